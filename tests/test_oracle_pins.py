@@ -1,0 +1,413 @@
+"""Pins for the float64 oracle: each check ties it to something other than itself.
+
+Hand-derived closed forms (tests/golden), library routines (torch SDPA, sklearn
+K-means), limits where MuSe is exact, calculus identities (the dipole is the
+Jacobian of softmax attention), invariances, and the truncation-error order.
+No GPU is used here.
+"""
+import glob
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import muse_oracle as mo
+from clustered_softmax_attention_b200.inputs import small_problem
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _closed(expr_tree):
+    """Evaluate nested lists of closed-form expression strings with math only."""
+    env = {"exp": math.exp, "log": math.log, "__builtins__": {}}
+    if isinstance(expr_tree, str):
+        return eval(expr_tree, env)  # noqa: S307 - fixture expressions are ours
+    return [_closed(e) for e in expr_tree]
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------- goldens
+
+@pytest.mark.parametrize("name", sorted(os.path.basename(p) for p in glob.glob(os.path.join(GOLDEN, "*.json"))))
+def test_golden_closed_forms(name):
+    g = _load(name)
+    Q, K, V = (np.array(g[k], float) for k in ("Q", "K", "V"))
+    s = g["scale"]
+    ql, kl = np.array(g["q_labels"]), np.array(g["k_labels"])
+    exp = g["expected"]
+    qbar = mo.cluster_means(Q, ql, g["Cq"])
+    logZ, mu_k, mu_v, cov = mo.tilted_summaries(qbar, K, V, kl, g["Ck"], s)
+    np.testing.assert_allclose(logZ, np.array(_closed(exp["logZ"])), rtol=1e-13, atol=1e-14)
+    for key, val in (("mu_k", mu_k), ("mu_v", mu_v), ("cov", cov)):
+        if key in exp:
+            np.testing.assert_allclose(val, np.array(_closed(exp[key])), rtol=1e-13, atol=1e-14)
+    O = mo.refine(Q, ql, qbar, logZ, mu_k, mu_v, cov, s)
+    np.testing.assert_allclose(O, np.array(_closed(exp["O"])), rtol=1e-12, atol=1e-14)
+    if "E" in exp:
+        E = mo.exact_attention(Q, K, V, s)
+        np.testing.assert_allclose(E, np.array(_closed(exp["E"])), rtol=1e-13)
+    if "kmeans_rounds" in g:
+        for t, want in g["kmeans_rounds"].items():
+            lab, cen = mo.kmeans(K, g["Ck"], int(t))
+            assert lab.tolist() == want["labels"]
+            np.testing.assert_allclose(cen, np.array(_closed(want["centroids"])), rtol=0, atol=1e-15)
+
+
+# --------------------------------------------------------------------------- exact attention
+
+def test_exact_attention_matches_torch_sdpa():
+    import torch
+    Q, K, V = small_problem(1, 50, 8, 5, 4, 0.3)
+    for causal in (False, True):
+        for s in (1.0, 0.7):
+            E = mo.exact_attention(Q, K, V, s, causal=causal)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.tensor(Q)[None], torch.tensor(K)[None], torch.tensor(V)[None],
+                is_causal=causal, scale=s)[0].numpy()
+            np.testing.assert_allclose(E, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_merge_partials_is_joint_softmax():
+    Q, K, V = small_problem(2, 40, 6, 3, 4, 0.4)
+    parts = []
+    for lo, hi in ((0, 7), (7, 30), (30, 40)):
+        o, l = mo.exact_attention(Q, K[lo:hi], V[lo:hi], 1.3, return_lse=True)
+        parts.append((l, o))
+    np.testing.assert_allclose(mo.merge_partials(parts), mo.exact_attention(Q, K, V, 1.3),
+                               rtol=1e-12, atol=1e-14)
+
+
+def test_rse_and_max_rel_err_definitions():
+    E = np.array([[3.0, 4.0], [0.0, 0.0]])
+    O = E + np.array([[0.0, 0.0], [1.0, 0.0]])
+    assert mo.rse(O, E) == pytest.approx(1.0 / 25.0)
+    assert mo.max_rel_err(O, E) == pytest.approx(1.0 / 4.0)
+
+
+# --------------------------------------------------------------------------- K-means
+
+def test_kmeans_matches_sklearn_lloyd_per_round():
+    from sklearn.cluster import KMeans
+    X, _, _ = small_problem(3, 300, 5, 1, 6, 0.25)
+    C = 6
+    for T in (1, 2, 3):
+        lab, cen = mo.kmeans(X, C, T)
+        assert np.bincount(lab, minlength=C).min() > 0
+        km = KMeans(n_clusters=C, init=X[:C].copy(), n_init=1, max_iter=T, tol=0.0,
+                    algorithm="lloyd").fit(X)
+        if km.n_iter_ == T:
+            np.testing.assert_allclose(cen, km.cluster_centers_, rtol=1e-12, atol=1e-13)
+            # sklearn's labels are the assignment to its final centroids
+            assert (mo.kmeans_assign(X, cen) == km.labels_).all()
+
+
+def test_kmeans_converged_matches_sklearn():
+    from sklearn.cluster import KMeans
+    X, _, _ = small_problem(4, 400, 6, 1, 5, 0.2)
+    lab, cen = mo.kmeans(X, 5, 60)
+    km = KMeans(n_clusters=5, init=X[:5].copy(), n_init=1, max_iter=60, tol=0.0,
+                algorithm="lloyd").fit(X)
+    assert (lab == km.labels_).all()
+    np.testing.assert_allclose(cen, km.cluster_centers_, rtol=1e-12, atol=1e-13)
+
+
+def test_kmeans_recovers_separated_mixture():
+    rng = np.random.default_rng(7)
+    comps, D = 8, 6
+    means = rng.standard_normal((comps, D)) * 10.0
+    idx = np.concatenate([np.arange(comps), rng.integers(0, comps, 500)])
+    X = means[idx] + 0.01 * rng.standard_normal((idx.size, D))
+    lab, cen = mo.kmeans(X, comps, 5)
+    # the first C rows are one point per component, so cluster c is component c
+    assert (lab == idx).all()
+    np.testing.assert_allclose(cen, means, atol=0.01)
+
+
+def test_kmeans_objective_nonincreasing():
+    X, _, _ = small_problem(5, 500, 8, 1, 20, 0.5)
+    _, _, hist = mo.kmeans(X, 16, 12, history=True)
+    objs = []
+    for C in hist:
+        lab = mo.kmeans_assign(X, C)
+        objs.append(mo.kmeans_objective(X, lab, C))
+    assert all(b <= a + 1e-12 for a, b in zip(objs, objs[1:]))
+
+
+def test_kmeans_empty_cluster_keeps_centroid_and_gap():
+    X = np.array([[0.0], [0.1], [10.0]])
+    C0 = np.array([[0.0], [5.0], [100.0]])
+    lab = mo.kmeans_assign(X, C0)
+    assert lab.tolist() == [0, 0, 1]
+    C1 = mo.kmeans_update(X, lab, C0)
+    assert C1[2, 0] == 100.0 and C1[0, 0] == pytest.approx(0.05) and C1[1, 0] == 10.0
+    lab2, gap = mo.kmeans_assign_gap(np.array([[1.0]]), np.array([[0.0], [2.0]]))
+    assert lab2[0] == 0 and gap[0] == 0.0
+
+
+# --------------------------------------------------------------------------- limits where MuSe is exact
+
+def test_singleton_key_clusters_are_exact_for_any_query_clustering():
+    """Ck = N: every key is its own cluster, kt = 0, C = 0 -> exact attention."""
+    Q, K, V = small_problem(8, 48, 6, 4, 5, 0.3)
+    rng = np.random.default_rng(0)
+    for s in (1.0, 2.5):
+        ql = rng.integers(0, 5, size=48)
+        O = mo.muse_from_labels(Q, K, V, ql, np.arange(48), 5, 48, s)
+        np.testing.assert_allclose(O, mo.exact_attention(Q, K, V, s), rtol=1e-10, atol=1e-12)
+
+
+def test_singleton_query_clusters_are_exact_for_any_key_clustering():
+    """Cq = N: qt = 0 -> exact attention, whatever the key clusters."""
+    Q, K, V = small_problem(9, 40, 5, 3, 4, 0.3)
+    rng = np.random.default_rng(1)
+    for s in (1.0, 3.0):
+        kl = rng.integers(0, 3, size=40)
+        O = mo.muse_from_labels(Q, K, V, np.arange(40), kl, 40, 3, s)
+        np.testing.assert_allclose(O, mo.exact_attention(Q, K, V, s), rtol=1e-10, atol=1e-12)
+    # the full pipeline with Cq = N: the first-N start makes every query its own centroid
+    O = mo.muse_acausal(Q, K, V, 40, 3, 4, 1.0)
+    np.testing.assert_allclose(O, mo.exact_attention(Q, K, V, 1.0), rtol=1e-10, atol=1e-12)
+
+
+def test_zero_residual_is_exact_attention_at_the_centroid():
+    """qt := 0 gives sum_j softmax(logZ_ij) mu_v,ij = exact attention evaluated at qbar_i."""
+    Q, K, V = small_problem(10, 60, 6, 4, 6, 0.4)
+    ql, qc = mo.kmeans(Q, 5, 3)
+    kl, _ = mo.kmeans(K, 7, 3)
+    O = mo.muse_from_labels(Q, K, V, ql, kl, 5, 7, 1.7, qbar=qc, zero_residual=True)
+    E = mo.exact_attention(qc[ql], K, V, 1.7)
+    np.testing.assert_allclose(O, E, rtol=1e-10, atol=1e-12)
+
+
+def test_single_key_cluster_is_first_order_taylor_of_attention():
+    """Ck = 1: O(q) = E(qbar) + J(qbar) qt with J the Jacobian of softmax attention.
+
+    The dipole s*C must equal dE/dq at the centroid (central differences, float64),
+    which fixes its sign, its transpose (Dv x D with D != Dv) and the factor s.
+    """
+    Q, K, V = small_problem(11, 30, 4, 3, 3, 0.5)
+    s = 1.6
+    qbar = Q.mean(0, keepdims=True)
+    logZ, mu_k, mu_v, cov = mo.tilted_summaries(qbar, K, V, np.zeros(30, int), 1, s)
+    h = 1e-5
+    J = np.zeros((3, 4))
+    for d in range(4):
+        e = np.zeros((1, 4))
+        e[0, d] = h
+        J[:, d] = (mo.exact_attention(qbar + e, K, V, s) - mo.exact_attention(qbar - e, K, V, s))[0] / (2 * h)
+    np.testing.assert_allclose(s * cov[0, 0], J, rtol=1e-7, atol=1e-10)
+    np.testing.assert_allclose(mu_v[0, 0], mo.exact_attention(qbar, K, V, s)[0], rtol=1e-12)
+    O = mo.refine(Q, np.zeros(30, int), qbar, logZ, mu_k, mu_v, cov, s)
+    np.testing.assert_allclose(O, mu_v[0, 0][None] + (Q - qbar) @ (s * cov[0, 0]).T, rtol=1e-12)
+
+
+# --------------------------------------------------------------------------- invariances
+
+def test_key_translation_invariance_and_query_translation_dependence():
+    Q, K, V = small_problem(12, 80, 6, 4, 4, 0.15)
+    O = mo.muse_acausal(Q, K, V, 6, 5, 6, 1.0)
+    rng = np.random.default_rng(3)
+    for norm in (0.5, 10.0):
+        t = rng.standard_normal(6)
+        t *= norm / np.linalg.norm(t)
+        Ot = mo.muse_acausal(Q, K + t, V, 6, 5, 6, 1.0)
+        np.testing.assert_allclose(Ot, O, rtol=1e-9, atol=1e-11)
+    t = rng.standard_normal(6)
+    Oq = mo.muse_acausal(Q + t, K, V, 6, 5, 6, 1.0)
+    assert np.abs(Oq - O).max() > 1e-3
+
+
+# --------------------------------------------------------------------------- truncation-error order
+
+def _order_problem(eq, ek, seed=0, N=64, D=4, Dv=3, cq=4, ck=4):
+    rng = np.random.default_rng(seed)
+    qc = rng.standard_normal((cq, D))
+    kc = rng.standard_normal((ck, D))
+    ql = np.arange(N) % cq
+    kl = np.arange(N) % ck
+    nq = rng.standard_normal((N, D))
+    nk = rng.standard_normal((N, D))
+    V = rng.standard_normal((N, Dv))
+    return qc[ql] + eq * nq, kc[kl] + ek * nk, V, ql, kl
+
+
+def _err(eq, ek, cq=4, ck=4):
+    Q, K, V, ql, kl = _order_problem(eq, ek, cq=cq, ck=ck)
+    O = mo.muse_from_labels(Q, K, V, ql, kl, cq, ck, 1.0)
+    return np.abs(O - mo.exact_attention(Q, K, V, 1.0)).max()
+
+
+def test_truncation_error_is_second_order_in_each_residual():
+    """Dropping only qt.kt leaves an error of order Tr(Cov(qt)Cov(kt)) ~ eq^2 ek^2."""
+    eps = np.array([1e-3, 3e-3, 1e-2, 3e-2, 1e-1])
+    fixed = 0.05
+    eq_err = np.array([_err(e, fixed) for e in eps])
+    ek_err = np.array([_err(fixed, e) for e in eps])
+    slope_q = np.polyfit(np.log(eps), np.log(eq_err), 1)[0]
+    slope_k = np.polyfit(np.log(eps), np.log(ek_err), 1)[0]
+    assert 1.8 <= slope_q <= 2.2, slope_q
+    assert 1.8 <= slope_k <= 2.2, slope_k
+    # error / (Tr Cov qt * Tr Cov kt) stays bounded as both shrink
+    ratios = [_err(e, e) / (e * e * e * e) for e in (1e-2, 3e-3, 1e-3)]
+    assert max(ratios) / min(ratios) < 2.0
+
+
+def test_monopole_only_would_be_first_order():
+    """Without the dipole the error would fall only linearly: guards the dipole's presence."""
+    def err_no_dip(eq):
+        Q, K, V, ql, kl = _order_problem(eq, 0.05)
+        qbar = mo.cluster_means(Q, ql, 4)
+        logZ, mu_k, mu_v, cov = mo.tilted_summaries(qbar, K, V, kl, 4, 1.0)
+        O = mo.refine(Q, ql, qbar, logZ, mu_k, mu_v, 0 * cov, 1.0)
+        return np.abs(O - mo.exact_attention(Q, K, V, 1.0)).max()
+    eps = np.array([1e-3, 1e-2, 1e-1])
+    slope = np.polyfit(np.log(eps), np.log([err_no_dip(e) for e in eps]), 1)[0]
+    assert 0.8 <= slope <= 1.2
+
+
+# --------------------------------------------------------------------------- tiny brute force
+
+def _bruteforce_muse(Q, K, V, ql, kl, Cq, Ck, s):
+    """Same definitions, written as scalar loops (N <= 16)."""
+    N, D = len(Q), len(Q[0])
+    Dv = len(V[0])
+    qbar = []
+    for i in range(Cq):
+        mem = [Q[n] for n in range(N) if ql[n] == i]
+        qbar.append([sum(m[d] for m in mem) / len(mem) if mem else 0.0 for d in range(D)])
+    out = []
+    for n in range(N):
+        i = ql[n]
+        qt = [Q[n][d] - qbar[i][d] for d in range(D)]
+        a, terms = [], []
+        for j in range(Ck):
+            mem = [k for k in range(N) if kl[k] == j]
+            if not mem:
+                continue
+            ell = [s * sum(qbar[i][d] * K[k][d] for d in range(D)) for k in mem]
+            mx = max(ell)
+            lz = mx + math.log(sum(math.exp(x - mx) for x in ell))
+            w = [math.exp(x - lz) for x in ell]
+            muk = [sum(w[t] * K[k][d] for t, k in enumerate(mem)) for d in range(D)]
+            muv = [sum(w[t] * V[k][e] for t, k in enumerate(mem)) for e in range(Dv)]
+            cq_ = [sum(w[t] * (V[k][e] - muv[e]) * sum((K[k][d] - muk[d]) * qt[d] for d in range(D))
+                       for t, k in enumerate(mem)) for e in range(Dv)]
+            a.append(lz + s * sum(qt[d] * muk[d] for d in range(D)))
+            terms.append([muv[e] + s * cq_[e] for e in range(Dv)])
+        mx = max(a)
+        p = [math.exp(x - mx) for x in a]
+        tot = sum(p)
+        out.append([sum(p[t] * terms[t][e] for t in range(len(a))) / tot for e in range(Dv)])
+    return np.array(out)
+
+
+def test_tiny_bruteforce_agrees():
+    Q, K, V = small_problem(13, 14, 3, 2, 3, 0.6)
+    ql = np.array([0, 1, 2, 0, 1, 2, 0, 0, 1, 1, 2, 2, 0, 1])
+    kl = np.array([0, 0, 1, 1, 2, 2, 3, 3, 0, 1, 2, 3, 0, 1])
+    for s in (1.0, 0.4):
+        O = mo.muse_from_labels(Q, K, V, ql, kl, 3, 5, s)   # key cluster 4 is empty
+        ref = _bruteforce_muse(Q.tolist(), K.tolist(), V.tolist(), ql.tolist(), kl.tolist(), 3, 5, s)
+        np.testing.assert_allclose(O, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_row_subset_matches_full():
+    Q, K, V = small_problem(14, 90, 5, 4, 5, 0.3)
+    ql, qc = mo.kmeans(Q, 6, 3)
+    kl, _ = mo.kmeans(K, 6, 3)
+    full = mo.muse_from_labels(Q, K, V, ql, kl, 6, 6, 1.0)
+    rows = np.array([0, 17, 44, 89])
+    sub = mo.muse_from_labels(Q, K, V, ql, kl, 6, 6, 1.0, rows=rows)
+    np.testing.assert_allclose(sub[rows], full[rows], rtol=1e-13)
+
+
+# --------------------------------------------------------------------------- causal decomposition
+
+def test_causal_squares_cover_each_prefix_once():
+    for N, S in ((64, 8), (72, 8), (40, 8), (16, 16)):
+        cover = np.zeros((N, N), int)
+        for n in range(N):
+            b = n // S
+            cover[n, b * S:n + 1] += 1
+        for (lev, r, q0, q1, k0, k1) in mo.causal_squares(N, S):
+            cover[q0:q1, k0:k1] += 1
+        assert (cover == np.tril(np.ones((N, N), int))).all(), (N, S)
+
+
+def test_causal_limits_are_exact():
+    Q, K, V = small_problem(15, 64, 5, 3, 4, 0.3)
+    E = mo.exact_attention(Q, K, V, 1.0, causal=True)
+    # one block: the diagonal is the whole causal attention
+    np.testing.assert_allclose(mo.muse_causal(Q, K, V, 64, 4, 4, 3, 1.0), E, rtol=1e-12)
+    # C >= range length in every square: singleton clusters everywhere -> exact
+    np.testing.assert_allclose(mo.muse_causal(Q, K, V, 8, 64, 64, 3, 1.0), E, rtol=1e-10, atol=1e-12)
+    # ragged N (not a power-of-two multiple of S)
+    Q2, K2, V2 = Q[:44], K[:44], V[:44]
+    E2 = mo.exact_attention(Q2, K2, V2, 1.0, causal=True)
+    np.testing.assert_allclose(mo.muse_causal(Q2, K2, V2, 8, 64, 64, 3, 1.0), E2, rtol=1e-10, atol=1e-12)
+
+
+def test_causal_is_close_to_exact_on_clustered_data():
+    Q, K, V = small_problem(16, 128, 6, 4, 4, 0.05)
+    O = mo.muse_causal(Q, K, V, 16, 4, 4, 5, 1.0)
+    assert mo.rse(O, mo.exact_attention(Q, K, V, 1.0, causal=True)) < 1e-4
+
+
+# --------------------------------------------------------------------------- retrieval
+
+def test_block_logz_merges_to_cluster_logz():
+    Q, K, V = small_problem(17, 64, 5, 3, 4, 0.3)
+    ql, qc = mo.kmeans(Q, 4, 3)
+    kl, _ = mo.kmeans(K, 5, 3)
+    lzb = mo.block_logZ(qc, K, kl, 5, 16, 1.3)
+    lz, _, _, _ = mo.tilted_summaries(qc, K, V, kl, 5, 1.3, want_cov=False)
+    np.testing.assert_allclose(np.logaddexp.reduce(lzb, axis=2), lz, rtol=1e-12)
+
+
+def test_retrieval_select_against_bruteforce_ranking():
+    rng = np.random.default_rng(5)
+    lzb = rng.standard_normal((3, 6, 5))
+    lzb[rng.random(lzb.shape) < 0.3] = -np.inf
+    lzb[1, 2, :] = lzb[1, 3, :]          # exact ties between clusters 2 and 3
+    sel = mo.retrieval_select(lzb, 2, 2)
+    for i in range(3):
+        assert (sel[i, 0] == -1).all()
+        for b in range(1, 5):
+            sig = {j: np.logaddexp.reduce(lzb[i, j, :b]) for j in range(6)}
+            ranked = [j for j, v in sorted(sig.items(), key=lambda kv: (-kv[1], kv[0])) if v > -np.inf][:2]
+            want = []
+            for j in ranked:
+                bl = [bb for bb, v in sorted(enumerate(lzb[i, j, :b]), key=lambda kv: (-kv[1], kv[0]))
+                      if v > -np.inf][:2]
+                want += [(j, bb) for bb in bl] + [(-1, -1)] * (2 - len(bl))
+            want += [(-1, -1)] * (4 - len(want))
+            assert [tuple(x) for x in sel[i, b]] == want
+
+
+def test_retrieval_limits_are_exact():
+    Q, K, V = small_problem(18, 64, 5, 3, 4, 0.3)
+    S = 16
+    E = mo.exact_attention(Q, K, V, 1.0, causal=True)
+    # everything retrieved: exact
+    O = mo.muse_retrieval(Q, K, V, S, 4, 5, 3, k1=5, k2=4, scale=1.0)
+    np.testing.assert_allclose(O, E, rtol=1e-10, atol=1e-12)
+    # singleton queries (qt = 0): exact whatever is retrieved
+    for k1, k2 in ((0, 0), (2, 1), (1, 3)):
+        O = mo.muse_retrieval(Q, K, V, S, 64, 5, 3, k1=k1, k2=k2, scale=1.0)
+        np.testing.assert_allclose(O, E, rtol=1e-10, atol=1e-12)
+    # singleton keys, nothing retrieved: the remainder summaries are exact
+    O = mo.muse_retrieval(Q, K, V, S, 4, 64, 3, k1=0, k2=0, scale=1.0)
+    np.testing.assert_allclose(O, E, rtol=1e-10, atol=1e-12)
+
+
+def test_retrieval_block_zero_uses_only_the_diagonal():
+    Q, K, V = small_problem(19, 48, 4, 3, 3, 0.3)
+    O = mo.muse_retrieval(Q, K, V, 16, 3, 3, 2, k1=1, k2=1, scale=1.0)
+    E0 = mo.exact_attention(Q[:16], K[:16], V[:16], 1.0, causal=True)
+    np.testing.assert_allclose(O[:16], E0, rtol=1e-12)
