@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""MuSe forward benchmark: tokens/s per head on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl muse|reference]
+                    [--workload acausal_n8k_bf16|causal_n16k_bf16|...]
+
+A step is one whole forward pass (both K-means, summaries, refinement; plus the
+diagonal blocks and merge on the causal workload) over one batch of seeded
+synthetic inputs already resident in HBM.  Steps are replayed from a CUDA graph,
+timed one by one with CUDA events on the launching stream, with a 256 MiB write
+between steps to flush L2.  value = B*H*N*ranks / (mean step time), taking the
+max over ranks.  ``e2e`` repeats the measurement through the public API with the
+inputs copied from pinned host memory and the output copied back inside the
+timed region.  ``--impl reference`` times the float64 oracle on the host cores on
+a bounded sample (one head per step) of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from clustered_softmax_attention_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "MuSe fwd tokens/s per head at N=8k/16k on 1 B200; % roofline; rel sq err"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # 148 SMs x 128 FP32 lanes x FMA x max clock
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="muse", choices=["muse", "reference"])
+    ap.add_argument("--workload", default="acausal_n8k_bf16", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_info():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_flops(w):
+    """Flops of the refinement contraction per launch (all problems).
+
+    Per problem the tilted dipole contraction costs 2*Cq*N*D*Dv and the refinement
+    2*N*Ck*D*Dv (acausal); the kernel evaluates the same contraction as
+    sum over query/key pairs, 2*nq*nk*(D+Dv), equal to it when Cq*D*Dv*... matches:
+    we count the smaller of the two per instance (the work the method needs).
+    """
+    def inst(nq, nk, cq, ck, D, Dv):
+        s_form = 2.0 * cq * nk * D * Dv + 2.0 * nq * ck * D * Dv
+        n_form = 2.0 * nq * nk * (D + Dv)
+        return min(s_form, n_form)
+    P = w.B * w.H
+    if w.mode == "acausal":
+        return P * inst(w.N, w.N, w.Cq, w.Ck, w.D, w.Dv)
+    if w.mode == "causal":
+        tot = 0.0
+        s = w.block
+        while s < w.N:
+            r = 1
+            while r * s < w.N:
+                nq = min((r + 1) * s, w.N) - r * s
+                tot += inst(nq, s, min(w.Cq, nq), min(w.Ck, s), w.D, w.Dv)
+                r += 2
+            s *= 2
+        return P * tot
+    raise ValueError(w.mode)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.sel = device_index
+
+    def start(self):
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.sel is not None:
+                cmd += ["-i", str(self.sel)]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def nvsmi_index(local_rank):
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(local_rank)
+        bus = getattr(p, "pci_bus_id", None)
+        dom = getattr(p, "pci_domain_id", None)
+        devid = getattr(p, "pci_device_id", None)
+        if bus is not None and dom is not None and devid is not None:
+            return f"{dom:08X}:{bus:02X}:{devid:02X}.0"
+    except Exception:
+        pass
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v for v in vis.split(",") if v.strip().isdigit()]
+    return ids[local_rank] if local_rank < len(ids) else local_rank
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, head=0):
+    """The float64 oracle on one head of the workload: (seconds, tokens)."""
+    from oracle import muse_oracle as mo
+    Q, K, V = make_inputs(w, heads=[head])
+    t0 = time.perf_counter()
+    if w.mode == "acausal":
+        mo.muse_acausal(Q[0, 0], K[0, 0], V[0, 0], w.Cq, w.Ck, w.iters, w.scale)
+    elif w.mode == "causal":
+        mo.muse_causal(Q[0, 0], K[0, 0], V[0, 0], w.block, w.Cq, w.Ck, w.iters, w.scale)
+    else:
+        raise ValueError(w.mode)
+    return time.perf_counter() - t0, w.N
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        oracle_sample(w)
+    secs = []
+    for k in range(args.steps):
+        s, n = oracle_sample(w, head=k % w.problems)
+        secs.append(s)
+    mean = sum(secs) / len(secs)
+    value = w.N / mean
+    cores = cpu_threads()
+    sample = f"one (b,h) problem of {w.name} per step (N={w.N} tokens), float64 numpy oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, graph=False),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, graph):
+    c = {"workload": w.name, "mode": w.mode, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "Dv": w.Dv,
+         "Cq": w.Cq, "Ck": w.Ck, "iters": w.iters, "scale": w.scale,
+         "l2": "flushed between timed steps (256 MiB write)", "cuda_graph": graph,
+         "parallelism": "replicas (every rank runs the whole workload; no collective)"}
+    if w.mode != "acausal":
+        c["block"] = w.block
+    if w.mode == "retrieval":
+        c.update(k1=w.k1, k2=w.k2)
+    return c
+
+
+def main():
+    args = parse()
+    rank, local_rank, world = dist_info()
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl" if args.impl == "muse" else "gloo",
+                                timeout=datetime.timedelta(seconds=300))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    from clustered_softmax_attention_b200 import muse as m
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[args.workload]
+    Qn, Kn, Vn = make_inputs(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    Qh = torch.from_numpy(Qn).to(tdt).pin_memory()
+    Kh = torch.from_numpy(Kn).to(tdt).pin_memory()
+    Vh = torch.from_numpy(Vn).to(tdt).pin_memory()
+    Qd, Kd, Vd = (x.to(dev) for x in (Qh, Kh, Vh))
+    Od = torch.empty(w.B, w.H, w.N, w.Dv, dtype=tdt, device=dev)
+    Oh = torch.empty_like(Od, device="cpu").pin_memory()
+    d = m.dims(Qd, Vd, w.scale)
+    if w.mode == "acausal":
+        ws = m.workspace("muse_forward", d, w.Cq, w.Ck)
+
+        def step(Q=Qd, K=Kd, V=Vd, O=Od):
+            m.muse_forward(Q, K, V, w.Cq, w.Ck, w.iters, w.scale, out=O, ws=ws)
+    elif w.mode == "causal":
+        ws = m.workspace("muse_causal_blocks", d, w.Cq, w.Ck, w.block)
+
+        def step(Q=Qd, K=Kd, V=Vd, O=Od):
+            m.muse_causal_blocks(Q, K, V, w.block, w.Cq, w.Ck, w.iters, w.scale, out=O, ws=ws)
+    else:
+        raise SystemExit(f"workload {w.name} is not benchmarked yet")
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    kev0, kev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kev0.record(stream)   # creates the underlying cudaEvent_t
+    kev1.record(stream)
+    m.lib().muse_set_profile_events(ctypes_ptr(kev0), ctypes_ptr(kev1))
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    n0 = m.lib().muse_launch_counter()
+    step()
+    torch.cuda.synchronize()
+    launches_per_step = int(m.lib().muse_launch_counter() - n0)
+    assert m.muse_last_device_status() == 0
+
+    graph = None
+    if not args.no_graph:
+        try:
+            s = torch.cuda.Stream()
+            s.wait_stream(stream)
+            with torch.cuda.stream(s):
+                step()
+            stream.wait_stream(s)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step()
+            torch.cuda.synchronize()
+            for _ in range(2):
+                graph.replay()
+            torch.cuda.synchronize()
+        except Exception as e:  # capture refused: time eager launches instead
+            print(f"cuda graph capture failed ({e}); timing eager launches", file=sys.stderr)
+            graph = None
+
+    def run_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(nvsmi_index(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    step_ms, kern_ms = [], []
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        run_step()
+        ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        step_ms.append(ev[k][0].elapsed_time(ev[k][1]))
+        kern_ms.append(kev0.elapsed_time(kev1))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(total, op=dist.ReduceOp.MAX)
+    mean_ms = float(total.item()) / args.steps
+    tokens = w.B * w.H * w.N
+    value = world * tokens / (mean_ms / 1e3)
+    assert m.muse_last_device_status() == 0
+
+    # end to end through the public API: pinned host inputs -> device -> output -> host
+    m.lib().muse_set_profile_events(None, None)
+    e2e_ms = []
+    for k in range(max(2, args.steps // 2)):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        Qd.copy_(Qh, non_blocking=True)
+        Kd.copy_(Kh, non_blocking=True)
+        Vd.copy_(Vh, non_blocking=True)
+        step()
+        Oh.copy_(Od, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    e2e_t = torch.tensor([sum(e2e_ms) / len(e2e_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = world * tokens / (float(e2e_t.item()) / 1e3)
+    h2d = sum(x.numel() * x.element_size() for x in (Qh, Kh, Vh))
+    d2h = Oh.numel() * Oh.element_size()
+
+    # roofline of the dominant kernel (the refinement), timed live above
+    peaks, peak_src = load_peaks()
+    kmean = sum(kern_ms) / len(kern_ms)
+    flops = algorithmic_flops(w)
+    achieved = flops / (kmean / 1e3) / 1e12
+    if w.dtype == "bf16":
+        peak, bound, unit = float(peaks["bf16_tflops"]), "tensor", "TFLOP/s"
+    else:
+        peak, bound, unit = FP32_SIMT_TFLOPS, "alu", "TFLOP/s"
+    roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": None, "kernel": "refinement",
+            "kernel_ms": kmean, "flops_per_launch": flops,
+            "peak_source": f"{peak_src} bf16_tflops (burst)" if w.dtype == "bf16"
+            else "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
+    if rank == 0:
+        try:
+            from oracle import muse_oracle as mo
+            rng = np.random.default_rng(0)
+            rows = rng.choice(w.N, 64, replace=False)
+            On = Od[0, 0].float().cpu().numpy().astype(np.float64)
+            E = mo.exact_attention(Qn[0, 0], Kn[0, 0], Vn[0, 0], w.scale, rows=rows,
+                                   causal=(w.mode != "acausal"))
+            rse = float(((On[rows] - E[rows]) ** 2).sum() / (E[rows] ** 2).sum())
+        except Exception:
+            rse = None
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            secs, n = oracle_sample(w)
+            cpu = {"value": n / secs, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                   "sample": f"one (b,h) problem of {w.name} (N={w.N} tokens), float64 numpy "
+                             f"oracle, {secs:.1f} s"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded Gaussian-mixture Q/K, normal V)",
+            "config": config_of(w, graph is not None),
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk, "rse_vs_exact_sampled": rse,
+            "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms),
+        }
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def ctypes_ptr(ev):
+    import ctypes
+    return ctypes.c_void_p(ev.cuda_event)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,86 @@
+// Shared device helpers for libmuse (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+
+#include "../../include/muse.h"
+
+namespace muse {
+
+// ---------------------------------------------------------------------------
+// Element I/O: inputs are float32 or bfloat16; arithmetic is float32.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ld_elem(const float *p) { return *p; }
+__device__ __forceinline__ float ld_elem(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void st_elem(float *p, float v) { *p = v; }
+__device__ __forceinline__ void st_elem(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+// ---------------------------------------------------------------------------
+// Segment table: the row ranges of the sequence axis that are clustered
+// separately.  The same table applies to every (b,h) problem.
+//   acausal / retrieval: one segment covering [0, N)
+//   causal: one segment per below-diagonal square (its query range on the query
+//           side, its key range on the key side)
+// Per problem p and segment s:
+//   row-indexed arrays (labels, perm, sorted copies) start at p*row_stride + lab0[s]
+//   cluster-indexed arrays (centroids, counts)       start at p*cen_stride + cen0[s]
+//   offsets arrays (C+1 entries)                      start at p*off_stride + off0[s]
+// ---------------------------------------------------------------------------
+constexpr int kMaxSeg = 128;
+constexpr int kMaxClusters = 1024;
+
+struct SegTable {
+  int nseg;
+  int row_stride, cen_stride, off_stride;
+  int max_rows, max_C;
+  int row0[kMaxSeg];
+  int nrow[kMaxSeg];
+  int C[kMaxSeg];
+  int lab0[kMaxSeg];
+  int cen0[kMaxSeg];
+  int off0[kMaxSeg];
+};
+
+// A task is one (problem, segment) pair.
+struct Task {
+  int p, s;
+  int row0, n, C;
+  int64_t lab, cen, off;  // absolute element offsets of the task's arrays
+};
+
+__host__ __device__ __forceinline__ Task make_task(const SegTable &t, int task) {
+  Task k;
+  k.p = task / t.nseg;
+  k.s = task - k.p * t.nseg;
+  k.row0 = t.row0[k.s];
+  k.n = t.nrow[k.s];
+  k.C = t.C[k.s];
+  k.lab = (int64_t)k.p * t.row_stride + t.lab0[k.s];
+  k.cen = (int64_t)k.p * t.cen_stride + t.cen0[k.s];
+  k.off = (int64_t)k.p * t.off_stride + t.off0[k.s];
+  return k;
+}
+
+// ---------------------------------------------------------------------------
+// Device status word (MUSE_OK / MUSE_ERR_TIMEOUT / MUSE_ERR_DEVICE).  Kernels get
+// its address as a parameter; the first error wins.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void report(int *status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+}  // namespace muse

@@ -1,0 +1,83 @@
+// Host-side declarations shared by the libmuse translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace muse {
+
+inline size_t align_up(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Host-side count of enqueued kernels (muse_launch_counter).
+void count_launches(int n);
+
+// Per-instance offsets of the stage buffers.  An instance pairs query segment s
+// with key segment s (acausal: the one whole-sequence segment; causal: one square).
+struct InstTable {
+  int ninst;
+  int w_stride;   // per problem: floats of W (sum over instances of Cq_s * nk_s)
+  int z_stride;   // per problem: entries of logZ (sum of Cq_s * Ck_s)
+  int c_stride;   // per problem: floats of each coefficient array (sum of Ck_s * nq_s)
+  int out_stride; // per problem: rows of the output / partial arrays
+  int w0[kMaxSeg], z0[kMaxSeg], cc0[kMaxSeg], out0[kMaxSeg];
+};
+
+struct MuseTables {
+  SegTable q, k;
+  InstTable in;
+};
+
+struct KmeansOut {
+  int32_t *labels;
+  float *centroids;
+  int32_t *perm;
+  int32_t *offsets;
+};
+
+size_t kmeans_ws_bytes(const SegTable &t, int P);
+cudaError_t run_kmeans(const void *X, int dtype, int D, int N, const SegTable &tab, int P,
+                       int iters, const KmeansOut &o, char *ws, int *status, cudaStream_t st);
+
+// Sorted working copies of one side (rows in cluster order).
+struct SortedSide {
+  void *rows;        // [P][row_stride][width] in the input dtype (queries: residuals q - qbar)
+  int32_t *cluster;  // [P][row_stride] cluster of each sorted position
+};
+
+// Stage buffers for the summaries + refinement of every instance.
+struct StageBufs {
+  float *W;        // [P][w_stride]  tilt logits, then tilt weights w_ik
+  float *logZ;     // [P][z_stride]
+  float *mu_k;     // [P][z_stride][D]
+  float *mu_v;     // [P][z_stride][Dv] (optional)
+  float *cov;      // [P][z_stride][Dv][D] (optional)
+  float *c0, *c1;  // [P][c_stride]
+  float *lse;      // [P][q.row_stride] logsumexp_j a_j per sorted query position
+};
+
+cudaError_t run_sort_side(const void *X, int dtype, int width, int N, const SegTable &tab, int P,
+                          const int32_t *perm, const int32_t *offsets, const float *centroids,
+                          SortedSide out, cudaStream_t st);
+cudaError_t run_summaries(const MuseTables &mt, int dtype, int D, int Dv, int P, float scale,
+                          const float *q_centroids, SortedSide ks, const void *vs_rows,
+                          const int32_t *k_offsets, StageBufs b, cudaStream_t st);
+// W = exp(s qbar_i.k - logZ_ij) for given logZ (the refinement's tilt weights).
+cudaError_t run_tilt_weights(const MuseTables &mt, int dtype, int D, int P, float scale,
+                             const float *q_centroids, SortedSide ks, const float *logZ, float *W,
+                             cudaStream_t st);
+cudaError_t run_coeffs(const MuseTables &mt, int dtype, int D, int P, float scale,
+                       SortedSide qs, const int32_t *q_offsets, StageBufs b, cudaStream_t st);
+// Refinement: acausal writes O[p][row][:] (row = sequence row); partial mode writes
+// part_o[p][out0 + row][:] (float32) and part_lse[p][out0 + row].
+cudaError_t run_refine(const MuseTables &mt, int dtype, int D, int Dv, int N, int P,
+                       SortedSide qs, const int32_t *q_perm, SortedSide ks, const void *vs_rows,
+                       StageBufs b, void *O, float *part_o, float *part_lse, cudaStream_t st);
+size_t muse_retrieval_ws(const muse_dims &d, int block, int Cq, int Ck, int k1, int k2);
+cudaError_t run_diag_merge(const void *Q, const void *K, const void *V, int dtype, int D, int Dv,
+                           int N, int P, int block, int levels, float scale,
+                           const float *part_o, const float *part_lse, void *O, cudaStream_t st);
+
+}  // namespace muse

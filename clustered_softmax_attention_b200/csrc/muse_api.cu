@@ -1,0 +1,559 @@
+// extern "C" entry points of libmuse: argument validation, segment tables,
+// workspace layout and the launch sequence of every call.  Declarations and the
+// meaning of every argument: include/muse.h.
+#include <math.h>
+
+#include <atomic>
+#include <mutex>
+#include <string.h>
+#include <vector>
+
+#include "internal.h"
+#include "tc.h"
+
+namespace muse {
+
+// ---------------------------------------------------------------------------
+// Device status word: one per device, read and cleared by muse_last_device_status.
+// ---------------------------------------------------------------------------
+static __device__ int g_status_word;
+
+static std::atomic<uint64_t> g_launches{0};
+static std::atomic<void *> g_prof_start{nullptr}, g_prof_stop{nullptr};
+
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+static int *status_ptr() {
+  static std::mutex mu;
+  static int *ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int *>(p);
+  }
+  return ptrs[dev];
+}
+
+// ---------------------------------------------------------------------------
+// Workspace: a bump allocator over the caller's buffer (or a size count when
+// base == nullptr).  Every piece is 256-byte aligned.
+// ---------------------------------------------------------------------------
+struct Bump {
+  char *base;
+  size_t off = 0;
+  explicit Bump(void *b) : base(static_cast<char *>(b)) {}
+  template <typename T>
+  T *take(size_t count) {
+    const size_t o = off;
+    off = align_up(off + count * sizeof(T));
+    return base ? reinterpret_cast<T *>(base + o) : nullptr;
+  }
+};
+
+static size_t elem_size(int dtype) { return dtype == MUSE_F32 ? 4 : 2; }
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static muse_status check_dims(const muse_dims &d, bool need_dv) {
+  if (d.dtype != MUSE_F32 && d.dtype != MUSE_BF16) return MUSE_ERR_DTYPE;
+  if (d.B <= 0 || d.H <= 0 || d.N <= 0) return MUSE_ERR_SHAPE;
+  if (d.D != 64 && d.D != 128) return MUSE_ERR_SHAPE;
+  if (need_dv && d.Dv != 64 && d.Dv != 128) return MUSE_ERR_SHAPE;
+  if ((int64_t)d.B * d.H > 65535) return MUSE_ERR_SHAPE;
+  if ((int64_t)d.N * 128 > (int64_t)1 << 31) return MUSE_ERR_SHAPE;
+  if (!isfinite(d.scale)) return MUSE_ERR_INVALID_ARG;
+  return MUSE_OK;
+}
+
+static bool valid_C(int C, int n) { return C >= 1 && C <= n && C <= kMaxClusters; }
+
+// One segment covering the whole sequence.
+static SegTable whole_side(int N, int C) {
+  SegTable t;
+  memset(&t, 0, sizeof(t));
+  t.nseg = 1;
+  t.row_stride = N;
+  t.cen_stride = C;
+  t.off_stride = C + 1;
+  t.max_rows = N;
+  t.max_C = C;
+  t.row0[0] = 0;
+  t.nrow[0] = N;
+  t.C[0] = C;
+  return t;
+}
+
+static InstTable whole_inst(int N, int Cq, int Ck) {
+  InstTable in;
+  memset(&in, 0, sizeof(in));
+  in.ninst = 1;
+  in.w_stride = Cq * N;
+  in.z_stride = Cq * Ck;
+  in.c_stride = Ck * N;
+  in.out_stride = N;
+  return in;
+}
+
+// Squares of the causal decomposition: level l (side s = block*2^(l-1)), odd r with
+// r*s < N: queries [r s, min((r+1) s, N)), keys [(r-1) s, r s).
+struct Square {
+  int lev, q0, q1, k0, k1;
+};
+static std::vector<Square> causal_squares(int N, int block) {
+  std::vector<Square> out;
+  int lev = 1;
+  for (int64_t s = block; s < N; s *= 2, ++lev)
+    for (int64_t r = 1; r * s < N; r += 2)
+      out.push_back({lev, (int)(r * s), (int)std::min<int64_t>((r + 1) * s, N), (int)((r - 1) * s),
+                     (int)(r * s)});
+  return out;
+}
+
+}  // namespace muse
+
+using namespace muse;
+
+extern "C" int muse_causal_levels(int N, int block) {
+  if (N <= 0 || block <= 0) return 0;
+  int L = 0;
+  for (int64_t s = block; s < N; s *= 2) ++L;
+  return L;
+}
+
+namespace muse {
+
+static bool build_causal(int N, int block, int Cq, int Ck, MuseTables &mt, int &levels) {
+  levels = muse_causal_levels(N, block);
+  std::vector<Square> sq = causal_squares(N, block);
+  if ((int)sq.size() > kMaxSeg || sq.empty()) return false;
+  memset(&mt, 0, sizeof(mt));
+  SegTable &q = mt.q, &k = mt.k;
+  InstTable &in = mt.in;
+  q.nseg = k.nseg = in.ninst = (int)sq.size();
+  int cq_acc = 0, ck_acc = 0, oq = 0, ok = 0, w = 0, z = 0, c = 0;
+  for (size_t s = 0; s < sq.size(); ++s) {
+    const Square &x = sq[s];
+    const int nq = x.q1 - x.q0, nk = x.k1 - x.k0;
+    const int cq = std::min(Cq, nq), ck = std::min(Ck, nk);
+    q.row0[s] = x.q0; q.nrow[s] = nq; q.C[s] = cq; q.lab0[s] = (x.lev - 1) * N + x.q0;
+    q.cen0[s] = cq_acc; q.off0[s] = oq;
+    k.row0[s] = x.k0; k.nrow[s] = nk; k.C[s] = ck; k.lab0[s] = (x.lev - 1) * N + x.k0;
+    k.cen0[s] = ck_acc; k.off0[s] = ok;
+    in.w0[s] = w; in.z0[s] = z; in.cc0[s] = c; in.out0[s] = (x.lev - 1) * N;
+    cq_acc += cq; ck_acc += ck; oq += cq + 1; ok += ck + 1;
+    w += cq * nk; z += cq * ck; c += ck * nq;
+    q.max_rows = std::max(q.max_rows, nq); k.max_rows = std::max(k.max_rows, nk);
+    q.max_C = std::max(q.max_C, cq); k.max_C = std::max(k.max_C, ck);
+  }
+  q.row_stride = k.row_stride = levels * N;
+  q.cen_stride = cq_acc; k.cen_stride = ck_acc;
+  q.off_stride = oq; k.off_stride = ok;
+  in.w_stride = w; in.z_stride = z; in.c_stride = c; in.out_stride = levels * N;
+  return true;
+}
+
+// Workspace of the refinement (sorted copies, tilt weights, coefficients).
+struct RefineWs {
+  SortedSide qs, ks;
+  void *vs;
+  int32_t *v_cluster;
+  StageBufs sb;
+};
+
+static void plan_refine(Bump &bp, const MuseTables &mt, const muse_dims &d, int P, RefineWs &r,
+                        bool need_logZ_mu) {
+  const size_t es = elem_size(d.dtype);
+  const size_t qrows = (size_t)P * mt.q.row_stride, krows = (size_t)P * mt.k.row_stride;
+  r.qs.rows = bp.take<char>(qrows * d.D * es);
+  r.qs.cluster = bp.take<int32_t>(qrows);
+  r.ks.rows = bp.take<char>(krows * d.D * es);
+  r.ks.cluster = bp.take<int32_t>(krows);
+  r.vs = bp.take<char>(krows * d.Dv * es);
+  r.v_cluster = bp.take<int32_t>(krows);
+  memset(&r.sb, 0, sizeof(r.sb));
+  r.sb.W = bp.take<float>((size_t)P * mt.in.w_stride);
+  if (need_logZ_mu) {
+    r.sb.logZ = bp.take<float>((size_t)P * mt.in.z_stride);
+    r.sb.mu_k = bp.take<float>((size_t)P * mt.in.z_stride * d.D);
+  }
+  r.sb.c0 = bp.take<float>((size_t)P * mt.in.c_stride);
+  r.sb.c1 = bp.take<float>((size_t)P * mt.in.c_stride);
+  r.sb.lse = bp.take<float>(qrows);
+}
+
+struct KmWs {
+  KmeansOut q, k;
+  char *scratch;
+};
+
+static void plan_kmeans_pair(Bump &bp, const MuseTables &mt, const muse_dims &d, int P, KmWs &w) {
+  auto side = [&](const SegTable &t, KmeansOut &o) {
+    o.labels = bp.take<int32_t>((size_t)P * t.row_stride);
+    o.centroids = bp.take<float>((size_t)P * t.cen_stride * d.D);
+    o.perm = bp.take<int32_t>((size_t)P * t.row_stride);
+    o.offsets = bp.take<int32_t>((size_t)P * t.off_stride);
+  };
+  side(mt.q, w.q);
+  side(mt.k, w.k);
+  w.scratch = bp.take<char>(std::max(kmeans_ws_bytes(mt.q, P), kmeans_ws_bytes(mt.k, P)));
+}
+
+#define MUSE_TRY(expr)                                  \
+  do {                                                  \
+    cudaError_t e_ = (expr);                            \
+    if (e_ != cudaSuccess) return MUSE_ERR_CUDA;        \
+  } while (0)
+
+// The refinement launch sequence shared by every path.
+static muse_status refine_path(const void *Q, const void *K, const void *V, const muse_dims &d,
+                               int P, const MuseTables &mt, const float *q_centroids,
+                               const int32_t *q_perm, const int32_t *q_offsets,
+                               const int32_t *k_perm, const int32_t *k_offsets,
+                               const float *logZ_in, const float *mu_k_in, RefineWs &r, void *O,
+                               float *part_o, float *part_lse, cudaStream_t st) {
+  MUSE_TRY(run_sort_side(Q, d.dtype, d.D, d.N, mt.q, P, q_perm, q_offsets, q_centroids, r.qs, st));
+  MUSE_TRY(run_sort_side(K, d.dtype, d.D, d.N, mt.k, P, k_perm, k_offsets, nullptr, r.ks, st));
+  SortedSide vsd{r.vs, r.v_cluster};
+  MUSE_TRY(run_sort_side(V, d.dtype, d.Dv, d.N, mt.k, P, k_perm, k_offsets, nullptr, vsd, st));
+  StageBufs sb = r.sb;
+  if (logZ_in) {
+    sb.logZ = const_cast<float *>(logZ_in);
+    sb.mu_k = const_cast<float *>(mu_k_in);
+    MUSE_TRY(run_tilt_weights(mt, d.dtype, d.D, P, d.scale, q_centroids, r.ks, logZ_in, sb.W, st));
+  } else {
+    MUSE_TRY(run_summaries(mt, d.dtype, d.D, d.Dv, P, d.scale, q_centroids, r.ks, nullptr,
+                           k_offsets, sb, st));
+  }
+  MUSE_TRY(run_coeffs(mt, d.dtype, d.D, P, d.scale, r.qs, q_offsets, sb, st));
+  void *ev0 = g_prof_start.load(), *ev1 = g_prof_stop.load();
+  if (ev0 && ev1) MUSE_TRY(cudaEventRecordWithFlags((cudaEvent_t)ev0, st, cudaEventRecordExternal));
+  if (tc_supported(d.dtype, d.D, d.Dv)) {
+    MUSE_TRY(run_refine_tc(mt, d.D, d.Dv, d.N, P, r.qs, q_perm, r.ks, r.vs, sb, O, part_o,
+                           part_lse, status_ptr(), st));
+  } else {
+    MUSE_TRY(run_refine(mt, d.dtype, d.D, d.Dv, d.N, P, r.qs, q_perm, r.ks, r.vs, sb, O, part_o,
+                        part_lse, st));
+  }
+  if (ev0 && ev1) MUSE_TRY(cudaEventRecordWithFlags((cudaEvent_t)ev1, st, cudaEventRecordExternal));
+  return MUSE_OK;
+}
+
+}  // namespace muse
+
+// ===========================================================================
+// Entry points
+// ===========================================================================
+
+extern "C" const char *muse_status_string(muse_status s) {
+  switch (s) {
+    case MUSE_OK: return "MUSE_OK";
+    case MUSE_ERR_INVALID_ARG: return "MUSE_ERR_INVALID_ARG";
+    case MUSE_ERR_SHAPE: return "MUSE_ERR_SHAPE";
+    case MUSE_ERR_DTYPE: return "MUSE_ERR_DTYPE";
+    case MUSE_ERR_WORKSPACE: return "MUSE_ERR_WORKSPACE";
+    case MUSE_ERR_CUDA: return "MUSE_ERR_CUDA";
+    case MUSE_ERR_TIMEOUT: return "MUSE_ERR_TIMEOUT";
+    case MUSE_ERR_DEVICE: return "MUSE_ERR_DEVICE";
+  }
+  return "MUSE_ERR_UNKNOWN";
+}
+
+extern "C" uint64_t muse_launch_counter(void) { return g_launches.load(); }
+
+extern "C" void muse_set_profile_events(void *start, void *stop) {
+  g_prof_start.store(start);
+  g_prof_stop.store(stop);
+}
+
+extern "C" muse_status muse_last_device_status(muse_stream_t st) {
+  if (cudaStreamSynchronize((cudaStream_t)st) != cudaSuccess) return MUSE_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof(int)) != cudaSuccess) return MUSE_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int)) != cudaSuccess) return MUSE_ERR_CUDA;
+  return (muse_status)v;
+}
+
+// --------------------------------------------------------------------------- sizes
+
+static size_t ws_kmeans(const muse_dims &d, int C) {
+  SegTable t = whole_side(d.N, C);
+  return kmeans_ws_bytes(t, d.B * d.H);
+}
+
+static size_t ws_summaries(const muse_dims &d, int Cq, int Ck, bool need_v, bool need_mu) {
+  const int P = d.B * d.H;
+  MuseTables mt;
+  mt.q = whole_side(d.N, Cq);
+  mt.k = whole_side(d.N, Ck);
+  mt.in = whole_inst(d.N, Cq, Ck);
+  Bump bp(nullptr);
+  const size_t es = elem_size(d.dtype);
+  bp.take<char>((size_t)P * d.N * d.D * es);
+  bp.take<int32_t>((size_t)P * d.N);
+  if (need_v) bp.take<char>((size_t)P * d.N * d.Dv * es);
+  bp.take<float>((size_t)P * mt.in.w_stride);
+  if (need_mu) {
+    bp.take<float>((size_t)P * mt.in.z_stride * d.D);
+    bp.take<float>((size_t)P * mt.in.z_stride * d.Dv);
+  }
+  return bp.off;
+}
+
+static size_t ws_refine(const muse_dims &d, int Cq, int Ck) {
+  MuseTables mt;
+  mt.q = whole_side(d.N, Cq);
+  mt.k = whole_side(d.N, Ck);
+  mt.in = whole_inst(d.N, Cq, Ck);
+  Bump bp(nullptr);
+  RefineWs r;
+  plan_refine(bp, mt, d, d.B * d.H, r, false);
+  return bp.off;
+}
+
+static size_t ws_forward(const muse_dims &d, int Cq, int Ck) {
+  MuseTables mt;
+  mt.q = whole_side(d.N, Cq);
+  mt.k = whole_side(d.N, Ck);
+  mt.in = whole_inst(d.N, Cq, Ck);
+  Bump bp(nullptr);
+  KmWs kw;
+  plan_kmeans_pair(bp, mt, d, d.B * d.H, kw);
+  RefineWs r;
+  plan_refine(bp, mt, d, d.B * d.H, r, true);
+  return bp.off;
+}
+
+static size_t ws_causal(const muse_dims &d, int block, int Cq, int Ck) {
+  MuseTables mt;
+  int L = 0;
+  if (!build_causal(d.N, block, Cq, Ck, mt, L)) return 0;
+  const int P = d.B * d.H;
+  Bump bp(nullptr);
+  KmWs kw;
+  plan_kmeans_pair(bp, mt, d, P, kw);
+  RefineWs r;
+  plan_refine(bp, mt, d, P, r, true);
+  bp.take<float>((size_t)P * L * d.N * d.Dv);
+  bp.take<float>((size_t)P * L * d.N);
+  return bp.off;
+}
+
+extern "C" size_t muse_workspace_size(const char *entry, muse_dims d, int Cq, int Ck, int block,
+                                      int k1, int k2) {
+  if (!entry) return 0;
+  const bool dv_needed = strcmp(entry, "muse_kmeans") != 0;
+  if (check_dims(d, dv_needed) != MUSE_OK) return 0;
+  if (!strcmp(entry, "muse_kmeans")) return valid_C(Cq, d.N) ? ws_kmeans(d, Cq) : 0;
+  if (!valid_C(Cq, d.N) && strcmp(entry, "muse_causal_blocks") != 0) return 0;
+  if (!strcmp(entry, "muse_tilted_summaries"))
+    return valid_C(Ck, d.N) ? ws_summaries(d, Cq, Ck, true, true) : 0;
+  if (!strcmp(entry, "muse_dipole_refine")) return valid_C(Ck, d.N) ? ws_refine(d, Cq, Ck) : 0;
+  if (!strcmp(entry, "muse_forward")) return valid_C(Ck, d.N) ? ws_forward(d, Cq, Ck) : 0;
+  if (!strcmp(entry, "muse_causal_blocks")) {
+    if (block <= 0 || block % 64 || d.N % block || Cq < 1 || Ck < 1 || Cq > kMaxClusters ||
+        Ck > kMaxClusters)
+      return 0;
+    return ws_causal(d, block, Cq, Ck);
+  }
+  if (!strcmp(entry, "muse_retrieve_exact")) return muse_retrieval_ws(d, block, Cq, Ck, k1, k2);
+  return 0;
+}
+
+// --------------------------------------------------------------------------- muse_kmeans
+
+extern "C" muse_status muse_kmeans(const void *X, muse_dims d, int C, int iters, int32_t *labels,
+                                   float *centroids, int32_t *perm, int32_t *offsets, void *ws,
+                                   size_t ws_bytes, muse_stream_t st) {
+  muse_status s = check_dims(d, false);
+  if (s != MUSE_OK) return s;
+  if (!X || !labels || !centroids || !perm || !offsets) return MUSE_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(labels) || !aligned16(centroids) || !aligned16(perm) ||
+      !aligned16(offsets))
+    return MUSE_ERR_INVALID_ARG;
+  if (!valid_C(C, d.N) || iters < 1 || iters > 1000) return MUSE_ERR_INVALID_ARG;
+  const size_t need = ws_kmeans(d, C);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
+  SegTable t = whole_side(d.N, C);
+  KmeansOut o{labels, centroids, perm, offsets};
+  if (run_kmeans(X, d.dtype, d.D, d.N, t, d.B * d.H, iters, o, (char *)ws, status_ptr(),
+                 (cudaStream_t)st) != cudaSuccess)
+    return MUSE_ERR_CUDA;
+  return MUSE_OK;
+}
+
+// --------------------------------------------------------------------------- summaries
+
+extern "C" muse_status muse_tilted_summaries(const float *q_centroids, const void *K,
+                                             const void *V, const int32_t *k_perm,
+                                             const int32_t *k_offsets, muse_dims d, int Cq, int Ck,
+                                             float *logZ, float *mu_k, float *mu_v, float *cov,
+                                             void *ws, size_t ws_bytes, muse_stream_t st) {
+  const bool need_v = mu_v || cov;
+  muse_status s = check_dims(d, need_v);
+  if (s != MUSE_OK) return s;
+  if (!q_centroids || !K || !k_perm || !k_offsets || !logZ || (need_v && !V))
+    return MUSE_ERR_INVALID_ARG;
+  for (const void *p : {(const void *)q_centroids, K, V, (const void *)k_perm,
+                        (const void *)k_offsets, (const void *)logZ, (const void *)mu_k,
+                        (const void *)mu_v, (const void *)cov})
+    if (p && !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  if (!valid_C(Cq, d.N) || !valid_C(Ck, d.N)) return MUSE_ERR_INVALID_ARG;
+  const size_t need = ws_summaries(d, Cq, Ck, true, true);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
+  const int P = d.B * d.H;
+  MuseTables mt;
+  mt.q = whole_side(d.N, Cq);
+  mt.k = whole_side(d.N, Ck);
+  mt.in = whole_inst(d.N, Cq, Ck);
+  Bump bp(ws);
+  const size_t es = elem_size(d.dtype);
+  SortedSide ks{bp.take<char>((size_t)P * d.N * d.D * es), bp.take<int32_t>((size_t)P * d.N)};
+  void *vs = bp.take<char>((size_t)P * d.N * d.Dv * es);
+  StageBufs sb;
+  memset(&sb, 0, sizeof(sb));
+  sb.W = bp.take<float>((size_t)P * mt.in.w_stride);
+  float *mk_int = bp.take<float>((size_t)P * mt.in.z_stride * d.D);
+  float *mv_int = bp.take<float>((size_t)P * mt.in.z_stride * d.Dv);
+  sb.logZ = logZ;
+  sb.mu_k = mu_k ? mu_k : (cov ? mk_int : nullptr);
+  sb.mu_v = mu_v ? mu_v : (cov ? mv_int : nullptr);
+  sb.cov = cov;
+  cudaStream_t cs = (cudaStream_t)st;
+  if (run_sort_side(K, d.dtype, d.D, d.N, mt.k, P, k_perm, k_offsets, nullptr, ks, cs) !=
+      cudaSuccess)
+    return MUSE_ERR_CUDA;
+  if (need_v) {
+    SortedSide vsd{vs, ks.cluster};
+    if (run_sort_side(V, d.dtype, d.Dv, d.N, mt.k, P, k_perm, k_offsets, nullptr, vsd, cs) !=
+        cudaSuccess)
+      return MUSE_ERR_CUDA;
+  }
+  if (run_summaries(mt, d.dtype, d.D, d.Dv, P, d.scale, q_centroids, ks, vs, k_offsets, sb, cs) !=
+      cudaSuccess)
+    return MUSE_ERR_CUDA;
+  return MUSE_OK;
+}
+
+// --------------------------------------------------------------------------- refine
+
+extern "C" muse_status muse_dipole_refine(const void *Q, const void *K, const void *V,
+                                          const float *q_centroids, const int32_t *q_perm,
+                                          const int32_t *q_offsets, const int32_t *k_perm,
+                                          const int32_t *k_offsets, const float *logZ,
+                                          const float *mu_k, muse_dims d, int Cq, int Ck, void *O,
+                                          void *ws, size_t ws_bytes, muse_stream_t st) {
+  muse_status s = check_dims(d, true);
+  if (s != MUSE_OK) return s;
+  const void *ptrs[] = {Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offsets, logZ, mu_k, O};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  if (!valid_C(Cq, d.N) || !valid_C(Ck, d.N)) return MUSE_ERR_INVALID_ARG;
+  const size_t need = ws_refine(d, Cq, Ck);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
+  const int P = d.B * d.H;
+  MuseTables mt;
+  mt.q = whole_side(d.N, Cq);
+  mt.k = whole_side(d.N, Ck);
+  mt.in = whole_inst(d.N, Cq, Ck);
+  Bump bp(ws);
+  RefineWs r;
+  plan_refine(bp, mt, d, P, r, false);
+  return refine_path(Q, K, V, d, P, mt, q_centroids, q_perm, q_offsets, k_perm, k_offsets, logZ,
+                     mu_k, r, O, nullptr, nullptr, (cudaStream_t)st);
+}
+
+// --------------------------------------------------------------------------- forward
+
+extern "C" muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims d,
+                                    int Cq, int Ck, int iters, void *O, void *ws, size_t ws_bytes,
+                                    muse_stream_t st) {
+  muse_status s = check_dims(d, true);
+  if (s != MUSE_OK) return s;
+  const void *ptrs[] = {Q, K, V, O};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  if (!valid_C(Cq, d.N) || !valid_C(Ck, d.N) || iters < 1 || iters > 1000)
+    return MUSE_ERR_INVALID_ARG;
+  const size_t need = ws_forward(d, Cq, Ck);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
+  const int P = d.B * d.H;
+  MuseTables mt;
+  mt.q = whole_side(d.N, Cq);
+  mt.k = whole_side(d.N, Ck);
+  mt.in = whole_inst(d.N, Cq, Ck);
+  Bump bp(ws);
+  KmWs kw;
+  plan_kmeans_pair(bp, mt, d, P, kw);
+  RefineWs r;
+  plan_refine(bp, mt, d, P, r, true);
+  cudaStream_t cs = (cudaStream_t)st;
+  int *stat = status_ptr();
+  if (run_kmeans(Q, d.dtype, d.D, d.N, mt.q, P, iters, kw.q, kw.scratch, stat, cs) != cudaSuccess)
+    return MUSE_ERR_CUDA;
+  if (run_kmeans(K, d.dtype, d.D, d.N, mt.k, P, iters, kw.k, kw.scratch, stat, cs) != cudaSuccess)
+    return MUSE_ERR_CUDA;
+  return refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets, kw.k.perm,
+                     kw.k.offsets, nullptr, nullptr, r, O, nullptr, nullptr, cs);
+}
+
+// --------------------------------------------------------------------------- causal
+
+extern "C" muse_status muse_causal_blocks(const void *Q, const void *K, const void *V,
+                                          muse_dims d, int block, int Cq, int Ck, int iters,
+                                          void *O, int32_t *q_labels_out, int32_t *k_labels_out,
+                                          void *ws, size_t ws_bytes, muse_stream_t st) {
+  muse_status s = check_dims(d, true);
+  if (s != MUSE_OK) return s;
+  const void *ptrs[] = {Q, K, V, O};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  if ((q_labels_out && !aligned16(q_labels_out)) || (k_labels_out && !aligned16(k_labels_out)))
+    return MUSE_ERR_INVALID_ARG;
+  if (block <= 0 || block % 64 || d.N % block) return MUSE_ERR_SHAPE;
+  if (Cq < 1 || Ck < 1 || Cq > kMaxClusters || Ck > kMaxClusters || iters < 1 || iters > 1000)
+    return MUSE_ERR_INVALID_ARG;
+  if (causal_squares(d.N, block).size() > (size_t)kMaxSeg) return MUSE_ERR_SHAPE;
+  const int P = d.B * d.H;
+  const int levels = muse_causal_levels(d.N, block);
+  cudaStream_t cs = (cudaStream_t)st;
+  if (levels == 0) {
+    // one block: the diagonal is the whole causal attention
+    if (run_diag_merge(Q, K, V, d.dtype, d.D, d.Dv, d.N, P, block, 0, d.scale, nullptr, nullptr,
+                       O, cs) != cudaSuccess)
+      return MUSE_ERR_CUDA;
+    return MUSE_OK;
+  }
+  MuseTables mt;
+  int L = 0;
+  build_causal(d.N, block, Cq, Ck, mt, L);
+  if ((int64_t)P * mt.q.nseg > 65535) return MUSE_ERR_SHAPE;
+  const size_t need = ws_causal(d, block, Cq, Ck);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
+  Bump bp(ws);
+  KmWs kw;
+  plan_kmeans_pair(bp, mt, d, P, kw);
+  RefineWs r;
+  plan_refine(bp, mt, d, P, r, true);
+  float *part_o = bp.take<float>((size_t)P * L * d.N * d.Dv);
+  float *part_lse = bp.take<float>((size_t)P * L * d.N);
+  if (q_labels_out) kw.q.labels = q_labels_out;
+  if (k_labels_out) kw.k.labels = k_labels_out;
+  // rows outside every square of a level keep label -1
+  if (cudaMemsetAsync(kw.q.labels, 0xff, (size_t)P * L * d.N * sizeof(int32_t), cs) != cudaSuccess ||
+      cudaMemsetAsync(kw.k.labels, 0xff, (size_t)P * L * d.N * sizeof(int32_t), cs) != cudaSuccess)
+    return MUSE_ERR_CUDA;
+  int *stat = status_ptr();
+  if (run_kmeans(Q, d.dtype, d.D, d.N, mt.q, P, iters, kw.q, kw.scratch, stat, cs) != cudaSuccess)
+    return MUSE_ERR_CUDA;
+  if (run_kmeans(K, d.dtype, d.D, d.N, mt.k, P, iters, kw.k, kw.scratch, stat, cs) != cudaSuccess)
+    return MUSE_ERR_CUDA;
+  s = refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets, kw.k.perm,
+                  kw.k.offsets, nullptr, nullptr, r, nullptr, part_o, part_lse, cs);
+  if (s != MUSE_OK) return s;
+  if (run_diag_merge(Q, K, V, d.dtype, d.D, d.Dv, d.N, P, block, L, d.scale, part_o, part_lse, O,
+                     cs) != cudaSuccess)
+    return MUSE_ERR_CUDA;
+  return MUSE_OK;
+}

@@ -1,0 +1,593 @@
+// Stage kernels (CUDA cores) of the MuSe forward pass, batched over
+// (problem, instance): sorted copies, tilt logits / log-normalisers / weights,
+// tilted moments, the refinement coefficients, and the refinement itself.
+//
+// Stage 1 (tilted monopole summaries and dipole): pith.science review of arXiv
+// 2509.10406, "What carries the argument" and "Assumptions & free parameters"
+// (M_j(q) = E exp(q.k)); referee minor comment on Algorithm 3 (tilted Cov_ij(v,k)).
+// Stage 2 (refinement that drops only qt.kt): same page, "What carries the
+// argument"; gist.science "Technische Samenvatting", "Kernmechanismen" 1-2.
+//
+// The refinement uses the identity
+//   mu_v,ij + s C_ij qt = sum_{k in S_j} w_ik (1 - s qt.mu_k,ij + s qt.k) v_k
+// (the weights w_ik sum to one and sum_k w_ik (k - mu_k,ij) = 0), so with
+//   c0_nj = p_nj (1 - s u_nj),  c1_nj = s p_nj,  u_nj = qt_n.mu_k,ij,
+//   O_n = sum_k w_{i(n),k} (c0_{n,j(k)} + c1_{n,j(k)} qt_n.k) v_k :
+// two contractions over the cluster-sorted keys with an element-wise step between
+// them, and C_ij is never formed.
+#include "internal.h"
+
+namespace muse {
+
+__device__ __forceinline__ Task q_task(const MuseTables &mt, int p, int s) {
+  return make_task(mt.q, p * mt.q.nseg + s);
+}
+__device__ __forceinline__ Task k_task(const MuseTables &mt, int p, int s) {
+  return make_task(mt.k, p * mt.k.nseg + s);
+}
+
+// ---------------------------------------------------------------------------
+// Sorted copies: position m of a task's perm holds row perm[m] (minus its
+// cluster's centroid when `centroids` is given: the query residuals).
+// One CTA per (cluster, task).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void sort_side(const T *__restrict__ X, int N, int W, SegTable tab,
+                          const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
+                          const float *__restrict__ centroids, T *__restrict__ rows,
+                          int32_t *__restrict__ cluster) {
+  const Task tk = make_task(tab, blockIdx.y);
+  const int c = blockIdx.x;
+  if (c >= tk.C) return;
+  const int b = offsets[tk.off + c], e = offsets[tk.off + c + 1];
+  const float *cen = centroids ? centroids + (tk.cen + c) * W : nullptr;
+  for (int m = b; m < e; ++m) {
+    const int row = perm[tk.lab + m];
+    const T *src = X + ((int64_t)tk.p * N + row) * W;
+    T *dst = rows + (tk.lab + m) * W;
+    for (int d = threadIdx.x; d < W; d += blockDim.x) {
+      float v = ld_elem(src + d);
+      if (cen) v -= cen[d];
+      st_elem(dst + d, v);
+    }
+    if (threadIdx.x == 0) cluster[tk.lab + m] = c;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tilt logits W[i][pos] = s qbar_i . k_pos over the sorted keys (64 x 64 tiles).
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+tilt_logits(MuseTables mt, float scale, const float *__restrict__ qcen, const T *__restrict__ ks,
+            float *__restrict__ W) {
+  const int p = blockIdx.z / mt.in.ninst, s = blockIdx.z % mt.in.ninst;
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int Cq = q.C, nk = k.n;
+  const int i0 = blockIdx.y * 64, k0 = blockIdx.x * 64;
+  if (i0 >= Cq || k0 >= nk) return;
+  __shared__ float As[32][65];
+  __shared__ float Bs[32][65];
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const float *qc = qcen + (q.cen + i0) * D;
+  const T *kr = ks + (k.lab + k0) * D;
+  for (int d0 = 0; d0 < D; d0 += 32) {
+    for (int e = threadIdx.x; e < 64 * 32; e += 256) {
+      const int r = e >> 5, dd = e & 31;
+      As[dd][r] = (i0 + r < Cq) ? qc[(int64_t)r * D + d0 + dd] : 0.f;
+      Bs[dd][r] = (k0 + r < nk) ? ld_elem(kr + (int64_t)r * D + d0 + dd) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int dd = 0; dd < 32; ++dd) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) av[a] = As[dd][ty * 4 + a];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) bv[b] = Bs[dd][tx * 4 + b];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
+    }
+    __syncthreads();
+  }
+  float *wo = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + ty * 4 + a;
+    if (i >= Cq) continue;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int kk = k0 + tx * 4 + b;
+      if (kk < nk) wo[(int64_t)i * nk + kk] = scale * acc[a][b];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// logZ_ij = logsumexp of W[i][S_j] (one warp per (i, j)), then W <- exp(W - logZ).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+tilt_lse(MuseTables mt, const int32_t *__restrict__ k_offsets, float *__restrict__ W,
+         float *__restrict__ logZ) {
+  const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int Cq = q.C, Ck = k.C, nk = k.n;
+  const int wid = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (wid >= Cq * Ck) return;
+  const int i = wid / Ck, j = wid % Ck;
+  const int b = k_offsets[k.off + j], e = k_offsets[k.off + j + 1];
+  float *w = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * nk;
+  float m = -CUDART_INF_F;
+  for (int pos = b + lane; pos < e; pos += 32) m = fmaxf(m, w[pos]);
+  m = warp_max(m);
+  float l = 0.f;
+  for (int pos = b + lane; pos < e; pos += 32) l += expf(w[pos] - m);
+  l = warp_sum(l);
+  const float lz = (e > b) ? m + logf(l) : -CUDART_INF_F;
+  for (int pos = b + lane; pos < e; pos += 32) w[pos] = expf(w[pos] - lz);
+  if (lane == 0) logZ[(int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck + j] = lz;
+}
+
+// ---------------------------------------------------------------------------
+// W <- exp(W - logZ[i][j(pos)]) for externally supplied log-normalisers.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+tilt_weights(MuseTables mt, const int32_t *__restrict__ k_cluster, const float *__restrict__ logZ,
+             float *__restrict__ W) {
+  const int p = blockIdx.z / mt.in.ninst, s = blockIdx.z % mt.in.ninst;
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int i = blockIdx.y;
+  if (i >= q.C) return;
+  const int pos = blockIdx.x * 256 + threadIdx.x;
+  if (pos >= k.n) return;
+  const int j = k_cluster[k.lab + pos];
+  const float lz = logZ[(int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * k.C + j];
+  float *w = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * k.n + pos;
+  *w = expf(*w - lz);
+}
+
+// ---------------------------------------------------------------------------
+// Tilted means mu[i][j][:] = sum_{pos in S_j} w_i,pos x_pos (x = keys or values).
+// CTA per (j, group of 32 query centroids); a warp handles 4 centroids, lanes
+// cover the coordinates.
+// ---------------------------------------------------------------------------
+template <typename T, int WD>
+__global__ void __launch_bounds__(256)
+tilt_moments(MuseTables mt, const int32_t *__restrict__ k_offsets, const float *__restrict__ W,
+             const T *__restrict__ xs, float *__restrict__ mu) {
+  const int p = blockIdx.z / mt.in.ninst, s = blockIdx.z % mt.in.ninst;
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int Cq = q.C, Ck = k.C, nk = k.n;
+  const int j = blockIdx.x;
+  if (j >= Ck) return;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int ib = blockIdx.y * 32 + wid * 4;
+  if (ib >= Cq) return;
+  const int b = k_offsets[k.off + j], e = k_offsets[k.off + j + 1];
+  constexpr int PER = WD / 32;
+  float acc[4][PER];
+#pragma unroll
+  for (int t = 0; t < 4; ++t)
+#pragma unroll
+    for (int u = 0; u < PER; ++u) acc[t][u] = 0.f;
+  const float *wb = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s];
+  for (int pos = b; pos < e; ++pos) {
+    float xv[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) xv[u] = ld_elem(xs + (k.lab + pos) * WD + lane + 32 * u);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int i = ib + t;
+      const float w = (i < Cq) ? wb[(int64_t)i * nk + pos] : 0.f;
+#pragma unroll
+      for (int u = 0; u < PER; ++u) acc[t][u] = fmaf(w, xv[u], acc[t][u]);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int i = ib + t;
+    if (i >= Cq) continue;
+    float *o = mu + ((int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck + j) * WD;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) o[lane + 32 * u] = acc[t][u];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tilted dipole C_ij = sum_k w (v - mu_v)(k - mu_k)^T, centred (inspection only:
+// the forward pass never materialises it).  CTA per (j, i, task).
+// ---------------------------------------------------------------------------
+template <typename T, int D, int DV>
+__global__ void __launch_bounds__(256)
+tilt_cov(MuseTables mt, const int32_t *__restrict__ k_offsets, const float *__restrict__ W,
+         const T *__restrict__ ks, const T *__restrict__ vs, const float *__restrict__ mu_k,
+         const float *__restrict__ mu_v, float *__restrict__ cov) {
+  const int p = blockIdx.z / mt.in.ninst, s = blockIdx.z % mt.in.ninst;
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int Cq = q.C, Ck = k.C, nk = k.n;
+  const int j = blockIdx.x, i = blockIdx.y;
+  if (j >= Ck || i >= Cq) return;
+  const int b = k_offsets[k.off + j], e = k_offsets[k.off + j + 1];
+  const int64_t z = (int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck + j;
+  const float *mk = mu_k + z * D;
+  const float *mv = mu_v + z * DV;
+  const float *w = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * nk;
+  float *out = cov + z * DV * D;
+  for (int e2 = threadIdx.x; e2 < DV * D; e2 += blockDim.x) {
+    const int dv = e2 / D, d = e2 % D;
+    float acc = 0.f;
+    for (int pos = b; pos < e; ++pos)
+      acc = fmaf(w[pos] * (ld_elem(vs + (k.lab + pos) * DV + dv) - mv[dv]),
+                 ld_elem(ks + (k.lab + pos) * D + d) - mk[d], acc);
+    out[e2] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Refinement coefficients for every sorted query position n of cluster i:
+//   a_j = logZ_ij + s u_j, u_j = qt.mu_k,ij;  p = softmax_j(a);
+//   c0[j][n] = p_j (1 - s u_j), c1[j][n] = s p_j,  lse[n] = logsumexp_j a_j.
+// CTA per (query cluster, task), one thread per query.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128)
+refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
+              const int32_t *__restrict__ q_offsets, const float *__restrict__ logZ,
+              const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
+              float *__restrict__ lse) {
+  extern __shared__ float sm[];
+  const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int Cq = q.C, Ck = k.C, nq = q.n;
+  const int i = blockIdx.x;
+  if (i >= Cq) return;
+  const int b = q_offsets[q.off + i], e = q_offsets[q.off + i + 1];
+  if (e <= b) return;
+  float *lz = sm;               // [Ck]
+  float *mk = sm + kMaxClusters;  // [32][D]
+  const int64_t zrow = (int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck;
+  for (int j = threadIdx.x; j < Ck; j += blockDim.x) lz[j] = logZ[zrow + j];
+  float *C0 = c0 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
+  float *C1 = c1 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
+  for (int n0 = b; n0 < e; n0 += blockDim.x) {
+    const int n = n0 + threadIdx.x;
+    const bool v = n < e;
+    float qt[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) qt[d] = v ? ld_elem(qt_rows + (q.lab + n) * D + d) : 0.f;
+    float m = -CUDART_INF_F;
+    for (int j0 = 0; j0 < Ck; j0 += 32) {
+      const int jt = min(32, Ck - j0);
+      __syncthreads();
+      for (int e2 = threadIdx.x; e2 < jt * D; e2 += blockDim.x)
+        mk[e2] = mu_k[(zrow + j0) * D + e2];
+      __syncthreads();
+      if (v) {
+        for (int jj = 0; jj < jt; ++jj) {
+          float u = 0.f;
+#pragma unroll
+          for (int d = 0; d < D; ++d) u = fmaf(qt[d], mk[jj * D + d], u);
+          const int j = j0 + jj;
+          const float a = lz[j] + scale * u;
+          C0[(int64_t)j * nq + n] = a;
+          C1[(int64_t)j * nq + n] = u;
+          m = fmaxf(m, a);
+        }
+      }
+    }
+    if (v) {
+      float l = 0.f;
+      for (int j = 0; j < Ck; ++j) l += expf(C0[(int64_t)j * nq + n] - m);
+      const float inv = 1.f / l;
+      for (int j = 0; j < Ck; ++j) {
+        const float a = C0[(int64_t)j * nq + n];
+        const float u = C1[(int64_t)j * nq + n];
+        const float pj = expf(a - m) * inv;
+        C0[(int64_t)j * nq + n] = pj * (1.f - scale * u);
+        C1[(int64_t)j * nq + n] = scale * pj;
+      }
+      lse[(int64_t)p * mt.q.row_stride + q.lab + n] = m + logf(l);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Refinement on CUDA cores: 64 sorted queries per CTA, 4 threads per query
+// (coordinates interleaved by 4), keys staged 32 at a time.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int DV>
+__global__ void __launch_bounds__(256)
+refine_simt(MuseTables mt, int N, const T *__restrict__ qt_rows, const int32_t *__restrict__ q_perm,
+            const int32_t *__restrict__ q_cluster, const T *__restrict__ ks,
+            const int32_t *__restrict__ k_cluster, const T *__restrict__ vs,
+            const float *__restrict__ W, const float *__restrict__ c0,
+            const float *__restrict__ c1, const float *__restrict__ lse, T *__restrict__ O,
+            float *__restrict__ part_o, float *__restrict__ part_lse) {
+  const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int nq = q.n, nk = k.n;
+  const int n0 = blockIdx.x * 64;
+  if (n0 >= nq) return;
+  __shared__ float Ks[32][D];
+  __shared__ float Vs[32][DV];
+  __shared__ int Js[32];
+  const int g = threadIdx.x & 3;
+  const int n = n0 + (threadIdx.x >> 2);
+  const bool v = n < nq;
+  constexpr int PD = D / 4, PV = DV / 4;
+  float qt[PD];
+#pragma unroll
+  for (int t = 0; t < PD; ++t) qt[t] = v ? ld_elem(qt_rows + (q.lab + n) * D + g + 4 * t) : 0.f;
+  const int i = v ? q_cluster[q.lab + n] : 0;
+  const float *wrow = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * nk;
+  const float *C0 = c0 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
+  const float *C1 = c1 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
+  float acc[PV];
+#pragma unroll
+  for (int t = 0; t < PV; ++t) acc[t] = 0.f;
+  int curj = -1;
+  float a0 = 0.f, a1 = 0.f;
+  for (int k0 = 0; k0 < nk; k0 += 32) {
+    const int kt = min(32, nk - k0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < kt * D; e += blockDim.x)
+      Ks[e / D][e % D] = ld_elem(ks + (k.lab + k0) * D + e);
+    for (int e = threadIdx.x; e < kt * DV; e += blockDim.x)
+      Vs[e / DV][e % DV] = ld_elem(vs + (k.lab + k0) * DV + e);
+    if (threadIdx.x < kt) Js[threadIdx.x] = k_cluster[k.lab + k0 + threadIdx.x];
+    __syncthreads();
+    for (int kk = 0; kk < kt; ++kk) {
+      float x = 0.f;
+#pragma unroll
+      for (int t = 0; t < PD; ++t) x = fmaf(qt[t], Ks[kk][g + 4 * t], x);
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
+      const int j = Js[kk];
+      if (j != curj) {
+        curj = j;
+        a0 = v ? C0[(int64_t)j * nq + n] : 0.f;
+        a1 = v ? C1[(int64_t)j * nq + n] : 0.f;
+      }
+      const float P = v ? wrow[k0 + kk] * fmaf(a1, x, a0) : 0.f;
+#pragma unroll
+      for (int t = 0; t < PV; ++t) acc[t] = fmaf(P, Vs[kk][g + 4 * t], acc[t]);
+    }
+  }
+  if (!v) return;
+  const int row = q_perm[q.lab + n];
+  if (O) {
+    T *o = O + ((int64_t)p * N + row) * DV;
+#pragma unroll
+    for (int t = 0; t < PV; ++t) st_elem(o + g + 4 * t, acc[t]);
+  } else {
+    const int64_t r = (int64_t)p * mt.in.out_stride + mt.in.out0[s] + row;
+#pragma unroll
+    for (int t = 0; t < PV; ++t) part_o[r * DV + g + 4 * t] = acc[t];
+    if (g == 0) part_lse[r] = lse[(int64_t)p * mt.q.row_stride + q.lab + n];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Causal: exact attention inside each diagonal block (keys [b*S, n]) merged with
+// the level partials of the squares that hold the row (levels whose bit of b is
+// set).  64 queries per CTA, 4 threads per query.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int DV>
+__global__ void __launch_bounds__(256)
+diag_merge(const T *__restrict__ Qg, const T *__restrict__ Kg, const T *__restrict__ Vg, int N,
+           int block, int levels, float scale, const float *__restrict__ part_o,
+           const float *__restrict__ part_lse, T *__restrict__ O) {
+  const int p = blockIdx.y;
+  const int n0 = blockIdx.x * 64;
+  const int bidx = n0 / block;
+  const int ks0 = bidx * block;
+  __shared__ float Ks[32][D];
+  __shared__ float Vs[32][DV];
+  const int g = threadIdx.x & 3;
+  const int n = n0 + (threadIdx.x >> 2);
+  constexpr int PD = D / 4, PV = DV / 4;
+  const T *Qp = Qg + (int64_t)p * N * D;
+  const T *Kp = Kg + (int64_t)p * N * D;
+  const T *Vp = Vg + (int64_t)p * N * DV;
+  float qv[PD];
+#pragma unroll
+  for (int t = 0; t < PD; ++t) qv[t] = ld_elem(Qp + (int64_t)n * D + g + 4 * t) * scale;
+  float m = -CUDART_INF_F, l = 0.f;
+  float acc[PV];
+#pragma unroll
+  for (int t = 0; t < PV; ++t) acc[t] = 0.f;
+  const int kend = min(n0 + 64, N);
+  for (int k0 = ks0; k0 < kend; k0 += 32) {
+    const int kt = min(32, kend - k0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < kt * D; e += blockDim.x)
+      Ks[e / D][e % D] = ld_elem(Kp + (int64_t)k0 * D + e);
+    for (int e = threadIdx.x; e < kt * DV; e += blockDim.x)
+      Vs[e / DV][e % DV] = ld_elem(Vp + (int64_t)k0 * DV + e);
+    __syncthreads();
+    for (int kk = 0; kk < kt; ++kk) {
+      float x = 0.f;
+#pragma unroll
+      for (int t = 0; t < PD; ++t) x = fmaf(qv[t], Ks[kk][g + 4 * t], x);
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
+      if (k0 + kk <= n) {
+        const float mn = fmaxf(m, x);
+        const float corr = expf(m - mn);
+        const float pe = expf(x - mn);
+        l = l * corr + pe;
+#pragma unroll
+        for (int t = 0; t < PV; ++t) acc[t] = fmaf(pe, Vs[kk][g + 4 * t], acc[t] * corr);
+        m = mn;
+      }
+    }
+  }
+  for (int lev = 1; lev <= levels; ++lev) {
+    if (!((bidx >> (lev - 1)) & 1)) continue;
+    const int64_t r = ((int64_t)p * levels + (lev - 1)) * N + n;
+    const float L = part_lse[r];
+    if (!(L > -CUDART_INF_F)) continue;
+    const float mn = fmaxf(m, L);
+    const float ca = expf(m - mn), cb = expf(L - mn);
+    l = l * ca + cb;
+#pragma unroll
+    for (int t = 0; t < PV; ++t) acc[t] = acc[t] * ca + cb * part_o[r * DV + g + 4 * t];
+    m = mn;
+  }
+  const float inv = 1.f / l;
+  T *o = O + ((int64_t)p * N + n) * DV;
+#pragma unroll
+  for (int t = 0; t < PV; ++t) st_elem(o + g + 4 * t, acc[t] * inv);
+}
+
+// ===========================================================================
+// Host launchers
+// ===========================================================================
+
+cudaError_t run_sort_side(const void *X, int dtype, int width, int N, const SegTable &tab, int P,
+                          const int32_t *perm, const int32_t *offsets, const float *centroids,
+                          SortedSide out, cudaStream_t st) {
+  dim3 grid(tab.max_C, P * tab.nseg);
+  const int threads = width;
+  count_launches(1);
+  if (dtype == MUSE_F32)
+    sort_side<float><<<grid, threads, 0, st>>>((const float *)X, N, width, tab, perm, offsets,
+                                               centroids, (float *)out.rows, out.cluster);
+  else
+    sort_side<__nv_bfloat16><<<grid, threads, 0, st>>>(
+        (const __nv_bfloat16 *)X, N, width, tab, perm, offsets, centroids,
+        (__nv_bfloat16 *)out.rows, out.cluster);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int DV>
+static cudaError_t summaries_t(const MuseTables &mt, int P, float scale, const float *qcen,
+                               SortedSide ks, const void *vs, const int32_t *k_offsets,
+                               StageBufs b, cudaStream_t st) {
+  const int tasks = P * mt.in.ninst;
+  const int maxCq = mt.q.max_C, maxCk = mt.k.max_C, maxnk = mt.k.max_rows;
+  tilt_logits<T, D><<<dim3((maxnk + 63) / 64, (maxCq + 63) / 64, tasks), 256, 0, st>>>(
+      mt, scale, qcen, (const T *)ks.rows, b.W);
+  tilt_lse<<<dim3((maxCq * maxCk + 7) / 8, tasks), 256, 0, st>>>(mt, k_offsets, b.W, b.logZ);
+  count_launches(2 + (b.mu_k != nullptr) + (b.mu_v != nullptr) + (b.cov != nullptr));
+  if (b.mu_k)
+    tilt_moments<T, D><<<dim3(maxCk, (maxCq + 31) / 32, tasks), 256, 0, st>>>(
+        mt, k_offsets, b.W, (const T *)ks.rows, b.mu_k);
+  if (b.mu_v)
+    tilt_moments<T, DV><<<dim3(maxCk, (maxCq + 31) / 32, tasks), 256, 0, st>>>(
+        mt, k_offsets, b.W, (const T *)vs, b.mu_v);
+  if (b.cov)
+    tilt_cov<T, D, DV><<<dim3(maxCk, maxCq, tasks), 256, 0, st>>>(
+        mt, k_offsets, b.W, (const T *)ks.rows, (const T *)vs, b.mu_k, b.mu_v, b.cov);
+  return cudaGetLastError();
+}
+
+#define MUSE_DISPATCH_DDV(dtype, D, Dv, FN, ...)                                        \
+  do {                                                                                  \
+    if ((dtype) == MUSE_F32) {                                                          \
+      if ((D) == 64 && (Dv) == 64) return FN<float, 64, 64>(__VA_ARGS__);               \
+      if ((D) == 64 && (Dv) == 128) return FN<float, 64, 128>(__VA_ARGS__);             \
+      if ((D) == 128 && (Dv) == 64) return FN<float, 128, 64>(__VA_ARGS__);             \
+      return FN<float, 128, 128>(__VA_ARGS__);                                          \
+    }                                                                                   \
+    if ((D) == 64 && (Dv) == 64) return FN<__nv_bfloat16, 64, 64>(__VA_ARGS__);         \
+    if ((D) == 64 && (Dv) == 128) return FN<__nv_bfloat16, 64, 128>(__VA_ARGS__);       \
+    if ((D) == 128 && (Dv) == 64) return FN<__nv_bfloat16, 128, 64>(__VA_ARGS__);       \
+    return FN<__nv_bfloat16, 128, 128>(__VA_ARGS__);                                    \
+  } while (0)
+
+cudaError_t run_summaries(const MuseTables &mt, int dtype, int D, int Dv, int P, float scale,
+                          const float *q_centroids, SortedSide ks, const void *vs_rows,
+                          const int32_t *k_offsets, StageBufs b, cudaStream_t st) {
+  MUSE_DISPATCH_DDV(dtype, D, Dv, summaries_t, mt, P, scale, q_centroids, ks, vs_rows, k_offsets,
+                    b, st);
+}
+
+template <typename T, int D>
+static cudaError_t weights_t(const MuseTables &mt, int P, float scale, const float *qcen,
+                             SortedSide ks, const float *logZ, float *W, cudaStream_t st) {
+  const int tasks = P * mt.in.ninst;
+  tilt_logits<T, D><<<dim3((mt.k.max_rows + 63) / 64, (mt.q.max_C + 63) / 64, tasks), 256, 0,
+                      st>>>(mt, scale, qcen, (const T *)ks.rows, W);
+  tilt_weights<<<dim3((mt.k.max_rows + 255) / 256, mt.q.max_C, tasks), 256, 0, st>>>(
+      mt, ks.cluster, logZ, W);
+  count_launches(2);
+  return cudaGetLastError();
+}
+
+cudaError_t run_tilt_weights(const MuseTables &mt, int dtype, int D, int P, float scale,
+                             const float *q_centroids, SortedSide ks, const float *logZ, float *W,
+                             cudaStream_t st) {
+  if (dtype == MUSE_F32)
+    return D == 64 ? weights_t<float, 64>(mt, P, scale, q_centroids, ks, logZ, W, st)
+                   : weights_t<float, 128>(mt, P, scale, q_centroids, ks, logZ, W, st);
+  return D == 64 ? weights_t<__nv_bfloat16, 64>(mt, P, scale, q_centroids, ks, logZ, W, st)
+                 : weights_t<__nv_bfloat16, 128>(mt, P, scale, q_centroids, ks, logZ, W, st);
+}
+
+template <typename T, int D>
+static cudaError_t coeffs_t(const MuseTables &mt, int P, float scale, SortedSide qs,
+                            const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
+  const size_t smem = (kMaxClusters + 32 * D) * sizeof(float);
+  cudaError_t err = cudaFuncSetAttribute(refine_coeffs<T, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  refine_coeffs<T, D><<<dim3(mt.q.max_C, P * mt.in.ninst), 128, smem, st>>>(
+      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t run_coeffs(const MuseTables &mt, int dtype, int D, int P, float scale, SortedSide qs,
+                       const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
+  if (dtype == MUSE_F32)
+    return D == 64 ? coeffs_t<float, 64>(mt, P, scale, qs, q_offsets, b, st)
+                   : coeffs_t<float, 128>(mt, P, scale, qs, q_offsets, b, st);
+  return D == 64 ? coeffs_t<__nv_bfloat16, 64>(mt, P, scale, qs, q_offsets, b, st)
+                 : coeffs_t<__nv_bfloat16, 128>(mt, P, scale, qs, q_offsets, b, st);
+}
+
+template <typename T, int D, int DV>
+static cudaError_t refine_t(const MuseTables &mt, int N, int P, SortedSide qs,
+                            const int32_t *q_perm, SortedSide ks, const void *vs, StageBufs b,
+                            void *O, float *part_o, float *part_lse, cudaStream_t st) {
+  dim3 grid((mt.q.max_rows + 63) / 64, P * mt.in.ninst);
+  refine_simt<T, D, DV><<<grid, 256, 0, st>>>(
+      mt, N, (const T *)qs.rows, q_perm, qs.cluster, (const T *)ks.rows, ks.cluster,
+      (const T *)vs, b.W, b.c0, b.c1, b.lse, (T *)O, part_o, part_lse);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t run_refine(const MuseTables &mt, int dtype, int D, int Dv, int N, int P,
+                       SortedSide qs, const int32_t *q_perm, SortedSide ks, const void *vs_rows,
+                       StageBufs b, void *O, float *part_o, float *part_lse, cudaStream_t st) {
+  MUSE_DISPATCH_DDV(dtype, D, Dv, refine_t, mt, N, P, qs, q_perm, ks, vs_rows, b, O, part_o,
+                    part_lse, st);
+}
+
+template <typename T, int D, int DV>
+static cudaError_t diag_t(const void *Q, const void *K, const void *V, int N, int P, int block,
+                          int levels, float scale, const float *part_o, const float *part_lse,
+                          void *O, cudaStream_t st) {
+  diag_merge<T, D, DV><<<dim3(N / 64, P), 256, 0, st>>>(
+      (const T *)Q, (const T *)K, (const T *)V, N, block, levels, scale, part_o, part_lse, (T *)O);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t run_diag_merge(const void *Q, const void *K, const void *V, int dtype, int D, int Dv,
+                           int N, int P, int block, int levels, float scale,
+                           const float *part_o, const float *part_lse, void *O, cudaStream_t st) {
+  MUSE_DISPATCH_DDV(dtype, D, Dv, diag_t, Q, K, V, N, P, block, levels, scale, part_o, part_lse,
+                    O, st);
+}
+
+}  // namespace muse

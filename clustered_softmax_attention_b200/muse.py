@@ -1,0 +1,262 @@
+"""Python binding of libmuse.so (ctypes).  Argument marshalling only.
+
+Every function here has the name of the C entry point it calls (include/muse.h)
+and does nothing but check shapes, allocate the caller-owned outputs and
+workspace with torch, and pass device pointers plus the current CUDA stream.
+All arithmetic runs in the library's CUDA kernels; if the library is missing,
+the import of this module fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmuse.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "muse.h")
+
+MUSE_F32, MUSE_BF16 = 0, 1
+STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_SHAPE", 3: "MUSE_ERR_DTYPE",
+          4: "MUSE_ERR_WORKSPACE", 5: "MUSE_ERR_CUDA", 6: "MUSE_ERR_TIMEOUT", 7: "MUSE_ERR_DEVICE"}
+
+
+class MuseError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class MuseDims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
+                ("D", ctypes.c_int), ("Dv", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("scale", ctypes.c_float)]
+
+
+_vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_SIGS = {
+    "muse_kmeans": [_vp, MuseDims, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
+    "muse_tilted_summaries": [_vp, _vp, _vp, _vp, _vp, MuseDims, _i, _i, _vp, _vp, _vp, _vp,
+                              _vp, _sz, _vp],
+    "muse_dipole_refine": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, MuseDims, _i, _i,
+                           _vp, _vp, _sz, _vp],
+    "muse_forward": [_vp, _vp, _vp, MuseDims, _i, _i, _i, _vp, _vp, _sz, _vp],
+    "muse_causal_levels": [_i, _i],
+    "muse_causal_blocks": [_vp, _vp, _vp, MuseDims, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz,
+                           _vp],
+    "muse_retrieve_exact": [_vp, _vp, _vp, MuseDims, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp,
+                            _vp, _sz, _vp],
+    "muse_workspace_size": [ctypes.c_char_p, MuseDims, _i, _i, _i, _i, _i],
+    "muse_status_string": [_i],
+    "muse_last_device_status": [_vp],
+}
+_RES = {"muse_workspace_size": _sz, "muse_status_string": ctypes.c_char_p,
+        "muse_causal_levels": _i}
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m clustered_softmax_attention_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, args in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = _RES.get(name, _i)
+    return lib
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is None:
+        _LIB = load_library()
+    return _LIB
+
+
+def declared_entry_points(header: str = HEADER):
+    """Names of the functions declared in include/muse.h."""
+    text = open(header).read()
+    return sorted(set(re.findall(r"^\s*(?:muse_status|size_t|int|const char \*)\s*\**(muse_\w+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise MuseError(code, where)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MUSE_F32
+    if t.dtype == torch.bfloat16:
+        return MUSE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def dims(X: torch.Tensor, V: Optional[torch.Tensor] = None, scale: float = 1.0) -> MuseDims:
+    B, H, N, D = X.shape
+    Dv = V.shape[-1] if V is not None else D
+    return MuseDims(B, H, N, D, Dv, _dtype_code(X), float(scale))
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def muse_workspace_size(entry: str, d: MuseDims, Cq: int, Ck: int = 0, block: int = 0,
+                        k1: int = 0, k2: int = 0) -> int:
+    return int(lib().muse_workspace_size(entry.encode(), d, Cq, Ck, block, k1, k2))
+
+
+def workspace(entry: str, d: MuseDims, Cq: int, Ck: int = 0, block: int = 0, k1: int = 0,
+              k2: int = 0, device="cuda") -> torch.Tensor:
+    n = muse_workspace_size(entry, d, Cq, Ck, block, k1, k2)
+    if n == 0:
+        raise MuseError(2, f"muse_workspace_size({entry})")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def muse_status_string(code: int) -> str:
+    return lib().muse_status_string(code).decode()
+
+
+def muse_last_device_status() -> int:
+    return int(lib().muse_last_device_status(_stream()))
+
+
+def muse_causal_levels(N: int, block: int) -> int:
+    return int(lib().muse_causal_levels(N, block))
+
+
+def muse_kmeans(X: torch.Tensor, C: int, iters: int, ws: Optional[torch.Tensor] = None):
+    """K-means of every (b,h) row set of X [B,H,N,D]: (labels, centroids, perm, offsets)."""
+    _contig(X)
+    d = dims(X)
+    B, H, N, D = X.shape
+    dev = X.device
+    labels = torch.empty(B, H, N, dtype=torch.int32, device=dev)
+    cen = torch.empty(B, H, C, D, dtype=torch.float32, device=dev)
+    perm = torch.empty(B, H, N, dtype=torch.int32, device=dev)
+    offs = torch.empty(B, H, C + 1, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace("muse_kmeans", d, C)
+    _check(lib().muse_kmeans(_p(X), d, C, iters, _p(labels), _p(cen), _p(perm), _p(offs), _p(ws),
+                             ws.numel(), _stream()), "muse_kmeans")
+    return labels, cen, perm, offs
+
+
+def muse_tilted_summaries(q_centroids, K, V, k_perm, k_offsets, Ck: int, scale: float = 1.0,
+                          want_mu_k: bool = True, want_mu_v: bool = True, want_cov: bool = False):
+    """Stage 1 summaries: dict with logZ and the requested mu_k / mu_v / cov."""
+    _contig(q_centroids, K, V, k_perm, k_offsets)
+    B, H, Cq, D = q_centroids.shape
+    d = dims(K, V, scale)
+    dev = K.device
+    Dv = d.Dv
+    out = {"logZ": torch.empty(B, H, Cq, Ck, dtype=torch.float32, device=dev)}
+    if want_mu_k:
+        out["mu_k"] = torch.empty(B, H, Cq, Ck, D, dtype=torch.float32, device=dev)
+    if want_mu_v:
+        out["mu_v"] = torch.empty(B, H, Cq, Ck, Dv, dtype=torch.float32, device=dev)
+    if want_cov:
+        out["cov"] = torch.empty(B, H, Cq, Ck, Dv, D, dtype=torch.float32, device=dev)
+    ws = workspace("muse_tilted_summaries", d, Cq, Ck)
+    _check(lib().muse_tilted_summaries(
+        _p(q_centroids), _p(K), _p(V), _p(k_perm), _p(k_offsets), d, Cq, Ck, _p(out["logZ"]),
+        _p(out.get("mu_k")), _p(out.get("mu_v")), _p(out.get("cov")), _p(ws), ws.numel(),
+        _stream()), "muse_tilted_summaries")
+    return out
+
+
+def muse_dipole_refine(Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offsets, logZ, mu_k,
+                       scale: float = 1.0):
+    """Stage 2 refinement: O [B,H,N,Dv] in Q's dtype."""
+    _contig(Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offsets, logZ, mu_k)
+    d = dims(Q, V, scale)
+    Cq, Ck = q_centroids.shape[2], logZ.shape[3]
+    O = torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], d.Dv, dtype=Q.dtype, device=Q.device)
+    ws = workspace("muse_dipole_refine", d, Cq, Ck)
+    _check(lib().muse_dipole_refine(
+        _p(Q), _p(K), _p(V), _p(q_centroids), _p(q_perm), _p(q_offsets), _p(k_perm),
+        _p(k_offsets), _p(logZ), _p(mu_k), d, Cq, Ck, _p(O), _p(ws), ws.numel(), _stream()),
+        "muse_dipole_refine")
+    return O
+
+
+def muse_forward(Q, K, V, Cq: int, Ck: int, iters: int, scale: float = 1.0,
+                 out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+    """The whole acausal forward pass."""
+    _contig(Q, K, V, out, ws)
+    d = dims(Q, V, scale)
+    if out is None:
+        out = torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], d.Dv, dtype=Q.dtype, device=Q.device)
+    if ws is None:
+        ws = workspace("muse_forward", d, Cq, Ck)
+    _check(lib().muse_forward(_p(Q), _p(K), _p(V), d, Cq, Ck, iters, _p(out), _p(ws), ws.numel(),
+                              _stream()), "muse_forward")
+    return out
+
+
+def muse_causal_blocks(Q, K, V, block: int, Cq: int, Ck: int, iters: int, scale: float = 1.0,
+                       return_labels: bool = False, out: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None):
+    """Causal MuSe (hierarchical block decomposition).  Labels are [B,H,L,N] (-1 = none)."""
+    _contig(Q, K, V, out, ws)
+    d = dims(Q, V, scale)
+    B, H, N, _ = Q.shape
+    if out is None:
+        out = torch.empty(B, H, N, d.Dv, dtype=Q.dtype, device=Q.device)
+    L = muse_causal_levels(N, block)
+    ql = kl = None
+    if return_labels and L > 0:
+        ql = torch.empty(B, H, L, N, dtype=torch.int32, device=Q.device)
+        kl = torch.empty(B, H, L, N, dtype=torch.int32, device=Q.device)
+    if ws is None:
+        n = muse_workspace_size("muse_causal_blocks", d, Cq, Ck, block)
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=Q.device)
+    _check(lib().muse_causal_blocks(_p(Q), _p(K), _p(V), d, block, Cq, Ck, iters, _p(out), _p(ql),
+                                    _p(kl), _p(ws), ws.numel(), _stream()), "muse_causal_blocks")
+    if return_labels:
+        return out, ql, kl
+    return out
+
+
+def muse_retrieve_exact(Q, K, V, block: int, Cq: int, Ck: int, iters: int, k1: int, k2: int,
+                        scale: float = 1.0, return_all: bool = False,
+                        out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+    """Causal MuSe with top-k1 cluster / top-k2 block retrieval."""
+    _contig(Q, K, V, out, ws)
+    d = dims(Q, V, scale)
+    B, H, N, _ = Q.shape
+    if out is None:
+        out = torch.empty(B, H, N, d.Dv, dtype=Q.dtype, device=Q.device)
+    ql = kl = sel = None
+    if return_all:
+        ql = torch.empty(B, H, N, dtype=torch.int32, device=Q.device)
+        kl = torch.empty(B, H, N, dtype=torch.int32, device=Q.device)
+        sel = torch.empty(B, H, Cq, N // block, max(1, k1 * k2), 2, dtype=torch.int32,
+                          device=Q.device)
+    if ws is None:
+        ws = workspace("muse_retrieve_exact", d, Cq, Ck, block, k1, k2)
+    _check(lib().muse_retrieve_exact(_p(Q), _p(K), _p(V), d, block, Cq, Ck, iters, k1, k2, _p(ql),
+                                     _p(kl), _p(sel), _p(out), _p(ws), ws.numel(), _stream()),
+           "muse_retrieve_exact")
+    if return_all:
+        return out, ql, kl, sel
+    return out

@@ -385,20 +385,25 @@ def diagonal_exact(Q, K, V, S: int, scale: float):
 
 def muse_causal(Q, K, V, S: int, Cq: int, Ck: int, iters: int, scale: float,
                 labels: Optional[Dict[Tuple[int, int], Tuple[np.ndarray, np.ndarray]]] = None,
-                return_labels: bool = False):
+                return_labels: bool = False, rows: Optional[np.ndarray] = None):
     """Causal MuSe: exact diagonal blocks + one acausal MuSe instance per square.
 
     Each square clusters its own query range and key range with
     C_eff = min(C, range length).  ``labels`` maps (level, r) to the (query, key)
     labels of that square (teacher forcing); otherwise K-means runs here.
+    ``rows`` restricts the work to the squares and outputs of those query rows
+    (the other rows of the result are not meaningful).
     """
     Q = np.asarray(Q, np.float64)
     K = np.asarray(K, np.float64)
     V = np.asarray(V, np.float64)
     N = Q.shape[0]
+    rws = None if rows is None else np.asarray(rows)
     parts = [diagonal_exact(Q, K, V, S, scale)]
     used = {}
     for (lev, r, q0, q1, k0, k1) in causal_squares(N, S):
+        if rws is not None and not ((rws >= q0) & (rws < q1)).any():
+            continue
         cq = min(Cq, q1 - q0)
         ck = min(Ck, k1 - k0)
         if labels is not None and (lev, r) in labels:
@@ -408,8 +413,9 @@ def muse_causal(Q, K, V, S: int, Cq: int, Ck: int, iters: int, scale: float,
             ql, qbar = kmeans(Q[q0:q1], cq, iters)
             kl, _ = kmeans(K[k0:k1], ck, iters)
         used[(lev, r)] = (ql, kl)
+        sub = None if rws is None else rws[(rws >= q0) & (rws < q1)] - q0
         o, l = muse_from_labels(Q[q0:q1], K[k0:k1], V[k0:k1], ql, kl, cq, ck, scale,
-                                qbar=qbar, return_lse=True)
+                                qbar=qbar, return_lse=True, rows=sub)
         lse = np.full(N, NEG_INF)
         oo = np.zeros((N, V.shape[1]))
         lse[q0:q1] = l

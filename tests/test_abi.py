@@ -1,0 +1,88 @@
+"""The C-ABI library: it loads, exports every declared entry point, sizes its
+workspace, and rejects bad arguments before launching anything (no GPU needed)."""
+import ctypes
+
+import pytest
+
+from clustered_softmax_attention_b200 import muse as m
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return m.load_library()
+
+
+def test_every_declared_entry_point_is_exported(lib):
+    names = m.declared_entry_points()
+    assert {"muse_kmeans", "muse_tilted_summaries", "muse_dipole_refine", "muse_forward",
+            "muse_causal_blocks", "muse_retrieve_exact", "muse_workspace_size",
+            "muse_status_string", "muse_last_device_status", "muse_causal_levels"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in m.STATUS.items():
+        assert lib.muse_status_string(code).decode() == name
+    assert lib.muse_status_string(99).decode() == "MUSE_ERR_UNKNOWN"
+
+
+def _d(B=1, H=2, N=1024, D=64, Dv=64, dtype=m.MUSE_BF16, scale=1.0):
+    return m.MuseDims(B, H, N, D, Dv, dtype, scale)
+
+
+def test_workspace_sizes(lib):
+    d = _d()
+    for entry in ("muse_kmeans", "muse_tilted_summaries", "muse_dipole_refine", "muse_forward"):
+        assert lib.muse_workspace_size(entry.encode(), d, 32, 32, 0, 0, 0) > 0, entry
+    assert lib.muse_workspace_size(b"muse_causal_blocks", d, 32, 32, 128, 0, 0) > 0
+    assert lib.muse_workspace_size(b"muse_causal_blocks", d, 32, 32, 100, 0, 0) == 0
+    assert lib.muse_workspace_size(b"nope", d, 32, 32, 0, 0, 0) == 0
+    assert lib.muse_workspace_size(b"muse_forward", _d(D=32), 32, 32, 0, 0, 0) == 0
+    assert lib.muse_workspace_size(b"muse_forward", d, 0, 32, 0, 0, 0) == 0
+    assert lib.muse_workspace_size(b"muse_forward", d, 2048, 32, 0, 0, 0) == 0
+    # forward = two clusterings + refinement buffers: grows with N
+    assert (lib.muse_workspace_size(b"muse_forward", _d(N=2048), 32, 32, 0, 0, 0)
+            > lib.muse_workspace_size(b"muse_forward", d, 32, 32, 0, 0, 0))
+
+
+def test_causal_levels(lib):
+    assert lib.muse_causal_levels(16384, 512) == 5
+    assert lib.muse_causal_levels(512, 512) == 0
+    assert lib.muse_causal_levels(1536, 512) == 2
+    assert lib.muse_causal_levels(0, 512) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)       # aligned, never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p((1 << 20) + 4)
+
+
+def test_argument_validation_enqueues_nothing(lib):
+    st = ctypes.c_void_p(0)
+    f = FAKE
+    # wrong dtype / shape
+    assert lib.muse_forward(f, f, f, _d(dtype=7), 8, 8, 2, f, f, 1 << 30, st) == 3
+    assert lib.muse_forward(f, f, f, _d(D=96), 8, 8, 2, f, f, 1 << 30, st) == 2
+    assert lib.muse_forward(f, f, f, _d(Dv=32), 8, 8, 2, f, f, 1 << 30, st) == 2
+    assert lib.muse_forward(f, f, f, _d(N=0), 8, 8, 2, f, f, 1 << 30, st) == 2
+    # null / misaligned pointers, cluster counts, iterations
+    assert lib.muse_forward(None, f, f, _d(), 8, 8, 2, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward(MISALIGNED, f, f, _d(), 8, 8, 2, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward(f, f, f, _d(), 0, 8, 2, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward(f, f, f, _d(N=64), 65, 8, 2, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward(f, f, f, _d(), 8, 8, 0, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward(f, f, f, _d(scale=float("nan")), 8, 8, 2, f, f, 1 << 30, st) == 1
+    # workspace too small or missing
+    assert lib.muse_forward(f, f, f, _d(), 8, 8, 2, f, f, 16, st) == 4
+    assert lib.muse_forward(f, f, f, _d(), 8, 8, 2, f, None, 1 << 30, st) == 4
+    assert lib.muse_kmeans(f, _d(), 8, 2, f, f, f, f, f, 0, st) == 4
+    assert lib.muse_kmeans(f, _d(), 8, 2, None, f, f, f, f, 1 << 30, st) == 1
+    assert lib.muse_kmeans(f, _d(), 8, 1001, f, f, f, f, f, 1 << 30, st) == 1
+    assert lib.muse_tilted_summaries(f, f, None, f, f, _d(), 8, 8, f, None, f, None, f, 1 << 30,
+                                     st) == 1
+    assert lib.muse_dipole_refine(f, f, f, f, f, f, f, f, f, None, _d(), 8, 8, f, f, 1 << 30,
+                                  st) == 1
+    assert lib.muse_causal_blocks(f, f, f, _d(), 100, 8, 8, 2, f, None, None, f, 1 << 30, st) == 2
+    assert lib.muse_causal_blocks(f, f, f, _d(N=1000), 128, 8, 8, 2, f, None, None, f, 1 << 30,
+                                  st) == 2
+    assert lib.muse_causal_blocks(f, f, f, _d(), 128, 8, 8, 2, f, None, None, f, 0, st) == 4

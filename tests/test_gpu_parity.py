@@ -1,0 +1,220 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Every comparison feeds the oracle the GPU's own clustering (teacher forcing), so a
+legal near-tie flip in K-means cannot fail an output tolerance; K-means itself is
+checked round by round, labels bit-exact except near-ties (top-2 gap < 1e-5 of
+||x||^2 + ||c||^2, counted).  Output tolerance: max|O - O*| / max|O*| per (b,h)
+<= 1e-4 (float32 path) and <= 2e-2 (bfloat16 inputs, float32 accumulation).
+"""
+import numpy as np
+import pytest
+import torch
+
+from clustered_softmax_attention_b200 import muse as m
+from clustered_softmax_attention_b200.inputs import WORKLOADS, make_inputs, small_problem
+from oracle import muse_oracle as mo
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+TDT = {"f32": torch.float32, "bf16": torch.bfloat16}
+NEAR_TIE = 1e-5
+
+
+def dev(a, dt):
+    return torch.tensor(np.ascontiguousarray(a), dtype=torch.float32).to(TDT[dt]).cuda().contiguous()
+
+
+def host(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def mixture(seed, B, H, N, D, Dv, comps, sigma, dt):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    from clustered_softmax_attention_b200.inputs import draw_problem, round_to_bf16
+    Qs, Ks, Vs = [], [], []
+    for _ in range(B * H):
+        Q, K, V = draw_problem(rng, N, D, Dv, comps, sigma)
+        Qs.append(Q); Ks.append(K); Vs.append(V)
+    cast = round_to_bf16 if dt == "bf16" else (lambda a: a.astype(np.float32))
+    f = lambda L, W: np.stack([cast(x) for x in L]).reshape(B, H, N, W)
+    return f(Qs, D), f(Ks, D), f(Vs, Dv)
+
+
+def check_kmeans_rounds(X, C, T, dt):
+    """Every round: labels vs the oracle's assignment from the GPU's previous centroids."""
+    Xd = dev(X, dt)
+    Xf = host(Xd)
+    B, H, N, D = X.shape
+    excused = 0
+    prev = None
+    for t in range(1, T + 1):
+        lab, cen, perm, offs = m.muse_kmeans(Xd, C, t)
+        lab, cen, perm, offs = (x.cpu().numpy() for x in (lab, cen, perm, offs))
+        for b in range(B):
+            for h in range(H):
+                x = Xf[b, h]
+                c_prev = x[:C] if prev is None else prev[b, h].astype(np.float64)
+                lo, gap = mo.kmeans_assign_gap(x, c_prev)
+                bad = lo != lab[b, h]
+                assert (gap[bad] < NEAR_TIE).all(), (t, b, h, int(bad.sum()))
+                excused += int(bad.sum())
+                # centroids: the oracle's update from the GPU labels
+                c_ref = mo.kmeans_update(x, lab[b, h], c_prev)
+                np.testing.assert_allclose(cen[b, h], c_ref, rtol=2e-5, atol=2e-6)
+                # CSR layout: stable sort by label, offsets = cumulative counts
+                np.testing.assert_array_equal(perm[b, h], np.argsort(lab[b, h], kind="stable"))
+                cnt = np.bincount(lab[b, h], minlength=C)
+                np.testing.assert_array_equal(offs[b, h], np.concatenate([[0], np.cumsum(cnt)]))
+        prev = cen
+    return excused
+
+
+@pytest.mark.parametrize("dt,N,D,C,H", [("f32", 1024, 64, 32, 1), ("bf16", 2048, 128, 64, 2),
+                                         ("bf16", 1000, 64, 37, 1)])
+def test_kmeans_rounds_teacher_forced(dt, N, D, C, H):
+    Q, K, V = mixture(11, 1, H, N, D, D, 48, 0.3 / np.sqrt(D), dt)
+    ex = check_kmeans_rounds(Q, C, 6, dt)
+    assert ex <= 3
+
+
+def run_gpu_pipeline(Q, K, V, Cq, Ck, T, s, dt, with_cov=False):
+    Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
+    ql, qc, qp, qo = m.muse_kmeans(Qd, Cq, T)
+    kl, kc, kp, ko = m.muse_kmeans(Kd, Ck, T)
+    summ = m.muse_tilted_summaries(qc, Kd, Vd, kp, ko, Ck, s, want_cov=with_cov)
+    O = m.muse_dipole_refine(Qd, Kd, Vd, qc, qp, qo, kp, ko, summ["logZ"], summ["mu_k"], s)
+    return dict(Qd=Qd, Kd=Kd, Vd=Vd, ql=ql, qc=qc, kl=kl, summ=summ, O=O)
+
+
+def normwise(O, ref):
+    return max(mo.max_rel_err(O[b, h], ref[b, h]) for b in range(O.shape[0]) for h in range(O.shape[1]))
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_summaries_and_refine_vs_oracle(dt):
+    N, D, Cq, Ck = 512, 64, 16, 24
+    Q, K, V = mixture(3, 1, 2, N, D, D, 20, 0.4 / np.sqrt(D), dt)
+    for s in (1.0, 0.125):
+        r = run_gpu_pipeline(Q, K, V, Cq, Ck, 5, s, dt, with_cov=True)
+        Qf, Kf, Vf = host(r["Qd"]), host(r["Kd"]), host(r["Vd"])
+        for h in range(2):
+            ql = r["ql"][0, h].cpu().numpy()
+            kl = r["kl"][0, h].cpu().numpy()
+            qbar = r["qc"][0, h].cpu().numpy().astype(np.float64)
+            lz, mk, mv, cv = mo.tilted_summaries(qbar, Kf[0, h], Vf[0, h], kl, Ck, s)
+            g = {k: v[0, h].cpu().numpy() for k, v in r["summ"].items()}
+            fin = np.isfinite(lz)
+            assert (np.isfinite(g["logZ"]) == fin).all()
+            np.testing.assert_allclose(g["logZ"][fin], lz[fin], rtol=1e-5, atol=1e-5)
+            for key, ref in (("mu_k", mk), ("mu_v", mv), ("cov", cv)):
+                err = np.abs(g[key] - ref).max() / max(np.abs(ref).max(), 1e-30)
+                assert err < 1e-4, (key, err)
+            O_ref = mo.refine(Qf[0, h], ql, qbar, lz, mk, mv, cv, s)
+            err = mo.max_rel_err(host(r["O"])[0, h], O_ref)
+            assert err <= TOL[dt], err
+
+
+def test_forward_end_to_end_small_f32():
+    w = WORKLOADS["acausal_n1k_f32"]
+    Q, K, V = make_inputs(w)
+    Qd, Kd, Vd = dev(Q, "f32"), dev(K, "f32"), dev(V, "f32")
+    O = host(m.muse_forward(Qd, Kd, Vd, w.Cq, w.Ck, w.iters, w.scale))
+    ql, qc, _, _ = m.muse_kmeans(Qd, w.Cq, w.iters)
+    kl, _, _, _ = m.muse_kmeans(Kd, w.Ck, w.iters)
+    ref = mo.muse_from_labels(Q[0, 0], K[0, 0], V[0, 0], ql[0, 0].cpu().numpy(),
+                              kl[0, 0].cpu().numpy(), w.Cq, w.Ck, w.scale)
+    assert mo.max_rel_err(O[0, 0], ref) <= 1e-4
+    # and against the oracle's own K-means (labels may differ only at near-ties)
+    ref2, ql2, kl2 = mo.muse_acausal(Q[0, 0], K[0, 0], V[0, 0], w.Cq, w.Ck, w.iters, w.scale,
+                                     return_labels=True)
+    if (ql2 == ql[0, 0].cpu().numpy()).all() and (kl2 == kl[0, 0].cpu().numpy()).all():
+        assert mo.max_rel_err(O[0, 0], ref2) <= 1e-4
+    E = mo.exact_attention(Q[0, 0], K[0, 0], V[0, 0], w.scale)
+    assert mo.rse(O[0, 0], E) < 0.2
+
+
+def test_forward_bf16_multihead():
+    Q, K, V = mixture(5, 2, 2, 2048, 64, 64, 64, 0.5 / 8, "bf16")
+    Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
+    O = host(m.muse_forward(Qd, Kd, Vd, 64, 48, 6, 1.0))
+    ql = m.muse_kmeans(Qd, 64, 6)[0].cpu().numpy()
+    kl = m.muse_kmeans(Kd, 48, 6)[0].cpu().numpy()
+    Qf, Kf, Vf = host(Qd), host(Kd), host(Vd)
+    for b in range(2):
+        for h in range(2):
+            ref = mo.muse_from_labels(Qf[b, h], Kf[b, h], Vf[b, h], ql[b, h], kl[b, h], 64, 48, 1.0)
+            assert mo.max_rel_err(O[b, h], ref) <= TOL["bf16"]
+
+
+def test_singleton_query_clusters_give_exact_attention_on_gpu():
+    Q, K, V = small_problem(21, 256, 64, 64, 16, 0.3)
+    Qd, Kd, Vd = (dev(x[None, None], "f32") for x in (Q, K, V))
+    O = host(m.muse_forward(Qd, Kd, Vd, 256, 16, 3, 1.0))[0, 0]
+    E = mo.exact_attention(host(Qd)[0, 0], host(Kd)[0, 0], host(Vd)[0, 0], 1.0)
+    assert mo.max_rel_err(O, E) <= 1e-4
+
+
+def test_forward_is_deterministic():
+    Q, K, V = mixture(6, 1, 2, 1024, 64, 64, 32, 0.4 / 8, "bf16")
+    Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
+    a = m.muse_forward(Qd, Kd, Vd, 32, 32, 4, 1.0)
+    b = m.muse_forward(Qd, Kd, Vd, 32, 32, 4, 1.0)
+    assert torch.equal(a, b)
+    assert m.muse_last_device_status() == 0
+
+
+def causal_labels(ql, kl, N, S):
+    out = {}
+    for (lev, r, q0, q1, k0, k1) in mo.causal_squares(N, S):
+        out[(lev, r)] = (ql[lev - 1, q0:q1], kl[lev - 1, k0:k1])
+    return out
+
+
+@pytest.mark.parametrize("dt,N,S,C", [("f32", 1024, 128, 16), ("bf16", 1024, 128, 16),
+                                       ("bf16", 1536, 256, 40)])
+def test_causal_vs_oracle(dt, N, S, C):
+    Q, K, V = mixture(7, 1, 2, N, 64, 64, 16, 0.3 / 8, dt)
+    Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
+    O, ql, kl = m.muse_causal_blocks(Qd, Kd, Vd, S, C, C, 4, 1.0, return_labels=True)
+    O = host(O)
+    ql, kl = ql.cpu().numpy(), kl.cpu().numpy()
+    Qf, Kf, Vf = host(Qd), host(Kd), host(Vd)
+    for h in range(2):
+        labels = causal_labels(ql[0, h], kl[0, h], N, S)
+        # rows outside every square of a level are labelled -1
+        L = m.muse_causal_levels(N, S)
+        for lev in range(1, L + 1):
+            inside = np.zeros(N, bool)
+            for (lv, r, q0, q1, k0, k1) in mo.causal_squares(N, S):
+                if lv == lev:
+                    inside[q0:q1] = True
+            assert (ql[0, h, lev - 1][~inside] == -1).all()
+            assert (ql[0, h, lev - 1][inside] >= 0).all()
+        ref = mo.muse_causal(Qf[0, h], Kf[0, h], Vf[0, h], S, C, C, 4, 1.0, labels=labels)
+        assert mo.max_rel_err(O[0, h], ref) <= TOL[dt]
+
+
+def test_causal_single_block_is_exact():
+    Q, K, V = small_problem(22, 256, 64, 64, 8, 0.3)
+    Qd, Kd, Vd = (dev(x[None, None], "f32") for x in (Q, K, V))
+    O = host(m.muse_causal_blocks(Qd, Kd, Vd, 256, 8, 8, 2, 1.0))[0, 0]
+    E = mo.exact_attention(host(Qd)[0, 0], host(Kd)[0, 0], host(Vd)[0, 0], 1.0, causal=True)
+    assert mo.max_rel_err(O, E) <= 1e-4
+
+
+def test_full_size_acausal_n8k_sampled_rows():
+    """The benchmarked workload at full size, checked on sampled rows of two heads."""
+    w = WORKLOADS["acausal_n8k_bf16"]
+    Q, K, V = make_inputs(w)
+    Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
+    O = host(m.muse_forward(Qd, Kd, Vd, w.Cq, w.Ck, w.iters, w.scale))
+    ql = m.muse_kmeans(Qd, w.Cq, w.iters)[0].cpu().numpy()
+    kl = m.muse_kmeans(Kd, w.Ck, w.iters)[0].cpu().numpy()
+    rng = np.random.default_rng(0)
+    for h in (0, w.H - 1):
+        rows = np.concatenate([rng.choice(w.N, 48, replace=False), [0, w.N - 1]])
+        ref = mo.muse_from_labels(Q[0, h], K[0, h], V[0, h], ql[0, h], kl[0, h], w.Cq, w.Ck,
+                                  w.scale, rows=rows)
+        err = np.abs(O[0, h][rows] - ref[rows]).max() / np.abs(ref[rows]).max()
+        assert err <= TOL["bf16"], err
