@@ -206,6 +206,17 @@ static void plan_kmeans_pair(Bump &bp, const MuseTables &mt, const muse_dims &d,
     if (e_ != cudaSuccess) return MUSE_ERR_CUDA;        \
   } while (0)
 
+// Inside a stream capture the event becomes an event-record node of the graph, so
+// every replay records it; outside a capture it is an ordinary record.
+static cudaError_t record_profile_event(void *ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  if (cs == cudaStreamCaptureStatusActive)
+    return cudaEventRecordWithFlags((cudaEvent_t)ev, st, cudaEventRecordExternal);
+  return cudaEventRecord((cudaEvent_t)ev, st);
+}
+
 // The refinement launch sequence shared by every path.
 static muse_status refine_path(const void *Q, const void *K, const void *V, const muse_dims &d,
                                int P, const MuseTables &mt, const float *q_centroids,
@@ -228,7 +239,7 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
   }
   MUSE_TRY(run_coeffs(mt, d.dtype, d.D, P, d.scale, r.qs, q_offsets, sb, st));
   void *ev0 = g_prof_start.load(), *ev1 = g_prof_stop.load();
-  if (ev0 && ev1) MUSE_TRY(cudaEventRecordWithFlags((cudaEvent_t)ev0, st, cudaEventRecordExternal));
+  if (ev0 && ev1) MUSE_TRY(record_profile_event(ev0, st));
   if (tc_supported(d.dtype, d.D, d.Dv)) {
     MUSE_TRY(run_refine_tc(mt, d.D, d.Dv, d.N, P, r.qs, q_perm, r.ks, r.vs, sb, O, part_o,
                            part_lse, status_ptr(), st));
@@ -236,7 +247,7 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
     MUSE_TRY(run_refine(mt, d.dtype, d.D, d.Dv, d.N, P, r.qs, q_perm, r.ks, r.vs, sb, O, part_o,
                         part_lse, st));
   }
-  if (ev0 && ev1) MUSE_TRY(cudaEventRecordWithFlags((cudaEvent_t)ev1, st, cudaEventRecordExternal));
+  if (ev0 && ev1) MUSE_TRY(record_profile_event(ev1, st));
   return MUSE_OK;
 }
 
