@@ -14,6 +14,9 @@ inline size_t align_up(size_t b) { return (b + 255) & ~(size_t)255; }
 // Host-side count of enqueued kernels (muse_launch_counter).
 void count_launches(int n);
 
+// Device address of the current device's status word (NULL if unavailable).
+int *device_status_word();
+
 // Per-instance offsets of the stage buffers.  An instance pairs query segment s
 // with key segment s (acausal: the one whole-sequence segment; causal: one square).
 struct InstTable {

@@ -37,6 +37,8 @@ static int *status_ptr() {
   return ptrs[dev];
 }
 
+int *device_status_word() { return status_ptr(); }
+
 // ---------------------------------------------------------------------------
 // Workspace: a bump allocator over the caller's buffer (or a size count when
 // base == nullptr).  Every piece is 256-byte aligned.

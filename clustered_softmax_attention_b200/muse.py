@@ -39,6 +39,7 @@ class MuseDims(ctypes.Structure):
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 _SIGS = {
     "muse_kmeans": [_vp, MuseDims, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
+    "muse_kmeans_noalloc": [_vp, MuseDims, _i, _i, _vp, _vp, _vp, _vp, _vp],
     "muse_tilted_summaries": [_vp, _vp, _vp, _vp, _vp, MuseDims, _i, _i, _vp, _vp, _vp, _vp,
                               _vp, _sz, _vp],
     "muse_dipole_refine": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, MuseDims, _i, _i,

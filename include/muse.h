@@ -91,6 +91,30 @@ muse_status muse_kmeans(const void *X, muse_dims d, int C, int iters, int32_t *l
                         size_t ws_bytes, muse_stream_t st);
 
 /*
+ * muse_kmeans_noalloc - muse_kmeans for callers that cannot allocate device memory
+ * and so cannot hand over a workspace: code running inside another runtime's memory
+ * pool that offers no allocation hook, code called while a global-mode stream
+ * capture is active (cudaMalloc is an error there), latency-critical loops that
+ * cannot pay for cudaMalloc's synchronisation.  The paper has no counterpart: this
+ * is a deployment variant of the same computation, with identical results.
+ *   Same arguments and outputs as muse_kmeans, minus the workspace.  Its scratch is
+ *   a static device array of MUSE_NOALLOC_SCRATCH_BYTES (16 MiB) inside the library,
+ *   held by every GPU that loads it until the process exits.  A problem whose
+ *   scratch need (muse_workspace_size("muse_kmeans", ...)) exceeds that returns
+ *   MUSE_ERR_WORKSPACE before anything is enqueued; e.g. B*H = 8, N = 8192,
+ *   C = 128 needs about 0.5 MiB.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.  The library
+ *   allocates nothing and calls no allocating routine.  Every call shares the one
+ *   array and leaves its contents behind: calls that overlap on the GPU (several
+ *   streams, or several threads) race on it and must be serialised by the caller.
+ */
+#define MUSE_NOALLOC_SCRATCH_BYTES (16u << 20)
+muse_status muse_kmeans_noalloc(const void *X, muse_dims d, int C, int iters, int32_t *labels,
+                                float *centroids, int32_t *perm, int32_t *offsets,
+                                muse_stream_t st);
+
+/*
  * muse_tilted_summaries - stage 1: for every query centroid i and key cluster j
  *     l_k = s qbar_i.k (k in S_j);  log Z_ij = log sum_k exp(l_k);
  *     w_k = exp(l_k - log Z_ij);    mu_k,ij = sum_k w_k k;  mu_v,ij = sum_k w_k v;
