@@ -44,6 +44,12 @@ struct SegTable {
   int off0[kMaxSeg];
 };
 
+// Row stride of the tilt-weight matrix W of an instance with nk sorted keys: padded
+// to 8 floats so every row starts 32-byte aligned.
+__host__ __device__ __forceinline__ int w_ld(int nk) { return (nk + 7) & ~7; }
+// Row stride of the transposed sorted values (keys innermost): 8 elements (16 bytes).
+__host__ __device__ __forceinline__ int vt_ld(int row_stride) { return (row_stride + 7) & ~7; }
+
 // A task is one (problem, segment) pair.
 struct Task {
   int p, s;

@@ -64,6 +64,9 @@ struct StageBufs {
 cudaError_t run_sort_side(const void *X, int dtype, int width, int N, const SegTable &tab, int P,
                           const int32_t *perm, const int32_t *offsets, const float *centroids,
                           SortedSide out, cudaStream_t st);
+// Transposed sorted copy (keys innermost) for the tensor-core refinement.
+cudaError_t run_sort_side_t(const void *X, int dtype, int width, int N, const SegTable &tab,
+                            int P, const int32_t *perm, void *vt, cudaStream_t st);
 cudaError_t run_summaries(const MuseTables &mt, int dtype, int D, int Dv, int P, float scale,
                           const float *q_centroids, SortedSide ks, const void *vs_rows,
                           const int32_t *k_offsets, StageBufs b, cudaStream_t st);

@@ -91,7 +91,7 @@ static InstTable whole_inst(int N, int Cq, int Ck) {
   InstTable in;
   memset(&in, 0, sizeof(in));
   in.ninst = 1;
-  in.w_stride = Cq * N;
+  in.w_stride = Cq * w_ld(N);
   in.z_stride = Cq * Ck;
   in.c_stride = Ck * N;
   in.out_stride = N;
@@ -145,7 +145,7 @@ static bool build_causal(int N, int block, int Cq, int Ck, MuseTables &mt, int &
     k.cen0[s] = ck_acc; k.off0[s] = ok;
     in.w0[s] = w; in.z0[s] = z; in.cc0[s] = c; in.out0[s] = (x.lev - 1) * N;
     cq_acc += cq; ck_acc += ck; oq += cq + 1; ok += ck + 1;
-    w += cq * nk; z += cq * ck; c += ck * nq;
+    w += cq * w_ld(nk); z += cq * ck; c += ck * nq;
     q.max_rows = std::max(q.max_rows, nq); k.max_rows = std::max(k.max_rows, nk);
     q.max_C = std::max(q.max_C, cq); k.max_C = std::max(k.max_C, ck);
   }
@@ -172,7 +172,7 @@ static void plan_refine(Bump &bp, const MuseTables &mt, const muse_dims &d, int 
   r.qs.cluster = bp.take<int32_t>(qrows);
   r.ks.rows = bp.take<char>(krows * d.D * es);
   r.ks.cluster = bp.take<int32_t>(krows);
-  r.vs = bp.take<char>(krows * d.Dv * es);
+  r.vs = bp.take<char>((size_t)P * d.Dv * vt_ld(mt.k.row_stride) * es);
   r.v_cluster = bp.take<int32_t>(krows);
   memset(&r.sb, 0, sizeof(r.sb));
   r.sb.W = bp.take<float>((size_t)P * mt.in.w_stride);
@@ -228,8 +228,13 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
                                float *part_o, float *part_lse, cudaStream_t st) {
   MUSE_TRY(run_sort_side(Q, d.dtype, d.D, d.N, mt.q, P, q_perm, q_offsets, q_centroids, r.qs, st));
   MUSE_TRY(run_sort_side(K, d.dtype, d.D, d.N, mt.k, P, k_perm, k_offsets, nullptr, r.ks, st));
-  SortedSide vsd{r.vs, r.v_cluster};
-  MUSE_TRY(run_sort_side(V, d.dtype, d.Dv, d.N, mt.k, P, k_perm, k_offsets, nullptr, vsd, st));
+  const bool use_tc = tc_supported(d.dtype, d.D, d.Dv);
+  if (use_tc) {
+    MUSE_TRY(run_sort_side_t(V, d.dtype, d.Dv, d.N, mt.k, P, k_perm, r.vs, st));
+  } else {
+    SortedSide vsd{r.vs, r.v_cluster};
+    MUSE_TRY(run_sort_side(V, d.dtype, d.Dv, d.N, mt.k, P, k_perm, k_offsets, nullptr, vsd, st));
+  }
   StageBufs sb = r.sb;
   if (logZ_in) {
     sb.logZ = const_cast<float *>(logZ_in);
@@ -242,9 +247,9 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
   MUSE_TRY(run_coeffs(mt, d.dtype, d.D, P, d.scale, r.qs, q_offsets, sb, st));
   void *ev0 = g_prof_start.load(), *ev1 = g_prof_stop.load();
   if (ev0 && ev1) MUSE_TRY(record_profile_event(ev0, st));
-  if (tc_supported(d.dtype, d.D, d.Dv)) {
-    MUSE_TRY(run_refine_tc(mt, d.D, d.Dv, d.N, P, r.qs, q_perm, r.ks, r.vs, sb, O, part_o,
-                           part_lse, status_ptr(), st));
+  if (use_tc) {
+    MUSE_TRY(run_refine_tc(mt, d.D, d.Dv, d.N, P, r.qs, q_perm, r.ks, k_offsets, r.vs, sb, O,
+                           part_o, part_lse, status_ptr(), st));
   } else {
     MUSE_TRY(run_refine(mt, d.dtype, d.D, d.Dv, d.N, P, r.qs, q_perm, r.ks, r.vs, sb, O, part_o,
                         part_lse, st));

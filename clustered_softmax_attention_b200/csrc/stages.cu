@@ -55,6 +55,44 @@ __global__ void sort_side(const T *__restrict__ X, int N, int W, SegTable tab,
 }
 
 // ---------------------------------------------------------------------------
+// Transposed sorted copy: vt[p][c][lab0 + m] = X[p][perm[m]][c] (keys innermost,
+// row length vt_ld(row_stride)), so that the values are a K-major operand of the
+// P.V contraction.  64 sorted positions per CTA, staged through shared memory.
+// ---------------------------------------------------------------------------
+template <typename T, int W>
+__global__ void __launch_bounds__(256)
+sort_side_t(const T *__restrict__ X, int N, SegTable tab, const int32_t *__restrict__ perm,
+            T *__restrict__ vt) {
+  const Task tk = make_task(tab, blockIdx.y);
+  const int m0 = blockIdx.x * 64;
+  if (m0 >= tk.n) return;
+  __shared__ T buf[64][W + 2];
+  const int mt = min(64, tk.n - m0);
+  for (int e = threadIdx.x; e < mt * W; e += blockDim.x) {
+    const int mm = e / W, c = e % W;
+    const int row = perm[tk.lab + m0 + mm];
+    buf[mm][c] = X[((int64_t)tk.p * N + row) * W + c];
+  }
+  __syncthreads();
+  const int ld = vt_ld(tab.row_stride);
+  const int64_t col0 = (int64_t)(tk.lab - (int64_t)tk.p * tab.row_stride) + m0;
+  for (int e = threadIdx.x; e < mt * W; e += blockDim.x) {
+    const int c = e / mt, mm = e % mt;
+    vt[((int64_t)tk.p * W + c) * ld + col0 + mm] = buf[mm][c];
+  }
+  // The 16 columns after the segment are read (and multiplied by zero weights) by a
+  // key tile that overhangs the segment's end: make them zeros, not stale memory.
+  if (m0 + 64 >= tk.n) {
+    const int64_t end = (int64_t)(tk.lab - (int64_t)tk.p * tab.row_stride) + tk.n;
+    for (int e = threadIdx.x; e < 16 * W; e += blockDim.x) {
+      const int c = e >> 4;
+      const int64_t col = end + (e & 15);
+      if (col < ld) vt[((int64_t)tk.p * W + c) * ld + col] = T(0.f);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Tilt logits W[i][pos] = s qbar_i . k_pos over the sorted keys (64 x 64 tiles).
 // ---------------------------------------------------------------------------
 template <typename T, int D>
@@ -105,7 +143,7 @@ tilt_logits(MuseTables mt, float scale, const float *__restrict__ qcen, const T 
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       const int kk = k0 + tx * 4 + b;
-      if (kk < nk) wo[(int64_t)i * nk + kk] = scale * acc[a][b];
+      if (kk < nk) wo[(int64_t)i * w_ld(nk) + kk] = scale * acc[a][b];
     }
   }
 }
@@ -123,7 +161,7 @@ tilt_lse(MuseTables mt, const int32_t *__restrict__ k_offsets, float *__restrict
   if (wid >= Cq * Ck) return;
   const int i = wid / Ck, j = wid % Ck;
   const int b = k_offsets[k.off + j], e = k_offsets[k.off + j + 1];
-  float *w = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * nk;
+  float *w = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * w_ld(nk);
   float m = -CUDART_INF_F;
   for (int pos = b + lane; pos < e; pos += 32) m = fmaxf(m, w[pos]);
   m = warp_max(m);
@@ -149,7 +187,7 @@ tilt_weights(MuseTables mt, const int32_t *__restrict__ k_cluster, const float *
   if (pos >= k.n) return;
   const int j = k_cluster[k.lab + pos];
   const float lz = logZ[(int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * k.C + j];
-  float *w = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * k.n + pos;
+  float *w = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * w_ld(k.n) + pos;
   *w = expf(*w - lz);
 }
 
@@ -185,7 +223,7 @@ tilt_moments(MuseTables mt, const int32_t *__restrict__ k_offsets, const float *
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const int i = ib + t;
-      const float w = (i < Cq) ? wb[(int64_t)i * nk + pos] : 0.f;
+      const float w = (i < Cq) ? wb[(int64_t)i * w_ld(nk) + pos] : 0.f;
 #pragma unroll
       for (int u = 0; u < PER; ++u) acc[t][u] = fmaf(w, xv[u], acc[t][u]);
     }
@@ -218,7 +256,7 @@ tilt_cov(MuseTables mt, const int32_t *__restrict__ k_offsets, const float *__re
   const int64_t z = (int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck + j;
   const float *mk = mu_k + z * D;
   const float *mv = mu_v + z * DV;
-  const float *w = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * nk;
+  const float *w = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * w_ld(nk);
   float *out = cov + z * DV * D;
   for (int e2 = threadIdx.x; e2 < DV * D; e2 += blockDim.x) {
     const int dv = e2 / D, d = e2 % D;
@@ -326,7 +364,7 @@ refine_simt(MuseTables mt, int N, const T *__restrict__ qt_rows, const int32_t *
 #pragma unroll
   for (int t = 0; t < PD; ++t) qt[t] = v ? ld_elem(qt_rows + (q.lab + n) * D + g + 4 * t) : 0.f;
   const int i = v ? q_cluster[q.lab + n] : 0;
-  const float *wrow = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * nk;
+  const float *wrow = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * w_ld(nk);
   const float *C0 = c0 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
   const float *C1 = c1 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
   float acc[PV];
@@ -464,6 +502,22 @@ cudaError_t run_sort_side(const void *X, int dtype, int width, int N, const SegT
     sort_side<__nv_bfloat16><<<grid, threads, 0, st>>>(
         (const __nv_bfloat16 *)X, N, width, tab, perm, offsets, centroids,
         (__nv_bfloat16 *)out.rows, out.cluster);
+  return cudaGetLastError();
+}
+
+cudaError_t run_sort_side_t(const void *X, int dtype, int width, int N, const SegTable &tab,
+                            int P, const int32_t *perm, void *vt, cudaStream_t st) {
+  dim3 grid((tab.max_rows + 63) / 64, P * tab.nseg);
+  count_launches(1);
+  if (dtype == MUSE_F32) {
+    if (width == 64) sort_side_t<float, 64><<<grid, 256, 0, st>>>((const float *)X, N, tab, perm, (float *)vt);
+    else sort_side_t<float, 128><<<grid, 256, 0, st>>>((const float *)X, N, tab, perm, (float *)vt);
+  } else {
+    if (width == 64)
+      sort_side_t<__nv_bfloat16, 64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)X, N, tab, perm, (__nv_bfloat16 *)vt);
+    else
+      sort_side_t<__nv_bfloat16, 128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)X, N, tab, perm, (__nv_bfloat16 *)vt);
+  }
   return cudaGetLastError();
 }
 
