@@ -40,9 +40,15 @@ struct KmeansOut {
   int32_t *offsets;
 };
 
-size_t kmeans_ws_bytes(const SegTable &t, int P);
+size_t kmeans_ws_bytes(const SegTable &t, int P, int D);
+size_t kmeans_pair_ws_bytes(const SegTable *tq, const SegTable *tk, int P, int D);
 cudaError_t run_kmeans(const void *X, int dtype, int D, int N, const SegTable &tab, int P,
                        int iters, const KmeansOut &o, char *ws, int *status, cudaStream_t st);
+// Queries and keys clustered in the same launches.
+cudaError_t run_kmeans_pair(const void *Xq, const SegTable &tq, const KmeansOut &oq,
+                            const void *Xk, const SegTable &tk, const KmeansOut &ok, int dtype,
+                            int D, int N, int P, int iters, char *ws, int *status,
+                            cudaStream_t st);
 
 // Sorted working copies of one side (rows in cluster order).
 struct SortedSide {

@@ -66,7 +66,7 @@ extern "C" muse_status muse_kmeans_noalloc(const void *X, muse_dims d, int C, in
   const int P = d.B * d.H;
   // The scratch holds per-chunk label counts, chunk bases and in-chunk ranks; a
   // problem needing more than the array holds is refused before anything runs.
-  if (kmeans_ws_bytes(t, P) > (size_t)MUSE_NOALLOC_SCRATCH_BYTES) return MUSE_ERR_WORKSPACE;
+  if (kmeans_ws_bytes(t, P, d.D) > (size_t)MUSE_NOALLOC_SCRATCH_BYTES) return MUSE_ERR_WORKSPACE;
 
   char *scratch = nullptr;
   if (kmeans_scratch_address(&scratch) != cudaSuccess) return MUSE_ERR_CUDA;

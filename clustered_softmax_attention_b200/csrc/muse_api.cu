@@ -93,7 +93,7 @@ static InstTable whole_inst(int N, int Cq, int Ck) {
   in.ninst = 1;
   in.w_stride = Cq * w_ld(N);
   in.z_stride = Cq * Ck;
-  in.c_stride = Ck * N;
+  in.c_stride = Ck * w_ld(N);
   in.out_stride = N;
   return in;
 }
@@ -145,7 +145,7 @@ static bool build_causal(int N, int block, int Cq, int Ck, MuseTables &mt, int &
     k.cen0[s] = ck_acc; k.off0[s] = ok;
     in.w0[s] = w; in.z0[s] = z; in.cc0[s] = c; in.out0[s] = (x.lev - 1) * N;
     cq_acc += cq; ck_acc += ck; oq += cq + 1; ok += ck + 1;
-    w += cq * w_ld(nk); z += cq * ck; c += ck * nq;
+    w += cq * w_ld(nk); z += cq * ck; c += ck * w_ld(nq);
     q.max_rows = std::max(q.max_rows, nq); k.max_rows = std::max(k.max_rows, nk);
     q.max_C = std::max(q.max_C, cq); k.max_C = std::max(k.max_C, ck);
   }
@@ -199,7 +199,7 @@ static void plan_kmeans_pair(Bump &bp, const MuseTables &mt, const muse_dims &d,
   };
   side(mt.q, w.q);
   side(mt.k, w.k);
-  w.scratch = bp.take<char>(std::max(kmeans_ws_bytes(mt.q, P), kmeans_ws_bytes(mt.k, P)));
+  w.scratch = bp.take<char>(kmeans_pair_ws_bytes(&mt.q, &mt.k, P, d.D));
 }
 
 #define MUSE_TRY(expr)                                  \
@@ -297,7 +297,7 @@ extern "C" muse_status muse_last_device_status(muse_stream_t st) {
 
 static size_t ws_kmeans(const muse_dims &d, int C) {
   SegTable t = whole_side(d.N, C);
-  return kmeans_ws_bytes(t, d.B * d.H);
+  return kmeans_ws_bytes(t, d.B * d.H, d.D);
 }
 
 static size_t ws_summaries(const muse_dims &d, int Cq, int Ck, bool need_v, bool need_mu) {
@@ -508,9 +508,8 @@ extern "C" muse_status muse_forward(const void *Q, const void *K, const void *V,
   plan_refine(bp, mt, d, P, r, true);
   cudaStream_t cs = (cudaStream_t)st;
   int *stat = status_ptr();
-  if (run_kmeans(Q, d.dtype, d.D, d.N, mt.q, P, iters, kw.q, kw.scratch, stat, cs) != cudaSuccess)
-    return MUSE_ERR_CUDA;
-  if (run_kmeans(K, d.dtype, d.D, d.N, mt.k, P, iters, kw.k, kw.scratch, stat, cs) != cudaSuccess)
+  if (run_kmeans_pair(Q, mt.q, kw.q, K, mt.k, kw.k, d.dtype, d.D, d.N, P, iters, kw.scratch, stat,
+                      cs) != cudaSuccess)
     return MUSE_ERR_CUDA;
   return refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets, kw.k.perm,
                      kw.k.offsets, nullptr, nullptr, r, O, nullptr, nullptr, cs);
@@ -563,9 +562,8 @@ extern "C" muse_status muse_causal_blocks(const void *Q, const void *K, const vo
       cudaMemsetAsync(kw.k.labels, 0xff, (size_t)P * L * d.N * sizeof(int32_t), cs) != cudaSuccess)
     return MUSE_ERR_CUDA;
   int *stat = status_ptr();
-  if (run_kmeans(Q, d.dtype, d.D, d.N, mt.q, P, iters, kw.q, kw.scratch, stat, cs) != cudaSuccess)
-    return MUSE_ERR_CUDA;
-  if (run_kmeans(K, d.dtype, d.D, d.N, mt.k, P, iters, kw.k, kw.scratch, stat, cs) != cudaSuccess)
+  if (run_kmeans_pair(Q, mt.q, kw.q, K, mt.k, kw.k, d.dtype, d.D, d.N, P, iters, kw.scratch, stat,
+                      cs) != cudaSuccess)
     return MUSE_ERR_CUDA;
   s = refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets, kw.k.perm,
                   kw.k.offsets, nullptr, nullptr, r, nullptr, part_o, part_lse, cs);

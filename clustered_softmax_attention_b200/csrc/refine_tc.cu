@@ -9,162 +9,61 @@
 //
 // One CTA = 128 consecutive sorted query rows of one instance (their residuals are
 // the A operand of the first contraction, resident in shared memory).  The CTA walks
-// the key clusters; a key tile is one cluster (chunks of at most 112 keys), widened
+// the key clusters; a key tile is one cluster (chunks of at most BN-16 keys), widened
 // to an 8-key-aligned start so the transposed values can be fetched by TMA, padded to
-// a multiple of 16 columns; out-of-cluster columns are masked to zero.
+// a multiple of 16 columns; out-of-cluster columns are masked to zero.  With every
+// key/value tile the producer also stages, by cp.async into the same stage, the tile's
+// tilt weights for up to 8 query clusters of the CTA and the tile's coefficients
+// c0, c1 for the CTA's 128 rows.
 //   S  = Qt . K_tile^T            (tcgen05, 128 x npad, fp32 in TMEM, double-buffered)
 //   P  = w .* (c0 + c1 .* S)      (epilogue warps: TMEM -> registers -> bf16 SMEM)
 //   O += P . V_tile               (tcgen05, 128 x Dv, fp32 in TMEM)
-// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner),
-// warps 2-5 = epilogue (TMEM lane quadrant = warp % 4).  Every wait on an mbarrier is
+// Warp roles: warp 0 = producer (TMA + cp.async), warp 1 = MMA issuer (+ TMEM
+// owner), warps 2-9 = epilogue (TMEM lane quadrant = warp % 4; two warps per quadrant
+// split the 16-column chunks).  Every wait on an mbarrier is
 // bounded: past the limit the kernel records MUSE_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 
 #include "tc.h"
+#include "tc_ptx.cuh"
 
 namespace muse {
 namespace tcr {
 
 constexpr int BM = 128;      // query rows per CTA
-constexpr int BN = 128;      // max keys per tile
-constexpr int CHUNK = 112;   // keys of one cluster per tile (<= 7 alignment keys in front)
-constexpr int NST = 2;       // K / V^T stages
-constexpr int kThreads = 192;
-constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr int NST = 3;       // K / V^T stages
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kSlots = 8;    // query clusters per CTA whose tilt weights are staged
+
+// Widest key tile: 128 keys when D = Dv = 64, else 64 (shared memory budget).
+template <int D, int DV>
+struct TileCfg {
+  static constexpr int BN = (D == 64 && DV == 64) ? 128 : 64;
+  static constexpr int CHUNK = BN - 16;  // keys of one cluster per tile (<= 7 alignment keys in front)
+};
 
 template <int D, int DV>
 struct __align__(1024) Smem {
+  static constexpr int BN = TileCfg<D, DV>::BN;
   __nv_bfloat16 q[D / 64][BM * 64];            // residual tile, K-major SW128 blocks
   __nv_bfloat16 k[NST][D / 64][BN * 64];       // key tiles
   __nv_bfloat16 vt[NST][BN / 64][DV * 64];     // transposed value tiles
   __nv_bfloat16 p[2][BN / 64][BM * 64];        // P tiles (A operand of the second MMA)
+  float w[NST][kSlots][BN];                    // tilt weights of the CTA's query clusters
+  float c0[NST][BM], c1[NST][BM];              // coefficients of the tile's key cluster
   uint64_t full[NST], empty[NST], sfull[2], sfree[2], pready[2], pfree[2], qbar, obar;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// ------------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint32_t saddr(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t now_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(saddr(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: false when the limit ran out or another role has aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile int *abort_flag,
-                                          int *status) {
-  if (mbar_try(b, parity)) return true;
-  const uint64_t t0 = now_ns();
-  while (true) {
-    if (mbar_try(b, parity)) return true;
-    if (*abort_flag) return false;
-    if (now_ns() - t0 > kTimeoutNs) {
-      *abort_flag = 1;
-      report(status, MUSE_ERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-// Bounded wait that ignores the abort flag: used to let in-flight copies and MMAs
-// finish before the CTA releases its shared memory and TMEM.
-__device__ __forceinline__ void mbar_drain(uint64_t *b, uint32_t parity, int *status) {
-  const uint64_t t0 = now_ns();
-  while (!mbar_try(b, parity)) {
-    if (now_ns() - t0 > kTimeoutNs) {
-      report(status, MUSE_ERR_TIMEOUT);
-      return;
-    }
-  }
-}
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
-                                            uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(saddr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(saddr(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint64_t *bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          saddr(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// 16 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(r[e]);
-}
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
-__device__ __forceinline__ uint64_t sdesc(const void *p) {
-  const uint32_t a = saddr(p);
-  uint64_t d = 0;
-  d |= (uint64_t)((a & 0x3FFFFu) >> 4);
-  d |= (uint64_t)1 << 16;            // leading byte offset (unused for swizzled K-major)
-  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset
-  d |= (uint64_t)1 << 46;            // descriptor version (sm_100)
-  d |= (uint64_t)2 << 61;            // SWIZZLE_128B
-  return d;
-}
-// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, both K-major.
-__host__ __device__ constexpr uint32_t idesc(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
+using namespace ptx;
 
 // Key tiles of an instance: cluster j's keys [b, e) in chunks of CHUNK.
 struct KTile {
   int j, c, n, x0, npad;
 };
+template <int CHUNK>
 struct TileIter {
   const int32_t *off;
   int C, j, c;
@@ -207,6 +106,8 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                  const float *__restrict__ c0g, const float *__restrict__ c1g,
                  const float *__restrict__ lse, __nv_bfloat16 *__restrict__ O,
                  float *__restrict__ part_o, float *__restrict__ part_lse, int *status) {
+  constexpr int BN = TileCfg<D, DV>::BN;
+  constexpr int CHUNK = TileCfg<D, DV>::CHUNK;
   const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
   const Task q = make_task(mt.q, p * mt.q.nseg + s);
   const Task k = make_task(mt.k, p * mt.k.nseg + s);
@@ -221,13 +122,13 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
-      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.full[i], 1 + 32);  // producer's expect_tx + one cp.async arrival per lane
       mbar_init(&sm.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.sfull[i], 1);
-      mbar_init(&sm.sfree[i], 4);
-      mbar_init(&sm.pready[i], 4);
+      mbar_init(&sm.sfree[i], kEpiWarps);
+      mbar_init(&sm.pready[i], kEpiWarps);
       mbar_init(&sm.pfree[i], 1);
     }
     mbar_init(&sm.qbar, 1);
@@ -249,19 +150,28 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   const uint32_t tmem_o = tmem + 256;
   const int32_t *koff = k_offsets + k.off;
   const int kcol0 = (int)(k.lab - (int64_t)p * mt.k.row_stride);  // instance's first key column
+  const int wl = w_ld(k.n), cl = w_ld(q.n);
+  const float *Wi = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s];      // row i: Wi + i*wl
+  const float *C0 = c0g + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];   // row j: C0 + j*cl
+  const float *C1 = c1g + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
+  const int i_first = q_cluster[q.lab + r0];  // query clusters i_first.. get staged weights
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ producer
+    TileIter<CHUNK> it;
+    it.begin(koff, k.C);
+    int t = 0;
     if (lane == 0) {
       mbar_expect_tx(&sm.qbar, (uint32_t)(D / 64) * BM * 128);
       for (int kb = 0; kb < D / 64; ++kb) tma_load_2d(sm.q[kb], &map_q, kb * 64, (int)(q.lab + r0), &sm.qbar);
-      TileIter it;
-      it.begin(koff, k.C);
-      int t = 0;
-      for (; !it.done(); it.next(), ++t) {
-        const KTile kt = it.get();
-        const int st = t % NST;
-        if (t >= NST && !mbar_wait(&sm.empty[st], ((t / NST) - 1) & 1, abort_flag, status)) break;
+    }
+    for (; !it.done(); it.next(), ++t) {
+      const KTile kt = it.get();
+      const int st = t % NST;
+      bool ok = true;
+      if (t >= NST) ok = mbar_wait(&sm.empty[st], ((t / NST) - 1) & 1, abort_flag, status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (lane == 0) {
         const int nbox = kt.npad > 64 ? 2 : 1;
         mbar_expect_tx(&sm.full[st], (uint32_t)nbox * ((D / 64) * 64 * 128 + DV * 128));
         for (int rb = 0; rb < nbox; ++rb) {
@@ -271,15 +181,34 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           tma_load_2d(sm.vt[st][rb], &map_vt, kcol0 + kt.x0 + rb * 64, p * DV, &sm.full[st]);
         }
       }
-      // copies still in flight land before the CTA may exit
-      for (int u = max(0, t - NST); u < t; ++u) mbar_drain(&sm.full[u % NST], (u / NST) & 1, status);
+      // tilt weights of the staged query clusters over the tile's columns
+      for (int e = lane; e < kSlots * (BN / 4); e += 32) {
+        const int sl = e / (BN / 4), v = e % (BN / 4);
+        const int col = kt.x0 + 4 * v, i = i_first + sl;
+        const bool in = i < q.C && col < wl && 4 * v < kt.npad;
+        cp_async16(&sm.w[st][sl][4 * v], in ? (const void *)(Wi + (int64_t)i * wl + col) : (const void *)W,
+                   in ? 16u : 0u);
+      }
+      // coefficients of the tile's key cluster for the CTA's rows
+      {
+        const int row = r0 + 4 * lane;
+        const bool in = row < cl;
+        cp_async16(&sm.c0[st][4 * lane], in ? (const void *)(C0 + (int64_t)kt.j * cl + row) : (const void *)W,
+                   in ? 16u : 0u);
+        cp_async16(&sm.c1[st][4 * lane], in ? (const void *)(C1 + (int64_t)kt.j * cl + row) : (const void *)W,
+                   in ? 16u : 0u);
+      }
+      cp_async_arrive(&sm.full[st]);
     }
+    // copies still in flight land before the CTA may exit
+    if (lane == 0)
+      for (int u = max(0, t - NST); u < t; ++u) mbar_drain(&sm.full[u % NST], (u / NST) & 1, status);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(&sm.qbar, 0, abort_flag, status);
       tc_fence_after();
-      TileIter it;
+      TileIter<CHUNK> it;
       it.begin(koff, k.C);
       int t = 0, prev_npad = 0;
       auto gemm2 = [&](int u, int npad) -> bool {
@@ -319,47 +248,55 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   } else {
     // ------------------------------------------------------------ epilogue warps
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;  // which 16-column chunks this warp takes
     const int r = quad * 32 + lane;
     const int n = r0 + r;
     const bool valid = n < q.n;
-    const int i = valid ? q_cluster[q.lab + n] : 0;
-    const float *wrow = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * w_ld(k.n);
-    const int wl = w_ld(k.n);
-    const float *C0 = c0g + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
-    const float *C1 = c1g + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
+    const int i = valid ? q_cluster[q.lab + n] : i_first;
+    const int slot = i - i_first;
+    const bool staged = slot < kSlots;
+    const float *wrow = Wi + (int64_t)i * wl;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    TileIter it;
+    TileIter<CHUNK> it;
     it.begin(koff, k.C);
     int t = 0;
     bool ok = true;
     for (; !it.done(); it.next(), ++t) {
       const KTile kt = it.get();
-      const int buf = t & 1;
+      const int buf = t & 1, st = t % NST;
       if (!mbar_wait(&sm.sfull[buf], (t >> 1) & 1, abort_flag, status)) { ok = false; break; }
+      if (!mbar_wait(&sm.full[st], (t / NST) & 1, abort_flag, status)) { ok = false; break; }
       tc_fence_after();
       if (t >= 2 && !mbar_wait(&sm.pfree[buf], ((t - 2) >> 1) & 1, abort_flag, status)) { ok = false; break; }
-      const float a0 = valid ? C0[(int64_t)kt.j * q.n + n] : 0.f;
-      const float a1 = valid ? C1[(int64_t)kt.j * q.n + n] : 0.f;
-      for (int cb = 0; cb < kt.npad / 16; ++cb) {
+      const float a0 = sm.c0[st][r], a1 = sm.c1[st][r];
+      const int lo = kt.c - kt.x0, hi = kt.c + kt.n - kt.x0;  // unmasked columns [lo, hi)
+      const float *ws = staged ? &sm.w[st][slot][0] : wrow + kt.x0;
+      for (int cb = half; cb < kt.npad / 16; cb += 2) {
         float x[16];
         tmem_ld16(tmem + lane_base + buf * 128 + cb * 16, x);
-        const int col0 = kt.x0 + cb * 16;
+        const int col0 = cb * 16;
         float w[16];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (col0 + 4 * u < wl) v = *reinterpret_cast<const float4 *>(wrow + col0 + 4 * u);
-          w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
+          float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (staged || kt.x0 + col0 + 4 * u < wl) v4 = *reinterpret_cast<const float4 *>(ws + col0 + 4 * u);
+          w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
+        }
+        float pv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pv[e] = w[e] * fmaf(a1, x[e], a0);
+        if (!valid) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pv[e] = 0.f;
+        } else if (col0 < lo || col0 + 16 > hi) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (col0 + e < lo || col0 + e >= hi) pv[e] = 0.f;
         }
         uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
-          const int key = col0 + e;
-          const bool m0 = valid && key >= kt.c && key < kt.c + kt.n;
-          const bool m1 = valid && key + 1 >= kt.c && key + 1 < kt.c + kt.n;
-          const float p0 = m0 ? w[e] * fmaf(a1, x[e], a0) : 0.f;
-          const float p1 = m1 ? w[e + 1] * fmaf(a1, x[e + 1], a0) : 0.f;
-          __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+          __nv_bfloat162 h = __floats2bfloat162_rn(pv[e], pv[e + 1]);
           pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
         }
         // two 16-byte chunks of row r in the 128-byte-swizzled K-major block cb/4
@@ -379,7 +316,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     if (ok && t > 0 && mbar_wait(&sm.obar, 0, abort_flag, status)) {
       tc_fence_after();
       const int row = valid ? q_perm[q.lab + n] : 0;
-      for (int cb = 0; cb < DV / 16; ++cb) {
+      for (int cb = half; cb < DV / 16; cb += 2) {
         float o[16];
         tmem_ld16(tmem_o + lane_base + cb * 16, o);
         if (!valid) continue;
@@ -400,11 +337,11 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           for (int u = 0; u < 4; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
         }
       }
-      if (valid && !O) {
+      if (valid && !O && half == 0) {
         const int64_t rr = (int64_t)p * mt.in.out_stride + mt.in.out0[s] + row;
         part_lse[rr] = lse[(int64_t)p * mt.q.row_stride + q.lab + n];
       }
-    } else if (t == 0 && valid) {
+    } else if (t == 0 && valid && half == 0) {
       // an instance with no keys cannot occur (every key range is non-empty)
       report(status, MUSE_ERR_DEVICE);
     }
@@ -420,38 +357,6 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 }
 
 // ------------------------------------------------------------------ host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 2-D bf16 map: inner extent `inner` elements, `rows` rows of `ld` elements, box {64, box_rows}.
-static bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t ld,
-                     uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int DV>
 static cudaError_t launch(const MuseTables &mt, int N, int P, SortedSide qs, const int32_t *q_perm,
                           SortedSide ks, const int32_t *k_offsets, const void *vt, StageBufs b,

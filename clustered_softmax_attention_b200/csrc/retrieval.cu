@@ -1,12 +1,645 @@
-// Causal MuSe with retrieval (placeholder).
+// Causal MuSe with causal accumulation and top-k retrieval (CUDA cores).
+//
+// gist.science "Technische Samenvatting: Multipole Semantic Attention (MuSe)",
+// "Kernmechanismen" item 3 (the context is cut into spatial blocks; a block sees the
+// summaries of all preceding blocks) and item 4 (top-k1 key clusters by tilted
+// summary score, then top-k2 spatial blocks inside them; exact attention on the
+// retrieved (cluster, block) pairs and the local block diagonal; the remaining
+// interactions through the approximate summaries).
+//
+// Clusters are global (one K-means over each problem's queries and keys).  Inside
+// a key cluster the sorted keys keep their token order, so the keys of cluster j in
+// block b' form one contiguous run; pend[j][b'] counts the keys of cluster j in
+// blocks < b'.
+//
+// For query n (block b, cluster i, qt = q - qbar_i):
+//   selection: sigma_j = logsumexp_{b'<b} logZb_{i,j,b'}; the k1 largest (ties to the
+//     lower j); inside each, the k2 largest logZb_{i,j,b'}, b' < b (ties to lower b');
+//   remainder R_j = keys of cluster j in blocks < b minus the selected runs, tilted by
+//     qbar_i: logZR_{i,b,j}, and with W_ik = exp(s qbar_i.k - logZ_ij) (the whole
+//     cluster's tilt), w^R_ik = W_ik exp(logZ_ij - logZR_{i,b,j});
+//     u_j = sum_{k in R_j} w^R_ik qt.k ;  a_j = logZR + s u_j ;  p = softmax_j(a);
+//     remainder output = sum_j p_j sum_{k in R_j} w^R_ik (1 - s u_j + s qt.k) v_k
+//     (the monopole + dipole refinement of the acausal path, restricted to R_j);
+//   exact part: keys of the selected runs and the diagonal keys [bS, n];
+//   both parts are merged into one softmax through their logsumexps.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+
 #include "internal.h"
 
 namespace muse {
-size_t muse_retrieval_ws(const muse_dims &, int, int, int, int, int) { return 0; }
+namespace ret {
+
+struct Geo {
+  int N, S, nb, Cq, Ck, K12, k1, k2;
+};
+
+__device__ __forceinline__ float lse_add(float a, float b) {
+  if (a == -CUDART_INF_F) return b;
+  if (b == -CUDART_INF_F) return a;
+  const float m = fmaxf(a, b);
+  return m + logf(expf(a - m) + expf(b - m));
+}
+
+// cnt[p][j][b'] = keys of cluster j in block b' (integer atomics: exact).
+__global__ void block_counts(Geo g, const int32_t *__restrict__ k_labels, int32_t *__restrict__ cnt) {
+  const int p = blockIdx.y;
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= g.N) return;
+  const int j = k_labels[(int64_t)p * g.N + k];
+  atomicAdd(&cnt[((int64_t)p * g.Ck + j) * g.nb + k / g.S], 1);
+}
+
+// pend[p][j][b'] = keys of cluster j in blocks < b' (b' = 0..nb).
+__global__ void block_prefix(Geo g, int P, const int32_t *__restrict__ cnt, int32_t *__restrict__ pend) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= P * g.Ck) return;
+  const int32_t *c = cnt + (int64_t)t * g.nb;
+  int32_t *o = pend + (int64_t)t * (g.nb + 1);
+  int run = 0;
+  for (int b = 0; b < g.nb; ++b) {
+    o[b] = run;
+    run += c[b];
+  }
+  o[g.nb] = run;
+}
+
+// logZb[p][i][j][b'] = logZ_ij + log(sum of W_ik over the run of (j, b')); one warp per (i, j).
+__global__ void __launch_bounds__(256)
+block_lse(Geo g, int P, const float *__restrict__ W, int w_stride, const float *__restrict__ logZ,
+          const int32_t *__restrict__ k_offsets, const int32_t *__restrict__ pend,
+          float *__restrict__ logZb) {
+  const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= (int64_t)P * g.Cq * g.Ck) return;
+  const int j = (int)(wid % g.Ck);
+  const int i = (int)((wid / g.Ck) % g.Cq);
+  const int p = (int)(wid / ((int64_t)g.Ck * g.Cq));
+  const float *w = W + (int64_t)p * w_stride + (int64_t)i * w_ld(g.N);
+  const int off = k_offsets[(int64_t)p * (g.Ck + 1) + j];
+  const int32_t *pe = pend + ((int64_t)p * g.Ck + j) * (g.nb + 1);
+  const float lz = logZ[((int64_t)p * g.Cq + i) * g.Ck + j];
+  float *out = logZb + (((int64_t)p * g.Cq + i) * g.Ck + j) * g.nb;
+  for (int b = 0; b < g.nb; ++b) {
+    const int s0 = off + pe[b], s1 = off + pe[b + 1];
+    float acc = 0.f;
+    for (int pos = s0 + lane; pos < s1; pos += 32) acc += w[pos];
+    acc = warp_sum(acc);
+    if (lane == 0) out[b] = (s1 > s0) ? lz + logf(acc) : -CUDART_INF_F;
+  }
+}
+
+// One warp per (p, i, b): the selection and the remainder log-normalisers.
+// sel[p][i][b][slot] = (j, b'), slot = t*k2 + u; logZR[p][i][b][j].
+__global__ void __launch_bounds__(256)
+select_blocks(Geo g, int P, const float *__restrict__ logZb, int32_t *__restrict__ sel,
+              float *__restrict__ logZR) {
+  constexpr int MAXJ = kMaxClusters / 32;  // clusters per lane
+  const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= (int64_t)P * g.Cq * g.nb) return;
+  const int b = (int)(wid % g.nb);
+  const int i = (int)((wid / g.nb) % g.Cq);
+  const int p = (int)(wid / ((int64_t)g.nb * g.Cq));
+  const float *lzb = logZb + ((int64_t)p * g.Cq + i) * g.Ck * g.nb;  // [j][b']
+  int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
+  float *zr = logZR + (((int64_t)p * g.Cq + i) * g.nb + b) * g.Ck;
+  for (int e = lane; e < g.K12 * 2; e += 32) so[e] = -1;
+  // sigma_j for this lane's clusters j = lane + 32 m
+  float sig[MAXJ];
+  bool taken[MAXJ];
+#pragma unroll
+  for (int m = 0; m < MAXJ; ++m) {
+    sig[m] = -CUDART_INF_F;
+    taken[m] = false;
+    const int j = lane + 32 * m;
+    if (j < g.Ck)
+      for (int bb = 0; bb < b; ++bb) sig[m] = lse_add(sig[m], lzb[(int64_t)j * g.nb + bb]);
+  }
+  int chosen[64];
+  int nchosen = 0;
+  for (int t = 0; t < g.k1 && b > 0; ++t) {
+    // warp argmax of sigma over untaken finite clusters, ties to the lower j
+    float bv = -CUDART_INF_F;
+    int bj = 0x7fffffff;
+#pragma unroll
+    for (int m = 0; m < MAXJ; ++m) {
+      const int j = lane + 32 * m;
+      if (j < g.Ck && !taken[m] && sig[m] > -CUDART_INF_F && (sig[m] > bv || (sig[m] == bv && j < bj))) {
+        bv = sig[m];
+        bj = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+      if (ov > bv || (ov == bv && oj < bj)) {
+        bv = ov;
+        bj = oj;
+      }
+    }
+    if (bj == 0x7fffffff) break;  // fewer candidates than k1
+    if ((bj & 31) == lane) taken[bj >> 5] = true;
+    chosen[nchosen++] = bj;
+    // top-k2 blocks of cluster bj among b' < b (lanes over b')
+    const float *row = lzb + (int64_t)bj * g.nb;
+    unsigned used = 0u;  // bit m: block lane + 32 m already chosen
+    for (int u = 0; u < g.k2; ++u) {
+      float vv = -CUDART_INF_F;
+      int vb = 0x7fffffff;
+      for (int m = 0; m * 32 < b; ++m) {
+        const int bb = lane + 32 * m;
+        if (bb < b && !((used >> m) & 1u)) {
+          const float x = row[bb];
+          if (x > -CUDART_INF_F && (x > vv || (x == vv && bb < vb))) {
+            vv = x;
+            vb = bb;
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, vv, o);
+        const int ob = __shfl_xor_sync(0xffffffffu, vb, o);
+        if (ov > vv || (ov == vv && ob < vb)) {
+          vv = ov;
+          vb = ob;
+        }
+      }
+      if (vb == 0x7fffffff) break;
+      if ((vb & 31) == lane) used |= 1u << (vb >> 5);
+      if (lane == 0) {
+        so[(t * g.k2 + u) * 2] = bj;
+        so[(t * g.k2 + u) * 2 + 1] = vb;
+      }
+    }
+  }
+  __syncwarp();
+  // remainder log-normalisers: blocks b' < b, minus the selected runs
+#pragma unroll
+  for (int m = 0; m < MAXJ; ++m) {
+    const int j = lane + 32 * m;
+    if (j >= g.Ck) continue;
+    int tj = -1;
+    for (int t = 0; t < nchosen; ++t)
+      if (chosen[t] == j) tj = t;
+    float acc = -CUDART_INF_F;
+    for (int bb = 0; bb < b; ++bb) {
+      bool ex = false;
+      if (tj >= 0)
+        for (int u = 0; u < g.k2; ++u) ex |= (so[(tj * g.k2 + u) * 2 + 1] == bb);
+      if (!ex) acc = lse_add(acc, lzb[(int64_t)j * g.nb + bb]);
+    }
+    zr[j] = acc;
+  }
+}
+
+// Excluded blocks of cluster j for a query whose selection row is `so` (<= 64 slots).
+__device__ __forceinline__ int excluded_blocks(const int32_t *so, int K12, int j, int (&xb)[8]) {
+  int n = 0;
+  for (int s = 0; s < K12 && n < 8; ++s)
+    if (so[2 * s] == j) xb[n++] = so[2 * s + 1];
+  return n;
+}
+__device__ __forceinline__ bool in_list(int v, const int (&xb)[8], int n) {
+  bool r = false;
+#pragma unroll
+  for (int a = 0; a < 8; ++a) r |= (a < n && xb[a] == v);
+  return r;
+}
+
+// Passes over the remainder keys of every cluster, 64 queries (one block b) per CTA,
+// 4 threads per query.  MODE 0: T[j][n] = sum_{k in R_j} W_ik qt.k.
+// MODE 1: o_n = sum_j sum_{k in R_j} W_ik (c0'_{jn} + c1'_{jn} qt.k) v_k.
+template <typename T, int D, int DV, int MODE>
+__global__ void __launch_bounds__(256)
+remainder_pass(Geo g, const T *__restrict__ Q, const float *__restrict__ qcen,
+               const int32_t *__restrict__ q_labels, const T *__restrict__ ks,
+               const T *__restrict__ vs, const int32_t *__restrict__ k_perm,
+               const int32_t *__restrict__ k_offsets, const int32_t *__restrict__ pend,
+               const float *__restrict__ W, int w_stride, const int32_t *__restrict__ sel,
+               float *__restrict__ Tbuf, const float *__restrict__ c0, const float *__restrict__ c1,
+               float *__restrict__ part_o) {
+  const int p = blockIdx.y;
+  const int n0 = blockIdx.x * 64;
+  const int b = n0 / g.S;
+  if (b == 0) return;  // block 0 has no remainder
+  __shared__ float Ks[32][D];
+  __shared__ float Vs[MODE ? 32 : 1][DV];
+  __shared__ int Bk[32];
+  const int gq = threadIdx.x & 3;
+  const int n = n0 + (threadIdx.x >> 2);
+  constexpr int PD = D / 4, PV = DV / 4;
+  const int i = q_labels[(int64_t)p * g.N + n];
+  float qt[PD];
+#pragma unroll
+  for (int t = 0; t < PD; ++t)
+    qt[t] = ld_elem(Q + ((int64_t)p * g.N + n) * D + gq + 4 * t) - qcen[((int64_t)p * g.Cq + i) * D + gq + 4 * t];
+  const float *wrow = W + (int64_t)p * w_stride + (int64_t)i * w_ld(g.N);
+  const int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
+  float acc[MODE ? PV : 1];
+#pragma unroll
+  for (int t = 0; t < (MODE ? PV : 1); ++t) acc[t] = 0.f;
+  const int32_t *koff = k_offsets + (int64_t)p * (g.Ck + 1);
+  const T *kp = ks + (int64_t)p * g.N * D;
+  const T *vp = vs + (int64_t)p * g.N * DV;
+  for (int j = 0; j < g.Ck; ++j) {
+    const int s0 = koff[j];
+    const int s1 = s0 + pend[((int64_t)p * g.Ck + j) * (g.nb + 1) + b];
+    if (s1 <= s0) continue;  // CTA-uniform
+    int xb[8];
+    const int nx = excluded_blocks(so, g.K12, j, xb);
+    float tsum = 0.f, a0 = 0.f, a1 = 0.f;
+    if (MODE) {
+      a0 = c0[((int64_t)p * g.Ck + j) * g.N + n];
+      a1 = c1[((int64_t)p * g.Ck + j) * g.N + n];
+    }
+    for (int k0 = s0; k0 < s1; k0 += 32) {
+      const int kt = min(32, s1 - k0);
+      __syncthreads();
+      for (int e = threadIdx.x; e < kt * D; e += blockDim.x) Ks[e / D][e % D] = ld_elem(kp + (int64_t)k0 * D + e);
+      if (MODE)
+        for (int e = threadIdx.x; e < kt * DV; e += blockDim.x)
+          Vs[e / DV][e % DV] = ld_elem(vp + (int64_t)k0 * DV + e);
+      if (threadIdx.x < kt) Bk[threadIdx.x] = k_perm[(int64_t)p * g.N + k0 + threadIdx.x] / g.S;
+      __syncthreads();
+      for (int kk = 0; kk < kt; ++kk) {
+        float x = 0.f;
+#pragma unroll
+        for (int t = 0; t < PD; ++t) x = fmaf(qt[t], Ks[kk][gq + 4 * t], x);
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        x += __shfl_xor_sync(0xffffffffu, x, 2);
+        if (nx && in_list(Bk[kk], xb, nx)) continue;
+        const float w = wrow[k0 + kk];
+        if (MODE) {
+          const float P = w * fmaf(a1, x, a0);
+#pragma unroll
+          for (int t = 0; t < PV; ++t) acc[t] = fmaf(P, Vs[kk][gq + 4 * t], acc[t]);
+        } else {
+          tsum = fmaf(w, x, tsum);
+        }
+      }
+    }
+    if (!MODE && gq == 0) Tbuf[((int64_t)p * g.Ck + j) * g.N + n] = tsum;
+  }
+  if (MODE) {
+#pragma unroll
+    for (int t = 0; t < PV; ++t) part_o[((int64_t)p * g.N + n) * DV + gq + 4 * t] = acc[t];
+  }
+}
+
+// Remainder coefficients per query (natural order):
+//   U_j = exp(logZ_ij - logZR) T_j;  a_j = logZR + s U_j;  p = softmax(a);
+//   c0'_j = p_j (1 - s U_j) exp(logZ_ij - logZR),  c1'_j = s p_j exp(logZ_ij - logZR).
+__global__ void __launch_bounds__(128)
+remainder_coeffs(Geo g, int P, float scale, const int32_t *__restrict__ q_labels,
+                 const float *__restrict__ logZ, const float *__restrict__ logZR,
+                 const float *__restrict__ Tbuf, float *__restrict__ c0, float *__restrict__ c1,
+                 float *__restrict__ lse_r) {
+  const int p = blockIdx.y;
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= g.N) return;
+  const int b = n / g.S;
+  const int i = q_labels[(int64_t)p * g.N + n];
+  const float *lz = logZ + ((int64_t)p * g.Cq + i) * g.Ck;
+  const float *zr = logZR + (((int64_t)p * g.Cq + i) * g.nb + b) * g.Ck;
+  float m = -CUDART_INF_F, l = 0.f;
+  for (int pass = 0; pass < 2; ++pass) {
+    const float inv = pass ? 1.f / l : 0.f;
+    for (int j = 0; j < g.Ck; ++j) {
+      const int64_t at = ((int64_t)p * g.Ck + j) * g.N + n;
+      const float r = zr[j];
+      if (b == 0 || !(r > -CUDART_INF_F)) {
+        if (pass) {
+          c0[at] = 0.f;
+          c1[at] = 0.f;
+        }
+        continue;
+      }
+      const float f = expf(lz[j] - r);
+      const float U = f * Tbuf[at];
+      const float a = r + scale * U;
+      if (!pass) {
+        if (a > m) {
+          l = l * expf(m - a) + 1.f;
+          m = a;
+        } else {
+          l += expf(a - m);
+        }
+      } else {
+        const float pj = expf(a - m) * inv;
+        c0[at] = pj * (1.f - scale * U) * f;
+        c1[at] = scale * pj * f;
+      }
+    }
+  }
+  lse_r[(int64_t)p * g.N + n] = (l > 0.f) ? m + logf(l) : -CUDART_INF_F;
+}
+
+// Exact part (diagonal keys [bS, n] and the selected runs) with online softmax, merged
+// with the remainder partial (lse_r, o_r).  64 queries per CTA, 4 threads per query.
+template <typename T, int D, int DV>
+__global__ void __launch_bounds__(256)
+exact_merge(Geo g, float scale, const T *__restrict__ Q, const T *__restrict__ K,
+            const T *__restrict__ V, const int32_t *__restrict__ q_labels,
+            const T *__restrict__ ks, const T *__restrict__ vs,
+            const int32_t *__restrict__ k_offsets, const int32_t *__restrict__ pend,
+            const int32_t *__restrict__ sel, const float *__restrict__ part_o,
+            const float *__restrict__ lse_r, T *__restrict__ O) {
+  const int p = blockIdx.y;
+  const int n0 = blockIdx.x * 64;
+  const int b = n0 / g.S;
+  __shared__ float Ks[32][D];
+  __shared__ float Vs[32][DV];
+  const int gq = threadIdx.x & 3;
+  const int n = n0 + (threadIdx.x >> 2);
+  constexpr int PD = D / 4, PV = DV / 4;
+  float qv[PD];
+#pragma unroll
+  for (int t = 0; t < PD; ++t) qv[t] = ld_elem(Q + ((int64_t)p * g.N + n) * D + gq + 4 * t) * scale;
+  float m = -CUDART_INF_F, l = 0.f;
+  float acc[PV];
+#pragma unroll
+  for (int t = 0; t < PV; ++t) acc[t] = 0.f;
+  auto add = [&](float x, const float *vrow, int stride) {
+    const float mn = fmaxf(m, x);
+    const float corr = expf(m - mn), pe = expf(x - mn);
+    l = l * corr + pe;
+#pragma unroll
+    for (int t = 0; t < PV; ++t) acc[t] = fmaf(pe, vrow[t * stride], acc[t] * corr);
+    m = mn;
+  };
+  // diagonal block, keys [bS, n]
+  const int kend = n0 + 64;
+  for (int k0 = b * g.S; k0 < kend; k0 += 32) {
+    const int kt = min(32, kend - k0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < kt * D; e += blockDim.x)
+      Ks[e / D][e % D] = ld_elem(K + ((int64_t)p * g.N + k0) * D + e);
+    for (int e = threadIdx.x; e < kt * DV; e += blockDim.x)
+      Vs[e / DV][e % DV] = ld_elem(V + ((int64_t)p * g.N + k0) * DV + e);
+    __syncthreads();
+    for (int kk = 0; kk < kt; ++kk) {
+      float x = 0.f;
+#pragma unroll
+      for (int t = 0; t < PD; ++t) x = fmaf(qv[t], Ks[kk][gq + 4 * t], x);
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
+      if (k0 + kk <= n) add(x, &Vs[kk][gq], 4);
+    }
+  }
+  // selected runs (sorted positions), per query
+  if (b > 0) {
+    const int i = q_labels[(int64_t)p * g.N + n];
+    const int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
+    const int32_t *koff = k_offsets + (int64_t)p * (g.Ck + 1);
+    for (int s = 0; s < g.K12; ++s) {
+      const int j = so[2 * s], bb = so[2 * s + 1];
+      if (j < 0) continue;
+      const int32_t *pe = pend + ((int64_t)p * g.Ck + j) * (g.nb + 1);
+      const int s0 = koff[j] + pe[bb], s1 = koff[j] + pe[bb + 1];
+      for (int pos = s0; pos < s1; ++pos) {
+        const T *kr = ks + ((int64_t)p * g.N + pos) * D;
+        float x = 0.f;
+#pragma unroll
+        for (int t = 0; t < PD; ++t) x = fmaf(qv[t], ld_elem(kr + gq + 4 * t), x);
+        // the 4 lanes of this query follow the same runs
+        const unsigned gm = 0xFu << ((threadIdx.x & 31) & ~3);
+        x += __shfl_xor_sync(gm, x, 1);
+        x += __shfl_xor_sync(gm, x, 2);
+        float vr[PV];
+        const T *vrp = vs + ((int64_t)p * g.N + pos) * DV;
+#pragma unroll
+        for (int t = 0; t < PV; ++t) vr[t] = ld_elem(vrp + gq + 4 * t);
+        add(x, vr, 1);
+      }
+    }
+    const float L = lse_r[(int64_t)p * g.N + n];
+    if (L > -CUDART_INF_F) {
+      const float mn = fmaxf(m, L);
+      const float ca = expf(m - mn), cb = expf(L - mn);
+      l = l * ca + cb;
+#pragma unroll
+      for (int t = 0; t < PV; ++t)
+        acc[t] = acc[t] * ca + cb * part_o[((int64_t)p * g.N + n) * DV + gq + 4 * t];
+      m = mn;
+    }
+  }
+  const float inv = 1.f / l;
+  T *o = O + ((int64_t)p * g.N + n) * DV;
+#pragma unroll
+  for (int t = 0; t < PV; ++t) st_elem(o + gq + 4 * t, acc[t] * inv);
+}
+
+// Workspace layout.
+struct Ws {
+  KmeansOut q, k;
+  char *km_scratch;
+  SortedSide ks;
+  void *vs;
+  int32_t *v_cluster;
+  float *W, *logZ;
+  int32_t *cnt, *pend, *sel;
+  float *logZb, *logZR, *T, *c0, *c1, *lse_r, *part_o;
+};
+
+struct Bump2 {
+  char *base;
+  size_t off = 0;
+  explicit Bump2(void *b) : base(static_cast<char *>(b)) {}
+  template <typename X>
+  X *take(size_t count) {
+    const size_t o = off;
+    off = align_up(off + count * sizeof(X));
+    return base ? reinterpret_cast<X *>(base + o) : nullptr;
+  }
+};
+
+static SegTable whole(int N, int C) {
+  SegTable t;
+  memset(&t, 0, sizeof(t));
+  t.nseg = 1;
+  t.row_stride = N;
+  t.cen_stride = C;
+  t.off_stride = C + 1;
+  t.max_rows = N;
+  t.max_C = C;
+  t.nrow[0] = N;
+  t.C[0] = C;
+  return t;
+}
+
+static MuseTables tables(int N, int Cq, int Ck) {
+  MuseTables mt;
+  memset(&mt, 0, sizeof(mt));
+  mt.q = whole(N, Cq);
+  mt.k = whole(N, Ck);
+  mt.in.ninst = 1;
+  mt.in.w_stride = Cq * w_ld(N);
+  mt.in.z_stride = Cq * Ck;
+  mt.in.c_stride = Ck * w_ld(N);
+  mt.in.out_stride = N;
+  return mt;
+}
+
+static void plan(Bump2 &bp, const muse_dims &d, const Geo &g, Ws &w) {
+  const int P = d.B * d.H;
+  const size_t es = d.dtype == MUSE_F32 ? 4 : 2;
+  MuseTables mt = tables(d.N, g.Cq, g.Ck);
+  auto side = [&](const SegTable &t, KmeansOut &o) {
+    o.labels = bp.take<int32_t>((size_t)P * t.row_stride);
+    o.centroids = bp.take<float>((size_t)P * t.cen_stride * d.D);
+    o.perm = bp.take<int32_t>((size_t)P * t.row_stride);
+    o.offsets = bp.take<int32_t>((size_t)P * t.off_stride);
+  };
+  side(mt.q, w.q);
+  side(mt.k, w.k);
+  w.km_scratch = bp.take<char>(kmeans_pair_ws_bytes(&mt.q, &mt.k, P, d.D));
+  w.ks.rows = bp.take<char>((size_t)P * d.N * d.D * es);
+  w.ks.cluster = bp.take<int32_t>((size_t)P * d.N);
+  w.vs = bp.take<char>((size_t)P * d.N * d.Dv * es);
+  w.v_cluster = bp.take<int32_t>((size_t)P * d.N);
+  w.W = bp.take<float>((size_t)P * mt.in.w_stride);
+  w.logZ = bp.take<float>((size_t)P * g.Cq * g.Ck);
+  w.cnt = bp.take<int32_t>((size_t)P * g.Ck * g.nb);
+  w.pend = bp.take<int32_t>((size_t)P * g.Ck * (g.nb + 1));
+  w.sel = bp.take<int32_t>((size_t)P * g.Cq * g.nb * g.K12 * 2);
+  w.logZb = bp.take<float>((size_t)P * g.Cq * g.Ck * g.nb);
+  w.logZR = bp.take<float>((size_t)P * g.Cq * g.nb * g.Ck);
+  w.T = bp.take<float>((size_t)P * g.Ck * d.N);
+  w.c0 = bp.take<float>((size_t)P * g.Ck * d.N);
+  w.c1 = bp.take<float>((size_t)P * g.Ck * d.N);
+  w.lse_r = bp.take<float>((size_t)P * d.N);
+  w.part_o = bp.take<float>((size_t)P * d.N * d.Dv);
+}
+
+static bool valid_geo(const muse_dims &d, int block, int Cq, int Ck, int k1, int k2, Geo &g) {
+  if (block <= 0 || block % 64 || d.N % block) return false;
+  if (Cq < 1 || Ck < 1 || Cq > d.N || Ck > d.N || Cq > kMaxClusters || Ck > kMaxClusters) return false;
+  const int nb = d.N / block;
+  if (nb > 1024) return false;
+  if (k1 < 0 || k2 < 0 || k1 > Ck || k2 > nb || k1 * k2 > 64) return false;
+  if (k2 == 0) k1 = 0;  // a cluster retrieved with no block excludes nothing
+  g.N = d.N;
+  g.S = block;
+  g.nb = nb;
+  g.Cq = Cq;
+  g.Ck = Ck;
+  g.k1 = k1;
+  g.k2 = k2;
+  g.K12 = std::max(1, k1 * k2);
+  return true;
+}
+
+template <typename T, int D, int DV>
+static cudaError_t run_t(const void *Q, const void *K, const void *V, const muse_dims &d,
+                         const Geo &g, int iters, Ws &w, void *O, int *status, cudaStream_t st) {
+  const int P = d.B * d.H;
+  MuseTables mt = tables(d.N, g.Cq, g.Ck);
+  cudaError_t e;
+  if ((e = run_kmeans_pair(Q, mt.q, w.q, K, mt.k, w.k, d.dtype, D, d.N, P, iters, w.km_scratch,
+                           status, st)) != cudaSuccess)
+    return e;
+  if ((e = run_sort_side(K, d.dtype, D, d.N, mt.k, P, w.k.perm, w.k.offsets, nullptr, w.ks, st)) !=
+      cudaSuccess)
+    return e;
+  SortedSide vsd{w.vs, w.v_cluster};
+  if ((e = run_sort_side(V, d.dtype, DV, d.N, mt.k, P, w.k.perm, w.k.offsets, nullptr, vsd, st)) !=
+      cudaSuccess)
+    return e;
+  StageBufs sb;
+  memset(&sb, 0, sizeof(sb));
+  sb.W = w.W;
+  sb.logZ = w.logZ;
+  if ((e = run_summaries(mt, d.dtype, D, DV, P, d.scale, w.q.centroids, w.ks, nullptr, w.k.offsets,
+                         sb, st)) != cudaSuccess)
+    return e;
+  if ((e = cudaMemsetAsync(w.cnt, 0, (size_t)P * g.Ck * g.nb * sizeof(int32_t), st)) != cudaSuccess)
+    return e;
+  block_counts<<<dim3((d.N + 255) / 256, P), 256, 0, st>>>(g, w.k.labels, w.cnt);
+  block_prefix<<<(P * g.Ck + 127) / 128, 128, 0, st>>>(g, P, w.cnt, w.pend);
+  const int64_t nw = (int64_t)P * g.Cq * g.Ck;
+  block_lse<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(g, P, w.W, mt.in.w_stride, w.logZ,
+                                                      w.k.offsets, w.pend, w.logZb);
+  const int64_t ns = (int64_t)P * g.Cq * g.nb;
+  select_blocks<<<(unsigned)((ns + 7) / 8), 256, 0, st>>>(g, P, w.logZb, w.sel, w.logZR);
+  dim3 qg(d.N / 64, P);
+  remainder_pass<T, D, DV, 0><<<qg, 256, 0, st>>>(
+      g, (const T *)Q, w.q.centroids, w.q.labels, (const T *)w.ks.rows, (const T *)w.vs, w.k.perm,
+      w.k.offsets, w.pend, w.W, mt.in.w_stride, w.sel, w.T, nullptr, nullptr, nullptr);
+  remainder_coeffs<<<dim3((d.N + 127) / 128, P), 128, 0, st>>>(g, P, d.scale, w.q.labels, w.logZ,
+                                                                w.logZR, w.T, w.c0, w.c1, w.lse_r);
+  remainder_pass<T, D, DV, 1><<<qg, 256, 0, st>>>(
+      g, (const T *)Q, w.q.centroids, w.q.labels, (const T *)w.ks.rows, (const T *)w.vs, w.k.perm,
+      w.k.offsets, w.pend, w.W, mt.in.w_stride, w.sel, nullptr, w.c0, w.c1, w.part_o);
+  exact_merge<T, D, DV><<<qg, 256, 0, st>>>(g, d.scale, (const T *)Q, (const T *)K, (const T *)V,
+                                            w.q.labels, (const T *)w.ks.rows, (const T *)w.vs,
+                                            w.k.offsets, w.pend, w.sel, w.part_o, w.lse_r, (T *)O);
+  count_launches(8);
+  return cudaGetLastError();
+}
+
+}  // namespace ret
+
+size_t muse_retrieval_ws(const muse_dims &d, int block, int Cq, int Ck, int k1, int k2) {
+  ret::Geo g;
+  if (!ret::valid_geo(d, block, Cq, Ck, k1, k2, g)) return 0;
+  ret::Bump2 bp(nullptr);
+  ret::Ws w;
+  ret::plan(bp, d, g, w);
+  return bp.off;
+}
+
+int *device_status_word();
+
 }  // namespace muse
 
-extern "C" muse_status muse_retrieve_exact(const void *, const void *, const void *, muse_dims,
-                                           int, int, int, int, int, int, int32_t *, int32_t *,
-                                           int32_t *, void *, void *, size_t, muse_stream_t) {
-  return MUSE_ERR_SHAPE;
+using namespace muse;
+
+extern "C" muse_status muse_retrieve_exact(const void *Q, const void *K, const void *V, muse_dims d,
+                                           int block, int Cq, int Ck, int iters, int k1, int k2,
+                                           int32_t *q_labels_out, int32_t *k_labels_out,
+                                           int32_t *selected_pairs, void *O, void *ws,
+                                           size_t ws_bytes, muse_stream_t st) {
+  if (d.dtype != MUSE_F32 && d.dtype != MUSE_BF16) return MUSE_ERR_DTYPE;
+  if (d.B <= 0 || d.H <= 0 || d.N <= 0 || (d.D != 64 && d.D != 128) || (d.Dv != 64 && d.Dv != 128))
+    return MUSE_ERR_SHAPE;
+  if ((int64_t)d.B * d.H > 65535 || (int64_t)d.N * 128 > ((int64_t)1 << 31)) return MUSE_ERR_SHAPE;
+  if (!isfinite(d.scale)) return MUSE_ERR_INVALID_ARG;
+  for (const void *p : {Q, K, V, (const void *)O})
+    if (!p || (reinterpret_cast<uintptr_t>(p) & 15u)) return MUSE_ERR_INVALID_ARG;
+  for (const void *p : {(const void *)q_labels_out, (const void *)k_labels_out,
+                        (const void *)selected_pairs})
+    if (p && (reinterpret_cast<uintptr_t>(p) & 15u)) return MUSE_ERR_INVALID_ARG;
+  if (block <= 0 || block % 64 || d.N % block) return MUSE_ERR_SHAPE;
+  if (iters < 1 || iters > 1000) return MUSE_ERR_INVALID_ARG;
+  ret::Geo g;
+  if (!ret::valid_geo(d, block, Cq, Ck, k1, k2, g)) return MUSE_ERR_INVALID_ARG;
+  const size_t need = muse_retrieval_ws(d, block, Cq, Ck, k1, k2);
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) return MUSE_ERR_WORKSPACE;
+  ret::Bump2 bp(ws);
+  ret::Ws w;
+  ret::plan(bp, d, g, w);
+  if (q_labels_out) w.q.labels = q_labels_out;
+  if (k_labels_out) w.k.labels = k_labels_out;
+  if (selected_pairs) w.sel = selected_pairs;
+  cudaError_t e;
+  int *status = device_status_word();
+  cudaStream_t cs = (cudaStream_t)st;
+  if (d.dtype == MUSE_F32) {
+    if (d.D == 64 && d.Dv == 64) e = ret::run_t<float, 64, 64>(Q, K, V, d, g, iters, w, O, status, cs);
+    else if (d.D == 64) e = ret::run_t<float, 64, 128>(Q, K, V, d, g, iters, w, O, status, cs);
+    else if (d.Dv == 64) e = ret::run_t<float, 128, 64>(Q, K, V, d, g, iters, w, O, status, cs);
+    else e = ret::run_t<float, 128, 128>(Q, K, V, d, g, iters, w, O, status, cs);
+  } else {
+    if (d.D == 64 && d.Dv == 64) e = ret::run_t<__nv_bfloat16, 64, 64>(Q, K, V, d, g, iters, w, O, status, cs);
+    else if (d.D == 64) e = ret::run_t<__nv_bfloat16, 64, 128>(Q, K, V, d, g, iters, w, O, status, cs);
+    else if (d.Dv == 64) e = ret::run_t<__nv_bfloat16, 128, 64>(Q, K, V, d, g, iters, w, O, status, cs);
+    else e = ret::run_t<__nv_bfloat16, 128, 128>(Q, K, V, d, g, iters, w, O, status, cs);
+  }
+  return e == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
 }

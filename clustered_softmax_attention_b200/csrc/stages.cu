@@ -32,25 +32,30 @@ __device__ __forceinline__ Task k_task(const MuseTables &mt, int p, int s) {
 // One CTA per (cluster, task).
 // ---------------------------------------------------------------------------
 template <typename T>
-__global__ void sort_side(const T *__restrict__ X, int N, int W, SegTable tab,
-                          const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
-                          const float *__restrict__ centroids, T *__restrict__ rows,
-                          int32_t *__restrict__ cluster) {
+__global__ void __launch_bounds__(256)
+sort_side(const T *__restrict__ X, int N, int W, SegTable tab, const int32_t *__restrict__ perm,
+          const int32_t *__restrict__ offsets, const float *__restrict__ centroids,
+          T *__restrict__ rows, int32_t *__restrict__ cluster) {
+  constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte vector
   const Task tk = make_task(tab, blockIdx.y);
   const int c = blockIdx.x;
   if (c >= tk.C) return;
   const int b = offsets[tk.off + c], e = offsets[tk.off + c + 1];
-  const float *cen = centroids ? centroids + (tk.cen + c) * W : nullptr;
-  for (int m = b; m < e; ++m) {
+  const int vpr = W / VEC, slots = 256 / vpr;
+  const int v = threadIdx.x % vpr, slot = threadIdx.x / vpr;
+  float cv[VEC];
+#pragma unroll
+  for (int u = 0; u < VEC; ++u) cv[u] = centroids ? centroids[(tk.cen + c) * W + v * VEC + u] : 0.f;
+  for (int m = b + slot; m < e; m += slots) {
     const int row = perm[tk.lab + m];
-    const T *src = X + ((int64_t)tk.p * N + row) * W;
-    T *dst = rows + (tk.lab + m) * W;
-    for (int d = threadIdx.x; d < W; d += blockDim.x) {
-      float v = ld_elem(src + d);
-      if (cen) v -= cen[d];
-      st_elem(dst + d, v);
+    uint4 raw = *reinterpret_cast<const uint4 *>(X + ((int64_t)tk.p * N + row) * W + v * VEC);
+    if (centroids) {
+      T *el = reinterpret_cast<T *>(&raw);
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) st_elem(el + u, ld_elem(el + u) - cv[u]);
     }
-    if (threadIdx.x == 0) cluster[tk.lab + m] = c;
+    *reinterpret_cast<uint4 *>(rows + (tk.lab + m) * W + v * VEC) = raw;
+    if (v == 0) cluster[tk.lab + m] = c;
   }
 }
 
@@ -200,41 +205,54 @@ template <typename T, int WD>
 __global__ void __launch_bounds__(256)
 tilt_moments(MuseTables mt, const int32_t *__restrict__ k_offsets, const float *__restrict__ W,
              const T *__restrict__ xs, float *__restrict__ mu) {
+  constexpr int PW = WD / 16;  // coordinates per thread (interleaved by 16)
+  __shared__ float Ws[64][33];
+  __shared__ float Xs[32][WD + 4];
   const int p = blockIdx.z / mt.in.ninst, s = blockIdx.z % mt.in.ninst;
   const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
   const int Cq = q.C, Ck = k.C, nk = k.n;
-  const int j = blockIdx.x;
-  if (j >= Ck) return;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int ib = blockIdx.y * 32 + wid * 4;
-  if (ib >= Cq) return;
+  const int j = blockIdx.x, i0 = blockIdx.y * 64;
+  if (j >= Ck || i0 >= Cq) return;
   const int b = k_offsets[k.off + j], e = k_offsets[k.off + j + 1];
-  constexpr int PER = WD / 32;
-  float acc[4][PER];
+  const int ti = threadIdx.x >> 4, td = threadIdx.x & 15;
+  float acc[4][PW];
 #pragma unroll
-  for (int t = 0; t < 4; ++t)
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int u = 0; u < PER; ++u) acc[t][u] = 0.f;
+    for (int u = 0; u < PW; ++u) acc[a][u] = 0.f;
   const float *wb = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s];
-  for (int pos = b; pos < e; ++pos) {
-    float xv[PER];
+  const int wl = w_ld(nk);
+  for (int pc = b; pc < e; pc += 32) {
+    const int pt = min(32, e - pc);
+    __syncthreads();
+    for (int x = threadIdx.x; x < 64 * 32; x += 256) {
+      const int ii = x >> 5, pp = x & 31;
+      Ws[ii][pp] = (i0 + ii < Cq && pp < pt) ? wb[(int64_t)(i0 + ii) * wl + pc + pp] : 0.f;
+    }
+    for (int x = threadIdx.x; x < 32 * WD; x += 256) {
+      const int pp = x / WD, d = x % WD;
+      Xs[pp][d] = pp < pt ? ld_elem(xs + (k.lab + pc + pp) * WD + d) : 0.f;
+    }
+    __syncthreads();
+    for (int pp = 0; pp < pt; ++pp) {
+      float xv[PW];
 #pragma unroll
-    for (int u = 0; u < PER; ++u) xv[u] = ld_elem(xs + (k.lab + pos) * WD + lane + 32 * u);
+      for (int u = 0; u < PW; ++u) xv[u] = Xs[pp][td + 16 * u];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int i = ib + t;
-      const float w = (i < Cq) ? wb[(int64_t)i * w_ld(nk) + pos] : 0.f;
+      for (int a = 0; a < 4; ++a) {
+        const float w = Ws[ti * 4 + a][pp];
 #pragma unroll
-      for (int u = 0; u < PER; ++u) acc[t][u] = fmaf(w, xv[u], acc[t][u]);
+        for (int u = 0; u < PW; ++u) acc[a][u] = fmaf(w, xv[u], acc[a][u]);
+      }
     }
   }
 #pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const int i = ib + t;
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + ti * 4 + a;
     if (i >= Cq) continue;
     float *o = mu + ((int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck + j) * WD;
 #pragma unroll
-    for (int u = 0; u < PER; ++u) o[lane + 32 * u] = acc[t][u];
+    for (int u = 0; u < PW; ++u) o[td + 16 * u] = acc[a][u];
   }
 }
 
@@ -288,7 +306,7 @@ refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
   if (i >= Cq) return;
   const int b = q_offsets[q.off + i], e = q_offsets[q.off + i + 1];
   if (e <= b) return;
-  float *lz = sm;               // [Ck]
+  float *lz = sm;                 // [Ck]
   float *mk = sm + kMaxClusters;  // [32][D]
   const int64_t zrow = (int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck;
   for (int j = threadIdx.x; j < Ck; j += blockDim.x) lz[j] = logZ[zrow + j];
@@ -300,39 +318,44 @@ refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
     float qt[D];
 #pragma unroll
     for (int d = 0; d < D; ++d) qt[d] = v ? ld_elem(qt_rows + (q.lab + n) * D + d) : 0.f;
-    float m = -CUDART_INF_F;
-    for (int j0 = 0; j0 < Ck; j0 += 32) {
-      const int jt = min(32, Ck - j0);
-      __syncthreads();
-      for (int e2 = threadIdx.x; e2 < jt * D; e2 += blockDim.x)
-        mk[e2] = mu_k[(zrow + j0) * D + e2];
-      __syncthreads();
-      if (v) {
+    // pass 0: running max and sum of exp(a_j - max); pass 1: the coefficients
+    float m = -CUDART_INF_F, l = 0.f;
+    for (int pass = 0; pass < 2; ++pass) {
+      const float inv = pass ? 1.f / l : 0.f;
+      for (int j0 = 0; j0 < Ck; j0 += 32) {
+        const int jt = min(32, Ck - j0);
+        __syncthreads();
+        for (int e2 = threadIdx.x; e2 < jt * D; e2 += blockDim.x)
+          mk[e2] = mu_k[(zrow + j0) * D + e2];
+        __syncthreads();
+        if (!v) continue;
         for (int jj = 0; jj < jt; ++jj) {
           float u = 0.f;
+          const float4 *m4 = reinterpret_cast<const float4 *>(mk + jj * D);
 #pragma unroll
-          for (int d = 0; d < D; ++d) u = fmaf(qt[d], mk[jj * D + d], u);
+          for (int d4 = 0; d4 < D / 4; ++d4) {
+            const float4 w4 = m4[d4];
+            u = fmaf(qt[4 * d4], w4.x, fmaf(qt[4 * d4 + 1], w4.y,
+                     fmaf(qt[4 * d4 + 2], w4.z, fmaf(qt[4 * d4 + 3], w4.w, u))));
+          }
           const int j = j0 + jj;
           const float a = lz[j] + scale * u;
-          C0[(int64_t)j * nq + n] = a;
-          C1[(int64_t)j * nq + n] = u;
-          m = fmaxf(m, a);
+          if (pass == 0) {
+            if (a > m) {
+              l = l * __expf(m - a) + 1.f;
+              m = a;
+            } else if (a > -CUDART_INF_F) {
+              l += __expf(a - m);
+            }
+          } else {
+            const float pj = (a > -CUDART_INF_F) ? __expf(a - m) * inv : 0.f;
+            C0[(int64_t)j * w_ld(nq) + n] = pj * (1.f - scale * u);
+            C1[(int64_t)j * w_ld(nq) + n] = scale * pj;
+          }
         }
       }
     }
-    if (v) {
-      float l = 0.f;
-      for (int j = 0; j < Ck; ++j) l += expf(C0[(int64_t)j * nq + n] - m);
-      const float inv = 1.f / l;
-      for (int j = 0; j < Ck; ++j) {
-        const float a = C0[(int64_t)j * nq + n];
-        const float u = C1[(int64_t)j * nq + n];
-        const float pj = expf(a - m) * inv;
-        C0[(int64_t)j * nq + n] = pj * (1.f - scale * u);
-        C1[(int64_t)j * nq + n] = scale * pj;
-      }
-      lse[(int64_t)p * mt.q.row_stride + q.lab + n] = m + logf(l);
-    }
+    if (v) lse[(int64_t)p * mt.q.row_stride + q.lab + n] = m + logf(l);
   }
 }
 
@@ -390,8 +413,8 @@ refine_simt(MuseTables mt, int N, const T *__restrict__ qt_rows, const int32_t *
       const int j = Js[kk];
       if (j != curj) {
         curj = j;
-        a0 = v ? C0[(int64_t)j * nq + n] : 0.f;
-        a1 = v ? C1[(int64_t)j * nq + n] : 0.f;
+        a0 = v ? C0[(int64_t)j * w_ld(nq) + n] : 0.f;
+        a1 = v ? C1[(int64_t)j * w_ld(nq) + n] : 0.f;
       }
       const float P = v ? wrow[k0 + kk] * fmaf(a1, x, a0) : 0.f;
 #pragma unroll
@@ -493,7 +516,7 @@ cudaError_t run_sort_side(const void *X, int dtype, int width, int N, const SegT
                           const int32_t *perm, const int32_t *offsets, const float *centroids,
                           SortedSide out, cudaStream_t st) {
   dim3 grid(tab.max_C, P * tab.nseg);
-  const int threads = width;
+  const int threads = 256;
   count_launches(1);
   if (dtype == MUSE_F32)
     sort_side<float><<<grid, threads, 0, st>>>((const float *)X, N, width, tab, perm, offsets,
@@ -532,10 +555,10 @@ static cudaError_t summaries_t(const MuseTables &mt, int P, float scale, const f
   tilt_lse<<<dim3((maxCq * maxCk + 7) / 8, tasks), 256, 0, st>>>(mt, k_offsets, b.W, b.logZ);
   count_launches(2 + (b.mu_k != nullptr) + (b.mu_v != nullptr) + (b.cov != nullptr));
   if (b.mu_k)
-    tilt_moments<T, D><<<dim3(maxCk, (maxCq + 31) / 32, tasks), 256, 0, st>>>(
+    tilt_moments<T, D><<<dim3(maxCk, (maxCq + 63) / 64, tasks), 256, 0, st>>>(
         mt, k_offsets, b.W, (const T *)ks.rows, b.mu_k);
   if (b.mu_v)
-    tilt_moments<T, DV><<<dim3(maxCk, (maxCq + 31) / 32, tasks), 256, 0, st>>>(
+    tilt_moments<T, DV><<<dim3(maxCk, (maxCq + 63) / 64, tasks), 256, 0, st>>>(
         mt, k_offsets, b.W, (const T *)vs, b.mu_v);
   if (b.cov)
     tilt_cov<T, D, DV><<<dim3(maxCk, maxCq, tasks), 256, 0, st>>>(

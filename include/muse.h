@@ -205,9 +205,10 @@ muse_status muse_causal_blocks(const void *Q, const void *K, const void *V, muse
  *   blocks) and 4 (top-k1 clusters, top-k2 blocks, exact on retrieved pairs plus
  *   the local diagonal, summaries for the rest).
  * Optional outputs: q_labels_out, k_labels_out int32 [B,H,N];
- *   selected_pairs int32 [B,H,Cq,N/block,k1*k2,2]: (cluster, block) of slot
+ *   selected_pairs int32 [B,H,Cq,N/block,max(1,k1*k2),2]: (cluster, block) of slot
  *   t*k2+u = the u-th block of the t-th cluster, (-1,-1) when unused.
- * N % block == 0; 0 <= k1 <= Ck; 0 <= k2 <= N/block; k1*k2 <= 64.
+ * N % block == 0, block a multiple of 64, N/block <= 1024; 0 <= k1 <= Ck;
+ * 0 <= k2 <= N/block; k1*k2 <= 64.  Runs on the CUDA cores (float32 arithmetic).
  */
 muse_status muse_retrieve_exact(const void *Q, const void *K, const void *V, muse_dims d,
                                 int block, int Cq, int Ck, int iters, int k1, int k2,

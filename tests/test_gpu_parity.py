@@ -218,3 +218,52 @@ def test_full_size_acausal_n8k_sampled_rows():
                                   w.scale, rows=rows)
         err = np.abs(O[0, h][rows] - ref[rows]).max() / np.abs(ref[rows]).max()
         assert err <= TOL["bf16"], err
+
+
+# --------------------------------------------------------------------------- retrieval
+
+def retrieval_case(dt, N, S, C, k1, k2, seed=9, H=2, scale=1.0, outliers=0.0):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    from clustered_softmax_attention_b200.inputs import draw_problem, round_to_bf16
+    cast = round_to_bf16 if dt == "bf16" else (lambda a: a.astype(np.float32))
+    Qs, Ks, Vs = zip(*[draw_problem(rng, N, 64, 64, 24, 0.3 / 8, outliers, 4.0) for _ in range(H)])
+    Q, K, V = (np.stack([cast(x) for x in L])[None] for L in (Qs, Ks, Vs))
+    Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
+    O, ql, kl, sel = m.muse_retrieve_exact(Qd, Kd, Vd, S, C, C, 4, k1, k2, scale, return_all=True)
+    return host(Qd), host(Kd), host(Vd), host(O), ql.cpu().numpy(), kl.cpu().numpy(), sel.cpu().numpy()
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_retrieval_vs_oracle(dt):
+    N, S, C, k1, k2 = 1024, 128, 16, 2, 2
+    Q, K, V, O, ql, kl, sel = retrieval_case(dt, N, S, C, k1, k2, outliers=0.05)
+    for h in range(2):
+        # the selection equals the oracle's from the same clustering (near-ties aside)
+        qbar = mo.cluster_means(Q[0, h], ql[0, h], C)
+        lzb = mo.block_logZ(qbar, K[0, h], kl[0, h], C, S, 1.0)
+        want = mo.retrieval_select(lzb, k1, k2)
+        agree = (want == sel[0, h]).all(axis=-1).mean()
+        assert agree > 0.98, agree
+        ref = mo.muse_retrieval(Q[0, h], K[0, h], V[0, h], S, C, C, 4, k1, k2, 1.0,
+                                q_labels=ql[0, h], k_labels=kl[0, h], selection=sel[0, h])
+        err = mo.max_rel_err(O[0, h], ref)
+        assert err <= TOL[dt], err
+
+
+def test_retrieval_exact_limits_on_gpu():
+    N, S = 256, 64
+    # every query its own cluster: exact whatever is retrieved
+    Q, K, V, O, *_ = retrieval_case("f32", N, S, N, 1, 1, H=1)
+    E = mo.exact_attention(Q[0, 0], K[0, 0], V[0, 0], 1.0, causal=True)
+    assert mo.max_rel_err(O[0, 0], E) <= 1e-4
+    # every (cluster, block) pair retrieved: exact
+    Q, K, V, O, *_ = retrieval_case("f32", N, S, 4, 4, 4, H=1)
+    E = mo.exact_attention(Q[0, 0], K[0, 0], V[0, 0], 1.0, causal=True)
+    assert mo.max_rel_err(O[0, 0], E) <= 1e-4
+    # nothing retrieved, singleton keys: the remainder summaries are exact
+    rng = np.random.Generator(np.random.PCG64(3))
+    Qn, Kn, Vn = small_problem(23, N, 64, 64, 8, 0.3)
+    Qd, Kd, Vd = (dev(x[None, None], "f32") for x in (Qn, Kn, Vn))
+    O = host(m.muse_retrieve_exact(Qd, Kd, Vd, S, 8, N, 3, 0, 0, 1.0))[0, 0]
+    E = mo.exact_attention(host(Qd)[0, 0], host(Kd)[0, 0], host(Vd)[0, 0], 1.0, causal=True)
+    assert mo.max_rel_err(O, E) <= 1e-4
