@@ -55,6 +55,18 @@ def dist_info():
             int(os.environ.get("WORLD_SIZE", "1")))
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The maximum of `value` over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    dev = device if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -322,10 +334,7 @@ def main():
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    total = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(total, op=dist.ReduceOp.MAX)
-    mean_ms = float(total.item()) / args.steps
+    mean_ms = max_over_ranks(sum(step_ms), dev) / args.steps
     tokens = w.B * w.H * w.N
     value = world * tokens / (mean_ms / 1e3)
     assert m.muse_last_device_status() == 0
@@ -345,10 +354,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms.append(e0.elapsed_time(e1))
-    e2e_t = torch.tensor([sum(e2e_ms) / len(e2e_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = world * tokens / (float(e2e_t.item()) / 1e3)
+    e2e_value = world * tokens / (max_over_ranks(sum(e2e_ms) / len(e2e_ms), dev) / 1e3)
     h2d = sum(x.numel() * x.element_size() for x in (Qh, Kh, Vh))
     d2h = Oh.numel() * Oh.element_size()
 

@@ -62,34 +62,32 @@ __device__ __forceinline__ KmCtx km_ctx(const KmJobs &J, int tg) {
   return c;
 }
 
+// Initial centroids (the first C rows), their bf16 split and squared norms; one warp
+// per centroid row, rows C..CP-1 are padding (+inf norm: never the nearest).
 template <typename T, int D>
-__global__ void km_init(KmJobs J, int N) {
-  __shared__ float nrm[256];
-  const KmCtx k = km_ctx(J, blockIdx.x);
-  const T *x = static_cast<const T *>(k.job->X) + ((int64_t)k.tk.p * N + k.tk.row0) * D;
-  float *c = k.job->out.centroids + k.tk.cen * D;
-  for (int e = threadIdx.x; e < k.tk.C * D; e += blockDim.x) c[e] = ld_elem(x + e);
-  if (!J.chi) return;
-  // split copies, squared norms (+inf on the padding rows, which must never win)
-  for (int cc = 0; cc < J.CP; ++cc) {
-    float sq = 0.f;
-    for (int d = threadIdx.x; d < D; d += blockDim.x) {
-      const float v = cc < k.tk.C ? ld_elem(x + (int64_t)cc * D + d) : 0.f;
+__global__ void __launch_bounds__(256)
+km_init(KmJobs J, int N) {
+  const KmCtx k = km_ctx(J, blockIdx.y);
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (c >= J.CP) return;
+  const bool real = c < k.tk.C;
+  const T *x = static_cast<const T *>(k.job->X) + ((int64_t)k.tk.p * N + k.tk.row0 + c) * D;
+  float sq = 0.f;
+#pragma unroll
+  for (int u = 0; u < D / 32; ++u) {
+    const int d = lane + 32 * u;
+    const float v = real ? ld_elem(x + d) : 0.f;
+    if (real) k.job->out.centroids[(k.tk.cen + c) * D + d] = v;
+    if (J.chi) {
       const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-      J.chi[((int64_t)k.tg * J.CP + cc) * D + d] = hi;
-      J.clo[((int64_t)k.tg * J.CP + cc) * D + d] = lo;
-      sq = fmaf(v, v, sq);
+      J.chi[((int64_t)k.tg * J.CP + c) * D + d] = hi;
+      J.clo[((int64_t)k.tg * J.CP + c) * D + d] = __float2bfloat16_rn(v - __bfloat162float(hi));
     }
-    nrm[threadIdx.x] = sq;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float t = 0.f;
-      for (int u = 0; u < (int)blockDim.x; ++u) t += nrm[u];
-      J.cn[(int64_t)k.tg * J.CP + cc] = cc < k.tk.C ? t : CUDART_INF_F;
-    }
-    __syncthreads();
+    sq = fmaf(v, v, sq);
   }
+  sq = warp_sum(sq);
+  if (J.chi && lane == 0) J.cn[(int64_t)k.tg * J.CP + c] = real ? sq : CUDART_INF_F;
 }
 
 // Per-chunk label histogram (cluster-major counts[tg][c][chunk]) and the stable rank
@@ -501,7 +499,7 @@ static cudaError_t run_kmeans_t(KmJobs &J, int N, int P, int iters, char *ws, in
                                (int)smem);
     if (err != cudaSuccess) return err;
   }
-  km_init<T, D><<<tasks, 256, 0, st>>>(J, N);
+  km_init<T, D><<<dim3((J.CP + 7) / 8, tasks), 256, 0, st>>>(J, N);
   count_launches(1 + 4 * iters);
   for (int it = 0; it < iters; ++it) {
     if (kTc)

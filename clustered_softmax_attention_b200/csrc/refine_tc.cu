@@ -339,7 +339,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       }
       if (valid && !O && half == 0) {
         const int64_t rr = (int64_t)p * mt.in.out_stride + mt.in.out0[s] + row;
-        part_lse[rr] = lse[(int64_t)p * mt.q.row_stride + q.lab + n];
+        part_lse[rr] = lse[q.lab + n];
       }
     } else if (t == 0 && valid && half == 0) {
       // an instance with no keys cannot occur (every key range is non-empty)

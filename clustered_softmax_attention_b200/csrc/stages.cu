@@ -329,33 +329,41 @@ refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
           mk[e2] = mu_k[(zrow + j0) * D + e2];
         __syncthreads();
         if (!v) continue;
-        for (int jj = 0; jj < jt; ++jj) {
-          float u = 0.f;
-          const float4 *m4 = reinterpret_cast<const float4 *>(mk + jj * D);
+        for (int jq = 0; jq < jt; jq += 4) {
+          // four clusters at a time: independent accumulation chains
+          float u4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int d4 = 0; d4 < D / 4; ++d4) {
-            const float4 w4 = m4[d4];
-            u = fmaf(qt[4 * d4], w4.x, fmaf(qt[4 * d4 + 1], w4.y,
-                     fmaf(qt[4 * d4 + 2], w4.z, fmaf(qt[4 * d4 + 3], w4.w, u))));
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              const float4 w4 = reinterpret_cast<const float4 *>(mk + (jq + a) * D)[d4];
+              u4[a] = fmaf(qt[4 * d4], w4.x, fmaf(qt[4 * d4 + 1], w4.y,
+                           fmaf(qt[4 * d4 + 2], w4.z, fmaf(qt[4 * d4 + 3], w4.w, u4[a]))));
+            }
           }
-          const int j = j0 + jj;
-          const float a = lz[j] + scale * u;
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+          if (jq + a >= jt) break;
+          const float u = u4[a];
+          const int j = j0 + jq + a;
+          const float a_ = lz[j] + scale * u;
           if (pass == 0) {
-            if (a > m) {
-              l = l * __expf(m - a) + 1.f;
-              m = a;
-            } else if (a > -CUDART_INF_F) {
-              l += __expf(a - m);
+            if (a_ > m) {
+              l = l * __expf(m - a_) + 1.f;
+              m = a_;
+            } else if (a_ > -CUDART_INF_F) {
+              l += __expf(a_ - m);
             }
           } else {
-            const float pj = (a > -CUDART_INF_F) ? __expf(a - m) * inv : 0.f;
+            const float pj = (a_ > -CUDART_INF_F) ? __expf(a_ - m) * inv : 0.f;
             C0[(int64_t)j * w_ld(nq) + n] = pj * (1.f - scale * u);
             C1[(int64_t)j * w_ld(nq) + n] = scale * pj;
+          }
           }
         }
       }
     }
-    if (v) lse[(int64_t)p * mt.q.row_stride + q.lab + n] = m + logf(l);
+    if (v) lse[q.lab + n] = m + logf(l);
   }
 }
 
@@ -431,7 +439,7 @@ refine_simt(MuseTables mt, int N, const T *__restrict__ qt_rows, const int32_t *
     const int64_t r = (int64_t)p * mt.in.out_stride + mt.in.out0[s] + row;
 #pragma unroll
     for (int t = 0; t < PV; ++t) part_o[r * DV + g + 4 * t] = acc[t];
-    if (g == 0) part_lse[r] = lse[(int64_t)p * mt.q.row_stride + q.lab + n];
+    if (g == 0) part_lse[r] = lse[q.lab + n];
   }
 }
 

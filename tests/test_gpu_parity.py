@@ -267,3 +267,97 @@ def test_retrieval_exact_limits_on_gpu():
     O = host(m.muse_retrieve_exact(Qd, Kd, Vd, S, 8, N, 3, 0, 0, 1.0))[0, 0]
     E = mo.exact_attention(host(Qd)[0, 0], host(Kd)[0, 0], host(Vd)[0, 0], 1.0, causal=True)
     assert mo.max_rel_err(O, E) <= 1e-4
+
+
+# --------------------------------------------------------------------------- full-size workloads
+# Sampled rows, oracle fed the GPU's clustering (and selection), same launch as bench.py.
+
+def test_full_size_causal_n16k_sampled_rows():
+    w = WORKLOADS["causal_n16k_bf16"]
+    heads = [0, w.problems - 1]
+    Q, K, V = make_inputs(w)
+    Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
+    O, ql, kl = m.muse_causal_blocks(Qd, Kd, Vd, w.block, w.Cq, w.Ck, w.iters, w.scale,
+                                     return_labels=True)
+    O = host(O)
+    ql, kl = ql.cpu().numpy(), kl.cpu().numpy()
+    rng = np.random.default_rng(1)
+    for p in heads:
+        b, h = divmod(p, w.H)
+        rows = np.concatenate([rng.choice(w.N, 24, replace=False), [0, w.block, w.N - 1]])
+        labels = causal_labels(ql[b, h], kl[b, h], w.N, w.block)
+        ref = mo.muse_causal(Q[b, h], K[b, h], V[b, h], w.block, w.Cq, w.Ck, w.iters, w.scale,
+                             labels=labels, rows=rows)
+        err = np.abs(O[b, h][rows] - ref[rows]).max() / np.abs(ref[rows]).max()
+        assert err <= TOL["bf16"], err
+
+
+def test_full_size_retrieval_n32k_sampled_rows():
+    w = WORKLOADS["retrieval_n32k_bf16"]
+    Q, K, V = make_inputs(w)
+    Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
+    O, ql, kl, sel = m.muse_retrieve_exact(Qd, Kd, Vd, w.block, w.Cq, w.Ck, w.iters, w.k1, w.k2,
+                                           w.scale, return_all=True)
+    O, ql, kl, sel = host(O), ql.cpu().numpy(), kl.cpu().numpy(), sel.cpu().numpy()
+    rng = np.random.default_rng(2)
+    for (b, h) in ((0, 0), (w.B - 1, w.H - 1)):
+        rows = np.concatenate([rng.choice(np.arange(w.block, w.N), 6, replace=False), [3, w.N - 1]])
+        ref = mo.muse_retrieval(Q[b, h], K[b, h], V[b, h], w.block, w.Cq, w.Ck, w.iters, w.k1,
+                                w.k2, w.scale, q_labels=ql[b, h], k_labels=kl[b, h],
+                                selection=sel[b, h], rows=rows)
+        err = np.abs(O[b, h][rows] - ref[rows]).max() / np.abs(ref[rows]).max()
+        assert err <= TOL["bf16"], err
+
+
+def test_full_size_acausal_n64k_d128_sampled_rows():
+    w = WORKLOADS["acausal_n64k_d128_bf16"]
+    heads = [0, w.H - 1]
+    Q, K, V = make_inputs(w, heads=heads)
+    Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
+    O = host(m.muse_forward(Qd, Kd, Vd, w.Cq, w.Ck, w.iters, w.scale))
+    ql = m.muse_kmeans(Qd, w.Cq, w.iters)[0].cpu().numpy()
+    kl = m.muse_kmeans(Kd, w.Ck, w.iters)[0].cpu().numpy()
+    rng = np.random.default_rng(3)
+    for h in range(len(heads)):
+        rows = np.concatenate([rng.choice(w.N, 10, replace=False), [0, w.N - 1]])
+        ref = mo.muse_from_labels(Q[0, h], K[0, h], V[0, h], ql[0, h], kl[0, h], w.Cq, w.Ck,
+                                  w.scale, rows=rows)
+        err = np.abs(O[0, h][rows] - ref[rows]).max() / np.abs(ref[rows]).max()
+        assert err <= TOL["bf16"], err
+
+
+# --------------------------------------------------------------------------- memory safety
+
+def _with_tail(nbytes, fill=0xAB, tail=1 << 16):
+    buf = torch.full((nbytes + tail,), fill, dtype=torch.uint8, device="cuda")
+    return buf, buf[:nbytes], buf[nbytes:]
+
+
+@pytest.mark.parametrize("entry", ["forward", "causal", "retrieval"])
+def test_workspace_and_output_tails_untouched(entry):
+    """Every write stays inside the caller's workspace and output (multi-problem batch)."""
+    B, H, N = 2, 3, 2048
+    Q, K, V = mixture(12, B, H, N, 64, 64, 32, 0.3 / 8, "bf16")
+    Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
+    d = m.dims(Qd, Vd, 1.0)
+    if entry == "forward":
+        need = m.muse_workspace_size("muse_forward", d, 32, 32)
+    elif entry == "causal":
+        need = m.muse_workspace_size("muse_causal_blocks", d, 32, 32, 256)
+    else:
+        need = m.muse_workspace_size("muse_retrieve_exact", d, 32, 32, 256, 2, 2)
+    wbuf, ws, wtail = _with_tail(need)
+    obytes = B * H * N * 64 * 2
+    obuf, ob, otail = _with_tail(obytes)
+    O = ob.view(torch.bfloat16).view(B, H, N, 64)
+    if entry == "forward":
+        m.muse_forward(Qd, Kd, Vd, 32, 32, 3, 1.0, out=O, ws=ws)
+    elif entry == "causal":
+        m.muse_causal_blocks(Qd, Kd, Vd, 256, 32, 32, 3, 1.0, out=O, ws=ws)
+    else:
+        m.muse_retrieve_exact(Qd, Kd, Vd, 256, 32, 32, 3, 2, 2, 1.0, out=O, ws=ws)
+    torch.cuda.synchronize()
+    assert (wtail == 0xAB).all(), "write past the workspace"
+    assert (otail == 0xAB).all(), "write past the output"
+    assert torch.isfinite(O.float()).all()
+    assert m.muse_last_device_status() == 0
