@@ -382,59 +382,72 @@ km_scatter(KmJobs J, const int32_t *__restrict__ base, int *status) {
   k.job->out.perm[tk.lab + pos] = tk.row0 + r;  // sequence row index
 }
 
-// One CTA per (cluster, task).  Thread t owns one 16-byte vector of the row and one
-// member slot; slots take members b+slot, b+slot+SLOTS, ... in order; the slots are
-// then summed in slot order.  The result depends only on the data.
+// One warp per (cluster, task), 8 clusters per CTA.  Lane t owns one 16-byte vector
+// of the row and one member slot; slots take members b+slot, b+slot+SLOTS, ... in
+// order and are then summed in slot order (shuffles): the result depends only on
+// the data.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 km_centroid(KmJobs J, int N) {
   constexpr int VEC = 16 / sizeof(T);
-  constexpr int VPR = D / VEC;
-  constexpr int SLOTS = 256 / VPR;
-  __shared__ float red[SLOTS][D + 1];
+  constexpr int VPR = D / VEC;      // lanes per row (8, 16 or 32)
+  constexpr int SLOTS = 32 / VPR;   // member slots per warp
   const KmCtx k = km_ctx(J, blockIdx.y);
   const Task &tk = k.tk;
-  const int c = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (c >= tk.C) return;
   const int32_t *offsets = k.job->out.offsets;
   const int b = offsets[tk.off + c], e = offsets[tk.off + c + 1];
   if (e <= b) return;  // empty: keep the previous centroid
-  const int v = threadIdx.x % VPR, slot = threadIdx.x / VPR;
+  const int v = lane % VPR, slot = lane / VPR;
   const T *xp = static_cast<const T *>(k.job->X) + (int64_t)tk.p * N * D;
   const int32_t *perm = k.job->out.perm + tk.lab;
   float acc[VEC];
 #pragma unroll
   for (int u = 0; u < VEC; ++u) acc[u] = 0.f;
-  for (int m = b + slot; m < e; m += SLOTS) {
-    const uint4 raw = *reinterpret_cast<const uint4 *>(xp + (int64_t)perm[m] * D + v * VEC);
-    const T *el = reinterpret_cast<const T *>(&raw);
+  // this slot's members b+slot, b+slot+SLOTS, ... in order, four loads in flight
+  for (int m0 = b + slot; m0 < e; m0 += 4 * SLOTS) {
+    int rows[4];
 #pragma unroll
-    for (int u = 0; u < VEC; ++u) acc[u] += ld_elem(el + u);
-  }
+    for (int t = 0; t < 4; ++t) rows[t] = (m0 + t * SLOTS < e) ? perm[m0 + t * SLOTS] : -1;
+    uint4 raw[4];
 #pragma unroll
-  for (int u = 0; u < VEC; ++u) red[slot][v * VEC + u] = acc[u];
-  __syncthreads();
-  float val = 0.f;
-  if (threadIdx.x < D) {
-    float s = 0.f;
-    for (int sl = 0; sl < SLOTS; ++sl) s += red[sl][threadIdx.x];
-    val = s / (float)(e - b);
-    k.job->out.centroids[(tk.cen + c) * D + threadIdx.x] = val;
+    for (int t = 0; t < 4; ++t)
+      raw[t] = rows[t] >= 0 ? *reinterpret_cast<const uint4 *>(xp + (int64_t)rows[t] * D + v * VEC)
+                            : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      if (rows[t] < 0) break;
+      const T *el = reinterpret_cast<const T *>(&raw[t]);
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) acc[u] += ld_elem(el + u);
+    }
   }
-  if (!J.chi) return;
-  __syncthreads();
-  if (threadIdx.x < D) {
-    const __nv_bfloat16 hi = __float2bfloat16_rn(val);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(val - __bfloat162float(hi));
-    J.chi[((int64_t)k.tg * J.CP + c) * D + threadIdx.x] = hi;
-    J.clo[((int64_t)k.tg * J.CP + c) * D + threadIdx.x] = lo;
-    red[0][threadIdx.x] = val * val;
+  // fixed-order reduction over the slots (lane bits above the vector index)
+#pragma unroll
+  for (int o = VPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+  const float inv = 1.f / (float)(e - b);
+  float sq = 0.f;
+  if (slot == 0) {
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) {
+      const float val = acc[u] * inv;
+      const int d = v * VEC + u;
+      k.job->out.centroids[(tk.cen + c) * D + d] = val;
+      if (J.chi) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(val);
+        J.chi[((int64_t)k.tg * J.CP + c) * D + d] = hi;
+        J.clo[((int64_t)k.tg * J.CP + c) * D + d] = __float2bfloat16_rn(val - __bfloat162float(hi));
+      }
+      sq = fmaf(val, val, sq);
+    }
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float t = 0.f;
-    for (int d = 0; d < D; ++d) t += red[0][d];
-    J.cn[(int64_t)k.tg * J.CP + c] = t;
+  if (J.chi) {
+    sq = warp_sum(sq);  // lanes of slot > 0 contribute 0
+    if (lane == 0) J.cn[(int64_t)k.tg * J.CP + c] = sq;
   }
 }
 
@@ -509,7 +522,7 @@ static cudaError_t run_kmeans_t(KmJobs &J, int N, int P, int iters, char *ws, in
       km_assign<T, D><<<dim3(nch, tasks), kChunk, smem, st>>>(J, N, counts);
     km_scan<<<tasks, 1024, 0, st>>>(J, counts, base);
     km_scatter<<<dim3(nch, tasks), kChunk, 0, st>>>(J, base, status);
-    km_centroid<T, D><<<dim3(J.maxC, tasks), 256, 0, st>>>(J, N);
+    km_centroid<T, D><<<dim3((J.maxC + 7) / 8, tasks), 256, 0, st>>>(J, N);
   }
   return cudaGetLastError();
 }

@@ -16,8 +16,10 @@
 // tilt weights for up to 8 query clusters of the CTA and the tile's coefficients
 // c0, c1 for the CTA's 128 rows.
 //   S  = Qt . K_tile^T            (tcgen05, 128 x npad, fp32 in TMEM, double-buffered)
-//   P  = w .* (c0 + c1 .* S)      (epilogue warps: TMEM -> registers -> bf16 SMEM)
-//   O += P . V_tile               (tcgen05, 128 x Dv, fp32 in TMEM)
+//   P  = w .* (c0 + c1 .* S)      (epilogue warps: TMEM -> registers -> bf16 TMEM)
+//   O += P . V_tile               (tcgen05, A = P from TMEM, 128 x Dv, fp32 in TMEM)
+// TMEM columns: S double buffer [0, 2 BN), P double buffer [2 BN, 3 BN) (bf16 packed
+// two per column), O [3 BN, 3 BN + Dv).
 // Warp roles: warp 0 = producer (TMA + cp.async), warp 1 = MMA issuer (+ TMEM
 // owner), warps 2-9 = epilogue (TMEM lane quadrant = warp % 4; two warps per quadrant
 // split the 16-column chunks).  Every wait on an mbarrier is
@@ -31,10 +33,11 @@ namespace muse {
 namespace tcr {
 
 constexpr int BM = 128;      // query rows per CTA
-constexpr int NST = 3;       // K / V^T stages
+constexpr int NST = 4;       // K / V^T stages
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kSlots = 8;    // query clusters per CTA whose tilt weights are staged
+constexpr int kTileSegs = 8; // key clusters packed into one tile at most
 
 // Widest key tile: 128 keys when D = Dv = 64, else 64 (shared memory budget).
 template <int D, int DV>
@@ -49,9 +52,10 @@ struct __align__(1024) Smem {
   __nv_bfloat16 q[D / 64][BM * 64];            // residual tile, K-major SW128 blocks
   __nv_bfloat16 k[NST][D / 64][BN * 64];       // key tiles
   __nv_bfloat16 vt[NST][BN / 64][DV * 64];     // transposed value tiles
-  __nv_bfloat16 p[2][BN / 64][BM * 64];        // P tiles (A operand of the second MMA)
   float w[NST][kSlots][BN];                    // tilt weights of the CTA's query clusters
-  float c0[NST][BM], c1[NST][BM];              // coefficients of the tile's key cluster
+  float c0[NST][kTileSegs][BM];                // coefficients of the tile's key clusters
+  float c1[NST][kTileSegs][BM];
+  unsigned char seg[NST][BN];                  // column -> cluster of the tile (0xFF: masked)
   uint64_t full[NST], empty[NST], sfull[2], sfree[2], pready[2], pfree[2], qbar, obar;
   uint32_t tmem_base;
   int abort_flag;
@@ -60,40 +64,57 @@ struct __align__(1024) Smem {
 using namespace ptx;
 
 // Key tiles of an instance: cluster j's keys [b, e) in chunks of CHUNK.
+// A key tile: keys [c, c+n) of the sorted keys, widened to start at x0 = c & ~7 and
+// padded to npad columns (multiple of 16).  Either a chunk of one large cluster, or
+// whole clusters j .. j+nseg-1 packed while they fit in BN columns.
 struct KTile {
-  int j, c, n, x0, npad;
+  int j, nseg, c, n, x0, npad;
 };
-template <int CHUNK>
+template <int BN, int CHUNK>
 struct TileIter {
   const int32_t *off;
-  int C, j, c;
+  int C;
+  KTile t;
   __device__ void begin(const int32_t *o, int Ck) {
     off = o;
     C = Ck;
-    j = 0;
-    c = __ldg(off);
-    skip();
+    make(0, __ldg(off));
   }
-  // Past the end of cluster j: move to the first key of the next non-empty cluster.
-  __device__ void skip() {
+  // The tile starting at key c of cluster j (skipping clusters with no key left).
+  __device__ void make(int j, int c) {
     while (j < C && c >= __ldg(off + j + 1)) {
       ++j;
       if (j < C) c = __ldg(off + j);
     }
-  }
-  __device__ bool done() const { return j >= C; }
-  __device__ KTile get() const {
-    KTile t;
     t.j = j;
     t.c = c;
-    t.n = min(CHUNK, __ldg(off + j + 1) - c);
+    if (j >= C) return;
     t.x0 = c & ~7;
-    t.npad = ((c + t.n - t.x0) + 15) & ~15;
-    return t;
+    const int e = __ldg(off + j + 1);
+    int end;
+    if (e - c > CHUNK) {
+      end = c + CHUNK;
+      t.nseg = 1;
+    } else {
+      end = e;
+      t.nseg = 1;
+      while (j + t.nseg < C && t.nseg < kTileSegs) {
+        const int e2 = __ldg(off + j + t.nseg + 1);
+        if (e2 - t.x0 > BN) break;
+        end = e2;
+        ++t.nseg;
+      }
+    }
+    t.n = end - c;
+    t.npad = ((end - t.x0) + 15) & ~15;
   }
+  __device__ bool done() const { return t.j >= C; }
+  __device__ KTile get() const { return t; }
   __device__ void next() {
-    c += CHUNK;
-    skip();
+    if (t.nseg == 1 && t.c + t.n < __ldg(off + t.j + 1))
+      make(t.j, t.c + t.n);  // next chunk of the same cluster
+    else
+      make(t.j + t.nseg, t.j + t.nseg < C ? __ldg(off + t.j + t.nseg) : 0);
   }
 };
 
@@ -122,7 +143,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
-      mbar_init(&sm.full[i], 1 + 32);  // producer's expect_tx + one cp.async arrival per lane
+      mbar_init(&sm.full[i], 1 + 32);  // producer lane 0 arrive + one cp.async arrival per lane
       mbar_init(&sm.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -147,7 +168,9 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t tmem_o = tmem + 256;
+  const uint32_t tmem_o = tmem + 3 * BN;
+  auto s_col = [](int buf) { return (uint32_t)(buf * BN); };
+  auto p_col = [](int buf) { return (uint32_t)(2 * BN + buf * (BN / 2)); };
   const int32_t *koff = k_offsets + k.off;
   const int kcol0 = (int)(k.lab - (int64_t)p * mt.k.row_stride);  // instance's first key column
   const int wl = w_ld(k.n), cl = w_ld(q.n);
@@ -158,7 +181,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    TileIter<CHUNK> it;
+    TileIter<BN, CHUNK> it;
     it.begin(koff, k.C);
     int t = 0;
     if (lane == 0) {
@@ -168,12 +191,12 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     for (; !it.done(); it.next(), ++t) {
       const KTile kt = it.get();
       const int st = t % NST;
-      bool ok = true;
-      if (t >= NST) ok = mbar_wait(&sm.empty[st], ((t / NST) - 1) & 1, abort_flag, status);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      int ok = 1;
+      if (t >= NST && lane == 0) ok = mbar_wait(&sm.empty[st], ((t / NST) - 1) & 1, abort_flag, status);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       if (lane == 0) {
         const int nbox = kt.npad > 64 ? 2 : 1;
-        mbar_expect_tx(&sm.full[st], (uint32_t)nbox * ((D / 64) * 64 * 128 + DV * 128));
+        mbar_expect_tx_only(&sm.full[st], (uint32_t)nbox * ((D / 64) * 64 * 128 + DV * 128));
         for (int rb = 0; rb < nbox; ++rb) {
           for (int kb = 0; kb < D / 64; ++kb)
             tma_load_2d(sm.k[st][kb] + rb * 64 * 64, &map_k, kb * 64, (int)(k.lab + kt.x0 + rb * 64),
@@ -189,16 +212,27 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         cp_async16(&sm.w[st][sl][4 * v], in ? (const void *)(Wi + (int64_t)i * wl + col) : (const void *)W,
                    in ? 16u : 0u);
       }
-      // coefficients of the tile's key cluster for the CTA's rows
-      {
+      // coefficients of the tile's key clusters for the CTA's rows
+      for (int sg = 0; sg < kt.nseg; ++sg) {
         const int row = r0 + 4 * lane;
         const bool in = row < cl;
-        cp_async16(&sm.c0[st][4 * lane], in ? (const void *)(C0 + (int64_t)kt.j * cl + row) : (const void *)W,
-                   in ? 16u : 0u);
-        cp_async16(&sm.c1[st][4 * lane], in ? (const void *)(C1 + (int64_t)kt.j * cl + row) : (const void *)W,
-                   in ? 16u : 0u);
+        const int64_t at = (int64_t)(kt.j + sg) * cl + row;
+        cp_async16(&sm.c0[st][sg][4 * lane], in ? (const void *)(C0 + at) : (const void *)W, in ? 16u : 0u);
+        cp_async16(&sm.c1[st][sg][4 * lane], in ? (const void *)(C1 + at) : (const void *)W, in ? 16u : 0u);
       }
       cp_async_arrive(&sm.full[st]);
+      // column -> segment (0xFF outside [c, c+n))
+      for (int col = lane; col < BN; col += 32) {
+        const int key = kt.x0 + col;
+        int sg = 0xFF;
+        if (col < kt.npad && key >= kt.c && key < kt.c + kt.n) {
+          sg = 0;
+          while (sg + 1 < kt.nseg && key >= __ldg(koff + kt.j + sg + 1)) ++sg;
+        }
+        sm.seg[st][col] = (unsigned char)sg;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.full[st]);  // releases the segment map with the stage
     }
     // copies still in flight land before the CTA may exit
     if (lane == 0)
@@ -208,7 +242,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     if (lane == 0) {
       bool ok = mbar_wait(&sm.qbar, 0, abort_flag, status);
       tc_fence_after();
-      TileIter<CHUNK> it;
+      TileIter<BN, CHUNK> it;
       it.begin(koff, k.C);
       int t = 0, prev_npad = 0;
       auto gemm2 = [&](int u, int npad) -> bool {
@@ -217,9 +251,8 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         tc_fence_after();
         const uint32_t id = idesc(BM, DV);
         for (int kk = 0; kk < npad / 16; ++kk) {
-          const uint64_t a = sdesc(sm.p[buf][kk >> 2] + (kk & 3) * 16);
           const uint64_t b = sdesc(sm.vt[st][kk >> 2] + (kk & 3) * 16);
-          tc_mma(tmem_o, a, b, id, (u > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem_o, tmem + p_col(buf) + kk * 8, b, id, (u > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&sm.pfree[buf]);
         tc_commit(&sm.empty[st]);
@@ -235,7 +268,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t a = sdesc(sm.q[kk >> 2] + (kk & 3) * 16);
           const uint64_t b = sdesc(sm.k[st][kk >> 2] + (kk & 3) * 16);
-          tc_mma(tmem + buf * 128, a, b, id, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + s_col(buf), a, b, id, kk > 0 ? 1u : 0u);
         }
         tc_commit(&sm.sfull[buf]);
         if (t >= 1 && !gemm2(t - 1, prev_npad)) { ok = false; break; }
@@ -257,7 +290,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const bool staged = slot < kSlots;
     const float *wrow = Wi + (int64_t)i * wl;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    TileIter<CHUNK> it;
+    TileIter<BN, CHUNK> it;
     it.begin(koff, k.C);
     int t = 0;
     bool ok = true;
@@ -268,12 +301,12 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       if (!mbar_wait(&sm.full[st], (t / NST) & 1, abort_flag, status)) { ok = false; break; }
       tc_fence_after();
       if (t >= 2 && !mbar_wait(&sm.pfree[buf], ((t - 2) >> 1) & 1, abort_flag, status)) { ok = false; break; }
-      const float a0 = sm.c0[st][r], a1 = sm.c1[st][r];
+      const float a0 = sm.c0[st][0][r], a1 = sm.c1[st][0][r];
       const int lo = kt.c - kt.x0, hi = kt.c + kt.n - kt.x0;  // unmasked columns [lo, hi)
       const float *ws = staged ? &sm.w[st][slot][0] : wrow + kt.x0;
       for (int cb = half; cb < kt.npad / 16; cb += 2) {
         float x[16];
-        tmem_ld16(tmem + lane_base + buf * 128 + cb * 16, x);
+        tmem_ld16(tmem + lane_base + s_col(buf) + cb * 16, x);
         const int col0 = cb * 16;
         float w[16];
 #pragma unroll
@@ -283,15 +316,28 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
         }
         float pv[16];
+        if (kt.nseg == 1) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) pv[e] = w[e] * fmaf(a1, x[e], a0);
-        if (!valid) {
+          for (int e = 0; e < 16; ++e) pv[e] = w[e] * fmaf(a1, x[e], a0);
+          if (!valid) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pv[e] = 0.f;
-        } else if (col0 < lo || col0 + 16 > hi) {
+            for (int e = 0; e < 16; ++e) pv[e] = 0.f;
+          } else if (col0 < lo || col0 + 16 > hi) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (col0 + e < lo || col0 + e >= hi) pv[e] = 0.f;
+            for (int e = 0; e < 16; ++e)
+              if (col0 + e < lo || col0 + e >= hi) pv[e] = 0.f;
+          }
+        } else {
+          // several clusters in the tile: coefficients per column from the segment map
+          const uint4 sgv = *reinterpret_cast<const uint4 *>(&sm.seg[st][col0]);
+          const unsigned char *sg = reinterpret_cast<const unsigned char *>(&sgv);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int g = sg[e];
+            float pe = 0.f;
+            if (valid && g != 0xFF) pe = w[e] * fmaf(sm.c1[st][g][r], x[e], sm.c0[st][g][r]);
+            pv[e] = pe;
+          }
         }
         uint32_t pk[8];
 #pragma unroll
@@ -299,13 +345,10 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           __nv_bfloat162 h = __floats2bfloat162_rn(pv[e], pv[e + 1]);
           pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
         }
-        // two 16-byte chunks of row r in the 128-byte-swizzled K-major block cb/4
-        unsigned char *blk = reinterpret_cast<unsigned char *>(sm.p[buf][cb >> 2]) + r * 128;
-        const int ch = (cb & 3) * 2;
-        *reinterpret_cast<uint4 *>(blk + (((ch) ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4 *>(blk + (((ch + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        // 16 bf16 of row r = 8 packed TMEM columns of the P buffer
+        tmem_st8(tmem + lane_base + p_col(buf) + cb * 8, pk);
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {

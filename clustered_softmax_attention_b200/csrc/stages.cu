@@ -295,75 +295,60 @@ tilt_cov(MuseTables mt, const int32_t *__restrict__ k_offsets, const float *__re
 template <typename T, int D>
 __global__ void __launch_bounds__(128)
 refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
-              const int32_t *__restrict__ q_offsets, const float *__restrict__ logZ,
+              const int32_t *__restrict__ q_cluster, const float *__restrict__ logZ,
               const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
-              float *__restrict__ lse) {
-  extern __shared__ float sm[];
+              float *__restrict__ lse, int keep_u) {
+  extern __shared__ float su[];  // [Ck][128] residual projections u_j (when keep_u)
   const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
   const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
-  const int Cq = q.C, Ck = k.C, nq = q.n;
-  const int i = blockIdx.x;
-  if (i >= Cq) return;
-  const int b = q_offsets[q.off + i], e = q_offsets[q.off + i + 1];
-  if (e <= b) return;
-  float *lz = sm;                 // [Ck]
-  float *mk = sm + kMaxClusters;  // [32][D]
+  const int Ck = k.C, nq = q.n;
+  const int n = blockIdx.x * 128 + threadIdx.x;
+  if (blockIdx.x * 128 >= nq) return;  // uniform
+  const bool v = n < nq;
+  const int i = v ? q_cluster[q.lab + n] : 0;
+  float qt[D];
+#pragma unroll
+  for (int d = 0; d < D; ++d) qt[d] = v ? ld_elem(qt_rows + (q.lab + n) * D + d) : 0.f;
   const int64_t zrow = (int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck;
-  for (int j = threadIdx.x; j < Ck; j += blockDim.x) lz[j] = logZ[zrow + j];
+  const float *lz = logZ + zrow;
+  const float4 *mk = reinterpret_cast<const float4 *>(mu_k + zrow * D);
   float *C0 = c0 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
   float *C1 = c1 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
-  for (int n0 = b; n0 < e; n0 += blockDim.x) {
-    const int n = n0 + threadIdx.x;
-    const bool v = n < e;
-    float qt[D];
+  const int cl = w_ld(nq);
+  auto proj = [&](int j) {
+    float u0 = 0.f, u1 = 0.f;
 #pragma unroll
-    for (int d = 0; d < D; ++d) qt[d] = v ? ld_elem(qt_rows + (q.lab + n) * D + d) : 0.f;
-    // pass 0: running max and sum of exp(a_j - max); pass 1: the coefficients
-    float m = -CUDART_INF_F, l = 0.f;
-    for (int pass = 0; pass < 2; ++pass) {
-      const float inv = pass ? 1.f / l : 0.f;
-      for (int j0 = 0; j0 < Ck; j0 += 32) {
-        const int jt = min(32, Ck - j0);
-        __syncthreads();
-        for (int e2 = threadIdx.x; e2 < jt * D; e2 += blockDim.x)
-          mk[e2] = mu_k[(zrow + j0) * D + e2];
-        __syncthreads();
-        if (!v) continue;
-        for (int jq = 0; jq < jt; jq += 4) {
-          // four clusters at a time: independent accumulation chains
-          float u4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int d4 = 0; d4 < D / 4; ++d4) {
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-              const float4 w4 = reinterpret_cast<const float4 *>(mk + (jq + a) * D)[d4];
-              u4[a] = fmaf(qt[4 * d4], w4.x, fmaf(qt[4 * d4 + 1], w4.y,
-                           fmaf(qt[4 * d4 + 2], w4.z, fmaf(qt[4 * d4 + 3], w4.w, u4[a]))));
-            }
-          }
-#pragma unroll
-          for (int a = 0; a < 4; ++a) {
-          if (jq + a >= jt) break;
-          const float u = u4[a];
-          const int j = j0 + jq + a;
-          const float a_ = lz[j] + scale * u;
-          if (pass == 0) {
-            if (a_ > m) {
-              l = l * __expf(m - a_) + 1.f;
-              m = a_;
-            } else if (a_ > -CUDART_INF_F) {
-              l += __expf(a_ - m);
-            }
-          } else {
-            const float pj = (a_ > -CUDART_INF_F) ? __expf(a_ - m) * inv : 0.f;
-            C0[(int64_t)j * w_ld(nq) + n] = pj * (1.f - scale * u);
-            C1[(int64_t)j * w_ld(nq) + n] = scale * pj;
-          }
-          }
-        }
+    for (int d4 = 0; d4 < D / 4; d4 += 2) {
+      const float4 a = __ldg(mk + (int64_t)j * (D / 4) + d4);
+      const float4 b = __ldg(mk + (int64_t)j * (D / 4) + d4 + 1);
+      u0 = fmaf(qt[4 * d4], a.x, fmaf(qt[4 * d4 + 1], a.y, fmaf(qt[4 * d4 + 2], a.z, fmaf(qt[4 * d4 + 3], a.w, u0))));
+      u1 = fmaf(qt[4 * d4 + 4], b.x, fmaf(qt[4 * d4 + 5], b.y, fmaf(qt[4 * d4 + 6], b.z, fmaf(qt[4 * d4 + 7], b.w, u1))));
+    }
+    return u0 + u1;
+  };
+  // pass 0: running max and sum of exp(a_j - max); pass 1: the coefficients
+  float m = -CUDART_INF_F, l = 0.f;
+  if (v) {
+    for (int j = 0; j < Ck; ++j) {
+      const float u = proj(j);
+      if (keep_u) su[j * 128 + threadIdx.x] = u;
+      const float a = lz[j] + scale * u;
+      if (a > m) {
+        l = l * __expf(m - a) + 1.f;
+        m = a;
+      } else if (a > -CUDART_INF_F) {
+        l += __expf(a - m);
       }
     }
-    if (v) lse[q.lab + n] = m + logf(l);
+    const float inv = 1.f / l;
+    for (int j = 0; j < Ck; ++j) {
+      const float u = keep_u ? su[j * 128 + threadIdx.x] : proj(j);
+      const float a = lz[j] + scale * u;
+      const float pj = (a > -CUDART_INF_F) ? __expf(a - m) * inv : 0.f;
+      C0[(int64_t)j * cl + n] = pj * (1.f - scale * u);
+      C1[(int64_t)j * cl + n] = scale * pj;
+    }
+    lse[q.lab + n] = m + logf(l);
   }
 }
 
@@ -620,12 +605,14 @@ cudaError_t run_tilt_weights(const MuseTables &mt, int dtype, int D, int P, floa
 template <typename T, int D>
 static cudaError_t coeffs_t(const MuseTables &mt, int P, float scale, SortedSide qs,
                             const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
-  const size_t smem = (kMaxClusters + 32 * D) * sizeof(float);
+  (void)q_offsets;
+  const int keep_u = mt.k.max_C <= 256 ? 1 : 0;
+  const size_t smem = keep_u ? (size_t)mt.k.max_C * 128 * sizeof(float) : 0;
   cudaError_t err = cudaFuncSetAttribute(refine_coeffs<T, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  refine_coeffs<T, D><<<dim3(mt.q.max_C, P * mt.in.ninst), 128, smem, st>>>(
-      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse);
+  refine_coeffs<T, D><<<dim3((mt.q.max_rows + 127) / 128, P * mt.in.ninst), 128, smem, st>>>(
+      mt, scale, (const T *)qs.rows, qs.cluster, b.logZ, b.mu_k, b.c0, b.c1, b.lse, keep_u);
   count_launches(1);
   return cudaGetLastError();
 }
