@@ -75,6 +75,39 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+KERNEL_SOURCES = ["clustered_softmax_attention_b200/csrc/refine_tc.cu",
+                  "clustered_softmax_attention_b200/csrc/tc_ptx.cuh"]
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the refinement kernel from the committed ncu summary of
+    this workload, if it was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"refine_tc_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def algorithmic_flops(w):
     """Flops of the refinement contraction per launch (all problems).
 
@@ -368,7 +401,7 @@ def main():
     else:
         peak, bound, unit = FP32_SIMT_TFLOPS, "alu", "TFLOP/s"
     roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": None, "kernel": "refinement",
+            "frac": achieved / peak, "traffic": recorded_traffic(w.name), "kernel": "refinement",
             "kernel_ms": kmean, "flops_per_launch": flops,
             "peak_source": f"{peak_src} bf16_tflops (burst)" if w.dtype == "bf16"
             else "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}

@@ -406,18 +406,18 @@ km_centroid(KmJobs J, int N) {
   float acc[VEC];
 #pragma unroll
   for (int u = 0; u < VEC; ++u) acc[u] = 0.f;
-  // this slot's members b+slot, b+slot+SLOTS, ... in order, four loads in flight
-  for (int m0 = b + slot; m0 < e; m0 += 4 * SLOTS) {
-    int rows[4];
+  // this slot's members b+slot, b+slot+SLOTS, ... in order, eight loads in flight
+  for (int m0 = b + slot; m0 < e; m0 += 8 * SLOTS) {
+    int rows[8];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) rows[t] = (m0 + t * SLOTS < e) ? perm[m0 + t * SLOTS] : -1;
-    uint4 raw[4];
+    for (int t = 0; t < 8; ++t) rows[t] = (m0 + t * SLOTS < e) ? perm[m0 + t * SLOTS] : -1;
+    uint4 raw[8];
 #pragma unroll
-    for (int t = 0; t < 4; ++t)
+    for (int t = 0; t < 8; ++t)
       raw[t] = rows[t] >= 0 ? *reinterpret_cast<const uint4 *>(xp + (int64_t)rows[t] * D + v * VEC)
                             : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
+    for (int t = 0; t < 8; ++t) {
       if (rows[t] < 0) break;
       const T *el = reinterpret_cast<const T *>(&raw[t]);
 #pragma unroll

@@ -20,9 +20,11 @@
 //   O += P . V_tile               (tcgen05, A = P from TMEM, 128 x Dv, fp32 in TMEM)
 // TMEM columns: S double buffer [0, 2 BN), P double buffer [2 BN, 3 BN) (bf16 packed
 // two per column), O [3 BN, 3 BN + Dv).
-// Warp roles: warp 0 = producer (TMA + cp.async), warp 1 = MMA issuer (+ TMEM
-// owner), warps 2-9 = epilogue (TMEM lane quadrant = warp % 4; two warps per quadrant
-// split the 16-column chunks).  Every wait on an mbarrier is
+// Warp roles: warp 0 = TMA producer (key and value tiles, each released as soon as
+// its MMA has consumed it), warp 1 = MMA issuer (+ TMEM owner), warps 2-9 = epilogue
+// in two groups of four (TMEM lane quadrant = warp % 4): group g takes the tiles of
+// parity g, i.e. S/P buffer g, so the groups overlap; warp 10 = cp.async producer of
+// the epilogue data.  Every wait on an mbarrier is
 // bounded: past the limit the kernel records MUSE_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 
@@ -35,7 +37,8 @@ namespace tcr {
 constexpr int BM = 128;      // query rows per CTA
 constexpr int NST = 4;       // K / V^T stages
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kThreads = 64 + 32 * kEpiWarps + 32;  // + the epilogue-data producer warp
+constexpr int kEWarp = 2 + kEpiWarps;               // that warp's index
 constexpr int kSlots = 8;    // query clusters per CTA whose tilt weights are staged
 constexpr int kTileSegs = 8; // key clusters packed into one tile at most
 
@@ -56,7 +59,11 @@ struct __align__(1024) Smem {
   float c0[NST][kTileSegs][BM];                // coefficients of the tile's key clusters
   float c1[NST][kTileSegs][BM];
   unsigned char seg[NST][BN];                  // column -> cluster of the tile (0xFF: masked)
-  uint64_t full[NST], empty[NST], sfull[2], sfree[2], pready[2], pfree[2], qbar, obar;
+  int koff[kMaxClusters + 1];                  // the instance's key-cluster offsets
+  // per stage: key tile (consumed by the first MMA), values (second MMA), epilogue
+  // data (tilt weights, coefficients, segment map; consumed by the epilogue)
+  uint64_t fullk[NST], emptyk[NST], fullv[NST], emptyv[NST], fulle[NST], emptye[NST];
+  uint64_t sfull[2], sfree[2], pready[2], pfree[2], qbar, obar;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -78,19 +85,19 @@ struct TileIter {
   __device__ void begin(const int32_t *o, int Ck) {
     off = o;
     C = Ck;
-    make(0, __ldg(off));
+    make(0, off[0]);
   }
   // The tile starting at key c of cluster j (skipping clusters with no key left).
   __device__ void make(int j, int c) {
-    while (j < C && c >= __ldg(off + j + 1)) {
+    while (j < C && c >= off[j + 1]) {
       ++j;
-      if (j < C) c = __ldg(off + j);
+      if (j < C) c = off[j];
     }
     t.j = j;
     t.c = c;
     if (j >= C) return;
     t.x0 = c & ~7;
-    const int e = __ldg(off + j + 1);
+    const int e = off[j + 1];
     int end;
     if (e - c > CHUNK) {
       end = c + CHUNK;
@@ -99,7 +106,7 @@ struct TileIter {
       end = e;
       t.nseg = 1;
       while (j + t.nseg < C && t.nseg < kTileSegs) {
-        const int e2 = __ldg(off + j + t.nseg + 1);
+        const int e2 = off[j + t.nseg + 1];
         if (e2 - t.x0 > BN) break;
         end = e2;
         ++t.nseg;
@@ -111,10 +118,10 @@ struct TileIter {
   __device__ bool done() const { return t.j >= C; }
   __device__ KTile get() const { return t; }
   __device__ void next() {
-    if (t.nseg == 1 && t.c + t.n < __ldg(off + t.j + 1))
+    if (t.nseg == 1 && t.c + t.n < off[t.j + 1])
       make(t.j, t.c + t.n);  // next chunk of the same cluster
     else
-      make(t.j + t.nseg, t.j + t.nseg < C ? __ldg(off + t.j + t.nseg) : 0);
+      make(t.j + t.nseg, t.j + t.nseg < C ? off[t.j + t.nseg] : 0);
   }
 };
 
@@ -143,13 +150,17 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
-      mbar_init(&sm.full[i], 1 + 32);  // producer lane 0 arrive + one cp.async arrival per lane
-      mbar_init(&sm.empty[i], 1);
+      mbar_init(&sm.fullk[i], 1);
+      mbar_init(&sm.emptyk[i], 1);
+      mbar_init(&sm.fullv[i], 1);
+      mbar_init(&sm.emptyv[i], 1);
+      mbar_init(&sm.fulle[i], 1 + 32);  // lane 0 arrive + one cp.async arrival per lane
+      mbar_init(&sm.emptye[i], kEpiWarps / 2);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.sfull[i], 1);
-      mbar_init(&sm.sfree[i], kEpiWarps);
-      mbar_init(&sm.pready[i], kEpiWarps);
+      mbar_init(&sm.sfree[i], kEpiWarps / 2);   // one warp group per buffer
+      mbar_init(&sm.pready[i], kEpiWarps / 2);
       mbar_init(&sm.pfree[i], 1);
     }
     mbar_init(&sm.qbar, 1);
@@ -164,6 +175,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  for (int j = threadIdx.x; j <= k.C; j += blockDim.x) sm.koff[j] = k_offsets[k.off + j];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -171,41 +183,61 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   const uint32_t tmem_o = tmem + 3 * BN;
   auto s_col = [](int buf) { return (uint32_t)(buf * BN); };
   auto p_col = [](int buf) { return (uint32_t)(2 * BN + buf * (BN / 2)); };
-  const int32_t *koff = k_offsets + k.off;
+  const int32_t *koff = sm.koff;
   const int kcol0 = (int)(k.lab - (int64_t)p * mt.k.row_stride);  // instance's first key column
   const int wl = w_ld(k.n), cl = w_ld(q.n);
   const float *Wi = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s];      // row i: Wi + i*wl
   const float *C0 = c0g + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];   // row j: C0 + j*cl
   const float *C1 = c1g + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
   const int i_first = q_cluster[q.lab + r0];  // query clusters i_first.. get staged weights
+  const int nslots = min(kSlots, q_cluster[q.lab + min(r0 + BM, q.n) - 1] - i_first + 1);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    TileIter<BN, CHUNK> it;
-    it.begin(koff, k.C);
-    int t = 0;
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       mbar_expect_tx(&sm.qbar, (uint32_t)(D / 64) * BM * 128);
       for (int kb = 0; kb < D / 64; ++kb) tma_load_2d(sm.q[kb], &map_q, kb * 64, (int)(q.lab + r0), &sm.qbar);
+      // K(t) then V(t); a stage is refilled once the MMA that read it has completed
+      TileIter<BN, CHUNK> it;
+      it.begin(koff, k.C);
+      int t = 0;
+      for (; !it.done(); it.next(), ++t) {
+        const KTile kt = it.get();
+        const int st = t % NST;
+        const int nbox = kt.npad > 64 ? 2 : 1;
+        if (t >= NST && !mbar_wait(&sm.emptyk[st], ((t / NST) - 1) & 1, abort_flag, status)) break;
+        mbar_expect_tx(&sm.fullk[st], (uint32_t)nbox * (D / 64) * 64 * 128);
+        for (int rb = 0; rb < nbox; ++rb)
+          for (int kb = 0; kb < D / 64; ++kb)
+            tma_load_2d(sm.k[st][kb] + rb * 64 * 64, &map_k, kb * 64, (int)(k.lab + kt.x0 + rb * 64),
+                        &sm.fullk[st]);
+        if (t >= NST && !mbar_wait(&sm.emptyv[st], ((t / NST) - 1) & 1, abort_flag, status)) {
+          mbar_drain(&sm.fullk[st], (t / NST) & 1, status);  // K(t) is in flight
+          break;
+        }
+        mbar_expect_tx(&sm.fullv[st], (uint32_t)nbox * DV * 128);
+        for (int rb = 0; rb < nbox; ++rb)
+          tma_load_2d(sm.vt[st][rb], &map_vt, kcol0 + kt.x0 + rb * 64, p * DV, &sm.fullv[st]);
+      }
+      // copies still in flight land before the CTA may exit
+      for (int u = max(0, t - NST); u < t; ++u) {
+        mbar_drain(&sm.fullk[u % NST], (u / NST) & 1, status);
+        mbar_drain(&sm.fullv[u % NST], (u / NST) & 1, status);
+      }
     }
+  } else if (warp == kEWarp) {
+    // ------------------------------------------------------------ epilogue-data producer
+    TileIter<BN, CHUNK> it;
+    it.begin(koff, k.C);
+    int t = 0;
     for (; !it.done(); it.next(), ++t) {
       const KTile kt = it.get();
       const int st = t % NST;
       int ok = 1;
-      if (t >= NST && lane == 0) ok = mbar_wait(&sm.empty[st], ((t / NST) - 1) & 1, abort_flag, status);
+      if (t >= NST && lane == 0) ok = mbar_wait(&sm.emptye[st], ((t / NST) - 1) & 1, abort_flag, status);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      if (lane == 0) {
-        const int nbox = kt.npad > 64 ? 2 : 1;
-        mbar_expect_tx_only(&sm.full[st], (uint32_t)nbox * ((D / 64) * 64 * 128 + DV * 128));
-        for (int rb = 0; rb < nbox; ++rb) {
-          for (int kb = 0; kb < D / 64; ++kb)
-            tma_load_2d(sm.k[st][kb] + rb * 64 * 64, &map_k, kb * 64, (int)(k.lab + kt.x0 + rb * 64),
-                        &sm.full[st]);
-          tma_load_2d(sm.vt[st][rb], &map_vt, kcol0 + kt.x0 + rb * 64, p * DV, &sm.full[st]);
-        }
-      }
       // tilt weights of the staged query clusters over the tile's columns
-      for (int e = lane; e < kSlots * (BN / 4); e += 32) {
+      for (int e = lane; e < nslots * (BN / 4); e += 32) {
         const int sl = e / (BN / 4), v = e % (BN / 4);
         const int col = kt.x0 + 4 * v, i = i_first + sl;
         const bool in = i < q.C && col < wl && 4 * v < kt.npad;
@@ -220,50 +252,39 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         cp_async16(&sm.c0[st][sg][4 * lane], in ? (const void *)(C0 + at) : (const void *)W, in ? 16u : 0u);
         cp_async16(&sm.c1[st][sg][4 * lane], in ? (const void *)(C1 + at) : (const void *)W, in ? 16u : 0u);
       }
-      cp_async_arrive(&sm.full[st]);
+      cp_async_arrive(&sm.fulle[st]);
       // column -> segment (0xFF outside [c, c+n))
       for (int col = lane; col < BN; col += 32) {
         const int key = kt.x0 + col;
         int sg = 0xFF;
         if (col < kt.npad && key >= kt.c && key < kt.c + kt.n) {
           sg = 0;
-          while (sg + 1 < kt.nseg && key >= __ldg(koff + kt.j + sg + 1)) ++sg;
+          while (sg + 1 < kt.nseg && key >= koff[kt.j + sg + 1]) ++sg;
         }
         sm.seg[st][col] = (unsigned char)sg;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.full[st]);  // releases the segment map with the stage
+      if (lane == 0) mbar_arrive(&sm.fulle[st]);  // releases the segment map with the stage
     }
-    // copies still in flight land before the CTA may exit
     if (lane == 0)
-      for (int u = max(0, t - NST); u < t; ++u) mbar_drain(&sm.full[u % NST], (u / NST) & 1, status);
+      for (int u = max(0, t - NST); u < t; ++u) mbar_drain(&sm.fulle[u % NST], (u / NST) & 1, status);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Fixed order S(0), S(1), then for every tile t: S(t+2) (its S buffer is released
+    // by the group reading S(t) before that group publishes P(t)), then O += P(t) V(t).
     if (lane == 0) {
       bool ok = mbar_wait(&sm.qbar, 0, abort_flag, status);
       tc_fence_after();
       TileIter<BN, CHUNK> it;
       it.begin(koff, k.C);
-      int t = 0, prev_npad = 0;
-      auto gemm2 = [&](int u, int npad) -> bool {
-        const int st = u % NST, buf = u & 1;
-        if (!mbar_wait(&sm.pready[buf], (u >> 1) & 1, abort_flag, status)) return false;
+      int g1 = 0;  // next tile of the first contraction
+      int npad_ring[4];
+      auto gemm1 = [&]() {
+        const int st = g1 % NST, buf = g1 & 1;
+        if (g1 >= 2 && !mbar_wait(&sm.sfree[buf], ((g1 - 2) >> 1) & 1, abort_flag, status)) return false;
+        if (!mbar_wait(&sm.fullk[st], (g1 / NST) & 1, abort_flag, status)) return false;
         tc_fence_after();
-        const uint32_t id = idesc(BM, DV);
-        for (int kk = 0; kk < npad / 16; ++kk) {
-          const uint64_t b = sdesc(sm.vt[st][kk >> 2] + (kk & 3) * 16);
-          tc_mma_ts(tmem_o, tmem + p_col(buf) + kk * 8, b, id, (u > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&sm.pfree[buf]);
-        tc_commit(&sm.empty[st]);
-        return true;
-      };
-      for (; ok && !it.done(); it.next(), ++t) {
         const KTile kt = it.get();
-        const int st = t % NST, buf = t & 1;
-        if (!mbar_wait(&sm.full[st], (t / NST) & 1, abort_flag, status)) { ok = false; break; }
-        if (t >= 2 && !mbar_wait(&sm.sfree[buf], ((t - 2) >> 1) & 1, abort_flag, status)) { ok = false; break; }
-        tc_fence_after();
         const uint32_t id = idesc(BM, kt.npad);
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t a = sdesc(sm.q[kk >> 2] + (kk & 3) * 16);
@@ -271,23 +292,44 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           tc_mma(tmem + s_col(buf), a, b, id, kk > 0 ? 1u : 0u);
         }
         tc_commit(&sm.sfull[buf]);
-        if (t >= 1 && !gemm2(t - 1, prev_npad)) { ok = false; break; }
-        prev_npad = kt.npad;
+        tc_commit(&sm.emptyk[st]);  // the key tile is consumed
+        npad_ring[g1 & 3] = kt.npad;
+        ++g1;
+        it.next();
+        return true;
+      };
+      for (int w = 0; ok && w < 2 && !it.done(); ++w) ok = gemm1();
+      for (int g2 = 0; ok && g2 < g1; ++g2) {
+        if (!it.done() && !(ok = gemm1())) break;
+        const int st = g2 % NST, buf = g2 & 1;
+        if (!mbar_wait(&sm.pready[buf], (g2 >> 1) & 1, abort_flag, status) ||
+            !mbar_wait(&sm.fullv[st], (g2 / NST) & 1, abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t id = idesc(BM, DV);
+        const int npad = npad_ring[g2 & 3];
+        for (int kk = 0; kk < npad / 16; ++kk) {
+          const uint64_t b = sdesc(sm.vt[st][kk >> 2] + (kk & 3) * 16);
+          tc_mma_ts(tmem_o, tmem + p_col(buf) + kk * 8, b, id, (g2 > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&sm.pfree[buf]);
+        tc_commit(&sm.emptyv[st]);
       }
-      if (ok && t >= 1) ok = gemm2(t - 1, prev_npad);
       tc_commit(&sm.obar);  // also tracks every MMA issued, on the abort path too
       mbar_drain(&sm.obar, 0, status);
     }
   } else {
     // ------------------------------------------------------------ epilogue warps
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;  // which 16-column chunks this warp takes
+    const int grp = (warp - 2) >> 2;  // tiles of parity grp (and, at the end, half of O)
     const int r = quad * 32 + lane;
     const int n = r0 + r;
     const bool valid = n < q.n;
     const int i = valid ? q_cluster[q.lab + n] : i_first;
     const int slot = i - i_first;
-    const bool staged = slot < kSlots;
+    const bool staged = slot < nslots;
     const float *wrow = Wi + (int64_t)i * wl;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     TileIter<BN, CHUNK> it;
@@ -295,18 +337,46 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     int t = 0;
     bool ok = true;
     for (; !it.done(); it.next(), ++t) {
+      if ((t & 1) != grp) continue;
       const KTile kt = it.get();
       const int buf = t & 1, st = t % NST;
-      if (!mbar_wait(&sm.sfull[buf], (t >> 1) & 1, abort_flag, status)) { ok = false; break; }
-      if (!mbar_wait(&sm.full[st], (t / NST) & 1, abort_flag, status)) { ok = false; break; }
+      // (a wait that gave up in one lane stops the whole warp: the TMEM accesses below
+      // are warp-collective)
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.sfull[buf], (t >> 1) & 1, abort_flag, status) &&
+                                       mbar_wait(&sm.fulle[st], (t / NST) & 1, abort_flag, status))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      if (t >= 2 && !mbar_wait(&sm.pfree[buf], ((t - 2) >> 1) & 1, abort_flag, status)) { ok = false; break; }
       const float a0 = sm.c0[st][0][r], a1 = sm.c1[st][0][r];
-      const int lo = kt.c - kt.x0, hi = kt.c + kt.n - kt.x0;  // unmasked columns [lo, hi)
       const float *ws = staged ? &sm.w[st][slot][0] : wrow + kt.x0;
-      for (int cb = half; cb < kt.npad / 16; cb += 2) {
+      constexpr int kBatch = 4;  // 16-column chunks loaded per TMEM wait
+      const int nch16 = kt.npad / 16;
+      for (int cb0 = 0; cb0 < nch16; cb0 += kBatch) {
+      uint32_t xr[kBatch][16];
+#pragma unroll
+      for (int qi = 0; qi < kBatch; ++qi)
+        if (cb0 + qi < nch16) tmem_ld16_async(tmem + lane_base + s_col(buf) + (cb0 + qi) * 16, xr[qi]);
+      tmem_ld_wait();
+      // P(t) overwrites P(t-2): wait until the MMA reading that has completed
+      if (cb0 == 0 && t >= 2 &&
+          !__all_sync(0xffffffffu, mbar_wait(&sm.pfree[buf], ((t - 2) >> 1) & 1, abort_flag, status))) {
+        ok = false;
+        break;
+      }
+      if (cb0 + kBatch >= nch16) {
+        // all of S read: its buffer can take the group's next tile while P is written
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sfree[buf]);
+      }
+#pragma unroll
+      for (int qi = 0; qi < kBatch; ++qi) {
+        const int cb = cb0 + qi;
+        if (cb >= nch16) break;
         float x[16];
-        tmem_ld16(tmem + lane_base + s_col(buf) + cb * 16, x);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(xr[qi][e]);
         const int col0 = cb * 16;
         float w[16];
 #pragma unroll
@@ -316,20 +386,23 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
         }
         float pv[16];
-        if (kt.nseg == 1) {
+        // the chunk's 16 columns: one cluster (the common case) or a boundary
+        const uint4 sgv = *reinterpret_cast<const uint4 *>(&sm.seg[st][col0]);
+        const unsigned g0 = sgv.x & 0xFFu, g15 = sgv.w >> 24;
+        if (g0 == g15 && g0 != 0xFFu) {
+          const float b0 = kt.nseg == 1 ? a0 : sm.c0[st][g0][r];
+          const float b1 = kt.nseg == 1 ? a1 : sm.c1[st][g0][r];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pv[e] = w[e] * fmaf(a1, x[e], a0);
+          for (int e = 0; e < 16; e += 2) {
+            float t0, t1;
+            fma2(t0, t1, b1, b1, x[e], x[e + 1], b0, b0);
+            mul2(pv[e], pv[e + 1], w[e], w[e + 1], t0, t1);
+          }
           if (!valid) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) pv[e] = 0.f;
-          } else if (col0 < lo || col0 + 16 > hi) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (col0 + e < lo || col0 + e >= hi) pv[e] = 0.f;
           }
         } else {
-          // several clusters in the tile: coefficients per column from the segment map
-          const uint4 sgv = *reinterpret_cast<const uint4 *>(&sm.seg[st][col0]);
           const unsigned char *sg = reinterpret_cast<const unsigned char *>(&sgv);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -348,18 +421,20 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         // 16 bf16 of row r = 8 packed TMEM columns of the P buffer
         tmem_st8(tmem + lane_base + p_col(buf) + cb * 8, pk);
       }
+      }
+      if (!ok) break;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&sm.pready[buf]);
-        mbar_arrive(&sm.sfree[buf]);
+        mbar_arrive(&sm.emptye[st]);  // the tile's epilogue data is consumed
       }
     }
-    if (ok && t > 0 && mbar_wait(&sm.obar, 0, abort_flag, status)) {
+    if (ok && t > 0 && __all_sync(0xffffffffu, mbar_wait(&sm.obar, 0, abort_flag, status))) {
       tc_fence_after();
       const int row = valid ? q_perm[q.lab + n] : 0;
-      for (int cb = half; cb < DV / 16; cb += 2) {
+      for (int cb = grp; cb < DV / 16; cb += 2) {
         float o[16];
         tmem_ld16(tmem_o + lane_base + cb * 16, o);
         if (!valid) continue;
@@ -380,11 +455,11 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           for (int u = 0; u < 4; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
         }
       }
-      if (valid && !O && half == 0) {
+      if (valid && !O && grp == 0) {
         const int64_t rr = (int64_t)p * mt.in.out_stride + mt.in.out0[s] + row;
         part_lse[rr] = lse[q.lab + n];
       }
-    } else if (t == 0 && valid && half == 0) {
+    } else if (t == 0 && valid && grp == 0) {
       // an instance with no keys cannot occur (every key range is non-empty)
       report(status, MUSE_ERR_DEVICE);
     }
