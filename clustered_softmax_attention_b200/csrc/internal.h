@@ -49,6 +49,11 @@ cudaError_t run_kmeans_pair(const void *Xq, const SegTable &tq, const KmeansOut 
                             const void *Xk, const SegTable &tk, const KmeansOut &ok, int dtype,
                             int D, int N, int P, int iters, char *ws, int *status,
                             cudaStream_t st);
+// Every round of K-means in one launch (kmeans_fused.cu): bfloat16, D = 64, C <= 128.
+bool kmeans_fused_supported(int dtype, int D, const SegTable &t);
+cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *const *tabs,
+                             const KmeansOut *outs, int N, int P, int iters, int *status,
+                             cudaStream_t st);
 
 // Sorted working copies of one side (rows in cluster order).
 struct SortedSide {

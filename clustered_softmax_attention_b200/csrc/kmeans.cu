@@ -538,6 +538,10 @@ static cudaError_t dispatch(KmJobs &J, int dtype, int D, int N, int P, int iters
 
 cudaError_t run_kmeans(const void *X, int dtype, int D, int N, const SegTable &tab, int P,
                        int iters, const KmeansOut &o, char *ws, int *status, cudaStream_t st) {
+  if (kmeans_fused_supported(dtype, D, tab)) {
+    const SegTable *t[1] = {&tab};
+    return run_kmeans_fused(1, &X, t, &o, N, P, iters, status, st);
+  }
   KmJobs J;
   J.njobs = 1;
   J.tasks0 = P * tab.nseg;
@@ -554,6 +558,12 @@ cudaError_t run_kmeans_pair(const void *Xq, const SegTable &tq, const KmeansOut 
                             const void *Xk, const SegTable &tk, const KmeansOut &ok, int dtype,
                             int D, int N, int P, int iters, char *ws, int *status,
                             cudaStream_t st) {
+  if (kmeans_fused_supported(dtype, D, tq) && kmeans_fused_supported(dtype, D, tk)) {
+    const void *X[2] = {Xq, Xk};
+    const SegTable *t[2] = {&tq, &tk};
+    const KmeansOut o[2] = {oq, ok};
+    return run_kmeans_fused(2, X, t, o, N, P, iters, status, st);
+  }
   KmJobs J;
   J.njobs = 2;
   J.tasks0 = P * tq.nseg;

@@ -1,0 +1,693 @@
+// Fused Lloyd K-means: every round of every task in ONE launch (bfloat16 rows, D = 64,
+// at most 128 clusters per task).
+//
+// Separate K-means over queries and over keys: pith.science review of arXiv
+// 2509.10406, "What carries the argument" / "Core claim"; gist.science
+// "Technische Samenvatting", "Kernmechanismen" item 1.  Same rounds as kmeans.cu:
+// start from the first C rows; a round assigns every row to its nearest centroid
+// (ties to the lowest index) and replaces every centroid by the mean of its members
+// (an empty cluster keeps its centroid); the labels of the last round are sorted
+// stably into the CSR layout (perm, offsets) that every later stage reads.
+//
+// A task (one segment of one problem) is owned by a group of g = 1, 2, 4 or 8 CTAs
+// of one thread-block cluster of 8; groups are packed into clusters on the host.
+// Each CTA streams its share of the task's 128-row tiles through shared memory (TMA,
+// 4 stages) every round and keeps the centroids in shared memory:
+//   S = X_tile . (c_hi + c_lo)^T      tcgen05.mma, M = 128 rows, N = clusters, fp32 TMEM
+//   label = argmin_c ||c||^2 - 2 S    8 epilogue warps, two column halves per row
+//   Sum += OneHot^T . X_tile          tcgen05.mma, M = 128 clusters, N = D, K = rows:
+//                                     the centroid sums as a contraction with the
+//                                     0/1 membership matrix (exact products, no atomics)
+// The centroid split c = c_hi + c_lo (bfloat16 parts) keeps the distance error below
+// 2^-18 (||x||^2 + ||c||^2), inside the near-tie band of the label parity rule.
+// End of a round: each CTA publishes its partial sums and member counts in shared
+// memory; the group's CTAs reduce disjoint cluster slices by reading every member's
+// partials through distributed shared memory in group order (deterministic), then
+// every CTA gathers the new centroids.  Three cluster barriers per round; the third
+// is split so that its wait overlaps the next round's tiles.
+//
+// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner), warps 2-9 =
+// epilogue.  Every mbarrier wait is bounded (MUSE_ERR_TIMEOUT); every CTA, idle
+// padding CTAs included, executes the same sequence of cluster barriers.
+#include <algorithm>
+#include <vector>
+
+#include "internal.h"
+#include "tc_ptx.cuh"
+
+namespace muse {
+namespace kmf {
+
+constexpr int TM = 128;        // rows per tile
+constexpr int D = 64;          // row width handled by this kernel
+constexpr int NSX = 4;         // row-tile stages
+constexpr int NOH = 2;         // one-hot buffers
+constexpr int CMAX = 128;      // clusters per task
+constexpr int GMAX = 8;        // CTAs per thread-block cluster
+constexpr int TPC = 8;         // row tiles per CTA that a group size aims for
+constexpr int kEpi = 8;        // epilogue warps
+constexpr int kThreads = 64 + 32 * kEpi;
+constexpr int PLD = D + 4;     // padded row stride (floats) of the partial sums
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSumCol = 256;  // TMEM column of the centroid-sum accumulator
+
+struct PlanEntry {
+  uint8_t seg, g;
+  uint16_t pos;  // first CTA of the group inside the problem's span
+};
+struct Job {
+  const void *X;
+  SegTable tab;
+  KmeansOut out;
+  int span;  // CTAs per problem (multiple of the job's largest group)
+  int base;  // first CTA of the job
+  int nent;
+  PlanEntry ent[kMaxSeg];
+};
+struct Params {
+  int njobs, P, N, iters;
+  Job job[2];
+};
+
+struct __align__(1024) Smem {
+  __nv_bfloat16 x[NSX][TM * 64];      // row tiles, rows of 128 B, 128-byte swizzle
+  __nv_bfloat16 oh[NOH][2][TM * 64];  // one-hot rows [row][cluster], two 64-cluster blocks
+  __nv_bfloat16 hi[CMAX * 64];        // centroid split, K-major, 128-byte swizzle
+  __nv_bfloat16 lo[CMAX * 64];
+  float part[CMAX * PLD];             // partial sums; the reducer's new centroids in place
+  float cn[CMAX];                     // squared centroid norms (+inf on padding rows)
+  int cnt[CMAX];                      // this CTA's member counts of the round
+  int tot[CMAX];                      // group totals of the clusters this CTA reduces
+  int totall[CMAX];                   // group totals of every cluster
+  int base[CMAX];                     // final sort: next position per cluster
+  int wc[4][CMAX];                    // final sort: members per (warp, cluster) of a tile
+  float xv[2][2][TM];                 // argmin of each column half, by tile parity
+  int xi[2][2][TM];
+  uint64_t xfull[NSX], xempty[NSX], sfull[2], sfree[2], ohfull[NOH], ohempty[NOH], xch[2];
+  uint64_t sumdone, fin;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+using namespace ptx;
+
+// ------------------------------------------------------------------ cluster helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory object in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t peer_addr(const void *p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_peer_f4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_peer_s32(uint32_t a) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Shared-memory descriptor of an MN-major operand with 128-byte swizzle: rows of
+// 128 B hold 64 consecutive M (or N) elements of one K index, 8 K-rows per 1024-B
+// atom (SBO), `lbo` bytes between successive 64-element blocks along M (or N).
+__device__ __forceinline__ uint64_t sdesc_mn(const void *p, uint32_t lbo) {
+  const uint32_t a = saddr(p);
+  uint64_t d = 0;
+  d |= (uint64_t)((a & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// kind::f16 instruction descriptor with both operands MN-major.
+__host__ __device__ constexpr uint32_t idesc_mn(int M, int N) {
+  return idesc(M, N) | (1u << 15) | (1u << 16);
+}
+
+
+// Writes half h (32 values) of centroid row c into the K-major split operands and
+// returns the partial squared norm.
+__device__ __forceinline__ float put_centroid(Smem &sm, int c, int h, const float (&v)[32]) {
+  float sq = 0.f;
+#pragma unroll
+  for (int j4 = 0; j4 < 4; ++j4) {
+    const int j = 4 * h + j4;
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const float a = v[8 * j4 + e], b = v[8 * j4 + e + 1];
+      const __nv_bfloat162 hh = __floats2bfloat162_rn(a, b);
+      const float2 hf = __bfloat1622float2(hh);
+      const __nv_bfloat162 ll = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+      hw[e >> 1] = *reinterpret_cast<const uint32_t *>(&hh);
+      lw[e >> 1] = *reinterpret_cast<const uint32_t *>(&ll);
+      sq = fmaf(a, a, sq);
+      sq = fmaf(b, b, sq);
+    }
+    const int off = c * 64 + ((j ^ (c & 7)) << 3);
+    *reinterpret_cast<uint4 *>(&sm.hi[off]) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4 *>(&sm.lo[off]) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+  return sq;
+}
+
+__global__ void __cluster_dims__(GMAX, 1, 1) __launch_bounds__(kThreads, 1)
+km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
+         const __grid_constant__ Params prm, int *status) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                       ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int *abort_flag = &sm.abort_flag;
+
+  // ---------------------------------------------- the group and task of this CTA
+  const int jb = (prm.njobs > 1 && (int)blockIdx.x >= prm.job[1].base) ? 1 : 0;
+  const Job &J = prm.job[jb];
+  const CUtensorMap *map = jb ? &map1 : &map0;
+  const int local = (int)blockIdx.x - J.base;
+  const int p = local / J.span, lp = local - p * J.span;
+  int seg = -1, g = 1, rank = 0;
+  if (p < prm.P)
+    for (int e = 0; e < J.nent; ++e) {
+      const int pos = J.ent[e].pos, ge = J.ent[e].g;
+      if (lp >= pos && lp < pos + ge) {
+        seg = J.ent[e].seg;
+        g = ge;
+        rank = lp - pos;
+        break;
+      }
+    }
+  const bool active = seg >= 0;  // uniform over the CTA
+  Task tk{};
+  if (active) tk = make_task(J.tab, p * J.tab.nseg + seg);
+  const int C = tk.C;
+  const int CP = (C + 31) & ~31;                      // assign N: both halves multiples of 16
+  const uint32_t gb = cluster_rank() - (uint32_t)rank;  // cluster rank of the group's first CTA
+  const int ntt = (tk.n + TM - 1) / TM;
+  const int tpc = (ntt + g - 1) / g;
+  const int t0 = rank * tpc;
+  const int nt = active ? max(0, min(ntt - t0, tpc)) : 0;  // this CTA's row tiles
+  const int64_t grow0 = (int64_t)p * prm.N + tk.row0;
+  const int T = prm.iters;
+
+  // ---------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NSX; ++i) {
+      mbar_init(&sm.xfull[i], 1);
+      mbar_init(&sm.xempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.sfull[i], 1);
+      mbar_init(&sm.sfree[i], kEpi);
+      mbar_init(&sm.xch[i], kEpi);
+    }
+    for (int i = 0; i < NOH; ++i) {
+      mbar_init(&sm.ohfull[i], kEpi);
+      mbar_init(&sm.ohempty[i], 1);
+    }
+    mbar_init(&sm.sumdone, 1);
+    mbar_init(&sm.fin, 1);
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (active && warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     saddr(&sm.tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (active) {
+    // starting centroids: the first C rows of the task
+    for (int tid = threadIdx.x; tid < 2 * CMAX; tid += kThreads) {
+      const int c = tid >> 1, h = tid & 1;
+      float v[32];
+      const __nv_bfloat16 *xr = static_cast<const __nv_bfloat16 *>(J.X) + (grow0 + c) * D + h * 32;
+#pragma unroll
+      for (int k = 0; k < 32; k += 8) {
+        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+        if (c < C) raw = *reinterpret_cast<const uint4 *>(xr + k);
+        const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(b2[e]);
+          v[k + 2 * e] = f.x;
+          v[k + 2 * e + 1] = f.y;
+        }
+      }
+      float sq = put_centroid(sm, c, h, v);
+      sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+      if (c < C && c % g == rank) {  // the reducer of c keeps the current centroid in memory
+        float4 *gc = reinterpret_cast<float4 *>(J.out.centroids + (tk.cen + c) * D + h * 32);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) gc[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+      }
+      if (h == 0) {
+        sm.cn[c] = c < C ? sq : CUDART_INF_F;
+        sm.cnt[c] = 0;
+      }
+    }
+    for (int e = threadIdx.x; e < 4 * CMAX; e += kThreads) (&sm.wc[0][0])[e] = 0;
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  int loaded = 0;  // producer: row tiles issued, counted over all rounds
+  for (int r = 0; r < T; ++r) {
+    const bool last = r == T - 1;
+    const int u0 = r * nt;
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0 && nt > 0 && !*abort_flag) {
+        // this round's tiles, then the next round's first stages (the rows do not change)
+        const int target = (r + 1) * nt + (last ? 0 : min(NSX, nt));
+        for (; loaded < target; ++loaded) {
+          const int u = loaded, st = u % NSX, t = u % nt;
+          if (u >= NSX && !mbar_wait(&sm.xempty[st], ((u / NSX) - 1) & 1, abort_flag, status)) break;
+          mbar_expect_tx(&sm.xfull[st], TM * 128);
+          tma_load_2d(sm.x[st], map, 0, (int)(grow0 + (int64_t)(t0 + t) * TM), &sm.xfull[st]);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0 && nt > 0 && !*abort_flag) {
+        auto assign = [&](int u) -> bool {
+          const int st = u % NSX, buf = u & 1;
+          if (!mbar_wait(&sm.xfull[st], (u / NSX) & 1, abort_flag, status)) return false;
+          if (u >= 2 && !mbar_wait(&sm.sfree[buf], ((u - 2) >> 1) & 1, abort_flag, status)) return false;
+          tc_fence_after();
+          const uint32_t id = idesc(TM, CP);
+          for (int kk = 0; kk < D / 16; ++kk)
+            tc_mma(tmem + buf * 128, sdesc(sm.x[st] + kk * 16), sdesc(sm.hi + kk * 16), id, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk)
+            tc_mma(tmem + buf * 128, sdesc(sm.x[st] + kk * 16), sdesc(sm.lo + kk * 16), id, 1u);
+          tc_commit(&sm.sfull[buf]);
+          return true;
+        };
+        auto sums = [&](int u, bool first) -> bool {
+          const int st = u % NSX, ob = u % NOH;
+          if (!mbar_wait(&sm.ohfull[ob], (u / NOH) & 1, abort_flag, status)) return false;
+          tc_fence_after();
+          const uint32_t id = idesc_mn(TM, D);
+          for (int ks = 0; ks < TM / 16; ++ks)
+            tc_mma(tmem + kSumCol, sdesc_mn(sm.oh[ob][0] + ks * 16 * 64, TM * 64 * 2),
+                   sdesc_mn(sm.x[st] + ks * 16 * 64, TM * 64 * 2), id, (first && ks == 0) ? 0u : 1u);
+          tc_commit(&sm.ohempty[ob]);
+          tc_commit(&sm.xempty[st]);
+          return true;
+        };
+        bool ok = assign(u0) && (nt < 2 || assign(u0 + 1));
+        for (int t = 0; ok && t < nt; ++t) {
+          if (t + 2 < nt && !(ok = assign(u0 + t + 2))) break;
+          ok = sums(u0 + t, t == 0);
+        }
+        tc_commit(&sm.sumdone);  // tracks every MMA issued this round, on the abort path too
+      }
+      __syncwarp();
+    } else {
+      // ------------------------------------------------------------ epilogue
+      const int half = (warp - 2) >> 2, quad = warp & 3;
+      const int rr = quad * 32 + lane;
+      const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+      const int hc = CP >> 1;  // columns of this half
+      const int col0 = half * hc;
+      for (int t = 0; t < nt; ++t) {
+        const int u = u0 + t, buf = u & 1, ob = u % NOH, xb = u & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.sfull[buf], (u >> 1) & 1, abort_flag, status))) break;
+        tc_fence_after();
+        uint32_t raw[4][16];
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+          if (ch * 16 < hc) tmem_ld16_async(tmem + lane_base + buf * 128 + col0 + ch * 16, raw[ch]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sfree[buf]);
+        // four independent chains (one per 16-column chunk), merged in column order
+        float best[4];
+        int bi[4];
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          best[ch] = CUDART_INF_F;
+          bi[ch] = col0;
+          if (ch * 16 < hc) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c = col0 + ch * 16 + e;
+              const float dd = fmaf(-2.f, __uint_as_float(raw[ch][e]), sm.cn[c]);
+              if (dd < best[ch]) {  // strict: the lowest index wins a tie
+                best[ch] = dd;
+                bi[ch] = c;
+              }
+            }
+          }
+        }
+        float bv = best[0];
+        int bc = bi[0];
+#pragma unroll
+        for (int ch = 1; ch < 4; ++ch)
+          if (best[ch] < bv) {
+            bv = best[ch];
+            bc = bi[ch];
+          }
+        sm.xv[xb][half][rr] = bv;
+        sm.xi[xb][half][rr] = bc;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.xch[xb]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.xch[xb], (u >> 1) & 1, abort_flag, status))) break;
+        const float v0 = sm.xv[xb][0][rr], v1 = sm.xv[xb][1][rr];
+        const int row = (t0 + t) * TM + rr;
+        const bool valid = row < tk.n;
+        const int L = !valid ? -1 : min(v1 < v0 ? sm.xi[xb][1][rr] : sm.xi[xb][0][rr], C - 1);
+        if (valid && half == 0) {
+          atomicAdd(&sm.cnt[L], 1);  // integer: exact in any order
+          if (last) J.out.labels[tk.lab + row] = L;
+        }
+        // this row's 64 one-hot entries of block `half` (bf16 1.0 = 0x3F80)
+        if (u >= NOH &&
+            !__all_sync(0xffffffffu, mbar_wait(&sm.ohempty[ob], ((u / NOH) - 1) & 1, abort_flag, status)))
+          break;
+        unsigned char *dst = reinterpret_cast<unsigned char *>(sm.oh[ob][half]) + rr * 128;
+        const int lc = L - half * 64;
+        const bool hit = lc >= 0 && lc < 64;
+        const uint32_t one = (lc & 1) ? 0x3F800000u : 0x00003F80u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const bool here = hit && (lc >> 3) == j;
+          const int w = (lc & 7) >> 1;
+          const uint4 val = make_uint4(here && w == 0 ? one : 0u, here && w == 1 ? one : 0u,
+                                       here && w == 2 ? one : 0u, here && w == 3 ? one : 0u);
+          *reinterpret_cast<uint4 *>(dst + ((j ^ (rr & 7)) << 4)) = val;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.ohfull[ob]);
+      }
+    }
+
+    // ---------------------------------------------------------------- end of the round
+    // (1) this CTA's partial sums (TMEM lane = cluster) into `part`, once every peer has
+    //     finished reading the previous round's contents
+    if (r > 0) cluster_wait();
+    if (active && warp >= 2) {
+      const int half = (warp - 2) >> 2, quad = warp & 3;
+      const int c = quad * 32 + lane;
+      float v[32];
+      bool have = false;
+      if (nt > 0) have = __all_sync(0xffffffffu, mbar_wait(&sm.sumdone, r & 1, abort_flag, status));
+      if (have) {
+        tc_fence_after();
+        float a[16], b[16];
+        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + kSumCol + half * 32, a);
+        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + kSumCol + half * 32 + 16, b);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          v[e] = a[e];
+          v[16 + e] = b[e];
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+      }
+      float4 *dst = reinterpret_cast<float4 *>(&sm.part[c * PLD + half * 32]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+      tc_fence_before();
+    }
+    __syncwarp();
+    cluster_arrive();
+    cluster_wait();
+    // (2) reduction: this CTA owns the clusters c = rank + g k; members summed in group order
+    if (active) {
+      const int nslice = (C - rank + g - 1) / g;
+      for (int it = threadIdx.x; it < nslice * (D / 4); it += kThreads) {
+        const int c = rank + g * (it / (D / 4)), v4 = it % (D / 4);
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        int total = 0;
+        for (int m = 0; m < g; ++m) {
+          const float4 a = ld_peer_f4(peer_addr(&sm.part[c * PLD + 4 * v4], gb + m));
+          s.x += a.x;
+          s.y += a.y;
+          s.z += a.z;
+          s.w += a.w;
+          total += ld_peer_s32(peer_addr(&sm.cnt[c], gb + m));
+        }
+        float4 *gc = reinterpret_cast<float4 *>(J.out.centroids + (tk.cen + c) * D + 4 * v4);
+        float4 nv;
+        if (total > 0) {
+          const float inv = 1.f / (float)total;
+          nv = make_float4(s.x * inv, s.y * inv, s.z * inv, s.w * inv);
+        } else {
+          nv = *gc;  // empty: keeps its centroid
+        }
+        *reinterpret_cast<float4 *>(&sm.part[c * PLD + 4 * v4]) = nv;
+        *gc = nv;
+        if (v4 == 0) sm.tot[c] = total;
+      }
+    }
+    __syncwarp();
+    cluster_arrive();
+    cluster_wait();
+    // (3) every CTA gathers the new centroids (split operands, norms) and the totals
+    if (active) {
+      for (int tid = threadIdx.x; tid < 2 * CMAX; tid += kThreads) {
+        const int c = tid >> 1, h = tid & 1;
+        const uint32_t q = gb + (uint32_t)(c % g);
+        float v[32];
+        if (c < C) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float4 a = ld_peer_f4(peer_addr(&sm.part[c * PLD + h * 32 + 4 * k], q));
+            v[4 * k] = a.x;
+            v[4 * k + 1] = a.y;
+            v[4 * k + 2] = a.z;
+            v[4 * k + 3] = a.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0.f;
+        }
+        float sq = put_centroid(sm, c, h, v);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+        if (h == 0) {
+          sm.cn[c] = c < C ? sq : CUDART_INF_F;
+          sm.totall[c] = c < C ? ld_peer_s32(peer_addr(&sm.tot[c], q)) : 0;
+          if (!last) sm.cnt[c] = 0;
+        }
+      }
+      if (last) {
+        // CSR offsets (exclusive scan of the totals) and, for this CTA's rows, the first
+        // position of each cluster: offsets + the members held by earlier CTAs of the group
+        __syncthreads();
+        if (warp == 2) {
+          int tv[4], s = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            tv[k] = sm.totall[4 * lane + k];
+            s += tv[k];
+          }
+          int inc = s;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+          }
+          int run = inc - s;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int c = 4 * lane + k;
+            if (c < C) {
+              sm.base[c] = run;
+              if (rank == 0) J.out.offsets[tk.off + c] = run;
+            }
+            run += tv[k];
+          }
+          if (lane == 31 && rank == 0) J.out.offsets[tk.off + C] = run;
+        }
+        __syncthreads();
+        if (threadIdx.x < C) {
+          int b = sm.base[threadIdx.x];
+          for (int m = 0; m < rank; ++m) b += ld_peer_s32(peer_addr(&sm.cnt[threadIdx.x], gb + m));
+          sm.base[threadIdx.x] = b;
+        }
+      }
+    }
+    __syncwarp();
+    cluster_arrive();  // its wait comes before the next write of `part` (or before exit)
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+
+  // ------------------------------------------------ stable scatter of the last labels
+  const bool aborted = *abort_flag != 0;  // read after the barrier above: uniform
+  if (active && !aborted && warp >= 2 && warp < 6) {
+    const int quad = warp & 3, rr = quad * 32 + lane;
+    for (int t = 0; t < nt; ++t) {
+      const int row = (t0 + t) * TM + rr;
+      const bool valid = row < tk.n;
+      const int L = valid ? J.out.labels[tk.lab + row] : -1;  // written by this thread
+      const unsigned peers = __match_any_sync(0xffffffffu, L);
+      const int wrank = __popc(peers & ((1u << lane) - 1u));
+      if (valid && wrank == 0) sm.wc[quad][L] = __popc(peers);
+      named_sync(1, 128);
+      if (valid) {
+        int pos = sm.base[L] + wrank;
+        for (int q2 = 0; q2 < quad; ++q2) pos += sm.wc[q2][L];
+        if (pos >= 0 && pos < tk.n)
+          J.out.perm[tk.lab + pos] = tk.row0 + row;
+        else
+          report(status, MUSE_ERR_DEVICE);
+      }
+      named_sync(1, 128);
+      if (rr < C) {
+        int s = 0;
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2) {
+          s += sm.wc[q2][rr];
+          sm.wc[q2][rr] = 0;
+        }
+        sm.base[rr] += s;
+      }
+      named_sync(1, 128);
+    }
+  }
+
+  cluster_wait();  // every peer has finished reading this CTA's shared memory
+  // ------------------------------------------------ teardown
+  if (warp == 0 && lane == 0)
+    for (int u = max(0, loaded - NSX); u < loaded; ++u) mbar_drain(&sm.xfull[u % NSX], (u / NSX) & 1, status);
+  if (active && warp == 1 && lane == 0) {
+    tc_commit(&sm.fin);
+    mbar_drain(&sm.fin, 0, status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (active && warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host side
+// CTAs of a task's group: enough for about TPC row tiles each, a power of two <= 8.
+static int group_size(int n) {
+  const int tiles = (n + TM - 1) / TM;
+  const int want = (tiles + TPC - 1) / TPC;
+  int g = 1;
+  while (g < want && g < GMAX) g <<= 1;
+  return g;
+}
+
+// Lays the segments of one problem out in CTA slots, largest groups first, so every
+// group starts at a multiple of its size and never straddles a cluster of 8.  Returns
+// the largest group.
+static int plan_job(Job &J, const SegTable &t) {
+  std::vector<int> order(t.nseg);
+  for (int s = 0; s < t.nseg; ++s) order[s] = s;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    return group_size(t.nrow[a]) > group_size(t.nrow[b]);
+  });
+  int pos = 0, gmax = 1;
+  for (int e = 0; e < t.nseg; ++e) {
+    const int s = order[e], g = group_size(t.nrow[s]);
+    J.ent[e].seg = (uint8_t)s;
+    J.ent[e].g = (uint8_t)g;
+    J.ent[e].pos = (uint16_t)pos;
+    pos += g;
+    gmax = std::max(gmax, g);
+  }
+  J.nent = t.nseg;
+  J.span = (pos + gmax - 1) / gmax * gmax;
+  return gmax;
+}
+
+}  // namespace kmf
+
+bool kmeans_fused_supported(int dtype, int D, const SegTable &t) {
+  if (dtype != MUSE_BF16 || D != kmf::D || t.max_C > kmf::CMAX || t.nseg > 255) return false;
+  int span = 0;
+  for (int s = 0; s < t.nseg; ++s) span += kmf::group_size(t.nrow[s]);
+  if (span > 65535) return false;
+  // one 8-CTA cluster of this kernel must fit on the device
+  static int fits = -1;
+  if (fits < 0) {
+    const size_t smem = sizeof(kmf::Smem) + 1024;
+    fits = cudaFuncSetAttribute(kmf::km_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+           cudaSuccess;
+    if (fits) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(kmf::GMAX);
+      cfg.blockDim = dim3(kmf::kThreads);
+      cfg.dynamicSmemBytes = smem;
+      int n = 0;
+      fits = cudaOccupancyMaxActiveClusters(&n, kmf::km_fused, &cfg) == cudaSuccess && n > 0;
+    }
+    if (!fits) cudaGetLastError();  // the old path takes over; leave no error behind
+  }
+  return fits == 1;
+}
+
+cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *const *tabs,
+                             const KmeansOut *outs, int N, int P, int iters, int *status,
+                             cudaStream_t st) {
+  using namespace kmf;
+  Params prm{};
+  prm.njobs = njobs;
+  prm.P = P;
+  prm.N = N;
+  prm.iters = iters;
+  int cursor = 0;
+  for (int j = 0; j < njobs; ++j) {
+    Job &J = prm.job[j];
+    J.X = X[j];
+    J.tab = *tabs[j];
+    J.out = outs[j];
+    const int gmax = plan_job(J, *tabs[j]);
+    cursor = (cursor + gmax - 1) / gmax * gmax;
+    J.base = cursor;
+    cursor += P * J.span;
+  }
+  const int grid = (cursor + GMAX - 1) / GMAX * GMAX;
+  CUtensorMap m0, m1;
+  if (!ptx::make_map(&m0, X[0], D, (uint64_t)P * N, D, TM) ||
+      !ptx::make_map(&m1, X[njobs > 1 ? 1 : 0], D, (uint64_t)P * N, D, TM))
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(km_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  km_fused<<<grid, kThreads, smem, st>>>(m0, m1, prm, status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace muse

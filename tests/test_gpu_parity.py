@@ -70,12 +70,16 @@ def check_kmeans_rounds(X, C, T, dt):
     return excused
 
 
+# bf16 with D = 64 and C <= 128 runs the single-launch K-means; the sizes give groups of
+# 1, 2, 4 and 8 CTAs per task, ragged last tiles and (N = 4200) a CTA with no row tile.
 @pytest.mark.parametrize("dt,N,D,C,H", [("f32", 1024, 64, 32, 1), ("bf16", 2048, 128, 64, 2),
-                                         ("bf16", 1000, 64, 37, 1)])
+                                         ("bf16", 1000, 64, 37, 1), ("bf16", 1500, 64, 16, 1),
+                                         ("bf16", 2100, 64, 64, 1), ("bf16", 4200, 64, 128, 1),
+                                         ("bf16", 8192, 64, 128, 2)])
 def test_kmeans_rounds_teacher_forced(dt, N, D, C, H):
     Q, K, V = mixture(11, 1, H, N, D, D, 48, 0.3 / np.sqrt(D), dt)
     ex = check_kmeans_rounds(Q, C, 6, dt)
-    assert ex <= 3
+    assert ex <= 3 + 1e-4 * N * H * 6  # excused near-ties stay rare
 
 
 def run_gpu_pipeline(Q, K, V, Cq, Ck, T, s, dt, with_cov=False):
