@@ -41,6 +41,7 @@ constexpr int kThreads = 64 + 32 * kEpiWarps + 32;  // + the epilogue-data produ
 constexpr int kEWarp = 2 + kEpiWarps;               // that warp's index
 constexpr int kSlots = 8;    // query clusters per CTA whose tilt weights are staged
 constexpr int kTileSegs = 8; // key clusters packed into one tile at most
+constexpr int kMixed = 0xFE; // chunk code: more than one key cluster among the valid columns
 
 // Widest key tile: 128 keys when D = Dv = 64, else 64 (shared memory budget).
 template <int D, int DV>
@@ -59,6 +60,7 @@ struct __align__(1024) Smem {
   float c0[NST][kTileSegs][BM];                // coefficients of the tile's key clusters
   float c1[NST][kTileSegs][BM];
   unsigned char seg[NST][BN];                  // column -> cluster of the tile (0xFF: masked)
+  int chunk[NST][BN / 16];                     // per 16 columns: valid mask << 8 | cluster (or kMixed)
   int koff[kMaxClusters + 1];                  // the instance's key-cluster offsets
   // per stage: key tile (consumed by the first MMA), values (second MMA), epilogue
   // data (tilt weights, coefficients, segment map; consumed by the epilogue)
@@ -69,6 +71,36 @@ struct __align__(1024) Smem {
 };
 
 using namespace ptx;
+
+struct F16 {
+  float v[16];
+};
+struct P8 {
+  uint32_t v[8];
+};
+
+// P for a 16-column chunk whose valid columns belong to more than one key cluster, or
+// for a warp with a row whose tilt weights are not staged: per-column cluster lookup.
+// Rare, so kept out of line (the hot loop stays small).
+template <int D, int DV>
+static __device__ __noinline__ P8 mixed_chunk(const Smem<D, DV> &sm, int st, int cb, int r,
+                                              const float *wp, F16 x) {
+  P8 out;
+  const int col0 = cb * 16;
+#pragma unroll
+  for (int e = 0; e < 16; e += 2) {
+    float pv[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int col = col0 + e + h;
+      const int g = sm.seg[st][col];
+      pv[h] = g == 0xFF ? 0.f : wp[col] * fmaf(sm.c1[st][g][r], x.v[e + h], sm.c0[st][g][r]);
+    }
+    __nv_bfloat162 hh = __floats2bfloat162_rn(pv[0], pv[1]);
+    out.v[e >> 1] = *reinterpret_cast<uint32_t *>(&hh);
+  }
+  return out;
+}
 
 // Key tiles of an instance: cluster j's keys [b, e) in chunks of CHUNK.
 // A key tile: keys [c, c+n) of the sorted keys, widened to start at x0 = c & ~7 and
@@ -262,6 +294,21 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           while (sg + 1 < kt.nseg && key >= koff[kt.j + sg + 1]) ++sg;
         }
         sm.seg[st][col] = (unsigned char)sg;
+        // per 16-column chunk: valid-column mask, and the chunk's key cluster when all
+        // its valid columns share one (else kMixed)
+        const bool in = sg != 0xFF;
+        const unsigned bal = __ballot_sync(0xffffffffu, in);
+        unsigned lo = in ? (unsigned)sg : 255u, hi = in ? (unsigned)sg : 0u;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {  // within each 16-lane half
+          lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+          hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        if ((lane & 15) == 0) {
+          const unsigned m16 = lane < 16 ? (bal & 0xFFFFu) : (bal >> 16);
+          const int g = m16 == 0 ? 0 : (lo == hi ? (int)lo : kMixed);
+          sm.chunk[st][col >> 4] = (int)(m16 << 8) | g;
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.fulle[st]);  // releases the segment map with the stage
@@ -330,6 +377,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int i = valid ? q_cluster[q.lab + n] : i_first;
     const int slot = i - i_first;
     const bool staged = slot < nslots;
+    const bool wfast = __all_sync(0xffffffffu, staged);  // every row of the warp has staged weights
     const float *wrow = Wi + (int64_t)i * wl;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     TileIter<BN, CHUNK> it;
@@ -348,79 +396,71 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         break;
       }
       tc_fence_after();
-      const float a0 = sm.c0[st][0][r], a1 = sm.c1[st][0][r];
-      const float *ws = staged ? &sm.w[st][slot][0] : wrow + kt.x0;
-      constexpr int kBatch = 4;  // 16-column chunks loaded per TMEM wait
+      const float *wsm = &sm.w[st][staged ? slot : 0][0];
       const int nch16 = kt.npad / 16;
-      for (int cb0 = 0; cb0 < nch16; cb0 += kBatch) {
-      uint32_t xr[kBatch][16];
-#pragma unroll
-      for (int qi = 0; qi < kBatch; ++qi)
-        if (cb0 + qi < nch16) tmem_ld16_async(tmem + lane_base + s_col(buf) + (cb0 + qi) * 16, xr[qi]);
-      tmem_ld_wait();
-      // P(t) overwrites P(t-2): wait until the MMA reading that has completed
-      if (cb0 == 0 && t >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait(&sm.pfree[buf], ((t - 2) >> 1) & 1, abort_flag, status))) {
-        ok = false;
-        break;
-      }
-      if (cb0 + kBatch >= nch16) {
-        // all of S read: its buffer can take the group's next tile while P is written
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.sfree[buf]);
-      }
-#pragma unroll
-      for (int qi = 0; qi < kBatch; ++qi) {
-        const int cb = cb0 + qi;
-        if (cb >= nch16) break;
-        float x[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(xr[qi][e]);
-        const int col0 = cb * 16;
-        float w[16];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (staged || kt.x0 + col0 + 4 * u < wl) v4 = *reinterpret_cast<const float4 *>(ws + col0 + 4 * u);
-          w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
+      for (int cb0 = 0; cb0 < nch16; cb0 += 2) {
+        const bool two = cb0 + 1 < nch16;  // uniform
+        uint32_t xr[2][16];
+        tmem_ld16_async(tmem + lane_base + s_col(buf) + cb0 * 16, xr[0]);
+        if (two) tmem_ld16_async(tmem + lane_base + s_col(buf) + (cb0 + 1) * 16, xr[1]);
+        tmem_ld_wait();
+        if (cb0 + 2 >= nch16) {
+          // all of S read: its buffer can take the group's next tile while P is written
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.sfree[buf]);
         }
-        float pv[16];
-        // the chunk's 16 columns: one cluster (the common case) or a boundary
-        const uint4 sgv = *reinterpret_cast<const uint4 *>(&sm.seg[st][col0]);
-        const unsigned g0 = sgv.x & 0xFFu, g15 = sgv.w >> 24;
-        if (g0 == g15 && g0 != 0xFFu) {
-          const float b0 = kt.nseg == 1 ? a0 : sm.c0[st][g0][r];
-          const float b1 = kt.nseg == 1 ? a1 : sm.c1[st][g0][r];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float t0, t1;
-            fma2(t0, t1, b1, b1, x[e], x[e + 1], b0, b0);
-            mul2(pv[e], pv[e + 1], w[e], w[e + 1], t0, t1);
-          }
-          if (!valid) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pv[e] = 0.f;
-          }
-        } else {
-          const unsigned char *sg = reinterpret_cast<const unsigned char *>(&sgv);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int g = sg[e];
-            float pe = 0.f;
-            if (valid && g != 0xFF) pe = w[e] * fmaf(sm.c1[st][g][r], x[e], sm.c0[st][g][r]);
-            pv[e] = pe;
-          }
+        // P(t) overwrites P(t-2): wait until the MMA reading that has completed
+        if (cb0 == 0 && t >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(&sm.pfree[buf], ((t - 2) >> 1) & 1, abort_flag, status))) {
+          ok = false;
+          break;
         }
-        uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          __nv_bfloat162 h = __floats2bfloat162_rn(pv[e], pv[e + 1]);
-          pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
+        for (int qi = 0; qi < 2; ++qi) {
+          if (qi == 1 && !two) break;
+          const int cb = cb0 + qi;
+          const int code = sm.chunk[st][cb];
+          uint32_t pk[8];
+          if (wfast && (code & 0xFF) != kMixed) {
+            // one key cluster over the chunk's valid columns (common case)
+            const int g = code & 0xFF;
+            const uint32_t msk = (uint32_t)code >> 8;
+            const float b0 = sm.c0[st][g][r], b1 = sm.c1[st][g][r];
+            float w[16];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float4 v4 = *reinterpret_cast<const float4 *>(wsm + cb * 16 + 4 * u);
+              w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
+            }
+            float pv[16];
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              float t0, t1;
+              fma2(t0, t1, b1, b1, __uint_as_float(xr[qi][e]), __uint_as_float(xr[qi][e + 1]), b0, b0);
+              mul2(pv[e], pv[e + 1], w[e], w[e + 1], t0, t1);
+            }
+            if (msk != 0xFFFFu) {
+              // columns outside the tile's keys: their S may come from unrelated rows
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pv[e] = ((msk >> e) & 1u) ? pv[e] : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(pv[e], pv[e + 1]);
+              pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
+            }
+          } else {
+            F16 xv;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) xv.v[e] = __uint_as_float(xr[qi][e]);
+            const P8 pr = mixed_chunk<D, DV>(sm, st, cb, r, staged ? wsm : wrow + kt.x0, xv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pk[e] = pr.v[e];
+          }
+          // 16 bf16 of row r = 8 packed TMEM columns of the P buffer
+          tmem_st8(tmem + lane_base + p_col(buf) + cb * 8, pk);
         }
-        // 16 bf16 of row r = 8 packed TMEM columns of the P buffer
-        tmem_st8(tmem + lane_base + p_col(buf) + cb * 8, pk);
-      }
       }
       if (!ok) break;
       tmem_st_wait();

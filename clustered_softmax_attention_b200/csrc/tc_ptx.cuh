@@ -37,8 +37,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *b) {
 }
 // One bounded probe of the phase: the warp may sleep (up to 50 us) until it completes,
 // so waiting roles do not take issue slots from working ones.
+#ifndef MUSE_WAIT_MODE
+#define MUSE_WAIT_MODE 1
+#endif
 __device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
   uint32_t ok;
+#if MUSE_WAIT_MODE == 0
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
@@ -46,6 +50,23 @@ __device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
       : "=r"(ok)
       : "r"(saddr(b)), "r"(parity), "r"(50000)
       : "memory");
+#elif MUSE_WAIT_MODE == 1
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(saddr(b)), "r"(parity)
+      : "memory");
+#else
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(saddr(b)), "r"(parity)
+      : "memory");
+#endif
   return ok != 0;
 }
 // Non-blocking test of the phase.
@@ -60,10 +81,10 @@ __device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false when the limit ran out or another role has aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile int *abort_flag,
-                                          int *status) {
-  if (mbar_try(b, parity)) return true;
+// Bounded wait: false when the limit ran out or another role has aborted.  The first
+// probe is inlined; the polling loop is a call, which keeps the hot loops small.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t *b, uint32_t parity,
+                                                   volatile int *abort_flag, int *status) {
   const uint64_t t0 = now_ns();
   while (true) {
     if (mbar_try(b, parity)) return true;
@@ -74,6 +95,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile int *abort_flag,
+                                          int *status) {
+  if (mbar_try(b, parity)) return true;
+  return mbar_wait_slow(b, parity, abort_flag, status);
 }
 // Bounded wait that ignores the abort flag: used to let in-flight copies and MMAs
 // finish before the CTA releases its shared memory and TMEM.
