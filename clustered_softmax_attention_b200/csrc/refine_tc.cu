@@ -285,30 +285,38 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         cp_async16(&sm.c1[st][sg][4 * lane], in ? (const void *)(C1 + at) : (const void *)W, in ? 16u : 0u);
       }
       cp_async_arrive(&sm.fulle[st]);
-      // column -> segment (0xFF outside [c, c+n))
+      // column -> key cluster of the tile (0xFF outside [c, c+n)), by comparison with
+      // the tile's cluster boundaries held in registers
+      int bnd[kTileSegs - 1];  // first key of the tile's clusters 1 .. nseg-1
+#pragma unroll
+      for (int b = 0; b < kTileSegs - 1; ++b) bnd[b] = b + 1 < kt.nseg ? koff[kt.j + b + 1] : 0x7FFFFFFF;
       for (int col = lane; col < BN; col += 32) {
         const int key = kt.x0 + col;
         int sg = 0xFF;
         if (col < kt.npad && key >= kt.c && key < kt.c + kt.n) {
           sg = 0;
-          while (sg + 1 < kt.nseg && key >= koff[kt.j + sg + 1]) ++sg;
+#pragma unroll
+          for (int b = 0; b < kTileSegs - 1; ++b) sg += key >= bnd[b] ? 1 : 0;
         }
         sm.seg[st][col] = (unsigned char)sg;
-        // per 16-column chunk: valid-column mask, and the chunk's key cluster when all
-        // its valid columns share one (else kMixed)
-        const bool in = sg != 0xFF;
-        const unsigned bal = __ballot_sync(0xffffffffu, in);
-        unsigned lo = in ? (unsigned)sg : 255u, hi = in ? (unsigned)sg : 0u;
+      }
+      // per 16-column chunk: valid-column mask (a contiguous run), and the chunk's key
+      // cluster when its first and last valid columns share one (else kMixed)
+      if (lane < BN / 16) {
+        const int cx = kt.x0 + 16 * lane;
+        const int k0 = max(kt.c, cx), k1 = min(kt.c + kt.n, cx + 16);
+        int code = 0;
+        if (16 * lane < kt.npad && k0 < k1) {
+          int s0 = 0, s1 = 0;
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) {  // within each 16-lane half
-          lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-          hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+          for (int b = 0; b < kTileSegs - 1; ++b) {
+            s0 += k0 >= bnd[b] ? 1 : 0;
+            s1 += k1 - 1 >= bnd[b] ? 1 : 0;
+          }
+          const uint32_t m16 = ((1u << (k1 - cx)) - 1u) & ~((1u << (k0 - cx)) - 1u);
+          code = (int)(m16 << 8) | (s0 == s1 ? s0 : kMixed);
         }
-        if ((lane & 15) == 0) {
-          const unsigned m16 = lane < 16 ? (bal & 0xFFFFu) : (bal >> 16);
-          const int g = m16 == 0 ? 0 : (lo == hi ? (int)lo : kMixed);
-          sm.chunk[st][col >> 4] = (int)(m16 << 8) | g;
-        }
+        sm.chunk[st][lane] = code;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.fulle[st]);  // releases the segment map with the stage
