@@ -23,8 +23,8 @@
 // Warp roles: warp 0 = TMA producer (key and value tiles, each released as soon as
 // its MMA has consumed it), warp 1 = MMA issuer (+ TMEM owner), warps 2-9 = epilogue
 // in two groups of four (TMEM lane quadrant = warp % 4): group g takes the tiles of
-// parity g, i.e. S/P buffer g, so the groups overlap; warp 10 = cp.async producer of
-// the epilogue data.  Every wait on an mbarrier is
+// parity g, i.e. S/P buffer g, so the groups overlap; warps 10-11 = cp.async producers
+// of the epilogue data (tiles of parity 0 and 1).  Every wait on an mbarrier is
 // bounded: past the limit the kernel records MUSE_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 
@@ -37,8 +37,8 @@ namespace tcr {
 constexpr int BM = 128;      // query rows per CTA
 constexpr int NST = 4;       // K / V^T stages
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps + 32;  // + the epilogue-data producer warp
-constexpr int kEWarp = 2 + kEpiWarps;               // that warp's index
+constexpr int kThreads = 64 + 32 * kEpiWarps + 64;  // + two epilogue-data producer warps
+constexpr int kEWarp = 2 + kEpiWarps;               // the first of them (tiles of parity 0)
 constexpr int kSlots = 8;    // query clusters per CTA whose tilt weights are staged
 constexpr int kTileSegs = 8; // key clusters packed into one tile at most
 constexpr int kMixed = 0xFE; // chunk code: more than one key cluster among the valid columns
@@ -257,12 +257,15 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         mbar_drain(&sm.fullv[u % NST], (u / NST) & 1, status);
       }
     }
-  } else if (warp == kEWarp) {
-    // ------------------------------------------------------------ epilogue-data producer
+  } else if (warp >= kEWarp) {
+    // ------------------------------------------------------------ epilogue-data producers
+    // warp kEWarp + par stages the tiles of parity par (stages par, par + 2, ...)
+    const int par = warp - kEWarp;
     TileIter<BN, CHUNK> it;
     it.begin(koff, k.C);
     int t = 0;
     for (; !it.done(); it.next(), ++t) {
+      if ((t & 1) != par) continue;
       const KTile kt = it.get();
       const int st = t % NST;
       int ok = 1;
@@ -322,7 +325,8 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       if (lane == 0) mbar_arrive(&sm.fulle[st]);  // releases the segment map with the stage
     }
     if (lane == 0)
-      for (int u = max(0, t - NST); u < t; ++u) mbar_drain(&sm.fulle[u % NST], (u / NST) & 1, status);
+      for (int u = max(0, t - NST); u < t; ++u)
+        if ((u & 1) == par) mbar_drain(&sm.fulle[u % NST], (u / NST) & 1, status);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // Fixed order S(0), S(1), then for every tile t: S(t+2) (its S buffer is released
