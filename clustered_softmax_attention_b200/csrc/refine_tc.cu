@@ -18,10 +18,11 @@
 //   S  = Qt . K_tile^T            (tcgen05, 128 x npad, fp32 in TMEM, double-buffered)
 //   P  = w .* (c0 + c1 .* S)      (epilogue warps: TMEM -> registers -> bf16 TMEM)
 //   O += P . V_tile               (tcgen05, A = P from TMEM, 128 x Dv, fp32 in TMEM)
-// TMEM columns: S double buffer [0, 2 BN), P double buffer [2 BN, 3 BN) (bf16 packed
-// two per column), O [3 BN, 3 BN + Dv).
-// Warp roles: warp 0 = TMA producer (key and value tiles, each released as soon as
-// its MMA has consumed it), warp 1 = MMA issuer (+ TMEM owner), warps 2-9 = epilogue
+// TMEM columns: S double buffer [0, 2 BN), P ring of three [2 BN, 3.5 BN) (bf16 packed
+// two per column), O [3.5 BN, 3.5 BN + Dv).
+// Warp roles: warp 0 = TMA producer of the key tiles, warp 12 = of the value tiles
+// (each stage released as soon as its MMA has consumed it), warp 1 = MMA issuer
+// (+ TMEM owner), warps 2-9 = epilogue
 // in two groups of four (TMEM lane quadrant = warp % 4): group g takes the tiles of
 // parity g, i.e. S/P buffer g, so the groups overlap; warps 10-11 = cp.async producers
 // of the epilogue data (tiles of parity 0 and 1).  Every wait on an mbarrier is
@@ -37,11 +38,13 @@ namespace tcr {
 constexpr int BM = 128;      // query rows per CTA
 constexpr int NST = 4;       // K / V^T stages
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps + 64;  // + two epilogue-data producer warps
-constexpr int kEWarp = 2 + kEpiWarps;               // the first of them (tiles of parity 0)
+constexpr int kThreads = 64 + 32 * kEpiWarps + 96;  // + two epilogue-data producers, value loader
+constexpr int kEWarp = 2 + kEpiWarps;               // first epilogue-data producer (parity 0)
+constexpr int kVWarp = kEWarp + 2;                  // value-tile TMA producer
 constexpr int kSlots = 8;    // query clusters per CTA whose tilt weights are staged
 constexpr int kTileSegs = 8; // key clusters packed into one tile at most
 constexpr int kMixed = 0xFE; // chunk code: more than one key cluster among the valid columns
+constexpr int kPBuf = 3;     // P buffers (tile t uses t % 3): P(t) waits only for O += P(t-3) V
 
 // Widest key tile: 128 keys when D = Dv = 64, else 64 (shared memory budget).
 template <int D, int DV>
@@ -62,10 +65,11 @@ struct __align__(1024) Smem {
   unsigned char seg[NST][BN];                  // column -> cluster of the tile (0xFF: masked)
   int chunk[NST][BN / 16];                     // per 16 columns: valid mask << 8 | cluster (or kMixed)
   int koff[kMaxClusters + 1];                  // the instance's key-cluster offsets
+  int tnpad[4];                                // padded width of the tiles in flight (MMA issuer)
   // per stage: key tile (consumed by the first MMA), values (second MMA), epilogue
   // data (tilt weights, coefficients, segment map; consumed by the epilogue)
   uint64_t fullk[NST], emptyk[NST], fullv[NST], emptyv[NST], fulle[NST], emptye[NST];
-  uint64_t sfull[2], sfree[2], pready[2], pfree[2], qbar, obar;
+  uint64_t sfull[2], sfree[2], pready[kPBuf], pfree[kPBuf], qbar, obar;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -192,6 +196,8 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.sfull[i], 1);
       mbar_init(&sm.sfree[i], kEpiWarps / 2);   // one warp group per buffer
+    }
+    for (int i = 0; i < kPBuf; ++i) {
       mbar_init(&sm.pready[i], kEpiWarps / 2);
       mbar_init(&sm.pfree[i], 1);
     }
@@ -212,7 +218,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t tmem_o = tmem + 3 * BN;
+  const uint32_t tmem_o = tmem + 2 * BN + kPBuf * (BN / 2);
   auto s_col = [](int buf) { return (uint32_t)(buf * BN); };
   auto p_col = [](int buf) { return (uint32_t)(2 * BN + buf * (BN / 2)); };
   const int32_t *koff = sm.koff;
@@ -224,12 +230,19 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   const int i_first = q_cluster[q.lab + r0];  // query clusters i_first.. get staged weights
   const int nslots = min(kSlots, q_cluster[q.lab + min(r0 + BM, q.n) - 1] - i_first + 1);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == kVWarp) {
+    // ------------------------------------------------------------ TMA producers
+    // warp 0: residual tile and key tiles; warp kVWarp: value tiles.  A stage is
+    // refilled once the MMA that read it has completed; the key tiles run ahead of
+    // the value tiles, whose stages free up only after the second contraction.
+    const bool keys = warp == 0;
     if (lane == 0) {
-      mbar_expect_tx(&sm.qbar, (uint32_t)(D / 64) * BM * 128);
-      for (int kb = 0; kb < D / 64; ++kb) tma_load_2d(sm.q[kb], &map_q, kb * 64, (int)(q.lab + r0), &sm.qbar);
-      // K(t) then V(t); a stage is refilled once the MMA that read it has completed
+      if (keys) {
+        mbar_expect_tx(&sm.qbar, (uint32_t)(D / 64) * BM * 128);
+        for (int kb = 0; kb < D / 64; ++kb) tma_load_2d(sm.q[kb], &map_q, kb * 64, (int)(q.lab + r0), &sm.qbar);
+      }
+      uint64_t *full = keys ? sm.fullk : sm.fullv;
+      uint64_t *empty = keys ? sm.emptyk : sm.emptyv;
       TileIter<BN, CHUNK> it;
       it.begin(koff, k.C);
       int t = 0;
@@ -237,27 +250,23 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const KTile kt = it.get();
         const int st = t % NST;
         const int nbox = kt.npad > 64 ? 2 : 1;
-        if (t >= NST && !mbar_wait(&sm.emptyk[st], ((t / NST) - 1) & 1, abort_flag, status)) break;
-        mbar_expect_tx(&sm.fullk[st], (uint32_t)nbox * (D / 64) * 64 * 128);
-        for (int rb = 0; rb < nbox; ++rb)
-          for (int kb = 0; kb < D / 64; ++kb)
-            tma_load_2d(sm.k[st][kb] + rb * 64 * 64, &map_k, kb * 64, (int)(k.lab + kt.x0 + rb * 64),
-                        &sm.fullk[st]);
-        if (t >= NST && !mbar_wait(&sm.emptyv[st], ((t / NST) - 1) & 1, abort_flag, status)) {
-          mbar_drain(&sm.fullk[st], (t / NST) & 1, status);  // K(t) is in flight
-          break;
+        if (t >= NST && !mbar_wait(&empty[st], ((t / NST) - 1) & 1, abort_flag, status)) break;
+        if (keys) {
+          mbar_expect_tx(&full[st], (uint32_t)nbox * (D / 64) * 64 * 128);
+          for (int rb = 0; rb < nbox; ++rb)
+            for (int kb = 0; kb < D / 64; ++kb)
+              tma_load_2d(sm.k[st][kb] + rb * 64 * 64, &map_k, kb * 64, (int)(k.lab + kt.x0 + rb * 64),
+                          &full[st]);
+        } else {
+          mbar_expect_tx(&full[st], (uint32_t)nbox * DV * 128);
+          for (int rb = 0; rb < nbox; ++rb)
+            tma_load_2d(sm.vt[st][rb], &map_vt, kcol0 + kt.x0 + rb * 64, p * DV, &full[st]);
         }
-        mbar_expect_tx(&sm.fullv[st], (uint32_t)nbox * DV * 128);
-        for (int rb = 0; rb < nbox; ++rb)
-          tma_load_2d(sm.vt[st][rb], &map_vt, kcol0 + kt.x0 + rb * 64, p * DV, &sm.fullv[st]);
       }
       // copies still in flight land before the CTA may exit
-      for (int u = max(0, t - NST); u < t; ++u) {
-        mbar_drain(&sm.fullk[u % NST], (u / NST) & 1, status);
-        mbar_drain(&sm.fullv[u % NST], (u / NST) & 1, status);
-      }
+      for (int u = max(0, t - NST); u < t; ++u) mbar_drain(&full[u % NST], (u / NST) & 1, status);
     }
-  } else if (warp >= kEWarp) {
+  } else if (warp >= kEWarp && warp < kVWarp) {
     // ------------------------------------------------------------ epilogue-data producers
     // warp kEWarp + par stages the tiles of parity par (stages par, par + 2, ...)
     const int par = warp - kEWarp;
@@ -329,52 +338,75 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         if ((u & 1) == par) mbar_drain(&sm.fulle[u % NST], (u / NST) & 1, status);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Fixed order S(0), S(1), then for every tile t: S(t+2) (its S buffer is released
-    // by the group reading S(t) before that group publishes P(t)), then O += P(t) V(t).
+    // Two in-order streams: S(t) = Qt . K(t)^T (needs K(t), and the S buffer of tile
+    // t-2 read by its group) and O += P(t) V(t) (needs P(t) and V(t)).  Whichever is
+    // ready is issued, the first contraction first, so that neither epilogue group
+    // waits behind the other.
     if (lane == 0) {
       bool ok = mbar_wait(&sm.qbar, 0, abort_flag, status);
       tc_fence_after();
       TileIter<BN, CHUNK> it;
       it.begin(koff, k.C);
-      int g1 = 0;  // next tile of the first contraction
-      int npad_ring[4];
-      auto gemm1 = [&]() {
-        const int st = g1 % NST, buf = g1 & 1;
-        if (g1 >= 2 && !mbar_wait(&sm.sfree[buf], ((g1 - 2) >> 1) & 1, abort_flag, status)) return false;
-        if (!mbar_wait(&sm.fullk[st], (g1 / NST) & 1, abort_flag, status)) return false;
-        tc_fence_after();
-        const KTile kt = it.get();
-        const uint32_t id = idesc(BM, kt.npad);
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sdesc(sm.q[kk >> 2] + (kk & 3) * 16);
-          const uint64_t b = sdesc(sm.k[st][kk >> 2] + (kk & 3) * 16);
-          tc_mma(tmem + s_col(buf), a, b, id, kk > 0 ? 1u : 0u);
+      int g1 = 0, g2 = 0;  // next tile of each contraction
+      int idle = 0;
+      uint64_t t_idle = 0;
+      while (ok && (!it.done() || g2 < g1)) {
+        bool progressed = false;
+        if (!it.done()) {
+          const int st = g1 % NST, buf = g1 & 1;
+          if ((g1 < 2 || mbar_test(&sm.sfree[buf], ((g1 - 2) >> 1) & 1)) &&
+              mbar_test(&sm.fullk[st], (g1 / NST) & 1)) {
+            tc_fence_after();
+            const KTile kt = it.get();
+            const uint32_t id = idesc(BM, kt.npad);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t a = sdesc(sm.q[kk >> 2] + (kk & 3) * 16);
+              const uint64_t b = sdesc(sm.k[st][kk >> 2] + (kk & 3) * 16);
+              tc_mma(tmem + s_col(buf), a, b, id, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&sm.sfull[buf]);
+            tc_commit(&sm.emptyk[st]);  // the key tile is consumed
+            sm.tnpad[g1 & 3] = kt.npad;
+            ++g1;
+            it.next();
+            progressed = true;
+          }
         }
-        tc_commit(&sm.sfull[buf]);
-        tc_commit(&sm.emptyk[st]);  // the key tile is consumed
-        npad_ring[g1 & 3] = kt.npad;
-        ++g1;
-        it.next();
-        return true;
-      };
-      for (int w = 0; ok && w < 2 && !it.done(); ++w) ok = gemm1();
-      for (int g2 = 0; ok && g2 < g1; ++g2) {
-        if (!it.done() && !(ok = gemm1())) break;
-        const int st = g2 % NST, buf = g2 & 1;
-        if (!mbar_wait(&sm.pready[buf], (g2 >> 1) & 1, abort_flag, status) ||
-            !mbar_wait(&sm.fullv[st], (g2 / NST) & 1, abort_flag, status)) {
-          ok = false;
-          break;
+        if (g2 < g1) {
+          const int st = g2 % NST, pb = g2 % kPBuf;
+          if (mbar_test(&sm.pready[pb], (g2 / kPBuf) & 1) && mbar_test(&sm.fullv[st], (g2 / NST) & 1)) {
+            tc_fence_after();
+            const uint32_t id = idesc(BM, DV);
+            const int npad = sm.tnpad[g2 & 3];
+            for (int kk = 0; kk < npad / 16; ++kk) {
+              const uint64_t b = sdesc(sm.vt[st][kk >> 2] + (kk & 3) * 16);
+              tc_mma_ts(tmem_o, tmem + p_col(pb) + kk * 8, b, id, (g2 > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&sm.pfree[pb]);
+            tc_commit(&sm.emptyv[st]);
+            ++g2;
+            progressed = true;
+          }
         }
-        tc_fence_after();
-        const uint32_t id = idesc(BM, DV);
-        const int npad = npad_ring[g2 & 3];
-        for (int kk = 0; kk < npad / 16; ++kk) {
-          const uint64_t b = sdesc(sm.vt[st][kk >> 2] + (kk & 3) * 16);
-          tc_mma_ts(tmem_o, tmem + p_col(buf) + kk * 8, b, id, (g2 > 0 || kk > 0) ? 1u : 0u);
+        if (progressed) {
+          idle = 0;
+          continue;
         }
-        tc_commit(&sm.pfree[buf]);
-        tc_commit(&sm.emptyv[st]);
+        // nothing ready: poll again, within the same time limit as every other wait
+        if ((++idle & 255) == 0) {
+          if (*abort_flag) {
+            ok = false;
+          } else {
+            const uint64_t now = now_ns();
+            if (idle == 256) {
+              t_idle = now;
+            } else if (now - t_idle > kTimeoutNs) {
+              *abort_flag = 1;
+              report(status, MUSE_ERR_TIMEOUT);
+              ok = false;
+            }
+          }
+        }
       }
       tc_commit(&sm.obar);  // also tracks every MMA issued, on the abort path too
       mbar_drain(&sm.obar, 0, status);
@@ -410,76 +442,87 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       tc_fence_after();
       const float *wsm = &sm.w[st][staged ? slot : 0][0];
       const int nch16 = kt.npad / 16;
-      for (int cb0 = 0; cb0 < nch16; cb0 += 2) {
-        const bool two = cb0 + 1 < nch16;  // uniform
-        uint32_t xr[2][16];
-        tmem_ld16_async(tmem + lane_base + s_col(buf) + cb0 * 16, xr[0]);
-        if (two) tmem_ld16_async(tmem + lane_base + s_col(buf) + (cb0 + 1) * 16, xr[1]);
+      const int pb = t % kPBuf;
+      // P(t) overwrites P(t-3): wait until the MMA reading that has completed
+      if (t >= kPBuf &&
+          !__all_sync(0xffffffffu, mbar_wait(&sm.pfree[pb], ((t / kPBuf) - 1) & 1, abort_flag, status))) {
+        ok = false;
+        break;
+      }
+      // P for 16 columns of S held in x, stored as 8 packed bf16 columns of buffer pb
+      auto chunk = [&](int cb, const uint32_t(&x)[16]) {
+        const int code = sm.chunk[st][cb];
+        uint32_t pk[8];
+        if (wfast && (code & 0xFF) != kMixed) {
+          // one key cluster over the chunk's valid columns (common case)
+          const int g = code & 0xFF;
+          const uint32_t msk = (uint32_t)code >> 8;
+          const float b0 = sm.c0[st][g][r], b1 = sm.c1[st][g][r];
+          float w[16];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 v4 = *reinterpret_cast<const float4 *>(wsm + cb * 16 + 4 * u);
+            w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
+          }
+          float pv[16];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float t0, t1;
+            fma2(t0, t1, b1, b1, __uint_as_float(x[e]), __uint_as_float(x[e + 1]), b0, b0);
+            mul2(pv[e], pv[e + 1], w[e], w[e + 1], t0, t1);
+          }
+          if (msk != 0xFFFFu) {
+            // columns outside the tile's keys: their S may come from unrelated rows
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pv[e] = ((msk >> e) & 1u) ? pv[e] : 0.f;
+          }
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(pv[e], pv[e + 1]);
+            pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
+          }
+        } else {
+          F16 xv;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) xv.v[e] = __uint_as_float(x[e]);
+          const P8 pr = mixed_chunk<D, DV>(sm, st, cb, r, staged ? wsm : wrow + kt.x0, xv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pk[e] = pr.v[e];
+        }
+        tmem_st8(tmem + lane_base + p_col(pb) + cb * 8, pk);
+      };
+      // S chunks alternate between two register sets: the load of chunk cb+1 is in
+      // flight while chunk cb is processed
+      uint32_t xa[16], xb[16];
+      int nl = 1;  // chunks whose load has been issued
+      bool freed = false;
+      auto landed = [&]() {
         tmem_ld_wait();
-        if (cb0 + 2 >= nch16) {
+        if (!freed && nl == nch16) {
           // all of S read: its buffer can take the group's next tile while P is written
+          freed = true;
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.sfree[buf]);
         }
-        // P(t) overwrites P(t-2): wait until the MMA reading that has completed
-        if (cb0 == 0 && t >= 2 &&
-            !__all_sync(0xffffffffu, mbar_wait(&sm.pfree[buf], ((t - 2) >> 1) & 1, abort_flag, status))) {
-          ok = false;
-          break;
-        }
-#pragma unroll
-        for (int qi = 0; qi < 2; ++qi) {
-          if (qi == 1 && !two) break;
-          const int cb = cb0 + qi;
-          const int code = sm.chunk[st][cb];
-          uint32_t pk[8];
-          if (wfast && (code & 0xFF) != kMixed) {
-            // one key cluster over the chunk's valid columns (common case)
-            const int g = code & 0xFF;
-            const uint32_t msk = (uint32_t)code >> 8;
-            const float b0 = sm.c0[st][g][r], b1 = sm.c1[st][g][r];
-            float w[16];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float4 v4 = *reinterpret_cast<const float4 *>(wsm + cb * 16 + 4 * u);
-              w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
-            }
-            float pv[16];
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              float t0, t1;
-              fma2(t0, t1, b1, b1, __uint_as_float(xr[qi][e]), __uint_as_float(xr[qi][e + 1]), b0, b0);
-              mul2(pv[e], pv[e + 1], w[e], w[e + 1], t0, t1);
-            }
-            if (msk != 0xFFFFu) {
-              // columns outside the tile's keys: their S may come from unrelated rows
-#pragma unroll
-              for (int e = 0; e < 16; ++e) pv[e] = ((msk >> e) & 1u) ? pv[e] : 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              __nv_bfloat162 h = __floats2bfloat162_rn(pv[e], pv[e + 1]);
-              pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
-            }
-          } else {
-            F16 xv;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) xv.v[e] = __uint_as_float(xr[qi][e]);
-            const P8 pr = mixed_chunk<D, DV>(sm, st, cb, r, staged ? wsm : wrow + kt.x0, xv);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) pk[e] = pr.v[e];
-          }
-          // 16 bf16 of row r = 8 packed TMEM columns of the P buffer
-          tmem_st8(tmem + lane_base + p_col(buf) + cb * 8, pk);
-        }
+      };
+      tmem_ld16_async(tmem + lane_base + s_col(buf), xa);
+      landed();
+      for (int cb = 0; cb < nch16; cb += 2) {
+        if (nl < nch16) tmem_ld16_async(tmem + lane_base + s_col(buf) + (nl++) * 16, xb);
+        chunk(cb, xa);
+        landed();
+        if (cb + 1 >= nch16) break;
+        if (nl < nch16) tmem_ld16_async(tmem + lane_base + s_col(buf) + (nl++) * 16, xa);
+        chunk(cb + 1, xb);
+        landed();
       }
       if (!ok) break;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sm.pready[buf]);
+        mbar_arrive(&sm.pready[pb]);
         mbar_arrive(&sm.emptye[st]);  // the tile's epilogue data is consumed
       }
     }

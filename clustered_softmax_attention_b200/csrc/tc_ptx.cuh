@@ -37,6 +37,9 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *b) {
 }
 // One bounded probe of the phase: the warp may sleep (up to 50 us) until it completes,
 // so waiting roles do not take issue slots from working ones.
+#ifndef MUSE_SPIN_PROBES
+#define MUSE_SPIN_PROBES 0
+#endif
 #ifndef MUSE_WAIT_MODE
 #define MUSE_WAIT_MODE 1
 #endif
@@ -85,6 +88,11 @@ __device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
 // probe is inlined; the polling loop is a call, which keeps the hot loops small.
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t *b, uint32_t parity,
                                                    volatile int *abort_flag, int *status) {
+#if MUSE_SPIN_PROBES > 0
+  // short waits: poll without suspending (a suspended waiter resumes late)
+  for (int i = 0; i < MUSE_SPIN_PROBES; ++i)
+    if (mbar_test(b, parity)) return true;
+#endif
   const uint64_t t0 = now_ns();
   while (true) {
     if (mbar_try(b, parity)) return true;
