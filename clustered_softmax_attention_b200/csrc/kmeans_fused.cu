@@ -14,7 +14,8 @@
 // Each CTA streams its share of the task's 128-row tiles through shared memory (TMA,
 // 4 stages) every round and keeps the centroids in shared memory:
 //   S = X_tile . (c_hi + c_lo)^T      tcgen05.mma, M = 128 rows, N = clusters, fp32 TMEM
-//   label = argmin_c ||c||^2 - 2 S    8 epilogue warps, two column halves per row
+//   label = argmin_c ||c||^2 - 2 S    two groups of 4 epilogue warps (tiles by parity),
+//                                     a thread per row
 //   Sum += OneHot^T . X_tile          tcgen05.mma, M = 128 clusters, N = D, K = rows:
 //                                     the centroid sums as a contraction with the
 //                                     0/1 membership matrix (exact products, no atomics)
@@ -81,9 +82,7 @@ struct __align__(1024) Smem {
   int totall[CMAX];                   // group totals of every cluster
   int base[CMAX];                     // final sort: next position per cluster
   int wc[4][CMAX];                    // final sort: members per (warp, cluster) of a tile
-  float xv[2][2][TM];                 // argmin of each column half, by tile parity
-  int xi[2][2][TM];
-  uint64_t xfull[NSX], xempty[NSX], sfull[2], sfree[2], ohfull[NOH], ohempty[NOH], xch[2];
+  uint64_t xfull[NSX], xempty[NSX], sfull[2], sfree[2], ohfull[NOH], ohempty[NOH];
   uint64_t sumdone, fin;
   uint32_t tmem_base;
   int abort_flag;
@@ -220,11 +219,10 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.sfull[i], 1);
-      mbar_init(&sm.sfree[i], kEpi);
-      mbar_init(&sm.xch[i], kEpi);
+      mbar_init(&sm.sfree[i], kEpi / 2);  // one group per S buffer
     }
     for (int i = 0; i < NOH; ++i) {
-      mbar_init(&sm.ohfull[i], kEpi);
+      mbar_init(&sm.ohfull[i], kEpi / 2);
       mbar_init(&sm.ohempty[i], 1);
     }
     mbar_init(&sm.sumdone, 1);
@@ -296,114 +294,148 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
       __syncwarp();
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
+      // Two in-order streams, whichever is ready goes first: distances of tile u
+      // (needs the rows and the S buffer of tile u-2 read by its group) and the
+      // centroid sums of tile u (needs its one-hot rows).
       if (lane == 0 && nt > 0 && !*abort_flag) {
-        auto assign = [&](int u) -> bool {
-          const int st = u % NSX, buf = u & 1;
-          if (!mbar_wait(&sm.xfull[st], (u / NSX) & 1, abort_flag, status)) return false;
-          if (u >= 2 && !mbar_wait(&sm.sfree[buf], ((u - 2) >> 1) & 1, abort_flag, status)) return false;
-          tc_fence_after();
-          const uint32_t id = idesc(TM, CP);
-          for (int kk = 0; kk < D / 16; ++kk)
-            tc_mma(tmem + buf * 128, sdesc(sm.x[st] + kk * 16), sdesc(sm.hi + kk * 16), id, kk > 0 ? 1u : 0u);
-          for (int kk = 0; kk < D / 16; ++kk)
-            tc_mma(tmem + buf * 128, sdesc(sm.x[st] + kk * 16), sdesc(sm.lo + kk * 16), id, 1u);
-          tc_commit(&sm.sfull[buf]);
-          return true;
-        };
-        auto sums = [&](int u, bool first) -> bool {
-          const int st = u % NSX, ob = u % NOH;
-          if (!mbar_wait(&sm.ohfull[ob], (u / NOH) & 1, abort_flag, status)) return false;
-          tc_fence_after();
-          const uint32_t id = idesc_mn(TM, D);
-          for (int ks = 0; ks < TM / 16; ++ks)
-            tc_mma(tmem + kSumCol, sdesc_mn(sm.oh[ob][0] + ks * 16 * 64, TM * 64 * 2),
-                   sdesc_mn(sm.x[st] + ks * 16 * 64, TM * 64 * 2), id, (first && ks == 0) ? 0u : 1u);
-          tc_commit(&sm.ohempty[ob]);
-          tc_commit(&sm.xempty[st]);
-          return true;
-        };
-        bool ok = assign(u0) && (nt < 2 || assign(u0 + 1));
-        for (int t = 0; ok && t < nt; ++t) {
-          if (t + 2 < nt && !(ok = assign(u0 + t + 2))) break;
-          ok = sums(u0 + t, t == 0);
+        int a = 0, sidx = 0;  // next tile of each stream (within the round)
+        int idle = 0;
+        uint64_t t_idle = 0;
+        bool ok = true;
+        while (ok && sidx < nt) {
+          bool progressed = false;
+          if (a < nt) {
+            const int u = u0 + a, st = u % NSX, buf = u & 1;
+            if (mbar_test(&sm.xfull[st], (u / NSX) & 1) &&
+                (u < 2 || mbar_test(&sm.sfree[buf], ((u - 2) >> 1) & 1))) {
+              tc_fence_after();
+              const uint32_t id = idesc(TM, CP);
+              for (int kk = 0; kk < D / 16; ++kk)
+                tc_mma(tmem + buf * 128, sdesc(sm.x[st] + kk * 16), sdesc(sm.hi + kk * 16), id, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < D / 16; ++kk)
+                tc_mma(tmem + buf * 128, sdesc(sm.x[st] + kk * 16), sdesc(sm.lo + kk * 16), id, 1u);
+              tc_commit(&sm.sfull[buf]);
+              ++a;
+              progressed = true;
+            }
+          }
+          if (sidx < a) {
+            const int u = u0 + sidx, st = u % NSX, ob = u % NOH;
+            if (mbar_test(&sm.ohfull[ob], (u / NOH) & 1)) {
+              tc_fence_after();
+              const uint32_t id = idesc_mn(TM, D);
+              for (int ks = 0; ks < TM / 16; ++ks)
+                tc_mma(tmem + kSumCol, sdesc_mn(sm.oh[ob][0] + ks * 16 * 64, TM * 64 * 2),
+                       sdesc_mn(sm.x[st] + ks * 16 * 64, TM * 64 * 2), id, (sidx == 0 && ks == 0) ? 0u : 1u);
+              tc_commit(&sm.ohempty[ob]);
+              tc_commit(&sm.xempty[st]);
+              ++sidx;
+              progressed = true;
+            }
+          }
+          if (progressed) {
+            idle = 0;
+            continue;
+          }
+          if ((++idle & 255) == 0) {  // the same time limit as every other wait
+            if (*abort_flag) {
+              ok = false;
+            } else {
+              const uint64_t now = now_ns();
+              if (idle == 256) {
+                t_idle = now;
+              } else if (now - t_idle > kTimeoutNs) {
+                *abort_flag = 1;
+                report(status, MUSE_ERR_TIMEOUT);
+                ok = false;
+              }
+            }
+          }
         }
         tc_commit(&sm.sumdone);  // tracks every MMA issued this round, on the abort path too
       }
       __syncwarp();
     } else {
       // ------------------------------------------------------------ epilogue
-      const int half = (warp - 2) >> 2, quad = warp & 3;
+      // Two groups of four warps take the tiles of parity 0 and 1; a thread owns one
+      // row (TMEM lane) and scans all CP distance columns.
+      const int grp = (warp - 2) >> 2, quad = warp & 3;
       const int rr = quad * 32 + lane;
       const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-      const int hc = CP >> 1;  // columns of this half
-      const int col0 = half * hc;
       for (int t = 0; t < nt; ++t) {
-        const int u = u0 + t, buf = u & 1, ob = u % NOH, xb = u & 1;
+        const int u = u0 + t, buf = u & 1, ob = u % NOH;
+        if (buf != grp) continue;
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.sfull[buf], (u >> 1) & 1, abort_flag, status))) break;
         tc_fence_after();
-        uint32_t raw[4][16];
+        // 16-column chunks in batches of four, one chain per chunk; chains and
+        // batches are merged in column order (strict <: the lowest index wins a tie)
+        float bv = CUDART_INF_F;
+        int bc = 0;
+        for (int c0 = 0; c0 < CP; c0 += 64) {
+          uint32_t raw[4][16];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-          if (ch * 16 < hc) tmem_ld16_async(tmem + lane_base + buf * 128 + col0 + ch * 16, raw[ch]);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.sfree[buf]);
-        // four independent chains (one per 16-column chunk), merged in column order
-        float best[4];
-        int bi[4];
+          for (int ch = 0; ch < 4; ++ch)
+            if (c0 + ch * 16 < CP) tmem_ld16_async(tmem + lane_base + buf * 128 + c0 + ch * 16, raw[ch]);
+          tmem_ld_wait();
+          if (c0 + 64 >= CP) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.sfree[buf]);
+          }
+          float best[4];
+          int bi[4];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          best[ch] = CUDART_INF_F;
-          bi[ch] = col0;
-          if (ch * 16 < hc) {
+          for (int ch = 0; ch < 4; ++ch) {
+            best[ch] = CUDART_INF_F;
+            bi[ch] = 0;
+            if (c0 + ch * 16 < CP) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c = col0 + ch * 16 + e;
-              const float dd = fmaf(-2.f, __uint_as_float(raw[ch][e]), sm.cn[c]);
-              if (dd < best[ch]) {  // strict: the lowest index wins a tie
-                best[ch] = dd;
-                bi[ch] = c;
+              for (int e4 = 0; e4 < 4; ++e4) {
+                const float4 n4 = *reinterpret_cast<const float4 *>(&sm.cn[c0 + ch * 16 + 4 * e4]);
+                const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float dd = fmaf(-2.f, __uint_as_float(raw[ch][4 * e4 + e]), nn[e]);
+                  if (dd < best[ch]) {
+                    best[ch] = dd;
+                    bi[ch] = c0 + ch * 16 + 4 * e4 + e;
+                  }
+                }
               }
             }
           }
-        }
-        float bv = best[0];
-        int bc = bi[0];
 #pragma unroll
-        for (int ch = 1; ch < 4; ++ch)
-          if (best[ch] < bv) {
-            bv = best[ch];
-            bc = bi[ch];
-          }
-        sm.xv[xb][half][rr] = bv;
-        sm.xi[xb][half][rr] = bc;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.xch[xb]);
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.xch[xb], (u >> 1) & 1, abort_flag, status))) break;
-        const float v0 = sm.xv[xb][0][rr], v1 = sm.xv[xb][1][rr];
+          for (int ch = 0; ch < 4; ++ch)
+            if (best[ch] < bv) {
+              bv = best[ch];
+              bc = bi[ch];
+            }
+        }
         const int row = (t0 + t) * TM + rr;
         const bool valid = row < tk.n;
-        const int L = !valid ? -1 : min(v1 < v0 ? sm.xi[xb][1][rr] : sm.xi[xb][0][rr], C - 1);
-        if (valid && half == 0) {
+        const int L = valid ? min(bc, C - 1) : -1;
+        if (valid) {
           atomicAdd(&sm.cnt[L], 1);  // integer: exact in any order
           if (last) J.out.labels[tk.lab + row] = L;
         }
-        // this row's 64 one-hot entries of block `half` (bf16 1.0 = 0x3F80)
+        // this row's one-hot entries (bf16 1.0 = 0x3F80), both 64-cluster blocks
         if (u >= NOH &&
             !__all_sync(0xffffffffu, mbar_wait(&sm.ohempty[ob], ((u / NOH) - 1) & 1, abort_flag, status)))
           break;
-        unsigned char *dst = reinterpret_cast<unsigned char *>(sm.oh[ob][half]) + rr * 128;
-        const int lc = L - half * 64;
-        const bool hit = lc >= 0 && lc < 64;
-        const uint32_t one = (lc & 1) ? 0x3F800000u : 0x00003F80u;
+        const uint32_t one = (L & 1) ? 0x3F800000u : 0x00003F80u;
+        const int w = (L & 7) >> 1;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const bool here = hit && (lc >> 3) == j;
-          const int w = (lc & 7) >> 1;
-          const uint4 val = make_uint4(here && w == 0 ? one : 0u, here && w == 1 ? one : 0u,
-                                       here && w == 2 ? one : 0u, here && w == 3 ? one : 0u);
-          *reinterpret_cast<uint4 *>(dst + ((j ^ (rr & 7)) << 4)) = val;
+        for (int half = 0; half < 2; ++half) {
+          unsigned char *dst = reinterpret_cast<unsigned char *>(sm.oh[ob][half]) + rr * 128;
+          const int lc = L - half * 64;
+          const bool hit = lc >= 0 && lc < 64;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const bool here = hit && (lc >> 3) == j;
+            const uint4 val = make_uint4(here && w == 0 ? one : 0u, here && w == 1 ? one : 0u,
+                                         here && w == 2 ? one : 0u, here && w == 3 ? one : 0u);
+            *reinterpret_cast<uint4 *>(dst + ((j ^ (rr & 7)) << 4)) = val;
+          }
         }
         fence_async_smem();
         __syncwarp();
@@ -599,10 +631,10 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
 }
 
 // ------------------------------------------------------------------ host side
-// CTAs of a task's group: enough for about TPC row tiles each, a power of two <= 8.
-static int group_size(int n) {
+// CTAs of a task's group: enough for about tpc row tiles each, a power of two <= 8.
+static int group_size(int n, int tpc = TPC) {
   const int tiles = (n + TM - 1) / TM;
-  const int want = (tiles + TPC - 1) / TPC;
+  const int want = (tiles + tpc - 1) / tpc;
   int g = 1;
   while (g < want && g < GMAX) g <<= 1;
   return g;
@@ -611,15 +643,15 @@ static int group_size(int n) {
 // Lays the segments of one problem out in CTA slots, largest groups first, so every
 // group starts at a multiple of its size and never straddles a cluster of 8.  Returns
 // the largest group.
-static int plan_job(Job &J, const SegTable &t) {
+static int plan_job(Job &J, const SegTable &t, int tpc) {
   std::vector<int> order(t.nseg);
   for (int s = 0; s < t.nseg; ++s) order[s] = s;
   std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
-    return group_size(t.nrow[a]) > group_size(t.nrow[b]);
+    return group_size(t.nrow[a], tpc) > group_size(t.nrow[b], tpc);
   });
   int pos = 0, gmax = 1;
   for (int e = 0; e < t.nseg; ++e) {
-    const int s = order[e], g = group_size(t.nrow[s]);
+    const int s = order[e], g = group_size(t.nrow[s], tpc);
     J.ent[e].seg = (uint8_t)s;
     J.ent[e].g = (uint8_t)g;
     J.ent[e].pos = (uint16_t)pos;
@@ -633,28 +665,32 @@ static int plan_job(Job &J, const SegTable &t) {
 
 }  // namespace kmf
 
+// CTAs of the fused kernel that can be resident at once (0: not even one cluster fits).
+static int kmf_capacity() {
+  static int cap = -1;
+  if (cap < 0) {
+    const size_t smem = sizeof(kmf::Smem) + 1024;
+    int n = 0;
+    if (cudaFuncSetAttribute(kmf::km_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(kmf::GMAX);
+      cfg.blockDim = dim3(kmf::kThreads);
+      cfg.dynamicSmemBytes = smem;
+      if (cudaOccupancyMaxActiveClusters(&n, kmf::km_fused, &cfg) != cudaSuccess) n = 0;
+    }
+    if (n <= 0) cudaGetLastError();  // the multi-launch path takes over; leave no error behind
+    cap = n * kmf::GMAX;
+  }
+  return cap;
+}
+
 bool kmeans_fused_supported(int dtype, int D, const SegTable &t) {
   if (dtype != MUSE_BF16 || D != kmf::D || t.max_C > kmf::CMAX || t.nseg > 255) return false;
   int span = 0;
   for (int s = 0; s < t.nseg; ++s) span += kmf::group_size(t.nrow[s]);
   if (span > 65535) return false;
-  // one 8-CTA cluster of this kernel must fit on the device
-  static int fits = -1;
-  if (fits < 0) {
-    const size_t smem = sizeof(kmf::Smem) + 1024;
-    fits = cudaFuncSetAttribute(kmf::km_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
-           cudaSuccess;
-    if (fits) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(kmf::GMAX);
-      cfg.blockDim = dim3(kmf::kThreads);
-      cfg.dynamicSmemBytes = smem;
-      int n = 0;
-      fits = cudaOccupancyMaxActiveClusters(&n, kmf::km_fused, &cfg) == cudaSuccess && n > 0;
-    }
-    if (!fits) cudaGetLastError();  // the old path takes over; leave no error behind
-  }
-  return fits == 1;
+  return kmf_capacity() > 0;
 }
 
 cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *const *tabs,
@@ -666,18 +702,37 @@ cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *co
   prm.P = P;
   prm.N = N;
   prm.iters = iters;
-  int cursor = 0;
-  for (int j = 0; j < njobs; ++j) {
-    Job &J = prm.job[j];
-    J.X = X[j];
-    J.tab = *tabs[j];
-    J.out = outs[j];
-    const int gmax = plan_job(J, *tabs[j]);
-    cursor = (cursor + gmax - 1) / gmax * gmax;
-    J.base = cursor;
-    cursor += P * J.span;
+  // group sizes: about TPC row tiles per CTA, or more (smaller groups) when that lets
+  // every CTA of the launch be resident at once
+  const int cap = kmf_capacity();
+  int grid = 0;
+  for (int tpc = TPC; tpc <= 8 * TPC; tpc *= 2) {
+    int cursor = 0;
+    for (int j = 0; j < njobs; ++j) {
+      Job &J = prm.job[j];
+      J.X = X[j];
+      J.tab = *tabs[j];
+      J.out = outs[j];
+      const int gmax = plan_job(J, *tabs[j], tpc);
+      cursor = (cursor + gmax - 1) / gmax * gmax;
+      J.base = cursor;
+      cursor += P * J.span;
+    }
+    const int g = (cursor + GMAX - 1) / GMAX * GMAX;
+    if (tpc == TPC || g <= cap) grid = g;
+    if (g <= cap) break;
+    if (tpc == 8 * TPC) {  // nothing fits in one wave: back to the default group sizes
+      cursor = 0;
+      for (int j = 0; j < njobs; ++j) {
+        Job &J = prm.job[j];
+        const int gmax = plan_job(J, *tabs[j], TPC);
+        cursor = (cursor + gmax - 1) / gmax * gmax;
+        J.base = cursor;
+        cursor += P * J.span;
+      }
+      grid = (cursor + GMAX - 1) / GMAX * GMAX;
+    }
   }
-  const int grid = (cursor + GMAX - 1) / GMAX * GMAX;
   CUtensorMap m0, m1;
   if (!ptx::make_map(&m0, X[0], D, (uint64_t)P * N, D, TM) ||
       !ptx::make_map(&m1, X[njobs > 1 ? 1 : 0], D, (uint64_t)P * N, D, TM))

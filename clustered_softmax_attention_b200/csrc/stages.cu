@@ -353,6 +353,138 @@ refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
 }
 
 // ---------------------------------------------------------------------------
+// The same coefficients as a register-tiled contraction per query cluster i:
+// U = Qt_i . mu_k,i^T (rows of cluster i against its Ck tilted key means), one
+// CTA per (query cluster, instance) looping over 64-row chunks of the cluster.
+// Thread (tq, tj): rows 4 tq .. 4 tq + 3 of the chunk and key clusters tj + 16 e;
+// the 16 threads of a row are consecutive lanes (softmax by shuffles); each thread
+// stores its 4 consecutive rows of a cluster j as one 16-byte vector.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int JPT>
+__global__ void __launch_bounds__(256)
+refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
+                    const int32_t *__restrict__ q_offsets, const float *__restrict__ logZ,
+                    const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
+                    float *__restrict__ lse) {
+  constexpr int CJ = 16 * JPT;  // key clusters per pass (all of them)
+  constexpr int MS = CJ + 1;    // padded strides: transposed writes hit distinct banks
+  constexpr int QS = 68;
+  extern __shared__ float sm[];
+  float *Ms = sm;              // [D][MS] tilted key means of cluster i (transposed)
+  float *Qs = Ms + D * MS;     // [D][QS] residual rows of the chunk (transposed)
+  float *lz = Qs + D * QS;     // [CJ]
+  const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int i = blockIdx.x;
+  if (i >= q.C) return;  // uniform
+  const int Ck = k.C;
+  const int b = q_offsets[q.off + i], e = q_offsets[q.off + i + 1];
+  if (e <= b) return;
+  const int64_t zrow = (int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck;
+  // Ms[d][j]: consecutive threads take consecutive clusters j of one 4-float group
+  for (int x = threadIdx.x; x < (D / 4) * CJ; x += 256) {
+    const int d4 = x / CJ, j = x % CJ;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < Ck) v = *reinterpret_cast<const float4 *>(mu_k + (zrow + j) * D + 4 * d4);
+    Ms[(4 * d4) * MS + j] = v.x;
+    Ms[(4 * d4 + 1) * MS + j] = v.y;
+    Ms[(4 * d4 + 2) * MS + j] = v.z;
+    Ms[(4 * d4 + 3) * MS + j] = v.w;
+  }
+  for (int j = threadIdx.x; j < CJ; j += 256) lz[j] = j < Ck ? logZ[zrow + j] : -CUDART_INF_F;
+  const int tq = threadIdx.x >> 4, tj = threadIdx.x & 15;
+  float *C0 = c0 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
+  float *C1 = c1 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
+  const int cl = w_ld(q.n);
+  // chunks start on 4-row boundaries of the coefficient arrays (16-byte stores);
+  // rows outside [b, e) belong to other clusters and are neither read nor written
+  for (int r0 = b & ~3; r0 < e; r0 += 64) {
+    __syncthreads();
+    // Qs[d][rr]: consecutive threads take consecutive rows of one 4-element group
+    for (int x = threadIdx.x; x < (D / 4) * 64; x += 256) {
+      const int d4 = x >> 6, rr = x & 63;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (r0 + rr >= b && r0 + rr < e) {
+        const T *src = qt_rows + (q.lab + r0 + rr) * D + 4 * d4;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = ld_elem(src + u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) Qs[(4 * d4 + u) * QS + rr] = v[u];
+    }
+    __syncthreads();
+    float acc[4][JPT];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int u = 0; u < JPT; ++u) acc[a][u] = 0.f;
+#pragma unroll 4
+    for (int d = 0; d < D; ++d) {
+      const float4 qv = *reinterpret_cast<const float4 *>(&Qs[d * QS + 4 * tq]);
+      float mv[JPT];
+#pragma unroll
+      for (int u = 0; u < JPT; ++u) mv[u] = Ms[d * MS + tj + 16 * u];
+#pragma unroll
+      for (int u = 0; u < JPT; ++u) {
+        acc[0][u] = fmaf(qv.x, mv[u], acc[0][u]);
+        acc[1][u] = fmaf(qv.y, mv[u], acc[1][u]);
+        acc[2][u] = fmaf(qv.z, mv[u], acc[2][u]);
+        acc[3][u] = fmaf(qv.w, mv[u], acc[3][u]);
+      }
+    }
+    // a_j = logZ_ij + s u_j; p = softmax_j(a) over the 16 lanes of each row
+    float pv[4][JPT];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      float m = -CUDART_INF_F;
+#pragma unroll
+      for (int u = 0; u < JPT; ++u) m = fmaxf(m, lz[tj + 16 * u] + scale * acc[a][u]);
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float l = 0.f;
+#pragma unroll
+      for (int u = 0; u < JPT; ++u) {
+        const float av = lz[tj + 16 * u] + scale * acc[a][u];
+        l += av > -CUDART_INF_F ? __expf(av - m) : 0.f;
+      }
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int u = 0; u < JPT; ++u) {
+        const float av = lz[tj + 16 * u] + scale * acc[a][u];
+        const float pj = av > -CUDART_INF_F ? __expf(av - m) * inv : 0.f;
+        acc[a][u] = pj * (1.f - scale * acc[a][u]);  // c0; c1 = s p is recomputed below
+        pv[a][u] = scale * pj;
+      }
+      const int n = r0 + 4 * tq + a;
+      if (tj == 0 && n >= b && n < e) lse[q.lab + n] = m + logf(l);
+    }
+    // rows n0 .. n0+3 of every cluster j this thread holds
+    const int n0 = r0 + 4 * tq;
+    const bool full = n0 >= b && n0 + 3 < e;
+#pragma unroll
+    for (int u = 0; u < JPT; ++u) {
+      const int j = tj + 16 * u;
+      if (j >= Ck) break;
+      float *d0 = C0 + (int64_t)j * cl + n0;
+      float *d1 = C1 + (int64_t)j * cl + n0;
+      if (full) {
+        *reinterpret_cast<float4 *>(d0) = make_float4(acc[0][u], acc[1][u], acc[2][u], acc[3][u]);
+        *reinterpret_cast<float4 *>(d1) = make_float4(pv[0][u], pv[1][u], pv[2][u], pv[3][u]);
+      } else {
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+          if (n0 + a >= b && n0 + a < e) {
+            d0[a] = acc[a][u];
+            d1[a] = pv[a][u];
+          }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Refinement on CUDA cores: 64 sorted queries per CTA, 4 threads per query
 // (coordinates interleaved by 4), keys staged 32 at a time.
 // ---------------------------------------------------------------------------
@@ -602,10 +734,35 @@ cudaError_t run_tilt_weights(const MuseTables &mt, int dtype, int D, int P, floa
                  : weights_t<__nv_bfloat16, 128>(mt, P, scale, q_centroids, ks, logZ, W, st);
 }
 
+template <typename T, int D, int JPT>
+static cudaError_t coeffs_tiled_t(const MuseTables &mt, int P, float scale, SortedSide qs,
+                                  const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
+  constexpr int CJ = 16 * JPT;
+  const size_t smem = ((size_t)D * (CJ + 1) + D * 68 + CJ) * sizeof(float);
+  cudaError_t err = cudaFuncSetAttribute(refine_coeffs_tiled<T, D, JPT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  refine_coeffs_tiled<T, D, JPT><<<dim3(mt.q.max_C, P * mt.in.ninst), 256, smem, st>>>(
+      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 template <typename T, int D>
 static cudaError_t coeffs_t(const MuseTables &mt, int P, float scale, SortedSide qs,
                             const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
-  (void)q_offsets;
+  // the tiled form stages each query cluster's tilted key means once, which pays off
+  // when clusters hold a few dozen rows or more on average
+  int64_t rows = 0, clusters = 0;
+  for (int si = 0; si < mt.in.ninst; ++si) {
+    rows += mt.q.nrow[si];
+    clusters += mt.q.C[si];
+  }
+  if (rows >= 32 * clusters) {
+    if (mt.k.max_C <= 64) return coeffs_tiled_t<T, D, 4>(mt, P, scale, qs, q_offsets, b, st);
+    if (mt.k.max_C <= 128) return coeffs_tiled_t<T, D, 8>(mt, P, scale, qs, q_offsets, b, st);
+    if (mt.k.max_C <= 256 && D == 64) return coeffs_tiled_t<T, D, 16>(mt, P, scale, qs, q_offsets, b, st);
+  }
   const int keep_u = mt.k.max_C <= 256 ? 1 : 0;
   const size_t smem = keep_u ? (size_t)mt.k.max_C * 128 * sizeof(float) : 0;
   cudaError_t err = cudaFuncSetAttribute(refine_coeffs<T, D>,
