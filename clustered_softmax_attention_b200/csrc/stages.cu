@@ -179,6 +179,32 @@ tilt_lse(MuseTables mt, const int32_t *__restrict__ k_offsets, float *__restrict
 }
 
 // ---------------------------------------------------------------------------
+// The same for short key clusters (a few keys each): one warp per row i, one lane
+// per key cluster j, each lane scanning its cluster's keys in order.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+tilt_lse_short(MuseTables mt, const int32_t *__restrict__ k_offsets, float *__restrict__ W,
+               float *__restrict__ logZ) {
+  const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (i >= q.C) return;
+  const int Ck = k.C;
+  float *w = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s] + (int64_t)i * w_ld(k.n);
+  float *lzr = logZ + (int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck;
+  for (int j = lane; j < Ck; j += 32) {
+    const int b = k_offsets[k.off + j], e = k_offsets[k.off + j + 1];
+    float m = -CUDART_INF_F;
+    for (int pos = b; pos < e; ++pos) m = fmaxf(m, w[pos]);
+    float l = 0.f;
+    for (int pos = b; pos < e; ++pos) l += expf(w[pos] - m);
+    const float lz = (e > b) ? m + logf(l) : -CUDART_INF_F;
+    for (int pos = b; pos < e; ++pos) w[pos] = expf(w[pos] - lz);
+    lzr[j] = lz;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // W <- exp(W - logZ[i][j(pos)]) for externally supplied log-normalisers.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
@@ -677,7 +703,15 @@ static cudaError_t summaries_t(const MuseTables &mt, int P, float scale, const f
   const int maxCq = mt.q.max_C, maxCk = mt.k.max_C, maxnk = mt.k.max_rows;
   tilt_logits<T, D><<<dim3((maxnk + 63) / 64, (maxCq + 63) / 64, tasks), 256, 0, st>>>(
       mt, scale, qcen, (const T *)ks.rows, b.W);
-  tilt_lse<<<dim3((maxCq * maxCk + 7) / 8, tasks), 256, 0, st>>>(mt, k_offsets, b.W, b.logZ);
+  int64_t keys = 0, clusters = 0;
+  for (int si = 0; si < mt.in.ninst; ++si) {
+    keys += mt.k.nrow[si];
+    clusters += mt.k.C[si];
+  }
+  if (keys <= 32 * clusters)  // a few keys per cluster: a lane per cluster
+    tilt_lse_short<<<dim3((maxCq + 7) / 8, tasks), 256, 0, st>>>(mt, k_offsets, b.W, b.logZ);
+  else
+    tilt_lse<<<dim3((maxCq * maxCk + 7) / 8, tasks), 256, 0, st>>>(mt, k_offsets, b.W, b.logZ);
   count_launches(2 + (b.mu_k != nullptr) + (b.mu_v != nullptr) + (b.cov != nullptr));
   if (b.mu_k)
     tilt_moments<T, D><<<dim3(maxCk, (maxCq + 63) / 64, tasks), 256, 0, st>>>(
