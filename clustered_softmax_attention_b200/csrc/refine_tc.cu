@@ -9,9 +9,9 @@
 //
 // One CTA = 128 consecutive sorted query rows of one instance (their residuals are
 // the A operand of the first contraction, resident in shared memory).  The CTA walks
-// the key clusters; a key tile is one cluster (chunks of at most BN-16 keys), widened
-// to an 8-key-aligned start so the transposed values can be fetched by TMA, padded to
-// a multiple of 16 columns; out-of-cluster columns are masked to zero.  With every
+// the cluster-sorted keys in windows of BN keys (8-key-aligned starts, so the
+// transposed values can be fetched by TMA); a window holds up to 8 key clusters or
+// parts of them, and columns outside it are masked to zero.  With every
 // key/value tile the producer also stages, by cp.async into the same stage, the tile's
 // tilt weights for up to 8 query clusters of the CTA and the tile's coefficients
 // c0, c1 for the CTA's 128 rows.
@@ -50,7 +50,6 @@ constexpr int kPBuf = 3;     // P buffers (tile t uses t % 3): P(t) waits only f
 template <int D, int DV>
 struct TileCfg {
   static constexpr int BN = (D == 64 && DV == 64) ? 128 : 64;
-  static constexpr int CHUNK = BN - 16;  // keys of one cluster per tile (<= 7 alignment keys in front)
 };
 
 template <int D, int DV>
@@ -106,14 +105,15 @@ static __device__ __noinline__ P8 mixed_chunk(const Smem<D, DV> &sm, int st, int
   return out;
 }
 
-// Key tiles of an instance: cluster j's keys [b, e) in chunks of CHUNK.
-// A key tile: keys [c, c+n) of the sorted keys, widened to start at x0 = c & ~7 and
-// padded to npad columns (multiple of 16).  Either a chunk of one large cluster, or
-// whole clusters j .. j+nseg-1 packed while they fit in BN columns.
+// Key tiles of an instance: windows of at most BN consecutive sorted keys [c, c+n),
+// starting 8-key aligned at x0 = c & ~7 (so the transposed values can be fetched by TMA)
+// and padded to npad columns (multiple of 16).  A window spans the key clusters
+// j .. j+nseg-1 (at most kTileSegs; it ends early at the start of cluster j+kTileSegs)
+// and may start or end inside a cluster, whose keys then fall in two tiles.
 struct KTile {
   int j, nseg, c, n, x0, npad;
 };
-template <int BN, int CHUNK>
+template <int BN>
 struct TileIter {
   const int32_t *off;
   int C;
@@ -123,42 +123,24 @@ struct TileIter {
     C = Ck;
     make(0, off[0]);
   }
-  // The tile starting at key c of cluster j (skipping clusters with no key left).
+  // The window starting at key c, which lies in cluster j or a later one.
   __device__ void make(int j, int c) {
-    while (j < C && c >= off[j + 1]) {
-      ++j;
-      if (j < C) c = off[j];
-    }
+    while (j < C && c >= off[j + 1]) ++j;
     t.j = j;
     t.c = c;
     if (j >= C) return;
     t.x0 = c & ~7;
-    const int e = off[j + 1];
-    int end;
-    if (e - c > CHUNK) {
-      end = c + CHUNK;
-      t.nseg = 1;
-    } else {
-      end = e;
-      t.nseg = 1;
-      while (j + t.nseg < C && t.nseg < kTileSegs) {
-        const int e2 = off[j + t.nseg + 1];
-        if (e2 - t.x0 > BN) break;
-        end = e2;
-        ++t.nseg;
-      }
-    }
+    int end = min(t.x0 + BN, off[C]);
+    if (j + kTileSegs < C) end = min(end, off[j + kTileSegs]);
+    int last = j;  // cluster holding key end-1
+    while (last + 1 < C && off[last + 1] < end) ++last;
+    t.nseg = last - j + 1;
     t.n = end - c;
     t.npad = ((end - t.x0) + 15) & ~15;
   }
   __device__ bool done() const { return t.j >= C; }
   __device__ KTile get() const { return t; }
-  __device__ void next() {
-    if (t.nseg == 1 && t.c + t.n < off[t.j + 1])
-      make(t.j, t.c + t.n);  // next chunk of the same cluster
-    else
-      make(t.j + t.nseg, t.j + t.nseg < C ? off[t.j + t.nseg] : 0);
-  }
+  __device__ void next() { make(t.j + t.nseg - 1, t.c + t.n); }
 };
 
 template <int D, int DV>
@@ -171,7 +153,6 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                  const float *__restrict__ lse, __nv_bfloat16 *__restrict__ O,
                  float *__restrict__ part_o, float *__restrict__ part_lse, int *status) {
   constexpr int BN = TileCfg<D, DV>::BN;
-  constexpr int CHUNK = TileCfg<D, DV>::CHUNK;
   const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
   const Task q = make_task(mt.q, p * mt.q.nseg + s);
   const Task k = make_task(mt.k, p * mt.k.nseg + s);
@@ -243,7 +224,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       }
       uint64_t *full = keys ? sm.fullk : sm.fullv;
       uint64_t *empty = keys ? sm.emptyk : sm.emptyv;
-      TileIter<BN, CHUNK> it;
+      TileIter<BN> it;
       it.begin(koff, k.C);
       int t = 0;
       for (; !it.done(); it.next(), ++t) {
@@ -270,7 +251,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     // ------------------------------------------------------------ epilogue-data producers
     // warp kEWarp + par stages the tiles of parity par (stages par, par + 2, ...)
     const int par = warp - kEWarp;
-    TileIter<BN, CHUNK> it;
+    TileIter<BN> it;
     it.begin(koff, k.C);
     int t = 0;
     for (; !it.done(); it.next(), ++t) {
@@ -345,7 +326,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     if (lane == 0) {
       bool ok = mbar_wait(&sm.qbar, 0, abort_flag, status);
       tc_fence_after();
-      TileIter<BN, CHUNK> it;
+      TileIter<BN> it;
       it.begin(koff, k.C);
       int g1 = 0, g2 = 0;  // next tile of each contraction
       int idle = 0;
@@ -424,7 +405,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const bool wfast = __all_sync(0xffffffffu, staged);  // every row of the warp has staged weights
     const float *wrow = Wi + (int64_t)i * wl;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    TileIter<BN, CHUNK> it;
+    TileIter<BN> it;
     it.begin(koff, k.C);
     int t = 0;
     bool ok = true;
