@@ -43,7 +43,7 @@ constexpr int kEWarp = 2 + kEpiWarps;               // first epilogue-data produ
 constexpr int kVWarp = kEWarp + 2;                  // value-tile TMA producer
 constexpr int kSlots = 8;    // query clusters per CTA whose tilt weights are staged
 constexpr int kTileSegs = 8; // key clusters packed into one tile at most
-constexpr int kMixed = 0xFE; // chunk code: more than one key cluster among the valid columns
+constexpr int kComplex = 1 << 13;  // chunk code flag: more than two key clusters in 16 columns
 constexpr int kPBuf = 3;     // P buffers (tile t uses t % 3): P(t) waits only for O += P(t-3) V
 
 // Widest key tile: 128 keys when D = Dv = 64, else 64 (shared memory budget).
@@ -62,7 +62,7 @@ struct __align__(1024) Smem {
   float c0[NST][kTileSegs][BM];                // coefficients of the tile's key clusters
   float c1[NST][kTileSegs][BM];
   unsigned char seg[NST][BN];                  // column -> cluster of the tile (0xFF: masked)
-  int chunk[NST][BN / 16];                     // per 16 columns: valid mask << 8 | cluster (or kMixed)
+  int chunk[NST][BN / 16];                     // per 16 columns: mask, clusters, split (or kComplex)
   int koff[kMaxClusters + 1];                  // the instance's key-cluster offsets
   int tnpad[4];                                // padded width of the tiles in flight (MMA issuer)
   // per stage: key tile (consumed by the first MMA), values (second MMA), epilogue
@@ -82,7 +82,7 @@ struct P8 {
   uint32_t v[8];
 };
 
-// P for a 16-column chunk whose valid columns belong to more than one key cluster, or
+// P for a 16-column chunk whose valid columns belong to more than two key clusters, or
 // for a warp with a row whose tilt weights are not staged: per-column cluster lookup.
 // Rare, so kept out of line (the hot loop stays small).
 template <int D, int DV>
@@ -293,21 +293,27 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         }
         sm.seg[st][col] = (unsigned char)sg;
       }
-      // per 16-column chunk: valid-column mask (a contiguous run), and the chunk's key
-      // cluster when its first and last valid columns share one (else kMixed)
+      // per 16-column chunk: valid-column mask (a contiguous run) << 16, the key
+      // clusters of its first and last valid columns (bits 0-3, 4-7) and the first
+      // column of the second one (bits 8-12; 16 for one cluster), or kComplex when
+      // more than two clusters share the chunk
       if (lane < BN / 16) {
         const int cx = kt.x0 + 16 * lane;
         const int k0 = max(kt.c, cx), k1 = min(kt.c + kt.n, cx + 16);
-        int code = 0;
+        int code = 16 << 8;  // no valid column: mask 0, P = 0
         if (16 * lane < kt.npad && k0 < k1) {
-          int s0 = 0, s1 = 0;
+          int s0 = 0, s1 = 0, split = 16;
 #pragma unroll
           for (int b = 0; b < kTileSegs - 1; ++b) {
             s0 += k0 >= bnd[b] ? 1 : 0;
             s1 += k1 - 1 >= bnd[b] ? 1 : 0;
           }
+#pragma unroll
+          for (int b = 0; b < kTileSegs - 1; ++b)
+            if (b == s0 && s1 == s0 + 1) split = bnd[b] - cx;
           const uint32_t m16 = ((1u << (k1 - cx)) - 1u) & ~((1u << (k0 - cx)) - 1u);
-          code = (int)(m16 << 8) | (s0 == s1 ? s0 : kMixed);
+          code = s1 > s0 + 1 ? kComplex : (s0 | (s1 << 4) | (split << 8));
+          code |= (int)(m16 << 16);
         }
         sm.chunk[st][lane] = code;
       }
@@ -434,11 +440,11 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       auto chunk = [&](int cb, const uint32_t(&x)[16]) {
         const int code = sm.chunk[st][cb];
         uint32_t pk[8];
-        if (wfast && (code & 0xFF) != kMixed) {
-          // one key cluster over the chunk's valid columns (common case)
-          const int g = code & 0xFF;
-          const uint32_t msk = (uint32_t)code >> 8;
-          const float b0 = sm.c0[st][g][r], b1 = sm.c1[st][g][r];
+        if (wfast && !(code & kComplex)) {
+          // at most two key clusters over the chunk's valid columns
+          const int glo = code & 15, ghi = (code >> 4) & 15, split = (code >> 8) & 31;
+          const uint32_t msk = (uint32_t)code >> 16;
+          const float b0 = sm.c0[st][glo][r], b1 = sm.c1[st][glo][r];
           float w[16];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -446,11 +452,23 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             w[4 * u] = v4.x; w[4 * u + 1] = v4.y; w[4 * u + 2] = v4.z; w[4 * u + 3] = v4.w;
           }
           float pv[16];
+          if (glo == ghi) {
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float t0, t1;
-            fma2(t0, t1, b1, b1, __uint_as_float(x[e]), __uint_as_float(x[e + 1]), b0, b0);
-            mul2(pv[e], pv[e + 1], w[e], w[e + 1], t0, t1);
+            for (int e = 0; e < 16; e += 2) {
+              float t0, t1;
+              fma2(t0, t1, b1, b1, __uint_as_float(x[e]), __uint_as_float(x[e + 1]), b0, b0);
+              mul2(pv[e], pv[e + 1], w[e], w[e + 1], t0, t1);
+            }
+          } else {
+            const float h0 = sm.c0[st][ghi][r], h1 = sm.c1[st][ghi][r];
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const bool lo0 = e < split, lo1 = e + 1 < split;
+              float t0, t1;
+              fma2(t0, t1, lo0 ? b1 : h1, lo1 ? b1 : h1, __uint_as_float(x[e]), __uint_as_float(x[e + 1]),
+                   lo0 ? b0 : h0, lo1 ? b0 : h0);
+              mul2(pv[e], pv[e + 1], w[e], w[e + 1], t0, t1);
+            }
           }
           if (msk != 0xFFFFu) {
             // columns outside the tile's keys: their S may come from unrelated rows
