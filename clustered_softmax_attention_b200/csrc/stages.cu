@@ -381,7 +381,7 @@ refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
 // ---------------------------------------------------------------------------
 // The same coefficients as a register-tiled contraction per query cluster i:
 // U = Qt_i . mu_k,i^T (rows of cluster i against its Ck tilted key means), one
-// CTA per (query cluster, instance) looping over 64-row chunks of the cluster.
+// CTA per 64-row chunk of a query cluster (the largest clusters set no tail).
 // Thread (tq, tj): rows 4 tq .. 4 tq + 3 of the chunk and key clusters tj + 16 e;
 // the 16 threads of a row are consecutive lanes (softmax by shuffles); each thread
 // stores its 4 consecutive rows of a cluster j as one 16-byte vector.
@@ -401,11 +401,46 @@ refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
   float *lz = Qs + D * QS;     // [CJ]
   const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
   const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
-  const int i = blockIdx.x;
-  if (i >= q.C) return;  // uniform
+  // this CTA's 64-row chunk: chunk g of the instance, counting ceil(rows/64) chunks
+  // per query cluster in cluster order (rows start on 4-row boundaries)
+  __shared__ int s_i, s_r0;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int run = 0, found = -1, fr0 = 0;
+    for (int c0 = 0; c0 < q.C && found < 0; c0 += 32) {
+      const int c = c0 + lane;
+      int nch = 0, bb = 0;
+      if (c < q.C) {
+        bb = q_offsets[q.off + c];
+        const int ee = q_offsets[q.off + c + 1];
+        nch = ee > bb ? (ee - (bb & ~3) + 63) / 64 : 0;
+      }
+      int inc = nch;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const int first = run + inc - nch;  // chunk index of this cluster's first chunk
+      const bool mine = (int)blockIdx.x >= first && (int)blockIdx.x < first + nch;
+      const unsigned bal = __ballot_sync(0xffffffffu, mine);
+      if (bal) {
+        const int src = __ffs(bal) - 1;
+        found = __shfl_sync(0xffffffffu, c, src);
+        fr0 = __shfl_sync(0xffffffffu, (bb & ~3) + 64 * ((int)blockIdx.x - first), src);
+      }
+      run += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) {
+      s_i = found;
+      s_r0 = fr0;
+    }
+  }
+  __syncthreads();
+  const int i = s_i;
+  if (i < 0) return;  // uniform: past the instance's last chunk
   const int Ck = k.C;
   const int b = q_offsets[q.off + i], e = q_offsets[q.off + i + 1];
-  if (e <= b) return;
   const int64_t zrow = (int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck;
   // Ms[d][j]: consecutive threads take consecutive clusters j of one 4-float group
   for (int x = threadIdx.x; x < (D / 4) * CJ; x += 256) {
@@ -424,7 +459,8 @@ refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
   const int cl = w_ld(q.n);
   // chunks start on 4-row boundaries of the coefficient arrays (16-byte stores);
   // rows outside [b, e) belong to other clusters and are neither read nor written
-  for (int r0 = b & ~3; r0 < e; r0 += 64) {
+  {
+    const int r0 = s_r0;
     __syncthreads();
     // Qs[d][rr]: consecutive threads take consecutive rows of one 4-element group
     for (int x = threadIdx.x; x < (D / 4) * 64; x += 256) {
@@ -776,7 +812,9 @@ static cudaError_t coeffs_tiled_t(const MuseTables &mt, int P, float scale, Sort
   cudaError_t err = cudaFuncSetAttribute(refine_coeffs_tiled<T, D, JPT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  refine_coeffs_tiled<T, D, JPT><<<dim3(mt.q.max_C, P * mt.in.ninst), 256, smem, st>>>(
+  // chunks of an instance: at most rows/64 + one partial chunk per cluster
+  refine_coeffs_tiled<T, D, JPT><<<dim3((mt.q.max_rows + 63) / 64 + mt.q.max_C, P * mt.in.ninst), 256,
+                                  smem, st>>>(
       mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse);
   count_launches(1);
   return cudaGetLastError();
