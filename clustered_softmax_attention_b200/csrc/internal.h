@@ -93,6 +93,12 @@ cudaError_t run_refine(const MuseTables &mt, int dtype, int D, int Dv, int N, in
                        SortedSide qs, const int32_t *q_perm, SortedSide ks, const void *vs_rows,
                        StageBufs b, void *O, float *part_o, float *part_lse, cudaStream_t st);
 size_t muse_retrieval_ws(const muse_dims &d, int block, int Cq, int Ck, int k1, int k2);
+// The exact diagonal on the tensor cores (diag_tc.cu): bf16, D = Dv = 64, block a
+// multiple of 128 and at most 512.
+bool diag_tc_supported(int dtype, int D, int Dv, int N, int block);
+cudaError_t run_diag_tc(const void *Q, const void *K, const void *V, int N, int P, int block,
+                        int levels, float scale, const float *part_o, const float *part_lse,
+                        void *O, int *status, cudaStream_t st);
 cudaError_t run_diag_merge(const void *Q, const void *K, const void *V, int dtype, int D, int Dv,
                            int N, int P, int block, int levels, float scale,
                            const float *part_o, const float *part_lse, void *O, cudaStream_t st);

@@ -887,6 +887,8 @@ static cudaError_t diag_t(const void *Q, const void *K, const void *V, int N, in
 cudaError_t run_diag_merge(const void *Q, const void *K, const void *V, int dtype, int D, int Dv,
                            int N, int P, int block, int levels, float scale,
                            const float *part_o, const float *part_lse, void *O, cudaStream_t st) {
+  if (diag_tc_supported(dtype, D, Dv, N, block))
+    return run_diag_tc(Q, K, V, N, P, block, levels, scale, part_o, part_lse, O, device_status_word(), st);
   MUSE_DISPATCH_DDV(dtype, D, Dv, diag_t, Q, K, V, N, P, block, levels, scale, part_o, part_lse,
                     O, st);
 }
