@@ -70,6 +70,33 @@ __host__ __device__ __forceinline__ Task make_task(const SegTable &t, int task) 
   return k;
 }
 
+// Blocks of `rows` consecutive rows of every segment of a table, numbered segment
+// after segment: a compact grid (no block lies past its segment's rows, which matters
+// when the segments differ in size, as the squares of the causal decomposition do).
+struct BlockMap {
+  int total;
+  int pre[kMaxSeg + 1];  // first block of segment s; pre[nseg] = total
+};
+inline BlockMap make_block_map(const SegTable &t, int rows) {
+  BlockMap m;
+  m.pre[0] = 0;
+  for (int s = 0; s < t.nseg; ++s) m.pre[s + 1] = m.pre[s] + (t.nrow[s] + rows - 1) / rows;
+  for (int s = t.nseg + 1; s <= kMaxSeg; ++s) m.pre[s] = m.pre[t.nseg];
+  m.total = m.pre[t.nseg];
+  return m;
+}
+// Segment of block b (the last segment whose first block is <= b) and its first block.
+__device__ __forceinline__ int map_block(const BlockMap &m, int nseg, int b, int &first) {
+  int lo = 0, hi = nseg - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (m.pre[mid] <= b) lo = mid;
+    else hi = mid - 1;
+  }
+  first = m.pre[lo];
+  return lo;
+}
+
 // ---------------------------------------------------------------------------
 // Device status word (MUSE_OK / MUSE_ERR_TIMEOUT / MUSE_ERR_DEVICE).  Kernels get
 // its address as a parameter; the first error wins.

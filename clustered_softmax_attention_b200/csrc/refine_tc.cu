@@ -151,12 +151,15 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                  const int32_t *__restrict__ k_offsets, const float *__restrict__ W,
                  const float *__restrict__ c0g, const float *__restrict__ c1g,
                  const float *__restrict__ lse, __nv_bfloat16 *__restrict__ O,
-                 float *__restrict__ part_o, float *__restrict__ part_lse, int *status) {
+                 float *__restrict__ part_o, float *__restrict__ part_lse, int *status,
+                 const __grid_constant__ BlockMap bm) {
   constexpr int BN = TileCfg<D, DV>::BN;
-  const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
+  // blockIdx.x: a 128-row block of one instance (compact grid), blockIdx.y: the problem
+  int bfirst;
+  const int p = blockIdx.y, s = map_block(bm, mt.in.ninst, blockIdx.x, bfirst);
   const Task q = make_task(mt.q, p * mt.q.nseg + s);
   const Task k = make_task(mt.k, p * mt.k.nseg + s);
-  const int r0 = blockIdx.x * BM;
+  const int r0 = ((int)blockIdx.x - bfirst) * BM;
   if (r0 >= q.n) return;  // uniform: nothing allocated yet
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -583,10 +586,11 @@ static cudaError_t launch(const MuseTables &mt, int N, int P, SortedSide qs, con
   cudaError_t e = cudaFuncSetAttribute(refine_tc_kernel<D, DV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((mt.q.max_rows + BM - 1) / BM, P * mt.in.ninst);
+  const BlockMap bm = make_block_map(mt.q, BM);
+  dim3 grid(bm.total, P);
   refine_tc_kernel<D, DV><<<grid, kThreads, smem, st>>>(
       mq, mk, mv, mt, N, q_perm, qs.cluster, k_offsets, b.W, b.c0, b.c1, b.lse,
-      (__nv_bfloat16 *)O, part_o, part_lse, status);
+      (__nv_bfloat16 *)O, part_o, part_lse, status, bm);
   count_launches(1);
   return cudaGetLastError();
 }

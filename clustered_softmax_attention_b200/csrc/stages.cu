@@ -67,9 +67,11 @@ sort_side(const T *__restrict__ X, int N, int W, SegTable tab, const int32_t *__
 template <typename T, int W>
 __global__ void __launch_bounds__(256)
 sort_side_t(const T *__restrict__ X, int N, SegTable tab, const int32_t *__restrict__ perm,
-            T *__restrict__ vt) {
-  const Task tk = make_task(tab, blockIdx.y);
-  const int m0 = blockIdx.x * 64;
+            T *__restrict__ vt, BlockMap bm) {
+  int bfirst;
+  const int sg = map_block(bm, tab.nseg, blockIdx.x, bfirst);
+  const Task tk = make_task(tab, blockIdx.y * tab.nseg + sg);
+  const int m0 = ((int)blockIdx.x - bfirst) * 64;
   if (m0 >= tk.n) return;
   __shared__ T buf[64][W + 2];
   const int mt = min(64, tk.n - m0);
@@ -103,11 +105,13 @@ sort_side_t(const T *__restrict__ X, int N, SegTable tab, const int32_t *__restr
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 tilt_logits(MuseTables mt, float scale, const float *__restrict__ qcen, const T *__restrict__ ks,
-            float *__restrict__ W) {
-  const int p = blockIdx.z / mt.in.ninst, s = blockIdx.z % mt.in.ninst;
+            float *__restrict__ W, BlockMap bm) {
+  // blockIdx.x: a 64-key block of one instance (compact grid), blockIdx.z: the problem
+  int bfirst;
+  const int p = blockIdx.z, s = map_block(bm, mt.in.ninst, blockIdx.x, bfirst);
   const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
   const int Cq = q.C, nk = k.n;
-  const int i0 = blockIdx.y * 64, k0 = blockIdx.x * 64;
+  const int i0 = blockIdx.y * 64, k0 = ((int)blockIdx.x - bfirst) * 64;
   if (i0 >= Cq || k0 >= nk) return;
   __shared__ float As[32][65];
   __shared__ float Bs[32][65];
@@ -323,13 +327,16 @@ __global__ void __launch_bounds__(128)
 refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
               const int32_t *__restrict__ q_cluster, const float *__restrict__ logZ,
               const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
-              float *__restrict__ lse, int keep_u) {
+              float *__restrict__ lse, int keep_u, BlockMap bm) {
   extern __shared__ float su[];  // [Ck][128] residual projections u_j (when keep_u)
-  const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
+  // blockIdx.x: a 128-row block of one instance (compact grid), blockIdx.y: the problem
+  int bfirst;
+  const int p = blockIdx.y, s = map_block(bm, mt.in.ninst, blockIdx.x, bfirst);
   const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
   const int Ck = k.C, nq = q.n;
-  const int n = blockIdx.x * 128 + threadIdx.x;
-  if (blockIdx.x * 128 >= nq) return;  // uniform
+  const int rb0 = ((int)blockIdx.x - bfirst) * 128;
+  const int n = rb0 + threadIdx.x;
+  if (rb0 >= nq) return;  // uniform
   const bool v = n < nq;
   const int i = v ? q_cluster[q.lab + n] : 0;
   float qt[D];
@@ -717,16 +724,17 @@ cudaError_t run_sort_side(const void *X, int dtype, int width, int N, const SegT
 
 cudaError_t run_sort_side_t(const void *X, int dtype, int width, int N, const SegTable &tab,
                             int P, const int32_t *perm, void *vt, cudaStream_t st) {
-  dim3 grid((tab.max_rows + 63) / 64, P * tab.nseg);
+  const BlockMap bm = make_block_map(tab, 64);
+  dim3 grid(bm.total, P);
   count_launches(1);
   if (dtype == MUSE_F32) {
-    if (width == 64) sort_side_t<float, 64><<<grid, 256, 0, st>>>((const float *)X, N, tab, perm, (float *)vt);
-    else sort_side_t<float, 128><<<grid, 256, 0, st>>>((const float *)X, N, tab, perm, (float *)vt);
+    if (width == 64) sort_side_t<float, 64><<<grid, 256, 0, st>>>((const float *)X, N, tab, perm, (float *)vt, bm);
+    else sort_side_t<float, 128><<<grid, 256, 0, st>>>((const float *)X, N, tab, perm, (float *)vt, bm);
   } else {
     if (width == 64)
-      sort_side_t<__nv_bfloat16, 64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)X, N, tab, perm, (__nv_bfloat16 *)vt);
+      sort_side_t<__nv_bfloat16, 64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)X, N, tab, perm, (__nv_bfloat16 *)vt, bm);
     else
-      sort_side_t<__nv_bfloat16, 128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)X, N, tab, perm, (__nv_bfloat16 *)vt);
+      sort_side_t<__nv_bfloat16, 128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)X, N, tab, perm, (__nv_bfloat16 *)vt, bm);
   }
   return cudaGetLastError();
 }
@@ -737,8 +745,9 @@ static cudaError_t summaries_t(const MuseTables &mt, int P, float scale, const f
                                StageBufs b, cudaStream_t st) {
   const int tasks = P * mt.in.ninst;
   const int maxCq = mt.q.max_C, maxCk = mt.k.max_C, maxnk = mt.k.max_rows;
-  tilt_logits<T, D><<<dim3((maxnk + 63) / 64, (maxCq + 63) / 64, tasks), 256, 0, st>>>(
-      mt, scale, qcen, (const T *)ks.rows, b.W);
+  const BlockMap kbm = make_block_map(mt.k, 64);
+  tilt_logits<T, D><<<dim3(kbm.total, (maxCq + 63) / 64, P), 256, 0, st>>>(
+      mt, scale, qcen, (const T *)ks.rows, b.W, kbm);
   int64_t keys = 0, clusters = 0;
   for (int si = 0; si < mt.in.ninst; ++si) {
     keys += mt.k.nrow[si];
@@ -786,8 +795,9 @@ template <typename T, int D>
 static cudaError_t weights_t(const MuseTables &mt, int P, float scale, const float *qcen,
                              SortedSide ks, const float *logZ, float *W, cudaStream_t st) {
   const int tasks = P * mt.in.ninst;
-  tilt_logits<T, D><<<dim3((mt.k.max_rows + 63) / 64, (mt.q.max_C + 63) / 64, tasks), 256, 0,
-                      st>>>(mt, scale, qcen, (const T *)ks.rows, W);
+  const BlockMap kbm = make_block_map(mt.k, 64);
+  tilt_logits<T, D><<<dim3(kbm.total, (mt.q.max_C + 63) / 64, P), 256, 0, st>>>(
+      mt, scale, qcen, (const T *)ks.rows, W, kbm);
   tilt_weights<<<dim3((mt.k.max_rows + 255) / 256, mt.q.max_C, tasks), 256, 0, st>>>(
       mt, ks.cluster, logZ, W);
   count_launches(2);
@@ -840,8 +850,9 @@ static cudaError_t coeffs_t(const MuseTables &mt, int P, float scale, SortedSide
   cudaError_t err = cudaFuncSetAttribute(refine_coeffs<T, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  refine_coeffs<T, D><<<dim3((mt.q.max_rows + 127) / 128, P * mt.in.ninst), 128, smem, st>>>(
-      mt, scale, (const T *)qs.rows, qs.cluster, b.logZ, b.mu_k, b.c0, b.c1, b.lse, keep_u);
+  const BlockMap bm = make_block_map(mt.q, 128);
+  refine_coeffs<T, D><<<dim3(bm.total, P), 128, smem, st>>>(
+      mt, scale, (const T *)qs.rows, qs.cluster, b.logZ, b.mu_k, b.c0, b.c1, b.lse, keep_u, bm);
   count_launches(1);
   return cudaGetLastError();
 }
