@@ -175,8 +175,13 @@ def causal_labels(ql, kl, N, S):
     return out
 
 
+# block sizes: 128 and 256 (several levels), 512 at N = 2048 (the tensor-core diagonal
+# with four key tiles per block), S = N/2 (a single level), and 1024 (the CUDA-core
+# diagonal, beyond the tensor-core kernel's 512)
 @pytest.mark.parametrize("dt,N,S,C", [("f32", 1024, 128, 16), ("bf16", 1024, 128, 16),
-                                       ("bf16", 1536, 256, 40)])
+                                       ("bf16", 1536, 256, 40), ("bf16", 2048, 512, 32),
+                                       ("bf16", 1024, 512, 32), ("bf16", 2048, 1024, 48),
+                                       ("f32", 2048, 512, 32)])
 def test_causal_vs_oracle(dt, N, S, C):
     Q, K, V = mixture(7, 1, 2, N, 64, 64, 16, 0.3 / 8, dt)
     Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
