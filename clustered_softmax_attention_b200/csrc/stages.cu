@@ -15,6 +15,7 @@
 //   O_n = sum_k w_{i(n),k} (c0_{n,j(k)} + c1_{n,j(k)} qt_n.k) v_k :
 // two contractions over the cluster-sorted keys with an element-wise step between
 // them, and C_ij is never formed.
+#include <type_traits>
 #include "internal.h"
 
 namespace muse {
@@ -283,6 +284,288 @@ tilt_moments(MuseTables mt, const int32_t *__restrict__ k_offsets, const float *
     float *o = mu + ((int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck + j) * WD;
 #pragma unroll
     for (int u = 0; u < PW; ++u) o[td + 16 * u] = acc[a][u];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// logits, log-normalisers, tilt weights and tilted key means in one kernel.  CTA per
+// (G consecutive key clusters, 64 query centroids, instance), G chosen per instance so
+// that a CTA covers about one chunk of keys (G = 1 for large clusters, up to 16 for
+// clusters of a few keys); the centroids are staged once for all G clusters.  A cluster
+// of at most KC keys takes one step: its logits stay in registers, give logZ by a
+// 16-lane reduction and then the weights and the tilted key mean.  A larger cluster takes
+// a first pass over chunks of KC keys (running maximum and sum) and a second pass that
+// recomputes the logits.  The next step's keys are loaded into registers while the
+// current step computes.  Thread (ti, td): centroids 4 ti .. 4 ti + 3, keys td + 16 c of
+// a chunk, coordinates 4 td + 64 h of the means (the 16 threads of a centroid are
+// consecutive lanes).
+// ---------------------------------------------------------------------------
+template <typename T, int D> struct TiltCfg {
+  static constexpr int KC = 16384 / (D * (int)sizeof(T));  // keys per chunk (16 KB)
+  static constexpr int UR = D * (int)sizeof(T) / 16;       // 16-byte units per key row
+  static constexpr int EPU = 16 / (int)sizeof(T);          // elements per unit
+  static constexpr int QS = D + 4, WS = 68;                // shared-memory row strides
+  static constexpr int GMAX = 16;
+  // centroids, keys (fp32), weights, and the raw key chunk the next step copies into
+  static constexpr size_t smem = ((size_t)64 * QS + (size_t)KC * QS + (size_t)KC * WS) * 4 + 16384;
+};
+
+// 16-byte asynchronous global -> shared copy (src_bytes = 0 writes zeros), its commit
+// and the wait for all of this thread's copies.
+__device__ __forceinline__ void tilt_cp16(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void tilt_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void tilt_cp_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// clusters per CTA for an instance of n keys in C clusters
+__host__ __device__ __forceinline__ int tilt_group(int n, int C, int kc) {
+  if (C <= 0 || n <= 0) return TiltCfg<float, 64>::GMAX;
+  const int64_t g = (int64_t)kc * C / n;
+  return (int)(g < 1 ? 1 : g > TiltCfg<float, 64>::GMAX ? TiltCfg<float, 64>::GMAX : g);
+}
+
+__device__ __forceinline__ void tilt_unpack(const uint4 u, float *o) {  // 8 bf16
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    const float2 f = __bfloat1622float2(h[x]);
+    o[2 * x] = f.x;
+    o[2 * x + 1] = f.y;
+  }
+}
+
+struct TiltStep {
+  int j, b, e, pc, pass;  // pass 0: the whole cluster in one chunk; 1, 2: first, second pass
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 2)
+tilt_fused(MuseTables mt, float scale, const float *__restrict__ qcen, const T *__restrict__ ks,
+           const int32_t *__restrict__ k_offsets, float *__restrict__ W, float *__restrict__ logZ,
+           float *__restrict__ mu, const __grid_constant__ BlockMap bm) {
+  // blockIdx.x: a group of G key clusters of one instance (compact grid), blockIdx.z: the problem
+  using Cf = TiltCfg<T, D>;
+  constexpr int KC = Cf::KC, QS = Cf::QS, WS = Cf::WS, PQ = D / 64;
+  extern __shared__ float4 tilt_smem[];
+  float *Qs = reinterpret_cast<float *>(tilt_smem);  // [64][QS] the group's centroids
+  float *Ks = Qs + 64 * QS;                           // [KC][QS] a chunk of keys
+  float *Ws = Ks + KC * QS;                           // [KC][WS] the chunk's weights
+  uint4 *Kr = reinterpret_cast<uint4 *>(Ws + KC * WS); // [1024] raw 16-byte units of a chunk
+  __shared__ int offs[Cf::GMAX + 1];
+  int bfirst;
+  const int p = blockIdx.z, s = map_block(bm, mt.in.ninst, blockIdx.x, bfirst);
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int Cq = q.C, Ck = k.C, nk = k.n;
+  const int G = tilt_group(nk, Ck, KC);
+  const int j0 = ((int)blockIdx.x - bfirst) * G, j1 = min(Ck, j0 + G), i0 = blockIdx.y * 64;
+  if (j0 >= Ck || i0 >= Cq) return;  // uniform
+  const int tid = threadIdx.x, ti = tid >> 4, td = tid & 15;
+  if (tid <= j1 - j0) offs[tid] = k_offsets[k.off + j0 + tid];
+  {
+    constexpr int QU = D / 4, NR = 64 * QU / 256;
+    float4 v[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      const int u = tid + 256 * r, ii = u / QU;
+      v[r] = i0 + ii < Cq ? __ldg(reinterpret_cast<const float4 *>(qcen + (q.cen + i0 + ii) * D) + u % QU)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      const int u = tid + 256 * r;
+      *reinterpret_cast<float4 *>(Qs + (u / QU) * QS + 4 * (u % QU)) = v[r];
+    }
+  }
+  __syncthreads();
+  float *wb = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s];
+  const int wl = w_ld(nk);
+  const int64_t zrow = (int64_t)p * mt.in.z_stride + mt.in.z0[s];
+  // outputs of cluster j: logZ and the tilted mean of each of the thread's centroids
+  auto put = [&](int j, const float (&lz)[4], const float (&acc)[4][PQ][4]) {
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int i = i0 + ti * 4 + a;
+      if (i >= Cq) continue;
+      const int64_t z = zrow + (int64_t)i * Ck + j;
+      if (td == 0) logZ[z] = lz[a];
+#pragma unroll
+      for (int h = 0; h < PQ; ++h)
+        *reinterpret_cast<float4 *>(mu + z * D + 64 * h + 4 * td) =
+            make_float4(acc[a][h][0], acc[a][h][1], acc[a][h][2], acc[a][h][3]);
+    }
+  };
+  float lz[4], m[4], l[4], acc[4][PQ][4];
+  auto clear_acc = [&]() {
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int h = 0; h < PQ; ++h)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) acc[a][h][x] = 0.f;
+  };
+  // first non-empty cluster from j on (empty clusters get logZ = -inf and a zero mean)
+  auto open = [&](int j) {
+    while (j < j1 && offs[j - j0 + 1] == offs[j - j0]) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const int i = i0 + ti * 4 + a;
+        if (i >= Cq) continue;
+        const int64_t z = zrow + (int64_t)i * Ck + j;
+        if (td == 0) logZ[z] = -CUDART_INF_F;
+#pragma unroll
+        for (int h = 0; h < PQ; ++h)
+          *reinterpret_cast<float4 *>(mu + z * D + 64 * h + 4 * td) = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      ++j;
+    }
+    TiltStep t;
+    t.j = j;
+    t.b = j < j1 ? offs[j - j0] : 0;
+    t.e = j < j1 ? offs[j - j0 + 1] : 0;
+    t.pc = t.b;
+    t.pass = t.e - t.b > KC ? 1 : 0;
+    return t;
+  };
+  auto advance = [&](TiltStep t) {
+    if (t.pc + KC < t.e) {
+      t.pc += KC;
+      return t;
+    }
+    if (t.pass == 1) {
+      t.pass = 2;
+      t.pc = t.b;
+      return t;
+    }
+    return open(t.j + 1);
+  };
+  // each thread copies, and later converts, the same four 16-byte units of a chunk
+  auto fetch = [&](const TiltStep &t) {
+    const int pt = min(KC, t.e - t.pc);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int u = tid + 256 * r, row = u / Cf::UR;
+      const bool in = row < pt;
+      tilt_cp16(Kr + u, in ? (const void *)(reinterpret_cast<const uint4 *>(ks + (k.lab + t.pc + row) * D) + u % Cf::UR)
+                           : (const void *)ks, in ? 16u : 0u);
+    }
+    tilt_cp_commit();
+  };
+  TiltStep cur = open(j0);
+  if (cur.j < j1) fetch(cur);
+  while (cur.j < j1) {
+    const int pt = min(KC, cur.e - cur.pc);
+    __syncthreads();  // the previous step is done with Ks and Ws
+    tilt_cp_wait();
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int u = tid + 256 * r;
+      float *dst = Ks + (u / Cf::UR) * QS + (u % Cf::UR) * Cf::EPU;
+      const uint4 raw = Kr[u];
+      if constexpr (sizeof(T) == 2) {
+        float f[8];
+        tilt_unpack(raw, f);
+        *reinterpret_cast<float4 *>(dst) = make_float4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<float4 *>(dst + 4) = make_float4(f[4], f[5], f[6], f[7]);
+      } else {
+        *reinterpret_cast<uint4 *>(dst) = raw;
+      }
+    }
+    const TiltStep nxt = advance(cur);
+    if (nxt.j < j1) fetch(nxt);
+    __syncthreads();
+    const bool first = cur.pc == cur.b, last = cur.pc + KC >= cur.e;
+    auto body = [&](auto ncv) {
+      constexpr int NC = decltype(ncv)::value;
+      float L[4][NC];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < NC; ++c) L[a][c] = 0.f;
+#pragma unroll 2
+      for (int d = 0; d < D; d += 4) {
+        float4 qv[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4 *>(Qs + (ti * 4 + a) * QS + d);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          const float4 kv = *reinterpret_cast<const float4 *>(Ks + (td + 16 * c) * QS + d);
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            L[a][c] = fmaf(qv[a].x, kv.x, L[a][c]);
+            L[a][c] = fmaf(qv[a].y, kv.y, L[a][c]);
+            L[a][c] = fmaf(qv[a].z, kv.z, L[a][c]);
+            L[a][c] = fmaf(qv[a].w, kv.w, L[a][c]);
+          }
+        }
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < NC; ++c) L[a][c] = td + 16 * c < pt ? scale * L[a][c] : -CUDART_INF_F;
+      if (cur.pass != 2) {  // running maximum and sum of exp over the cluster's keys
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          if (first) {
+            m[a] = -CUDART_INF_F;
+            l[a] = 0.f;
+          }
+          float cm = L[a][0];
+#pragma unroll
+          for (int c = 1; c < NC; ++c) cm = fmaxf(cm, L[a][c]);
+#pragma unroll
+          for (int o = 1; o < 16; o <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+          const float mn = fmaxf(m[a], cm);
+          float cs = 0.f;
+#pragma unroll
+          for (int c = 0; c < NC; ++c) cs += L[a][c] > -CUDART_INF_F ? expf(L[a][c] - mn) : 0.f;
+#pragma unroll
+          for (int o = 1; o < 16; o <<= 1) cs += __shfl_xor_sync(0xffffffffu, cs, o);
+          l[a] = (m[a] > -CUDART_INF_F ? l[a] * expf(m[a] - mn) : 0.f) + cs;
+          m[a] = mn;
+          if (last) lz[a] = m[a] + logf(l[a]);
+        }
+        if (cur.pass == 1) return;
+      }
+      if (first) clear_acc();
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int kk = td + 16 * c;
+        float w[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          w[a] = kk < pt ? expf(L[a][c] - lz[a]) : 0.f;
+          if (kk < pt && i0 + ti * 4 + a < Cq) wb[(int64_t)(i0 + ti * 4 + a) * wl + cur.pc + kk] = w[a];
+        }
+        *reinterpret_cast<float4 *>(Ws + kk * WS + 4 * ti) = make_float4(w[0], w[1], w[2], w[3]);
+      }
+      __syncthreads();
+      for (int pp = 0; pp < pt; ++pp) {
+        const float4 wv = *reinterpret_cast<const float4 *>(Ws + pp * WS + 4 * ti);
+        const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int h = 0; h < PQ; ++h) {
+          const float4 kv = *reinterpret_cast<const float4 *>(Ks + pp * QS + 64 * h + 4 * td);
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            acc[a][h][0] = fmaf(wa[a], kv.x, acc[a][h][0]);
+            acc[a][h][1] = fmaf(wa[a], kv.y, acc[a][h][1]);
+            acc[a][h][2] = fmaf(wa[a], kv.z, acc[a][h][2]);
+            acc[a][h][3] = fmaf(wa[a], kv.w, acc[a][h][3]);
+          }
+        }
+      }
+      if (last) put(cur.j, lz, acc);
+    };
+    const int nc = (pt + 15) >> 4;
+    if (nc <= 1) body(std::integral_constant<int, 1>{});
+    else if (nc <= 2) body(std::integral_constant<int, 2>{});
+    else if (nc <= 4 || KC < 128) body(std::integral_constant<int, (KC / 16 < 4 ? KC / 16 : 4)>{});
+    else body(std::integral_constant<int, KC / 16>{});
+    cur = nxt;
   }
 }
 
@@ -739,12 +1022,39 @@ cudaError_t run_sort_side_t(const void *X, int dtype, int width, int N, const Se
   return cudaGetLastError();
 }
 
+template <typename T, int D>
+static cudaError_t launch_tilt_fused(const MuseTables &mt, int P, float scale, const float *qcen,
+                                     SortedSide ks, const int32_t *k_offsets, StageBufs b,
+                                     cudaStream_t st) {
+  using Cf = TiltCfg<T, D>;
+  BlockMap bm;  // ceil(C / G) blocks per instance
+  bm.pre[0] = 0;
+  for (int si = 0; si < mt.in.ninst; ++si) {
+    const int C = mt.k.C[si], g = tilt_group(mt.k.nrow[si], C, Cf::KC);
+    bm.pre[si + 1] = bm.pre[si] + (C + g - 1) / g;
+  }
+  for (int si = mt.in.ninst + 1; si <= kMaxSeg; ++si) bm.pre[si] = bm.pre[mt.in.ninst];
+  bm.total = bm.pre[mt.in.ninst];
+  if (bm.total == 0) return cudaSuccess;
+  cudaError_t err = cudaFuncSetAttribute(tilt_fused<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cf::smem);
+  if (err != cudaSuccess) return err;
+  tilt_fused<T, D><<<dim3(bm.total, (mt.q.max_C + 63) / 64, P), 256, Cf::smem, st>>>(
+      mt, scale, qcen, (const T *)ks.rows, k_offsets, b.W, b.logZ, b.mu_k, bm);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 template <typename T, int D, int DV>
 static cudaError_t summaries_t(const MuseTables &mt, int P, float scale, const float *qcen,
                                SortedSide ks, const void *vs, const int32_t *k_offsets,
                                StageBufs b, cudaStream_t st) {
   const int tasks = P * mt.in.ninst;
-  const int maxCq = mt.q.max_C, maxCk = mt.k.max_C, maxnk = mt.k.max_rows;
+  const int maxCq = mt.q.max_C, maxCk = mt.k.max_C;
+  if (b.mu_k && !b.mu_v && !b.cov) {
+    // the forward pass: logits, log-normalisers, weights and key means in one launch
+    return launch_tilt_fused<T, D>(mt, P, scale, qcen, ks, k_offsets, b, st);
+  }
   const BlockMap kbm = make_block_map(mt.k, 64);
   tilt_logits<T, D><<<dim3(kbm.total, (maxCq + 63) / 64, P), 256, 0, st>>>(
       mt, scale, qcen, (const T *)ks.rows, b.W, kbm);

@@ -119,6 +119,49 @@ def test_summaries_and_refine_vs_oracle(dt):
             assert err <= TOL[dt], err
 
 
+# logZ and mu_k alone take the one-launch tilt kernel: key clusters of 0, 1, 15-17, 64-65,
+# 127-129 and 300 keys (one chunk, several chunks, several clusters per CTA), 70 centroids
+# (a ragged second group of 64), given directly as a permutation and offsets.
+@pytest.mark.parametrize("dt,D,Ck", [("bf16", 64, 16), ("bf16", 64, 40), ("f32", 64, 40),
+                                      ("bf16", 128, 40), ("f32", 128, 16)])
+def test_key_means_cluster_layouts(dt, D, Ck):
+    rng = np.random.Generator(np.random.PCG64(100 + Ck + D))
+    N, Cq, s = 1200, 70, 0.35
+    fixed = [300, 0, 1, 15, 16, 17, 64, 65, 127, 128, 129, 0]
+    rest = Ck - len(fixed)
+    left = N - sum(fixed)
+    if rest > 0:
+        cuts = np.sort(rng.integers(0, left + 1, rest - 1))
+        sizes = fixed + list(np.diff(np.concatenate([[0], cuts, [left]])))
+    else:
+        sizes = fixed[:Ck - 1] + [N - sum(fixed[:Ck - 1])]
+    sizes = np.array(sizes)
+    assert sizes.sum() == N and (sizes >= 0).all() and len(sizes) == Ck
+    K = 0.6 * rng.standard_normal((1, 1, N, D))
+    V = rng.standard_normal((1, 1, N, D))
+    qc = rng.standard_normal((1, 1, Cq, D)).astype(np.float32)
+    perm = rng.permutation(N).astype(np.int32)
+    offs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    labels = np.empty(N, np.int64)
+    for j in range(Ck):
+        labels[perm[offs[j]:offs[j + 1]]] = j
+    Kd, Vd = dev(K, dt), dev(V, dt)
+    g = m.muse_tilted_summaries(torch.tensor(qc).cuda(), Kd, Vd,
+                                torch.tensor(perm[None, None]).cuda().contiguous(),
+                                torch.tensor(offs[None, None]).cuda().contiguous(), Ck, s,
+                                want_mu_v=False)
+    lz, mk, _, _ = mo.tilted_summaries(qc[0, 0].astype(np.float64), host(Kd)[0, 0], host(Vd)[0, 0],
+                                       labels, Ck, s, want_cov=False)
+    glz = g["logZ"][0, 0].cpu().numpy()
+    gmk = g["mu_k"][0, 0].cpu().numpy()
+    fin = np.isfinite(lz)
+    assert (np.isfinite(glz) == fin).all() and (glz[~fin] == -np.inf).all()
+    np.testing.assert_allclose(glz[fin], lz[fin], rtol=1e-5, atol=1e-5)
+    assert (gmk[~fin] == 0).all()
+    err = np.abs(gmk - mk).max() / np.abs(mk).max()
+    assert err < 1e-5, err
+
+
 def test_forward_end_to_end_small_f32():
     w = WORKLOADS["acausal_n1k_f32"]
     Q, K, V = make_inputs(w)
