@@ -31,6 +31,7 @@
 // epilogue.  Every mbarrier wait is bounded (MUSE_ERR_TIMEOUT); every CTA, idle
 // padding CTAs included, executes the same sequence of cluster barriers.
 #include <algorithm>
+#include <numeric>
 #include <vector>
 
 #include "internal.h"
@@ -44,7 +45,7 @@ constexpr int D = 64;          // row width handled by this kernel
 constexpr int NSX = 4;         // row-tile stages
 constexpr int NOH = 2;         // one-hot buffers
 constexpr int CMAX = 128;      // clusters per task
-constexpr int GMAX = 8;        // CTAs per thread-block cluster
+constexpr int GMAX = 8;        // CTAs per thread-block cluster (at most)
 constexpr int TPC = 8;         // row tiles per CTA that a group size aims for
 constexpr int kEpi = 8;        // epilogue warps
 constexpr int kThreads = 64 + 32 * kEpi;
@@ -172,7 +173,7 @@ __device__ __forceinline__ float put_centroid(Smem &sm, int c, int h, const floa
   return sq;
 }
 
-__global__ void __cluster_dims__(GMAX, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
          const __grid_constant__ Params prm, int *status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -631,66 +632,102 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
 }
 
 // ------------------------------------------------------------------ host side
-// CTAs of a task's group: enough for about tpc row tiles each, a power of two <= 8.
-static int group_size(int n, int tpc = TPC) {
+// Thread-block clusters of Z = 8 or 6 CTAs (a launch attribute); a task's group is a
+// divisor of Z, so that groups placed at multiples of their size never straddle a
+// cluster.  Clusters of 6 fit 22 to a B200 at this kernel's shared memory, clusters of
+// 8 only 15: for 16 tasks of 64 row tiles, groups of 6 (11 tiles per CTA) then beat
+// groups of 4 (16 tiles per CTA).
+static int group_size(int n, int tpc, int Z) {
   const int tiles = (n + TM - 1) / TM;
   const int want = (tiles + tpc - 1) / tpc;
-  int g = 1;
-  while (g < want && g < GMAX) g <<= 1;
-  return g;
+  for (int g = 1; g < Z; ++g)
+    if (Z % g == 0 && g >= want) return g;
+  return Z;
 }
 
-// Lays the segments of one problem out in CTA slots, largest groups first, so every
-// group starts at a multiple of its size and never straddles a cluster of 8.  Returns
-// the largest group.
-static int plan_job(Job &J, const SegTable &t, int tpc) {
+// Lays the segments of one problem out in CTA slots, largest groups first, each group at
+// a multiple of its size.  Returns the least common multiple of the group sizes, the
+// alignment of the problem's span and of the job's first CTA.
+static int plan_job(Job &J, const SegTable &t, int tpc, int Z) {
   std::vector<int> order(t.nseg);
   for (int s = 0; s < t.nseg; ++s) order[s] = s;
   std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
-    return group_size(t.nrow[a], tpc) > group_size(t.nrow[b], tpc);
+    return group_size(t.nrow[a], tpc, Z) > group_size(t.nrow[b], tpc, Z);
   });
-  int pos = 0, gmax = 1;
+  int pos = 0, L = 1;
   for (int e = 0; e < t.nseg; ++e) {
-    const int s = order[e], g = group_size(t.nrow[s], tpc);
+    const int s = order[e], g = group_size(t.nrow[s], tpc, Z);
+    pos = (pos + g - 1) / g * g;
     J.ent[e].seg = (uint8_t)s;
     J.ent[e].g = (uint8_t)g;
     J.ent[e].pos = (uint16_t)pos;
     pos += g;
-    gmax = std::max(gmax, g);
+    L = std::lcm(L, g);
   }
   J.nent = t.nseg;
-  J.span = (pos + gmax - 1) / gmax * gmax;
-  return gmax;
+  J.span = (pos + L - 1) / L * L;
+  return L;
+}
+
+// Plans every job for cluster size Z and group target tpc; returns the grid (a multiple
+// of Z) and the largest number of row tiles a CTA takes.
+static int plan_all(Params &prm, int njobs, const void *const *X, const SegTable *const *tabs,
+                    const KmeansOut *outs, int tpc, int Z, int &max_tiles) {
+  int cursor = 0;
+  max_tiles = 0;
+  for (int j = 0; j < njobs; ++j) {
+    Job &J = prm.job[j];
+    J.X = X[j];
+    J.tab = *tabs[j];
+    J.out = outs[j];
+    const int L = plan_job(J, *tabs[j], tpc, Z);
+    cursor = (cursor + L - 1) / L * L;
+    J.base = cursor;
+    cursor += prm.P * J.span;
+    for (int e = 0; e < J.nent; ++e) {
+      const int tiles = (J.tab.nrow[J.ent[e].seg] + TM - 1) / TM;
+      max_tiles = std::max(max_tiles, (tiles + J.ent[e].g - 1) / J.ent[e].g);
+    }
+  }
+  return (cursor + Z - 1) / Z * Z;
 }
 
 }  // namespace kmf
 
-// CTAs of the fused kernel that can be resident at once (0: not even one cluster fits).
-static int kmf_capacity() {
-  static int cap = -1;
-  if (cap < 0) {
+// CTAs of the fused kernel that can be resident at once in clusters of Z (0: not even
+// one cluster fits).
+static int kmf_capacity(int Z) {
+  static int cap[kmf::GMAX + 1] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+  if (cap[Z] < 0) {
     const size_t smem = sizeof(kmf::Smem) + 1024;
     int n = 0;
     if (cudaFuncSetAttribute(kmf::km_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
         cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(kmf::GMAX);
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = Z;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(Z);
       cfg.blockDim = dim3(kmf::kThreads);
       cfg.dynamicSmemBytes = smem;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
       if (cudaOccupancyMaxActiveClusters(&n, kmf::km_fused, &cfg) != cudaSuccess) n = 0;
     }
     if (n <= 0) cudaGetLastError();  // the multi-launch path takes over; leave no error behind
-    cap = n * kmf::GMAX;
+    cap[Z] = n * Z;
   }
-  return cap;
+  return cap[Z];
 }
 
 bool kmeans_fused_supported(int dtype, int D, const SegTable &t) {
   if (dtype != MUSE_BF16 || D != kmf::D || t.max_C > kmf::CMAX || t.nseg > 255) return false;
   int span = 0;
-  for (int s = 0; s < t.nseg; ++s) span += kmf::group_size(t.nrow[s]);
-  if (span > 65535) return false;
-  return kmf_capacity() > 0;
+  for (int s = 0; s < t.nseg; ++s) span += kmf::group_size(t.nrow[s], kmf::TPC, kmf::GMAX);
+  if (span > 65535 / 3) return false;  // positions of any plan (groups of 6 are at most 1.5x, padding < 2x) fit 16 bits
+  return kmf_capacity(kmf::GMAX) > 0;
 }
 
 cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *const *tabs,
@@ -702,37 +739,25 @@ cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *co
   prm.P = P;
   prm.N = N;
   prm.iters = iters;
-  // group sizes: about TPC row tiles per CTA, or more (smaller groups) when that lets
-  // every CTA of the launch be resident at once
-  const int cap = kmf_capacity();
-  int grid = 0;
-  for (int tpc = TPC; tpc <= 8 * TPC; tpc *= 2) {
-    int cursor = 0;
-    for (int j = 0; j < njobs; ++j) {
-      Job &J = prm.job[j];
-      J.X = X[j];
-      J.tab = *tabs[j];
-      J.out = outs[j];
-      const int gmax = plan_job(J, *tabs[j], tpc);
-      cursor = (cursor + gmax - 1) / gmax * gmax;
-      J.base = cursor;
-      cursor += P * J.span;
-    }
-    const int g = (cursor + GMAX - 1) / GMAX * GMAX;
-    if (tpc == TPC || g <= cap) grid = g;
-    if (g <= cap) break;
-    if (tpc == 8 * TPC) {  // nothing fits in one wave: back to the default group sizes
-      cursor = 0;
-      for (int j = 0; j < njobs; ++j) {
-        Job &J = prm.job[j];
-        const int gmax = plan_job(J, *tabs[j], TPC);
-        cursor = (cursor + gmax - 1) / gmax * gmax;
-        J.base = cursor;
-        cursor += P * J.span;
+  // Among the plans whose CTAs are all resident at once (clusters of 8 or 6, about
+  // 8 .. 64 row tiles per CTA), the one with the fewest row tiles per CTA; if none fits,
+  // clusters of 8 with about 8 tiles per CTA, in several waves.
+  int bestZ = GMAX, best_tpc = TPC, best_tiles = 1 << 30;
+  for (int Z : {GMAX, 6}) {
+    const int cap = kmf_capacity(Z);
+    if (cap <= 0) continue;
+    for (int tpc = TPC; tpc <= 8 * TPC; tpc *= 2) {
+      int tiles = 0;
+      const int grid = plan_all(prm, njobs, X, tabs, outs, tpc, Z, tiles);
+      if (grid <= cap && tiles < best_tiles) {
+        best_tiles = tiles;
+        bestZ = Z;
+        best_tpc = tpc;
       }
-      grid = (cursor + GMAX - 1) / GMAX * GMAX;
     }
   }
+  int tiles = 0;
+  const int grid = plan_all(prm, njobs, X, tabs, outs, best_tpc, bestZ, tiles);
   CUtensorMap m0, m1;
   if (!ptx::make_map(&m0, X[0], D, (uint64_t)P * N, D, TM) ||
       !ptx::make_map(&m1, X[njobs > 1 ? 1 : 0], D, (uint64_t)P * N, D, TM))
@@ -740,8 +765,21 @@ cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *co
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(km_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  km_fused<<<grid, kThreads, smem, st>>>(m0, m1, prm, status);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = bestZ;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, km_fused, m0, m1, prm, status);
   count_launches(1);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -71,11 +71,14 @@ def check_kmeans_rounds(X, C, T, dt):
 
 
 # bf16 with D = 64 and C <= 128 runs the single-launch K-means; the sizes give groups of
-# 1, 2, 4 and 8 CTAs per task, ragged last tiles and (N = 4200) a CTA with no row tile.
+# 1, 2, 4 and 8 CTAs per task in clusters of 8, ragged last tiles and (N = 4200) a CTA
+# with no row tile; 16 tasks of 64 tiles take groups of 6 and 40 tasks of 24 tiles
+# groups of 3, in clusters of 6.
 @pytest.mark.parametrize("dt,N,D,C,H", [("f32", 1024, 64, 32, 1), ("bf16", 2048, 128, 64, 2),
                                          ("bf16", 1000, 64, 37, 1), ("bf16", 1500, 64, 16, 1),
                                          ("bf16", 2100, 64, 64, 1), ("bf16", 4200, 64, 128, 1),
-                                         ("bf16", 8192, 64, 128, 2)])
+                                         ("bf16", 8192, 64, 128, 2), ("bf16", 8192, 64, 128, 16),
+                                         ("bf16", 3072, 64, 128, 40)])
 def test_kmeans_rounds_teacher_forced(dt, N, D, C, H):
     Q, K, V = mixture(11, 1, H, N, D, D, 48, 0.3 / np.sqrt(D), dt)
     ex = check_kmeans_rounds(Q, C, 6, dt)
