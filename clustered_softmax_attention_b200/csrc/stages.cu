@@ -599,6 +599,11 @@ tilt_cov(MuseTables mt, const int32_t *__restrict__ k_offsets, const float *__re
   }
 }
 
+// Instances a kernel leaves to another one (bit s: instance s).
+struct InstMask {
+  uint32_t w[kMaxSeg / 32];
+};
+
 // ---------------------------------------------------------------------------
 // Refinement coefficients for every sorted query position n of cluster i:
 //   a_j = logZ_ij + s u_j, u_j = qt.mu_k,ij;  p = softmax_j(a);
@@ -681,7 +686,7 @@ __global__ void __launch_bounds__(256)
 refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
                     const int32_t *__restrict__ q_offsets, const float *__restrict__ logZ,
                     const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
-                    float *__restrict__ lse) {
+                    float *__restrict__ lse, InstMask skip) {
   constexpr int CJ = 16 * JPT;  // key clusters per pass (all of them)
   constexpr int MS = CJ + 1;    // padded strides: transposed writes hit distinct banks
   constexpr int QS = 68;
@@ -690,6 +695,7 @@ refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
   float *Qs = Ms + D * MS;     // [D][QS] residual rows of the chunk (transposed)
   float *lz = Qs + D * QS;     // [CJ]
   const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
+  if ((skip.w[s >> 5] >> (s & 31)) & 1u) return;  // uniform: another kernel's instance
   const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
   // this CTA's 64-row chunk: chunk g of the instance, counting ceil(rows/64) chunks
   // per query cluster in cluster order (rows start on 4-row boundaries)
@@ -833,6 +839,200 @@ refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
           }
       }
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The same coefficients for query clusters of a few rows (the causal squares' small
+// instances): CTA per G consecutive query clusters of one instance (compact grid), passes
+// of 16 rows of one cluster.  The cluster's Ck tilted key means and log-normalisers and
+// the pass's residual rows arrive by cp.async one pass ahead.  Thread (tr, tj): row tr
+// of the pass, key clusters tj + 16 u; the softmax runs over the 16 lanes of a row; the
+// coefficients go through shared memory so that each key cluster's rows leave as one
+// contiguous run.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int JPT> struct CoefCfg {
+  static constexpr int CJ = 16 * JPT;                  // key clusters (all of them)
+  static constexpr int MSD = D + 4;                    // row stride of the means (floats)
+  static constexpr int QRB = D * (int)sizeof(T) + 16;  // row stride of the raw rows (bytes)
+  static constexpr int GMAX = 16;
+  static constexpr size_t smem = 2 * (size_t)CJ * MSD * 4 + 2 * (size_t)CJ * 4 + 2 * 16 * (size_t)QRB +
+                                 2 * (size_t)CJ * 17 * 4;
+};
+
+// query clusters per CTA for an instance of n rows in C clusters (about 64 rows a CTA)
+__host__ __device__ __forceinline__ int coef_group(int n, int C) {
+  if (C <= 0 || n <= 0) return 16;
+  const int64_t g = 64ll * C / n;
+  return (int)(g < 1 ? 1 : g > 16 ? 16 : g);
+}
+
+__device__ __forceinline__ void coef_cp16(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void coef_cp4(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+template <typename T, int D, int JPT>
+__global__ void __launch_bounds__(256)
+refine_coeffs_grouped(MuseTables mt, float scale, const T *__restrict__ qt_rows,
+                      const int32_t *__restrict__ q_offsets, const float *__restrict__ logZ,
+                      const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
+                      float *__restrict__ lse, const __grid_constant__ BlockMap bm) {
+  using Cf = CoefCfg<T, D, JPT>;
+  constexpr int CJ = Cf::CJ, MSD = Cf::MSD, QRB = Cf::QRB;
+  extern __shared__ float4 coef_smem[];
+  float *Ms = reinterpret_cast<float *>(coef_smem);               // [2][CJ][MSD] means
+  float *Lz = Ms + 2 * CJ * MSD;                                  // [2][CJ] logZ row
+  unsigned char *Qr = reinterpret_cast<unsigned char *>(Lz + 2 * CJ);  // [2][16][QRB] rows
+  float *Cs = reinterpret_cast<float *>(Qr + 2 * 16 * QRB);       // [2][CJ][17] c0, c1
+  __shared__ int offs[Cf::GMAX + 1];
+  int bfirst;
+  const int p = blockIdx.y, s = map_block(bm, mt.in.ninst, blockIdx.x, bfirst);
+  const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
+  const int Cq = q.C, Ck = k.C;
+  const int G = coef_group(q.n, Cq);
+  const int i0 = ((int)blockIdx.x - bfirst) * G, i1 = min(Cq, i0 + G);
+  if (i0 >= Cq) return;  // uniform
+  const int tid = threadIdx.x, tr = tid >> 4, tj = tid & 15;
+  if (tid <= i1 - i0) offs[tid] = q_offsets[q.off + i0 + tid];
+  __syncthreads();
+  const int64_t zbase = (int64_t)p * mt.in.z_stride + mt.in.z0[s];
+  float *C0 = c0 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
+  float *C1 = c1 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
+  const int cl = w_ld(q.n);
+  // a pass: rows r0 .. r0 + 15 (clipped to e) of cluster i
+  struct Pass {
+    int i, e, r0, mb;  // mb: the means buffer of cluster i
+  };
+  auto first_of = [&](int i, int mb) {
+    while (i < i1 && offs[i - i0 + 1] == offs[i - i0]) ++i;
+    Pass t;
+    t.i = i;
+    t.r0 = i < i1 ? offs[i - i0] : 0;
+    t.e = i < i1 ? offs[i - i0 + 1] : 0;
+    t.mb = mb;
+    return t;
+  };
+  auto next_of = [&](const Pass &t) {
+    if (t.r0 + 16 < t.e) {
+      Pass n = t;
+      n.r0 += 16;
+      return n;
+    }
+    return first_of(t.i + 1, t.mb ^ 1);
+  };
+  // copies of pass t's inputs: the rows into row buffer qb and, for a cluster's first
+  // pass, its means and log-normalisers into means buffer t.mb
+  auto fetch = [&](const Pass &t, int qb, bool means) {
+    constexpr int UR = D * (int)sizeof(T) / 16;  // 16-byte units per row
+    for (int u = tid; u < 16 * UR; u += 256) {
+      const int r = u / UR, c = u % UR;
+      const bool in = t.r0 + r < t.e;
+      coef_cp16(Qr + (qb * 16 + r) * QRB + 16 * c,
+                in ? (const void *)(reinterpret_cast<const uint4 *>(qt_rows + (q.lab + t.r0 + r) * D) + c)
+                   : (const void *)qt_rows,
+                in ? 16u : 0u);
+    }
+    if (means) {
+      const int64_t zrow = zbase + (int64_t)t.i * Ck;
+      for (int u = tid; u < CJ * (D / 4); u += 256) {
+        const int j = u / (D / 4), c = u % (D / 4);
+        const bool in = j < Ck;
+        coef_cp16(Ms + (t.mb * CJ + j) * MSD + 4 * c,
+                  in ? (const void *)(mu_k + (zrow + j) * D + 4 * c) : (const void *)mu_k, in ? 16u : 0u);
+      }
+      for (int j = tid; j < CJ; j += 256)
+        coef_cp4(Lz + t.mb * CJ + j, j < Ck ? (const void *)(logZ + zrow + j) : (const void *)logZ,
+                 j < Ck ? 4u : 0u);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  Pass cur = first_of(i0, 0);
+  if (cur.i >= i1) return;  // uniform: every cluster of the group is empty
+  int qb = 0;
+  fetch(cur, qb, true);
+  while (cur.i < i1) {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();  // this pass's inputs have landed; the previous pass is done
+    const Pass nxt = next_of(cur);
+    if (nxt.i < i1) fetch(nxt, qb ^ 1, nxt.i != cur.i);
+    const float *M = Ms + cur.mb * CJ * MSD;
+    const float *lz = Lz + cur.mb * CJ;
+    const unsigned char *qrow = Qr + (qb * 16 + tr) * QRB;
+    float acc[JPT];
+#pragma unroll
+    for (int u = 0; u < JPT; ++u) acc[u] = 0.f;
+#pragma unroll 4
+    for (int d = 0; d < D; d += 4) {
+      float qv[4];
+      if constexpr (sizeof(T) == 2) {
+        const uint2 raw = *reinterpret_cast<const uint2 *>(qrow + 2 * d);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+        qv[0] = a.x;
+        qv[1] = a.y;
+        qv[2] = b.x;
+        qv[3] = b.y;
+      } else {
+        const float4 a = *reinterpret_cast<const float4 *>(qrow + 4 * d);
+        qv[0] = a.x;
+        qv[1] = a.y;
+        qv[2] = a.z;
+        qv[3] = a.w;
+      }
+#pragma unroll
+      for (int u = 0; u < JPT; ++u) {
+        const float4 m4 = *reinterpret_cast<const float4 *>(M + (tj + 16 * u) * MSD + d);
+        acc[u] = fmaf(qv[0], m4.x, acc[u]);
+        acc[u] = fmaf(qv[1], m4.y, acc[u]);
+        acc[u] = fmaf(qv[2], m4.z, acc[u]);
+        acc[u] = fmaf(qv[3], m4.w, acc[u]);
+      }
+    }
+    // a_j = logZ_ij + s u_j; p = softmax_j(a) over the 16 lanes of the row
+    float m = -CUDART_INF_F;
+#pragma unroll
+    for (int u = 0; u < JPT; ++u)
+      m = fmaxf(m, tj + 16 * u < Ck ? lz[tj + 16 * u] + scale * acc[u] : -CUDART_INF_F);
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+#pragma unroll
+    for (int u = 0; u < JPT; ++u) {
+      const float av = tj + 16 * u < Ck ? lz[tj + 16 * u] + scale * acc[u] : -CUDART_INF_F;
+      l += av > -CUDART_INF_F ? __expf(av - m) : 0.f;
+    }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int u = 0; u < JPT; ++u) {
+      const int j = tj + 16 * u;
+      const float av = j < Ck ? lz[j] + scale * acc[u] : -CUDART_INF_F;
+      const float pj = av > -CUDART_INF_F ? __expf(av - m) * inv : 0.f;
+      Cs[j * 17 + tr] = pj * (1.f - scale * acc[u]);
+      Cs[(CJ + j) * 17 + tr] = scale * pj;
+    }
+    const int nr = min(16, cur.e - cur.r0);
+    if (tj == 0 && tr < nr) lse[q.lab + cur.r0 + tr] = m + logf(l);
+    __syncthreads();
+    for (int x = tid; x < Ck * 16; x += 256) {
+      const int j = x >> 4, r = x & 15;
+      if (r < nr) {
+        C0[(int64_t)j * cl + cur.r0 + r] = Cs[j * 17 + r];
+        C1[(int64_t)j * cl + cur.r0 + r] = Cs[(CJ + j) * 17 + r];
+      }
+    }
+    cur = nxt;
+    qb ^= 1;
   }
 }
 
@@ -1126,7 +1326,8 @@ cudaError_t run_tilt_weights(const MuseTables &mt, int dtype, int D, int P, floa
 
 template <typename T, int D, int JPT>
 static cudaError_t coeffs_tiled_t(const MuseTables &mt, int P, float scale, SortedSide qs,
-                                  const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
+                                  const int32_t *q_offsets, StageBufs b, InstMask skip,
+                                  cudaStream_t st) {
   constexpr int CJ = 16 * JPT;
   const size_t smem = ((size_t)D * (CJ + 1) + D * 68 + CJ) * sizeof(float);
   cudaError_t err = cudaFuncSetAttribute(refine_coeffs_tiled<T, D, JPT>,
@@ -1135,26 +1336,63 @@ static cudaError_t coeffs_tiled_t(const MuseTables &mt, int P, float scale, Sort
   // chunks of an instance: at most rows/64 + one partial chunk per cluster
   refine_coeffs_tiled<T, D, JPT><<<dim3((mt.q.max_rows + 63) / 64 + mt.q.max_C, P * mt.in.ninst), 256,
                                   smem, st>>>(
-      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse);
+      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse, skip);
   count_launches(1);
   return cudaGetLastError();
+}
+
+template <typename T, int D, int JPT>
+static cudaError_t coeffs_grouped_t(const MuseTables &mt, int P, float scale, SortedSide qs,
+                                    const int32_t *q_offsets, StageBufs b, InstMask skip,
+                                    cudaStream_t st) {
+  using Cf = CoefCfg<T, D, JPT>;
+  BlockMap bm;  // ceil(C / G) blocks per instance this kernel takes
+  bm.pre[0] = 0;
+  for (int si = 0; si < mt.in.ninst; ++si) {
+    const int C = mt.q.C[si], g = coef_group(mt.q.nrow[si], C);
+    const bool mine = !((skip.w[si >> 5] >> (si & 31)) & 1u);
+    bm.pre[si + 1] = bm.pre[si] + (mine ? (C + g - 1) / g : 0);
+  }
+  for (int si = mt.in.ninst + 1; si <= kMaxSeg; ++si) bm.pre[si] = bm.pre[mt.in.ninst];
+  bm.total = bm.pre[mt.in.ninst];
+  if (bm.total == 0) return cudaSuccess;
+  cudaError_t err = cudaFuncSetAttribute(refine_coeffs_grouped<T, D, JPT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::smem);
+  if (err != cudaSuccess) return err;
+  refine_coeffs_grouped<T, D, JPT><<<dim3(bm.total, P), 256, Cf::smem, st>>>(
+      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse, bm);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// Instances whose query clusters hold fewer than 32 rows on average take the grouped
+// kernel (passes of 16 rows), the others the tiled one (chunks of 64 rows); both run when
+// the instances differ (the causal squares).
+template <typename T, int D, int JPT>
+static cudaError_t coeffs_split_t(const MuseTables &mt, int P, float scale, SortedSide qs,
+                                  const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
+  InstMask small{}, large{};
+  bool any_small = false, any_large = false;
+  for (int si = 0; si < mt.in.ninst; ++si) {
+    const bool sm = (int64_t)mt.q.nrow[si] < 32ll * mt.q.C[si];
+    (sm ? large : small).w[si >> 5] |= 1u << (si & 31);  // the mask lists the skipped ones
+    any_small |= sm;
+    any_large |= !sm;
+  }
+  cudaError_t err = cudaSuccess;
+  if (any_large) err = coeffs_tiled_t<T, D, JPT>(mt, P, scale, qs, q_offsets, b, large, st);
+  if (err == cudaSuccess && any_small)
+    err = coeffs_grouped_t<T, D, JPT>(mt, P, scale, qs, q_offsets, b, small, st);
+  return err;
 }
 
 template <typename T, int D>
 static cudaError_t coeffs_t(const MuseTables &mt, int P, float scale, SortedSide qs,
                             const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
-  // the tiled form stages each query cluster's tilted key means once, which pays off
-  // when clusters hold a few dozen rows or more on average
-  int64_t rows = 0, clusters = 0;
-  for (int si = 0; si < mt.in.ninst; ++si) {
-    rows += mt.q.nrow[si];
-    clusters += mt.q.C[si];
-  }
-  if (rows >= 32 * clusters) {
-    if (mt.k.max_C <= 64) return coeffs_tiled_t<T, D, 4>(mt, P, scale, qs, q_offsets, b, st);
-    if (mt.k.max_C <= 128) return coeffs_tiled_t<T, D, 8>(mt, P, scale, qs, q_offsets, b, st);
-    if (mt.k.max_C <= 256 && D == 64) return coeffs_tiled_t<T, D, 16>(mt, P, scale, qs, q_offsets, b, st);
-  }
+  // both forms stage each query cluster's tilted key means once in shared memory
+  if (mt.k.max_C <= 64) return coeffs_split_t<T, D, 4>(mt, P, scale, qs, q_offsets, b, st);
+  if (mt.k.max_C <= 128) return coeffs_split_t<T, D, 8>(mt, P, scale, qs, q_offsets, b, st);
+  if (mt.k.max_C <= 256 && D == 64) return coeffs_split_t<T, D, 16>(mt, P, scale, qs, q_offsets, b, st);
   const int keep_u = mt.k.max_C <= 256 ? 1 : 0;
   const size_t smem = keep_u ? (size_t)mt.k.max_C * 128 * sizeof(float) : 0;
   cudaError_t err = cudaFuncSetAttribute(refine_coeffs<T, D>,
