@@ -676,24 +676,40 @@ refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
 // ---------------------------------------------------------------------------
 // The same coefficients as a register-tiled contraction per query cluster i:
 // U = Qt_i . mu_k,i^T (rows of cluster i against its Ck tilted key means), one
-// CTA per 64-row chunk of a query cluster (the largest clusters set no tail).
-// Thread (tq, tj): rows 4 tq .. 4 tq + 3 of the chunk and key clusters tj + 16 e;
-// the 16 threads of a row are consecutive lanes (softmax by shuffles); each thread
-// stores its 4 consecutive rows of a cluster j as one 16-byte vector.
+// CTA per 64-row chunk of a query cluster (the largest clusters set no tail).  The
+// means and the chunk's rows are copied as stored by cp.async (no transpose); thread
+// (tq, tj) takes rows 4 tq .. 4 tq + 3 and key clusters tj + 16 e and reads 4
+// coordinates at a time of each; the 16 threads of a row are consecutive lanes
+// (softmax by shuffles); each thread stores its 4 consecutive rows of a cluster j as
+// one 16-byte vector.
 // ---------------------------------------------------------------------------
+// 16- and 4-byte asynchronous global -> shared copies (src_bytes = 0 writes zeros).
+__device__ __forceinline__ void coef_cp16(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void coef_cp4(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
 template <typename T, int D, int JPT>
 __global__ void __launch_bounds__(256)
 refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
                     const int32_t *__restrict__ q_offsets, const float *__restrict__ logZ,
                     const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
                     float *__restrict__ lse, InstMask skip) {
-  constexpr int CJ = 16 * JPT;  // key clusters per pass (all of them)
-  constexpr int MS = CJ + 1;    // padded strides: transposed writes hit distinct banks
-  constexpr int QS = 68;
-  extern __shared__ float sm[];
-  float *Ms = sm;              // [D][MS] tilted key means of cluster i (transposed)
-  float *Qs = Ms + D * MS;     // [D][QS] residual rows of the chunk (transposed)
-  float *lz = Qs + D * QS;     // [CJ]
+  constexpr int CJ = 16 * JPT;                         // key clusters (all of them)
+  constexpr int MSD = D + 4;                           // row stride of the means (floats)
+  constexpr int QRB = D * (int)sizeof(T) + 16;         // row stride of the raw rows (bytes)
+  extern __shared__ float4 tiled_smem[];
+  float *Ms = reinterpret_cast<float *>(tiled_smem);   // [CJ][MSD] tilted key means of cluster i
+  float *lz = Ms + CJ * MSD;                           // [CJ]
+  unsigned char *Qr = reinterpret_cast<unsigned char *>(lz + CJ);  // [64][QRB] residual rows
   const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
   if ((skip.w[s >> 5] >> (s & 31)) & 1u) return;  // uniform: another kernel's instance
   const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
@@ -738,16 +754,27 @@ refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
   const int Ck = k.C;
   const int b = q_offsets[q.off + i], e = q_offsets[q.off + i + 1];
   const int64_t zrow = (int64_t)p * mt.in.z_stride + mt.in.z0[s] + (int64_t)i * Ck;
-  // Ms[d][j]: consecutive threads take consecutive clusters j of one 4-float group
-  for (int x = threadIdx.x; x < (D / 4) * CJ; x += 256) {
-    const int d4 = x / CJ, j = x % CJ;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j < Ck) v = *reinterpret_cast<const float4 *>(mu_k + (zrow + j) * D + 4 * d4);
-    Ms[(4 * d4) * MS + j] = v.x;
-    Ms[(4 * d4 + 1) * MS + j] = v.y;
-    Ms[(4 * d4 + 2) * MS + j] = v.z;
-    Ms[(4 * d4 + 3) * MS + j] = v.w;
+  const int r0 = s_r0;
+  // Ms[j][d]: the cluster's tilted key means as stored (rows of D floats, padded);
+  // Qr: the chunk's residual rows as stored (rows outside [b, e) zero); both by cp.async
+  for (int u = threadIdx.x; u < CJ * (D / 4); u += 256) {
+    const int j = u / (D / 4), c = u % (D / 4);
+    const bool in = j < Ck;
+    coef_cp16(Ms + j * MSD + 4 * c, in ? (const void *)(mu_k + (zrow + j) * D + 4 * c) : (const void *)mu_k,
+              in ? 16u : 0u);
   }
+  {
+    constexpr int UR = D * (int)sizeof(T) / 16;
+    for (int u = threadIdx.x; u < 64 * UR; u += 256) {
+      const int rr = u / UR, c = u % UR;
+      const bool in = r0 + rr >= b && r0 + rr < e;
+      coef_cp16(Qr + rr * QRB + 16 * c,
+                in ? (const void *)(reinterpret_cast<const uint4 *>(qt_rows + (q.lab + r0 + rr) * D) + c)
+                   : (const void *)qt_rows,
+                in ? 16u : 0u);
+    }
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
   for (int j = threadIdx.x; j < CJ; j += 256) lz[j] = j < Ck ? logZ[zrow + j] : -CUDART_INF_F;
   const int tq = threadIdx.x >> 4, tj = threadIdx.x & 15;
   float *C0 = c0 + (int64_t)p * mt.in.c_stride + mt.in.cc0[s];
@@ -756,38 +783,45 @@ refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
   // chunks start on 4-row boundaries of the coefficient arrays (16-byte stores);
   // rows outside [b, e) belong to other clusters and are neither read nor written
   {
-    const int r0 = s_r0;
-    __syncthreads();
-    // Qs[d][rr]: consecutive threads take consecutive rows of one 4-element group
-    for (int x = threadIdx.x; x < (D / 4) * 64; x += 256) {
-      const int d4 = x >> 6, rr = x & 63;
-      float v[4] = {0.f, 0.f, 0.f, 0.f};
-      if (r0 + rr >= b && r0 + rr < e) {
-        const T *src = qt_rows + (q.lab + r0 + rr) * D + 4 * d4;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) v[u] = ld_elem(src + u);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) Qs[(4 * d4 + u) * QS + rr] = v[u];
-    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
     float acc[4][JPT];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
       for (int u = 0; u < JPT; ++u) acc[a][u] = 0.f;
-#pragma unroll 4
-    for (int d = 0; d < D; ++d) {
-      const float4 qv = *reinterpret_cast<const float4 *>(&Qs[d * QS + 4 * tq]);
-      float mv[JPT];
+#pragma unroll 2
+    for (int d = 0; d < D; d += 4) {
+      float qv[4][4];
 #pragma unroll
-      for (int u = 0; u < JPT; ++u) mv[u] = Ms[d * MS + tj + 16 * u];
+      for (int a = 0; a < 4; ++a) {
+        const unsigned char *qrow = Qr + (4 * tq + a) * QRB;
+        if constexpr (sizeof(T) == 2) {
+          const uint2 raw = *reinterpret_cast<const uint2 *>(qrow + 2 * d);
+          const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+          const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+          qv[a][0] = x.x;
+          qv[a][1] = x.y;
+          qv[a][2] = y.x;
+          qv[a][3] = y.y;
+        } else {
+          const float4 x = *reinterpret_cast<const float4 *>(qrow + 4 * d);
+          qv[a][0] = x.x;
+          qv[a][1] = x.y;
+          qv[a][2] = x.z;
+          qv[a][3] = x.w;
+        }
+      }
 #pragma unroll
       for (int u = 0; u < JPT; ++u) {
-        acc[0][u] = fmaf(qv.x, mv[u], acc[0][u]);
-        acc[1][u] = fmaf(qv.y, mv[u], acc[1][u]);
-        acc[2][u] = fmaf(qv.z, mv[u], acc[2][u]);
-        acc[3][u] = fmaf(qv.w, mv[u], acc[3][u]);
+        const float4 m4 = *reinterpret_cast<const float4 *>(Ms + (tj + 16 * u) * MSD + d);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          acc[a][u] = fmaf(qv[a][0], m4.x, acc[a][u]);
+          acc[a][u] = fmaf(qv[a][1], m4.y, acc[a][u]);
+          acc[a][u] = fmaf(qv[a][2], m4.z, acc[a][u]);
+          acc[a][u] = fmaf(qv[a][3], m4.w, acc[a][u]);
+        }
       }
     }
     // a_j = logZ_ij + s u_j; p = softmax_j(a) over the 16 lanes of each row
@@ -867,18 +901,6 @@ __host__ __device__ __forceinline__ int coef_group(int n, int C) {
   return (int)(g < 1 ? 1 : g > 16 ? 16 : g);
 }
 
-__device__ __forceinline__ void coef_cp16(void *dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
-                   (uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void coef_cp4(void *dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(
-                   (uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src), "r"(src_bytes)
-               : "memory");
-}
 
 template <typename T, int D, int JPT>
 __global__ void __launch_bounds__(256)
@@ -1329,7 +1351,7 @@ static cudaError_t coeffs_tiled_t(const MuseTables &mt, int P, float scale, Sort
                                   const int32_t *q_offsets, StageBufs b, InstMask skip,
                                   cudaStream_t st) {
   constexpr int CJ = 16 * JPT;
-  const size_t smem = ((size_t)D * (CJ + 1) + D * 68 + CJ) * sizeof(float);
+  const size_t smem = (size_t)CJ * (D + 4) * 4 + CJ * 4 + 64 * (D * sizeof(T) + 16);
   cudaError_t err = cudaFuncSetAttribute(refine_coeffs_tiled<T, D, JPT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
