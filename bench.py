@@ -17,6 +17,7 @@ a bounded sample (one head per step) of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import os
@@ -47,7 +48,22 @@ def parse():
     ap.add_argument("--workload", default="acausal_n8k_bf16", choices=sorted(WORKLOADS))
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", type=int, default=0,
+                    help="causal/retrieval block size S (default: the workload's); "
+                         "N/2 gives the single-level decomposition")
     return ap.parse_args()
+
+
+def workload_of(args):
+    """The named workload, with the block size overridden if --block is given."""
+    w = WORKLOADS[args.workload]
+    if args.block:
+        if w.mode == "acausal":
+            raise SystemExit("--block applies to the causal and retrieval workloads")
+        if args.block <= 0 or w.N % args.block:
+            raise SystemExit(f"--block must divide N={w.N}")
+        w = dataclasses.replace(w, block=args.block)
+    return w
 
 
 def dist_info():
@@ -228,7 +244,7 @@ def oracle_sample(w, head=0):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
+    w = workload_of(args)
     for _ in range(args.warmup):
         oracle_sample(w)
     secs = []
@@ -281,7 +297,7 @@ def main():
     from clustered_softmax_attention_b200 import muse as m
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = WORKLOADS[args.workload]
+    w = workload_of(args)
     Qn, Kn, Vn = make_inputs(w)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     Qh = torch.from_numpy(Qn).to(tdt).pin_memory()
