@@ -10,8 +10,10 @@
 //
 // One CTA = 128 query rows inside one block (block a multiple of 128); it attends the
 // key tiles t = 0 .. qt of its block (qt = the query tile's index in the block; tile qt
-// is the diagonal one, masked k <= n).  TMA brings the residual-free query tile and all
-// key and value tiles at once.  Two passes over the key tiles:
+// is the diagonal one, masked k <= n).  TMA brings the residual-free query tile and, when
+// at most four key tiles are attended, all key and value tiles at once; otherwise the
+// key tiles (pass 1) and the key and value tiles (pass 2) come in groups of four.  Two
+// passes over the key tiles:
 //   pass 1: S = Q . K_t^T (tcgen05, fp32 in TMEM) -> running row maximum of s S
 //   pass 2: S again; P = exp(s S - m) (bf16, TMEM); l += sum P; O += P . V_t
 //           (tcgen05, A = P from TMEM, B = V_t as stored: keys x Dv, Dv innermost)
@@ -25,7 +27,7 @@ namespace dtc {
 
 constexpr int TM = 128;       // query rows per CTA and keys per tile
 constexpr int D = 64;
-constexpr int MAXT = 4;       // key tiles per block at most (block <= 512)
+constexpr int MAXT = 4;       // key and value tiles resident at once
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kS = 0, kP = 128, kO = 192;  // TMEM columns: S, P (packed bf16), O
 
@@ -89,17 +91,35 @@ diag_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUten
   const uint32_t tmem = sm.tmem_base;
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
+  const bool one = qt < MAXT;  // every key and value tile resident from the start
   if (t == 0) {
-    mbar_expect_tx(&sm.lbar, (uint32_t)(1 + 2 * (qt + 1)) * TM * 128);
+    const int nk = one ? qt + 1 : MAXT;
+    mbar_expect_tx(&sm.lbar, (uint32_t)(1 + (one ? 2 : 1) * nk) * TM * 128);
     tma_load_2d(sm.q, &map_q, 0, (int)(row0 + n0), &sm.lbar);
-    for (int kt = 0; kt <= qt; ++kt) {
+    for (int kt = 0; kt < nk; ++kt) {
       tma_load_2d(sm.k[kt], &map_k, 0, (int)(row0 + ks0 + kt * TM), &sm.lbar);
-      tma_load_2d(sm.v[kt], &map_v, 0, (int)(row0 + ks0 + kt * TM), &sm.lbar);
+      if (one) tma_load_2d(sm.v[kt], &map_v, 0, (int)(row0 + ks0 + kt * TM), &sm.lbar);
     }
   }
   // (every decision to go on is made CTA-wide: a wait that gives up in one thread stops
   // all of them at the next barrier)
   bool ok = __syncthreads_and(mbar_wait(&sm.lbar, 0, abort_flag, status));
+  uint32_t lph = 1;  // loads issued on lbar (each one phase)
+  // key tiles g0 .. g0 + cnt - 1 (and their value tiles) into slots 0 .. cnt - 1; called
+  // by every thread after a CTA barrier that follows the last MMA reading the slots
+  auto load_group = [&](int g0, bool withv) -> bool {
+    const int cnt = min(MAXT, qt + 1 - g0);
+    if (t == 0) {
+      mbar_expect_tx(&sm.lbar, (uint32_t)((withv ? 2 : 1) * cnt) * TM * 128);
+      for (int i = 0; i < cnt; ++i) {
+        tma_load_2d(sm.k[i], &map_k, 0, (int)(row0 + ks0 + (g0 + i) * TM), &sm.lbar);
+        if (withv) tma_load_2d(sm.v[i], &map_v, 0, (int)(row0 + ks0 + (g0 + i) * TM), &sm.lbar);
+      }
+    }
+    const bool r = mbar_wait(&sm.lbar, lph & 1, abort_flag, status);
+    ++lph;
+    return __syncthreads_and(r);
+  };
   uint32_t mph = 0;  // phase of the MMA barrier
   // S = Q . K_kt^T into TMEM columns [kS, kS + 128); every thread waits for it
   auto qk = [&](int kt) -> bool {
@@ -107,7 +127,7 @@ diag_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUten
       tc_fence_after();
       const uint32_t id = idesc(TM, TM);
       for (int kk = 0; kk < D / 16; ++kk)
-        tc_mma(tmem + kS, sdesc(sm.q + kk * 16), sdesc(sm.k[kt] + kk * 16), id, kk > 0 ? 1u : 0u);
+        tc_mma(tmem + kS, sdesc(sm.q + kk * 16), sdesc(sm.k[kt % MAXT] + kk * 16), id, kk > 0 ? 1u : 0u);
       tc_commit(&sm.mbar);
     }
     const bool r = mbar_wait(&sm.mbar, mph & 1, abort_flag, status);
@@ -120,6 +140,7 @@ diag_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUten
   float m2 = -CUDART_INF_F;  // running maximum of c S over the valid keys of the row
   // ------------------------------------------------ pass 1: row maxima
   for (int kt = 0; ok && kt <= qt; ++kt) {
+    if (kt > 0 && kt % MAXT == 0 && !(ok = load_group(kt, false))) break;
     const bool r = qk(kt);
     const int lim = kt < qt ? TM : t + 1;  // valid columns of this row
     for (int cb = 0; r && cb < TM / 16; ++cb) {
@@ -135,6 +156,7 @@ diag_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUten
   // ------------------------------------------------ pass 2: P, l and O += P V
   float l = 0.f;
   for (int kt = 0; ok && kt <= qt; ++kt) {
+    if (!one && kt % MAXT == 0 && !(ok = load_group(kt, true))) break;
     const bool r = qk(kt);
     const int lim = kt < qt ? TM : t + 1;
     for (int cb = 0; r && cb < TM / 16; ++cb) {
@@ -159,7 +181,7 @@ diag_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUten
       // B = V_kt as stored (keys x Dv, Dv innermost): MN-major operand
       const uint32_t id = idesc(TM, D) | (1u << 16);
       for (int kk = 0; kk < TM / 16; ++kk)
-        tc_mma_ts(tmem + kO, tmem + kP + kk * 8, sdesc_mn(sm.v[kt] + kk * 16 * 64), id,
+        tc_mma_ts(tmem + kO, tmem + kP + kk * 8, sdesc_mn(sm.v[kt % MAXT] + kk * 16 * 64), id,
                   (kt > 0 || kk > 0) ? 1u : 0u);
       tc_commit(&sm.mbar);
     }
@@ -216,7 +238,7 @@ diag_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUten
   }
   // copies and MMAs still in flight land before the CTA releases its memory
   if (t == 0) {
-    mbar_drain(&sm.lbar, 0, status);
+    mbar_drain(&sm.lbar, (lph - 1) & 1, status);  // the last load issued
     tc_commit(&sm.mbar);
     mbar_drain(&sm.mbar, mph & 1, status);
   }
@@ -233,8 +255,7 @@ diag_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUten
 }  // namespace dtc
 
 bool diag_tc_supported(int dtype, int D, int Dv, int N, int block) {
-  return dtype == MUSE_BF16 && D == dtc::D && Dv == dtc::D && block % dtc::TM == 0 &&
-         block / dtc::TM <= dtc::MAXT && N % block == 0;
+  return dtype == MUSE_BF16 && D == dtc::D && Dv == dtc::D && block % dtc::TM == 0 && N % block == 0;
 }
 
 cudaError_t run_diag_tc(const void *Q, const void *K, const void *V, int N, int P, int block,

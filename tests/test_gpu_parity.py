@@ -222,12 +222,14 @@ def causal_labels(ql, kl, N, S):
 
 
 # block sizes: 128 and 256 (several levels), 512 at N = 2048 (the tensor-core diagonal
-# with four key tiles per block), S = N/2 (a single level), and 1024 (the CUDA-core
-# diagonal, beyond the tensor-core kernel's 512)
+# with four key tiles per block, all resident), S = N/2 (a single level), 1024 and 2048
+# (the tensor-core diagonal streaming key and value tiles in groups of four), and the
+# CUDA-core diagonal of the float32 path at 512 and 1024
 @pytest.mark.parametrize("dt,N,S,C", [("f32", 1024, 128, 16), ("bf16", 1024, 128, 16),
                                        ("bf16", 1536, 256, 40), ("bf16", 2048, 512, 32),
                                        ("bf16", 1024, 512, 32), ("bf16", 2048, 1024, 48),
-                                       ("f32", 2048, 512, 32)])
+                                       ("bf16", 4096, 2048, 32), ("f32", 2048, 512, 32),
+                                       ("f32", 2048, 1024, 48)])
 def test_causal_vs_oracle(dt, N, S, C):
     Q, K, V = mixture(7, 1, 2, N, 64, 64, 16, 0.3 / 8, dt)
     Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
