@@ -18,7 +18,7 @@ q = qbar_i + qt (the residual), k = k_j + kt ([summary] "Kernmechanismen", item 
 
 Every routine is float64.  Inputs are the already-rounded values the GPU sees.
 
-Readings taken where the pages leave a step open (each is listed in the design doc):
+Readings taken where the pages leave a step open:
   * K-means starts from the first C rows, runs T rounds of (assign, update); the
     labels are those of round T and the centroids are the update after it.  An
     empty cluster keeps its previous centroid.  Ties go to the lowest cluster index.
@@ -208,7 +208,7 @@ def tilted_summaries(qbar: np.ndarray, K: np.ndarray, V: np.ndarray,
 def refine(Q: np.ndarray, q_labels: np.ndarray, qbar: np.ndarray, logZ: np.ndarray,
            mu_k: np.ndarray, mu_v: np.ndarray, cov: np.ndarray, scale: float,
            zero_residual: bool = False, rows: Optional[np.ndarray] = None,
-           return_lse: bool = False):
+           return_lse: bool = False, dipole: bool = True):
     """For query n in cluster i, qt = q_n - qbar_i:
 
       a_j  = logZ_ij + s * qt . mu_k,ij
@@ -216,6 +216,9 @@ def refine(Q: np.ndarray, q_labels: np.ndarray, qbar: np.ndarray, logZ: np.ndarr
       O_n  = sum_j p_j (mu_v,ij + s * C_ij qt)
 
     ``zero_residual`` forces qt = 0 (the monopole-only result at the centroid).
+    ``dipole=False`` drops the s C_ij qt term: the monopole-only ablation ([review]
+    "invented entities": the dipole correction, whose removal the paper's Table 3
+    measures), O_n = sum_j p_j mu_v,ij with the same weights p.
     ``rows`` restricts the output to those query rows (others are left zero).
     With ``return_lse`` also returns logsumexp_j a_j per row (for merging partial sums).
     """
@@ -241,7 +244,7 @@ def refine(Q: np.ndarray, q_labels: np.ndarray, qbar: np.ndarray, logZ: np.ndarr
         p = e / l[:, None]
         Ck, Dv_, D = cov[i].shape
         dip = (cov[i].reshape(Ck * Dv_, D) @ Qt.T).reshape(Ck, Dv_, idx.size)  # C_ij qt
-        term = mu_v[i][:, :, None] + scale * dip                    # [Ck, Dv, n_i]
+        term = mu_v[i][:, :, None] + (scale * dip if dipole else 0.0)  # [Ck, Dv, n_i]
         O[idx] = np.einsum("nj,jvn->nv", p, term)
         lse[idx] = m + np.log(l)
     if return_lse:
@@ -251,7 +254,8 @@ def refine(Q: np.ndarray, q_labels: np.ndarray, qbar: np.ndarray, logZ: np.ndarr
 
 def muse_from_labels(Q, K, V, q_labels, k_labels, Cq: int, Ck: int, scale: float,
                      qbar: Optional[np.ndarray] = None, rows: Optional[np.ndarray] = None,
-                     return_lse: bool = False, zero_residual: bool = False):
+                     return_lse: bool = False, zero_residual: bool = False,
+                     dipole: bool = True):
     """MuSe output from given clusterings.  qbar defaults to the member means.
 
     With ``rows`` the summaries are built only for the query clusters those rows use.
@@ -268,18 +272,19 @@ def muse_from_labels(Q, K, V, q_labels, k_labels, Cq: int, Ck: int, scale: float
         logZ, mu_k, mu_v, cov = tilted_summaries(qbar[used], K, V, k_labels, Ck, scale)
         lab = np.where(q_labels >= 0, remap[np.clip(q_labels, 0, Cq - 1)], -1)
         return refine(Q, lab, qbar[used], logZ, mu_k, mu_v, cov, scale,
-                      zero_residual=zero_residual, rows=rows, return_lse=return_lse)
+                      zero_residual=zero_residual, rows=rows, return_lse=return_lse,
+                      dipole=dipole)
     logZ, mu_k, mu_v, cov = tilted_summaries(qbar, K, V, k_labels, Ck, scale)
     return refine(Q, q_labels, qbar, logZ, mu_k, mu_v, cov, scale,
-                  zero_residual=zero_residual, return_lse=return_lse)
+                  zero_residual=zero_residual, return_lse=return_lse, dipole=dipole)
 
 
 def muse_acausal(Q, K, V, Cq: int, Ck: int, iters: int, scale: float,
-                 return_labels: bool = False):
+                 return_labels: bool = False, dipole: bool = True):
     """Full acausal MuSe: K-means on Q and on K, summaries, refinement."""
     ql, qc = kmeans(Q, Cq, iters)
     kl, _ = kmeans(K, Ck, iters)
-    O = muse_from_labels(Q, K, V, ql, kl, Cq, Ck, scale, qbar=qc)
+    O = muse_from_labels(Q, K, V, ql, kl, Cq, Ck, scale, qbar=qc, dipole=dipole)
     if return_labels:
         return O, ql, kl
     return O

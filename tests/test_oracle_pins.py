@@ -264,11 +264,41 @@ def test_monopole_only_would_be_first_order():
         Q, K, V, ql, kl = _order_problem(eq, 0.05)
         qbar = mo.cluster_means(Q, ql, 4)
         logZ, mu_k, mu_v, cov = mo.tilted_summaries(qbar, K, V, kl, 4, 1.0)
-        O = mo.refine(Q, ql, qbar, logZ, mu_k, mu_v, 0 * cov, 1.0)
+        O = mo.refine(Q, ql, qbar, logZ, mu_k, mu_v, cov, 1.0, dipole=False)
         return np.abs(O - mo.exact_attention(Q, K, V, 1.0)).max()
     eps = np.array([1e-3, 1e-2, 1e-1])
     slope = np.polyfit(np.log(eps), np.log([err_no_dip(e) for e in eps]), 1)[0]
     assert 0.8 <= slope <= 1.2
+
+
+def test_monopole_only_single_key_cluster_is_attention_at_the_centroid():
+    """Monopole only, Ck = 1: every query of cluster i gets sum_k softmax(s qbar_i.k) v_k,
+    exact attention evaluated at its centroid, whatever its residual."""
+    rng = np.random.default_rng(21)
+    N, D, Dv, Cq, s = 48, 5, 3, 4, 0.7
+    Q = rng.standard_normal((N, D))
+    K = rng.standard_normal((N, D))
+    V = rng.standard_normal((N, Dv))
+    ql = rng.integers(0, Cq, N)
+    ql[:Cq] = np.arange(Cq)
+    O = mo.muse_from_labels(Q, K, V, ql, np.zeros(N, np.int64), Cq, 1, s, dipole=False)
+    qbar = mo.cluster_means(Q, ql, Cq)
+    at_centroid = mo.exact_attention(qbar, K, V, s)
+    np.testing.assert_allclose(O, at_centroid[ql], rtol=1e-12, atol=1e-12)
+    # the dipole term is what moves the output off the centroid's value
+    O_dip = mo.muse_from_labels(Q, K, V, ql, np.zeros(N, np.int64), Cq, 1, s)
+    assert np.abs(O_dip - O).max() > 1e-3
+
+
+def test_monopole_only_singleton_queries_is_exact():
+    """Monopole only with Cq = N: qt = 0, so the dropped term vanishes and the result is
+    exact attention for any key clustering."""
+    rng = np.random.default_rng(22)
+    N, D, Dv = 40, 4, 3
+    Q, K, V = rng.standard_normal((N, D)), rng.standard_normal((N, D)), rng.standard_normal((N, Dv))
+    kl = rng.integers(0, 5, N)
+    O = mo.muse_from_labels(Q, K, V, np.arange(N), kl, N, 5, 1.0, dipole=False)
+    np.testing.assert_allclose(O, mo.exact_attention(Q, K, V, 1.0), rtol=1e-10, atol=1e-12)
 
 
 # --------------------------------------------------------------------------- tiny brute force
