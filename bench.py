@@ -51,6 +51,12 @@ def parse():
     ap.add_argument("--block", type=int, default=0,
                     help="causal/retrieval block size S (default: the workload's); "
                          "N/2 gives the single-level decomposition")
+    ap.add_argument("--clusters", type=int, default=0,
+                    help="Cq = Ck override (default: the workload's)")
+    ap.add_argument("--iters", type=int, default=0,
+                    help="K-means rounds override (default: the workload's)")
+    ap.add_argument("--monopole", action="store_true",
+                    help="acausal: the monopole-only ablation (dipole term dropped)")
     return ap.parse_args()
 
 
@@ -63,6 +69,14 @@ def workload_of(args):
         if args.block <= 0 or w.N % args.block:
             raise SystemExit(f"--block must divide N={w.N}")
         w = dataclasses.replace(w, block=args.block)
+    if args.clusters:
+        if not 1 <= args.clusters <= w.N:
+            raise SystemExit(f"--clusters must be in [1, N={w.N}]")
+        w = dataclasses.replace(w, Cq=args.clusters, Ck=args.clusters)
+    if args.iters:
+        w = dataclasses.replace(w, iters=args.iters)
+    if args.monopole and w.mode != "acausal":
+        raise SystemExit("--monopole applies to the acausal workloads")
     return w
 
 
@@ -310,8 +324,10 @@ def main():
     if w.mode == "acausal":
         ws = m.workspace("muse_forward", d, w.Cq, w.Ck)
 
+        flags = m.MUSE_FLAG_MONOPOLE if args.monopole else 0
+
         def step(Q=Qd, K=Kd, V=Vd, O=Od):
-            m.muse_forward(Q, K, V, w.Cq, w.Ck, w.iters, w.scale, out=O, ws=ws)
+            m.muse_forward_ex(Q, K, V, w.Cq, w.Ck, w.iters, w.scale, flags=flags, out=O, ws=ws)
     elif w.mode == "causal":
         ws = m.workspace("muse_causal_blocks", d, w.Cq, w.Ck, w.block)
 
@@ -443,7 +459,8 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic (seeded Gaussian-mixture Q/K, normal V)",
-            "config": config_of(w, graph is not None),
+            "config": dict(config_of(w, graph is not None),
+                           **({"monopole": True} if args.monopole else {})),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

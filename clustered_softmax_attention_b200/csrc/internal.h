@@ -85,8 +85,10 @@ cudaError_t run_summaries(const MuseTables &mt, int dtype, int D, int Dv, int P,
 cudaError_t run_tilt_weights(const MuseTables &mt, int dtype, int D, int P, float scale,
                              const float *q_centroids, SortedSide ks, const float *logZ, float *W,
                              cudaStream_t st);
+// sdip: the factor of the dipole terms (the logit scale, or 0 for the monopole only).
 cudaError_t run_coeffs(const MuseTables &mt, int dtype, int D, int P, float scale,
-                       SortedSide qs, const int32_t *q_offsets, StageBufs b, cudaStream_t st);
+                       SortedSide qs, const int32_t *q_offsets, StageBufs b, float sdip,
+                       cudaStream_t st);
 // Refinement: acausal writes O[p][row][:] (row = sequence row); partial mode writes
 // part_o[p][out0 + row][:] (float32) and part_lse[p][out0 + row].
 cudaError_t run_refine(const MuseTables &mt, int dtype, int D, int Dv, int N, int P,

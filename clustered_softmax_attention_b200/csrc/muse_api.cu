@@ -225,7 +225,8 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
                                const int32_t *q_perm, const int32_t *q_offsets,
                                const int32_t *k_perm, const int32_t *k_offsets,
                                const float *logZ_in, const float *mu_k_in, RefineWs &r, void *O,
-                               float *part_o, float *part_lse, cudaStream_t st) {
+                               float *part_o, float *part_lse, cudaStream_t st,
+                               bool monopole = false) {
   MUSE_TRY(run_sort_side(Q, d.dtype, d.D, d.N, mt.q, P, q_perm, q_offsets, q_centroids, r.qs, st));
   MUSE_TRY(run_sort_side(K, d.dtype, d.D, d.N, mt.k, P, k_perm, k_offsets, nullptr, r.ks, st));
   const bool use_tc = tc_supported(d.dtype, d.D, d.Dv);
@@ -244,7 +245,8 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
     MUSE_TRY(run_summaries(mt, d.dtype, d.D, d.Dv, P, d.scale, q_centroids, r.ks, nullptr,
                            k_offsets, sb, st));
   }
-  MUSE_TRY(run_coeffs(mt, d.dtype, d.D, P, d.scale, r.qs, q_offsets, sb, st));
+  // the dipole terms carry the logit scale; the monopole-only ablation drops them
+  MUSE_TRY(run_coeffs(mt, d.dtype, d.D, P, d.scale, r.qs, q_offsets, sb, monopole ? 0.f : d.scale, st));
   void *ev0 = g_prof_start.load(), *ev1 = g_prof_stop.load();
   if (ev0 && ev1) MUSE_TRY(record_profile_event(ev0, st));
   if (use_tc) {
@@ -368,7 +370,8 @@ extern "C" size_t muse_workspace_size(const char *entry, muse_dims d, int Cq, in
   if (!strcmp(entry, "muse_tilted_summaries"))
     return valid_C(Ck, d.N) ? ws_summaries(d, Cq, Ck, true, true) : 0;
   if (!strcmp(entry, "muse_dipole_refine")) return valid_C(Ck, d.N) ? ws_refine(d, Cq, Ck) : 0;
-  if (!strcmp(entry, "muse_forward")) return valid_C(Ck, d.N) ? ws_forward(d, Cq, Ck) : 0;
+  if (!strcmp(entry, "muse_forward") || !strcmp(entry, "muse_forward_ex"))
+    return valid_C(Ck, d.N) ? ws_forward(d, Cq, Ck) : 0;
   if (!strcmp(entry, "muse_causal_blocks")) {
     if (block <= 0 || block % 64 || d.N % block || Cq < 1 || Ck < 1 || Cq > kMaxClusters ||
         Ck > kMaxClusters)
@@ -484,11 +487,12 @@ extern "C" muse_status muse_dipole_refine(const void *Q, const void *K, const vo
 
 // --------------------------------------------------------------------------- forward
 
-extern "C" muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims d,
-                                    int Cq, int Ck, int iters, void *O, void *ws, size_t ws_bytes,
-                                    muse_stream_t st) {
+extern "C" muse_status muse_forward_ex(const void *Q, const void *K, const void *V, muse_dims d,
+                                       int Cq, int Ck, int iters, unsigned flags, void *O, void *ws,
+                                       size_t ws_bytes, muse_stream_t st) {
   muse_status s = check_dims(d, true);
   if (s != MUSE_OK) return s;
+  if (flags & ~(unsigned)MUSE_FLAG_MONOPOLE) return MUSE_ERR_INVALID_ARG;
   const void *ptrs[] = {Q, K, V, O};
   for (const void *p : ptrs)
     if (!p || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
@@ -512,7 +516,14 @@ extern "C" muse_status muse_forward(const void *Q, const void *K, const void *V,
                       cs) != cudaSuccess)
     return MUSE_ERR_CUDA;
   return refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets, kw.k.perm,
-                     kw.k.offsets, nullptr, nullptr, r, O, nullptr, nullptr, cs);
+                     kw.k.offsets, nullptr, nullptr, r, O, nullptr, nullptr, cs,
+                     (flags & MUSE_FLAG_MONOPOLE) != 0);
+}
+
+extern "C" muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims d,
+                                    int Cq, int Ck, int iters, void *O, void *ws, size_t ws_bytes,
+                                    muse_stream_t st) {
+  return muse_forward_ex(Q, K, V, d, Cq, Ck, iters, 0u, O, ws, ws_bytes, st);
 }
 
 // --------------------------------------------------------------------------- causal

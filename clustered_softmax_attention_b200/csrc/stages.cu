@@ -607,7 +607,8 @@ struct InstMask {
 // ---------------------------------------------------------------------------
 // Refinement coefficients for every sorted query position n of cluster i:
 //   a_j = logZ_ij + s u_j, u_j = qt.mu_k,ij;  p = softmax_j(a);
-//   c0[j][n] = p_j (1 - s u_j), c1[j][n] = s p_j,  lse[n] = logsumexp_j a_j.
+//   c0[j][n] = p_j (1 - sd u_j), c1[j][n] = sd p_j,  lse[n] = logsumexp_j a_j,
+// with sd = s (monopole and dipole) or sd = 0 (monopole only: c0 = p, c1 = 0).
 // CTA per (query cluster, task), one thread per query.
 // ---------------------------------------------------------------------------
 template <typename T, int D>
@@ -615,7 +616,7 @@ __global__ void __launch_bounds__(128)
 refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
               const int32_t *__restrict__ q_cluster, const float *__restrict__ logZ,
               const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
-              float *__restrict__ lse, int keep_u, BlockMap bm) {
+              float *__restrict__ lse, int keep_u, BlockMap bm, float sdip) {
   extern __shared__ float su[];  // [Ck][128] residual projections u_j (when keep_u)
   // blockIdx.x: a 128-row block of one instance (compact grid), blockIdx.y: the problem
   int bfirst;
@@ -666,8 +667,8 @@ refine_coeffs(MuseTables mt, float scale, const T *__restrict__ qt_rows,
       const float u = keep_u ? su[j * 128 + threadIdx.x] : proj(j);
       const float a = lz[j] + scale * u;
       const float pj = (a > -CUDART_INF_F) ? __expf(a - m) * inv : 0.f;
-      C0[(int64_t)j * cl + n] = pj * (1.f - scale * u);
-      C1[(int64_t)j * cl + n] = scale * pj;
+      C0[(int64_t)j * cl + n] = pj * (1.f - sdip * u);
+      C1[(int64_t)j * cl + n] = sdip * pj;
     }
     lse[q.lab + n] = m + logf(l);
   }
@@ -702,7 +703,7 @@ __global__ void __launch_bounds__(256)
 refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
                     const int32_t *__restrict__ q_offsets, const float *__restrict__ logZ,
                     const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
-                    float *__restrict__ lse, InstMask skip) {
+                    float *__restrict__ lse, InstMask skip, float sdip) {
   constexpr int CJ = 16 * JPT;                         // key clusters (all of them)
   constexpr int MSD = D + 4;                           // row stride of the means (floats)
   constexpr int QRB = D * (int)sizeof(T) + 16;         // row stride of the raw rows (bytes)
@@ -846,8 +847,8 @@ refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
       for (int u = 0; u < JPT; ++u) {
         const float av = lz[tj + 16 * u] + scale * acc[a][u];
         const float pj = av > -CUDART_INF_F ? __expf(av - m) * inv : 0.f;
-        acc[a][u] = pj * (1.f - scale * acc[a][u]);  // c0; c1 = s p is recomputed below
-        pv[a][u] = scale * pj;
+        acc[a][u] = pj * (1.f - sdip * acc[a][u]);  // c0
+        pv[a][u] = sdip * pj;                       // c1
       }
       const int n = r0 + 4 * tq + a;
       if (tj == 0 && n >= b && n < e) lse[q.lab + n] = m + logf(l);
@@ -907,7 +908,7 @@ __global__ void __launch_bounds__(256)
 refine_coeffs_grouped(MuseTables mt, float scale, const T *__restrict__ qt_rows,
                       const int32_t *__restrict__ q_offsets, const float *__restrict__ logZ,
                       const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
-                      float *__restrict__ lse, const __grid_constant__ BlockMap bm) {
+                      float *__restrict__ lse, const __grid_constant__ BlockMap bm, float sdip) {
   using Cf = CoefCfg<T, D, JPT>;
   constexpr int CJ = Cf::CJ, MSD = Cf::MSD, QRB = Cf::QRB;
   extern __shared__ float4 coef_smem[];
@@ -1040,8 +1041,8 @@ refine_coeffs_grouped(MuseTables mt, float scale, const T *__restrict__ qt_rows,
       const int j = tj + 16 * u;
       const float av = j < Ck ? lz[j] + scale * acc[u] : -CUDART_INF_F;
       const float pj = av > -CUDART_INF_F ? __expf(av - m) * inv : 0.f;
-      Cs[j * 17 + tr] = pj * (1.f - scale * acc[u]);
-      Cs[(CJ + j) * 17 + tr] = scale * pj;
+      Cs[j * 17 + tr] = pj * (1.f - sdip * acc[u]);
+      Cs[(CJ + j) * 17 + tr] = sdip * pj;
     }
     const int nr = min(16, cur.e - cur.r0);
     if (tj == 0 && tr < nr) lse[q.lab + cur.r0 + tr] = m + logf(l);
@@ -1349,7 +1350,7 @@ cudaError_t run_tilt_weights(const MuseTables &mt, int dtype, int D, int P, floa
 template <typename T, int D, int JPT>
 static cudaError_t coeffs_tiled_t(const MuseTables &mt, int P, float scale, SortedSide qs,
                                   const int32_t *q_offsets, StageBufs b, InstMask skip,
-                                  cudaStream_t st) {
+                                  float sdip, cudaStream_t st) {
   constexpr int CJ = 16 * JPT;
   const size_t smem = (size_t)CJ * (D + 4) * 4 + CJ * 4 + 64 * (D * sizeof(T) + 16);
   cudaError_t err = cudaFuncSetAttribute(refine_coeffs_tiled<T, D, JPT>,
@@ -1358,7 +1359,7 @@ static cudaError_t coeffs_tiled_t(const MuseTables &mt, int P, float scale, Sort
   // chunks of an instance: at most rows/64 + one partial chunk per cluster
   refine_coeffs_tiled<T, D, JPT><<<dim3((mt.q.max_rows + 63) / 64 + mt.q.max_C, P * mt.in.ninst), 256,
                                   smem, st>>>(
-      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse, skip);
+      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse, skip, sdip);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -1366,7 +1367,7 @@ static cudaError_t coeffs_tiled_t(const MuseTables &mt, int P, float scale, Sort
 template <typename T, int D, int JPT>
 static cudaError_t coeffs_grouped_t(const MuseTables &mt, int P, float scale, SortedSide qs,
                                     const int32_t *q_offsets, StageBufs b, InstMask skip,
-                                    cudaStream_t st) {
+                                    float sdip, cudaStream_t st) {
   using Cf = CoefCfg<T, D, JPT>;
   BlockMap bm;  // ceil(C / G) blocks per instance this kernel takes
   bm.pre[0] = 0;
@@ -1382,7 +1383,7 @@ static cudaError_t coeffs_grouped_t(const MuseTables &mt, int P, float scale, So
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::smem);
   if (err != cudaSuccess) return err;
   refine_coeffs_grouped<T, D, JPT><<<dim3(bm.total, P), 256, Cf::smem, st>>>(
-      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse, bm);
+      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse, bm, sdip);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -1392,7 +1393,8 @@ static cudaError_t coeffs_grouped_t(const MuseTables &mt, int P, float scale, So
 // the instances differ (the causal squares).
 template <typename T, int D, int JPT>
 static cudaError_t coeffs_split_t(const MuseTables &mt, int P, float scale, SortedSide qs,
-                                  const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
+                                  const int32_t *q_offsets, StageBufs b, float sdip,
+                                  cudaStream_t st) {
   InstMask small{}, large{};
   bool any_small = false, any_large = false;
   for (int si = 0; si < mt.in.ninst; ++si) {
@@ -1402,19 +1404,20 @@ static cudaError_t coeffs_split_t(const MuseTables &mt, int P, float scale, Sort
     any_large |= !sm;
   }
   cudaError_t err = cudaSuccess;
-  if (any_large) err = coeffs_tiled_t<T, D, JPT>(mt, P, scale, qs, q_offsets, b, large, st);
+  if (any_large) err = coeffs_tiled_t<T, D, JPT>(mt, P, scale, qs, q_offsets, b, large, sdip, st);
   if (err == cudaSuccess && any_small)
-    err = coeffs_grouped_t<T, D, JPT>(mt, P, scale, qs, q_offsets, b, small, st);
+    err = coeffs_grouped_t<T, D, JPT>(mt, P, scale, qs, q_offsets, b, small, sdip, st);
   return err;
 }
 
 template <typename T, int D>
 static cudaError_t coeffs_t(const MuseTables &mt, int P, float scale, SortedSide qs,
-                            const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
+                            const int32_t *q_offsets, StageBufs b, float sdip, cudaStream_t st) {
   // both forms stage each query cluster's tilted key means once in shared memory
-  if (mt.k.max_C <= 64) return coeffs_split_t<T, D, 4>(mt, P, scale, qs, q_offsets, b, st);
-  if (mt.k.max_C <= 128) return coeffs_split_t<T, D, 8>(mt, P, scale, qs, q_offsets, b, st);
-  if (mt.k.max_C <= 256 && D == 64) return coeffs_split_t<T, D, 16>(mt, P, scale, qs, q_offsets, b, st);
+  if (mt.k.max_C <= 64) return coeffs_split_t<T, D, 4>(mt, P, scale, qs, q_offsets, b, sdip, st);
+  if (mt.k.max_C <= 128) return coeffs_split_t<T, D, 8>(mt, P, scale, qs, q_offsets, b, sdip, st);
+  if (mt.k.max_C <= 256 && D == 64)
+    return coeffs_split_t<T, D, 16>(mt, P, scale, qs, q_offsets, b, sdip, st);
   const int keep_u = mt.k.max_C <= 256 ? 1 : 0;
   const size_t smem = keep_u ? (size_t)mt.k.max_C * 128 * sizeof(float) : 0;
   cudaError_t err = cudaFuncSetAttribute(refine_coeffs<T, D>,
@@ -1422,18 +1425,18 @@ static cudaError_t coeffs_t(const MuseTables &mt, int P, float scale, SortedSide
   if (err != cudaSuccess) return err;
   const BlockMap bm = make_block_map(mt.q, 128);
   refine_coeffs<T, D><<<dim3(bm.total, P), 128, smem, st>>>(
-      mt, scale, (const T *)qs.rows, qs.cluster, b.logZ, b.mu_k, b.c0, b.c1, b.lse, keep_u, bm);
+      mt, scale, (const T *)qs.rows, qs.cluster, b.logZ, b.mu_k, b.c0, b.c1, b.lse, keep_u, bm, sdip);
   count_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t run_coeffs(const MuseTables &mt, int dtype, int D, int P, float scale, SortedSide qs,
-                       const int32_t *q_offsets, StageBufs b, cudaStream_t st) {
+                       const int32_t *q_offsets, StageBufs b, float sdip, cudaStream_t st) {
   if (dtype == MUSE_F32)
-    return D == 64 ? coeffs_t<float, 64>(mt, P, scale, qs, q_offsets, b, st)
-                   : coeffs_t<float, 128>(mt, P, scale, qs, q_offsets, b, st);
-  return D == 64 ? coeffs_t<__nv_bfloat16, 64>(mt, P, scale, qs, q_offsets, b, st)
-                 : coeffs_t<__nv_bfloat16, 128>(mt, P, scale, qs, q_offsets, b, st);
+    return D == 64 ? coeffs_t<float, 64>(mt, P, scale, qs, q_offsets, b, sdip, st)
+                   : coeffs_t<float, 128>(mt, P, scale, qs, q_offsets, b, sdip, st);
+  return D == 64 ? coeffs_t<__nv_bfloat16, 64>(mt, P, scale, qs, q_offsets, b, sdip, st)
+                 : coeffs_t<__nv_bfloat16, 128>(mt, P, scale, qs, q_offsets, b, sdip, st);
 }
 
 template <typename T, int D, int DV>

@@ -45,6 +45,7 @@ _SIGS = {
     "muse_dipole_refine": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, MuseDims, _i, _i,
                            _vp, _vp, _sz, _vp],
     "muse_forward": [_vp, _vp, _vp, MuseDims, _i, _i, _i, _vp, _vp, _sz, _vp],
+    "muse_forward_ex": [_vp, _vp, _vp, MuseDims, _i, _i, _i, ctypes.c_uint, _vp, _vp, _sz, _vp],
     "muse_causal_levels": [_i, _i],
     "muse_causal_blocks": [_vp, _vp, _vp, MuseDims, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz,
                            _vp],
@@ -211,6 +212,23 @@ def muse_forward(Q, K, V, Cq: int, Ck: int, iters: int, scale: float = 1.0,
         ws = workspace("muse_forward", d, Cq, Ck)
     _check(lib().muse_forward(_p(Q), _p(K), _p(V), d, Cq, Ck, iters, _p(out), _p(ws), ws.numel(),
                               _stream()), "muse_forward")
+    return out
+
+
+MUSE_FLAG_MONOPOLE = 1
+
+
+def muse_forward_ex(Q, K, V, Cq: int, Ck: int, iters: int, scale: float = 1.0, flags: int = 0,
+                    out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+    """muse_forward with option flags (MUSE_FLAG_MONOPOLE: the monopole-only ablation)."""
+    _contig(Q, K, V, out, ws)
+    d = dims(Q, V, scale)
+    if out is None:
+        out = torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], d.Dv, dtype=Q.dtype, device=Q.device)
+    if ws is None:
+        ws = workspace("muse_forward_ex", d, Cq, Ck)
+    _check(lib().muse_forward_ex(_p(Q), _p(K), _p(V), d, Cq, Ck, iters, flags, _p(out), _p(ws),
+                                 ws.numel(), _stream()), "muse_forward_ex")
     return out
 
 

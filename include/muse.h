@@ -168,6 +168,21 @@ muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims 
                          muse_stream_t st);
 
 /*
+ * muse_forward_ex - muse_forward with option flags (0 = muse_forward).
+ *   MUSE_FLAG_MONOPOLE: the monopole-only ablation - the dipole term s C_ij qt is
+ *   dropped and O_n = sum_j p_j mu_v,ij with the same weights p_j = softmax_j(logZ_ij +
+ *   s qt.mu_k,ij) (pith.science review of arXiv 2509.10406, "invented entities": the
+ *   dipole correction, whose removal the paper's Table 3 measures).
+ * Same arguments, layouts, ownership and workspace as muse_forward
+ * (muse_workspace_size("muse_forward_ex", ...) = that of "muse_forward").  Unknown flag
+ * bits return MUSE_ERR_INVALID_ARG before anything is enqueued.
+ */
+#define MUSE_FLAG_MONOPOLE 1u
+muse_status muse_forward_ex(const void *Q, const void *K, const void *V, muse_dims d, int Cq,
+                            int Ck, int iters, unsigned flags, void *O, void *ws,
+                            size_t ws_bytes, muse_stream_t st);
+
+/*
  * muse_causal_levels - number of levels L of the causal decomposition of N rows
  * into blocks of `block` rows (levels with side block*2^(l-1) < N).
  */
@@ -218,7 +233,7 @@ muse_status muse_retrieve_exact(const void *Q, const void *K, const void *V, mus
 
 /*
  * muse_workspace_size - bytes of workspace `entry` needs ("muse_kmeans" with C = Cq,
- * "muse_tilted_summaries", "muse_dipole_refine", "muse_forward",
+ * "muse_tilted_summaries", "muse_dipole_refine", "muse_forward", "muse_forward_ex",
  * "muse_causal_blocks", "muse_retrieve_exact").  Arguments an entry does not
  * use are ignored.  Returns 0 for an unknown entry or invalid sizes.
  */

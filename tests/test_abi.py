@@ -15,7 +15,7 @@ def lib():
 def test_every_declared_entry_point_is_exported(lib):
     names = m.declared_entry_points()
     assert {"muse_kmeans", "muse_tilted_summaries", "muse_dipole_refine", "muse_forward",
-            "muse_causal_blocks", "muse_retrieve_exact", "muse_workspace_size",
+            "muse_forward_ex", "muse_causal_blocks", "muse_retrieve_exact", "muse_workspace_size",
             "muse_status_string", "muse_last_device_status", "muse_causal_levels"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
@@ -41,6 +41,8 @@ def test_workspace_sizes(lib):
     assert lib.muse_workspace_size(b"muse_forward", _d(D=32), 32, 32, 0, 0, 0) == 0
     assert lib.muse_workspace_size(b"muse_forward", d, 0, 32, 0, 0, 0) == 0
     assert lib.muse_workspace_size(b"muse_forward", d, 2048, 32, 0, 0, 0) == 0
+    assert (lib.muse_workspace_size(b"muse_forward_ex", d, 32, 32, 0, 0, 0)
+            == lib.muse_workspace_size(b"muse_forward", d, 32, 32, 0, 0, 0))
     # forward = two clusterings + refinement buffers: grows with N
     assert (lib.muse_workspace_size(b"muse_forward", _d(N=2048), 32, 32, 0, 0, 0)
             > lib.muse_workspace_size(b"muse_forward", d, 32, 32, 0, 0, 0))
@@ -86,3 +88,7 @@ def test_argument_validation_enqueues_nothing(lib):
     assert lib.muse_causal_blocks(f, f, f, _d(N=1000), 128, 8, 8, 2, f, None, None, f, 1 << 30,
                                   st) == 2
     assert lib.muse_causal_blocks(f, f, f, _d(), 128, 8, 8, 2, f, None, None, f, 0, st) == 4
+    # option flags: unknown bits are refused before the workspace is looked at
+    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 2, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 1, f, f, 16, st) == 4
+    assert lib.muse_forward_ex(f, f, f, _d(D=96), 8, 8, 2, 1, f, f, 1 << 30, st) == 2

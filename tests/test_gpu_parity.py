@@ -184,6 +184,27 @@ def test_forward_end_to_end_small_f32():
     assert mo.rse(O[0, 0], E) < 0.2
 
 
+# the monopole-only ablation (dipole term dropped) against the oracle's same mode, with
+# the GPU's clustering; it must be less accurate than the full method on these inputs
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_forward_monopole_only(dt):
+    N, C, T = 2048, 32, 6
+    Q, K, V = mixture(9, 1, 2, N, 64, 64, 48, 0.5 / 8, dt)
+    Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
+    Om = host(m.muse_forward_ex(Qd, Kd, Vd, C, C, T, 1.0, flags=m.MUSE_FLAG_MONOPOLE))
+    Od = host(m.muse_forward_ex(Qd, Kd, Vd, C, C, T, 1.0))
+    np.testing.assert_array_equal(Od, host(m.muse_forward(Qd, Kd, Vd, C, C, T, 1.0)))
+    ql, _, _, _ = m.muse_kmeans(Qd, C, T)
+    kl, _, _, _ = m.muse_kmeans(Kd, C, T)
+    Qf, Kf, Vf = host(Qd), host(Kd), host(Vd)
+    for h in range(2):
+        a = (Qf[0, h], Kf[0, h], Vf[0, h], ql[0, h].cpu().numpy(), kl[0, h].cpu().numpy(), C, C, 1.0)
+        ref_m = mo.muse_from_labels(*a, dipole=False)
+        assert mo.max_rel_err(Om[0, h], ref_m) <= TOL[dt]
+        E = mo.exact_attention(Qf[0, h], Kf[0, h], Vf[0, h], 1.0)
+        assert mo.rse(Od[0, h], E) < mo.rse(Om[0, h], E)
+
+
 def test_forward_bf16_multihead():
     Q, K, V = mixture(5, 2, 2, 2048, 64, 64, 64, 0.5 / 8, "bf16")
     Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
