@@ -279,6 +279,55 @@ def muse_from_labels(Q, K, V, q_labels, k_labels, Cq: int, Ck: int, scale: float
                   zero_residual=zero_residual, return_lse=return_lse, dipole=dipole)
 
 
+# ----------------------------------------------------------------------------
+# The partially specialised dipole ([review] "Axioms" / "ad hoc to paper": the
+# covariance of each key cluster is taken without the exponential tilt by the query
+# centroid, Cov_j(v,k) over the cluster's members, "aggregated per query cluster";
+# referee comment on Algorithm 3: it is Cov_j(v,k), not the tilted Cov_ij(v,k)).
+# The aggregation weights are not printed; the reading taken here weights cluster j
+# by the monopole softmax at the centroid, pi_ij = softmax_j(logZ_ij).
+# ----------------------------------------------------------------------------
+
+def key_cluster_covariances(K: np.ndarray, V: np.ndarray, k_labels: np.ndarray,
+                            n_kclusters: int) -> np.ndarray:
+    """Cov_j = (1/|S_j|) sum_{k in S_j} (v - vbar_j)(k - kbar_j)^T  [Ck, Dv, D]
+    (two-pass: means first; zero for an empty cluster)."""
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    out = np.zeros((n_kclusters, V.shape[1], K.shape[1]))
+    for j in range(n_kclusters):
+        idx = np.nonzero(k_labels == j)[0]
+        if idx.size == 0:
+            continue
+        kc = K[idx] - K[idx].mean(axis=0)
+        vc = V[idx] - V[idx].mean(axis=0)
+        out[j] = vc.T @ kc / idx.size
+    return out
+
+
+def muse_partial_dipole_from_labels(Q, K, V, q_labels, k_labels, Cq: int, Ck: int,
+                                    scale: float, qbar: Optional[np.ndarray] = None):
+    """O_n = sum_j p_j mu_v,ij + s Cbar_i qt_n, with p_j = softmax_j(logZ_ij + s qt.mu_k,ij)
+    (the monopole part of the full method) and Cbar_i = sum_j pi_ij Cov_j,
+    pi_ij = softmax_j(logZ_ij)."""
+    Q = np.asarray(Q, np.float64)
+    q_labels = np.asarray(q_labels)
+    if qbar is None:
+        qbar = cluster_means(Q, q_labels, Cq)
+    logZ, mu_k, mu_v, cov = tilted_summaries(qbar, K, V, k_labels, Ck, scale, want_cov=False)
+    O = refine(Q, q_labels, qbar, logZ, mu_k, mu_v, np.zeros((Cq, Ck, mu_v.shape[2], Q.shape[1])),
+               scale, dipole=False)
+    covs = key_cluster_covariances(K, V, k_labels, Ck)
+    for i in np.unique(q_labels):
+        m = logZ[i].max()
+        pi = np.exp(logZ[i] - m)          # exp(-inf) = 0 for empty clusters
+        pi /= pi.sum()
+        cbar = np.einsum("j,jvd->vd", pi, covs)
+        idx = np.nonzero(q_labels == i)[0]
+        O[idx] += scale * (Q[idx] - qbar[i][None, :]) @ cbar.T
+    return O
+
+
 def muse_acausal(Q, K, V, Cq: int, Ck: int, iters: int, scale: float,
                  return_labels: bool = False, dipole: bool = True):
     """Full acausal MuSe: K-means on Q and on K, summaries, refinement."""

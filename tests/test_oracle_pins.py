@@ -441,3 +441,54 @@ def test_retrieval_block_zero_uses_only_the_diagonal():
     O = mo.muse_retrieval(Q, K, V, 16, 3, 3, 2, k1=1, k2=1, scale=1.0)
     E0 = mo.exact_attention(Q[:16], K[:16], V[:16], 1.0, causal=True)
     np.testing.assert_allclose(O[:16], E0, rtol=1e-12)
+
+
+# --------------------------------------------------------------------------- partial dipole
+
+def test_partial_dipole_equals_full_when_the_centroid_is_zero():
+    """One query cluster whose centroid is 0 and one key cluster: the tilt by qbar = 0 is
+    uniform, so the tilted C_ij is the plain Cov_j and pi = 1; the partially specialised
+    dipole must then equal the full method (two different code paths)."""
+    rng = np.random.default_rng(31)
+    N, D, Dv, s = 40, 5, 3, 0.8
+    Q = 0.3 * rng.standard_normal((N, D))
+    Q -= Q.mean(axis=0)
+    K, V = rng.standard_normal((N, D)), rng.standard_normal((N, Dv))
+    ql, kl = np.zeros(N, np.int64), np.zeros(N, np.int64)
+    Op = mo.muse_partial_dipole_from_labels(Q, K, V, ql, kl, 1, 1, s)
+    Of = mo.muse_from_labels(Q, K, V, ql, kl, 1, 1, s)
+    np.testing.assert_allclose(Op, Of, rtol=1e-12, atol=1e-12)
+
+
+def test_key_cluster_covariance_is_numpy_cov():
+    """Cov_j against numpy's biased covariance of the stacked (v, k) members."""
+    rng = np.random.default_rng(32)
+    N, D, Dv = 50, 4, 3
+    K, V = rng.standard_normal((N, D)), rng.standard_normal((N, Dv))
+    kl = rng.integers(0, 3, N)
+    covs = mo.key_cluster_covariances(K, V, kl, 4)
+    for j in range(3):
+        idx = kl == j
+        full = np.cov(np.hstack([V[idx], K[idx]]).T, bias=True)
+        np.testing.assert_allclose(covs[j], full[:Dv, Dv:], rtol=1e-12, atol=1e-14)
+    assert (covs[3] == 0).all()
+
+
+def test_partial_dipole_is_first_order_in_the_centroid():
+    """The untilted covariance leaves an error linear in the query centroid (the pages'
+    O(qbar qt kt^2) bound): with one key cluster (so both weightings are 1), qt fixed and
+    qbar scaled, the partial dipole departs from the full one in proportion to qbar."""
+    rng = np.random.default_rng(33)
+    N, D, Dv = 60, 4, 3
+    base = rng.standard_normal(D)
+    noise = 0.05 * rng.standard_normal((N, D))
+    K, V = rng.standard_normal((N, D)), rng.standard_normal((N, Dv))
+    ql, kl = np.zeros(N, np.int64), np.zeros(N, np.int64)
+    diffs = []
+    for a in (1e-3, 1e-2, 1e-1):
+        Q = a * base[None, :] + noise - noise.mean(axis=0)
+        Op = mo.muse_partial_dipole_from_labels(Q, K, V, ql, kl, 1, 1, 1.0)
+        Of = mo.muse_from_labels(Q, K, V, ql, kl, 1, 1, 1.0)
+        diffs.append(np.abs(Op - Of).max())
+    slope = np.polyfit(np.log([1e-3, 1e-2, 1e-1]), np.log(diffs), 1)[0]
+    assert 0.8 <= slope <= 1.2, slope
