@@ -57,6 +57,8 @@ def parse():
                     help="K-means rounds override (default: the workload's)")
     ap.add_argument("--monopole", action="store_true",
                     help="acausal: the monopole-only ablation (dipole term dropped)")
+    ap.add_argument("--partial-dipole", action="store_true",
+                    help="acausal: the partially specialised dipole (untilted covariances)")
     return ap.parse_args()
 
 
@@ -75,8 +77,10 @@ def workload_of(args):
         w = dataclasses.replace(w, Cq=args.clusters, Ck=args.clusters)
     if args.iters:
         w = dataclasses.replace(w, iters=args.iters)
-    if args.monopole and w.mode != "acausal":
-        raise SystemExit("--monopole applies to the acausal workloads")
+    if (args.monopole or args.partial_dipole) and w.mode != "acausal":
+        raise SystemExit("--monopole and --partial-dipole apply to the acausal workloads")
+    if args.monopole and args.partial_dipole:
+        raise SystemExit("--monopole and --partial-dipole exclude each other")
     return w
 
 
@@ -322,9 +326,9 @@ def main():
     Oh = torch.empty_like(Od, device="cpu").pin_memory()
     d = m.dims(Qd, Vd, w.scale)
     if w.mode == "acausal":
-        ws = m.workspace("muse_forward", d, w.Cq, w.Ck)
-
-        flags = m.MUSE_FLAG_MONOPOLE if args.monopole else 0
+        ws = m.workspace("muse_forward_ex", d, w.Cq, w.Ck)
+        flags = (m.MUSE_FLAG_MONOPOLE if args.monopole else 0) | \
+            (m.MUSE_FLAG_PARTIAL_DIPOLE if args.partial_dipole else 0)
 
         def step(Q=Qd, K=Kd, V=Vd, O=Od):
             m.muse_forward_ex(Q, K, V, w.Cq, w.Ck, w.iters, w.scale, flags=flags, out=O, ws=ws)
@@ -460,7 +464,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic (seeded Gaussian-mixture Q/K, normal V)",
             "config": dict(config_of(w, graph is not None),
-                           **({"monopole": True} if args.monopole else {})),
+                           **({"monopole": True} if args.monopole else {}),
+                           **({"partial_dipole": True} if args.partial_dipole else {})),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

@@ -85,6 +85,13 @@ cudaError_t run_summaries(const MuseTables &mt, int dtype, int D, int Dv, int P,
 cudaError_t run_tilt_weights(const MuseTables &mt, int dtype, int D, int P, float scale,
                              const float *q_centroids, SortedSide ks, const float *logZ, float *W,
                              cudaStream_t st);
+// Partially specialised dipole (acausal tables): Cov_j per key cluster, Cbar_i per query
+// cluster, O += s Cbar_i qt.  ws holds P (Cq + Ck) D Dv floats.
+size_t partial_dipole_ws_floats(int P, int Cq, int Ck, int D, int Dv);
+cudaError_t run_partial_dipole(const MuseTables &mt, int dtype, int D, int Dv, int N, int P,
+                               float scale, SortedSide qs, const int32_t *q_perm, SortedSide ks,
+                               const void *V, const int32_t *k_perm, const int32_t *k_offsets,
+                               const float *logZ, float *ws, void *O, cudaStream_t st);
 // sdip: the factor of the dipole terms (the logit scale, or 0 for the monopole only).
 cudaError_t run_coeffs(const MuseTables &mt, int dtype, int D, int P, float scale,
                        SortedSide qs, const int32_t *q_offsets, StageBufs b, float sdip,

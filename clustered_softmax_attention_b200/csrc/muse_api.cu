@@ -332,6 +332,11 @@ static size_t ws_refine(const muse_dims &d, int Cq, int Ck) {
   return bp.off;
 }
 
+// the partially specialised dipole's covariances (after the forward pass's buffers)
+static size_t ws_partial_dipole(const muse_dims &d, int Cq, int Ck) {
+  return partial_dipole_ws_floats(d.B * d.H, Cq, Ck, d.D, d.Dv) * sizeof(float) + 256;
+}
+
 static size_t ws_forward(const muse_dims &d, int Cq, int Ck) {
   MuseTables mt;
   mt.q = whole_side(d.N, Cq);
@@ -370,8 +375,9 @@ extern "C" size_t muse_workspace_size(const char *entry, muse_dims d, int Cq, in
   if (!strcmp(entry, "muse_tilted_summaries"))
     return valid_C(Ck, d.N) ? ws_summaries(d, Cq, Ck, true, true) : 0;
   if (!strcmp(entry, "muse_dipole_refine")) return valid_C(Ck, d.N) ? ws_refine(d, Cq, Ck) : 0;
-  if (!strcmp(entry, "muse_forward") || !strcmp(entry, "muse_forward_ex"))
-    return valid_C(Ck, d.N) ? ws_forward(d, Cq, Ck) : 0;
+  if (!strcmp(entry, "muse_forward")) return valid_C(Ck, d.N) ? ws_forward(d, Cq, Ck) : 0;
+  if (!strcmp(entry, "muse_forward_ex"))
+    return valid_C(Ck, d.N) ? ws_forward(d, Cq, Ck) + ws_partial_dipole(d, Cq, Ck) : 0;
   if (!strcmp(entry, "muse_causal_blocks")) {
     if (block <= 0 || block % 64 || d.N % block || Cq < 1 || Ck < 1 || Cq > kMaxClusters ||
         Ck > kMaxClusters)
@@ -492,13 +498,15 @@ extern "C" muse_status muse_forward_ex(const void *Q, const void *K, const void 
                                        size_t ws_bytes, muse_stream_t st) {
   muse_status s = check_dims(d, true);
   if (s != MUSE_OK) return s;
-  if (flags & ~(unsigned)MUSE_FLAG_MONOPOLE) return MUSE_ERR_INVALID_ARG;
+  const unsigned known = MUSE_FLAG_MONOPOLE | MUSE_FLAG_PARTIAL_DIPOLE;
+  if ((flags & ~known) || (flags & known) == known) return MUSE_ERR_INVALID_ARG;
+  const bool partial = (flags & MUSE_FLAG_PARTIAL_DIPOLE) != 0;
   const void *ptrs[] = {Q, K, V, O};
   for (const void *p : ptrs)
     if (!p || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
   if (!valid_C(Cq, d.N) || !valid_C(Ck, d.N) || iters < 1 || iters > 1000)
     return MUSE_ERR_INVALID_ARG;
-  const size_t need = ws_forward(d, Cq, Ck);
+  const size_t need = ws_forward(d, Cq, Ck) + (partial ? ws_partial_dipole(d, Cq, Ck) : 0);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
   const int P = d.B * d.H;
   MuseTables mt;
@@ -510,14 +518,20 @@ extern "C" muse_status muse_forward_ex(const void *Q, const void *K, const void 
   plan_kmeans_pair(bp, mt, d, P, kw);
   RefineWs r;
   plan_refine(bp, mt, d, P, r, true);
+  float *pd_ws = partial ? bp.take<float>(partial_dipole_ws_floats(P, Cq, Ck, d.D, d.Dv)) : nullptr;
   cudaStream_t cs = (cudaStream_t)st;
   int *stat = status_ptr();
   if (run_kmeans_pair(Q, mt.q, kw.q, K, mt.k, kw.k, d.dtype, d.D, d.N, P, iters, kw.scratch, stat,
                       cs) != cudaSuccess)
     return MUSE_ERR_CUDA;
-  return refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets, kw.k.perm,
-                     kw.k.offsets, nullptr, nullptr, r, O, nullptr, nullptr, cs,
-                     (flags & MUSE_FLAG_MONOPOLE) != 0);
+  // the partially specialised dipole adds s Cbar_i qt to the monopole-only result
+  muse_status s2 = refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets,
+                               kw.k.perm, kw.k.offsets, nullptr, nullptr, r, O, nullptr, nullptr,
+                               cs, flags != 0);
+  if (s2 != MUSE_OK || !partial) return s2;
+  MUSE_TRY(run_partial_dipole(mt, d.dtype, d.D, d.Dv, d.N, P, d.scale, r.qs, kw.q.perm, r.ks, V,
+                              kw.k.perm, kw.k.offsets, r.sb.logZ, pd_ws, O, cs));
+  return MUSE_OK;
 }
 
 extern "C" muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims d,

@@ -216,11 +216,13 @@ def muse_forward(Q, K, V, Cq: int, Ck: int, iters: int, scale: float = 1.0,
 
 
 MUSE_FLAG_MONOPOLE = 1
+MUSE_FLAG_PARTIAL_DIPOLE = 2
 
 
 def muse_forward_ex(Q, K, V, Cq: int, Ck: int, iters: int, scale: float = 1.0, flags: int = 0,
                     out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
-    """muse_forward with option flags (MUSE_FLAG_MONOPOLE: the monopole-only ablation)."""
+    """muse_forward with option flags (MUSE_FLAG_MONOPOLE: the monopole-only ablation;
+    MUSE_FLAG_PARTIAL_DIPOLE: the partially specialised dipole)."""
     _contig(Q, K, V, out, ws)
     d = dims(Q, V, scale)
     if out is None:

@@ -173,11 +173,21 @@ muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims 
  *   dropped and O_n = sum_j p_j mu_v,ij with the same weights p_j = softmax_j(logZ_ij +
  *   s qt.mu_k,ij) (pith.science review of arXiv 2509.10406, "invented entities": the
  *   dipole correction, whose removal the paper's Table 3 measures).
- * Same arguments, layouts, ownership and workspace as muse_forward
- * (muse_workspace_size("muse_forward_ex", ...) = that of "muse_forward").  Unknown flag
- * bits return MUSE_ERR_INVALID_ARG before anything is enqueued.
+ *   MUSE_FLAG_PARTIAL_DIPOLE: the partially specialised dipole - the tilted C_ij is
+ *   replaced by the untilted covariance of each key cluster, Cov_j = mean over S_j of
+ *   (v - vbar_j)(k - kbar_j)^T, aggregated per query cluster with the weights
+ *   softmax_j(logZ_ij): O_n = sum_j p_j mu_v,ij + s (sum_j softmax_j(logZ_ij) Cov_j) qt_n
+ *   (same review: "Axioms", the covariance taken without the tilt by the query
+ *   centroid; "invented entities", an aggregated covariance per query cluster; the
+ *   weights are not printed, this is the reading taken).
+ * Same arguments, layouts and ownership as muse_forward.  Workspace: that of
+ * muse_forward, plus B*H*(Cq + Ck)*D*Dv floats and 256 bytes with
+ * MUSE_FLAG_PARTIAL_DIPOLE; muse_workspace_size("muse_forward_ex", ...) returns that
+ * larger size.  Unknown flag bits, or both flags at once, return MUSE_ERR_INVALID_ARG
+ * before anything is enqueued.
  */
 #define MUSE_FLAG_MONOPOLE 1u
+#define MUSE_FLAG_PARTIAL_DIPOLE 2u
 muse_status muse_forward_ex(const void *Q, const void *K, const void *V, muse_dims d, int Cq,
                             int Ck, int iters, unsigned flags, void *O, void *ws,
                             size_t ws_bytes, muse_stream_t st);

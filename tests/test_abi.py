@@ -41,8 +41,10 @@ def test_workspace_sizes(lib):
     assert lib.muse_workspace_size(b"muse_forward", _d(D=32), 32, 32, 0, 0, 0) == 0
     assert lib.muse_workspace_size(b"muse_forward", d, 0, 32, 0, 0, 0) == 0
     assert lib.muse_workspace_size(b"muse_forward", d, 2048, 32, 0, 0, 0) == 0
+    # forward_ex: the forward pass's buffers plus the partially specialised dipole's
+    # covariances, B*H*(Cq+Ck)*D*Dv floats and 256 bytes
     assert (lib.muse_workspace_size(b"muse_forward_ex", d, 32, 32, 0, 0, 0)
-            == lib.muse_workspace_size(b"muse_forward", d, 32, 32, 0, 0, 0))
+            == lib.muse_workspace_size(b"muse_forward", d, 32, 32, 0, 0, 0) + 2 * 64 * 64 * 64 * 4 + 256)
     # forward = two clusterings + refinement buffers: grows with N
     assert (lib.muse_workspace_size(b"muse_forward", _d(N=2048), 32, 32, 0, 0, 0)
             > lib.muse_workspace_size(b"muse_forward", d, 32, 32, 0, 0, 0))
@@ -89,6 +91,7 @@ def test_argument_validation_enqueues_nothing(lib):
                                   st) == 2
     assert lib.muse_causal_blocks(f, f, f, _d(), 128, 8, 8, 2, f, None, None, f, 0, st) == 4
     # option flags: unknown bits are refused before the workspace is looked at
-    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 2, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 4, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 3, f, f, 1 << 30, st) == 1
     assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 1, f, f, 16, st) == 4
     assert lib.muse_forward_ex(f, f, f, _d(D=96), 8, 8, 2, 1, f, f, 1 << 30, st) == 2

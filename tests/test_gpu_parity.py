@@ -205,6 +205,23 @@ def test_forward_monopole_only(dt):
         assert mo.rse(Od[0, h], E) < mo.rse(Om[0, h], E)
 
 
+# the partially specialised dipole (untilted key-cluster covariances aggregated per query
+# cluster) against the oracle's same reading, with the GPU's clustering
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_forward_partial_dipole(dt):
+    N, C, T = 2048, 32, 6
+    Q, K, V = mixture(10, 1, 2, N, 64, 64, 48, 0.5 / 8, dt)
+    Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
+    Op = host(m.muse_forward_ex(Qd, Kd, Vd, C, C, T, 1.0, flags=m.MUSE_FLAG_PARTIAL_DIPOLE))
+    ql, _, _, _ = m.muse_kmeans(Qd, C, T)
+    kl, _, _, _ = m.muse_kmeans(Kd, C, T)
+    Qf, Kf, Vf = host(Qd), host(Kd), host(Vd)
+    for h in range(2):
+        ref = mo.muse_partial_dipole_from_labels(Qf[0, h], Kf[0, h], Vf[0, h], ql[0, h].cpu().numpy(),
+                                                 kl[0, h].cpu().numpy(), C, C, 1.0)
+        assert mo.max_rel_err(Op[0, h], ref) <= TOL[dt]
+
+
 def test_forward_bf16_multihead():
     Q, K, V = mixture(5, 2, 2, 2048, 64, 64, 64, 0.5 / 8, "bf16")
     Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
