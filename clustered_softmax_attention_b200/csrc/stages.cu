@@ -339,7 +339,10 @@ __device__ __forceinline__ void tilt_unpack(const uint4 u, float *o) {  // 8 bf1
 }
 
 struct TiltStep {
-  int j, b, e, pc, pass;  // pass 0: the whole cluster in one chunk; 1, 2: first, second pass
+  // clusters j .. je-1, keys [b, e), chunk start pc; pass 0: one cluster in one chunk;
+  // 1, 2: first, second pass over a larger cluster; 3: a window of several whole
+  // clusters that fit in one chunk together
+  int j, je, b, e, pc, pass;
 };
 
 template <typename T, int D>
@@ -356,6 +359,8 @@ tilt_fused(MuseTables mt, float scale, const float *__restrict__ qcen, const T *
   float *Ws = Ks + KC * QS;                           // [KC][WS] the chunk's weights
   uint4 *Kr = reinterpret_cast<uint4 *>(Ws + KC * WS); // [1024] raw 16-byte units of a chunk
   __shared__ int offs[Cf::GMAX + 1];
+  __shared__ float LZs[Cf::GMAX * 64];  // window steps: logZ per (cluster, centroid)
+  __shared__ unsigned char segk[KC];    // window steps: cluster of each key of the chunk
   int bfirst;
   const int p = blockIdx.z, s = map_block(bm, mt.in.ninst, blockIdx.x, bfirst);
   const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
@@ -424,13 +429,24 @@ tilt_fused(MuseTables mt, float scale, const float *__restrict__ qcen, const T *
     }
     TiltStep t;
     t.j = j;
+    t.je = j + 1;
     t.b = j < j1 ? offs[j - j0] : 0;
     t.e = j < j1 ? offs[j - j0 + 1] : 0;
     t.pc = t.b;
     t.pass = t.e - t.b > KC ? 1 : 0;
+    if (j < j1 && t.pass == 0) {  // the following clusters that fit in the same chunk
+      int je = j + 1;
+      while (je < j1 && offs[je + 1 - j0] - t.b <= KC) ++je;
+      if (je - j >= 2) {
+        t.je = je;
+        t.e = offs[je - j0];
+        t.pass = 3;
+      }
+    }
     return t;
   };
   auto advance = [&](TiltStep t) {
+    if (t.pass == 3) return open(t.je);
     if (t.pc + KC < t.e) {
       t.pc += KC;
       return t;
@@ -440,7 +456,7 @@ tilt_fused(MuseTables mt, float scale, const float *__restrict__ qcen, const T *
       t.pc = t.b;
       return t;
     }
-    return open(t.j + 1);
+    return open(t.je);
   };
   // each thread copies, and later converts, the same four 16-byte units of a chunk
   auto fetch = [&](const TiltStep &t) {
@@ -474,6 +490,11 @@ tilt_fused(MuseTables mt, float scale, const float *__restrict__ qcen, const T *
         *reinterpret_cast<uint4 *>(dst) = raw;
       }
     }
+    if (cur.pass == 3 && tid < pt) {  // cluster of each key of the window
+      int cl = 0;
+      while (offs[cur.j + cl + 1 - j0] - cur.b <= tid) ++cl;
+      segk[tid] = (unsigned char)cl;
+    }
     const TiltStep nxt = advance(cur);
     if (nxt.j < j1) fetch(nxt);
     __syncthreads();
@@ -506,6 +527,64 @@ tilt_fused(MuseTables mt, float scale, const float *__restrict__ qcen, const T *
       for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int c = 0; c < NC; ++c) L[a][c] = td + 16 * c < pt ? scale * L[a][c] : -CUDART_INF_F;
+      if (cur.pass == 3) {
+        // a window of whole clusters: the logits go through shared memory, logZ per
+        // (cluster, centroid) by a scan of the cluster's keys, then the weights and one
+        // tilted mean per cluster from the same key tile
+        const int ncl = cur.je - cur.j;
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+          *reinterpret_cast<float4 *>(Ws + (td + 16 * c) * WS + 4 * ti) =
+              make_float4(L[0][c], L[1][c], L[2][c], L[3][c]);
+        __syncthreads();
+        for (int x = tid; x < 64 * ncl; x += 256) {
+          const int il = x & 63, cl = x >> 6;
+          const int kb = offs[cur.j + cl - j0] - cur.b, ke = offs[cur.j + cl + 1 - j0] - cur.b;
+          float mx = -CUDART_INF_F;
+          for (int kk = kb; kk < ke; ++kk) mx = fmaxf(mx, Ws[kk * WS + il]);
+          float sm = 0.f;
+          for (int kk = kb; kk < ke; ++kk) sm += expf(Ws[kk * WS + il] - mx);
+          LZs[cl * 64 + il] = ke > kb ? mx + logf(sm) : -CUDART_INF_F;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          const int kk = td + 16 * c;
+          const int cl = kk < pt ? segk[kk] : 0;
+          float w[4];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            w[a] = kk < pt ? expf(L[a][c] - LZs[cl * 64 + ti * 4 + a]) : 0.f;
+            if (kk < pt && i0 + ti * 4 + a < Cq) wb[(int64_t)(i0 + ti * 4 + a) * wl + cur.b + kk] = w[a];
+          }
+          *reinterpret_cast<float4 *>(Ws + kk * WS + 4 * ti) = make_float4(w[0], w[1], w[2], w[3]);
+        }
+        __syncthreads();
+        for (int cl = 0; cl < ncl; ++cl) {
+          const int kb = offs[cur.j + cl - j0] - cur.b, ke = offs[cur.j + cl + 1 - j0] - cur.b;
+          clear_acc();
+          for (int pp = kb; pp < ke; ++pp) {
+            const float4 wv = *reinterpret_cast<const float4 *>(Ws + pp * WS + 4 * ti);
+            const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+            for (int h = 0; h < PQ; ++h) {
+              const float4 kv = *reinterpret_cast<const float4 *>(Ks + pp * QS + 64 * h + 4 * td);
+#pragma unroll
+              for (int a = 0; a < 4; ++a) {
+                acc[a][h][0] = fmaf(wa[a], kv.x, acc[a][h][0]);
+                acc[a][h][1] = fmaf(wa[a], kv.y, acc[a][h][1]);
+                acc[a][h][2] = fmaf(wa[a], kv.z, acc[a][h][2]);
+                acc[a][h][3] = fmaf(wa[a], kv.w, acc[a][h][3]);
+              }
+            }
+          }
+          float lzw[4];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) lzw[a] = LZs[cl * 64 + ti * 4 + a];
+          put(cur.j + cl, lzw, acc);
+        }
+        return;
+      }
       if (cur.pass != 2) {  // running maximum and sum of exp over the cluster's keys
 #pragma unroll
         for (int a = 0; a < 4; ++a) {

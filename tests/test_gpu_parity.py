@@ -123,14 +123,16 @@ def test_summaries_and_refine_vs_oracle(dt):
 
 
 # logZ and mu_k alone take the one-launch tilt kernel: key clusters of 0, 1, 15-17, 64-65,
-# 127-129 and 300 keys (one chunk, several chunks, several clusters per CTA), 70 centroids
-# (a ragged second group of 64), given directly as a permutation and offsets.
+# 127-129 and 300 keys (one chunk, several chunks, several clusters per CTA, windows of
+# whole clusters with an empty one inside), 70 centroids (a ragged second group of 64),
+# given directly as a permutation and offsets; Ck = 128 makes most clusters a few keys.
 @pytest.mark.parametrize("dt,D,Ck", [("bf16", 64, 16), ("bf16", 64, 40), ("f32", 64, 40),
-                                      ("bf16", 128, 40), ("f32", 128, 16)])
+                                      ("bf16", 128, 40), ("f32", 128, 16), ("bf16", 64, 128),
+                                      ("f32", 128, 128)])
 def test_key_means_cluster_layouts(dt, D, Ck):
     rng = np.random.Generator(np.random.PCG64(100 + Ck + D))
     N, Cq, s = 1200, 70, 0.35
-    fixed = [300, 0, 1, 15, 16, 17, 64, 65, 127, 128, 129, 0]
+    fixed = [300, 0, 1, 15, 0, 16, 17, 64, 65, 127, 128, 129, 0]
     rest = Ck - len(fixed)
     left = N - sum(fixed)
     if rest > 0:
