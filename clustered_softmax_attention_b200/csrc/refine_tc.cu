@@ -15,16 +15,17 @@
 // key/value tile the producer also stages, by cp.async into the same stage, the tile's
 // tilt weights for up to 8 query clusters of the CTA and the tile's coefficients
 // c0, c1 for the CTA's 128 rows.
-//   S  = Qt . K_tile^T            (tcgen05, 128 x npad, fp32 in TMEM, double-buffered)
-//   P  = w .* (c0 + c1 .* S)      (epilogue warps: TMEM -> registers -> bf16 TMEM)
+//   S  = Qt . K_tile^T            (tcgen05, 128 x npad, fp32 in TMEM, three buffers)
+//   P  = w .* (c0 + c1 .* S)      (epilogue warps: TMEM -> registers -> bf16 TMEM, written
+//                                  over S(t) in its own buffer, two per column)
 //   O += P . V_tile               (tcgen05, A = P from TMEM, 128 x Dv, fp32 in TMEM)
-// TMEM columns: S double buffer [0, 2 BN), P ring of three [2 BN, 3.5 BN) (bf16 packed
-// two per column), O [3.5 BN, 3.5 BN + Dv).
+// TMEM columns: S/P buffers [0, 3 BN) (tile t uses buffer t % 3; it takes S(t + 3) once
+// O += P(t) V has completed), O [3 BN, 3 BN + Dv).
 // Warp roles: warp 0 = TMA producer of the key tiles, warp 12 = of the value tiles
 // (each stage released as soon as its MMA has consumed it), warp 1 = MMA issuer
 // (+ TMEM owner), warps 2-9 = epilogue
 // in two groups of four (TMEM lane quadrant = warp % 4): group g takes the tiles of
-// parity g, i.e. S/P buffer g, so the groups overlap; warps 10-11 = cp.async producers
+// parity g, so the groups overlap; warps 10-11 = cp.async producers
 // of the epilogue data (tiles of parity 0 and 1).  Every wait on an mbarrier is
 // bounded: past the limit the kernel records MUSE_ERR_TIMEOUT and winds down.
 #include <cuda.h>
@@ -44,7 +45,7 @@ constexpr int kVWarp = kEWarp + 2;                  // value-tile TMA producer
 constexpr int kSlots = 8;    // query clusters per CTA whose tilt weights are staged
 constexpr int kTileSegs = 8; // key clusters packed into one tile at most
 constexpr int kComplex = 1 << 13;  // chunk code flag: more than two key clusters in 16 columns
-constexpr int kPBuf = 3;     // P buffers (tile t uses t % 3): P(t) waits only for O += P(t-3) V
+constexpr int kSBuf = 3;     // S buffers (tile t uses t % 3); P(t) is written over S(t) in place
 
 // Widest key tile: 128 keys when D = Dv = 64, else 64 (shared memory budget).
 template <int D, int DV>
@@ -68,7 +69,8 @@ struct __align__(1024) Smem {
   // per stage: key tile (consumed by the first MMA), values (second MMA), epilogue
   // data (tilt weights, coefficients, segment map; consumed by the epilogue)
   uint64_t fullk[NST], emptyk[NST], fullv[NST], emptyv[NST], fulle[NST], emptye[NST];
-  uint64_t sfull[2], sfree[2], pready[kPBuf], pfree[kPBuf], qbar, obar;
+  // S(t) in TMEM; P(t) over it; O += P(t) V done (the buffer is free again)
+  uint64_t sfull[kSBuf], pready[kSBuf], spfree[kSBuf], qbar, obar;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -177,13 +179,10 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       mbar_init(&sm.fulle[i], 1 + 32);  // lane 0 arrive + one cp.async arrival per lane
       mbar_init(&sm.emptye[i], kEpiWarps / 2);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSBuf; ++i) {
       mbar_init(&sm.sfull[i], 1);
-      mbar_init(&sm.sfree[i], kEpiWarps / 2);   // one warp group per buffer
-    }
-    for (int i = 0; i < kPBuf; ++i) {
-      mbar_init(&sm.pready[i], kEpiWarps / 2);
-      mbar_init(&sm.pfree[i], 1);
+      mbar_init(&sm.pready[i], kEpiWarps / 2);  // the four warps of the tile's group
+      mbar_init(&sm.spfree[i], 1);
     }
     mbar_init(&sm.qbar, 1);
     mbar_init(&sm.obar, 1);
@@ -202,9 +201,8 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t tmem_o = tmem + 2 * BN + kPBuf * (BN / 2);
-  auto s_col = [](int buf) { return (uint32_t)(buf * BN); };
-  auto p_col = [](int buf) { return (uint32_t)(2 * BN + buf * (BN / 2)); };
+  const uint32_t tmem_o = tmem + kSBuf * BN;
+  auto s_col = [](int buf) { return (uint32_t)(buf * BN); };  // S(t) and, over it, P(t)
   const int32_t *koff = sm.koff;
   const int kcol0 = (int)(k.lab - (int64_t)p * mt.k.row_stride);  // instance's first key column
   const int wl = w_ld(k.n), cl = w_ld(q.n);
@@ -343,8 +341,9 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       while (ok && (!it.done() || g2 < g1)) {
         bool progressed = false;
         if (!it.done()) {
-          const int st = g1 % NST, buf = g1 & 1;
-          if ((g1 < 2 || mbar_test(&sm.sfree[buf], ((g1 - 2) >> 1) & 1)) &&
+          const int st = g1 % NST, buf = g1 % kSBuf;
+          // the buffer's previous tile has gone through O += P V
+          if ((g1 < kSBuf || mbar_test(&sm.spfree[buf], ((g1 / kSBuf) - 1) & 1)) &&
               mbar_test(&sm.fullk[st], (g1 / NST) & 1)) {
             tc_fence_after();
             const KTile kt = it.get();
@@ -363,16 +362,16 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           }
         }
         if (g2 < g1) {
-          const int st = g2 % NST, pb = g2 % kPBuf;
-          if (mbar_test(&sm.pready[pb], (g2 / kPBuf) & 1) && mbar_test(&sm.fullv[st], (g2 / NST) & 1)) {
+          const int st = g2 % NST, pb = g2 % kSBuf;
+          if (mbar_test(&sm.pready[pb], (g2 / kSBuf) & 1) && mbar_test(&sm.fullv[st], (g2 / NST) & 1)) {
             tc_fence_after();
             const uint32_t id = idesc(BM, DV);
             const int npad = sm.tnpad[g2 & 3];
             for (int kk = 0; kk < npad / 16; ++kk) {
               const uint64_t b = sdesc(sm.vt[st][kk >> 2] + (kk & 3) * 16);
-              tc_mma_ts(tmem_o, tmem + p_col(pb) + kk * 8, b, id, (g2 > 0 || kk > 0) ? 1u : 0u);
+              tc_mma_ts(tmem_o, tmem + s_col(pb) + kk * 8, b, id, (g2 > 0 || kk > 0) ? 1u : 0u);
             }
-            tc_commit(&sm.pfree[pb]);
+            tc_commit(&sm.spfree[pb]);
             tc_commit(&sm.emptyv[st]);
             ++g2;
             progressed = true;
@@ -421,10 +420,10 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     for (; !it.done(); it.next(), ++t) {
       if ((t & 1) != grp) continue;
       const KTile kt = it.get();
-      const int buf = t & 1, st = t % NST;
+      const int buf = t % kSBuf, st = t % NST;
       // (a wait that gave up in one lane stops the whole warp: the TMEM accesses below
       // are warp-collective)
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.sfull[buf], (t >> 1) & 1, abort_flag, status) &&
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.sfull[buf], (t / kSBuf) & 1, abort_flag, status) &&
                                        mbar_wait(&sm.fulle[st], (t / NST) & 1, abort_flag, status))) {
         ok = false;
         break;
@@ -432,14 +431,11 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       tc_fence_after();
       const float *wsm = &sm.w[st][staged ? slot : 0][0];
       const int nch16 = kt.npad / 16;
-      const int pb = t % kPBuf;
-      // P(t) overwrites P(t-3): wait until the MMA reading that has completed
-      if (t >= kPBuf &&
-          !__all_sync(0xffffffffu, mbar_wait(&sm.pfree[pb], ((t / kPBuf) - 1) & 1, abort_flag, status))) {
-        ok = false;
-        break;
-      }
-      // P for 16 columns of S held in x, stored as 8 packed bf16 columns of buffer pb
+      // P for 16 columns of S held in x, stored as 8 packed bf16 columns over the same
+      // buffer: chunk cb's P lands in S columns 8 cb .. 8 cb + 7, which belong to S chunk
+      // cb / 2, already read (and waited for) by this thread; the load in flight is of
+      // chunk cb + 1, columns 16 cb + 16 on
+
       auto chunk = [&](int cb, const uint32_t(&x)[16]) {
         const int code = sm.chunk[st][cb];
         uint32_t pk[8];
@@ -491,23 +487,13 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
           for (int e = 0; e < 8; ++e) pk[e] = pr.v[e];
         }
-        tmem_st8(tmem + lane_base + p_col(pb) + cb * 8, pk);
+        tmem_st8(tmem + lane_base + s_col(buf) + cb * 8, pk);
       };
       // S chunks alternate between two register sets: the load of chunk cb+1 is in
       // flight while chunk cb is processed
       uint32_t xa[16], xb[16];
       int nl = 1;  // chunks whose load has been issued
-      bool freed = false;
-      auto landed = [&]() {
-        tmem_ld_wait();
-        if (!freed && nl == nch16) {
-          // all of S read: its buffer can take the group's next tile while P is written
-          freed = true;
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.sfree[buf]);
-        }
-      };
+      auto landed = [&]() { tmem_ld_wait(); };
       tmem_ld16_async(tmem + lane_base + s_col(buf), xa);
       landed();
       for (int cb = 0; cb < nch16; cb += 2) {
@@ -524,7 +510,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sm.pready[pb]);
+        mbar_arrive(&sm.pready[buf]);
         mbar_arrive(&sm.emptye[st]);  // the tile's epilogue data is consumed
       }
     }
