@@ -30,24 +30,34 @@ __device__ __forceinline__ Task k_task(const MuseTables &mt, int p, int s) {
 // ---------------------------------------------------------------------------
 // Sorted copies: position m of a task's perm holds row perm[m] (minus its
 // cluster's centroid when `centroids` is given: the query residuals).
-// One CTA per (cluster, task).
+// One CTA per 64 sorted positions of a task (compact grid); a position's cluster is
+// the last one whose offset is <= it (a binary search over the task's offsets).
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256)
 sort_side(const T *__restrict__ X, int N, int W, SegTable tab, const int32_t *__restrict__ perm,
           const int32_t *__restrict__ offsets, const float *__restrict__ centroids,
-          T *__restrict__ rows, int32_t *__restrict__ cluster) {
+          T *__restrict__ rows, int32_t *__restrict__ cluster, const __grid_constant__ BlockMap bm) {
   constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte vector
-  const Task tk = make_task(tab, blockIdx.y);
-  const int c = blockIdx.x;
-  if (c >= tk.C) return;
-  const int b = offsets[tk.off + c], e = offsets[tk.off + c + 1];
+  int bfirst;
+  const int sg = map_block(bm, tab.nseg, blockIdx.x, bfirst);
+  const Task tk = make_task(tab, blockIdx.y * tab.nseg + sg);
+  const int m0 = ((int)blockIdx.x - bfirst) * 64, m1 = min(m0 + 64, tk.n);
+  if (m0 >= tk.n) return;
+  const int32_t *off = offsets + tk.off;
   const int vpr = W / VEC, slots = 256 / vpr;
   const int v = threadIdx.x % vpr, slot = threadIdx.x / vpr;
-  float cv[VEC];
+  for (int m = m0 + slot; m < m1; m += slots) {
+    int lo = 0, hi = tk.C - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(off + mid) <= m) lo = mid;
+      else hi = mid - 1;
+    }
+    const int c = lo;
+    float cv[VEC];
 #pragma unroll
-  for (int u = 0; u < VEC; ++u) cv[u] = centroids ? centroids[(tk.cen + c) * W + v * VEC + u] : 0.f;
-  for (int m = b + slot; m < e; m += slots) {
+    for (int u = 0; u < VEC; ++u) cv[u] = centroids ? centroids[(tk.cen + c) * W + v * VEC + u] : 0.f;
     const int row = perm[tk.lab + m];
     uint4 raw = *reinterpret_cast<const uint4 *>(X + ((int64_t)tk.p * N + row) * W + v * VEC);
     if (centroids) {
@@ -1294,16 +1304,18 @@ diag_merge(const T *__restrict__ Qg, const T *__restrict__ Kg, const T *__restri
 cudaError_t run_sort_side(const void *X, int dtype, int width, int N, const SegTable &tab, int P,
                           const int32_t *perm, const int32_t *offsets, const float *centroids,
                           SortedSide out, cudaStream_t st) {
-  dim3 grid(tab.max_C, P * tab.nseg);
+  const BlockMap bm = make_block_map(tab, 64);
+  if (bm.total == 0) return cudaSuccess;
+  dim3 grid(bm.total, P);
   const int threads = 256;
   count_launches(1);
   if (dtype == MUSE_F32)
     sort_side<float><<<grid, threads, 0, st>>>((const float *)X, N, width, tab, perm, offsets,
-                                               centroids, (float *)out.rows, out.cluster);
+                                               centroids, (float *)out.rows, out.cluster, bm);
   else
     sort_side<__nv_bfloat16><<<grid, threads, 0, st>>>(
         (const __nv_bfloat16 *)X, N, width, tab, perm, offsets, centroids,
-        (__nv_bfloat16 *)out.rows, out.cluster);
+        (__nv_bfloat16 *)out.rows, out.cluster, bm);
   return cudaGetLastError();
 }
 
