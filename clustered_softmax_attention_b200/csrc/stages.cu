@@ -86,10 +86,14 @@ sort_side_t(const T *__restrict__ X, int N, SegTable tab, const int32_t *__restr
   if (m0 >= tk.n) return;
   __shared__ T buf[64][W + 2];
   const int mt = min(64, tk.n - m0);
-  for (int e = threadIdx.x; e < mt * W; e += blockDim.x) {
-    const int mm = e / W, c = e % W;
+  constexpr int VEC = 16 / sizeof(T), VPR = W / VEC;  // 16-byte vectors per row
+  for (int e = threadIdx.x; e < mt * VPR; e += blockDim.x) {
+    const int mm = e / VPR, cv = e % VPR;
     const int row = perm[tk.lab + m0 + mm];
-    buf[mm][c] = X[((int64_t)tk.p * N + row) * W + c];
+    const uint4 raw = *reinterpret_cast<const uint4 *>(X + ((int64_t)tk.p * N + row) * W + cv * VEC);
+    const T *el = reinterpret_cast<const T *>(&raw);
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) buf[mm][cv * VEC + u] = el[u];
   }
   __syncthreads();
   const int ld = vt_ld(tab.row_stride);
