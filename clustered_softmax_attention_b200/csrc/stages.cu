@@ -946,25 +946,22 @@ refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
       const int n = r0 + 4 * tq + a;
       if (tj == 0 && n >= b && n < e) lse[q.lab + n] = m + logf(l);
     }
-    // rows n0 .. n0+3 of every cluster j this thread holds
-    const int n0 = r0 + 4 * tq;
-    const bool full = n0 >= b && n0 + 3 < e;
+    // c0, then c1, through shared memory (the means' space, free after the products):
+    // every key cluster's rows of the chunk leave as one contiguous run
+    float *Cs = Ms;  // [CJ][65]
+    const int lo = max(b, r0) - r0, hi = min(e, r0 + 64) - r0;  // the chunk's rows of cluster i
 #pragma unroll
-    for (int u = 0; u < JPT; ++u) {
-      const int j = tj + 16 * u;
-      if (j >= Ck) break;
-      float *d0 = C0 + (int64_t)j * cl + n0;
-      float *d1 = C1 + (int64_t)j * cl + n0;
-      if (full) {
-        *reinterpret_cast<float4 *>(d0) = make_float4(acc[0][u], acc[1][u], acc[2][u], acc[3][u]);
-        *reinterpret_cast<float4 *>(d1) = make_float4(pv[0][u], pv[1][u], pv[2][u], pv[3][u]);
-      } else {
+    for (int half = 0; half < 2; ++half) {
+      __syncthreads();  // the products (first half) or the previous stores are done
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-          if (n0 + a >= b && n0 + a < e) {
-            d0[a] = acc[a][u];
-            d1[a] = pv[a][u];
-          }
+      for (int u = 0; u < JPT; ++u)
+#pragma unroll
+        for (int a = 0; a < 4; ++a) Cs[(tj + 16 * u) * 65 + 4 * tq + a] = half ? pv[a][u] : acc[a][u];
+      __syncthreads();
+      float *dst = half ? C1 : C0;
+      for (int x = threadIdx.x; x < Ck * 64; x += 256) {
+        const int j = x >> 6, rr = x & 63;
+        if (rr >= lo && rr < hi) dst[(int64_t)j * cl + r0 + rr] = Cs[j * 65 + rr];
       }
     }
   }
