@@ -63,3 +63,48 @@ def test_reference_arm_under_torchrun_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _args(*argv):
+    sys.path.insert(0, ROOT)
+    import bench
+    old = sys.argv
+    sys.argv = ["bench.py", *argv]
+    try:
+        return bench, bench.parse()
+    finally:
+        sys.argv = old
+
+
+def test_workload_overrides():
+    """--block, --clusters, --iters change the named workload; invalid combinations stop
+    before anything runs."""
+    bench, a = _args("--workload", "causal_n16k_bf16", "--block", "1024", "--clusters", "32",
+                     "--iters", "3")
+    w = bench.workload_of(a)
+    assert (w.block, w.Cq, w.Ck, w.iters) == (1024, 32, 32, 3)
+    assert w.N == 16384 and w.name == "causal_n16k_bf16"
+    bench, a = _args("--monopole")
+    assert bench.workload_of(a).mode == "acausal"
+    for bad in (["--block", "512"],                                   # acausal has no blocks
+                ["--workload", "causal_n16k_bf16", "--block", "1000"],  # does not divide N
+                ["--workload", "causal_n16k_bf16", "--monopole"],
+                ["--monopole", "--partial-dipole"],
+                ["--clusters", "100000"]):
+        bench, a = _args(*bad)
+        with pytest.raises(SystemExit):
+            bench.workload_of(a)
+
+
+def test_algorithmic_flops_of_the_block_sweep():
+    """The refinement's algorithmic flops per launch: at S = N/2 one square of N/2 x N/2,
+    and the multi-level count sums the squares of every level."""
+    bench, a = _args("--workload", "causal_n16k_bf16", "--block", "8192")
+    w = bench.workload_of(a)
+    n = 8192
+    one = min(2.0 * 64 * n * 64 * 64 + 2.0 * n * 64 * 64 * 64, 2.0 * n * n * 128)
+    assert bench.algorithmic_flops(w) == w.B * w.H * one
+    bench, a = _args("--workload", "causal_n16k_bf16", "--block", "4096")
+    w2 = bench.workload_of(a)
+    sq = lambda s: min(2.0 * 64 * s * 64 * 64 + 2.0 * s * 64 * 64 * 64, 2.0 * s * s * 128)
+    assert bench.algorithmic_flops(w2) == w2.B * w2.H * (sq(8192) + 2 * sq(4096))
