@@ -188,10 +188,10 @@ def test_forward_end_to_end_small_f32():
 
 # the monopole-only ablation (dipole term dropped) against the oracle's same mode, with
 # the GPU's clustering; it must be less accurate than the full method on these inputs
-@pytest.mark.parametrize("dt", ["f32", "bf16"])
-def test_forward_monopole_only(dt):
+@pytest.mark.parametrize("dt,D", [("f32", 64), ("bf16", 64), ("bf16", 128)])
+def test_forward_monopole_only(dt, D):
     N, C, T = 2048, 32, 6
-    Q, K, V = mixture(9, 1, 2, N, 64, 64, 48, 0.5 / 8, dt)
+    Q, K, V = mixture(9, 1, 2, N, D, D, 48, 0.5 / np.sqrt(D), dt)
     Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
     Om = host(m.muse_forward_ex(Qd, Kd, Vd, C, C, T, 1.0, flags=m.MUSE_FLAG_MONOPOLE))
     Od = host(m.muse_forward_ex(Qd, Kd, Vd, C, C, T, 1.0))
@@ -209,10 +209,11 @@ def test_forward_monopole_only(dt):
 
 # the partially specialised dipole (untilted key-cluster covariances aggregated per query
 # cluster) against the oracle's same reading, with the GPU's clustering
-@pytest.mark.parametrize("dt", ["f32", "bf16"])
-def test_forward_partial_dipole(dt):
+@pytest.mark.parametrize("dt,D,Dv", [("f32", 64, 64), ("bf16", 64, 64), ("bf16", 128, 128),
+                                     ("f32", 64, 128)])
+def test_forward_partial_dipole(dt, D, Dv):
     N, C, T = 2048, 32, 6
-    Q, K, V = mixture(10, 1, 2, N, 64, 64, 48, 0.5 / 8, dt)
+    Q, K, V = mixture(10, 1, 2, N, D, Dv, 48, 0.5 / np.sqrt(D), dt)
     Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
     Op = host(m.muse_forward_ex(Qd, Kd, Vd, C, C, T, 1.0, flags=m.MUSE_FLAG_PARTIAL_DIPOLE))
     ql, _, _, _ = m.muse_kmeans(Qd, C, T)
