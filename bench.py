@@ -171,6 +171,18 @@ def algorithmic_flops(w):
     raise ValueError(w.mode)
 
 
+def retrieval_flops(w):
+    """Algorithmic flops of one retrieval step (all problems): K-means of queries and keys,
+    the tilted summaries and the refinement over the whole causal prefix counted as in
+    the acausal case (2 Cq N D Dv + 2 N Ck D Dv), the exact diagonal (S N (D + Dv)) and
+    the retrieved runs (about S / Ck keys per (cluster, block) pair, k1 k2 pairs)."""
+    per = (2 * w.iters * 2.0 * w.N * w.Cq * w.D
+           + 2.0 * w.Cq * w.N * w.D * w.Dv + 2.0 * w.N * w.Ck * w.D * w.Dv
+           + float(w.block) * w.N * (w.D + w.Dv)
+           + 2.0 * w.N * w.k1 * w.k2 * (w.block / w.Ck) * (w.D + w.Dv))
+    return w.B * w.H * per
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -337,8 +349,14 @@ def main():
 
         def step(Q=Qd, K=Kd, V=Vd, O=Od):
             m.muse_causal_blocks(Q, K, V, w.block, w.Cq, w.Ck, w.iters, w.scale, out=O, ws=ws)
+    elif w.mode == "retrieval":
+        ws = m.workspace("muse_retrieve_exact", d, w.Cq, w.Ck, w.block, w.k1, w.k2)
+
+        def step(Q=Qd, K=Kd, V=Vd, O=Od):
+            m.muse_retrieve_exact(Q, K, V, w.block, w.Cq, w.Ck, w.iters, w.k1, w.k2, w.scale,
+                                  out=O, ws=ws)
     else:
-        raise SystemExit(f"workload {w.name} is not benchmarked yet")
+        raise SystemExit(f"workload {w.name} has an unknown mode")
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -427,20 +445,30 @@ def main():
     h2d = sum(x.numel() * x.element_size() for x in (Qh, Kh, Vh))
     d2h = Oh.numel() * Oh.element_size()
 
-    # roofline of the dominant kernel (the refinement), timed live above
+    # roofline of the dominant kernel (the refinement), timed live above; the retrieval
+    # path runs on CUDA cores only and is rated as a whole step against the FP32 peak
     peaks, peak_src = load_peaks()
-    kmean = sum(kern_ms) / len(kern_ms)
-    flops = algorithmic_flops(w)
-    achieved = flops / (kmean / 1e3) / 1e12
-    if w.dtype == "bf16":
-        peak, bound, unit = float(peaks["bf16_tflops"]), "tensor", "TFLOP/s"
+    if w.mode == "retrieval":
+        kmean = mean_ms
+        flops = retrieval_flops(w)
+        achieved = flops / (kmean / 1e3) / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_SIMT_TFLOPS, "traffic": None,
+                "kernel": "whole step (CUDA cores)", "kernel_ms": kmean, "flops_per_launch": flops,
+                "peak_source": "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
     else:
-        peak, bound, unit = FP32_SIMT_TFLOPS, "alu", "TFLOP/s"
-    roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": recorded_traffic(w.name), "kernel": "refinement",
-            "kernel_ms": kmean, "flops_per_launch": flops,
-            "peak_source": f"{peak_src} bf16_tflops (burst)" if w.dtype == "bf16"
-            else "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
+        kmean = sum(kern_ms) / len(kern_ms)
+        flops = algorithmic_flops(w)
+        achieved = flops / (kmean / 1e3) / 1e12
+        if w.dtype == "bf16":
+            peak, bound, unit = float(peaks["bf16_tflops"]), "tensor", "TFLOP/s"
+        else:
+            peak, bound, unit = FP32_SIMT_TFLOPS, "alu", "TFLOP/s"
+        roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": recorded_traffic(w.name),
+                "kernel": "refinement", "kernel_ms": kmean, "flops_per_launch": flops,
+                "peak_source": f"{peak_src} bf16_tflops (burst)" if w.dtype == "bf16"
+                else "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
     if rank == 0:
         try:
             from oracle import muse_oracle as mo
