@@ -238,6 +238,22 @@ def test_forward_bf16_multihead():
             assert mo.max_rel_err(O[b, h], ref) <= TOL["bf16"]
 
 
+# key and value widths that differ: the tensor-core refinement's 64-key tiles and a
+# 128-column O accumulator (Dv = 128), and 128-wide residuals and keys (D = 128)
+@pytest.mark.parametrize("D,Dv", [(64, 128), (128, 64)])
+def test_forward_bf16_unequal_widths(D, Dv):
+    Q, K, V = mixture(12, 1, 2, 2048, D, Dv, 48, 0.5 / np.sqrt(D), "bf16")
+    Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
+    O = host(m.muse_forward(Qd, Kd, Vd, 32, 40, 5, 1.0))
+    assert O.shape[-1] == Dv
+    ql = m.muse_kmeans(Qd, 32, 5)[0].cpu().numpy()
+    kl = m.muse_kmeans(Kd, 40, 5)[0].cpu().numpy()
+    Qf, Kf, Vf = host(Qd), host(Kd), host(Vd)
+    for h in range(2):
+        ref = mo.muse_from_labels(Qf[0, h], Kf[0, h], Vf[0, h], ql[0, h], kl[0, h], 32, 40, 1.0)
+        assert mo.max_rel_err(O[0, h], ref) <= TOL["bf16"]
+
+
 def test_singleton_query_clusters_give_exact_attention_on_gpu():
     Q, K, V = small_problem(21, 256, 64, 64, 16, 0.3)
     Qd, Kd, Vd = (dev(x[None, None], "f32") for x in (Q, K, V))
