@@ -271,6 +271,15 @@ def test_forward_is_deterministic():
     assert m.muse_last_device_status() == 0
 
 
+def test_causal_is_deterministic():
+    Q, K, V = mixture(16, 1, 2, 2048, 64, 64, 32, 0.3 / 8, "bf16")
+    Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
+    a = m.muse_causal_blocks(Qd, Kd, Vd, 256, 32, 32, 4, 1.0)
+    b = m.muse_causal_blocks(Qd, Kd, Vd, 256, 32, 32, 4, 1.0)
+    assert torch.equal(a, b)
+    assert m.muse_last_device_status() == 0
+
+
 def causal_labels(ql, kl, N, S):
     out = {}
     for (lev, r, q0, q1, k0, k1) in mo.causal_squares(N, S):
