@@ -492,3 +492,46 @@ def test_partial_dipole_is_first_order_in_the_centroid():
         diffs.append(np.abs(Op - Of).max())
     slope = np.polyfit(np.log([1e-3, 1e-2, 1e-1]), np.log(diffs), 1)[0]
     assert 0.8 <= slope <= 1.2, slope
+
+
+# --------------------------------------------------------------------------- the pages' trends
+
+def _trend_problem(seed):
+    from clustered_softmax_attention_b200.inputs import small_problem
+    return small_problem(seed, 512, 16, 8, 24, 0.25)
+
+
+def test_more_clusters_lower_error_and_the_dipole_helps():
+    """The pages' qualitative claims (review "free parameters": error falls from C = 32 to
+    C = 128; "invented entities": removing the dipole raises the error), on synthetic
+    mixtures: the RSE against exact attention falls as C grows, and the monopole-only
+    result is worse than the full method at every C."""
+    for seed in (1, 2):
+        Q, K, V = _trend_problem(seed)
+        E = mo.exact_attention(Q, K, V, 1.0)
+        errs, mono = [], []
+        for C in (4, 16, 64):
+            ql, qc = mo.kmeans(Q, C, 5)
+            kl, _ = mo.kmeans(K, C, 5)
+            errs.append(mo.rse(mo.muse_from_labels(Q, K, V, ql, kl, C, C, 1.0, qbar=qc), E))
+            mono.append(mo.rse(mo.muse_from_labels(Q, K, V, ql, kl, C, C, 1.0, qbar=qc,
+                                                   dipole=False), E))
+        assert errs[0] > errs[1] > errs[2], errs
+        assert all(m > e for m, e in zip(mono, errs)), (mono, errs)
+
+
+def test_more_kmeans_rounds_do_not_raise_the_error():
+    """Review "free parameters": the error drops from 1 to 5 K-means iterations."""
+    tot1 = tot5 = 0.0
+    for seed in (3, 4, 5):
+        Q, K, V = _trend_problem(seed)
+        E = mo.exact_attention(Q, K, V, 1.0)
+        for T in (1, 5):
+            ql, qc = mo.kmeans(Q, 16, T)
+            kl, _ = mo.kmeans(K, 16, T)
+            r = mo.rse(mo.muse_from_labels(Q, K, V, ql, kl, 16, 16, 1.0, qbar=qc), E)
+            if T == 1:
+                tot1 += r
+            else:
+                tot5 += r
+    assert tot5 < tot1, (tot1, tot5)
