@@ -115,6 +115,31 @@ def dims(X: torch.Tensor, V: Optional[torch.Tensor] = None, scale: float = 1.0) 
     return MuseDims(B, H, N, D, Dv, _dtype_code(X), float(scale))
 
 
+def _expect(t, shape, dtype, name):
+    """Shape and dtype of an argument the library reads or writes with sizes taken from
+    other arguments (a mismatch would make it read or write past the tensor)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+
+
+def _qkv(Q, K, V, out=None):
+    """Q, K [B,H,N,D] and V [B,H,N,Dv] of one dtype on one device; out [B,H,N,Dv]."""
+    if Q.dim() != 4:
+        raise ValueError(f"Q: expected [B,H,N,D], got shape {tuple(Q.shape)}")
+    B, H, N, D = Q.shape
+    _expect(K, (B, H, N, D), Q.dtype, "K")
+    if V.dim() != 4 or tuple(V.shape[:3]) != (B, H, N):
+        raise ValueError(f"V: shape {tuple(V.shape)}, expected [{B},{H},{N},Dv]")
+    _expect(V, V.shape, Q.dtype, "V")
+    if not (Q.device == K.device == V.device):
+        raise ValueError("Q, K, V must be on one device")
+    _expect(out, (B, H, N, V.shape[3]), Q.dtype, "out")
+
+
 def _contig(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -166,6 +191,11 @@ def muse_kmeans(X: torch.Tensor, C: int, iters: int, ws: Optional[torch.Tensor] 
 def muse_tilted_summaries(q_centroids, K, V, k_perm, k_offsets, Ck: int, scale: float = 1.0,
                           want_mu_k: bool = True, want_mu_v: bool = True, want_cov: bool = False):
     """Stage 1 summaries: dict with logZ and the requested mu_k / mu_v / cov."""
+    _qkv(K, K, V)
+    B, H, N, D = K.shape
+    _expect(q_centroids, (B, H, q_centroids.shape[2], D), torch.float32, "q_centroids")
+    _expect(k_perm, (B, H, N), torch.int32, "k_perm")
+    _expect(k_offsets, (B, H, Ck + 1), torch.int32, "k_offsets")
     _contig(q_centroids, K, V, k_perm, k_offsets)
     B, H, Cq, D = q_centroids.shape
     d = dims(K, V, scale)
@@ -189,6 +219,16 @@ def muse_tilted_summaries(q_centroids, K, V, k_perm, k_offsets, Ck: int, scale: 
 def muse_dipole_refine(Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offsets, logZ, mu_k,
                        scale: float = 1.0):
     """Stage 2 refinement: O [B,H,N,Dv] in Q's dtype."""
+    _qkv(Q, K, V)
+    B, H, N, D = Q.shape
+    Cq, Ck = q_centroids.shape[2], logZ.shape[3]
+    _expect(q_centroids, (B, H, Cq, D), torch.float32, "q_centroids")
+    _expect(q_perm, (B, H, N), torch.int32, "q_perm")
+    _expect(q_offsets, (B, H, Cq + 1), torch.int32, "q_offsets")
+    _expect(k_perm, (B, H, N), torch.int32, "k_perm")
+    _expect(k_offsets, (B, H, Ck + 1), torch.int32, "k_offsets")
+    _expect(logZ, (B, H, Cq, Ck), torch.float32, "logZ")
+    _expect(mu_k, (B, H, Cq, Ck, D), torch.float32, "mu_k")
     _contig(Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offsets, logZ, mu_k)
     d = dims(Q, V, scale)
     Cq, Ck = q_centroids.shape[2], logZ.shape[3]
@@ -204,6 +244,7 @@ def muse_dipole_refine(Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offset
 def muse_forward(Q, K, V, Cq: int, Ck: int, iters: int, scale: float = 1.0,
                  out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
     """The whole acausal forward pass."""
+    _qkv(Q, K, V, out)
     _contig(Q, K, V, out, ws)
     d = dims(Q, V, scale)
     if out is None:
@@ -223,6 +264,7 @@ def muse_forward_ex(Q, K, V, Cq: int, Ck: int, iters: int, scale: float = 1.0, f
                     out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
     """muse_forward with option flags (MUSE_FLAG_MONOPOLE: the monopole-only ablation;
     MUSE_FLAG_PARTIAL_DIPOLE: the partially specialised dipole)."""
+    _qkv(Q, K, V, out)
     _contig(Q, K, V, out, ws)
     d = dims(Q, V, scale)
     if out is None:
@@ -238,6 +280,7 @@ def muse_causal_blocks(Q, K, V, block: int, Cq: int, Ck: int, iters: int, scale:
                        return_labels: bool = False, out: Optional[torch.Tensor] = None,
                        ws: Optional[torch.Tensor] = None):
     """Causal MuSe (hierarchical block decomposition).  Labels are [B,H,L,N] (-1 = none)."""
+    _qkv(Q, K, V, out)
     _contig(Q, K, V, out, ws)
     d = dims(Q, V, scale)
     B, H, N, _ = Q.shape
@@ -262,6 +305,7 @@ def muse_retrieve_exact(Q, K, V, block: int, Cq: int, Ck: int, iters: int, k1: i
                         scale: float = 1.0, return_all: bool = False,
                         out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
     """Causal MuSe with top-k1 cluster / top-k2 block retrieval."""
+    _qkv(Q, K, V, out)
     _contig(Q, K, V, out, ws)
     d = dims(Q, V, scale)
     B, H, N, _ = Q.shape

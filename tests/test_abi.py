@@ -95,3 +95,25 @@ def test_argument_validation_enqueues_nothing(lib):
     assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 3, f, f, 1 << 30, st) == 1
     assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 1, f, f, 16, st) == 4
     assert lib.muse_forward_ex(f, f, f, _d(D=96), 8, 8, 2, 1, f, f, 1 << 30, st) == 2
+
+
+def test_binding_refuses_mismatched_tensors():
+    """The binding checks what the C ABI cannot (buffer extents): Q, K, V shapes, dtypes and
+    the output's shape, before anything reaches the library."""
+    import torch
+    Q = torch.zeros(1, 2, 256, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="K: shape"):
+        m.muse_forward(Q, torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16), Q, 8, 8, 2)
+    with pytest.raises(ValueError, match="K: dtype"):
+        m.muse_forward(Q, Q.float(), Q, 8, 8, 2)
+    with pytest.raises(ValueError, match="V: shape"):
+        m.muse_causal_blocks(Q, Q, torch.zeros(1, 2, 255, 64, dtype=torch.bfloat16), 128, 8, 8, 2)
+    with pytest.raises(ValueError, match="out: shape"):
+        m.muse_forward_ex(Q, Q, Q, 8, 8, 2, out=torch.zeros(1, 2, 256, 32, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="k_offsets: shape"):
+        m.muse_tilted_summaries(torch.zeros(1, 2, 8, 64), Q, Q,
+                                torch.zeros(1, 2, 256, dtype=torch.int32),
+                                torch.zeros(1, 2, 8, dtype=torch.int32), 8)
+    # consistent tensors on the host: refused for not being on the GPU
+    with pytest.raises(ValueError, match="CUDA"):
+        m.muse_forward(Q, Q, Q, 8, 8, 2)
