@@ -257,18 +257,29 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
+RETRIEVAL_SAMPLE_ROWS = 64  # the retrieval oracle costs seconds per query row at N = 32k
+
+
 def oracle_sample(w, head=0):
-    """The float64 oracle on one head of the workload: (seconds, tokens)."""
+    """The float64 oracle on one head of the workload: (seconds, tokens).  The retrieval
+    workload computes RETRIEVAL_SAMPLE_ROWS evenly spaced query rows (after the whole
+    problem's K-means and block selection), and counts those rows as its tokens."""
     from oracle import muse_oracle as mo
     Q, K, V = make_inputs(w, heads=[head])
     t0 = time.perf_counter()
+    n = w.N
     if w.mode == "acausal":
         mo.muse_acausal(Q[0, 0], K[0, 0], V[0, 0], w.Cq, w.Ck, w.iters, w.scale)
     elif w.mode == "causal":
         mo.muse_causal(Q[0, 0], K[0, 0], V[0, 0], w.block, w.Cq, w.Ck, w.iters, w.scale)
+    elif w.mode == "retrieval":
+        rows = np.linspace(0, w.N - 1, RETRIEVAL_SAMPLE_ROWS).astype(np.int64)
+        mo.muse_retrieval(Q[0, 0], K[0, 0], V[0, 0], w.block, w.Cq, w.Ck, w.iters, w.k1, w.k2,
+                          w.scale, rows=rows)
+        n = rows.size
     else:
         raise ValueError(w.mode)
-    return time.perf_counter() - t0, w.N
+    return time.perf_counter() - t0, n
 
 
 def run_reference(args, rank, world):
@@ -278,13 +289,18 @@ def run_reference(args, rank, world):
     for _ in range(args.warmup):
         oracle_sample(w)
     secs = []
+    n = w.N
     for k in range(args.steps):
         s, n = oracle_sample(w, head=k % w.problems)
         secs.append(s)
     mean = sum(secs) / len(secs)
-    value = w.N / mean
+    value = n / mean
     cores = cpu_threads()
-    sample = f"one (b,h) problem of {w.name} per step (N={w.N} tokens), float64 numpy oracle"
+    if w.mode == "retrieval":
+        sample = (f"{n} evenly spaced query rows of one (b,h) problem of {w.name} per step, "
+                  f"after that problem's whole K-means and block selection; float64 numpy oracle")
+    else:
+        sample = f"one (b,h) problem of {w.name} per step (N={w.N} tokens), float64 numpy oracle"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -483,9 +499,11 @@ def main():
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             secs, n = oracle_sample(w)
+            what = (f"{n} evenly spaced query rows of one (b,h) problem of {w.name} (after its "
+                    f"whole K-means and block selection)" if w.mode == "retrieval"
+                    else f"one (b,h) problem of {w.name} (N={w.N} tokens)")
             cpu = {"value": n / secs, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                   "sample": f"one (b,h) problem of {w.name} (N={w.N} tokens), float64 numpy "
-                             f"oracle, {secs:.1f} s"}
+                   "sample": f"{what}, float64 numpy oracle, {secs:.1f} s"}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
