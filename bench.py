@@ -258,17 +258,28 @@ def cpu_threads():
 
 
 RETRIEVAL_SAMPLE_ROWS = 64  # the retrieval oracle costs seconds per query row at N = 32k
+LARGE_SAMPLE_ROWS = 16      # acausal problems whose dipoles would not fit in 1 GiB of host memory
 
 
 def oracle_sample(w, head=0):
     """The float64 oracle on one head of the workload: (seconds, tokens).  The retrieval
     workload computes RETRIEVAL_SAMPLE_ROWS evenly spaced query rows (after the whole
-    problem's K-means and block selection), and counts those rows as its tokens."""
+    problem's K-means and block selection), an acausal workload too large for the oracle's
+    dense dipoles LARGE_SAMPLE_ROWS rows (after the whole K-means); those rows are the
+    tokens counted."""
     from oracle import muse_oracle as mo
     Q, K, V = make_inputs(w, heads=[head])
     t0 = time.perf_counter()
     n = w.N
-    if w.mode == "acausal":
+    if w.mode == "acausal" and w.Cq * w.Ck * w.D * w.Dv * 8 > (1 << 30):
+        # the oracle forms every C_ij: summaries only for the query clusters of a row sample
+        rows = np.linspace(0, w.N - 1, LARGE_SAMPLE_ROWS).astype(np.int64)
+        ql, qc = mo.kmeans(Q[0, 0], w.Cq, w.iters)
+        kl, _ = mo.kmeans(K[0, 0], w.Ck, w.iters)
+        mo.muse_from_labels(Q[0, 0], K[0, 0], V[0, 0], ql, kl, w.Cq, w.Ck, w.scale, qbar=qc,
+                            rows=rows)
+        n = rows.size
+    elif w.mode == "acausal":
         mo.muse_acausal(Q[0, 0], K[0, 0], V[0, 0], w.Cq, w.Ck, w.iters, w.scale)
     elif w.mode == "causal":
         mo.muse_causal(Q[0, 0], K[0, 0], V[0, 0], w.block, w.Cq, w.Ck, w.iters, w.scale)
@@ -296,9 +307,10 @@ def run_reference(args, rank, world):
     mean = sum(secs) / len(secs)
     value = n / mean
     cores = cpu_threads()
-    if w.mode == "retrieval":
+    if n != w.N:
         sample = (f"{n} evenly spaced query rows of one (b,h) problem of {w.name} per step, "
-                  f"after that problem's whole K-means and block selection; float64 numpy oracle")
+                  f"after that problem's whole K-means (and block selection); float64 numpy "
+                  f"oracle")
     else:
         sample = f"one (b,h) problem of {w.name} per step (N={w.N} tokens), float64 numpy oracle"
     line = {
@@ -500,7 +512,7 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             secs, n = oracle_sample(w)
             what = (f"{n} evenly spaced query rows of one (b,h) problem of {w.name} (after its "
-                    f"whole K-means and block selection)" if w.mode == "retrieval"
+                    f"whole K-means and block selection)" if n != w.N
                     else f"one (b,h) problem of {w.name} (N={w.N} tokens)")
             cpu = {"value": n / secs, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                    "sample": f"{what}, float64 numpy oracle, {secs:.1f} s"}
