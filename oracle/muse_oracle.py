@@ -53,10 +53,15 @@ NEG_INF = -np.inf
 # in the queries).
 # ----------------------------------------------------------------------------
 
-def kmeans_distances(X: np.ndarray, C: np.ndarray, chunk: int = 2048) -> np.ndarray:
-    """Squared Euclidean distances ||x_n - c_c||^2 by direct differences, [n, C]."""
+def kmeans_distances(X: np.ndarray, C: np.ndarray, chunk: int = 0) -> np.ndarray:
+    """Squared Euclidean distances ||x_n - c_c||^2 by direct differences, [n, C].
+
+    Rows go through in chunks (default: about 4M differences at a time) only to bound the
+    temporary array; every distance is the same sum of squared differences either way."""
     X = np.asarray(X, dtype=np.float64)
     C = np.asarray(C, dtype=np.float64)
+    if chunk <= 0:
+        chunk = max(1, (1 << 22) // max(1, C.shape[0] * C.shape[1]))
     out = np.empty((X.shape[0], C.shape[0]))
     for a in range(0, X.shape[0], chunk):
         diff = X[a:a + chunk, None, :] - C[None, :, :]

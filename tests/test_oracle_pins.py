@@ -21,7 +21,7 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 def _closed(expr_tree):
     """Evaluate nested lists of closed-form expression strings with math only."""
-    env = {"exp": math.exp, "log": math.log, "__builtins__": {}}
+    env = {"exp": math.exp, "log": math.log, "inf": math.inf, "__builtins__": {}}
     if isinstance(expr_tree, str):
         return eval(expr_tree, env)  # noqa: S307 - fixture expressions are ours
     return [_closed(e) for e in expr_tree]
@@ -34,7 +34,12 @@ def _load(name):
 
 # --------------------------------------------------------------------------- goldens
 
-@pytest.mark.parametrize("name", sorted(os.path.basename(p) for p in glob.glob(os.path.join(GOLDEN, "*.json"))))
+def _goldens(kind):
+    names = sorted(os.path.basename(p) for p in glob.glob(os.path.join(GOLDEN, "*.json")))
+    return [n for n in names if _load(n).get("kind", "muse") == kind]
+
+
+@pytest.mark.parametrize("name", _goldens("muse"))
 def test_golden_closed_forms(name):
     g = _load(name)
     Q, K, V = (np.array(g[k], float) for k in ("Q", "K", "V"))
@@ -57,6 +62,29 @@ def test_golden_closed_forms(name):
             lab, cen = mo.kmeans(K, g["Ck"], int(t))
             assert lab.tolist() == want["labels"]
             np.testing.assert_allclose(cen, np.array(_closed(want["centroids"])), rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("name", _goldens("kmeans_gap"))
+def test_golden_kmeans_gap_normaliser(name):
+    """The label-parity gap (d2 - d1) / (||x||^2 + ||c_a||^2) on hand-derived rows where d1 is
+    0, where the runner-up's norm differs from the assigned centroid's, and an exact tie."""
+    g = _load(name)
+    X, C = np.array(_closed(g["X"])), np.array(_closed(g["C"]))
+    lab, gap = mo.kmeans_assign_gap(X, C)
+    assert lab.tolist() == g["labels"]
+    assert mo.kmeans_assign(X, C).tolist() == g["labels"]
+    np.testing.assert_allclose(gap, np.array(_closed(g["gap"])), rtol=1e-13, atol=0)
+
+
+@pytest.mark.parametrize("name", _goldens("retrieval_select"))
+def test_golden_retrieval_selection(name):
+    """Cluster ranking by the prefix logsumexp, block ranking inside each chosen cluster,
+    ties to the lower index, -inf excluded, slot order, fewer candidates than k1 or k2."""
+    g = _load(name)
+    lzb = np.array(_closed(g["logZb"]), dtype=np.float64)
+    for case in g["cases"]:
+        sel = mo.retrieval_select(lzb, case["k1"], case["k2"])
+        assert sel.tolist() == case["slots"], (case["k1"], case["k2"])
 
 
 # --------------------------------------------------------------------------- exact attention
@@ -535,3 +563,23 @@ def test_more_kmeans_rounds_do_not_raise_the_error():
             else:
                 tot5 += r
     assert tot5 < tot1, (tot1, tot5)
+
+
+def test_retrieval_error_does_not_rise_with_k1_and_k2():
+    """gist.science "Kernmechanismen" item 4: retrieval is the accuracy upgrade of the causal
+    accumulation -- exact attention on the retrieved (cluster, block) pairs replaces their
+    summaries.  On seeded mixtures with 5 % outlier keys (x4 norm), the RSE against exact
+    causal attention must not rise as k1 and k2 grow, and retrieving every pair is exact."""
+    from clustered_softmax_attention_b200.inputs import draw_problem
+    steps = ((0, 0), (1, 1), (2, 2), (4, 4), (8, 4), (16, 8))
+    for seed in (1, 2, 3):
+        rng = np.random.Generator(np.random.PCG64(seed))
+        Q, K, V = draw_problem(rng, 1024, 16, 16, 24, 0.3 / 4, 0.05, 4.0)
+        E = mo.exact_attention(Q, K, V, 1.0, causal=True)
+        ql, _ = mo.kmeans(Q, 16, 5)
+        kl, _ = mo.kmeans(K, 16, 5)
+        errs = [mo.rse(mo.muse_retrieval(Q, K, V, 128, 16, 16, 5, k1, k2, 1.0,
+                                         q_labels=ql, k_labels=kl), E) for k1, k2 in steps]
+        assert all(b <= a * (1 + 1e-9) for a, b in zip(errs, errs[1:])), (seed, errs)
+        assert errs[0] > 10 * errs[4], (seed, errs)   # retrieval makes a real difference
+        assert errs[-1] < 1e-20, (seed, errs)          # k1 = Ck, k2 = nb: everything exact
