@@ -262,35 +262,69 @@ LARGE_SAMPLE_ROWS = 16      # acausal problems whose dipoles would not fit in 1 
 
 
 def oracle_sample(w, head=0):
-    """The float64 oracle on one head of the workload: (seconds, tokens).  The retrieval
-    workload computes RETRIEVAL_SAMPLE_ROWS evenly spaced query rows (after the whole
-    problem's K-means and block selection), an acausal workload too large for the oracle's
-    dense dipoles LARGE_SAMPLE_ROWS rows (after the whole K-means); those rows are the
-    tokens counted."""
+    """The float64 oracle on one head of the workload: (seconds, tokens, note).
+
+    Workloads the oracle finishes in seconds run whole (note None).  Two are too large
+    and are extrapolated to the whole problem from timed parts (the note says how):
+      * retrieval: both K-means and the block selection run whole; RETRIEVAL_SAMPLE_ROWS
+        evenly spaced query rows are computed, and their time is scaled by the number of
+        (query cluster, query block) groups of the problem over the sampled rows' groups
+        (each group builds its own remainder summaries, which dominate the per-row work);
+      * acausal problems whose dense C_ij would exceed 1 GiB: both K-means run whole;
+        the summaries are built for the query clusters of LARGE_SAMPLE_ROWS evenly spaced
+        rows and scaled by Cq over that count; the refinement of the sampled rows is
+        scaled by N over the rows."""
     from oracle import muse_oracle as mo
     Q, K, V = make_inputs(w, heads=[head])
+    Q, K, V = Q[0, 0], K[0, 0], V[0, 0]
     t0 = time.perf_counter()
-    n = w.N
     if w.mode == "acausal" and w.Cq * w.Ck * w.D * w.Dv * 8 > (1 << 30):
-        # the oracle forms every C_ij: summaries only for the query clusters of a row sample
         rows = np.linspace(0, w.N - 1, LARGE_SAMPLE_ROWS).astype(np.int64)
-        ql, qc = mo.kmeans(Q[0, 0], w.Cq, w.iters)
-        kl, _ = mo.kmeans(K[0, 0], w.Ck, w.iters)
-        mo.muse_from_labels(Q[0, 0], K[0, 0], V[0, 0], ql, kl, w.Cq, w.Ck, w.scale, qbar=qc,
-                            rows=rows)
-        n = rows.size
-    elif w.mode == "acausal":
-        mo.muse_acausal(Q[0, 0], K[0, 0], V[0, 0], w.Cq, w.Ck, w.iters, w.scale)
-    elif w.mode == "causal":
-        mo.muse_causal(Q[0, 0], K[0, 0], V[0, 0], w.block, w.Cq, w.Ck, w.iters, w.scale)
-    elif w.mode == "retrieval":
+        ql, qc = mo.kmeans(Q, w.Cq, w.iters)
+        kl, _ = mo.kmeans(K, w.Ck, w.iters)
+        t_km = time.perf_counter() - t0
+        used = np.unique(ql[rows])
+        t1 = time.perf_counter()
+        lz, mk, mv, cv = mo.tilted_summaries(qc[used], K, V, kl, w.Ck, w.scale)
+        t_sum = time.perf_counter() - t1
+        remap = -np.ones(w.Cq, np.int64)
+        remap[used] = np.arange(used.size)
+        t2 = time.perf_counter()
+        mo.refine(Q, remap[ql], qc[used], lz, mk, mv, cv, w.scale, rows=rows)
+        t_ref = time.perf_counter() - t2
+        secs = t_km + t_sum * w.Cq / used.size + t_ref * w.N / rows.size
+        note = (f"extrapolated: both K-means whole ({t_km:.1f} s), summaries of {used.size} of "
+                f"{w.Cq} query clusters ({t_sum:.1f} s) scaled x{w.Cq / used.size:.1f}, "
+                f"refinement of {rows.size} rows ({t_ref:.2f} s) scaled x{w.N / rows.size:.0f}")
+        return secs, w.N, note
+    if w.mode == "acausal":
+        mo.muse_acausal(Q, K, V, w.Cq, w.Ck, w.iters, w.scale)
+        return time.perf_counter() - t0, w.N, None
+    if w.mode == "causal":
+        mo.muse_causal(Q, K, V, w.block, w.Cq, w.Ck, w.iters, w.scale)
+        return time.perf_counter() - t0, w.N, None
+    if w.mode == "retrieval":
         rows = np.linspace(0, w.N - 1, RETRIEVAL_SAMPLE_ROWS).astype(np.int64)
-        mo.muse_retrieval(Q[0, 0], K[0, 0], V[0, 0], w.block, w.Cq, w.Ck, w.iters, w.k1, w.k2,
-                          w.scale, rows=rows)
-        n = rows.size
-    else:
-        raise ValueError(w.mode)
-    return time.perf_counter() - t0, n
+        ql, qc = mo.kmeans(Q, w.Cq, w.iters)
+        kl, _ = mo.kmeans(K, w.Ck, w.iters)
+        t_km = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        qbar = mo.cluster_means(Q, ql, w.Cq)
+        sel = mo.retrieval_select(mo.block_logZ(qbar, K, kl, w.Ck, w.block, w.scale), w.k1, w.k2)
+        t_sel = time.perf_counter() - t1
+        t2 = time.perf_counter()
+        mo.muse_retrieval(Q, K, V, w.block, w.Cq, w.Ck, w.iters, w.k1, w.k2, w.scale,
+                          q_labels=ql, k_labels=kl, selection=sel, rows=rows)
+        t_rows = time.perf_counter() - t2
+        blk = np.arange(w.N) // w.block
+        g_all = len(set(zip(ql.tolist(), blk.tolist())))
+        g_smp = len(set(zip(ql[rows].tolist(), blk[rows].tolist())))
+        secs = t_km + t_sel + t_rows * g_all / g_smp
+        note = (f"extrapolated: both K-means whole ({t_km:.1f} s), block selection whole "
+                f"({t_sel:.1f} s), {rows.size} evenly spaced query rows in {g_smp} (query "
+                f"cluster, block) groups ({t_rows:.1f} s) scaled to the problem's {g_all} groups")
+        return secs, w.N, note
+    raise ValueError(w.mode)
 
 
 def run_reference(args, rank, world):
@@ -300,19 +334,16 @@ def run_reference(args, rank, world):
     for _ in range(args.warmup):
         oracle_sample(w)
     secs = []
-    n = w.N
+    note = None
     for k in range(args.steps):
-        s, n = oracle_sample(w, head=k % w.problems)
+        s, n, note = oracle_sample(w, head=k % w.problems)
         secs.append(s)
     mean = sum(secs) / len(secs)
     value = n / mean
     cores = cpu_threads()
-    if n != w.N:
-        sample = (f"{n} evenly spaced query rows of one (b,h) problem of {w.name} per step, "
-                  f"after that problem's whole K-means (and block selection); float64 numpy "
-                  f"oracle")
-    else:
-        sample = f"one (b,h) problem of {w.name} per step (N={w.N} tokens), float64 numpy oracle"
+    sample = f"one (b,h) problem of {w.name} per step (N={w.N} tokens), float64 numpy oracle"
+    if note:
+        sample += f"; {note} (last step)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -510,10 +541,10 @@ def main():
             rse = None
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            secs, n = oracle_sample(w)
-            what = (f"{n} evenly spaced query rows of one (b,h) problem of {w.name} (after its "
-                    f"whole K-means and block selection)" if n != w.N
-                    else f"one (b,h) problem of {w.name} (N={w.N} tokens)")
+            secs, n, note = oracle_sample(w)
+            what = f"one (b,h) problem of {w.name} (N={w.N} tokens)"
+            if note:
+                what += f"; {note}"
             cpu = {"value": n / secs, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                    "sample": f"{what}, float64 numpy oracle, {secs:.1f} s"}
         line = {

@@ -98,9 +98,15 @@ __device__ __forceinline__ int map_block(const BlockMap &m, int nseg, int b, int
 }
 
 // ---------------------------------------------------------------------------
-// Device status word (MUSE_OK / MUSE_ERR_TIMEOUT / MUSE_ERR_DEVICE).  Kernels get
-// its address as a parameter; the first error wins.
+// Device status block, one per device.  Kernels get its address as a parameter.
+//   [0]    status word (MUSE_OK / MUSE_ERR_TIMEOUT / MUSE_ERR_DEVICE); first error wins
+//   [1]    test hooks (MUSE_TEST_* bits of muse_set_test_hooks; 0 in normal use)
+//   [2..3] wait limit in nanoseconds for the kernels that honour it (0 = default)
 // ---------------------------------------------------------------------------
+constexpr int kStatusInts = 4;
+__device__ __forceinline__ unsigned test_hooks(const int *status) {
+  return status ? (unsigned)*reinterpret_cast<const volatile int *>(status + 1) : 0u;
+}
 __device__ __forceinline__ void report(int *status, int code) {
   if (status) atomicCAS(status, 0, code);
 }

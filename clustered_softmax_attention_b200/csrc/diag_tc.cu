@@ -239,7 +239,11 @@ diag_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUten
   // copies and MMAs still in flight land before the CTA releases its memory
   if (t == 0) {
     mbar_drain(&sm.lbar, (lph - 1) & 1, status);  // the last load issued
+    // a wait that gave up leaves phase mph - 1 possibly incomplete: drain it first (a
+    // parity probe for phase mph alone would see the completed phase mph - 2), then the
+    // phase of a final commit that tracks every MMA issued
     tc_commit(&sm.mbar);
+    if (mph > 0) mbar_drain(&sm.mbar, (mph - 1) & 1, status);
     mbar_drain(&sm.mbar, mph & 1, status);
   }
   tc_fence_before();

@@ -64,9 +64,13 @@ extern "C" muse_status muse_kmeans_noalloc(const void *X, muse_dims d, int C, in
   t.nrow[0] = d.N;
   t.C[0] = C;
   const int P = d.B * d.H;
-  // The scratch holds per-chunk label counts, chunk bases and in-chunk ranks; a
-  // problem needing more than the array holds is refused before anything runs.
-  if (kmeans_ws_bytes(t, P, d.D) > (size_t)MUSE_NOALLOC_SCRATCH_BYTES) return MUSE_ERR_WORKSPACE;
+  // The multi-launch kernels keep per-chunk label counts, chunk bases and in-chunk ranks
+  // in the scratch; a problem of theirs needing more than the array holds is refused
+  // before anything runs.  The one-launch kernel (bfloat16, D = 64, C <= 128) keeps all
+  // of its state on chip and uses no scratch, so no size limit applies to it.
+  if (!kmeans_fused_supported(d.dtype, d.D, t) &&
+      kmeans_ws_bytes(t, P, d.D) > (size_t)MUSE_NOALLOC_SCRATCH_BYTES)
+    return MUSE_ERR_WORKSPACE;
 
   char *scratch = nullptr;
   if (kmeans_scratch_address(&scratch) != cudaSuccess) return MUSE_ERR_CUDA;

@@ -14,9 +14,10 @@
 namespace muse {
 
 // ---------------------------------------------------------------------------
-// Device status word: one per device, read and cleared by muse_last_device_status.
+// Device status block (common.cuh): one per device.  Its status word is read and
+// cleared by muse_last_device_status, its test-hook words set by muse_set_test_hooks.
 // ---------------------------------------------------------------------------
-static __device__ int g_status_word;
+static __device__ __align__(16) int g_status_word[kStatusInts];
 
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<void *> g_prof_start{nullptr}, g_prof_stop{nullptr};
@@ -293,6 +294,18 @@ extern "C" muse_status muse_last_device_status(muse_stream_t st) {
   if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof(int)) != cudaSuccess) return MUSE_ERR_CUDA;
   if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int)) != cudaSuccess) return MUSE_ERR_CUDA;
   return (muse_status)v;
+}
+
+extern "C" muse_status muse_set_test_hooks(unsigned hooks, uint64_t wait_limit_ns) {
+  if (hooks & ~(unsigned)MUSE_TEST_WITHHOLD_VALUES) return MUSE_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MUSE_ERR_CUDA;
+  int words[3];
+  words[0] = (int)hooks;
+  memcpy(&words[1], &wait_limit_ns, sizeof(uint64_t));
+  if (cudaMemcpyToSymbol(g_status_word, words, sizeof(words), sizeof(int)) != cudaSuccess)
+    return MUSE_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MUSE_ERR_CUDA;
+  return MUSE_OK;
 }
 
 // --------------------------------------------------------------------------- sizes

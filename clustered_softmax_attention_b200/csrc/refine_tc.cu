@@ -218,7 +218,9 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     // refilled once the MMA that read it has completed; the key tiles run ahead of
     // the value tiles, whose stages free up only after the second contraction.
     const bool keys = warp == 0;
-    if (lane == 0) {
+    // (test hook: the value tiles are never loaded, so the waits for them run out)
+    const bool withhold = !keys && (test_hooks(status) & MUSE_TEST_WITHHOLD_VALUES);
+    if (lane == 0 && !withhold) {
       if (keys) {
         mbar_expect_tx(&sm.qbar, (uint32_t)(D / 64) * BM * 128);
         for (int kb = 0; kb < D / 64; ++kb) tma_load_2d(sm.q[kb], &map_q, kb * 64, (int)(q.lab + r0), &sm.qbar);
@@ -232,7 +234,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const KTile kt = it.get();
         const int st = t % NST;
         const int nbox = kt.npad > 64 ? 2 : 1;
-        if (t >= NST && !mbar_wait(&empty[st], ((t / NST) - 1) & 1, abort_flag, status)) break;
+        if (t >= NST && !mbar_wait<true>(&empty[st], ((t / NST) - 1) & 1, abort_flag, status)) break;
         if (keys) {
           mbar_expect_tx(&full[st], (uint32_t)nbox * (D / 64) * 64 * 128);
           for (int rb = 0; rb < nbox; ++rb)
@@ -260,7 +262,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const KTile kt = it.get();
       const int st = t % NST;
       int ok = 1;
-      if (t >= NST && lane == 0) ok = mbar_wait(&sm.emptye[st], ((t / NST) - 1) & 1, abort_flag, status);
+      if (t >= NST && lane == 0) ok = mbar_wait<true>(&sm.emptye[st], ((t / NST) - 1) & 1, abort_flag, status);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       // tilt weights of the staged query clusters over the tile's columns
       for (int e = lane; e < nslots * (BN / 4); e += 32) {
@@ -331,13 +333,14 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     // ready is issued, the first contraction first, so that neither epilogue group
     // waits behind the other.
     if (lane == 0) {
-      bool ok = mbar_wait(&sm.qbar, 0, abort_flag, status);
+      bool ok = mbar_wait<true>(&sm.qbar, 0, abort_flag, status);
       tc_fence_after();
       TileIter<BN> it;
       it.begin(koff, k.C);
       int g1 = 0, g2 = 0;  // next tile of each contraction
       int idle = 0;
       uint64_t t_idle = 0;
+      const uint64_t idle_limit = wait_limit<true>(status);
       while (ok && (!it.done() || g2 < g1)) {
         bool progressed = false;
         if (!it.done()) {
@@ -389,7 +392,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const uint64_t now = now_ns();
             if (idle == 256) {
               t_idle = now;
-            } else if (now - t_idle > kTimeoutNs) {
+            } else if (now - t_idle > idle_limit) {
               *abort_flag = 1;
               report(status, MUSE_ERR_TIMEOUT);
               ok = false;
@@ -423,8 +426,8 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const int buf = t % kSBuf, st = t % NST;
       // (a wait that gave up in one lane stops the whole warp: the TMEM accesses below
       // are warp-collective)
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.sfull[buf], (t / kSBuf) & 1, abort_flag, status) &&
-                                       mbar_wait(&sm.fulle[st], (t / NST) & 1, abort_flag, status))) {
+      if (!__all_sync(0xffffffffu, mbar_wait<true>(&sm.sfull[buf], (t / kSBuf) & 1, abort_flag, status) &&
+                                       mbar_wait<true>(&sm.fulle[st], (t / NST) & 1, abort_flag, status))) {
         ok = false;
         break;
       }
@@ -514,7 +517,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         mbar_arrive(&sm.emptye[st]);  // the tile's epilogue data is consumed
       }
     }
-    if (ok && t > 0 && __all_sync(0xffffffffu, mbar_wait(&sm.obar, 0, abort_flag, status))) {
+    if (ok && t > 0 && __all_sync(0xffffffffu, mbar_wait<true>(&sm.obar, 0, abort_flag, status))) {
       tc_fence_after();
       const int row = valid ? q_perm[q.lab + n] : 0;
       for (int cb = grp; cb < DV / 16; cb += 2) {

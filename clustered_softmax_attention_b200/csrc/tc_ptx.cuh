@@ -84,8 +84,18 @@ __device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Limit of a bounded wait.  Kernels built with kRuntimeLimit read it from the status
+// block (status[2..3], nanoseconds, set by muse_set_test_hooks; 0 = kTimeoutNs) so that
+// a test can shorten it; the others always use kTimeoutNs.
+template <bool kRuntimeLimit>
+__device__ __forceinline__ uint64_t wait_limit(const int *status) {
+  if (!kRuntimeLimit || !status) return kTimeoutNs;
+  const uint64_t v = *reinterpret_cast<const volatile unsigned long long *>(status + 2);
+  return v ? v : kTimeoutNs;
+}
 // Bounded wait: false when the limit ran out or another role has aborted.  The first
 // probe is inlined; the polling loop is a call, which keeps the hot loops small.
+template <bool kRuntimeLimit>
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t *b, uint32_t parity,
                                                    volatile int *abort_flag, int *status) {
 #if MUSE_SPIN_PROBES > 0
@@ -93,21 +103,23 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t *b, uint32_t parity,
   for (int i = 0; i < MUSE_SPIN_PROBES; ++i)
     if (mbar_test(b, parity)) return true;
 #endif
+  const uint64_t limit = wait_limit<kRuntimeLimit>(status);
   const uint64_t t0 = now_ns();
   while (true) {
     if (mbar_try(b, parity)) return true;
     if (*abort_flag) return false;
-    if (now_ns() - t0 > kTimeoutNs) {
+    if (now_ns() - t0 > limit) {
       *abort_flag = 1;
       report(status, MUSE_ERR_TIMEOUT);
       return false;
     }
   }
 }
+template <bool kRuntimeLimit = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile int *abort_flag,
                                           int *status) {
   if (mbar_try(b, parity)) return true;
-  return mbar_wait_slow(b, parity, abort_flag, status);
+  return mbar_wait_slow<kRuntimeLimit>(b, parity, abort_flag, status);
 }
 // Bounded wait that ignores the abort flag: used to let in-flight copies and MMAs
 // finish before the CTA releases its shared memory and TMEM.

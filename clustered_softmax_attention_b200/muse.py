@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libmuse.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "muse.h")
 
 MUSE_F32, MUSE_BF16 = 0, 1
+NOALLOC_SCRATCH_BYTES = 16 << 20   # MUSE_NOALLOC_SCRATCH_BYTES of include/muse.h
 STATUS = {0: "MUSE_OK", 1: "MUSE_ERR_INVALID_ARG", 2: "MUSE_ERR_SHAPE", 3: "MUSE_ERR_DTYPE",
           4: "MUSE_ERR_WORKSPACE", 5: "MUSE_ERR_CUDA", 6: "MUSE_ERR_TIMEOUT", 7: "MUSE_ERR_DEVICE"}
 
@@ -54,6 +55,7 @@ _SIGS = {
     "muse_workspace_size": [ctypes.c_char_p, MuseDims, _i, _i, _i, _i, _i],
     "muse_status_string": [_i],
     "muse_last_device_status": [_vp],
+    "muse_set_test_hooks": [ctypes.c_uint, ctypes.c_uint64],
 }
 _RES = {"muse_workspace_size": _sz, "muse_status_string": ctypes.c_char_p,
         "muse_causal_levels": _i}
@@ -165,6 +167,15 @@ def muse_status_string(code: int) -> str:
 
 def muse_last_device_status() -> int:
     return int(lib().muse_last_device_status(_stream()))
+
+
+MUSE_TEST_WITHHOLD_VALUES = 1
+
+
+def muse_set_test_hooks(hooks: int = 0, wait_limit_ns: int = 0) -> None:
+    """Failure-path testing aid: make the refinement kernel's bounded waits run out
+    (see include/muse.h).  muse_set_test_hooks() restores normal operation."""
+    _check(lib().muse_set_test_hooks(hooks, wait_limit_ns), "muse_set_test_hooks")
 
 
 def muse_causal_levels(N: int, block: int) -> int:

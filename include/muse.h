@@ -99,10 +99,12 @@ muse_status muse_kmeans(const void *X, muse_dims d, int C, int iters, int32_t *l
  * is a deployment variant of the same computation, with identical results.
  *   Same arguments and outputs as muse_kmeans, minus the workspace.  Its scratch is
  *   a static device array of MUSE_NOALLOC_SCRATCH_BYTES (16 MiB) inside the library,
- *   held by every GPU that loads it until the process exits.  A problem whose
- *   scratch need (muse_workspace_size("muse_kmeans", ...)) exceeds that returns
- *   MUSE_ERR_WORKSPACE before anything is enqueued; e.g. B*H = 8, N = 8192,
- *   C = 128 needs about 0.5 MiB.
+ *   held by every GPU that loads it until the process exits.  Problems that take the
+ *   multi-launch kernels (float32 inputs, D = 128 or C > 128) use that scratch: one
+ *   whose need (muse_workspace_size("muse_kmeans", ...)) exceeds the array returns
+ *   MUSE_ERR_WORKSPACE before anything is enqueued; e.g. B*H = 8, N = 8192, C = 256,
+ *   D = 128 needs about 1 MiB.  The one-launch kernel (bfloat16, D = 64, C <= 128)
+ *   uses no scratch and has no size limit beyond muse_kmeans's.
  *   The first call on a device looks up the array's device address (with that
  *   device current); make that first call before any stream capture.  The library
  *   allocates nothing and calls no allocating routine.  Every call shares the one
@@ -260,6 +262,25 @@ const char *muse_status_string(muse_status s);
  * call on the device.
  */
 muse_status muse_last_device_status(muse_stream_t st);
+
+/*
+ * muse_set_test_hooks - failure-path testing aid (no counterpart in the method).
+ *   Every wait inside the library's tensor-core kernels is bounded: when it runs out
+ *   the kernel records MUSE_ERR_TIMEOUT in the device status word, every warp of the
+ *   block winds down (copies and tensor-core work in flight are drained, tensor memory
+ *   is freed) and the kernel returns, leaving the context usable.  This call lets a
+ *   test make such a wait run out without any fault:
+ *     hooks = MUSE_TEST_WITHHOLD_VALUES: the refinement kernel (the tensor-core path of
+ *       muse_dipole_refine, muse_forward, muse_causal_blocks) never loads its value
+ *       tiles, so the waits for them can only run out;
+ *     wait_limit_ns > 0: the limit of the refinement kernel's waits (default 2 s when 0).
+ *   The outputs of a call that timed out are undefined.  hooks = 0, wait_limit_ns = 0
+ *   restores normal operation.  Applies to the current device, synchronises it first,
+ *   and is process-wide: not for use while other work runs on the device.  Unknown hook
+ *   bits return MUSE_ERR_INVALID_ARG.
+ */
+#define MUSE_TEST_WITHHOLD_VALUES 1u
+muse_status muse_set_test_hooks(unsigned hooks, uint64_t wait_limit_ns);
 
 /*
  * Instrumentation (no counterpart in the method; used by the benchmark).

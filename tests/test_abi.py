@@ -117,3 +117,21 @@ def test_binding_refuses_mismatched_tensors():
     # consistent tensors on the host: refused for not being on the GPU
     with pytest.raises(ValueError, match="CUDA"):
         m.muse_forward(Q, Q, Q, 8, 8, 2)
+
+
+def test_noalloc_kmeans_refuses_a_multi_launch_problem_beyond_its_scratch(lib):
+    """float32 inputs take the multi-launch kernels, whose scratch (ranks of every row)
+    for B*H*N = 4M rows exceeds the 16 MiB array: refused before any CUDA call.  (The
+    one-launch bfloat16 path has no such limit; that acceptance needs real buffers and is
+    a GPU test.)"""
+    d = _d(B=8, H=8, N=65536, D=64, dtype=m.MUSE_F32)
+    assert lib.muse_workspace_size(b"muse_kmeans", d, 64, 0, 0, 0, 0) > m.NOALLOC_SCRATCH_BYTES
+    assert lib.muse_kmeans_noalloc(FAKE, d, 64, 2, FAKE, FAKE, FAKE, FAKE, ctypes.c_void_p(0)) == 4
+    d = _d(B=1, H=1, N=4096, D=128, dtype=m.MUSE_F32)
+    assert lib.muse_kmeans_noalloc(FAKE, d, 5000, 2, FAKE, FAKE, FAKE, FAKE, ctypes.c_void_p(0)) == 1
+
+
+def test_test_hooks_refuse_unknown_bits(lib):
+    """Unknown hook bits are refused before the device is touched."""
+    assert lib.muse_set_test_hooks(2, 0) == 1
+    assert lib.muse_set_test_hooks(0xFFFF, 5) == 1

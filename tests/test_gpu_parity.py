@@ -78,11 +78,17 @@ def check_kmeans_rounds(X, C, T, dt):
                                          ("bf16", 1000, 64, 37, 1), ("bf16", 1500, 64, 16, 1),
                                          ("bf16", 2100, 64, 64, 1), ("bf16", 4200, 64, 128, 1),
                                          ("bf16", 8192, 64, 128, 2), ("bf16", 8192, 64, 128, 16),
-                                         ("bf16", 3072, 64, 128, 40)])
-def test_kmeans_rounds_teacher_forced(dt, N, D, C, H):
-    Q, K, V = mixture(11, 1, H, N, D, D, 48, 0.3 / np.sqrt(D), dt)
-    ex = check_kmeans_rounds(Q, C, 6, dt)
-    assert ex <= 3 + 1e-4 * N * H * 6  # excused near-ties stay rare
+                                         ("bf16", 3072, 64, 128, 40), ("bf16", 4096, 64, 200, 2),
+                                         ("f32", 3000, 128, 300, 1), ("bf16", 16384, 128, 256, 1)])
+def test_kmeans_rounds_teacher_forced(dt, N, D, C, H, parity):
+    # C > 128 and D = 128 take the multi-launch kernels; the last case is the long-context
+    # workload's shape (N = 16384 rows of it, D = 128, C = 256)
+    comps = 48 if C <= 128 else 2 * C
+    Q, K, V = mixture(11, 1, H, N, D, D, comps, 0.3 / np.sqrt(D), dt)
+    T = 6 if N * C * D <= 8192 * 128 * 64 else 4
+    ex = check_kmeans_rounds(Q, C, T, dt)
+    parity("excused near-tie labels", ex)
+    assert ex <= 3 + 1e-4 * N * H * T  # excused near-ties stay rare
 
 
 def run_gpu_pipeline(Q, K, V, Cq, Ck, T, s, dt, with_cov=False):
@@ -99,7 +105,7 @@ def normwise(O, ref):
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
-def test_summaries_and_refine_vs_oracle(dt):
+def test_summaries_and_refine_vs_oracle(dt, parity):
     N, D, Cq, Ck = 512, 64, 16, 24
     Q, K, V = mixture(3, 1, 2, N, D, D, 20, 0.4 / np.sqrt(D), dt)
     for s in (1.0, 0.125):
@@ -116,9 +122,11 @@ def test_summaries_and_refine_vs_oracle(dt):
             np.testing.assert_allclose(g["logZ"][fin], lz[fin], rtol=1e-5, atol=1e-5)
             for key, ref in (("mu_k", mk), ("mu_v", mv), ("cov", cv)):
                 err = np.abs(g[key] - ref).max() / max(np.abs(ref).max(), 1e-30)
+                parity(f"{key} s={s} h={h}", err, 1e-4)
                 assert err < 1e-4, (key, err)
             O_ref = mo.refine(Qf[0, h], ql, qbar, lz, mk, mv, cv, s)
             err = mo.max_rel_err(host(r["O"])[0, h], O_ref)
+            parity(f"O s={s} h={h}", err, TOL[dt])
             assert err <= TOL[dt], err
 
 
@@ -129,7 +137,7 @@ def test_summaries_and_refine_vs_oracle(dt):
 @pytest.mark.parametrize("dt,D,Ck", [("bf16", 64, 16), ("bf16", 64, 40), ("f32", 64, 40),
                                       ("bf16", 128, 40), ("f32", 128, 16), ("bf16", 64, 128),
                                       ("f32", 128, 128)])
-def test_key_means_cluster_layouts(dt, D, Ck):
+def test_key_means_cluster_layouts(dt, D, Ck, parity):
     rng = np.random.Generator(np.random.PCG64(100 + Ck + D))
     N, Cq, s = 1200, 70, 0.35
     fixed = [300, 0, 1, 15, 0, 16, 17, 64, 65, 127, 128, 129, 0]
@@ -164,10 +172,11 @@ def test_key_means_cluster_layouts(dt, D, Ck):
     np.testing.assert_allclose(glz[fin], lz[fin], rtol=1e-5, atol=1e-5)
     assert (gmk[~fin] == 0).all()
     err = np.abs(gmk - mk).max() / np.abs(mk).max()
+    parity("mu_k", err, 1e-5)
     assert err < 1e-5, err
 
 
-def test_forward_end_to_end_small_f32():
+def test_forward_end_to_end_small_f32(parity):
     w = WORKLOADS["acausal_n1k_f32"]
     Q, K, V = make_inputs(w)
     Qd, Kd, Vd = dev(Q, "f32"), dev(K, "f32"), dev(V, "f32")
@@ -176,6 +185,7 @@ def test_forward_end_to_end_small_f32():
     kl, _, _, _ = m.muse_kmeans(Kd, w.Ck, w.iters)
     ref = mo.muse_from_labels(Q[0, 0], K[0, 0], V[0, 0], ql[0, 0].cpu().numpy(),
                               kl[0, 0].cpu().numpy(), w.Cq, w.Ck, w.scale)
+    parity("O", mo.max_rel_err(O[0, 0], ref), 1e-4)
     assert mo.max_rel_err(O[0, 0], ref) <= 1e-4
     # and against the oracle's own K-means (labels may differ only at near-ties)
     ref2, ql2, kl2 = mo.muse_acausal(Q[0, 0], K[0, 0], V[0, 0], w.Cq, w.Ck, w.iters, w.scale,
@@ -189,7 +199,7 @@ def test_forward_end_to_end_small_f32():
 # the monopole-only ablation (dipole term dropped) against the oracle's same mode, with
 # the GPU's clustering; it must be less accurate than the full method on these inputs
 @pytest.mark.parametrize("dt,D", [("f32", 64), ("bf16", 64), ("bf16", 128)])
-def test_forward_monopole_only(dt, D):
+def test_forward_monopole_only(dt, D, parity):
     N, C, T = 2048, 32, 6
     Q, K, V = mixture(9, 1, 2, N, D, D, 48, 0.5 / np.sqrt(D), dt)
     Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
@@ -202,6 +212,7 @@ def test_forward_monopole_only(dt, D):
     for h in range(2):
         a = (Qf[0, h], Kf[0, h], Vf[0, h], ql[0, h].cpu().numpy(), kl[0, h].cpu().numpy(), C, C, 1.0)
         ref_m = mo.muse_from_labels(*a, dipole=False)
+        parity(f"O h={h}", mo.max_rel_err(Om[0, h], ref_m), TOL[dt])
         assert mo.max_rel_err(Om[0, h], ref_m) <= TOL[dt]
         E = mo.exact_attention(Qf[0, h], Kf[0, h], Vf[0, h], 1.0)
         assert mo.rse(Od[0, h], E) < mo.rse(Om[0, h], E)
@@ -211,7 +222,7 @@ def test_forward_monopole_only(dt, D):
 # cluster) against the oracle's same reading, with the GPU's clustering
 @pytest.mark.parametrize("dt,D,Dv", [("f32", 64, 64), ("bf16", 64, 64), ("bf16", 128, 128),
                                      ("f32", 64, 128)])
-def test_forward_partial_dipole(dt, D, Dv):
+def test_forward_partial_dipole(dt, D, Dv, parity):
     N, C, T = 2048, 32, 6
     Q, K, V = mixture(10, 1, 2, N, D, Dv, 48, 0.5 / np.sqrt(D), dt)
     Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
@@ -222,10 +233,11 @@ def test_forward_partial_dipole(dt, D, Dv):
     for h in range(2):
         ref = mo.muse_partial_dipole_from_labels(Qf[0, h], Kf[0, h], Vf[0, h], ql[0, h].cpu().numpy(),
                                                  kl[0, h].cpu().numpy(), C, C, 1.0)
+        parity(f"O h={h}", mo.max_rel_err(Op[0, h], ref), TOL[dt])
         assert mo.max_rel_err(Op[0, h], ref) <= TOL[dt]
 
 
-def test_forward_bf16_multihead():
+def test_forward_bf16_multihead(parity):
     Q, K, V = mixture(5, 2, 2, 2048, 64, 64, 64, 0.5 / 8, "bf16")
     Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
     O = host(m.muse_forward(Qd, Kd, Vd, 64, 48, 6, 1.0))
@@ -235,13 +247,14 @@ def test_forward_bf16_multihead():
     for b in range(2):
         for h in range(2):
             ref = mo.muse_from_labels(Qf[b, h], Kf[b, h], Vf[b, h], ql[b, h], kl[b, h], 64, 48, 1.0)
+            parity(f"O b={b} h={h}", mo.max_rel_err(O[b, h], ref), TOL["bf16"])
             assert mo.max_rel_err(O[b, h], ref) <= TOL["bf16"]
 
 
 # key and value widths that differ: the tensor-core refinement's 64-key tiles and a
 # 128-column O accumulator (Dv = 128), and 128-wide residuals and keys (D = 128)
 @pytest.mark.parametrize("D,Dv", [(64, 128), (128, 64)])
-def test_forward_bf16_unequal_widths(D, Dv):
+def test_forward_bf16_unequal_widths(D, Dv, parity):
     Q, K, V = mixture(12, 1, 2, 2048, D, Dv, 48, 0.5 / np.sqrt(D), "bf16")
     Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
     O = host(m.muse_forward(Qd, Kd, Vd, 32, 40, 5, 1.0))
@@ -251,14 +264,16 @@ def test_forward_bf16_unequal_widths(D, Dv):
     Qf, Kf, Vf = host(Qd), host(Kd), host(Vd)
     for h in range(2):
         ref = mo.muse_from_labels(Qf[0, h], Kf[0, h], Vf[0, h], ql[0, h], kl[0, h], 32, 40, 1.0)
+        parity(f"O h={h}", mo.max_rel_err(O[0, h], ref), TOL["bf16"])
         assert mo.max_rel_err(O[0, h], ref) <= TOL["bf16"]
 
 
-def test_singleton_query_clusters_give_exact_attention_on_gpu():
+def test_singleton_query_clusters_give_exact_attention_on_gpu(parity):
     Q, K, V = small_problem(21, 256, 64, 64, 16, 0.3)
     Qd, Kd, Vd = (dev(x[None, None], "f32") for x in (Q, K, V))
     O = host(m.muse_forward(Qd, Kd, Vd, 256, 16, 3, 1.0))[0, 0]
     E = mo.exact_attention(host(Qd)[0, 0], host(Kd)[0, 0], host(Vd)[0, 0], 1.0)
+    parity("O vs exact", mo.max_rel_err(O, E), 1e-4)
     assert mo.max_rel_err(O, E) <= 1e-4
 
 
@@ -296,7 +311,7 @@ def causal_labels(ql, kl, N, S):
                                        ("bf16", 1024, 512, 32), ("bf16", 2048, 1024, 48),
                                        ("bf16", 4096, 2048, 32), ("f32", 2048, 512, 32),
                                        ("f32", 2048, 1024, 48)])
-def test_causal_vs_oracle(dt, N, S, C):
+def test_causal_vs_oracle(dt, N, S, C, parity):
     Q, K, V = mixture(7, 1, 2, N, 64, 64, 16, 0.3 / 8, dt)
     Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
     O, ql, kl = m.muse_causal_blocks(Qd, Kd, Vd, S, C, C, 4, 1.0, return_labels=True)
@@ -315,31 +330,53 @@ def test_causal_vs_oracle(dt, N, S, C):
             assert (ql[0, h, lev - 1][~inside] == -1).all()
             assert (ql[0, h, lev - 1][inside] >= 0).all()
         ref = mo.muse_causal(Qf[0, h], Kf[0, h], Vf[0, h], S, C, C, 4, 1.0, labels=labels)
+        parity(f"O h={h}", mo.max_rel_err(O[0, h], ref), TOL[dt])
         assert mo.max_rel_err(O[0, h], ref) <= TOL[dt]
 
 
-def test_causal_single_block_is_exact():
+def test_causal_single_block_is_exact(parity):
     Q, K, V = small_problem(22, 256, 64, 64, 8, 0.3)
     Qd, Kd, Vd = (dev(x[None, None], "f32") for x in (Q, K, V))
     O = host(m.muse_causal_blocks(Qd, Kd, Vd, 256, 8, 8, 2, 1.0))[0, 0]
     E = mo.exact_attention(host(Qd)[0, 0], host(Kd)[0, 0], host(Vd)[0, 0], 1.0, causal=True)
+    parity("O vs exact", mo.max_rel_err(O, E), 1e-4)
     assert mo.max_rel_err(O, E) <= 1e-4
 
 
-def test_full_size_acausal_n8k_sampled_rows():
+def check_last_kmeans_round(Xd, C, T, heads, parity, what):
+    """The last K-means round at full size: labels of round T against the oracle's
+    assignment from the GPU's centroids after round T - 1, bit-exact except near-ties
+    (counted).  Returns round T's labels [B,H,N]."""
+    Xf = host(Xd)
+    prev = m.muse_kmeans(Xd, C, T - 1)[1].cpu().numpy() if T > 1 else None
+    lab = m.muse_kmeans(Xd, C, T)[0].cpu().numpy()
+    excused = 0
+    for (b, h) in heads:
+        c_prev = Xf[b, h, :C] if prev is None else prev[b, h].astype(np.float64)
+        lo, gap = mo.kmeans_assign_gap(Xf[b, h], c_prev)
+        bad = lo != lab[b, h]
+        assert (gap[bad] < NEAR_TIE).all(), (what, b, h, int(bad.sum()))
+        excused += int(bad.sum())
+    parity(f"{what}: excused near-tie labels in round {T}", excused)
+    return lab
+
+
+def test_full_size_acausal_n8k_sampled_rows(parity):
     """The benchmarked workload at full size, checked on sampled rows of two heads."""
     w = WORKLOADS["acausal_n8k_bf16"]
     Q, K, V = make_inputs(w)
     Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
     O = host(m.muse_forward(Qd, Kd, Vd, w.Cq, w.Ck, w.iters, w.scale))
-    ql = m.muse_kmeans(Qd, w.Cq, w.iters)[0].cpu().numpy()
-    kl = m.muse_kmeans(Kd, w.Ck, w.iters)[0].cpu().numpy()
+    heads = [(0, 0), (0, w.H - 1)]
+    ql = check_last_kmeans_round(Qd, w.Cq, w.iters, heads, parity, "queries")
+    kl = check_last_kmeans_round(Kd, w.Ck, w.iters, heads, parity, "keys")
     rng = np.random.default_rng(0)
-    for h in (0, w.H - 1):
+    for _, h in heads:
         rows = np.concatenate([rng.choice(w.N, 48, replace=False), [0, w.N - 1]])
         ref = mo.muse_from_labels(Q[0, h], K[0, h], V[0, h], ql[0, h], kl[0, h], w.Cq, w.Ck,
                                   w.scale, rows=rows)
         err = np.abs(O[0, h][rows] - ref[rows]).max() / np.abs(ref[rows]).max()
+        parity(f"O sampled rows h={h}", err, TOL["bf16"])
         assert err <= TOL["bf16"], err
 
 
@@ -356,32 +393,85 @@ def retrieval_case(dt, N, S, C, k1, k2, seed=9, H=2, scale=1.0, outliers=0.0):
     return host(Qd), host(Kd), host(Vd), host(O), ql.cpu().numpy(), kl.cpu().numpy(), sel.cpu().numpy()
 
 
-@pytest.mark.parametrize("dt", ["f32", "bf16"])
-def test_retrieval_vs_oracle(dt):
-    N, S, C, k1, k2 = 1024, 128, 16, 2, 2
+def _close(a, b, tol=NEAR_TIE):
+    return abs(a - b) <= tol * max(1.0, abs(a), abs(b))
+
+
+def check_selection(lzb, got, k1, k2):
+    """The GPU's retrieval selection against the oracle's from the same clustering.
+
+    Slots must be equal, except where the oracle's ranking has a near-tie: a slot whose
+    cluster differs must hold a cluster whose prefix score is within 1e-5 (relative) of
+    the oracle's pick, and a block that differs a block whose score is within 1e-5 of the
+    oracle's.  Whatever differs must still be a valid selection (distinct clusters,
+    distinct blocks before the query block, finite scores).  Returns the number of
+    (query cluster, query block) rows excused as near-ties."""
+    want = mo.retrieval_select(lzb, k1, k2)
+    Cq, nb = want.shape[:2]
+    excused = 0
+    for i in range(Cq):
+        for b in range(nb):
+            if (want[i, b] == got[i, b]).all():
+                continue
+            sig = [mo._lse(lzb[i, j, :b]) for j in range(lzb.shape[1])]
+            gj = [int(got[i, b, t * k2, 0]) for t in range(k1)]
+            wj = [int(want[i, b, t * k2, 0]) for t in range(k1)]
+            chosen = [j for j in gj if j >= 0]
+            assert len(set(chosen)) == len(chosen), (i, b, gj)
+            for t in range(k1):
+                assert (gj[t] < 0) == (wj[t] < 0), (i, b, gj, wj)
+                if gj[t] < 0:
+                    continue
+                assert gj[t] == wj[t] or _close(sig[gj[t]], sig[wj[t]]), (i, b, t, gj, wj)
+                j = gj[t]
+                row = lzb[i, j, :b]
+                ranked = sorted((bb for bb in range(b) if np.isfinite(row[bb])),
+                                key=lambda bb: (-row[bb], bb))[:k2]
+                gb = [int(got[i, b, t * k2 + u, 1]) for u in range(k2)]
+                assert all(int(got[i, b, t * k2 + u, 0]) in (j, -1) for u in range(k2))
+                assert len(set(x for x in gb if x >= 0)) == len([x for x in gb if x >= 0])
+                for u in range(k2):
+                    eb = ranked[u] if u < len(ranked) else -1
+                    assert (gb[u] < 0) == (eb < 0), (i, b, t, gb, ranked)
+                    if gb[u] >= 0:
+                        assert gb[u] < b and np.isfinite(row[gb[u]])
+                        assert gb[u] == eb or _close(row[gb[u]], row[eb]), (i, b, t, gb, ranked)
+            excused += 1
+    return excused
+
+
+@pytest.mark.parametrize("dt,k1,k2", [("f32", 2, 2), ("bf16", 2, 2), ("bf16", 4, 1),
+                                       ("bf16", 1, 4)])
+def test_retrieval_vs_oracle(dt, k1, k2, parity):
+    N, S, C = 1024, 128, 16
     Q, K, V, O, ql, kl, sel = retrieval_case(dt, N, S, C, k1, k2, outliers=0.05)
+    nrows = 0
     for h in range(2):
-        # the selection equals the oracle's from the same clustering (near-ties aside)
+        # the selection equals the oracle's from the same clustering (near-ties counted)
         qbar = mo.cluster_means(Q[0, h], ql[0, h], C)
         lzb = mo.block_logZ(qbar, K[0, h], kl[0, h], C, S, 1.0)
-        want = mo.retrieval_select(lzb, k1, k2)
-        agree = (want == sel[0, h]).all(axis=-1).mean()
-        assert agree > 0.98, agree
+        ex = check_selection(lzb, sel[0, h], k1, k2)
+        parity(f"selection rows excused as near-ties h={h}", ex)
+        nrows += C * (N // S)
+        assert ex <= 2, ex
         ref = mo.muse_retrieval(Q[0, h], K[0, h], V[0, h], S, C, C, 4, k1, k2, 1.0,
                                 q_labels=ql[0, h], k_labels=kl[0, h], selection=sel[0, h])
         err = mo.max_rel_err(O[0, h], ref)
+        parity(f"O h={h}", err, TOL[dt])
         assert err <= TOL[dt], err
 
 
-def test_retrieval_exact_limits_on_gpu():
+def test_retrieval_exact_limits_on_gpu(parity):
     N, S = 256, 64
     # every query its own cluster: exact whatever is retrieved
     Q, K, V, O, *_ = retrieval_case("f32", N, S, N, 1, 1, H=1)
     E = mo.exact_attention(Q[0, 0], K[0, 0], V[0, 0], 1.0, causal=True)
+    parity("singleton queries vs exact", mo.max_rel_err(O[0, 0], E), 1e-4)
     assert mo.max_rel_err(O[0, 0], E) <= 1e-4
     # every (cluster, block) pair retrieved: exact
     Q, K, V, O, *_ = retrieval_case("f32", N, S, 4, 4, 4, H=1)
     E = mo.exact_attention(Q[0, 0], K[0, 0], V[0, 0], 1.0, causal=True)
+    parity("all retrieved vs exact", mo.max_rel_err(O[0, 0], E), 1e-4)
     assert mo.max_rel_err(O[0, 0], E) <= 1e-4
     # nothing retrieved, singleton keys: the remainder summaries are exact
     rng = np.random.Generator(np.random.PCG64(3))
@@ -389,13 +479,14 @@ def test_retrieval_exact_limits_on_gpu():
     Qd, Kd, Vd = (dev(x[None, None], "f32") for x in (Qn, Kn, Vn))
     O = host(m.muse_retrieve_exact(Qd, Kd, Vd, S, 8, N, 3, 0, 0, 1.0))[0, 0]
     E = mo.exact_attention(host(Qd)[0, 0], host(Kd)[0, 0], host(Vd)[0, 0], 1.0, causal=True)
+    parity("singleton keys, nothing retrieved, vs exact", mo.max_rel_err(O, E), 1e-4)
     assert mo.max_rel_err(O, E) <= 1e-4
 
 
 # --------------------------------------------------------------------------- full-size workloads
 # Sampled rows, oracle fed the GPU's clustering (and selection), same launch as bench.py.
 
-def test_full_size_causal_n16k_sampled_rows():
+def test_full_size_causal_n16k_sampled_rows(parity):
     w = WORKLOADS["causal_n16k_bf16"]
     heads = [0, w.problems - 1]
     Q, K, V = make_inputs(w)
@@ -404,6 +495,19 @@ def test_full_size_causal_n16k_sampled_rows():
                                      return_labels=True)
     O = host(O)
     ql, kl = ql.cpu().numpy(), kl.cpu().numpy()
+    # the largest square (top level: queries [N/2, N), keys [0, N/2)) clustered on its own
+    # through muse_kmeans, last round against the oracle; the causal launch's labels of
+    # that square must equal them except at those near-ties
+    L, half = ql.shape[2], w.N // 2
+    sq = [(0, 0), (w.B - 1, w.H - 1)]
+    lq = check_last_kmeans_round(Qd[:, :, half:].contiguous(), w.Cq, w.iters, sq, parity,
+                                 "top-level square, queries")
+    lk = check_last_kmeans_round(Kd[:, :, :half].contiguous(), w.Ck, w.iters, sq, parity,
+                                 "top-level square, keys")
+    differ = sum(int((ql[b, h, L - 1, half:] != lq[b, h]).sum()) +
+                 int((kl[b, h, L - 1, :half] != lk[b, h]).sum()) for b, h in sq)
+    parity("top-level square: causal-launch labels differing from muse_kmeans", differ)
+    assert differ <= 4, differ
     rng = np.random.default_rng(1)
     for p in heads:
         b, h = divmod(p, w.H)
@@ -412,40 +516,54 @@ def test_full_size_causal_n16k_sampled_rows():
         ref = mo.muse_causal(Q[b, h], K[b, h], V[b, h], w.block, w.Cq, w.Ck, w.iters, w.scale,
                              labels=labels, rows=rows)
         err = np.abs(O[b, h][rows] - ref[rows]).max() / np.abs(ref[rows]).max()
+        parity(f"O sampled rows p={p}", err, TOL["bf16"])
         assert err <= TOL["bf16"], err
 
 
-def test_full_size_retrieval_n32k_sampled_rows():
+def test_full_size_retrieval_n32k_sampled_rows(parity):
     w = WORKLOADS["retrieval_n32k_bf16"]
     Q, K, V = make_inputs(w)
     Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
     O, ql, kl, sel = m.muse_retrieve_exact(Qd, Kd, Vd, w.block, w.Cq, w.Ck, w.iters, w.k1, w.k2,
                                            w.scale, return_all=True)
     O, ql, kl, sel = host(O), ql.cpu().numpy(), kl.cpu().numpy(), sel.cpu().numpy()
+    heads = [(0, 0), (w.B - 1, w.H - 1)]
+    lq = check_last_kmeans_round(Qd, w.Cq, w.iters, heads, parity, "queries")
+    lk = check_last_kmeans_round(Kd, w.Ck, w.iters, heads, parity, "keys")
+    for (b, h) in heads:
+        assert (lq[b, h] == ql[b, h]).all() and (lk[b, h] == kl[b, h]).all()
+        # the whole selection of this head against the oracle's (near-ties counted)
+        qbar = mo.cluster_means(Q[b, h], ql[b, h], w.Cq)
+        lzb = mo.block_logZ(qbar, K[b, h], kl[b, h], w.Ck, w.block, w.scale)
+        ex = check_selection(lzb, sel[b, h], w.k1, w.k2)
+        parity(f"selection rows excused as near-ties b={b} h={h}", ex)
+        assert ex <= 8, ex
     rng = np.random.default_rng(2)
-    for (b, h) in ((0, 0), (w.B - 1, w.H - 1)):
+    for (b, h) in heads:
         rows = np.concatenate([rng.choice(np.arange(w.block, w.N), 6, replace=False), [3, w.N - 1]])
         ref = mo.muse_retrieval(Q[b, h], K[b, h], V[b, h], w.block, w.Cq, w.Ck, w.iters, w.k1,
                                 w.k2, w.scale, q_labels=ql[b, h], k_labels=kl[b, h],
                                 selection=sel[b, h], rows=rows)
         err = np.abs(O[b, h][rows] - ref[rows]).max() / np.abs(ref[rows]).max()
+        parity(f"O sampled rows b={b} h={h}", err, TOL["bf16"])
         assert err <= TOL["bf16"], err
 
 
-def test_full_size_acausal_n64k_d128_sampled_rows():
+def test_full_size_acausal_n64k_d128_sampled_rows(parity):
     w = WORKLOADS["acausal_n64k_d128_bf16"]
     heads = [0, w.H - 1]
     Q, K, V = make_inputs(w, heads=heads)
     Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
     O = host(m.muse_forward(Qd, Kd, Vd, w.Cq, w.Ck, w.iters, w.scale))
-    ql = m.muse_kmeans(Qd, w.Cq, w.iters)[0].cpu().numpy()
-    kl = m.muse_kmeans(Kd, w.Ck, w.iters)[0].cpu().numpy()
+    ql = check_last_kmeans_round(Qd, w.Cq, w.iters, [(0, 0)], parity, "queries")
+    kl = check_last_kmeans_round(Kd, w.Ck, w.iters, [(0, 0)], parity, "keys")
     rng = np.random.default_rng(3)
     for h in range(len(heads)):
         rows = np.concatenate([rng.choice(w.N, 10, replace=False), [0, w.N - 1]])
         ref = mo.muse_from_labels(Q[0, h], K[0, h], V[0, h], ql[0, h], kl[0, h], w.Cq, w.Ck,
                                   w.scale, rows=rows)
         err = np.abs(O[0, h][rows] - ref[rows]).max() / np.abs(ref[rows]).max()
+        parity(f"O sampled rows h={h}", err, TOL["bf16"])
         assert err <= TOL["bf16"], err
 
 
