@@ -333,6 +333,93 @@ def muse_partial_dipole_from_labels(Q, K, V, q_labels, k_labels, Cq: int, Ck: in
     return O
 
 
+# ----------------------------------------------------------------------------
+# Backward pass: the gradient of the same approximation.
+# [review] referee report and "What carries the argument": MuSe is used for pretraining,
+# so the approximation itself is differentiated (the pages never measure it).  Reading
+# taken: the clustering is held fixed (K-means assignments are discrete), the query
+# centroid qbar_i is the mean of its members (as K-means leaves it), so gradients flow
+# into Q through both qbar_i and the residuals; the key clustering enters only through
+# the member sets S_j.
+# ----------------------------------------------------------------------------
+
+def muse_backward_from_labels(Q, K, V, q_labels, k_labels, Cq: int, Ck: int, scale: float, dO):
+    """(dQ, dK, dV) = gradients of sum(O * dO) for O = muse_from_labels(Q, K, V, ...), labels
+    fixed, qbar the member means.  Chain rule through the definitions, in reverse order:
+
+      refinement   O_n = sum_j p_nj y_nj,  y_nj = mu_v,ij + s C_ij qt_n,
+                   p_n = softmax_j(a_nj),  a_nj = logZ_ij + s qt_n . mu_k,ij
+      summaries    w_ik = exp(s qbar_i.k - logZ_ij), mu_k = sum w k, mu_v = sum w v,
+                   C_ij = sum w v k^T - mu_v mu_k^T   (equal to the centred form)
+      centroids    qt_n = q_n - qbar_i,  qbar_i = mean of the members of cluster i
+    """
+    Q = np.asarray(Q, np.float64)
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    dO = np.asarray(dO, np.float64)
+    q_labels = np.asarray(q_labels)
+    k_labels = np.asarray(k_labels)
+    s = scale
+    N, D = Q.shape
+    Dv = V.shape[1]
+    qbar = cluster_means(Q, q_labels, Cq)
+    logZ, mu_k, mu_v, cov = tilted_summaries(qbar, K, V, k_labels, Ck, s)
+    dQt = np.zeros((N, D))
+    dlogZ = np.zeros((Cq, Ck))
+    dmuk = np.zeros((Cq, Ck, D))
+    dmuv = np.zeros((Cq, Ck, Dv))
+    dC = np.zeros((Cq, Ck, Dv, D))
+    live = np.isfinite(logZ)
+    # --- refinement, per query cluster
+    for i in np.unique(q_labels):
+        idx = np.nonzero(q_labels == i)[0]
+        Qt = Q[idx] - qbar[i][None, :]
+        a = np.where(live[i][None, :], logZ[i][None, :] + s * (Qt @ mu_k[i].T), NEG_INF)
+        m = a.max(axis=1)
+        p = np.exp(a - m[:, None])
+        p /= p.sum(axis=1)[:, None]
+        y = mu_v[i][None, :, :] + s * np.einsum("jvd,nd->njv", cov[i], Qt)   # [n, Ck, Dv]
+        dy = p[:, :, None] * dO[idx][:, None, :]                               # dO/dy
+        dp = np.einsum("nv,njv->nj", dO[idx], y)
+        da = p * (dp - (p * dp).sum(axis=1)[:, None])                         # softmax
+        dlogZ[i] += da.sum(axis=0)
+        dQt[idx] += s * (da @ mu_k[i]) + s * np.einsum("jvd,njv->nd", cov[i], dy)
+        dmuk[i] += s * (da.T @ Qt)
+        dmuv[i] += dy.sum(axis=0)
+        dC[i] += s * np.einsum("njv,nd->jvd", dy, Qt)
+    # --- summaries, per key cluster (all query centroids at once)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    dqbar = np.zeros((Cq, D))
+    for j in range(Ck):
+        kidx = np.nonzero(k_labels == j)[0]
+        if kidx.size == 0:
+            continue
+        Kj, Vj = K[kidx], V[kidx]
+        ell = s * (qbar @ Kj.T)                                  # [Cq, nj]
+        w = np.exp(ell - logZ[:, j][:, None])
+        G = dC[:, j]                                             # [Cq, Dv, D]
+        Gk = np.einsum("ivd,nd->inv", G, Kj)                     # G k_k
+        Gv = np.einsum("ivd,nv->ind", G, Vj)                     # G^T v_k
+        dmuv_t = dmuv[:, j] - np.einsum("ivd,id->iv", G, mu_k[:, j])   # through -mu_v mu_k^T
+        dmuk_t = dmuk[:, j] - np.einsum("ivd,iv->id", G, mu_v[:, j])
+        dw = (np.einsum("nv,inv->in", Vj, Gk)                    # v^T G k
+              + dmuk_t @ Kj.T + dmuv_t @ Vj.T)
+        dVj = np.einsum("in,inv->nv", w, Gk) + w.T @ dmuv_t
+        dKj = np.einsum("in,ind->nd", w, Gv) + w.T @ dmuk_t
+        dell = w * (dw - (w * dw).sum(axis=1)[:, None]) + w * dlogZ[:, j][:, None]
+        dqbar += s * (dell @ Kj)
+        dKj += s * (dell.T @ qbar)
+        dK[kidx] += dKj
+        dV[kidx] += dVj
+    # --- residuals and centroids
+    dQ = dQt.copy()
+    for i in np.unique(q_labels):
+        idx = np.nonzero(q_labels == i)[0]
+        dQ[idx] += (dqbar[i] - dQt[idx].sum(axis=0))[None, :] / idx.size
+    return dQ, dK, dV
+
+
 def muse_acausal(Q, K, V, Cq: int, Ck: int, iters: int, scale: float,
                  return_labels: bool = False, dipole: bool = True):
     """Full acausal MuSe: K-means on Q and on K, summaries, refinement."""

@@ -583,3 +583,54 @@ def test_retrieval_error_does_not_rise_with_k1_and_k2():
         assert all(b <= a * (1 + 1e-9) for a, b in zip(errs, errs[1:])), (seed, errs)
         assert errs[0] > 10 * errs[4], (seed, errs)   # retrieval makes a real difference
         assert errs[-1] < 1e-20, (seed, errs)          # k1 = Ck, k2 = nb: everything exact
+
+
+# --------------------------------------------------------------------------- backward pass
+
+def _fd_grad(f, X, h=1e-6):
+    g = np.zeros_like(X)
+    for idx in np.ndindex(X.shape):
+        Xp, Xm = X.copy(), X.copy()
+        Xp[idx] += h
+        Xm[idx] -= h
+        g[idx] = (f(Xp) - f(Xm)) / (2 * h)
+    return g
+
+
+@pytest.mark.parametrize("seed,D,Dv,s", [(0, 3, 2, 0.9), (1, 2, 4, 1.7), (2, 4, 4, 0.4)])
+def test_backward_matches_central_differences(seed, D, Dv, s):
+    """The backward pass against central finite differences of the forward oracle (labels
+    fixed, qbar the member means), with an empty key cluster and a singleton query cluster."""
+    rng = np.random.default_rng(seed)
+    N, Cq, Ck = 14, 3, 4
+    Q, K, V = rng.standard_normal((N, D)), rng.standard_normal((N, D)), rng.standard_normal((N, Dv))
+    ql = np.concatenate([[0, 1, 2], rng.integers(0, 2, N - 3)])   # cluster 2: one member
+    kl = np.concatenate([[0, 1, 2], rng.integers(0, 3, N - 3)])   # cluster 3: empty
+    dO = rng.standard_normal((N, Dv))
+    dQ, dK, dV = mo.muse_backward_from_labels(Q, K, V, ql, kl, Cq, Ck, s, dO)
+    loss = lambda Q_, K_, V_: float((mo.muse_from_labels(Q_, K_, V_, ql, kl, Cq, Ck, s) * dO).sum())
+    for got, fd in ((dQ, _fd_grad(lambda X: loss(X, K, V), Q)),
+                    (dK, _fd_grad(lambda X: loss(Q, X, V), K)),
+                    (dV, _fd_grad(lambda X: loss(Q, K, X), V))):
+        np.testing.assert_allclose(got, fd, rtol=0, atol=1e-7 * np.abs(fd).max())
+
+
+@pytest.mark.parametrize("case", ["singleton_keys", "singleton_queries"])
+def test_backward_is_exact_attention_gradient_in_the_exact_limits(case):
+    """Ck = N or Cq = N makes the approximation equal to exact attention as a function of
+    (Q, K, V), so its gradient must equal exact attention's, taken by torch autograd."""
+    import torch
+    Q, K, V = small_problem(41, 24, 5, 3, 4, 0.3)
+    rng = np.random.default_rng(9)
+    dO = rng.standard_normal((24, 3))
+    if case == "singleton_keys":
+        ql, kl, Cq, Ck = rng.integers(0, 4, 24), np.arange(24), 4, 24
+    else:
+        ql, kl, Cq, Ck = np.arange(24), rng.integers(0, 5, 24), 24, 5
+    dQ, dK, dV = mo.muse_backward_from_labels(Q, K, V, ql, kl, Cq, Ck, 1.3, dO)
+    t = [torch.tensor(x, requires_grad=True) for x in (Q, K, V)]
+    O = torch.nn.functional.scaled_dot_product_attention(t[0][None], t[1][None], t[2][None],
+                                                         scale=1.3)[0]
+    (O * torch.tensor(dO)).sum().backward()
+    for got, ref in zip((dQ, dK, dV), t):
+        np.testing.assert_allclose(got, ref.grad.numpy(), rtol=1e-10, atol=1e-12)
