@@ -11,8 +11,11 @@ timed one by one with CUDA events on the launching stream, with a 256 MiB write
 between steps to flush L2.  value = B*H*N*ranks / (mean step time), taking the
 max over ranks.  ``e2e`` repeats the measurement through the public API with the
 inputs copied from pinned host memory and the output copied back inside the
-timed region.  ``--impl reference`` times the float64 oracle on the host cores on
-a bounded sample (one head per step) of the same workload.
+timed region.  The default run (acausal N = 8k) also measures the metric's second
+headline size, the causal N = 16k workload, under the key ``second_headline``
+(``--no-second`` skips it).  ``--impl reference`` times the float64 oracle on the
+host cores, one (b,h) problem per step (extrapolated from timed parts where the
+problem is too large; the line says how).
 """
 from __future__ import annotations
 
@@ -34,6 +37,7 @@ sys.path.insert(0, ROOT)
 from clustered_softmax_attention_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "MuSe fwd tokens/s per head at N=8k/16k on 1 B200; % roofline; rel sq err"
+DEFAULT_WORKLOAD = "acausal_n8k_bf16"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # 148 SMs x 128 FP32 lanes x FMA x max clock
@@ -42,10 +46,12 @@ FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # 148 SMs x 128 FP32 lanes x
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="muse", choices=["muse", "reference"])
-    ap.add_argument("--workload", default="acausal_n8k_bf16", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-second", action="store_true",
+                    help="skip the second headline workload (causal N = 16k) of the default run")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--block", type=int, default=0,
@@ -157,6 +163,12 @@ def algorithmic_flops(w):
     P = w.B * w.H
     if w.mode == "acausal":
         return P * inst(w.N, w.N, w.Cq, w.Ck, w.D, w.Dv)
+    if w.mode == "retrieval":
+        # the remainder over every query's causal prefix: the method's count over the
+        # prefix (as in the acausal case) or the pair form over the causal pairs
+        s_form = 2.0 * w.Cq * w.N * w.D * w.Dv + 2.0 * w.N * w.Ck * w.D * w.Dv
+        n_form = 2.0 * (w.N * w.N / 2.0) * (w.D + w.Dv)
+        return P * min(s_form, n_form)
     if w.mode == "causal":
         tot = 0.0
         s = w.block
@@ -196,7 +208,7 @@ class ClockSampler:
     def start(self):
         try:
             cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                   "-lms", "100"]
+                   "-lms", "50"]
             if self.sel is not None:
                 cmd += ["-i", str(self.sel)]
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
@@ -369,24 +381,15 @@ def config_of(w, graph):
     return c
 
 
-def main():
-    args = parse()
-    rank, local_rank, world = dist_info()
-    import torch
-    import torch.distributed as dist
-    if world > 1:
-        dist.init_process_group("nccl" if args.impl == "muse" else "gloo",
-                                timeout=datetime.timedelta(seconds=300))
-    if args.impl == "reference":
-        run_reference(args, rank, world)
-        if world > 1:
-            dist.destroy_process_group()
-        return
+SECOND_HEADLINE = "causal_n16k_bf16"   # the metric's other headline size (N = 16k, causal)
 
+
+def measure(args, w, steps, warmup, world, rank, local_rank, cpu_baseline):
+    """Time `steps` whole forward passes of workload w on this rank; the JSON fields of
+    the measurement (rank 0: with the sampled RSE and, if asked, the CPU baseline)."""
+    import torch
     from clustered_softmax_attention_b200 import muse as m
-    torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = workload_of(args)
     Qn, Kn, Vn = make_inputs(w)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     Qh = torch.from_numpy(Qn).to(tdt).pin_memory()
@@ -396,10 +399,12 @@ def main():
     Od = torch.empty(w.B, w.H, w.N, w.Dv, dtype=tdt, device=dev)
     Oh = torch.empty_like(Od, device="cpu").pin_memory()
     d = m.dims(Qd, Vd, w.scale)
+    monopole = args.monopole and w.mode == "acausal"
+    partial = args.partial_dipole and w.mode == "acausal"
     if w.mode == "acausal":
         ws = m.workspace("muse_forward_ex", d, w.Cq, w.Ck)
-        flags = (m.MUSE_FLAG_MONOPOLE if args.monopole else 0) | \
-            (m.MUSE_FLAG_PARTIAL_DIPOLE if args.partial_dipole else 0)
+        flags = (m.MUSE_FLAG_MONOPOLE if monopole else 0) | \
+            (m.MUSE_FLAG_PARTIAL_DIPOLE if partial else 0)
 
         def step(Q=Qd, K=Kd, V=Vd, O=Od):
             m.muse_forward_ex(Q, K, V, w.Cq, w.Ck, w.iters, w.scale, flags=flags, out=O, ws=ws)
@@ -424,7 +429,7 @@ def main():
     kev1.record(stream)
     m.lib().muse_set_profile_events(ctypes_ptr(kev0), ctypes_ptr(kev1))
 
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         step()
     torch.cuda.synchronize()
     n0 = m.lib().muse_launch_counter()
@@ -460,15 +465,14 @@ def main():
             step()
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
+          for _ in range(steps)]
+    barrier(world)
     torch.cuda.synchronize()
     clocks = ClockSampler(nvsmi_index(local_rank))
     clocks.start()
     time.sleep(0.3)
     step_ms, kern_ms = [], []
-    for k in range(args.steps):
+    for k in range(steps):
         flush.zero_()
         ev[k][0].record(stream)
         run_step()
@@ -477,10 +481,9 @@ def main():
         step_ms.append(ev[k][0].elapsed_time(ev[k][1]))
         kern_ms.append(kev0.elapsed_time(kev1))
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     clk = clocks.stop()
-    mean_ms = max_over_ranks(sum(step_ms), dev) / args.steps
+    mean_ms = max_over_ranks(sum(step_ms), dev) / steps
     tokens = w.B * w.H * w.N
     value = world * tokens / (mean_ms / 1e3)
     assert m.muse_last_device_status() == 0
@@ -488,7 +491,7 @@ def main():
     # end to end through the public API: pinned host inputs -> device -> output -> host
     m.lib().muse_set_profile_events(None, None)
     e2e_ms = []
-    for k in range(max(2, args.steps // 2)):
+    for k in range(max(2, steps // 2)):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -504,30 +507,25 @@ def main():
     h2d = sum(x.numel() * x.element_size() for x in (Qh, Kh, Vh))
     d2h = Oh.numel() * Oh.element_size()
 
-    # roofline of the dominant kernel (the refinement), timed live above; the retrieval
-    # path runs on CUDA cores only and is rated as a whole step against the FP32 peak
+    # roofline of the dominant kernel (the refinement; on the retrieval workload its
+    # retrieval mode, the remainder), timed live above
     peaks, peak_src = load_peaks()
-    if w.mode == "retrieval":
-        kmean = mean_ms
-        flops = retrieval_flops(w)
-        achieved = flops / (kmean / 1e3) / 1e12
-        roof = {"bound": "alu", "achieved": achieved, "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
-                "frac": achieved / FP32_SIMT_TFLOPS, "traffic": None,
-                "kernel": "whole step (CUDA cores)", "kernel_ms": kmean, "flops_per_launch": flops,
-                "peak_source": "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
+    kmean = sum(kern_ms) / len(kern_ms)
+    flops = algorithmic_flops(w)
+    achieved = flops / (kmean / 1e3) / 1e12
+    if w.dtype == "bf16":
+        peak, bound, unit = float(peaks["bf16_tflops"]), "tensor", "TFLOP/s"
     else:
-        kmean = sum(kern_ms) / len(kern_ms)
-        flops = algorithmic_flops(w)
-        achieved = flops / (kmean / 1e3) / 1e12
-        if w.dtype == "bf16":
-            peak, bound, unit = float(peaks["bf16_tflops"]), "tensor", "TFLOP/s"
-        else:
-            peak, bound, unit = FP32_SIMT_TFLOPS, "alu", "TFLOP/s"
-        roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": recorded_traffic(w.name),
-                "kernel": "refinement", "kernel_ms": kmean, "flops_per_launch": flops,
-                "peak_source": f"{peak_src} bf16_tflops (burst)" if w.dtype == "bf16"
-                else "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
+        peak, bound, unit = FP32_SIMT_TFLOPS, "alu", "TFLOP/s"
+    roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": recorded_traffic(w.name),
+            "kernel": "refinement (retrieval remainder)" if w.mode == "retrieval"
+            else "refinement", "kernel_ms": kmean, "flops_per_launch": flops,
+            "peak_source": f"{peak_src} bf16_tflops (burst)" if w.dtype == "bf16"
+            else "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
+    if w.mode == "retrieval":
+        roof["step_flops"] = retrieval_flops(w)
+    out = None
     if rank == 0:
         try:
             from oracle import muse_oracle as mo
@@ -540,30 +538,70 @@ def main():
         except Exception:
             rse = None
         cpu = None
-        if world == 1 and not args.no_cpu_baseline:
+        if cpu_baseline:
             secs, n, note = oracle_sample(w)
             what = f"one (b,h) problem of {w.name} (N={w.N} tokens)"
             if note:
                 what += f"; {note}"
             cpu = {"value": n / secs, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                    "sample": f"{what}, float64 numpy oracle, {secs:.1f} s"}
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": w.dtype, "data": "synthetic (seeded Gaussian-mixture Q/K, normal V)",
+        out = {
+            "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": warmup,
+            "ms_per_step": mean_ms, "dtype": w.dtype,
             "config": dict(config_of(w, graph is not None),
-                           **({"monopole": True} if args.monopole else {}),
-                           **({"partial_dipole": True} if args.partial_dipole else {})),
+                           **({"monopole": True} if monopole else {}),
+                           **({"partial_dipole": True} if partial else {})),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": launches_per_step * steps,
             "clocks": clk, "rse_vs_exact_sampled": rse,
             "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms),
         }
-        print(json.dumps(line), flush=True)
     del graph
+    return out
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def main():
+    args = parse()
+    rank, local_rank, world = dist_info()
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl" if args.impl == "muse" else "gloo",
+                                timeout=datetime.timedelta(seconds=300))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    torch.cuda.set_device(local_rank)
+    w = workload_of(args)
+    res = measure(args, w, args.steps, args.warmup, world, rank, local_rank,
+                  cpu_baseline=(world == 1 and not args.no_cpu_baseline))
+    # the metric names two headline sizes: the default run also measures the causal 16k
+    # workload (every rank, same collective steps), reported under its own key
+    second = None
+    if args.workload == DEFAULT_WORKLOAD and not args.no_second and not (
+            args.block or args.clusters or args.iters or args.monopole or args.partial_dipole):
+        second = measure(args, WORKLOADS[SECOND_HEADLINE], max(10, args.steps // 4), args.warmup,
+                         world, rank, local_rank, cpu_baseline=False)
+    if rank == 0:
+        line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": res["dtype"], "data": "synthetic (seeded Gaussian-mixture Q/K, normal V)"}
+        line.update({k: v for k, v in res.items() if k not in line})
+        if second is not None:
+            line["second_headline"] = dict(second, workload=SECOND_HEADLINE)
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
 

@@ -203,9 +203,11 @@ diag_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUten
     // natural-log units from here: m = m2 / log2(e)
     float m = m2 * 0.6931471805599453f;
     if (n < N) {
-      for (int lev = 1; lev <= levels; ++lev) {
-        if (!((bidx >> (lev - 1)) & 1)) continue;
-        const int64_t r = ((int64_t)p * levels + (lev - 1)) * N + n;
+      // levels < 0: a single partial array, merged into every row
+      const int nlev = levels < 0 ? 1 : levels;
+      for (int lev = 1; lev <= nlev; ++lev) {
+        if (levels > 0 && !((bidx >> (lev - 1)) & 1)) continue;
+        const int64_t r = ((int64_t)p * nlev + (lev - 1)) * N + n;
         const float L = part_lse[r];
         if (!(L > -CUDART_INF_F)) continue;
         const float mn = fmaxf(m, L);
@@ -239,11 +241,13 @@ diag_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUten
   // copies and MMAs still in flight land before the CTA releases its memory
   if (t == 0) {
     mbar_drain(&sm.lbar, (lph - 1) & 1, status);  // the last load issued
-    // a wait that gave up leaves phase mph - 1 possibly incomplete: drain it first (a
-    // parity probe for phase mph alone would see the completed phase mph - 2), then the
-    // phase of a final commit that tracks every MMA issued
-    tc_commit(&sm.mbar);
+    // A wait that gave up may leave MMA phase mph - 1 incomplete: drain it before the final
+    // commit (once that commit has landed, the parity of phase mph - 1 is also that of the
+    // open phase mph + 1, and the probe would wait for good).  On the normal path phase
+    // mph - 1 is complete and the probe returns at once.  Then the final commit's phase,
+    // which tracks every MMA issued.
     if (mph > 0) mbar_drain(&sm.mbar, (mph - 1) & 1, status);
+    tc_commit(&sm.mbar);
     mbar_drain(&sm.mbar, mph & 1, status);
   }
   tc_fence_before();

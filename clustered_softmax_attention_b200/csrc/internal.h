@@ -17,6 +17,10 @@ void count_launches(int n);
 // Device address of the current device's status word (NULL if unavailable).
 int *device_status_word();
 
+// Records the event set by muse_set_profile_events before (start) or after the dominant
+// kernel of a call, when events are set; cudaSuccess otherwise.
+cudaError_t profile_mark(bool start, cudaStream_t st);
+
 // Per-instance offsets of the stage buffers.  An instance pairs query segment s
 // with key segment s (acausal: the one whole-sequence segment; causal: one square).
 struct InstTable {
@@ -101,9 +105,27 @@ cudaError_t run_coeffs(const MuseTables &mt, int dtype, int D, int P, float scal
 cudaError_t run_refine(const MuseTables &mt, int dtype, int D, int Dv, int N, int P,
                        SortedSide qs, const int32_t *q_perm, SortedSide ks, const void *vs_rows,
                        StageBufs b, void *O, float *part_o, float *part_lse, cudaStream_t st);
+// The refinement from materialised summaries (refine_summaries.cu): O_n = sum_j p_j
+// (mu_v,ij + s C_ij qt) with p = softmax_j(logZ_ij + s qt.mu_k,ij), float32 on the CUDA
+// cores.  q_labels (natural order) is optional; a row whose label disagrees with
+// q_perm / q_offsets is reported as MUSE_ERR_DEVICE.
+cudaError_t run_refine_summaries(int dtype, int D, int Dv, int N, int P, int Cq, int Ck,
+                                 float scale, const void *Q, const float *q_centroids,
+                                 const int32_t *q_perm, const int32_t *q_offsets,
+                                 const int32_t *q_labels, const float *logZ, const float *mu_k,
+                                 const float *mu_v, const float *cov, void *O, int *status,
+                                 cudaStream_t st);
+// Backward pass (backward.cu): dQ, dK, dV of sum(O * dO), clusterings fixed.
+size_t muse_backward_ws(const muse_dims &d, int Cq, int Ck);
+cudaError_t run_backward(const void *Q, const void *K, const void *V, const void *dO,
+                         const int32_t *q_perm, const int32_t *q_offsets, const int32_t *k_perm,
+                         const int32_t *k_offsets, const muse_dims &d, int Cq, int Ck, void *dQ,
+                         void *dK, void *dV, void *ws, cudaStream_t st);
 size_t muse_retrieval_ws(const muse_dims &d, int block, int Cq, int Ck, int k1, int k2);
 // The exact diagonal on the tensor cores (diag_tc.cu): bf16, D = Dv = 64, block a
-// multiple of 128 and at most 512.
+// multiple of 128.  levels > 0: the causal decomposition's level partials
+// part_*[P][levels][N] (level l merged into the rows of blocks whose bit l-1 is set);
+// levels < 0: one partial array part_*[P][N] merged into every row (retrieval).
 bool diag_tc_supported(int dtype, int D, int Dv, int N, int block);
 cudaError_t run_diag_tc(const void *Q, const void *K, const void *V, int N, int P, int block,
                         int levels, float scale, const float *part_o, const float *part_lse,

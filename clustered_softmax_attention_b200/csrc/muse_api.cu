@@ -220,6 +220,12 @@ static cudaError_t record_profile_event(void *ev, cudaStream_t st) {
   return cudaEventRecord((cudaEvent_t)ev, st);
 }
 
+cudaError_t profile_mark(bool start, cudaStream_t st) {
+  void *ev0 = g_prof_start.load(), *ev1 = g_prof_stop.load();
+  if (!ev0 || !ev1) return cudaSuccess;
+  return record_profile_event(start ? ev0 : ev1, st);
+}
+
 // The refinement launch sequence shared by every path.
 static muse_status refine_path(const void *Q, const void *K, const void *V, const muse_dims &d,
                                int P, const MuseTables &mt, const float *q_centroids,
@@ -248,8 +254,7 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
   }
   // the dipole terms carry the logit scale; the monopole-only ablation drops them
   MUSE_TRY(run_coeffs(mt, d.dtype, d.D, P, d.scale, r.qs, q_offsets, sb, monopole ? 0.f : d.scale, st));
-  void *ev0 = g_prof_start.load(), *ev1 = g_prof_stop.load();
-  if (ev0 && ev1) MUSE_TRY(record_profile_event(ev0, st));
+  MUSE_TRY(profile_mark(true, st));
   if (use_tc) {
     MUSE_TRY(run_refine_tc(mt, d.D, d.Dv, d.N, P, r.qs, q_perm, r.ks, k_offsets, r.vs, sb, O,
                            part_o, part_lse, status_ptr(), st));
@@ -257,7 +262,7 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
     MUSE_TRY(run_refine(mt, d.dtype, d.D, d.Dv, d.N, P, r.qs, q_perm, r.ks, r.vs, sb, O, part_o,
                         part_lse, st));
   }
-  if (ev0 && ev1) MUSE_TRY(record_profile_event(ev1, st));
+  MUSE_TRY(profile_mark(false, st));
   return MUSE_OK;
 }
 
@@ -398,6 +403,7 @@ extern "C" size_t muse_workspace_size(const char *entry, muse_dims d, int Cq, in
     return ws_causal(d, block, Cq, Ck);
   }
   if (!strcmp(entry, "muse_retrieve_exact")) return muse_retrieval_ws(d, block, Cq, Ck, k1, k2);
+  if (!strcmp(entry, "muse_backward")) return valid_C(Ck, d.N) ? muse_backward_ws(d, Cq, Ck) : 0;
   return 0;
 }
 
@@ -479,20 +485,33 @@ extern "C" muse_status muse_tilted_summaries(const float *q_centroids, const voi
 // --------------------------------------------------------------------------- refine
 
 extern "C" muse_status muse_dipole_refine(const void *Q, const void *K, const void *V,
-                                          const float *q_centroids, const int32_t *q_perm,
-                                          const int32_t *q_offsets, const int32_t *k_perm,
-                                          const int32_t *k_offsets, const float *logZ,
-                                          const float *mu_k, muse_dims d, int Cq, int Ck, void *O,
-                                          void *ws, size_t ws_bytes, muse_stream_t st) {
+                                          const int32_t *q_labels, const float *q_centroids,
+                                          const int32_t *q_perm, const int32_t *q_offsets,
+                                          const int32_t *k_perm, const int32_t *k_offsets,
+                                          const float *logZ, const float *mu_k,
+                                          const float *mu_v, const float *cov, muse_dims d,
+                                          int Cq, int Ck, void *O, void *ws, size_t ws_bytes,
+                                          muse_stream_t st) {
   muse_status s = check_dims(d, true);
   if (s != MUSE_OK) return s;
   const void *ptrs[] = {Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offsets, logZ, mu_k, O};
   for (const void *p : ptrs)
     if (!p || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  for (const void *p : {(const void *)q_labels, (const void *)mu_v, (const void *)cov})
+    if (p && !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  if (!mu_v != !cov) return MUSE_ERR_INVALID_ARG;  // both materialised, or neither
   if (!valid_C(Cq, d.N) || !valid_C(Ck, d.N)) return MUSE_ERR_INVALID_ARG;
   const size_t need = ws_refine(d, Cq, Ck);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
   const int P = d.B * d.H;
+  if (cov) {
+    // the summaries are given: the refinement reads them as they are
+    if (run_refine_summaries(d.dtype, d.D, d.Dv, d.N, P, Cq, Ck, d.scale, Q, q_centroids, q_perm,
+                             q_offsets, q_labels, logZ, mu_k, mu_v, cov, O, status_ptr(),
+                             (cudaStream_t)st) != cudaSuccess)
+      return MUSE_ERR_CUDA;
+    return MUSE_OK;
+  }
   MuseTables mt;
   mt.q = whole_side(d.N, Cq);
   mt.k = whole_side(d.N, Ck);
@@ -608,6 +627,27 @@ extern "C" muse_status muse_causal_blocks(const void *Q, const void *K, const vo
   if (s != MUSE_OK) return s;
   if (run_diag_merge(Q, K, V, d.dtype, d.D, d.Dv, d.N, P, block, L, d.scale, part_o, part_lse, O,
                      cs) != cudaSuccess)
+    return MUSE_ERR_CUDA;
+  return MUSE_OK;
+}
+
+// --------------------------------------------------------------------------- backward
+
+extern "C" muse_status muse_backward(const void *Q, const void *K, const void *V, const void *dO,
+                                     const int32_t *q_perm, const int32_t *q_offsets,
+                                     const int32_t *k_perm, const int32_t *k_offsets, muse_dims d,
+                                     int Cq, int Ck, void *dQ, void *dK, void *dV, void *ws,
+                                     size_t ws_bytes, muse_stream_t st) {
+  muse_status s = check_dims(d, true);
+  if (s != MUSE_OK) return s;
+  const void *ptrs[] = {Q, K, V, dO, q_perm, q_offsets, k_perm, k_offsets, dQ, dK, dV};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
+  if (!valid_C(Cq, d.N) || !valid_C(Ck, d.N)) return MUSE_ERR_INVALID_ARG;
+  const size_t need = muse_backward_ws(d, Cq, Ck);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
+  if (run_backward(Q, K, V, dO, q_perm, q_offsets, k_perm, k_offsets, d, Cq, Ck, dQ, dK, dV, ws,
+                   (cudaStream_t)st) != cudaSuccess)
     return MUSE_ERR_CUDA;
   return MUSE_OK;
 }

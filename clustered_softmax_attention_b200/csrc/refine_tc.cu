@@ -28,6 +28,17 @@
 // parity g, so the groups overlap; warps 10-11 = cp.async producers
 // of the epilogue data (tiles of parity 0 and 1).  Every wait on an mbarrier is
 // bounded: past the limit the kernel records MUSE_ERR_TIMEOUT and winds down.
+//
+// Retrieval mode (RET): the remainder of causal accumulation with retrieval
+// (gist.science "Kernmechanismen" items 3-4) has the same pair form over the global
+// clusters, restricted per query: query n (block b, cluster i) takes the keys of every
+// cluster in blocks b' < b, minus the (cluster, block) pairs selected for (i, b), which
+// are attended exactly elsewhere; c0, c1 then carry the remainder coefficients.  The
+// keys of a cluster are in token order, so for the CTA's latest query block b_hi each
+// cluster contributes a prefix of its sorted keys; the tiles walk those prefixes only.
+// Per element the epilogue masks key blocks b' >= b (a per-chunk block range decides
+// most chunks at once) and, for the few tiles holding a selected cluster of the row,
+// the selected blocks.
 #include <cuda.h>
 
 #include "tc.h"
@@ -65,6 +76,10 @@ struct __align__(1024) Smem {
   unsigned char seg[NST][BN];                  // column -> cluster of the tile (0xFF: masked)
   int chunk[NST][BN / 16];                     // per 16 columns: mask, clusters, split (or kComplex)
   int koff[kMaxClusters + 1];                  // the instance's key-cluster offsets
+  int kend[kMaxClusters];                      // RET: end of each cluster's causal prefix
+  unsigned short kblk[NST][BN];                // RET: key block of every column
+  int crng[NST][BN / 16];                      // RET: min | max << 16 key block per 16 columns
+  int wbhi[BM / 32];                           // RET: latest query block per row warp
   int tnpad[4];                                // padded width of the tiles in flight (MMA issuer)
   // per stage: key tile (consumed by the first MMA), values (second MMA), epilogue
   // data (tilt weights, coefficients, segment map; consumed by the epilogue)
@@ -115,19 +130,31 @@ static __device__ __noinline__ P8 mixed_chunk(const Smem<D, DV> &sm, int st, int
 struct KTile {
   int j, nseg, c, n, x0, npad;
 };
+// With `live` (retrieval mode) only the first live[j] - off[j] keys of cluster j are
+// walked: a window ends where a cluster's live keys end before the cluster does.
 template <int BN>
 struct TileIter {
   const int32_t *off;
+  const int32_t *live;
   int C;
   KTile t;
-  __device__ void begin(const int32_t *o, int Ck) {
+  __device__ void begin(const int32_t *o, int Ck, const int32_t *lv = nullptr) {
     off = o;
+    live = lv;
     C = Ck;
     make(0, off[0]);
   }
   // The window starting at key c, which lies in cluster j or a later one.
   __device__ void make(int j, int c) {
-    while (j < C && c >= off[j + 1]) ++j;
+    if (live) {
+      while (j < C) {
+        if (c < off[j]) c = off[j];
+        if (c < live[j]) break;
+        ++j;
+      }
+    } else {
+      while (j < C && c >= off[j + 1]) ++j;
+    }
     t.j = j;
     t.c = c;
     if (j >= C) return;
@@ -135,7 +162,18 @@ struct TileIter {
     int end = min(t.x0 + BN, off[C]);
     if (j + kTileSegs < C) end = min(end, off[j + kTileSegs]);
     int last = j;  // cluster holding key end-1
-    while (last + 1 < C && off[last + 1] < end) ++last;
+    if (live) {
+      while (true) {
+        if (live[last] < off[last + 1]) {  // dead keys follow: the window stops there
+          end = min(end, live[last]);
+          break;
+        }
+        if (last + 1 >= C || off[last + 1] >= end) break;
+        ++last;
+      }
+    } else {
+      while (last + 1 < C && off[last + 1] < end) ++last;
+    }
     t.nseg = last - j + 1;
     t.n = end - c;
     t.npad = ((end - t.x0) + 15) & ~15;
@@ -145,7 +183,45 @@ struct TileIter {
   __device__ void next() { make(t.j + t.nseg - 1, t.c + t.n); }
 };
 
+// Retrieval-mode arguments (unused by the plain refinement).
+struct RetArgs {
+  const int32_t *k_perm;  // [P][N] sorted key position -> token
+  const int32_t *pend;    // [P][Ck][nb + 1] keys of cluster j in blocks < b'
+  const int32_t *sel;     // [P][Cq][nb][K12][2] (cluster, block) pairs selected per (i, b)
+  int S, nb, k1, k2, K12, Cq;
+};
+
+// RET: columns of chunk cb whose key block precedes the row's block brow (the chunk's
+// block range was not enough to decide).
 template <int D, int DV>
+static __device__ __noinline__ uint32_t causal_bits(const Smem<D, DV> &sm, int st, int cb, int brow) {
+  uint32_t keep = 0;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) keep |= (sm.kblk[st][cb * 16 + e] < brow ? 1u : 0u) << e;
+  return keep;
+}
+// RET: columns of chunk cb that are not in a (cluster, block) pair selected for the row
+// (so, its k1 x k2 slots; xseg: the tile segments whose cluster the row selected).
+template <int D, int DV>
+static __device__ __noinline__ uint32_t excl_bits(const Smem<D, DV> &sm, int st, int cb,
+                                                  uint32_t xseg, int tj, const int32_t *so,
+                                                  int k1, int k2) {
+  uint32_t keep = 0xFFFFu;
+  for (int e = 0; e < 16; ++e) {
+    const int col = cb * 16 + e;
+    const int g = sm.seg[st][col];
+    if (g == 0xFF || !((xseg >> g) & 1u)) continue;
+    const int j = tj + g, b = sm.kblk[st][col];
+    for (int t = 0; t < k1; ++t) {
+      if (so[2 * t * k2] != j) continue;
+      for (int u = 0; u < k2; ++u)
+        if (so[2 * (t * k2 + u) + 1] == b) keep &= ~(1u << e);
+    }
+  }
+  return keep;
+}
+
+template <int D, int DV, bool RET>
 __global__ void __launch_bounds__(kThreads, 1)
 refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                  const __grid_constant__ CUtensorMap map_vt, MuseTables mt, int N,
@@ -154,7 +230,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                  const float *__restrict__ c0g, const float *__restrict__ c1g,
                  const float *__restrict__ lse, __nv_bfloat16 *__restrict__ O,
                  float *__restrict__ part_o, float *__restrict__ part_lse, int *status,
-                 const __grid_constant__ BlockMap bm) {
+                 const __grid_constant__ BlockMap bm, const RetArgs ra) {
   constexpr int BN = TileCfg<D, DV>::BN;
   // blockIdx.x: a 128-row block of one instance (compact grid), blockIdx.y: the problem
   int bfirst;
@@ -197,6 +273,22 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   for (int j = threadIdx.x; j <= k.C; j += blockDim.x) sm.koff[j] = k_offsets[k.off + j];
+  if constexpr (RET) {
+    // the CTA's latest query block b_hi: each key cluster takes the keys of blocks < b_hi
+    if (warp < BM / 32) {
+      const int n = r0 + threadIdx.x;
+      int b = n < q.n ? q_perm[q.lab + n] / ra.S : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) b = max(b, __shfl_xor_sync(0xffffffffu, b, o));
+      if (lane == 0) sm.wbhi[warp] = b;
+    }
+    __syncthreads();
+    int bhi = 0;
+#pragma unroll
+    for (int w = 0; w < BM / 32; ++w) bhi = max(bhi, sm.wbhi[w]);
+    const int32_t *pe = ra.pend + (int64_t)p * k.C * (ra.nb + 1) + bhi;
+    for (int j = threadIdx.x; j < k.C; j += blockDim.x) sm.kend[j] = sm.koff[j] + pe[(int64_t)j * (ra.nb + 1)];
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -204,6 +296,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   const uint32_t tmem_o = tmem + kSBuf * BN;
   auto s_col = [](int buf) { return (uint32_t)(buf * BN); };  // S(t) and, over it, P(t)
   const int32_t *koff = sm.koff;
+  const int32_t *kend = RET ? sm.kend : nullptr;
   const int kcol0 = (int)(k.lab - (int64_t)p * mt.k.row_stride);  // instance's first key column
   const int wl = w_ld(k.n), cl = w_ld(q.n);
   const float *Wi = W + (int64_t)p * mt.in.w_stride + mt.in.w0[s];      // row i: Wi + i*wl
@@ -228,7 +321,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       uint64_t *full = keys ? sm.fullk : sm.fullv;
       uint64_t *empty = keys ? sm.emptyk : sm.emptyv;
       TileIter<BN> it;
-      it.begin(koff, k.C);
+      it.begin(koff, k.C, kend);
       int t = 0;
       for (; !it.done(); it.next(), ++t) {
         const KTile kt = it.get();
@@ -255,7 +348,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     // warp kEWarp + par stages the tiles of parity par (stages par, par + 2, ...)
     const int par = warp - kEWarp;
     TileIter<BN> it;
-    it.begin(koff, k.C);
+    it.begin(koff, k.C, kend);
     int t = 0;
     for (; !it.done(); it.next(), ++t) {
       if ((t & 1) != par) continue;
@@ -295,6 +388,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           for (int b = 0; b < kTileSegs - 1; ++b) sg += key >= bnd[b] ? 1 : 0;
         }
         sm.seg[st][col] = (unsigned char)sg;
+        if constexpr (RET) sm.kblk[st][col] = (unsigned short)(sg == 0xFF ? 0xFFFF : ra.k_perm[k.lab + key] / ra.S);
       }
       // per 16-column chunk: valid-column mask (a contiguous run) << 16, the key
       // clusters of its first and last valid columns (bits 0-3, 4-7) and the first
@@ -321,6 +415,20 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         sm.chunk[st][lane] = code;
       }
       __syncwarp();
+      if constexpr (RET) {
+        // per 16 columns: the smallest and largest key block of the valid columns
+        if (lane < BN / 16) {
+          int lo = 0xFFFF, hi = 0;
+          for (int e = 0; e < 16; ++e) {
+            if (sm.seg[st][16 * lane + e] == 0xFF) continue;
+            const int b = sm.kblk[st][16 * lane + e];
+            lo = min(lo, b);
+            hi = max(hi, b);
+          }
+          sm.crng[st][lane] = lo | (hi << 16);
+        }
+        __syncwarp();
+      }
       if (lane == 0) mbar_arrive(&sm.fulle[st]);  // releases the segment map with the stage
     }
     if (lane == 0)
@@ -336,7 +444,7 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       bool ok = mbar_wait<true>(&sm.qbar, 0, abort_flag, status);
       tc_fence_after();
       TileIter<BN> it;
-      it.begin(koff, k.C);
+      it.begin(koff, k.C, kend);
       int g1 = 0, g2 = 0;  // next tile of each contraction
       int idle = 0;
       uint64_t t_idle = 0;
@@ -416,8 +524,16 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const bool wfast = __all_sync(0xffffffffu, staged);  // every row of the warp has staged weights
     const float *wrow = Wi + (int64_t)i * wl;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    int brow = 0;                 // RET: the row's query block (0 masks every key)
+    const int32_t *so = nullptr;  // RET: the row's selected (cluster, block) slots
+    if constexpr (RET) {
+      if (valid) {
+        brow = q_perm[q.lab + n] / ra.S;
+        so = ra.sel + (((int64_t)p * ra.Cq + i) * ra.nb + brow) * ra.K12 * 2;
+      }
+    }
     TileIter<BN> it;
-    it.begin(koff, k.C);
+    it.begin(koff, k.C, kend);
     int t = 0;
     bool ok = true;
     for (; !it.done(); it.next(), ++t) {
@@ -434,6 +550,14 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       tc_fence_after();
       const float *wsm = &sm.w[st][staged ? slot : 0][0];
       const int nch16 = kt.npad / 16;
+      uint32_t xseg = 0;  // RET: tile segments holding a cluster the row selected
+      if constexpr (RET) {
+        if (so && brow > 0)
+          for (int t1 = 0; t1 < ra.k1; ++t1) {
+            const int d = so[2 * t1 * ra.k2] - kt.j;
+            if (so[2 * t1 * ra.k2] >= 0 && d >= 0 && d < kt.nseg) xseg |= 1u << d;
+          }
+      }
       // P for 16 columns of S held in x, stored as 8 packed bf16 columns over the same
       // buffer: chunk cb's P lands in S columns 8 cb .. 8 cb + 7, which belong to S chunk
       // cb / 2, already read (and waited for) by this thread; the load in flight is of
@@ -441,11 +565,19 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
       auto chunk = [&](int cb, const uint32_t(&x)[16]) {
         const int code = sm.chunk[st][cb];
+        uint32_t keep = 0xFFFFu;  // RET: the row's causal and exclusion mask of the chunk
+        if constexpr (RET) {
+          const int rng = sm.crng[st][cb];
+          const int blo = rng & 0xFFFF, bhi = rng >> 16;
+          if (blo >= brow) keep = 0u;
+          else if (bhi >= brow) keep = causal_bits<D, DV>(sm, st, cb, brow);
+          if (xseg && keep) keep &= excl_bits<D, DV>(sm, st, cb, xseg, kt.j, so, ra.k1, ra.k2);
+        }
         uint32_t pk[8];
         if (wfast && !(code & kComplex)) {
           // at most two key clusters over the chunk's valid columns
           const int glo = code & 15, ghi = (code >> 4) & 15, split = (code >> 8) & 31;
-          const uint32_t msk = (uint32_t)code >> 16;
+          const uint32_t msk = ((uint32_t)code >> 16) & keep;
           const float b0 = sm.c0[st][glo][r], b1 = sm.c1[st][glo][r];
           float w[16];
 #pragma unroll
@@ -488,7 +620,11 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           for (int e = 0; e < 16; ++e) xv.v[e] = __uint_as_float(x[e]);
           const P8 pr = mixed_chunk<D, DV>(sm, st, cb, r, staged ? wsm : wrow + kt.x0, xv);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) pk[e] = pr.v[e];
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t hm = (((keep >> (2 * e)) & 1u) ? 0x0000FFFFu : 0u) |
+                                (((keep >> (2 * e + 1)) & 1u) ? 0xFFFF0000u : 0u);
+            pk[e] = pr.v[e] & hm;
+          }
         }
         tmem_st8(tmem + lane_base + s_col(buf) + cb * 8, pk);
       };
@@ -545,9 +681,18 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const int64_t rr = (int64_t)p * mt.in.out_stride + mt.in.out0[s] + row;
         part_lse[rr] = lse[q.lab + n];
       }
-    } else if (t == 0 && valid && grp == 0) {
-      // an instance with no keys cannot occur (every key range is non-empty)
-      report(status, MUSE_ERR_DEVICE);
+    } else if (t == 0 && valid) {
+      if constexpr (RET) {
+        // every row of the CTA lies in block 0: no key precedes it, the partial is empty
+        const int row = q_perm[q.lab + n];
+        const int64_t rr = (int64_t)p * mt.in.out_stride + mt.in.out0[s] + row;
+        float4 *dst = reinterpret_cast<float4 *>(part_o + rr * DV);
+        for (int c = grp; c < DV / 4; c += 2) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (grp == 0) part_lse[rr] = lse[q.lab + n];
+      } else if (grp == 0) {
+        // an instance with no keys cannot occur (every key range is non-empty)
+        report(status, MUSE_ERR_DEVICE);
+      }
     }
   }
   tc_fence_before();
@@ -561,10 +706,11 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 }
 
 // ------------------------------------------------------------------ host side
-template <int D, int DV>
+template <int D, int DV, bool RET>
 static cudaError_t launch(const MuseTables &mt, int N, int P, SortedSide qs, const int32_t *q_perm,
                           SortedSide ks, const int32_t *k_offsets, const void *vt, StageBufs b,
-                          void *O, float *part_o, float *part_lse, int *status, cudaStream_t st) {
+                          void *O, float *part_o, float *part_lse, int *status, cudaStream_t st,
+                          const RetArgs &ra) {
   CUtensorMap mq, mk, mv;
   const int ldv = vt_ld(mt.k.row_stride);
   if (!make_map(&mq, qs.rows, D, (uint64_t)P * mt.q.row_stride, D, BM) ||
@@ -572,14 +718,14 @@ static cudaError_t launch(const MuseTables &mt, int N, int P, SortedSide qs, con
       !make_map(&mv, vt, ldv, (uint64_t)P * DV, ldv, DV))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem<D, DV>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(refine_tc_kernel<D, DV>,
+  cudaError_t e = cudaFuncSetAttribute(refine_tc_kernel<D, DV, RET>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const BlockMap bm = make_block_map(mt.q, BM);
   dim3 grid(bm.total, P);
-  refine_tc_kernel<D, DV><<<grid, kThreads, smem, st>>>(
+  refine_tc_kernel<D, DV, RET><<<grid, kThreads, smem, st>>>(
       mq, mk, mv, mt, N, q_perm, qs.cluster, k_offsets, b.W, b.c0, b.c1, b.lse,
-      (__nv_bfloat16 *)O, part_o, part_lse, status, bm);
+      (__nv_bfloat16 *)O, part_o, part_lse, status, bm, ra);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -594,13 +740,44 @@ cudaError_t run_refine_tc(const MuseTables &mt, int D, int Dv, int N, int P, Sor
                           const int32_t *q_perm, SortedSide ks, const int32_t *k_offsets,
                           const void *vt, StageBufs b, void *O, float *part_o, float *part_lse,
                           int *status, cudaStream_t st) {
-  if (D == 64 && Dv == 64)
-    return tcr::launch<64, 64>(mt, N, P, qs, q_perm, ks, k_offsets, vt, b, O, part_o, part_lse, status, st);
-  if (D == 64 && Dv == 128)
-    return tcr::launch<64, 128>(mt, N, P, qs, q_perm, ks, k_offsets, vt, b, O, part_o, part_lse, status, st);
-  if (D == 128 && Dv == 64)
-    return tcr::launch<128, 64>(mt, N, P, qs, q_perm, ks, k_offsets, vt, b, O, part_o, part_lse, status, st);
-  return tcr::launch<128, 128>(mt, N, P, qs, q_perm, ks, k_offsets, vt, b, O, part_o, part_lse, status, st);
+  const tcr::RetArgs ra{};
+#define MUSE_REFINE_TC(DD, DDV)                                                              \
+  if (D == DD && Dv == DDV)                                                                  \
+    return tcr::launch<DD, DDV, false>(mt, N, P, qs, q_perm, ks, k_offsets, vt, b, O, part_o, \
+                                       part_lse, status, st, ra);
+  MUSE_REFINE_TC(64, 64)
+  MUSE_REFINE_TC(64, 128)
+  MUSE_REFINE_TC(128, 64)
+  MUSE_REFINE_TC(128, 128)
+#undef MUSE_REFINE_TC
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t run_refine_tc_ret(const MuseTables &mt, int D, int Dv, int N, int P, SortedSide qs,
+                              const int32_t *q_perm, SortedSide ks, const int32_t *k_offsets,
+                              const void *vt, StageBufs b, float *part_o, float *part_lse,
+                              const int32_t *k_perm, const int32_t *pend, const int32_t *sel,
+                              int S, int k1, int k2, int *status, cudaStream_t st) {
+  tcr::RetArgs ra;
+  ra.k_perm = k_perm;
+  ra.pend = pend;
+  ra.sel = sel;
+  ra.S = S;
+  ra.nb = N / S;
+  ra.k1 = k1;
+  ra.k2 = k2;
+  ra.K12 = k1 * k2 > 1 ? k1 * k2 : 1;
+  ra.Cq = mt.q.C[0];
+#define MUSE_REFINE_TC(DD, DDV)                                                                 \
+  if (D == DD && Dv == DDV)                                                                     \
+    return tcr::launch<DD, DDV, true>(mt, N, P, qs, q_perm, ks, k_offsets, vt, b, nullptr, part_o, \
+                                      part_lse, status, st, ra);
+  MUSE_REFINE_TC(64, 64)
+  MUSE_REFINE_TC(64, 128)
+  MUSE_REFINE_TC(128, 64)
+  MUSE_REFINE_TC(128, 128)
+#undef MUSE_REFINE_TC
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace muse

@@ -1,4 +1,4 @@
-// Causal MuSe with causal accumulation and top-k retrieval (CUDA cores).
+// Causal MuSe with causal accumulation and top-k retrieval.
 //
 // gist.science "Technische Samenvatting: Multipole Semantic Attention (MuSe)",
 // "Kernmechanismen" item 3 (the context is cut into spatial blocks; a block sees the
@@ -23,12 +23,19 @@
 //     (the monopole + dipole refinement of the acausal path, restricted to R_j);
 //   exact part: keys of the selected runs and the diagonal keys [bS, n];
 //   both parts are merged into one softmax through their logsumexps.
+//
+// bfloat16 inputs (D, Dv in {64, 128}) take the tensor-core path: u_j via running
+// prefixes over the key blocks (ret_T), the remainder output on tcgen05 (the
+// refinement kernel's retrieval mode), the selected runs exactly on the CUDA cores
+// (ret_runs) and the diagonal with the merge on tcgen05 (diag_tc) where it applies.
+// float32 inputs take the CUDA-core passes below (remainder_pass, exact_merge).
 #include <math.h>
 #include <string.h>
 
 #include <algorithm>
 
 #include "internal.h"
+#include "tc.h"
 
 namespace muse {
 namespace ret {
@@ -44,19 +51,20 @@ __device__ __forceinline__ float lse_add(float a, float b) {
   return m + logf(expf(a - m) + expf(b - m));
 }
 
-// cnt[p][j][b'] = keys of cluster j in block b' (integer atomics: exact).
-__global__ void block_counts(Geo g, const int32_t *__restrict__ k_labels, int32_t *__restrict__ cnt) {
+// cnt[p][j][b'] = rows of cluster j in block b' (integer atomics: exact); C clusters.
+__global__ void block_counts(Geo g, int C, const int32_t *__restrict__ labels, int32_t *__restrict__ cnt) {
   const int p = blockIdx.y;
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= g.N) return;
-  const int j = k_labels[(int64_t)p * g.N + k];
-  atomicAdd(&cnt[((int64_t)p * g.Ck + j) * g.nb + k / g.S], 1);
+  const int j = labels[(int64_t)p * g.N + k];
+  atomicAdd(&cnt[((int64_t)p * C + j) * g.nb + k / g.S], 1);
 }
 
-// pend[p][j][b'] = keys of cluster j in blocks < b' (b' = 0..nb).
-__global__ void block_prefix(Geo g, int P, const int32_t *__restrict__ cnt, int32_t *__restrict__ pend) {
+// pend[p][j][b'] = rows of cluster j in blocks < b' (b' = 0..nb).
+__global__ void block_prefix(Geo g, int P, int C, const int32_t *__restrict__ cnt,
+                             int32_t *__restrict__ pend) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= P * g.Ck) return;
+  if (t >= P * C) return;
   const int32_t *c = cnt + (int64_t)t * g.nb;
   int32_t *o = pend + (int64_t)t * (g.nb + 1);
   int run = 0;
@@ -435,6 +443,298 @@ exact_merge(Geo g, float scale, const T *__restrict__ Q, const T *__restrict__ K
   for (int t = 0; t < PV; ++t) st_elem(o + gq + 4 * t, acc[t] * inv);
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core path (bfloat16).  Query rows are in query-cluster order (sorted
+// residuals qt = q - qbar_i), keys in key-cluster order; inside a cluster both keep
+// token order, so the rows of (cluster i, block b) and the keys of (cluster j,
+// block b') are contiguous runs: [qoff_i + qpend_i(b), qoff_i + qpend_i(b+1)) and
+// [koff_j + pend_j(b'), koff_j + pend_j(b'+1)).
+// ---------------------------------------------------------------------------
+
+// T[p][j][r] = sum over the remainder keys k of cluster j of W_ik qt_r.k for sorted query
+// row r (cluster i, block b): the keys of j in blocks b' < b minus the runs selected for
+// (i, b).  A running sum m1_j = sum_{b' < b} sum_{k in (j, b')} W_ik k over the key blocks
+// gives qt_r.m1_j; the selected runs are subtracted key by key.  One CTA per (problem,
+// query cluster i, group of JPC key clusters); DP = D / 32 threads per cluster, 32
+// coordinates each.
+template <int D>
+__global__ void __launch_bounds__(256)
+ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q_offsets,
+      const int32_t *__restrict__ qpend, const __nv_bfloat16 *__restrict__ ks,
+      const int32_t *__restrict__ k_offsets, const int32_t *__restrict__ pend,
+      const float *__restrict__ W, int w_stride, const int32_t *__restrict__ sel,
+      float *__restrict__ Tout) {
+  constexpr int DP = D / 32, JPC = 256 / DP;
+  const int p = blockIdx.z, i = blockIdx.y;
+  const int jl = threadIdx.x / DP, dp = threadIdx.x % DP;
+  const int j = blockIdx.x * JPC + jl;
+  const bool live = j < g.Ck;
+  const int jj = live ? j : g.Ck - 1;
+  const int32_t *qo = q_offsets + (int64_t)p * (g.Cq + 1);
+  const int32_t *qpe = qpend + ((int64_t)p * g.Cq + i) * (g.nb + 1);
+  const int32_t *pe = pend + ((int64_t)p * g.Ck + jj) * (g.nb + 1);
+  const int kbase = k_offsets[(int64_t)p * (g.Ck + 1) + jj];
+  const float *wrow = W + (int64_t)p * w_stride + (int64_t)i * w_ld(g.N);
+  const __nv_bfloat16 *kp = ks + (int64_t)p * g.N * D + dp * 32;
+  const __nv_bfloat16 *qp = qs + (int64_t)p * g.N * D + dp * 32;
+  float *tout = Tout + ((int64_t)p * g.Ck + jj) * g.N;
+  const int r_first = qo[i];
+  float m1[32];
+#pragma unroll
+  for (int d = 0; d < 32; ++d) m1[d] = 0.f;
+  auto load32 = [](const __nv_bfloat16 *src, float (&x)[32]) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 u = reinterpret_cast<const uint4 *>(src)[v];
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
+        x[8 * v + 2 * h] = __low2float(b2);
+        x[8 * v + 2 * h + 1] = __high2float(b2);
+      }
+    }
+  };
+  for (int b = 0; b < g.nb; ++b) {
+    if (b > 0 && live) {
+      // the keys of (j, b - 1) join the prefix
+      for (int pos = kbase + pe[b - 1]; pos < kbase + pe[b]; ++pos) {
+        float x[32];
+        load32(kp + (int64_t)pos * D, x);
+        const float w = wrow[pos];
+#pragma unroll
+        for (int d = 0; d < 32; ++d) m1[d] = fmaf(w, x[d], m1[d]);
+      }
+    }
+    const int r0 = r_first + qpe[b], r1 = r_first + qpe[b + 1];
+    if (r0 >= r1) continue;  // CTA-uniform
+    // the slots of cluster j among those selected for (i, b): tj (or -1)
+    const int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
+    int tj = -1;
+    if (b > 0 && live)
+      for (int t = 0; t < g.k1; ++t)
+        if (so[2 * t * g.k2] == j) tj = t;
+    for (int r = r0; r < r1; ++r) {
+      float q[32];
+      load32(qp + (int64_t)r * D, q);
+      float acc = 0.f;
+      if (b > 0) {
+#pragma unroll
+        for (int d = 0; d < 32; ++d) acc = fmaf(q[d], m1[d], acc);
+        for (int u = 0; tj >= 0 && u < g.k2; ++u) {
+          const int bb = so[2 * (tj * g.k2 + u) + 1];
+          if (bb < 0) continue;
+          for (int pos = kbase + pe[bb]; pos < kbase + pe[bb + 1]; ++pos) {
+            float x[32];
+            load32(kp + (int64_t)pos * D, x);
+            float dot = 0.f;
+#pragma unroll
+            for (int d = 0; d < 32; ++d) dot = fmaf(q[d], x[d], dot);
+            acc = fmaf(-wrow[pos], dot, acc);
+          }
+        }
+      }
+#pragma unroll
+      for (int o = DP / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (live && dp == 0) tout[r] = acc;
+    }
+  }
+}
+
+// Remainder coefficients per sorted query row r (cluster i, block b):
+//   U_j = exp(logZ_ij - logZR) T_jr;  a_j = logZR + s U_j;  p = softmax(a);
+//   c0_jr = p_j (1 - s U_j) exp(logZ_ij - logZR),  c1_jr = s p_j exp(logZ_ij - logZR);
+// lse_r[p][r] = logsumexp_j a_j (-inf when nothing remains).
+__global__ void __launch_bounds__(128)
+ret_coeffs(Geo g, float scale, const int32_t *__restrict__ q_perm,
+           const int32_t *__restrict__ q_cluster, const float *__restrict__ logZ,
+           const float *__restrict__ logZR, const float *__restrict__ Tbuf,
+           float *__restrict__ c0, float *__restrict__ c1, float *__restrict__ lse_r) {
+  const int p = blockIdx.y;
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= g.N) return;
+  const int b = q_perm[(int64_t)p * g.N + r] / g.S;
+  const int i = q_cluster[(int64_t)p * g.N + r];
+  const float *lz = logZ + ((int64_t)p * g.Cq + i) * g.Ck;
+  const float *zr = logZR + (((int64_t)p * g.Cq + i) * g.nb + b) * g.Ck;
+  float m = -CUDART_INF_F, l = 0.f;
+  for (int pass = 0; pass < 2; ++pass) {
+    const float inv = pass ? 1.f / l : 0.f;
+    for (int j = 0; j < g.Ck; ++j) {
+      const int64_t at = ((int64_t)p * g.Ck + j) * g.N + r;
+      const float z = zr[j];
+      if (b == 0 || !(z > -CUDART_INF_F)) {
+        if (pass) {
+          c0[at] = 0.f;
+          c1[at] = 0.f;
+        }
+        continue;
+      }
+      const float f = expf(lz[j] - z);
+      const float U = f * Tbuf[at];
+      const float a = z + scale * U;
+      if (!pass) {
+        if (a > m) {
+          l = l * expf(m - a) + 1.f;
+          m = a;
+        } else {
+          l += expf(a - m);
+        }
+      } else {
+        const float pj = expf(a - m) * inv;
+        c0[at] = pj * (1.f - scale * U) * f;
+        c1[at] = scale * pj * f;
+      }
+    }
+  }
+  lse_r[(int64_t)p * g.N + r] = (l > 0.f) ? m + logf(l) : -CUDART_INF_F;
+}
+
+// Exact attention over the (cluster, block) runs selected for (query cluster i, query
+// block b), merged into the remainder partial of every row of the group (token order):
+// part_lse[p][n], part_o[p][n][:] become the joint (log-normaliser, normalised output) of
+// the remainder and the runs.  One CTA of four warps per (problem, i, b); the runs' keys
+// and values go through shared memory KC at a time; a warp takes one query row at a time
+// (lanes over keys for the logits, over output columns for the sums).
+template <int D, int DV>
+__global__ void __launch_bounds__(128)
+ret_runs(Geo g, float scale, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
+         const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ q_perm,
+         const int32_t *__restrict__ q_offsets, const int32_t *__restrict__ qpend,
+         const int32_t *__restrict__ k_perm, const int32_t *__restrict__ k_offsets,
+         const int32_t *__restrict__ pend, const int32_t *__restrict__ sel,
+         float *__restrict__ part_o, float *__restrict__ part_lse) {
+  constexpr int KC = (D + DV <= 128) ? 64 : 32;  // keys per chunk
+  constexpr int NK = KC / 32, PV = DV / 32;
+  __shared__ float Ks[KC][D + 1];
+  __shared__ float Vs[KC][DV];
+  __shared__ float qsh[4][D];
+  __shared__ float psh[4][KC];
+  __shared__ int runs[64], cum[65];  // run start (sorted key position), keys before it
+  __shared__ int nruns;
+  const int p = blockIdx.z, i = blockIdx.y, b = blockIdx.x;
+  if (b == 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t *qo = q_offsets + (int64_t)p * (g.Cq + 1);
+  const int32_t *qpe = qpend + ((int64_t)p * g.Cq + i) * (g.nb + 1);
+  const int r0 = qo[i] + qpe[b], r1 = qo[i] + qpe[b + 1];
+  if (r0 >= r1) return;  // uniform
+  if (threadIdx.x == 0) {
+    const int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
+    int n = 0;
+    cum[0] = 0;
+    for (int t = 0; t < g.K12; ++t) {
+      const int j = so[2 * t], bb = so[2 * t + 1];
+      if (j < 0) continue;
+      const int base = k_offsets[(int64_t)p * (g.Ck + 1) + j];
+      const int32_t *pe = pend + ((int64_t)p * g.Ck + j) * (g.nb + 1);
+      if (pe[bb + 1] > pe[bb]) {
+        runs[n] = base + pe[bb];
+        cum[n + 1] = cum[n] + pe[bb + 1] - pe[bb];
+        ++n;
+      }
+    }
+    nruns = n;
+  }
+  __syncthreads();
+  const int total = cum[nruns];
+  if (total == 0) return;  // uniform
+  const int32_t *kperm = k_perm + (int64_t)p * g.N;
+  for (int rb = r0; rb < r1; rb += 4) {
+    const int r = rb + warp;
+    const bool rv = r < r1;
+    const int n = rv ? q_perm[(int64_t)p * g.N + r] : 0;
+    if (rv)
+      for (int d = lane; d < D; d += 32)
+        qsh[warp][d] = __bfloat162float(Q[((int64_t)p * g.N + n) * D + d]) * scale;
+    float m = -CUDART_INF_F, l = 0.f, o[PV];
+#pragma unroll
+    for (int v = 0; v < PV; ++v) o[v] = 0.f;
+    for (int c0 = 0; c0 < total; c0 += KC) {
+      const int cnt = min(KC, total - c0);
+      __syncthreads();
+      if (threadIdx.x < cnt) {
+        const int gi = c0 + threadIdx.x;
+        int rr = 0;
+        while (cum[rr + 1] <= gi) ++rr;
+        const int tok = kperm[runs[rr] + gi - cum[rr]];
+        const uint4 *kr = reinterpret_cast<const uint4 *>(K + ((int64_t)p * g.N + tok) * D);
+        const uint4 *vr = reinterpret_cast<const uint4 *>(V + ((int64_t)p * g.N + tok) * DV);
+        for (int u = 0; u < D / 8; ++u) {
+          const uint4 x = kr[u];
+          const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+          for (int h = 0; h < 4; ++h) {
+            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
+            Ks[threadIdx.x][8 * u + 2 * h] = __low2float(b2);
+            Ks[threadIdx.x][8 * u + 2 * h + 1] = __high2float(b2);
+          }
+        }
+        for (int u = 0; u < DV / 8; ++u) {
+          const uint4 x = vr[u];
+          const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+          for (int h = 0; h < 4; ++h) {
+            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
+            Vs[threadIdx.x][8 * u + 2 * h] = __low2float(b2);
+            Vs[threadIdx.x][8 * u + 2 * h + 1] = __high2float(b2);
+          }
+        }
+      }
+      __syncthreads();
+      if (rv) {
+        float x[NK];
+        float cm = -CUDART_INF_F;
+#pragma unroll
+        for (int h = 0; h < NK; ++h) {
+          const int kk = lane + 32 * h;
+          x[h] = -CUDART_INF_F;
+          if (kk < cnt) {
+            float a = 0.f;
+            for (int d = 0; d < D; ++d) a = fmaf(qsh[warp][d], Ks[kk][d], a);
+            x[h] = a;
+          }
+          cm = fmaxf(cm, x[h]);
+        }
+        const float mn = fmaxf(m, warp_max(cm));
+        const float corr = expf(m - mn);
+        float ps = 0.f;
+#pragma unroll
+        for (int h = 0; h < NK; ++h) {
+          const float pe = lane + 32 * h < cnt ? expf(x[h] - mn) : 0.f;
+          psh[warp][lane + 32 * h] = pe;
+          ps += pe;
+        }
+        l = l * corr + warp_sum(ps);
+        __syncwarp();
+#pragma unroll
+        for (int v = 0; v < PV; ++v) {
+          float acc = o[v] * corr;
+          for (int k = 0; k < cnt; ++k) acc = fmaf(psh[warp][k], Vs[k][lane + 32 * v], acc);
+          o[v] = acc;
+        }
+        m = mn;
+        __syncwarp();
+      }
+    }
+    if (rv) {
+      // joint softmax with the remainder partial of the row
+      const int64_t at = (int64_t)p * g.N + n;
+      const float L = part_lse[at];
+      float *po = part_o + at * DV;
+      const bool has = L > -CUDART_INF_F;
+      const float mn = has ? fmaxf(m, L) : m;
+      const float ca = expf(m - mn), cb = has ? expf(L - mn) : 0.f;
+      const float lt = l * ca + cb;
+#pragma unroll
+      for (int v = 0; v < PV; ++v) {
+        const float prev = has ? po[lane + 32 * v] : 0.f;
+        po[lane + 32 * v] = (o[v] * ca + cb * prev) / lt;
+      }
+      __syncwarp();
+      if (lane == 0) part_lse[at] = mn + logf(lt);
+    }
+  }
+}
+
 // Workspace layout.
 struct Ws {
   KmeansOut q, k;
@@ -445,6 +745,9 @@ struct Ws {
   float *W, *logZ;
   int32_t *cnt, *pend, *sel;
   float *logZb, *logZR, *T, *c0, *c1, *lse_r, *part_o;
+  SortedSide qs;              // tensor-core path: sorted residuals
+  int32_t *qcnt, *qpend;      // rows of query cluster i in / before each block
+  float *part_lse;            // remainder + runs log-normaliser per token
 };
 
 struct Bump2 {
@@ -515,6 +818,11 @@ static void plan(Bump2 &bp, const muse_dims &d, const Geo &g, Ws &w) {
   w.c1 = bp.take<float>((size_t)P * g.Ck * d.N);
   w.lse_r = bp.take<float>((size_t)P * d.N);
   w.part_o = bp.take<float>((size_t)P * d.N * d.Dv);
+  w.qs.rows = bp.take<char>((size_t)P * d.N * d.D * es);
+  w.qs.cluster = bp.take<int32_t>((size_t)P * d.N);
+  w.qcnt = bp.take<int32_t>((size_t)P * g.Cq * g.nb);
+  w.qpend = bp.take<int32_t>((size_t)P * g.Cq * (g.nb + 1));
+  w.part_lse = bp.take<float>((size_t)P * d.N);
 }
 
 static bool valid_geo(const muse_dims &d, int block, int Cq, int Ck, int k1, int k2, Geo &g) {
@@ -533,6 +841,67 @@ static bool valid_geo(const muse_dims &d, int block, int Cq, int Ck, int k1, int
   g.k2 = k2;
   g.K12 = std::max(1, k1 * k2);
   return true;
+}
+
+// The tensor-core path (bfloat16): see the header of this file.
+template <int D, int DV>
+static cudaError_t run_tc(const void *Q, const void *K, const void *V, const muse_dims &d,
+                          const Geo &g, int iters, Ws &w, void *O, int *status, cudaStream_t st) {
+  const int P = d.B * d.H;
+  MuseTables mt = tables(d.N, g.Cq, g.Ck);
+  cudaError_t e;
+  if ((e = run_kmeans_pair(Q, mt.q, w.q, K, mt.k, w.k, d.dtype, D, d.N, P, iters, w.km_scratch,
+                           status, st)) != cudaSuccess)
+    return e;
+  if ((e = run_sort_side(Q, d.dtype, D, d.N, mt.q, P, w.q.perm, w.q.offsets, w.q.centroids, w.qs,
+                         st)) != cudaSuccess)
+    return e;
+  if ((e = run_sort_side(K, d.dtype, D, d.N, mt.k, P, w.k.perm, w.k.offsets, nullptr, w.ks, st)) !=
+      cudaSuccess)
+    return e;
+  if ((e = run_sort_side_t(V, d.dtype, DV, d.N, mt.k, P, w.k.perm, w.vs, st)) != cudaSuccess) return e;
+  StageBufs sb;
+  memset(&sb, 0, sizeof(sb));
+  sb.W = w.W;
+  sb.logZ = w.logZ;
+  if ((e = run_summaries(mt, d.dtype, D, DV, P, d.scale, w.q.centroids, w.ks, nullptr, w.k.offsets,
+                         sb, st)) != cudaSuccess)
+    return e;
+  if ((e = cudaMemsetAsync(w.cnt, 0, (size_t)P * g.Ck * g.nb * sizeof(int32_t), st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(w.qcnt, 0, (size_t)P * g.Cq * g.nb * sizeof(int32_t), st)) != cudaSuccess)
+    return e;
+  block_counts<<<dim3((d.N + 255) / 256, P), 256, 0, st>>>(g, g.Ck, w.k.labels, w.cnt);
+  block_prefix<<<(P * g.Ck + 127) / 128, 128, 0, st>>>(g, P, g.Ck, w.cnt, w.pend);
+  block_counts<<<dim3((d.N + 255) / 256, P), 256, 0, st>>>(g, g.Cq, w.q.labels, w.qcnt);
+  block_prefix<<<(P * g.Cq + 127) / 128, 128, 0, st>>>(g, P, g.Cq, w.qcnt, w.qpend);
+  const int64_t nw = (int64_t)P * g.Cq * g.Ck;
+  block_lse<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(g, P, w.W, mt.in.w_stride, w.logZ,
+                                                      w.k.offsets, w.pend, w.logZb);
+  const int64_t ns = (int64_t)P * g.Cq * g.nb;
+  select_blocks<<<(unsigned)((ns + 7) / 8), 256, 0, st>>>(g, P, w.logZb, w.sel, w.logZR);
+  constexpr int JPC = 256 / (D / 32);
+  ret_T<D><<<dim3((g.Ck + JPC - 1) / JPC, g.Cq, P), 256, 0, st>>>(
+      g, (const __nv_bfloat16 *)w.qs.rows, w.q.offsets, w.qpend, (const __nv_bfloat16 *)w.ks.rows,
+      w.k.offsets, w.pend, w.W, mt.in.w_stride, w.sel, w.T);
+  ret_coeffs<<<dim3((d.N + 127) / 128, P), 128, 0, st>>>(g, d.scale, w.q.perm, w.qs.cluster, w.logZ,
+                                                        w.logZR, w.T, w.c0, w.c1, w.lse_r);
+  count_launches(10);
+  sb.c0 = w.c0;
+  sb.c1 = w.c1;
+  sb.lse = w.lse_r;
+  if ((e = profile_mark(true, st)) != cudaSuccess) return e;
+  if ((e = run_refine_tc_ret(mt, D, DV, d.N, P, w.qs, w.q.perm, w.ks, w.k.offsets, w.vs, sb,
+                             w.part_o, w.part_lse, w.k.perm, w.pend, w.sel, g.S, g.k1, g.k2,
+                             status, st)) != cudaSuccess)
+    return e;
+  if ((e = profile_mark(false, st)) != cudaSuccess) return e;
+  ret_runs<D, DV><<<dim3(g.nb, g.Cq, P), 128, 0, st>>>(
+      g, d.scale, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V,
+      w.q.perm, w.q.offsets, w.qpend, w.k.perm, w.k.offsets, w.pend, w.sel, w.part_o, w.part_lse);
+  count_launches(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return run_diag_merge(Q, K, V, d.dtype, D, DV, d.N, P, g.S, -1, d.scale, w.part_o, w.part_lse, O,
+                        st);
 }
 
 template <typename T, int D, int DV>
@@ -560,8 +929,8 @@ static cudaError_t run_t(const void *Q, const void *K, const void *V, const muse
     return e;
   if ((e = cudaMemsetAsync(w.cnt, 0, (size_t)P * g.Ck * g.nb * sizeof(int32_t), st)) != cudaSuccess)
     return e;
-  block_counts<<<dim3((d.N + 255) / 256, P), 256, 0, st>>>(g, w.k.labels, w.cnt);
-  block_prefix<<<(P * g.Ck + 127) / 128, 128, 0, st>>>(g, P, w.cnt, w.pend);
+  block_counts<<<dim3((d.N + 255) / 256, P), 256, 0, st>>>(g, g.Ck, w.k.labels, w.cnt);
+  block_prefix<<<(P * g.Ck + 127) / 128, 128, 0, st>>>(g, P, g.Ck, w.cnt, w.pend);
   const int64_t nw = (int64_t)P * g.Cq * g.Ck;
   block_lse<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(g, P, w.W, mt.in.w_stride, w.logZ,
                                                       w.k.offsets, w.pend, w.logZb);
@@ -636,10 +1005,10 @@ extern "C" muse_status muse_retrieve_exact(const void *Q, const void *K, const v
     else if (d.Dv == 64) e = ret::run_t<float, 128, 64>(Q, K, V, d, g, iters, w, O, status, cs);
     else e = ret::run_t<float, 128, 128>(Q, K, V, d, g, iters, w, O, status, cs);
   } else {
-    if (d.D == 64 && d.Dv == 64) e = ret::run_t<__nv_bfloat16, 64, 64>(Q, K, V, d, g, iters, w, O, status, cs);
-    else if (d.D == 64) e = ret::run_t<__nv_bfloat16, 64, 128>(Q, K, V, d, g, iters, w, O, status, cs);
-    else if (d.Dv == 64) e = ret::run_t<__nv_bfloat16, 128, 64>(Q, K, V, d, g, iters, w, O, status, cs);
-    else e = ret::run_t<__nv_bfloat16, 128, 128>(Q, K, V, d, g, iters, w, O, status, cs);
+    if (d.D == 64 && d.Dv == 64) e = ret::run_tc<64, 64>(Q, K, V, d, g, iters, w, O, status, cs);
+    else if (d.D == 64) e = ret::run_tc<64, 128>(Q, K, V, d, g, iters, w, O, status, cs);
+    else if (d.Dv == 64) e = ret::run_tc<128, 64>(Q, K, V, d, g, iters, w, O, status, cs);
+    else e = ret::run_tc<128, 128>(Q, K, V, d, g, iters, w, O, status, cs);
   }
   return e == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
 }

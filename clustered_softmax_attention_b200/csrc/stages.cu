@@ -1280,9 +1280,11 @@ diag_merge(const T *__restrict__ Qg, const T *__restrict__ Kg, const T *__restri
       }
     }
   }
-  for (int lev = 1; lev <= levels; ++lev) {
-    if (!((bidx >> (lev - 1)) & 1)) continue;
-    const int64_t r = ((int64_t)p * levels + (lev - 1)) * N + n;
+  // levels < 0: a single partial array, merged into every row
+  const int nlev = levels < 0 ? 1 : levels;
+  for (int lev = 1; lev <= nlev; ++lev) {
+    if (levels > 0 && !((bidx >> (lev - 1)) & 1)) continue;
+    const int64_t r = ((int64_t)p * nlev + (lev - 1)) * N + n;
     const float L = part_lse[r];
     if (!(L > -CUDART_INF_F)) continue;
     const float mn = fmaxf(m, L);

@@ -43,8 +43,8 @@ _SIGS = {
     "muse_kmeans_noalloc": [_vp, MuseDims, _i, _i, _vp, _vp, _vp, _vp, _vp],
     "muse_tilted_summaries": [_vp, _vp, _vp, _vp, _vp, MuseDims, _i, _i, _vp, _vp, _vp, _vp,
                               _vp, _sz, _vp],
-    "muse_dipole_refine": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, MuseDims, _i, _i,
-                           _vp, _vp, _sz, _vp],
+    "muse_dipole_refine": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                           MuseDims, _i, _i, _vp, _vp, _sz, _vp],
     "muse_forward": [_vp, _vp, _vp, MuseDims, _i, _i, _i, _vp, _vp, _sz, _vp],
     "muse_forward_ex": [_vp, _vp, _vp, MuseDims, _i, _i, _i, ctypes.c_uint, _vp, _vp, _sz, _vp],
     "muse_causal_levels": [_i, _i],
@@ -56,6 +56,8 @@ _SIGS = {
     "muse_status_string": [_i],
     "muse_last_device_status": [_vp],
     "muse_set_test_hooks": [ctypes.c_uint, ctypes.c_uint64],
+    "muse_backward": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, MuseDims, _i, _i, _vp, _vp, _vp,
+                      _vp, _sz, _vp],
 }
 _RES = {"muse_workspace_size": _sz, "muse_status_string": ctypes.c_char_p,
         "muse_causal_levels": _i}
@@ -228,11 +230,13 @@ def muse_tilted_summaries(q_centroids, K, V, k_perm, k_offsets, Ck: int, scale: 
 
 
 def muse_dipole_refine(Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offsets, logZ, mu_k,
-                       scale: float = 1.0):
-    """Stage 2 refinement: O [B,H,N,Dv] in Q's dtype."""
+                       scale: float = 1.0, mu_v=None, cov=None, q_labels=None):
+    """Stage 2 refinement: O [B,H,N,Dv] in Q's dtype.  With mu_v and cov (materialised
+    summaries) the library evaluates the refinement from them as given."""
     _qkv(Q, K, V)
     B, H, N, D = Q.shape
     Cq, Ck = q_centroids.shape[2], logZ.shape[3]
+    Dv = V.shape[3]
     _expect(q_centroids, (B, H, Cq, D), torch.float32, "q_centroids")
     _expect(q_perm, (B, H, N), torch.int32, "q_perm")
     _expect(q_offsets, (B, H, Cq + 1), torch.int32, "q_offsets")
@@ -240,15 +244,18 @@ def muse_dipole_refine(Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offset
     _expect(k_offsets, (B, H, Ck + 1), torch.int32, "k_offsets")
     _expect(logZ, (B, H, Cq, Ck), torch.float32, "logZ")
     _expect(mu_k, (B, H, Cq, Ck, D), torch.float32, "mu_k")
-    _contig(Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offsets, logZ, mu_k)
+    _expect(mu_v, (B, H, Cq, Ck, Dv), torch.float32, "mu_v")
+    _expect(cov, (B, H, Cq, Ck, Dv, D), torch.float32, "cov")
+    _expect(q_labels, (B, H, N), torch.int32, "q_labels")
+    _contig(Q, K, V, q_centroids, q_perm, q_offsets, k_perm, k_offsets, logZ, mu_k, mu_v, cov,
+            q_labels)
     d = dims(Q, V, scale)
-    Cq, Ck = q_centroids.shape[2], logZ.shape[3]
     O = torch.empty(Q.shape[0], Q.shape[1], Q.shape[2], d.Dv, dtype=Q.dtype, device=Q.device)
     ws = workspace("muse_dipole_refine", d, Cq, Ck)
     _check(lib().muse_dipole_refine(
-        _p(Q), _p(K), _p(V), _p(q_centroids), _p(q_perm), _p(q_offsets), _p(k_perm),
-        _p(k_offsets), _p(logZ), _p(mu_k), d, Cq, Ck, _p(O), _p(ws), ws.numel(), _stream()),
-        "muse_dipole_refine")
+        _p(Q), _p(K), _p(V), _p(q_labels), _p(q_centroids), _p(q_perm), _p(q_offsets),
+        _p(k_perm), _p(k_offsets), _p(logZ), _p(mu_k), _p(mu_v), _p(cov), d, Cq, Ck, _p(O),
+        _p(ws), ws.numel(), _stream()), "muse_dipole_refine")
     return O
 
 
@@ -336,3 +343,23 @@ def muse_retrieve_exact(Q, K, V, block: int, Cq: int, Ck: int, iters: int, k1: i
     if return_all:
         return out, ql, kl, sel
     return out
+
+
+def muse_backward(Q, K, V, dO, q_perm, q_offsets, k_perm, k_offsets, scale: float = 1.0,
+                  ws: Optional[torch.Tensor] = None):
+    """Gradients (dQ, dK, dV) of sum(O * dO) for the acausal forward pass, clusterings fixed."""
+    _qkv(Q, K, V, dO)
+    B, H, N, D = Q.shape
+    Cq, Ck = q_offsets.shape[2] - 1, k_offsets.shape[2] - 1
+    for t, shape, name in ((q_perm, (B, H, N), "q_perm"), (q_offsets, (B, H, Cq + 1), "q_offsets"),
+                           (k_perm, (B, H, N), "k_perm"), (k_offsets, (B, H, Ck + 1), "k_offsets")):
+        _expect(t, shape, torch.int32, name)
+    _contig(Q, K, V, dO, q_perm, q_offsets, k_perm, k_offsets, ws)
+    d = dims(Q, V, scale)
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    if ws is None:
+        ws = workspace("muse_backward", d, Cq, Ck)
+    _check(lib().muse_backward(_p(Q), _p(K), _p(V), _p(dO), _p(q_perm), _p(q_offsets), _p(k_perm),
+                               _p(k_offsets), d, Cq, Ck, _p(dQ), _p(dK), _p(dV), _p(ws), ws.numel(),
+                               _stream()), "muse_backward")
+    return dQ, dK, dV

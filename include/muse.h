@@ -143,23 +143,34 @@ muse_status muse_tilted_summaries(const float *q_centroids, const void *K, const
  * muse_dipole_refine - stage 2: for query n in cluster i with qt = q_n - qbar_i,
  *     a_j = log Z_ij + s qt.mu_k,ij;   p = softmax_j(a);
  *     O_n = sum_j p_j (mu_v,ij + s C_ij qt)
- *   computed without materialising C_ij: with u_j = qt.mu_k,ij,
- *     O_n = sum_j sum_{k in S_j} w_ik p_j (1 - s u_j + s qt.k) v_k,
- *   an identity of the definition above (sum_k w_ik (k - mu_k,ij) = 0).
  *   Source: pith.science review, "What carries the argument" (drop only qt.kt);
  *   gist.science "Kernmechanismen" 1-2.
- * Inputs:  Q, K, V; q_centroids/q_perm/q_offsets from muse_kmeans on Q (Cq
- *          clusters); k_perm/k_offsets from muse_kmeans on K (Ck clusters);
- *          logZ and mu_k from muse_tilted_summaries (any values of the right
- *          shape are accepted, so the refinement can be fed reference summaries).
+ *   Two ways to evaluate it:
+ *   - mu_v = cov = NULL (the forward pass): C_ij is never materialised; with
+ *     u_j = qt.mu_k,ij the output is computed as
+ *       O_n = sum_j sum_{k in S_j} w_ik p_j (1 - s u_j + s qt.k) v_k,
+ *     an identity of the definition (sum_k w_ik (k - mu_k,ij) = 0), on the tensor
+ *     cores for bfloat16 inputs; the tilt weights w_ik are recomputed from logZ.
+ *   - mu_v and cov given: the formula above is evaluated as written from the
+ *     caller's materialised summaries (float32, CUDA cores; teacher forcing of the
+ *     dipole, or summaries from elsewhere).
+ * Inputs:  Q, K, V; q_labels int32 [B,H,N] (optional, may be NULL; when given, a row
+ *          whose label disagrees with q_perm/q_offsets sets MUSE_ERR_DEVICE in the
+ *          device status word); q_centroids/q_perm/q_offsets from muse_kmeans on Q
+ *          (Cq clusters); k_perm/k_offsets from muse_kmeans on K (Ck clusters); logZ
+ *          and mu_k from muse_tilted_summaries; mu_v f32 [B,H,Cq,Ck,Dv] and cov f32
+ *          [B,H,Cq,Ck,Dv,D] both NULL or both given (else MUSE_ERR_INVALID_ARG).  Any
+ *          values of the right shape are accepted, so the refinement can be fed
+ *          reference summaries.
  * Output:  O [B,H,N,Dv] in d.dtype.
  */
 muse_status muse_dipole_refine(const void *Q, const void *K, const void *V,
-                               const float *q_centroids,
+                               const int32_t *q_labels, const float *q_centroids,
                                const int32_t *q_perm, const int32_t *q_offsets,
                                const int32_t *k_perm, const int32_t *k_offsets,
-                               const float *logZ, const float *mu_k, muse_dims d, int Cq,
-                               int Ck, void *O, void *ws, size_t ws_bytes, muse_stream_t st);
+                               const float *logZ, const float *mu_k, const float *mu_v,
+                               const float *cov, muse_dims d, int Cq, int Ck, void *O,
+                               void *ws, size_t ws_bytes, muse_stream_t st);
 
 /*
  * muse_forward - the whole acausal forward pass: muse_kmeans on Q (Cq) and on K
@@ -244,9 +255,30 @@ muse_status muse_retrieve_exact(const void *Q, const void *K, const void *V, mus
                                 muse_stream_t st);
 
 /*
+ * muse_backward - gradients of the acausal forward pass: dQ, dK, dV of sum(O * dO) for
+ *   O = muse_forward's output, with the clusterings held fixed (K-means assignments are
+ *   discrete) and each query centroid the mean of its members, so gradients reach Q
+ *   through both the centroid and the residual.
+ *   Source: pith.science review of arXiv 2509.10406, referee report (the approximation
+ *   is used for pretraining, i.e. differentiated; the pages never measure it) and
+ *   "What carries the argument" (the quantities differentiated).
+ * Inputs:  Q, K, V, dO [B,H,N,*] (d.dtype); q_perm/q_offsets (Cq clusters) and
+ *          k_perm/k_offsets (Ck clusters): the clusterings of the forward pass, from
+ *          muse_kmeans.
+ * Outputs: dQ, dK [B,H,N,D], dV [B,H,N,Dv] in d.dtype.
+ * Float32 arithmetic on the CUDA cores, deterministic.  The forward summaries are
+ * recomputed; the workspace (muse_workspace_size("muse_backward", ...)) holds the
+ * materialised C_ij and its gradient, 8 B*H*Cq*Ck*Dv*D bytes among the rest.
+ */
+muse_status muse_backward(const void *Q, const void *K, const void *V, const void *dO,
+                          const int32_t *q_perm, const int32_t *q_offsets, const int32_t *k_perm,
+                          const int32_t *k_offsets, muse_dims d, int Cq, int Ck, void *dQ,
+                          void *dK, void *dV, void *ws, size_t ws_bytes, muse_stream_t st);
+
+/*
  * muse_workspace_size - bytes of workspace `entry` needs ("muse_kmeans" with C = Cq,
  * "muse_tilted_summaries", "muse_dipole_refine", "muse_forward", "muse_forward_ex",
- * "muse_causal_blocks", "muse_retrieve_exact").  Arguments an entry does not
+ * "muse_causal_blocks", "muse_retrieve_exact", "muse_backward").  Arguments an entry does not
  * use are ignored.  Returns 0 for an unknown entry or invalid sizes.
  */
 size_t muse_workspace_size(const char *entry, muse_dims d, int Cq, int Ck, int block, int k1,

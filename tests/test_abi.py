@@ -84,8 +84,15 @@ def test_argument_validation_enqueues_nothing(lib):
     assert lib.muse_kmeans(f, _d(), 8, 1001, f, f, f, f, f, 1 << 30, st) == 1
     assert lib.muse_tilted_summaries(f, f, None, f, f, _d(), 8, 8, f, None, f, None, f, 1 << 30,
                                      st) == 1
-    assert lib.muse_dipole_refine(f, f, f, f, f, f, f, f, f, None, _d(), 8, 8, f, f, 1 << 30,
-                                  st) == 1
+    assert lib.muse_dipole_refine(f, f, f, None, f, f, f, f, f, f, None, None, None, _d(), 8, 8,
+                                  f, f, 1 << 30, st) == 1
+    # mu_v and cov: both materialised or neither
+    assert lib.muse_dipole_refine(f, f, f, None, f, f, f, f, f, f, f, f, None, _d(), 8, 8,
+                                  f, f, 1 << 30, st) == 1
+    assert lib.muse_dipole_refine(f, f, f, None, f, f, f, f, f, f, f, None, f, _d(), 8, 8,
+                                  f, f, 1 << 30, st) == 1
+    assert lib.muse_dipole_refine(f, f, f, MISALIGNED, f, f, f, f, f, f, f, f, f, _d(), 8, 8,
+                                  f, f, 1 << 30, st) == 1
     assert lib.muse_causal_blocks(f, f, f, _d(), 100, 8, 8, 2, f, None, None, f, 1 << 30, st) == 2
     assert lib.muse_causal_blocks(f, f, f, _d(N=1000), 128, 8, 8, 2, f, None, None, f, 1 << 30,
                                   st) == 2
@@ -135,3 +142,18 @@ def test_test_hooks_refuse_unknown_bits(lib):
     """Unknown hook bits are refused before the device is touched."""
     assert lib.muse_set_test_hooks(2, 0) == 1
     assert lib.muse_set_test_hooks(0xFFFF, 5) == 1
+
+
+def test_backward_validation_and_workspace(lib):
+    st = ctypes.c_void_p(0)
+    f = FAKE
+    d = _d()
+    need = lib.muse_workspace_size(b"muse_backward", d, 16, 16, 0, 0, 0)
+    # the materialised C_ij and its gradient: 2 B*H*Cq*Ck*Dv*D floats at least
+    assert need >= 2 * 2 * 16 * 16 * 64 * 64 * 4
+    assert lib.muse_workspace_size(b"muse_backward", d, 16, 0, 0, 0, 0) == 0
+    assert lib.muse_backward(f, f, f, f, f, f, f, f, _d(dtype=5), 16, 16, f, f, f, f, need, st) == 3
+    assert lib.muse_backward(f, f, f, None, f, f, f, f, d, 16, 16, f, f, f, f, need, st) == 1
+    assert lib.muse_backward(f, f, f, f, f, f, f, f, d, 16, 16, f, f, MISALIGNED, f, need, st) == 1
+    assert lib.muse_backward(f, f, f, f, f, f, f, f, d, 0, 16, f, f, f, f, need, st) == 1
+    assert lib.muse_backward(f, f, f, f, f, f, f, f, d, 16, 16, f, f, f, f, need - 1, st) == 4

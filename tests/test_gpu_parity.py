@@ -97,7 +97,8 @@ def run_gpu_pipeline(Q, K, V, Cq, Ck, T, s, dt, with_cov=False):
     kl, kc, kp, ko = m.muse_kmeans(Kd, Ck, T)
     summ = m.muse_tilted_summaries(qc, Kd, Vd, kp, ko, Ck, s, want_cov=with_cov)
     O = m.muse_dipole_refine(Qd, Kd, Vd, qc, qp, qo, kp, ko, summ["logZ"], summ["mu_k"], s)
-    return dict(Qd=Qd, Kd=Kd, Vd=Vd, ql=ql, qc=qc, kl=kl, summ=summ, O=O)
+    return dict(Qd=Qd, Kd=Kd, Vd=Vd, ql=ql, qc=qc, qp=qp, qo=qo, kl=kl, kp=kp, ko=ko, summ=summ,
+                O=O)
 
 
 def normwise(O, ref):
@@ -128,6 +129,64 @@ def test_summaries_and_refine_vs_oracle(dt, parity):
             err = mo.max_rel_err(host(r["O"])[0, h], O_ref)
             parity(f"O s={s} h={h}", err, TOL[dt])
             assert err <= TOL[dt], err
+
+
+# the refinement from materialised summaries (muse_dipole_refine with mu_v and cov): fed the
+# oracle's own summaries (teacher forcing of the tilted dipole) it must reproduce the
+# oracle's refinement up to float32 rounding; fed the GPU's summaries it must agree with the
+# fused path (which never forms C_ij)
+@pytest.mark.parametrize("dt,D,Dv", [("f32", 64, 64), ("bf16", 64, 64), ("bf16", 128, 64),
+                                     ("f32", 64, 128)])
+def test_refine_from_materialised_summaries(dt, D, Dv, parity):
+    N, Cq, Ck, s = 768, 12, 20, 0.7
+    Q, K, V = mixture(14, 1, 2, N, D, Dv, 24, 0.4 / np.sqrt(D), dt)
+    r = run_gpu_pipeline(Q, K, V, Cq, Ck, 4, s, dt, with_cov=True)
+    Qf, Kf, Vf = host(r["Qd"]), host(r["Kd"]), host(r["Vd"])
+    ql, qc, qp, qo, kp, ko = (r[k] for k in ("ql", "qc", "qp", "qo", "kp", "ko"))
+    # the oracle's summaries from the GPU's clustering, as float32
+    oracle = {"logZ": [], "mu_k": [], "mu_v": [], "cov": []}
+    refs = []
+    for h in range(2):
+        qbar = qc[0, h].cpu().numpy().astype(np.float64)
+        lz, mk, mv, cv = mo.tilted_summaries(qbar, Kf[0, h], Vf[0, h], r["kl"][0, h].cpu().numpy(),
+                                             Ck, s)
+        for key, val in zip(("logZ", "mu_k", "mu_v", "cov"), (lz, mk, mv, cv)):
+            oracle[key].append(val)
+        refs.append(mo.refine(Qf[0, h], ql[0, h].cpu().numpy(), qbar, lz, mk, mv, cv, s))
+    t = {k: torch.tensor(np.stack(v)[None], dtype=torch.float32).cuda().contiguous()
+         for k, v in oracle.items()}
+    O_tf = host(m.muse_dipole_refine(r["Qd"], r["Kd"], r["Vd"], qc, qp, qo, kp, ko, t["logZ"],
+                                     t["mu_k"], s, mu_v=t["mu_v"], cov=t["cov"], q_labels=ql))
+    assert m.muse_last_device_status() == 0
+    # the materialised path computes in float32; only the output's own rounding remains
+    tol_tf = 1e-5 if dt == "f32" else 8e-3
+    for h in range(2):
+        err = mo.max_rel_err(O_tf[0, h], refs[h])
+        parity(f"teacher-forced dipole h={h}", err, tol_tf)
+        assert err <= tol_tf, err
+    g = r["summ"]
+    O_m = host(m.muse_dipole_refine(r["Qd"], r["Kd"], r["Vd"], qc, qp, qo, kp, ko, g["logZ"],
+                                    g["mu_k"], s, mu_v=g["mu_v"], cov=g["cov"]))
+    for h in range(2):
+        err = mo.max_rel_err(O_m[0, h], host(r["O"])[0, h])
+        parity(f"materialised vs fused h={h}", err, TOL[dt])
+        assert err <= TOL[dt], err
+
+
+def test_refine_reports_labels_that_disagree_with_the_permutation():
+    """A device-side consistency check that reports and returns (no fault): q_labels that do
+    not match q_perm / q_offsets give MUSE_ERR_DEVICE; a correct call afterwards is clean."""
+    N, C = 512, 8
+    Q, K, V = mixture(15, 1, 1, N, 64, 64, 16, 0.05, "f32")
+    r = run_gpu_pipeline(Q, K, V, C, C, 3, 1.0, "f32", with_cov=True)
+    qc, qp, qo, kp, ko = (r[k] for k in ("qc", "qp", "qo", "kp", "ko"))
+    g = r["summ"]
+    bad = ((r["ql"] + 1) % C).to(torch.int32).contiguous()
+    args = (r["Qd"], r["Kd"], r["Vd"], qc, qp, qo, kp, ko, g["logZ"], g["mu_k"], 1.0)
+    m.muse_dipole_refine(*args, mu_v=g["mu_v"], cov=g["cov"], q_labels=bad)
+    assert m.muse_last_device_status() == 7
+    m.muse_dipole_refine(*args, mu_v=g["mu_v"], cov=g["cov"], q_labels=r["ql"])
+    assert m.muse_last_device_status() == 0
 
 
 # logZ and mu_k alone take the one-launch tilt kernel: key clusters of 0, 1, 15-17, 64-65,
@@ -382,11 +441,12 @@ def test_full_size_acausal_n8k_sampled_rows(parity):
 
 # --------------------------------------------------------------------------- retrieval
 
-def retrieval_case(dt, N, S, C, k1, k2, seed=9, H=2, scale=1.0, outliers=0.0):
+def retrieval_case(dt, N, S, C, k1, k2, seed=9, H=2, scale=1.0, outliers=0.0, D=64, Dv=64):
     rng = np.random.Generator(np.random.PCG64(seed))
     from clustered_softmax_attention_b200.inputs import draw_problem, round_to_bf16
     cast = round_to_bf16 if dt == "bf16" else (lambda a: a.astype(np.float32))
-    Qs, Ks, Vs = zip(*[draw_problem(rng, N, 64, 64, 24, 0.3 / 8, outliers, 4.0) for _ in range(H)])
+    Qs, Ks, Vs = zip(*[draw_problem(rng, N, D, Dv, 24, 0.3 / np.sqrt(D), outliers, 4.0)
+                       for _ in range(H)])
     Q, K, V = (np.stack([cast(x) for x in L])[None] for L in (Qs, Ks, Vs))
     Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
     O, ql, kl, sel = m.muse_retrieve_exact(Qd, Kd, Vd, S, C, C, 4, k1, k2, scale, return_all=True)
@@ -397,21 +457,24 @@ def _close(a, b, tol=NEAR_TIE):
     return abs(a - b) <= tol * max(1.0, abs(a), abs(b))
 
 
-def check_selection(lzb, got, k1, k2):
-    """The GPU's retrieval selection against the oracle's from the same clustering.
+def check_selection(lzb, got, k1, k2, q_labels, S):
+    """The GPU's retrieval selection against the oracle's from the same clustering, on
+    every (query cluster, query block) group that holds a query (the others are never
+    read, and an empty query cluster keeps a centroid that is no member mean).
 
     Slots must be equal, except where the oracle's ranking has a near-tie: a slot whose
     cluster differs must hold a cluster whose prefix score is within 1e-5 (relative) of
     the oracle's pick, and a block that differs a block whose score is within 1e-5 of the
     oracle's.  Whatever differs must still be a valid selection (distinct clusters,
     distinct blocks before the query block, finite scores).  Returns the number of
-    (query cluster, query block) rows excused as near-ties."""
+    groups excused as near-ties."""
     want = mo.retrieval_select(lzb, k1, k2)
     Cq, nb = want.shape[:2]
+    used = set(zip(np.asarray(q_labels).tolist(), (np.arange(len(q_labels)) // S).tolist()))
     excused = 0
     for i in range(Cq):
         for b in range(nb):
-            if (want[i, b] == got[i, b]).all():
+            if (i, b) not in used or (want[i, b] == got[i, b]).all():
                 continue
             sig = [mo._lse(lzb[i, j, :b]) for j in range(lzb.shape[1])]
             gj = [int(got[i, b, t * k2, 0]) for t in range(k1)]
@@ -440,17 +503,22 @@ def check_selection(lzb, got, k1, k2):
     return excused
 
 
-@pytest.mark.parametrize("dt,k1,k2", [("f32", 2, 2), ("bf16", 2, 2), ("bf16", 4, 1),
-                                       ("bf16", 1, 4)])
-def test_retrieval_vs_oracle(dt, k1, k2, parity):
-    N, S, C = 1024, 128, 16
-    Q, K, V, O, ql, kl, sel = retrieval_case(dt, N, S, C, k1, k2, outliers=0.05)
+# bfloat16 takes the tensor-core path (remainder on tcgen05, diagonal on tcgen05 for
+# D = Dv = 64 and blocks of a multiple of 128), float32 the CUDA-core passes; N = 4096
+# with blocks of 256 gives clusters of several tiles whose causal prefixes end inside them
+@pytest.mark.parametrize("dt,N,S,C,k1,k2,D,Dv", [
+    ("f32", 1024, 128, 16, 2, 2, 64, 64), ("bf16", 1024, 128, 16, 2, 2, 64, 64),
+    ("bf16", 1024, 128, 16, 4, 1, 64, 64), ("bf16", 1024, 128, 16, 1, 4, 64, 64),
+    ("bf16", 1024, 128, 16, 2, 2, 64, 128), ("bf16", 1024, 128, 16, 2, 2, 128, 64),
+    ("bf16", 4096, 256, 32, 2, 3, 64, 64), ("bf16", 2048, 64, 24, 3, 2, 64, 64)])
+def test_retrieval_vs_oracle(dt, N, S, C, k1, k2, D, Dv, parity):
+    Q, K, V, O, ql, kl, sel = retrieval_case(dt, N, S, C, k1, k2, outliers=0.05, D=D, Dv=Dv)
     nrows = 0
     for h in range(2):
         # the selection equals the oracle's from the same clustering (near-ties counted)
         qbar = mo.cluster_means(Q[0, h], ql[0, h], C)
         lzb = mo.block_logZ(qbar, K[0, h], kl[0, h], C, S, 1.0)
-        ex = check_selection(lzb, sel[0, h], k1, k2)
+        ex = check_selection(lzb, sel[0, h], k1, k2, ql[0, h], S)
         parity(f"selection rows excused as near-ties h={h}", ex)
         nrows += C * (N // S)
         assert ex <= 2, ex
@@ -461,26 +529,26 @@ def test_retrieval_vs_oracle(dt, k1, k2, parity):
         assert err <= TOL[dt], err
 
 
-def test_retrieval_exact_limits_on_gpu(parity):
-    N, S = 256, 64
+@pytest.mark.parametrize("dt,S", [("f32", 64), ("bf16", 64), ("bf16", 128)])
+def test_retrieval_exact_limits_on_gpu(dt, S, parity):
+    N, tol = 256, TOL[dt]
     # every query its own cluster: exact whatever is retrieved
-    Q, K, V, O, *_ = retrieval_case("f32", N, S, N, 1, 1, H=1)
+    Q, K, V, O, *_ = retrieval_case(dt, N, S, N, 1, 1, H=1)
     E = mo.exact_attention(Q[0, 0], K[0, 0], V[0, 0], 1.0, causal=True)
-    parity("singleton queries vs exact", mo.max_rel_err(O[0, 0], E), 1e-4)
-    assert mo.max_rel_err(O[0, 0], E) <= 1e-4
+    parity("singleton queries vs exact", mo.max_rel_err(O[0, 0], E), tol)
+    assert mo.max_rel_err(O[0, 0], E) <= tol
     # every (cluster, block) pair retrieved: exact
-    Q, K, V, O, *_ = retrieval_case("f32", N, S, 4, 4, 4, H=1)
+    Q, K, V, O, *_ = retrieval_case(dt, N, S, 4, 4, N // S, H=1)
     E = mo.exact_attention(Q[0, 0], K[0, 0], V[0, 0], 1.0, causal=True)
-    parity("all retrieved vs exact", mo.max_rel_err(O[0, 0], E), 1e-4)
-    assert mo.max_rel_err(O[0, 0], E) <= 1e-4
+    parity("all retrieved vs exact", mo.max_rel_err(O[0, 0], E), tol)
+    assert mo.max_rel_err(O[0, 0], E) <= tol
     # nothing retrieved, singleton keys: the remainder summaries are exact
-    rng = np.random.Generator(np.random.PCG64(3))
     Qn, Kn, Vn = small_problem(23, N, 64, 64, 8, 0.3)
-    Qd, Kd, Vd = (dev(x[None, None], "f32") for x in (Qn, Kn, Vn))
+    Qd, Kd, Vd = (dev(x[None, None], dt) for x in (Qn, Kn, Vn))
     O = host(m.muse_retrieve_exact(Qd, Kd, Vd, S, 8, N, 3, 0, 0, 1.0))[0, 0]
     E = mo.exact_attention(host(Qd)[0, 0], host(Kd)[0, 0], host(Vd)[0, 0], 1.0, causal=True)
-    parity("singleton keys, nothing retrieved, vs exact", mo.max_rel_err(O, E), 1e-4)
-    assert mo.max_rel_err(O, E) <= 1e-4
+    parity("singleton keys, nothing retrieved, vs exact", mo.max_rel_err(O, E), tol)
+    assert mo.max_rel_err(O, E) <= tol
 
 
 # --------------------------------------------------------------------------- full-size workloads
@@ -535,7 +603,7 @@ def test_full_size_retrieval_n32k_sampled_rows(parity):
         # the whole selection of this head against the oracle's (near-ties counted)
         qbar = mo.cluster_means(Q[b, h], ql[b, h], w.Cq)
         lzb = mo.block_logZ(qbar, K[b, h], kl[b, h], w.Ck, w.block, w.scale)
-        ex = check_selection(lzb, sel[b, h], w.k1, w.k2)
+        ex = check_selection(lzb, sel[b, h], w.k1, w.k2, ql[b, h], w.block)
         parity(f"selection rows excused as near-ties b={b} h={h}", ex)
         assert ex <= 8, ex
     rng = np.random.default_rng(2)
