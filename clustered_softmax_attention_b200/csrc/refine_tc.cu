@@ -77,8 +77,8 @@ struct __align__(1024) Smem {
   int chunk[NST][BN / 16];                     // per 16 columns: mask, clusters, split (or kComplex)
   int koff[kMaxClusters + 1];                  // the instance's key-cluster offsets
   int kend[kMaxClusters];                      // RET: end of each cluster's causal prefix
-  unsigned short kblk[NST][BN];                // RET: key block of every column
-  int crng[NST][BN / 16];                      // RET: min | max << 16 key block per 16 columns
+  alignas(16) unsigned short kblk[NST][BN];    // RET: key block of every column (cp.async)
+  int kgrp[NST][BN / 8];                       // RET: min | max << 16 key block per 8 columns
   int wbhi[BM / 32];                           // RET: latest query block per row warp
   int tnpad[4];                                // padded width of the tiles in flight (MMA issuer)
   // per stage: key tile (consumed by the first MMA), values (second MMA), epilogue
@@ -185,9 +185,10 @@ struct TileIter {
 
 // Retrieval-mode arguments (unused by the plain refinement).
 struct RetArgs {
-  const int32_t *k_perm;  // [P][N] sorted key position -> token
-  const int32_t *pend;    // [P][Ck][nb + 1] keys of cluster j in blocks < b'
-  const int32_t *sel;     // [P][Cq][nb][K12][2] (cluster, block) pairs selected per (i, b)
+  const unsigned short *kblk;  // [P][N] block of every sorted key
+  const int *kgrp;             // [P][N / 8] min | max << 16 block of every 8 sorted keys
+  const int32_t *pend;         // [P][Ck][nb + 1] keys of cluster j in blocks < b'
+  const int32_t *sel;          // [P][Cq][nb][K12][2] (cluster, block) pairs selected per (i, b)
   int S, nb, k1, k2, K12, Cq;
 };
 
@@ -373,6 +374,17 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         cp_async16(&sm.c0[st][sg][4 * lane], in ? (const void *)(C0 + at) : (const void *)W, in ? 16u : 0u);
         cp_async16(&sm.c1[st][sg][4 * lane], in ? (const void *)(C1 + at) : (const void *)W, in ? 16u : 0u);
       }
+      if constexpr (RET) {
+        // the tile's key blocks (8 per copy) and their per-8 ranges (8-aligned tile start)
+        const int64_t g0 = (k.lab + kt.x0) / 8;
+        const int64_t gend = (k.lab + k.n + 7) / 8;  // the instance's groups end here
+        for (int v = lane; v < BN / 8; v += 32) {
+          const bool in = 8 * v < kt.npad && g0 + v < gend;
+          cp_async16(&sm.kblk[st][8 * v], in ? (const void *)(ra.kblk + 8 * (g0 + v)) : (const void *)W,
+                     in ? 16u : 0u);
+          cp_async4(&sm.kgrp[st][v], in ? (const void *)(ra.kgrp + g0 + v) : (const void *)W, in ? 4u : 0u);
+        }
+      }
       cp_async_arrive(&sm.fulle[st]);
       // column -> key cluster of the tile (0xFF outside [c, c+n)), by comparison with
       // the tile's cluster boundaries held in registers
@@ -388,7 +400,6 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           for (int b = 0; b < kTileSegs - 1; ++b) sg += key >= bnd[b] ? 1 : 0;
         }
         sm.seg[st][col] = (unsigned char)sg;
-        if constexpr (RET) sm.kblk[st][col] = (unsigned short)(sg == 0xFF ? 0xFFFF : ra.k_perm[k.lab + key] / ra.S);
       }
       // per 16-column chunk: valid-column mask (a contiguous run) << 16, the key
       // clusters of its first and last valid columns (bits 0-3, 4-7) and the first
@@ -415,20 +426,6 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         sm.chunk[st][lane] = code;
       }
       __syncwarp();
-      if constexpr (RET) {
-        // per 16 columns: the smallest and largest key block of the valid columns
-        if (lane < BN / 16) {
-          int lo = 0xFFFF, hi = 0;
-          for (int e = 0; e < 16; ++e) {
-            if (sm.seg[st][16 * lane + e] == 0xFF) continue;
-            const int b = sm.kblk[st][16 * lane + e];
-            lo = min(lo, b);
-            hi = max(hi, b);
-          }
-          sm.crng[st][lane] = lo | (hi << 16);
-        }
-        __syncwarp();
-      }
       if (lane == 0) mbar_arrive(&sm.fulle[st]);  // releases the segment map with the stage
     }
     if (lane == 0)
@@ -526,10 +523,19 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     int brow = 0;                 // RET: the row's query block (0 masks every key)
     const int32_t *so = nullptr;  // RET: the row's selected (cluster, block) slots
+    constexpr int kSelReg = 8;    // RET: selected clusters kept in registers
+    int selc[kSelReg];
+#pragma unroll
+    for (int t1 = 0; t1 < kSelReg; ++t1) selc[t1] = -1;
     if constexpr (RET) {
       if (valid) {
         brow = q_perm[q.lab + n] / ra.S;
         so = ra.sel + (((int64_t)p * ra.Cq + i) * ra.nb + brow) * ra.K12 * 2;
+        if (brow > 0) {
+#pragma unroll
+          for (int t1 = 0; t1 < kSelReg; ++t1)
+            if (t1 < ra.k1) selc[t1] = so[2 * t1 * ra.k2];
+        }
       }
     }
     TileIter<BN> it;
@@ -552,8 +558,13 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const int nch16 = kt.npad / 16;
       uint32_t xseg = 0;  // RET: tile segments holding a cluster the row selected
       if constexpr (RET) {
+#pragma unroll
+        for (int t1 = 0; t1 < kSelReg; ++t1) {
+          const int d = selc[t1] - kt.j;
+          if (selc[t1] >= 0 && d >= 0 && d < kt.nseg) xseg |= 1u << d;
+        }
         if (so && brow > 0)
-          for (int t1 = 0; t1 < ra.k1; ++t1) {
+          for (int t1 = kSelReg; t1 < ra.k1; ++t1) {
             const int d = so[2 * t1 * ra.k2] - kt.j;
             if (so[2 * t1 * ra.k2] >= 0 && d >= 0 && d < kt.nseg) xseg |= 1u << d;
           }
@@ -567,8 +578,9 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const int code = sm.chunk[st][cb];
         uint32_t keep = 0xFFFFu;  // RET: the row's causal and exclusion mask of the chunk
         if constexpr (RET) {
-          const int rng = sm.crng[st][cb];
-          const int blo = rng & 0xFFFF, bhi = rng >> 16;
+          // the chunk's block range, conservative: every key of its two 8-key groups
+          const int ga = sm.kgrp[st][2 * cb], gb = sm.kgrp[st][2 * cb + 1];
+          const int blo = min(ga & 0xFFFF, gb & 0xFFFF), bhi = max(ga >> 16, gb >> 16);
           if (blo >= brow) keep = 0u;
           else if (bhi >= brow) keep = causal_bits<D, DV>(sm, st, cb, brow);
           if (xseg && keep) keep &= excl_bits<D, DV>(sm, st, cb, xseg, kt.j, so, ra.k1, ra.k2);
@@ -756,10 +768,12 @@ cudaError_t run_refine_tc(const MuseTables &mt, int D, int Dv, int N, int P, Sor
 cudaError_t run_refine_tc_ret(const MuseTables &mt, int D, int Dv, int N, int P, SortedSide qs,
                               const int32_t *q_perm, SortedSide ks, const int32_t *k_offsets,
                               const void *vt, StageBufs b, float *part_o, float *part_lse,
-                              const int32_t *k_perm, const int32_t *pend, const int32_t *sel,
-                              int S, int k1, int k2, int *status, cudaStream_t st) {
+                              const unsigned short *kblk, const int *kgrp, const int32_t *pend,
+                              const int32_t *sel, int S, int k1, int k2, int *status,
+                              cudaStream_t st) {
   tcr::RetArgs ra;
-  ra.k_perm = k_perm;
+  ra.kblk = kblk;
+  ra.kgrp = kgrp;
   ra.pend = pend;
   ra.sel = sel;
   ra.S = S;

@@ -75,36 +75,51 @@ __global__ void block_prefix(Geo g, int P, int C, const int32_t *__restrict__ cn
   o[g.nb] = run;
 }
 
-// logZb[p][i][j][b'] = logZ_ij + log(sum of W_ik over the run of (j, b')); one warp per (i, j).
+// logZb[p][i][j][b'] = logZ_ij + log(sum of W_ik over the run of (j, b')); one thread per
+// (p, i, j, b'), the run's weights summed in key order (runs are a few keys long).
 __global__ void __launch_bounds__(256)
 block_lse(Geo g, int P, const float *__restrict__ W, int w_stride, const float *__restrict__ logZ,
           const int32_t *__restrict__ k_offsets, const int32_t *__restrict__ pend,
           float *__restrict__ logZb) {
-  const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (wid >= (int64_t)P * g.Cq * g.Ck) return;
-  const int j = (int)(wid % g.Ck);
-  const int i = (int)((wid / g.Ck) % g.Cq);
-  const int p = (int)(wid / ((int64_t)g.Ck * g.Cq));
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= (int64_t)P * g.Cq * g.Ck * g.nb) return;
+  const int b = (int)(t % g.nb);
+  const int64_t pij = t / g.nb;
+  const int j = (int)(pij % g.Ck);
+  const int i = (int)((pij / g.Ck) % g.Cq);
+  const int p = (int)(pij / ((int64_t)g.Ck * g.Cq));
   const float *w = W + (int64_t)p * w_stride + (int64_t)i * w_ld(g.N);
   const int off = k_offsets[(int64_t)p * (g.Ck + 1) + j];
   const int32_t *pe = pend + ((int64_t)p * g.Ck + j) * (g.nb + 1);
-  const float lz = logZ[((int64_t)p * g.Cq + i) * g.Ck + j];
-  float *out = logZb + (((int64_t)p * g.Cq + i) * g.Ck + j) * g.nb;
+  const int s0 = off + pe[b], s1 = off + pe[b + 1];
+  float acc = 0.f;
+  for (int pos = s0; pos < s1; ++pos) acc += w[pos];
+  logZb[t] = (s1 > s0) ? logZ[pij] + logf(acc) : -CUDART_INF_F;
+}
+
+// pref[p][i][b][j] = logsumexp_{b' < b} logZb[p][i][j][b'] (b = 0..nb), accumulated in block
+// order; one thread per (p, i, j).
+__global__ void __launch_bounds__(256)
+block_prefix_lse(Geo g, int P, const float *__restrict__ logZb, float *__restrict__ pref) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= (int64_t)P * g.Cq * g.Ck) return;
+  const int j = (int)(t % g.Ck);
+  const int64_t pi = t / g.Ck;
+  const float *lzb = logZb + t * g.nb;
+  float *out = pref + pi * (int64_t)(g.nb + 1) * g.Ck + j;
+  float acc = -CUDART_INF_F;
+  out[0] = acc;
   for (int b = 0; b < g.nb; ++b) {
-    const int s0 = off + pe[b], s1 = off + pe[b + 1];
-    float acc = 0.f;
-    for (int pos = s0 + lane; pos < s1; pos += 32) acc += w[pos];
-    acc = warp_sum(acc);
-    if (lane == 0) out[b] = (s1 > s0) ? lz + logf(acc) : -CUDART_INF_F;
+    acc = lse_add(acc, lzb[b]);
+    out[(int64_t)(b + 1) * g.Ck] = acc;
   }
 }
 
 // One warp per (p, i, b): the selection and the remainder log-normalisers.
 // sel[p][i][b][slot] = (j, b'), slot = t*k2 + u; logZR[p][i][b][j].
 __global__ void __launch_bounds__(256)
-select_blocks(Geo g, int P, const float *__restrict__ logZb, int32_t *__restrict__ sel,
-              float *__restrict__ logZR) {
+select_blocks(Geo g, int P, const float *__restrict__ logZb, const float *__restrict__ pref,
+              int32_t *__restrict__ sel, float *__restrict__ logZR) {
   constexpr int MAXJ = kMaxClusters / 32;  // clusters per lane
   const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -124,8 +139,7 @@ select_blocks(Geo g, int P, const float *__restrict__ logZb, int32_t *__restrict
     sig[m] = -CUDART_INF_F;
     taken[m] = false;
     const int j = lane + 32 * m;
-    if (j < g.Ck)
-      for (int bb = 0; bb < b; ++bb) sig[m] = lse_add(sig[m], lzb[(int64_t)j * g.nb + bb]);
+    if (j < g.Ck) sig[m] = pref[(((int64_t)p * g.Cq + i) * (g.nb + 1) + b) * g.Ck + j];
   }
   int chosen[64];
   int nchosen = 0;
@@ -187,7 +201,8 @@ select_blocks(Geo g, int P, const float *__restrict__ logZb, int32_t *__restrict
     }
   }
   __syncwarp();
-  // remainder log-normalisers: blocks b' < b, minus the selected runs
+  // remainder log-normalisers: blocks b' < b, minus the selected runs (an unselected
+  // cluster's is its prefix score, summed in the same order)
 #pragma unroll
   for (int m = 0; m < MAXJ; ++m) {
     const int j = lane + 32 * m;
@@ -195,11 +210,14 @@ select_blocks(Geo g, int P, const float *__restrict__ logZb, int32_t *__restrict
     int tj = -1;
     for (int t = 0; t < nchosen; ++t)
       if (chosen[t] == j) tj = t;
+    if (tj < 0) {
+      zr[j] = sig[m];
+      continue;
+    }
     float acc = -CUDART_INF_F;
     for (int bb = 0; bb < b; ++bb) {
       bool ex = false;
-      if (tj >= 0)
-        for (int u = 0; u < g.k2; ++u) ex |= (so[(tj * g.k2 + u) * 2 + 1] == bb);
+      for (int u = 0; u < g.k2; ++u) ex |= (so[(tj * g.k2 + u) * 2 + 1] == bb);
       if (!ex) acc = lse_add(acc, lzb[(int64_t)j * g.nb + bb]);
     }
     zr[j] = acc;
@@ -454,9 +472,10 @@ exact_merge(Geo g, float scale, const T *__restrict__ Q, const T *__restrict__ K
 // T[p][j][r] = sum over the remainder keys k of cluster j of W_ik qt_r.k for sorted query
 // row r (cluster i, block b): the keys of j in blocks b' < b minus the runs selected for
 // (i, b).  A running sum m1_j = sum_{b' < b} sum_{k in (j, b')} W_ik k over the key blocks
-// gives qt_r.m1_j; the selected runs are subtracted key by key.  One CTA per (problem,
-// query cluster i, group of JPC key clusters); DP = D / 32 threads per cluster, 32
-// coordinates each.
+// gives qt_r.m1_j; a selected cluster's runs are summed once per (i, b) group into e_j
+// and qt_r.e_j is subtracted (float32).  One CTA per (problem, query cluster i, group of
+// JPC key clusters); DP = D / 32 threads per cluster, 32 coordinates each; the group's
+// residual rows are staged in shared memory once per block.
 template <int D>
 __global__ void __launch_bounds__(256)
 ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q_offsets,
@@ -464,7 +483,9 @@ ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q
       const int32_t *__restrict__ k_offsets, const int32_t *__restrict__ pend,
       const float *__restrict__ W, int w_stride, const int32_t *__restrict__ sel,
       float *__restrict__ Tout) {
-  constexpr int DP = D / 32, JPC = 256 / DP;
+  constexpr int DP = D / 32, JPC = 256 / DP, RMAX = 2048 / D;
+  __shared__ float qsh[RMAX][D];
+  __shared__ float exsh[JPC][D + 1];
   const int p = blockIdx.z, i = blockIdx.y;
   const int jl = threadIdx.x / DP, dp = threadIdx.x % DP;
   const int j = blockIdx.x * JPC + jl;
@@ -476,68 +497,111 @@ ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q
   const int kbase = k_offsets[(int64_t)p * (g.Ck + 1) + jj];
   const float *wrow = W + (int64_t)p * w_stride + (int64_t)i * w_ld(g.N);
   const __nv_bfloat16 *kp = ks + (int64_t)p * g.N * D + dp * 32;
-  const __nv_bfloat16 *qp = qs + (int64_t)p * g.N * D + dp * 32;
+  const __nv_bfloat16 *qp = qs + (int64_t)p * g.N * D;
   float *tout = Tout + ((int64_t)p * g.Ck + jj) * g.N;
   const int r_first = qo[i];
   float m1[32];
 #pragma unroll
   for (int d = 0; d < 32; ++d) m1[d] = 0.f;
-  auto load32 = [](const __nv_bfloat16 *src, float (&x)[32]) {
+  // acc[d] += w * key[dp * 32 + d] for the key at sorted position pos
+  auto add_key = [&](int pos, float w, float (&acc)[32]) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(kp + (int64_t)pos * D);
+    uint4 u[4];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) u[v] = src[v];
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
-      const uint4 u = reinterpret_cast<const uint4 *>(src)[v];
-      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+      const uint32_t w4[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
-        x[8 * v + 2 * h] = __low2float(b2);
-        x[8 * v + 2 * h + 1] = __high2float(b2);
+        acc[8 * v + 2 * h] = fmaf(w, __low2float(b2), acc[8 * v + 2 * h]);
+        acc[8 * v + 2 * h + 1] = fmaf(w, __high2float(b2), acc[8 * v + 2 * h + 1]);
       }
     }
   };
   for (int b = 0; b < g.nb; ++b) {
     if (b > 0 && live) {
       // the keys of (j, b - 1) join the prefix
-      for (int pos = kbase + pe[b - 1]; pos < kbase + pe[b]; ++pos) {
-        float x[32];
-        load32(kp + (int64_t)pos * D, x);
-        const float w = wrow[pos];
-#pragma unroll
-        for (int d = 0; d < 32; ++d) m1[d] = fmaf(w, x[d], m1[d]);
+      const int e = kbase + pe[b];
+      int pos = kbase + pe[b - 1];
+      for (; pos + 1 < e; pos += 2) {
+        const float w0 = wrow[pos], w1 = wrow[pos + 1];
+        add_key(pos, w0, m1);
+        add_key(pos + 1, w1, m1);
       }
+      if (pos < e) add_key(pos, wrow[pos], m1);
     }
     const int r0 = r_first + qpe[b], r1 = r_first + qpe[b + 1];
     if (r0 >= r1) continue;  // CTA-uniform
-    // the slots of cluster j among those selected for (i, b): tj (or -1)
-    const int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
+    // a cluster the group selected: the sum of its selected runs, once for the group
     int tj = -1;
+    const int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
     if (b > 0 && live)
       for (int t = 0; t < g.k1; ++t)
         if (so[2 * t * g.k2] == j) tj = t;
-    for (int r = r0; r < r1; ++r) {
-      float q[32];
-      load32(qp + (int64_t)r * D, q);
-      float acc = 0.f;
-      if (b > 0) {
+    if (tj >= 0) {
+      float ex[32];
 #pragma unroll
-        for (int d = 0; d < 32; ++d) acc = fmaf(q[d], m1[d], acc);
-        for (int u = 0; tj >= 0 && u < g.k2; ++u) {
-          const int bb = so[2 * (tj * g.k2 + u) + 1];
-          if (bb < 0) continue;
-          for (int pos = kbase + pe[bb]; pos < kbase + pe[bb + 1]; ++pos) {
-            float x[32];
-            load32(kp + (int64_t)pos * D, x);
-            float dot = 0.f;
-#pragma unroll
-            for (int d = 0; d < 32; ++d) dot = fmaf(q[d], x[d], dot);
-            acc = fmaf(-wrow[pos], dot, acc);
-          }
-        }
+      for (int d = 0; d < 32; ++d) ex[d] = 0.f;
+      for (int u = 0; u < g.k2; ++u) {
+        const int bb = so[2 * (tj * g.k2 + u) + 1];
+        if (bb < 0) continue;
+        for (int pos = kbase + pe[bb]; pos < kbase + pe[bb + 1]; ++pos) add_key(pos, wrow[pos], ex);
       }
 #pragma unroll
-      for (int o = DP / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (live && dp == 0) tout[r] = acc;
+      for (int d = 0; d < 32; ++d) exsh[jl][dp * 32 + d] = ex[d];
     }
+    for (int rb = r0; rb < r1; rb += RMAX) {
+      const int nr = min(RMAX, r1 - rb);
+      __syncthreads();  // the previous rows are read
+      for (int e = threadIdx.x; e < nr * (D / 8); e += blockDim.x) {
+        const int rr = e / (D / 8), v = e % (D / 8);
+        const uint4 u = reinterpret_cast<const uint4 *>(qp + (int64_t)(rb + rr) * D)[v];
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
+          qsh[rr][8 * v + 2 * h] = __low2float(b2);
+          qsh[rr][8 * v + 2 * h + 1] = __high2float(b2);
+        }
+      }
+      __syncthreads();
+      for (int rr = 0; rr < nr; ++rr) {
+        float acc = 0.f;
+        if (b > 0) {
+#pragma unroll
+          for (int d = 0; d < 32; ++d) acc = fmaf(qsh[rr][dp * 32 + d], m1[d], acc);
+          if (tj >= 0) {
+#pragma unroll
+            for (int d = 0; d < 32; ++d) acc = fmaf(-qsh[rr][dp * 32 + d], exsh[jl][dp * 32 + d], acc);
+          }
+        }
+#pragma unroll
+        for (int o = DP / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (live && dp == 0) tout[rb + rr] = acc;
+      }
+    }
+  }
+}
+
+// kb[p][pos] = block of the key at sorted position pos; kg[p][pos / 8] = smallest | largest
+// << 16 block of the 8 keys pos & ~7 .. (pos & ~7) + 7 (N is a multiple of 8).
+__global__ void __launch_bounds__(256)
+key_blocks(Geo g, const int32_t *__restrict__ k_perm, unsigned short *__restrict__ kb,
+           int *__restrict__ kg) {
+  const int p = blockIdx.y;
+  const int pos = blockIdx.x * blockDim.x + threadIdx.x;
+  const int b = pos < g.N ? k_perm[(int64_t)p * g.N + pos] / g.S : 0;
+  int lo = b, hi = b;
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (pos < g.N) {
+    kb[(int64_t)p * g.N + pos] = (unsigned short)b;
+    if ((pos & 7) == 0) kg[(int64_t)p * (g.N / 8) + pos / 8] = lo | (hi << 16);
   }
 }
 
@@ -619,22 +683,40 @@ ret_runs(Geo g, float scale, const __nv_bfloat16 *__restrict__ Q, const __nv_bfl
   const int32_t *qpe = qpend + ((int64_t)p * g.Cq + i) * (g.nb + 1);
   const int r0 = qo[i] + qpe[b], r1 = qo[i] + qpe[b + 1];
   if (r0 >= r1) return;  // uniform
-  if (threadIdx.x == 0) {
-    const int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
-    int n = 0;
-    cum[0] = 0;
-    for (int t = 0; t < g.K12; ++t) {
+  // the selected runs: slot t (a warp pair reads the K12 <= 64 slots at once), then an
+  // inclusive scan of their lengths by warp 0
+  __shared__ int len[64];
+  if (threadIdx.x < 64) {
+    const int t = threadIdx.x;
+    int start = 0, n = 0;
+    if (t < g.K12) {
+      const int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
       const int j = so[2 * t], bb = so[2 * t + 1];
-      if (j < 0) continue;
-      const int base = k_offsets[(int64_t)p * (g.Ck + 1) + j];
-      const int32_t *pe = pend + ((int64_t)p * g.Ck + j) * (g.nb + 1);
-      if (pe[bb + 1] > pe[bb]) {
-        runs[n] = base + pe[bb];
-        cum[n + 1] = cum[n] + pe[bb + 1] - pe[bb];
-        ++n;
+      if (j >= 0) {
+        const int32_t *pe = pend + ((int64_t)p * g.Ck + j) * (g.nb + 1);
+        start = k_offsets[(int64_t)p * (g.Ck + 1) + j] + pe[bb];
+        n = pe[bb + 1] - pe[bb];
       }
     }
-    nruns = n;
+    runs[t] = start;
+    len[t] = n;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int a = len[2 * lane], c = len[2 * lane + 1];
+    int inc = a + c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const int excl = inc - a - c;
+    cum[2 * lane] = excl;
+    cum[2 * lane + 1] = excl + a;
+    if (lane == 31) {
+      cum[64] = inc;
+      nruns = 64;
+    }
   }
   __syncthreads();
   const int total = cum[nruns];
@@ -744,9 +826,11 @@ struct Ws {
   int32_t *v_cluster;
   float *W, *logZ;
   int32_t *cnt, *pend, *sel;
-  float *logZb, *logZR, *T, *c0, *c1, *lse_r, *part_o;
+  float *logZb, *logZR, *T, *c0, *c1, *lse_r, *part_o, *pref;
   SortedSide qs;              // tensor-core path: sorted residuals
   int32_t *qcnt, *qpend;      // rows of query cluster i in / before each block
+  unsigned short *kb;         // block of every sorted key
+  int *kg;                    // block range of every 8 sorted keys
   float *part_lse;            // remainder + runs log-normaliser per token
 };
 
@@ -812,6 +896,7 @@ static void plan(Bump2 &bp, const muse_dims &d, const Geo &g, Ws &w) {
   w.pend = bp.take<int32_t>((size_t)P * g.Ck * (g.nb + 1));
   w.sel = bp.take<int32_t>((size_t)P * g.Cq * g.nb * g.K12 * 2);
   w.logZb = bp.take<float>((size_t)P * g.Cq * g.Ck * g.nb);
+  w.pref = bp.take<float>((size_t)P * g.Cq * (g.nb + 1) * g.Ck);
   w.logZR = bp.take<float>((size_t)P * g.Cq * g.nb * g.Ck);
   w.T = bp.take<float>((size_t)P * g.Ck * d.N);
   w.c0 = bp.take<float>((size_t)P * g.Ck * d.N);
@@ -823,6 +908,8 @@ static void plan(Bump2 &bp, const muse_dims &d, const Geo &g, Ws &w) {
   w.qcnt = bp.take<int32_t>((size_t)P * g.Cq * g.nb);
   w.qpend = bp.take<int32_t>((size_t)P * g.Cq * (g.nb + 1));
   w.part_lse = bp.take<float>((size_t)P * d.N);
+  w.kb = bp.take<unsigned short>((size_t)P * d.N);
+  w.kg = bp.take<int>((size_t)P * (d.N / 8));
 }
 
 static bool valid_geo(const muse_dims &d, int block, int Cq, int Ck, int k1, int k2, Geo &g) {
@@ -875,23 +962,25 @@ static cudaError_t run_tc(const void *Q, const void *K, const void *V, const mus
   block_counts<<<dim3((d.N + 255) / 256, P), 256, 0, st>>>(g, g.Cq, w.q.labels, w.qcnt);
   block_prefix<<<(P * g.Cq + 127) / 128, 128, 0, st>>>(g, P, g.Cq, w.qcnt, w.qpend);
   const int64_t nw = (int64_t)P * g.Cq * g.Ck;
-  block_lse<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(g, P, w.W, mt.in.w_stride, w.logZ,
-                                                      w.k.offsets, w.pend, w.logZb);
+  block_lse<<<(unsigned)((nw * g.nb + 255) / 256), 256, 0, st>>>(g, P, w.W, mt.in.w_stride, w.logZ,
+                                                                  w.k.offsets, w.pend, w.logZb);
+  block_prefix_lse<<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(g, P, w.logZb, w.pref);
   const int64_t ns = (int64_t)P * g.Cq * g.nb;
-  select_blocks<<<(unsigned)((ns + 7) / 8), 256, 0, st>>>(g, P, w.logZb, w.sel, w.logZR);
+  select_blocks<<<(unsigned)((ns + 7) / 8), 256, 0, st>>>(g, P, w.logZb, w.pref, w.sel, w.logZR);
   constexpr int JPC = 256 / (D / 32);
   ret_T<D><<<dim3((g.Ck + JPC - 1) / JPC, g.Cq, P), 256, 0, st>>>(
       g, (const __nv_bfloat16 *)w.qs.rows, w.q.offsets, w.qpend, (const __nv_bfloat16 *)w.ks.rows,
       w.k.offsets, w.pend, w.W, mt.in.w_stride, w.sel, w.T);
   ret_coeffs<<<dim3((d.N + 127) / 128, P), 128, 0, st>>>(g, d.scale, w.q.perm, w.qs.cluster, w.logZ,
                                                         w.logZR, w.T, w.c0, w.c1, w.lse_r);
+  key_blocks<<<dim3((d.N + 255) / 256, P), 256, 0, st>>>(g, w.k.perm, w.kb, w.kg);
   count_launches(10);
   sb.c0 = w.c0;
   sb.c1 = w.c1;
   sb.lse = w.lse_r;
   if ((e = profile_mark(true, st)) != cudaSuccess) return e;
   if ((e = run_refine_tc_ret(mt, D, DV, d.N, P, w.qs, w.q.perm, w.ks, w.k.offsets, w.vs, sb,
-                             w.part_o, w.part_lse, w.k.perm, w.pend, w.sel, g.S, g.k1, g.k2,
+                             w.part_o, w.part_lse, w.kb, w.kg, w.pend, w.sel, g.S, g.k1, g.k2,
                              status, st)) != cudaSuccess)
     return e;
   if ((e = profile_mark(false, st)) != cudaSuccess) return e;
@@ -932,10 +1021,11 @@ static cudaError_t run_t(const void *Q, const void *K, const void *V, const muse
   block_counts<<<dim3((d.N + 255) / 256, P), 256, 0, st>>>(g, g.Ck, w.k.labels, w.cnt);
   block_prefix<<<(P * g.Ck + 127) / 128, 128, 0, st>>>(g, P, g.Ck, w.cnt, w.pend);
   const int64_t nw = (int64_t)P * g.Cq * g.Ck;
-  block_lse<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(g, P, w.W, mt.in.w_stride, w.logZ,
-                                                      w.k.offsets, w.pend, w.logZb);
+  block_lse<<<(unsigned)((nw * g.nb + 255) / 256), 256, 0, st>>>(g, P, w.W, mt.in.w_stride, w.logZ,
+                                                                  w.k.offsets, w.pend, w.logZb);
+  block_prefix_lse<<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(g, P, w.logZb, w.pref);
   const int64_t ns = (int64_t)P * g.Cq * g.nb;
-  select_blocks<<<(unsigned)((ns + 7) / 8), 256, 0, st>>>(g, P, w.logZb, w.sel, w.logZR);
+  select_blocks<<<(unsigned)((ns + 7) / 8), 256, 0, st>>>(g, P, w.logZb, w.pref, w.sel, w.logZR);
   dim3 qg(d.N / 64, P);
   remainder_pass<T, D, DV, 0><<<qg, 256, 0, st>>>(
       g, (const T *)Q, w.q.centroids, w.q.labels, (const T *)w.ks.rows, (const T *)w.vs, w.k.perm,
@@ -948,7 +1038,7 @@ static cudaError_t run_t(const void *Q, const void *K, const void *V, const muse
   exact_merge<T, D, DV><<<qg, 256, 0, st>>>(g, d.scale, (const T *)Q, (const T *)K, (const T *)V,
                                             w.q.labels, (const T *)w.ks.rows, (const T *)w.vs,
                                             w.k.offsets, w.pend, w.sel, w.part_o, w.lse_r, (T *)O);
-  count_launches(8);
+  count_launches(9);
   return cudaGetLastError();
 }
 

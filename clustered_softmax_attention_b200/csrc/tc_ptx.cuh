@@ -146,6 +146,12 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t 
                "r"(src_bytes)
                : "memory");
 }
+// 4-byte global -> shared copy; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(saddr(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
 // The barrier's phase also waits for this thread's earlier cp.async copies.
 __device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(saddr(bar)) : "memory");
