@@ -21,7 +21,10 @@
 //
 // Float32 on the CUDA cores, every sum in a fixed order (no floating-point atomics).
 // The forward summaries, C_ij included, are recomputed and materialised in the
-// workspace (Cq Ck Dv D floats per problem, twice with dC).
+// workspace (Cq Ck Dv D floats per problem, twice with dC).  Kernels: means (qbar),
+// the forward summaries, rows (per query cluster: softmax backward, dqt and the cluster
+// sums), keys (two passes per key cluster: the tilted-moment backward into dk, dv and the
+// logit gradients), queries (dqbar and the centroid correction), unsort.
 #include <string.h>
 
 #include "internal.h"
@@ -59,155 +62,220 @@ __device__ __forceinline__ int cluster_of(const int32_t *off, int C, int r) {
   return lo;
 }
 
-// Per sorted query row (one warp): p_nj and da_nj for every key cluster (PA, DA
-// [P][N][Ck]) and dqt_n (dQt [P][N][D], sorted rows).  Two passes over j: logits and
-// dp_nj (online softmax), then p, da and dqt.  u_j = C_ij^T dO_n is formed in both.
+// Per query cluster i (one CTA of eight warps): the rows of the cluster in passes of
+// RP = 32 (four per warp), and for every key cluster j with C_ij, mu_k,ij, mu_v,ij staged in
+// shared memory once per pass:
+//   pass A: a_nj = logZ_ij + s qt_n.mu_k,ij and dp_nj = dO_n.mu_v,ij + s qt_n.(C_ij^T dO_n)
+//           (online softmax statistics; a and dp kept in PA, DA [P][N][Ck], sorted rows);
+//   pass B: p_nj, da_nj = p_nj (dp_nj - sum_j' p_nj' dp_nj'), dqt_n += s (da_nj mu_k,ij +
+//           p_nj C_ij^T dO_n), and the cluster sums dlogZ_ij, dmu_k,ij, dmu_v,ij and
+//           dC_ij = s sum_n p_nj dO_n qt_n^T over the pass's rows (added pass by pass in
+//           row order: deterministic).
 template <typename T, int D, int DV>
 __global__ void __launch_bounds__(256)
 rows(Geo g, const T *__restrict__ Q, const T *__restrict__ dO, const int32_t *__restrict__ q_perm,
      const int32_t *__restrict__ q_offsets, const float *__restrict__ qbar,
      const float *__restrict__ logZ, const float *__restrict__ mu_k, const float *__restrict__ mu_v,
      const float *__restrict__ cov, float *__restrict__ PA, float *__restrict__ DA,
-     float *__restrict__ dQt) {
-  constexpr int PD = D / 32, PV = DV / 32;
-  __shared__ float do_sh[8][DV];
-  const int p = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * 8 + warp;
-  if (r >= g.N) return;  // whole warps
-  const int i = cluster_of(q_offsets + (int64_t)p * (g.Cq + 1), g.Cq, r);
-  const int n = q_perm[(int64_t)p * g.N + r];
-  float qt[PD];
-#pragma unroll
-  for (int t = 0; t < PD; ++t)
-    qt[t] = ld_elem(Q + ((int64_t)p * g.N + n) * D + lane + 32 * t) - qbar[((int64_t)p * g.Cq + i) * D + lane + 32 * t];
-  float dov[PV];
-#pragma unroll
-  for (int v = 0; v < PV; ++v) {
-    dov[v] = ld_elem(dO + ((int64_t)p * g.N + n) * DV + lane + 32 * v);
-    do_sh[warp][lane + 32 * v] = dov[v];
-  }
-  __syncwarp();
-  const int64_t ij0 = ((int64_t)p * g.Cq + i) * g.Ck;
-  float *pa = PA + ((int64_t)p * g.N + r) * g.Ck;
-  float *da = DA + ((int64_t)p * g.N + r) * g.Ck;
-  // u = C^T dO (lane owns coordinates lane + 32 t)
-  auto ctdo = [&](int j, float (&u)[PD]) {
-    const float *cj = cov + (ij0 + j) * DV * D;
-#pragma unroll
-    for (int t = 0; t < PD; ++t) u[t] = 0.f;
-    for (int v = 0; v < DV; ++v) {
-      const float dv = do_sh[warp][v];
-#pragma unroll
-      for (int t = 0; t < PD; ++t) u[t] = fmaf(cj[(int64_t)v * D + lane + 32 * t], dv, u[t]);
-    }
-  };
-  float m = -CUDART_INF_F, l = 0.f, sdp = 0.f;  // running max, sum of e^(a-m), sum of e^(a-m) dp
-  for (int j = 0; j < g.Ck; ++j) {
-    const float lz = logZ[ij0 + j];
-    if (!(lz > -CUDART_INF_F)) {
-      if (lane == 0) pa[j] = -CUDART_INF_F;
-      continue;
-    }
-    float u[PD];
-    ctdo(j, u);
-    float x = 0.f, y = 0.f, z = 0.f;
-#pragma unroll
-    for (int t = 0; t < PD; ++t) {
-      x = fmaf(qt[t], mu_k[(ij0 + j) * D + lane + 32 * t], x);
-      y = fmaf(qt[t], u[t], y);
-    }
-#pragma unroll
-    for (int v = 0; v < PV; ++v) z = fmaf(dov[v], mu_v[(ij0 + j) * DV + lane + 32 * v], z);
-    const float a = lz + g.s * warp_sum(x);
-    const float dp = fmaf(g.s, warp_sum(y), warp_sum(z));  // dO.(mu_v + s C qt)
-    const float mn = fmaxf(m, a);
-    const float c = expf(m - mn), e = expf(a - mn);
-    l = l * c + e;
-    sdp = sdp * c + e * dp;
-    m = mn;
-    if (lane == 0) {
-      pa[j] = a;
-      da[j] = dp;
-    }
-  }
-  __syncwarp();
-  const float lse = m + logf(l), mean_dp = sdp / l;
-  float dq[PD];
-#pragma unroll
-  for (int t = 0; t < PD; ++t) dq[t] = 0.f;
-  for (int j = 0; j < g.Ck; ++j) {
-    const float a = pa[j];
-    if (!(a > -CUDART_INF_F)) {
-      __syncwarp();
-      if (lane == 0) {
-        pa[j] = 0.f;
-        da[j] = 0.f;
-      }
-      continue;
-    }
-    const float pj = expf(a - lse);
-    const float daj = pj * (da[j] - mean_dp);
-    float u[PD];
-    ctdo(j, u);
-#pragma unroll
-    for (int t = 0; t < PD; ++t)
-      dq[t] = fmaf(g.s, fmaf(daj, mu_k[(ij0 + j) * D + lane + 32 * t], pj * u[t]), dq[t]);
-    __syncwarp();
-    if (lane == 0) {
-      pa[j] = pj;
-      da[j] = daj;
-    }
-  }
-#pragma unroll
-  for (int t = 0; t < PD; ++t) dQt[((int64_t)p * g.N + r) * D + lane + 32 * t] = dq[t];
-}
-
-// Per (query cluster i, key cluster j): sums over the rows of cluster i (sorted order):
-// dlogZ, dmu_k, dmu_v and dC [Dv][D].  256 threads, 16 (D = Dv = 64) to 64 entries of dC
-// each.
-template <typename T, int D, int DV>
-__global__ void __launch_bounds__(256)
-cluster_sums(Geo g, const T *__restrict__ Q, const T *__restrict__ dO,
-             const int32_t *__restrict__ q_perm, const int32_t *__restrict__ q_offsets,
-             const float *__restrict__ qbar, const float *__restrict__ PA,
-             const float *__restrict__ DA, float *__restrict__ dlogZ, float *__restrict__ dmuk,
-             float *__restrict__ dmuv, float *__restrict__ dC) {
-  constexpr int E = DV * D / 256;
-  __shared__ float qt[D], dov[DV], pd[2];
-  const int p = blockIdx.z, i = blockIdx.y, j = blockIdx.x;
+     float *__restrict__ dQt, float *__restrict__ dlogZ, float *__restrict__ dmuk,
+     float *__restrict__ dmuv, float *__restrict__ dC) {
+  constexpr int PD = D / 32, PV = DV / 32, RW = 4, RP = 8 * RW, E = DV * D / 256;
+  extern __shared__ float sm_raw[];
+  float *Cs = sm_raw;                 // [DV][D]
+  float *qt_sh = Cs + DV * D;         // [RP][D]
+  float *do_sh = qt_sh + RP * D;      // [RP][DV]
+  float *mk = do_sh + RP * DV;        // [D]
+  float *mv = mk + D;                 // [DV]
+  float *pj_sh = mv + DV;             // [RP]
+  float *da_sh = pj_sh + RP;          // [RP]
+  const int p = blockIdx.y, i = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t *off = q_offsets + (int64_t)p * (g.Cq + 1);
-  const int r0 = off[i], r1 = off[i + 1];
-  const int64_t ij = ((int64_t)p * g.Cq + i) * g.Ck + j;
-  float acc[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  float amk = 0.f, amv = 0.f, alz = 0.f;  // thread t < D: dmu_k[t]; t < DV: dmu_v[t]; t == 0: dlogZ
-  for (int r = r0; r < r1; ++r) {
+  const int R0 = off[i], R1 = off[i + 1];
+  const int64_t ij0 = ((int64_t)p * g.Cq + i) * g.Ck;
+  // C_ij, mu_k, mu_v of cluster j into shared memory (after a barrier of the caller)
+  auto stage = [&](int j) {
+    const float4 *src = reinterpret_cast<const float4 *>(cov + (ij0 + j) * DV * D);
+    for (int e = threadIdx.x; e < DV * D / 4; e += 256) reinterpret_cast<float4 *>(Cs)[e] = src[e];
+    if (threadIdx.x < D) mk[threadIdx.x] = mu_k[(ij0 + j) * D + threadIdx.x];
+    if (threadIdx.x >= 128 && threadIdx.x - 128 < DV) mv[threadIdx.x - 128] = mu_v[(ij0 + j) * DV + threadIdx.x - 128];
+  };
+  for (int pr0 = R0; pr0 < R1; pr0 += RP) {
+    const int nr = min(RP, R1 - pr0);
     __syncthreads();
-    const int n = q_perm[(int64_t)p * g.N + r];
-    if (threadIdx.x < D)
-      qt[threadIdx.x] = ld_elem(Q + ((int64_t)p * g.N + n) * D + threadIdx.x) - qbar[((int64_t)p * g.Cq + i) * D + threadIdx.x];
-    if (threadIdx.x < DV) dov[threadIdx.x] = ld_elem(dO + ((int64_t)p * g.N + n) * DV + threadIdx.x);
-    if (threadIdx.x == 0) {
-      pd[0] = PA[((int64_t)p * g.N + r) * g.Ck + j];
-      pd[1] = DA[((int64_t)p * g.N + r) * g.Ck + j];
+    // the pass's residuals and output gradients, float32
+    for (int e = threadIdx.x; e < RP * D; e += 256) {
+      const int rr = e / D, d = e % D;
+      float v = 0.f;
+      if (rr < nr) {
+        const int n = q_perm[(int64_t)p * g.N + pr0 + rr];
+        v = ld_elem(Q + ((int64_t)p * g.N + n) * D + d) - qbar[((int64_t)p * g.Cq + i) * D + d];
+      }
+      qt_sh[e] = v;
     }
-    __syncthreads();
-    const float pj = pd[0], daj = pd[1];
+    for (int e = threadIdx.x; e < RP * DV; e += 256) {
+      const int rr = e / DV, v = e % DV;
+      do_sh[e] = rr < nr ? ld_elem(dO + ((int64_t)p * g.N + q_perm[(int64_t)p * g.N + pr0 + rr]) * DV + v) : 0.f;
+    }
+    // this warp's rows: pr0 + warp + 8 q, q < RW
+    float m[RW], l[RW], sdp[RW];
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int idx = threadIdx.x + 256 * e;
-      acc[e] = fmaf(pj * dov[idx / D], qt[idx % D], acc[e]);
+    for (int q = 0; q < RW; ++q) {
+      m[q] = -CUDART_INF_F;
+      l[q] = 0.f;
+      sdp[q] = 0.f;
     }
-    if (threadIdx.x < D) amk = fmaf(daj, qt[threadIdx.x], amk);
-    if (threadIdx.x < DV) amv = fmaf(pj, dov[threadIdx.x], amv);
-    if (threadIdx.x == 0) alz += daj;
+    // u_q = C^T dO of row q (lane owns coordinates lane + 32 t)
+    auto ctdo = [&](float (&u)[RW][PD]) {
+#pragma unroll
+      for (int q = 0; q < RW; ++q)
+#pragma unroll
+        for (int t = 0; t < PD; ++t) u[q][t] = 0.f;
+      for (int v = 0; v < DV; ++v) {
+        float c[PD];
+#pragma unroll
+        for (int t = 0; t < PD; ++t) c[t] = Cs[v * D + lane + 32 * t];
+#pragma unroll
+        for (int q = 0; q < RW; ++q) {
+          const float dv = do_sh[(warp + 8 * q) * DV + v];
+#pragma unroll
+          for (int t = 0; t < PD; ++t) u[q][t] = fmaf(c[t], dv, u[q][t]);
+        }
+      }
+    };
+    // ---- pass A
+    for (int j = 0; j < g.Ck; ++j) {
+      const float lz = logZ[ij0 + j];
+      if (!(lz > -CUDART_INF_F)) continue;  // uniform
+      __syncthreads();
+      stage(j);
+      __syncthreads();
+      float u[RW][PD];
+      ctdo(u);
+#pragma unroll
+      for (int q = 0; q < RW; ++q) {
+        const int rr = warp + 8 * q;
+        float x = 0.f, y = 0.f, z = 0.f;
+#pragma unroll
+        for (int t = 0; t < PD; ++t) {
+          const float qv = qt_sh[rr * D + lane + 32 * t];
+          x = fmaf(qv, mk[lane + 32 * t], x);
+          y = fmaf(qv, u[q][t], y);
+        }
+#pragma unroll
+        for (int v = 0; v < PV; ++v) z = fmaf(do_sh[rr * DV + lane + 32 * v], mv[lane + 32 * v], z);
+        const float a = lz + g.s * warp_sum(x);
+        const float dp = fmaf(g.s, warp_sum(y), warp_sum(z));
+        const float mn = fmaxf(m[q], a);
+        const float c = expf(m[q] - mn), e = expf(a - mn);
+        l[q] = l[q] * c + e;
+        sdp[q] = sdp[q] * c + e * dp;
+        m[q] = mn;
+        if (lane == 0 && rr < nr) {
+          PA[((int64_t)p * g.N + pr0 + rr) * g.Ck + j] = a;
+          DA[((int64_t)p * g.N + pr0 + rr) * g.Ck + j] = dp;
+        }
+      }
+    }
+    float lse[RW], mdp[RW], dq[RW][PD];
+#pragma unroll
+    for (int q = 0; q < RW; ++q) {
+      lse[q] = m[q] + logf(l[q]);
+      mdp[q] = sdp[q] / l[q];
+#pragma unroll
+      for (int t = 0; t < PD; ++t) dq[q][t] = 0.f;
+    }
+    // ---- pass B
+    for (int j = 0; j < g.Ck; ++j) {
+      const float lz = logZ[ij0 + j];
+      const int64_t ij = ij0 + j;
+      if (!(lz > -CUDART_INF_F)) {
+        // an empty key cluster: no weight, and zero sums (written once, by the first pass)
+        if (pr0 == R0) {
+          for (int e = threadIdx.x; e < DV * D; e += 256) dC[ij * DV * D + e] = 0.f;
+          if (threadIdx.x < D) dmuk[ij * D + threadIdx.x] = 0.f;
+          if (threadIdx.x < DV) dmuv[ij * DV + threadIdx.x] = 0.f;
+          if (threadIdx.x == 0) dlogZ[ij] = 0.f;
+        }
+        if (threadIdx.x < nr) {
+          PA[((int64_t)p * g.N + pr0 + threadIdx.x) * g.Ck + j] = 0.f;
+          DA[((int64_t)p * g.N + pr0 + threadIdx.x) * g.Ck + j] = 0.f;
+        }
+        continue;
+      }
+      __syncthreads();
+      stage(j);
+      __syncthreads();
+      float u[RW][PD];
+      ctdo(u);
+#pragma unroll
+      for (int q = 0; q < RW; ++q) {
+        const int rr = warp + 8 * q;
+        float pj = 0.f, daj = 0.f;
+        if (rr < nr) {
+          const int64_t at = ((int64_t)p * g.N + pr0 + rr) * g.Ck + j;
+          pj = expf(PA[at] - lse[q]);
+          daj = pj * (DA[at] - mdp[q]);
+        }
+#pragma unroll
+        for (int t = 0; t < PD; ++t)
+          dq[q][t] = fmaf(g.s, fmaf(daj, mk[lane + 32 * t], pj * u[q][t]), dq[q][t]);
+        if (lane == 0) {
+          pj_sh[rr] = pj;
+          da_sh[rr] = daj;
+        }
+      }
+      __syncthreads();
+      // the cluster sums of this pass (rows in order), added to the earlier passes'
+      float acc[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = 0.f;
+      float amk = 0.f, amv = 0.f, alz = 0.f;
+      for (int rr = 0; rr < nr; ++rr) {
+        const float pjr = pj_sh[rr], dar = da_sh[rr];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int idx = threadIdx.x + 256 * e;
+          acc[e] = fmaf(pjr * do_sh[rr * DV + idx / D], qt_sh[rr * D + idx % D], acc[e]);
+        }
+        if (threadIdx.x < D) amk = fmaf(dar, qt_sh[rr * D + threadIdx.x], amk);
+        if (threadIdx.x >= 128 && threadIdx.x - 128 < DV) amv = fmaf(pjr, do_sh[rr * DV + threadIdx.x - 128], amv);
+        if (threadIdx.x == 0) alz += dar;
+      }
+      const bool first = pr0 == R0;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        float *dst = dC + ij * DV * D + threadIdx.x + 256 * e;
+        *dst = (first ? 0.f : *dst) + g.s * acc[e];
+      }
+      if (threadIdx.x < D) {
+        float *dst = dmuk + ij * D + threadIdx.x;
+        *dst = (first ? 0.f : *dst) + g.s * amk;
+      }
+      if (threadIdx.x >= 128 && threadIdx.x - 128 < DV) {
+        float *dst = dmuv + ij * DV + threadIdx.x - 128;
+        *dst = (first ? 0.f : *dst) + amv;
+      }
+      if (threadIdx.x == 0) dlogZ[ij] = (first ? 0.f : dlogZ[ij]) + alz;
+    }
+#pragma unroll
+    for (int q = 0; q < RW; ++q) {
+      const int rr = warp + 8 * q;
+      if (rr < nr)
+#pragma unroll
+        for (int t = 0; t < PD; ++t) dQt[((int64_t)p * g.N + pr0 + rr) * D + lane + 32 * t] = dq[q][t];
+    }
   }
-#pragma unroll
-  for (int e = 0; e < E; ++e) dC[ij * DV * D + threadIdx.x + 256 * e] = g.s * acc[e];
-  if (threadIdx.x < D) dmuk[ij * D + threadIdx.x] = g.s * amk;
-  if (threadIdx.x < DV) dmuv[ij * DV + threadIdx.x] = amv;
-  if (threadIdx.x == 0) dlogZ[ij] = alz;
+  if (R0 == R1) {
+    // an empty query cluster: zero cluster sums
+    for (int j = 0; j < g.Ck; ++j) {
+      const int64_t ij = ij0 + j;
+      for (int e = threadIdx.x; e < DV * D; e += 256) dC[ij * DV * D + e] = 0.f;
+      if (threadIdx.x < D) dmuk[ij * D + threadIdx.x] = 0.f;
+      if (threadIdx.x < DV) dmuv[ij * DV + threadIdx.x] = 0.f;
+      if (threadIdx.x == 0) dlogZ[ij] = 0.f;
+    }
+  }
 }
 
 // Per (key cluster j, problem): for every query centroid i, the corrected mean gradients
@@ -459,12 +527,13 @@ static cudaError_t run_t(const void *Q, const void *K, const void *V, const void
   if ((e = run_summaries(mt, d.dtype, D, DV, P, d.scale, w.qbar, w.ks, w.vs, k_offsets, w.sb, st)) !=
       cudaSuccess)
     return e;
-  rows<T, D, DV><<<dim3((N + 7) / 8, P), 256, 0, st>>>(g, (const T *)Q, (const T *)dO, q_perm, q_offsets,
-                                                      w.qbar, w.sb.logZ, w.sb.mu_k, w.sb.mu_v,
-                                                      w.sb.cov, w.PA, w.DA, w.dQt);
-  cluster_sums<T, D, DV><<<dim3(Ck, Cq, P), 256, 0, st>>>(g, (const T *)Q, (const T *)dO, q_perm,
-                                                         q_offsets, w.qbar, w.PA, w.DA, w.dlogZ,
-                                                         w.dmuk, w.dmuv, w.dC);
+  const size_t rsm = (size_t)(DV * D + 32 * (D + DV) + D + DV + 64) * sizeof(float);
+  if ((e = cudaFuncSetAttribute(rows<T, D, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)rsm)) != cudaSuccess)
+    return e;
+  rows<T, D, DV><<<dim3(Cq, P), 256, rsm, st>>>(g, (const T *)Q, (const T *)dO, q_perm, q_offsets,
+                                               w.qbar, w.sb.logZ, w.sb.mu_k, w.sb.mu_v, w.sb.cov,
+                                               w.PA, w.DA, w.dQt, w.dlogZ, w.dmuk, w.dmuv, w.dC);
   const size_t gsm = (size_t)DV * (D + 1) * sizeof(float);
   if ((e = cudaFuncSetAttribute(keys<T, D, DV, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)gsm)) != cudaSuccess ||
@@ -483,7 +552,7 @@ static cudaError_t run_t(const void *Q, const void *K, const void *V, const void
                                             w.dQt, (T *)dQ);
   unsort<T><<<dim3((unsigned)(((int64_t)N * D + 255) / 256), P), 256, 0, st>>>(N, D, k_perm, w.dKs, (T *)dK);
   unsort<T><<<dim3((unsigned)(((int64_t)N * DV + 255) / 256), P), 256, 0, st>>>(N, DV, k_perm, w.dVs, (T *)dV);
-  count_launches(9);
+  count_launches(7);
   return cudaGetLastError();
 }
 

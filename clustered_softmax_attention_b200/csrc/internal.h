@@ -17,6 +17,9 @@ void count_launches(int n);
 // Device address of the current device's status word (NULL if unavailable).
 int *device_status_word();
 
+// Records a CUDA error for muse_last_error_detail (this thread) and returns MUSE_ERR_CUDA.
+muse_status cuda_fail(cudaError_t e);
+
 // Records the event set by muse_set_profile_events before (start) or after the dominant
 // kernel of a call, when events are set; cudaSuccess otherwise.
 cudaError_t profile_mark(bool start, cudaStream_t st);

@@ -40,6 +40,12 @@ static int *status_ptr() {
 
 int *device_status_word() { return status_ptr(); }
 
+static thread_local cudaError_t t_last_cuda = cudaSuccess;
+muse_status cuda_fail(cudaError_t e) {
+  t_last_cuda = e;
+  return MUSE_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Workspace: a bump allocator over the caller's buffer (or a size count when
 // base == nullptr).  Every piece is 256-byte aligned.
@@ -206,7 +212,7 @@ static void plan_kmeans_pair(Bump &bp, const MuseTables &mt, const muse_dims &d,
 #define MUSE_TRY(expr)                                  \
   do {                                                  \
     cudaError_t e_ = (expr);                            \
-    if (e_ != cudaSuccess) return MUSE_ERR_CUDA;        \
+    if (e_ != cudaSuccess) return cuda_fail(e_);        \
   } while (0)
 
 // Inside a stream capture the event becomes an event-record node of the graph, so
@@ -307,8 +313,10 @@ extern "C" muse_status muse_set_test_hooks(unsigned hooks, uint64_t wait_limit_n
   int words[3];
   words[0] = (int)hooks;
   memcpy(&words[1], &wait_limit_ns, sizeof(uint64_t));
-  if (cudaMemcpyToSymbol(g_status_word, words, sizeof(words), sizeof(int)) != cudaSuccess)
-    return MUSE_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status_word, words, sizeof(words), sizeof(int)) != cudaSuccess) {
+    const cudaError_t e_ = cudaGetLastError();
+    return cuda_fail(e_ != cudaSuccess ? e_ : cudaErrorUnknown);
+  }
   if (cudaDeviceSynchronize() != cudaSuccess) return MUSE_ERR_CUDA;
   return MUSE_OK;
 }
@@ -424,8 +432,10 @@ extern "C" muse_status muse_kmeans(const void *X, muse_dims d, int C, int iters,
   SegTable t = whole_side(d.N, C);
   KmeansOut o{labels, centroids, perm, offsets};
   if (run_kmeans(X, d.dtype, d.D, d.N, t, d.B * d.H, iters, o, (char *)ws, status_ptr(),
-                 (cudaStream_t)st) != cudaSuccess)
-    return MUSE_ERR_CUDA;
+                 (cudaStream_t)st) != cudaSuccess) {
+    const cudaError_t e_ = cudaGetLastError();
+    return cuda_fail(e_ != cudaSuccess ? e_ : cudaErrorUnknown);
+  }
   return MUSE_OK;
 }
 
@@ -508,8 +518,10 @@ extern "C" muse_status muse_dipole_refine(const void *Q, const void *K, const vo
     // the summaries are given: the refinement reads them as they are
     if (run_refine_summaries(d.dtype, d.D, d.Dv, d.N, P, Cq, Ck, d.scale, Q, q_centroids, q_perm,
                              q_offsets, q_labels, logZ, mu_k, mu_v, cov, O, status_ptr(),
-                             (cudaStream_t)st) != cudaSuccess)
-      return MUSE_ERR_CUDA;
+                             (cudaStream_t)st) != cudaSuccess) {
+      const cudaError_t e_ = cudaGetLastError();
+      return cuda_fail(e_ != cudaSuccess ? e_ : cudaErrorUnknown);
+    }
     return MUSE_OK;
   }
   MuseTables mt;
@@ -554,8 +566,10 @@ extern "C" muse_status muse_forward_ex(const void *Q, const void *K, const void 
   cudaStream_t cs = (cudaStream_t)st;
   int *stat = status_ptr();
   if (run_kmeans_pair(Q, mt.q, kw.q, K, mt.k, kw.k, d.dtype, d.D, d.N, P, iters, kw.scratch, stat,
-                      cs) != cudaSuccess)
-    return MUSE_ERR_CUDA;
+                      cs) != cudaSuccess) {
+    const cudaError_t e_ = cudaGetLastError();
+    return cuda_fail(e_ != cudaSuccess ? e_ : cudaErrorUnknown);
+  }
   // the partially specialised dipole adds s Cbar_i qt to the monopole-only result
   muse_status s2 = refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets,
                                kw.k.perm, kw.k.offsets, nullptr, nullptr, r, O, nullptr, nullptr,
@@ -595,8 +609,10 @@ extern "C" muse_status muse_causal_blocks(const void *Q, const void *K, const vo
   if (levels == 0) {
     // one block: the diagonal is the whole causal attention
     if (run_diag_merge(Q, K, V, d.dtype, d.D, d.Dv, d.N, P, block, 0, d.scale, nullptr, nullptr,
-                       O, cs) != cudaSuccess)
-      return MUSE_ERR_CUDA;
+                       O, cs) != cudaSuccess) {
+      const cudaError_t e_ = cudaGetLastError();
+      return cuda_fail(e_ != cudaSuccess ? e_ : cudaErrorUnknown);
+    }
     return MUSE_OK;
   }
   MuseTables mt;
@@ -616,18 +632,24 @@ extern "C" muse_status muse_causal_blocks(const void *Q, const void *K, const vo
   if (k_labels_out) kw.k.labels = k_labels_out;
   // rows outside every square of a level keep label -1
   if (cudaMemsetAsync(kw.q.labels, 0xff, (size_t)P * L * d.N * sizeof(int32_t), cs) != cudaSuccess ||
-      cudaMemsetAsync(kw.k.labels, 0xff, (size_t)P * L * d.N * sizeof(int32_t), cs) != cudaSuccess)
-    return MUSE_ERR_CUDA;
+      cudaMemsetAsync(kw.k.labels, 0xff, (size_t)P * L * d.N * sizeof(int32_t), cs) != cudaSuccess) {
+    const cudaError_t e_ = cudaGetLastError();
+    return cuda_fail(e_ != cudaSuccess ? e_ : cudaErrorUnknown);
+  }
   int *stat = status_ptr();
   if (run_kmeans_pair(Q, mt.q, kw.q, K, mt.k, kw.k, d.dtype, d.D, d.N, P, iters, kw.scratch, stat,
-                      cs) != cudaSuccess)
-    return MUSE_ERR_CUDA;
+                      cs) != cudaSuccess) {
+    const cudaError_t e_ = cudaGetLastError();
+    return cuda_fail(e_ != cudaSuccess ? e_ : cudaErrorUnknown);
+  }
   s = refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets, kw.k.perm,
                   kw.k.offsets, nullptr, nullptr, r, nullptr, part_o, part_lse, cs);
   if (s != MUSE_OK) return s;
   if (run_diag_merge(Q, K, V, d.dtype, d.D, d.Dv, d.N, P, block, L, d.scale, part_o, part_lse, O,
-                     cs) != cudaSuccess)
-    return MUSE_ERR_CUDA;
+                     cs) != cudaSuccess) {
+    const cudaError_t e_ = cudaGetLastError();
+    return cuda_fail(e_ != cudaSuccess ? e_ : cudaErrorUnknown);
+  }
   return MUSE_OK;
 }
 
@@ -647,7 +669,13 @@ extern "C" muse_status muse_backward(const void *Q, const void *K, const void *V
   const size_t need = muse_backward_ws(d, Cq, Ck);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
   if (run_backward(Q, K, V, dO, q_perm, q_offsets, k_perm, k_offsets, d, Cq, Ck, dQ, dK, dV, ws,
-                   (cudaStream_t)st) != cudaSuccess)
-    return MUSE_ERR_CUDA;
+                   (cudaStream_t)st) != cudaSuccess) {
+    const cudaError_t e_ = cudaGetLastError();
+    return cuda_fail(e_ != cudaSuccess ? e_ : cudaErrorUnknown);
+  }
   return MUSE_OK;
+}
+
+extern "C" const char *muse_last_error_detail(void) {
+  return t_last_cuda == cudaSuccess ? "" : cudaGetErrorString(t_last_cuda);
 }

@@ -80,6 +80,7 @@ struct __align__(1024) Smem {
   alignas(16) unsigned short kblk[NST][BN];    // RET: key block of every column (cp.async)
   int kgrp[NST][BN / 8];                       // RET: min | max << 16 key block per 8 columns
   int wbhi[BM / 32];                           // RET: latest query block per row warp
+  int xblk[BM][17];                            // RET: each row's selected blocks (k1 k2 <= 16)
   int tnpad[4];                                // padded width of the tiles in flight (MMA issuer)
   // per stage: key tile (consumed by the first MMA), values (second MMA), epilogue
   // data (tilt weights, coefficients, segment map; consumed by the epilogue)
@@ -222,16 +223,39 @@ static __device__ __noinline__ uint32_t excl_bits(const Smem<D, DV> &sm, int st,
   return keep;
 }
 
+// RET: bit e set where the 16-bit block of column e (two per word, low half first) is
+// below `lim` (pair = lim in both halves).
+__device__ __forceinline__ uint32_t lt_bits16(const uint4 &a, const uint4 &b, uint32_t pair) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t c = __vcmpltu2(w[k], pair);  // 0xFFFF per half where below
+    m |= ((c & 1u) | ((c >> 15) & 2u)) << (2 * k);
+  }
+  return m;
+}
+// RET: bit e set where the block of column e equals `pair`'s.
+__device__ __forceinline__ uint32_t eq_bits16(const uint4 &a, const uint4 &b, uint32_t pair) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t c = __vcmpeq2(w[k], pair);
+    m |= ((c & 1u) | ((c >> 15) & 2u)) << (2 * k);
+  }
+  return m;
+}
+
 template <int D, int DV, bool RET>
-__global__ void __launch_bounds__(kThreads, 1)
-refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                 const __grid_constant__ CUtensorMap map_vt, MuseTables mt, int N,
-                 const int32_t *__restrict__ q_perm, const int32_t *__restrict__ q_cluster,
-                 const int32_t *__restrict__ k_offsets, const float *__restrict__ W,
-                 const float *__restrict__ c0g, const float *__restrict__ c1g,
-                 const float *__restrict__ lse, __nv_bfloat16 *__restrict__ O,
-                 float *__restrict__ part_o, float *__restrict__ part_lse, int *status,
-                 const __grid_constant__ BlockMap bm, const RetArgs ra) {
+__device__ __forceinline__ void
+refine_tc_body(const CUtensorMap &map_q, const CUtensorMap &map_k, const CUtensorMap &map_vt,
+               const MuseTables &mt, int N, const int32_t *__restrict__ q_perm,
+               const int32_t *__restrict__ q_cluster, const int32_t *__restrict__ k_offsets,
+               const float *__restrict__ W, const float *__restrict__ c0g,
+               const float *__restrict__ c1g, const float *__restrict__ lse,
+               __nv_bfloat16 *__restrict__ O, float *__restrict__ part_o,
+               float *__restrict__ part_lse, int *status, const BlockMap &bm, const RetArgs &ra) {
   constexpr int BN = TileCfg<D, DV>::BN;
   // blockIdx.x: a 128-row block of one instance (compact grid), blockIdx.y: the problem
   int bfirst;
@@ -535,9 +559,14 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
           for (int t1 = 0; t1 < kSelReg; ++t1)
             if (t1 < ra.k1) selc[t1] = so[2 * t1 * ra.k2];
+          if (ra.k1 <= kSelReg && ra.K12 <= 16 && grp == 0)
+            for (int e = 0; e < ra.K12; ++e) sm.xblk[r][e] = so[2 * e + 1];
         }
       }
     }
+    // the table is read by both groups' threads of the same row
+    if constexpr (RET) asm volatile("bar.sync 2, %0;" ::"r"(32 * kEpiWarps) : "memory");
+    const bool xfast = ra.k1 <= kSelReg && ra.K12 <= 16;  // selection held in registers/table
     TileIter<BN> it;
     it.begin(koff, k.C, kend);
     int t = 0;
@@ -557,11 +586,15 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const float *wsm = &sm.w[st][staged ? slot : 0][0];
       const int nch16 = kt.npad / 16;
       uint32_t xseg = 0;  // RET: tile segments holding a cluster the row selected
+      uint32_t tmap = 0xFFFFFFFFu;  // RET: 4 bits per tile segment: its selected slot (15: none)
       if constexpr (RET) {
 #pragma unroll
         for (int t1 = 0; t1 < kSelReg; ++t1) {
           const int d = selc[t1] - kt.j;
-          if (selc[t1] >= 0 && d >= 0 && d < kt.nseg) xseg |= 1u << d;
+          if (selc[t1] >= 0 && d >= 0 && d < kt.nseg) {
+            xseg |= 1u << d;
+            tmap = (tmap & ~(15u << (4 * d))) | ((uint32_t)t1 << (4 * d));
+          }
         }
         if (so && brow > 0)
           for (int t1 = kSelReg; t1 < ra.k1; ++t1) {
@@ -581,9 +614,36 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           // the chunk's block range, conservative: every key of its two 8-key groups
           const int ga = sm.kgrp[st][2 * cb], gb = sm.kgrp[st][2 * cb + 1];
           const int blo = min(ga & 0xFFFF, gb & 0xFFFF), bhi = max(ga >> 16, gb >> 16);
+          const bool straddle = blo < brow && bhi >= brow;
+          const bool xchunk = xseg != 0u && blo < brow;
           if (blo >= brow) keep = 0u;
-          else if (bhi >= brow) keep = causal_bits<D, DV>(sm, st, cb, brow);
-          if (xseg && keep) keep &= excl_bits<D, DV>(sm, st, cb, xseg, kt.j, so, ra.k1, ra.k2);
+          if (straddle || xchunk) {
+            const uint4 ka = *reinterpret_cast<const uint4 *>(&sm.kblk[st][cb * 16]);
+            const uint4 kb = *reinterpret_cast<const uint4 *>(&sm.kblk[st][cb * 16 + 8]);
+            if (straddle) keep = lt_bits16(ka, kb, (uint32_t)brow * 0x10001u);
+            if (xchunk) {
+              if (xfast && !(code & kComplex)) {
+                // the chunk's clusters: glo over columns [0, split), ghi over [split, 16)
+                const int glo = code & 15, ghi = (code >> 4) & 15, split = (code >> 8) & 31;
+                const uint32_t lomask = split >= 16 ? 0xFFFFu : ((1u << split) - 1u);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const int sg = h ? ghi : glo;
+                  if (h && ghi == glo) break;
+                  const uint32_t tt = (tmap >> (4 * sg)) & 15u;
+                  if (tt == 15u) continue;
+                  uint32_t ex = 0;
+                  for (int u = 0; u < ra.k2; ++u) {
+                    const int bb = sm.xblk[r][tt * ra.k2 + u];
+                    if (bb >= 0) ex |= eq_bits16(ka, kb, (uint32_t)bb * 0x10001u);
+                  }
+                  keep &= ~(ex & (h ? ~lomask & 0xFFFFu : lomask));
+                }
+              } else {
+                keep &= excl_bits<D, DV>(sm, st, cb, xseg, kt.j, so, ra.k1, ra.k2);
+              }
+            }
+          }
         }
         uint32_t pk[8];
         if (wfast && !(code & kComplex)) {
@@ -717,6 +777,21 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   }
 }
 
+// The refinement and its retrieval mode: one CTA per SM, 416 threads.
+template <int D, int DV, bool RET>
+__global__ void __launch_bounds__(kThreads, 1)
+refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                 const __grid_constant__ CUtensorMap map_vt, MuseTables mt, int N,
+                 const int32_t *__restrict__ q_perm, const int32_t *__restrict__ q_cluster,
+                 const int32_t *__restrict__ k_offsets, const float *__restrict__ W,
+                 const float *__restrict__ c0g, const float *__restrict__ c1g,
+                 const float *__restrict__ lse, __nv_bfloat16 *__restrict__ O,
+                 float *__restrict__ part_o, float *__restrict__ part_lse, int *status,
+                 const __grid_constant__ BlockMap bm, const RetArgs ra) {
+  refine_tc_body<D, DV, RET>(map_q, map_k, map_vt, mt, N, q_perm, q_cluster, k_offsets, W, c0g,
+                             c1g, lse, O, part_o, part_lse, status, bm, ra);
+}
+
 // ------------------------------------------------------------------ host side
 template <int D, int DV, bool RET>
 static cudaError_t launch(const MuseTables &mt, int N, int P, SortedSide qs, const int32_t *q_perm,
@@ -730,14 +805,17 @@ static cudaError_t launch(const MuseTables &mt, int N, int P, SortedSide qs, con
       !make_map(&mv, vt, ldv, (uint64_t)P * DV, ldv, DV))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem<D, DV>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(refine_tc_kernel<D, DV, RET>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = refine_tc_kernel<D, DV, RET>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+  if (fa.maxThreadsPerBlock < kThreads) return cudaErrorLaunchOutOfResources;
   const BlockMap bm = make_block_map(mt.q, BM);
   dim3 grid(bm.total, P);
-  refine_tc_kernel<D, DV, RET><<<grid, kThreads, smem, st>>>(
-      mq, mk, mv, mt, N, q_perm, qs.cluster, k_offsets, b.W, b.c0, b.c1, b.lse,
-      (__nv_bfloat16 *)O, part_o, part_lse, status, bm, ra);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mt, N, q_perm, qs.cluster, k_offsets, b.W, b.c0,
+                                     b.c1, b.lse, (__nv_bfloat16 *)O, part_o, part_lse, status, bm,
+                                     ra);
   count_launches(1);
   return cudaGetLastError();
 }

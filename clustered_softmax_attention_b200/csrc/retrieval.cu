@@ -671,7 +671,7 @@ ret_runs(Geo g, float scale, const __nv_bfloat16 *__restrict__ Q, const __nv_bfl
   constexpr int KC = (D + DV <= 128) ? 64 : 32;  // keys per chunk
   constexpr int NK = KC / 32, PV = DV / 32;
   __shared__ float Ks[KC][D + 1];
-  __shared__ float Vs[KC][DV];
+  __shared__ float Vs[KC][DV + 1];  // padded rows: a thread per key writes a row
   __shared__ float qsh[4][D];
   __shared__ float psh[4][KC];
   __shared__ int runs[64], cum[65];  // run start (sorted key position), keys before it
@@ -1100,5 +1100,5 @@ extern "C" muse_status muse_retrieve_exact(const void *Q, const void *K, const v
     else if (d.Dv == 64) e = ret::run_tc<128, 64>(Q, K, V, d, g, iters, w, O, status, cs);
     else e = ret::run_tc<128, 128>(Q, K, V, d, g, iters, w, O, status, cs);
   }
-  return e == cudaSuccess ? MUSE_OK : MUSE_ERR_CUDA;
+  return e == cudaSuccess ? MUSE_OK : cuda_fail(e);
 }

@@ -54,13 +54,14 @@ _SIGS = {
                             _vp, _sz, _vp],
     "muse_workspace_size": [ctypes.c_char_p, MuseDims, _i, _i, _i, _i, _i],
     "muse_status_string": [_i],
+    "muse_last_error_detail": [],
     "muse_last_device_status": [_vp],
     "muse_set_test_hooks": [ctypes.c_uint, ctypes.c_uint64],
     "muse_backward": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, MuseDims, _i, _i, _vp, _vp, _vp,
                       _vp, _sz, _vp],
 }
 _RES = {"muse_workspace_size": _sz, "muse_status_string": ctypes.c_char_p,
-        "muse_causal_levels": _i}
+        "muse_causal_levels": _i, "muse_last_error_detail": ctypes.c_char_p}
 
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
@@ -94,7 +95,8 @@ def declared_entry_points(header: str = HEADER):
 
 def _check(code: int, where: str):
     if code != 0:
-        raise MuseError(code, where)
+        detail = lib().muse_last_error_detail().decode() if code == 5 else ""
+        raise MuseError(code, where + (f" ({detail})" if detail else ""))
 
 
 def _p(t: Optional[torch.Tensor]):

@@ -288,6 +288,13 @@ size_t muse_workspace_size(const char *entry, muse_dims d, int Cq, int Ck, int b
 const char *muse_status_string(muse_status s);
 
 /*
+ * muse_last_error_detail - the CUDA runtime's description of the error behind the
+ * calling thread's most recent MUSE_ERR_CUDA ("" if none); valid until the next call
+ * into the library on this thread.
+ */
+const char *muse_last_error_detail(void);
+
+/*
  * muse_last_device_status - synchronises `st`, returns and clears the device status
  * word of the current device (MUSE_OK, MUSE_ERR_TIMEOUT or MUSE_ERR_DEVICE), or
  * MUSE_ERR_CUDA if the synchronisation itself failed.  The word is shared by every
