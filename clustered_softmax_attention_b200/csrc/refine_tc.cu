@@ -247,6 +247,30 @@ __device__ __forceinline__ uint32_t eq_bits16(const uint4 &a, const uint4 &b, ui
   return m;
 }
 
+// RET: columns of a chunk (at most two key clusters: glo over columns [0, split), ghi over
+// [split, 16)) that are not in a block the row selected for their cluster; xb: the row's
+// selected blocks, slot t * k2 + u; tmap: 4 bits per tile segment, its slot (15: none).
+// Out of line: only chunks of a selected cluster come here.
+static __device__ __noinline__ uint32_t excl_fast(uint4 ka, uint4 kb, int code, uint32_t tmap,
+                                                  const int *xb, int k2) {
+  const int glo = code & 15, ghi = (code >> 4) & 15, split = (code >> 8) & 31;
+  const uint32_t lomask = split >= 16 ? 0xFFFFu : ((1u << split) - 1u);
+  uint32_t keep = 0xFFFFu;
+  for (int h = 0; h < 2; ++h) {
+    const int sg = h ? ghi : glo;
+    if (h && ghi == glo) break;
+    const uint32_t tt = (tmap >> (4 * sg)) & 15u;
+    if (tt == 15u) continue;
+    uint32_t ex = 0;
+    for (int u = 0; u < k2; ++u) {
+      const int bb = xb[tt * k2 + u];
+      if (bb >= 0) ex |= eq_bits16(ka, kb, (uint32_t)bb * 0x10001u);
+    }
+    keep &= ~(ex & (h ? ~lomask & 0xFFFFu : lomask));
+  }
+  return keep;
+}
+
 template <int D, int DV, bool RET>
 __device__ __forceinline__ void
 refine_tc_body(const CUtensorMap &map_q, const CUtensorMap &map_k, const CUtensorMap &map_vt,
@@ -622,26 +646,10 @@ refine_tc_body(const CUtensorMap &map_q, const CUtensorMap &map_k, const CUtenso
             const uint4 kb = *reinterpret_cast<const uint4 *>(&sm.kblk[st][cb * 16 + 8]);
             if (straddle) keep = lt_bits16(ka, kb, (uint32_t)brow * 0x10001u);
             if (xchunk) {
-              if (xfast && !(code & kComplex)) {
-                // the chunk's clusters: glo over columns [0, split), ghi over [split, 16)
-                const int glo = code & 15, ghi = (code >> 4) & 15, split = (code >> 8) & 31;
-                const uint32_t lomask = split >= 16 ? 0xFFFFu : ((1u << split) - 1u);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                  const int sg = h ? ghi : glo;
-                  if (h && ghi == glo) break;
-                  const uint32_t tt = (tmap >> (4 * sg)) & 15u;
-                  if (tt == 15u) continue;
-                  uint32_t ex = 0;
-                  for (int u = 0; u < ra.k2; ++u) {
-                    const int bb = sm.xblk[r][tt * ra.k2 + u];
-                    if (bb >= 0) ex |= eq_bits16(ka, kb, (uint32_t)bb * 0x10001u);
-                  }
-                  keep &= ~(ex & (h ? ~lomask & 0xFFFFu : lomask));
-                }
-              } else {
+              if (xfast && !(code & kComplex))
+                keep &= excl_fast(ka, kb, code, tmap, sm.xblk[r], ra.k2);
+              else
                 keep &= excl_bits<D, DV>(sm, st, cb, xseg, kt.j, so, ra.k1, ra.k2);
-              }
             }
           }
         }

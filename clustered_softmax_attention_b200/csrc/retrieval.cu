@@ -473,9 +473,9 @@ exact_merge(Geo g, float scale, const T *__restrict__ Q, const T *__restrict__ K
 // row r (cluster i, block b): the keys of j in blocks b' < b minus the runs selected for
 // (i, b).  A running sum m1_j = sum_{b' < b} sum_{k in (j, b')} W_ik k over the key blocks
 // gives qt_r.m1_j; a selected cluster's runs are summed once per (i, b) group into e_j
-// and qt_r.e_j is subtracted (float32).  One CTA per (problem, query cluster i, group of
-// JPC key clusters); DP = D / 32 threads per cluster, 32 coordinates each; the group's
-// residual rows are staged in shared memory once per block.
+// and qt_r.(m1_j - e_j) is taken (float32).  One CTA per (problem, query cluster i, group
+// of JPC key clusters); DP = D / 32 threads per cluster, 32 coordinates each; no
+// block-wide barrier (a thread's work varies with its cluster's keys per block).
 template <int D>
 __global__ void __launch_bounds__(256)
 ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q_offsets,
@@ -483,9 +483,7 @@ ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q
       const int32_t *__restrict__ k_offsets, const int32_t *__restrict__ pend,
       const float *__restrict__ W, int w_stride, const int32_t *__restrict__ sel,
       float *__restrict__ Tout) {
-  constexpr int DP = D / 32, JPC = 256 / DP, RMAX = 2048 / D;
-  __shared__ float qsh[RMAX][D];
-  __shared__ float exsh[JPC][D + 1];
+  constexpr int DP = D / 32, JPC = 256 / DP;
   const int p = blockIdx.z, i = blockIdx.y;
   const int jl = threadIdx.x / DP, dp = threadIdx.x % DP;
   const int j = blockIdx.x * JPC + jl;
@@ -540,47 +538,40 @@ ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q
     if (b > 0 && live)
       for (int t = 0; t < g.k1; ++t)
         if (so[2 * t * g.k2] == j) tj = t;
-    if (tj >= 0) {
-      float ex[32];
+    float ex[32];
 #pragma unroll
-      for (int d = 0; d < 32; ++d) ex[d] = 0.f;
+    for (int d = 0; d < 32; ++d) ex[d] = 0.f;
+    if (tj >= 0) {
       for (int u = 0; u < g.k2; ++u) {
         const int bb = so[2 * (tj * g.k2 + u) + 1];
         if (bb < 0) continue;
         for (int pos = kbase + pe[bb]; pos < kbase + pe[bb + 1]; ++pos) add_key(pos, wrow[pos], ex);
       }
-#pragma unroll
-      for (int d = 0; d < 32; ++d) exsh[jl][dp * 32 + d] = ex[d];
     }
-    for (int rb = r0; rb < r1; rb += RMAX) {
-      const int nr = min(RMAX, r1 - rb);
-      __syncthreads();  // the previous rows are read
-      for (int e = threadIdx.x; e < nr * (D / 8); e += blockDim.x) {
-        const int rr = e / (D / 8), v = e % (D / 8);
-        const uint4 u = reinterpret_cast<const uint4 *>(qp + (int64_t)(rb + rr) * D)[v];
-        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+    // every row of the group: qt.(m1 - e), the thread's 32 coordinates read straight from
+    // the sorted residuals (the same addresses for every thread of a half: L1 broadcast)
+    for (int r = r0; r < r1; ++r) {
+      float acc = 0.f;
+      if (b > 0) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(qp + (int64_t)r * D + dp * 32);
+        uint4 u[4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
-          qsh[rr][8 * v + 2 * h] = __low2float(b2);
-          qsh[rr][8 * v + 2 * h + 1] = __high2float(b2);
-        }
-      }
-      __syncthreads();
-      for (int rr = 0; rr < nr; ++rr) {
-        float acc = 0.f;
-        if (b > 0) {
+        for (int v = 0; v < 4; ++v) u[v] = src[v];
 #pragma unroll
-          for (int d = 0; d < 32; ++d) acc = fmaf(qsh[rr][dp * 32 + d], m1[d], acc);
-          if (tj >= 0) {
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t w4[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
 #pragma unroll
-            for (int d = 0; d < 32; ++d) acc = fmaf(-qsh[rr][dp * 32 + d], exsh[jl][dp * 32 + d], acc);
+          for (int h = 0; h < 4; ++h) {
+            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
+            const int d = 8 * v + 2 * h;
+            acc = fmaf(__low2float(b2), m1[d] - ex[d], acc);
+            acc = fmaf(__high2float(b2), m1[d + 1] - ex[d + 1], acc);
           }
         }
-#pragma unroll
-        for (int o = DP / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (live && dp == 0) tout[rb + rr] = acc;
       }
+#pragma unroll
+      for (int o = DP / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (live && dp == 0) tout[r] = acc;
     }
   }
 }
@@ -657,163 +648,131 @@ ret_coeffs(Geo g, float scale, const int32_t *__restrict__ q_perm,
 // Exact attention over the (cluster, block) runs selected for (query cluster i, query
 // block b), merged into the remainder partial of every row of the group (token order):
 // part_lse[p][n], part_o[p][n][:] become the joint (log-normaliser, normalised output) of
-// the remainder and the runs.  One CTA of four warps per (problem, i, b); the runs' keys
-// and values go through shared memory KC at a time; a warp takes one query row at a time
-// (lanes over keys for the logits, over output columns for the sums).
+// the remainder and the runs.  One warp per (problem, i, b) group, no block-wide
+// barrier: the warp lists the runs (lanes over the slots, a shuffle scan of their
+// lengths), then for every row of the group walks the runs' keys 32 at a time -- lane k
+// forms the logit of key k against the row's query (held in shared memory), the warp
+// updates the online softmax, and lanes over output columns accumulate p_k v_k (value
+// rows read whole by the warp).
 template <int D, int DV>
-__global__ void __launch_bounds__(128)
-ret_runs(Geo g, float scale, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
+__global__ void __launch_bounds__(256)
+ret_runs(Geo g, int P, float scale, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
          const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ q_perm,
          const int32_t *__restrict__ q_offsets, const int32_t *__restrict__ qpend,
          const int32_t *__restrict__ k_perm, const int32_t *__restrict__ k_offsets,
          const int32_t *__restrict__ pend, const int32_t *__restrict__ sel,
          float *__restrict__ part_o, float *__restrict__ part_lse) {
-  constexpr int KC = (D + DV <= 128) ? 64 : 32;  // keys per chunk
-  constexpr int NK = KC / 32, PV = DV / 32;
-  __shared__ float Ks[KC][D + 1];
-  __shared__ float Vs[KC][DV + 1];  // padded rows: a thread per key writes a row
-  __shared__ float qsh[4][D];
-  __shared__ float psh[4][KC];
-  __shared__ int runs[64], cum[65];  // run start (sorted key position), keys before it
-  __shared__ int nruns;
-  const int p = blockIdx.z, i = blockIdx.y, b = blockIdx.x;
-  if (b == 0) return;
+  constexpr int PV = DV / 32;
+  __shared__ float qsh[8][D];
+  __shared__ int runs[8][64], cum[8][65];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gid = (int64_t)blockIdx.x * 8 + warp;  // (p, i, b)
+  if (gid >= (int64_t)g.nb * g.Cq * P) return;  // whole warps
+  const int b = (int)(gid % g.nb), i = (int)((gid / g.nb) % g.Cq), p = (int)(gid / ((int64_t)g.nb * g.Cq));
+  if (b == 0) return;
   const int32_t *qo = q_offsets + (int64_t)p * (g.Cq + 1);
   const int32_t *qpe = qpend + ((int64_t)p * g.Cq + i) * (g.nb + 1);
   const int r0 = qo[i] + qpe[b], r1 = qo[i] + qpe[b + 1];
-  if (r0 >= r1) return;  // uniform
-  // the selected runs: slot t (a warp pair reads the K12 <= 64 slots at once), then an
-  // inclusive scan of their lengths by warp 0
-  __shared__ int len[64];
-  if (threadIdx.x < 64) {
-    const int t = threadIdx.x;
-    int start = 0, n = 0;
+  if (r0 >= r1) return;
+  // the selected runs: slots lane and lane + 32
+  const int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
+  int start[2], len[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int t = lane + 32 * h;
+    start[h] = 0;
+    len[h] = 0;
     if (t < g.K12) {
-      const int32_t *so = sel + (((int64_t)p * g.Cq + i) * g.nb + b) * g.K12 * 2;
       const int j = so[2 * t], bb = so[2 * t + 1];
       if (j >= 0) {
         const int32_t *pe = pend + ((int64_t)p * g.Ck + j) * (g.nb + 1);
-        start = k_offsets[(int64_t)p * (g.Ck + 1) + j] + pe[bb];
-        n = pe[bb + 1] - pe[bb];
+        start[h] = k_offsets[(int64_t)p * (g.Ck + 1) + j] + pe[bb];
+        len[h] = pe[bb + 1] - pe[bb];
       }
     }
-    runs[t] = start;
-    len[t] = n;
   }
-  __syncthreads();
-  if (warp == 0) {
-    int a = len[2 * lane], c = len[2 * lane + 1];
-    int inc = a + c;
+  // exclusive scan over the 64 slots (lane-major halves: slots 0..31, then 32..63)
+  int inc0 = len[0], inc1 = len[1];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
-    }
-    const int excl = inc - a - c;
-    cum[2 * lane] = excl;
-    cum[2 * lane + 1] = excl + a;
-    if (lane == 31) {
-      cum[64] = inc;
-      nruns = 64;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y0 = __shfl_up_sync(0xffffffffu, inc0, o), y1 = __shfl_up_sync(0xffffffffu, inc1, o);
+    if (lane >= o) {
+      inc0 += y0;
+      inc1 += y1;
     }
   }
-  __syncthreads();
-  const int total = cum[nruns];
-  if (total == 0) return;  // uniform
+  const int tot0 = __shfl_sync(0xffffffffu, inc0, 31);
+  runs[warp][lane] = start[0];
+  runs[warp][lane + 32] = start[1];
+  cum[warp][lane] = inc0 - len[0];
+  cum[warp][lane + 32] = tot0 + inc1 - len[1];
+  if (lane == 31) cum[warp][64] = tot0 + inc1;
+  __syncwarp();
+  const int total = cum[warp][64];
+  if (total == 0) return;
   const int32_t *kperm = k_perm + (int64_t)p * g.N;
-  for (int rb = r0; rb < r1; rb += 4) {
-    const int r = rb + warp;
-    const bool rv = r < r1;
-    const int n = rv ? q_perm[(int64_t)p * g.N + r] : 0;
-    if (rv)
-      for (int d = lane; d < D; d += 32)
-        qsh[warp][d] = __bfloat162float(Q[((int64_t)p * g.N + n) * D + d]) * scale;
+  for (int r = r0; r < r1; ++r) {
+    const int n = q_perm[(int64_t)p * g.N + r];
+    __syncwarp();
+    for (int d = lane; d < D; d += 32) qsh[warp][d] = __bfloat162float(Q[((int64_t)p * g.N + n) * D + d]) * scale;
+    __syncwarp();
     float m = -CUDART_INF_F, l = 0.f, o[PV];
 #pragma unroll
     for (int v = 0; v < PV; ++v) o[v] = 0.f;
-    for (int c0 = 0; c0 < total; c0 += KC) {
-      const int cnt = min(KC, total - c0);
-      __syncthreads();
-      if (threadIdx.x < cnt) {
-        const int gi = c0 + threadIdx.x;
-        int rr = 0;
-        while (cum[rr + 1] <= gi) ++rr;
-        const int tok = kperm[runs[rr] + gi - cum[rr]];
+    int rr = 0;  // run of this lane's key (the lane's keys only move forward)
+    for (int c0 = 0; c0 < total; c0 += 32) {
+      const int gi = c0 + lane;
+      int tok = 0;
+      float x = -CUDART_INF_F;
+      if (gi < total) {
+        while (cum[warp][rr + 1] <= gi) ++rr;
+        tok = kperm[runs[warp][rr] + gi - cum[warp][rr]];
         const uint4 *kr = reinterpret_cast<const uint4 *>(K + ((int64_t)p * g.N + tok) * D);
-        const uint4 *vr = reinterpret_cast<const uint4 *>(V + ((int64_t)p * g.N + tok) * DV);
+        float a = 0.f;
+#pragma unroll
         for (int u = 0; u < D / 8; ++u) {
-          const uint4 x = kr[u];
-          const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+          const uint4 w4 = kr[u];
+          const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
           for (int h = 0; h < 4; ++h) {
-            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
-            Ks[threadIdx.x][8 * u + 2 * h] = __low2float(b2);
-            Ks[threadIdx.x][8 * u + 2 * h + 1] = __high2float(b2);
+            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&ww[h]);
+            a = fmaf(qsh[warp][8 * u + 2 * h], __low2float(b2), a);
+            a = fmaf(qsh[warp][8 * u + 2 * h + 1], __high2float(b2), a);
           }
         }
-        for (int u = 0; u < DV / 8; ++u) {
-          const uint4 x = vr[u];
-          const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
-          for (int h = 0; h < 4; ++h) {
-            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
-            Vs[threadIdx.x][8 * u + 2 * h] = __low2float(b2);
-            Vs[threadIdx.x][8 * u + 2 * h + 1] = __high2float(b2);
-          }
-        }
+        x = a;
       }
-      __syncthreads();
-      if (rv) {
-        float x[NK];
-        float cm = -CUDART_INF_F;
+      const float mn = fmaxf(m, warp_max(x));
+      const float corr = expf(m - mn);
+      const float pk = gi < total ? expf(x - mn) : 0.f;
+      l = l * corr + warp_sum(pk);
 #pragma unroll
-        for (int h = 0; h < NK; ++h) {
-          const int kk = lane + 32 * h;
-          x[h] = -CUDART_INF_F;
-          if (kk < cnt) {
-            float a = 0.f;
-            for (int d = 0; d < D; ++d) a = fmaf(qsh[warp][d], Ks[kk][d], a);
-            x[h] = a;
-          }
-          cm = fmaxf(cm, x[h]);
-        }
-        const float mn = fmaxf(m, warp_max(cm));
-        const float corr = expf(m - mn);
-        float ps = 0.f;
+      for (int v = 0; v < PV; ++v) o[v] *= corr;
+      const int cnt = min(32, total - c0);
+      for (int k = 0; k < cnt; ++k) {
+        const float pkk = __shfl_sync(0xffffffffu, pk, k);
+        const int tk = __shfl_sync(0xffffffffu, tok, k);
+        const __nv_bfloat16 *vr = V + ((int64_t)p * g.N + tk) * DV;
 #pragma unroll
-        for (int h = 0; h < NK; ++h) {
-          const float pe = lane + 32 * h < cnt ? expf(x[h] - mn) : 0.f;
-          psh[warp][lane + 32 * h] = pe;
-          ps += pe;
-        }
-        l = l * corr + warp_sum(ps);
-        __syncwarp();
-#pragma unroll
-        for (int v = 0; v < PV; ++v) {
-          float acc = o[v] * corr;
-          for (int k = 0; k < cnt; ++k) acc = fmaf(psh[warp][k], Vs[k][lane + 32 * v], acc);
-          o[v] = acc;
-        }
-        m = mn;
-        __syncwarp();
+        for (int v = 0; v < PV; ++v) o[v] = fmaf(pkk, __bfloat162float(vr[lane + 32 * v]), o[v]);
       }
+      m = mn;
     }
-    if (rv) {
-      // joint softmax with the remainder partial of the row
-      const int64_t at = (int64_t)p * g.N + n;
-      const float L = part_lse[at];
-      float *po = part_o + at * DV;
-      const bool has = L > -CUDART_INF_F;
-      const float mn = has ? fmaxf(m, L) : m;
-      const float ca = expf(m - mn), cb = has ? expf(L - mn) : 0.f;
-      const float lt = l * ca + cb;
+    // joint softmax with the remainder partial of the row
+    const int64_t at = (int64_t)p * g.N + n;
+    const float L = part_lse[at];
+    float *po = part_o + at * DV;
+    const bool has = L > -CUDART_INF_F;
+    const float mn = has ? fmaxf(m, L) : m;
+    const float ca = expf(m - mn), cb = has ? expf(L - mn) : 0.f;
+    const float lt = l * ca + cb;
 #pragma unroll
-      for (int v = 0; v < PV; ++v) {
-        const float prev = has ? po[lane + 32 * v] : 0.f;
-        po[lane + 32 * v] = (o[v] * ca + cb * prev) / lt;
-      }
-      __syncwarp();
-      if (lane == 0) part_lse[at] = mn + logf(lt);
+    for (int v = 0; v < PV; ++v) {
+      const float prev = has ? po[lane + 32 * v] : 0.f;
+      po[lane + 32 * v] = (o[v] * ca + cb * prev) / lt;
     }
+    __syncwarp();
+    if (lane == 0) part_lse[at] = mn + logf(lt);
   }
 }
 
@@ -984,8 +943,8 @@ static cudaError_t run_tc(const void *Q, const void *K, const void *V, const mus
                              status, st)) != cudaSuccess)
     return e;
   if ((e = profile_mark(false, st)) != cudaSuccess) return e;
-  ret_runs<D, DV><<<dim3(g.nb, g.Cq, P), 128, 0, st>>>(
-      g, d.scale, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V,
+  ret_runs<D, DV><<<(unsigned)(((int64_t)g.nb * g.Cq * P + 7) / 8), 256, 0, st>>>(
+      g, P, d.scale, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V,
       w.q.perm, w.q.offsets, w.qpend, w.k.perm, w.k.offsets, w.pend, w.sel, w.part_o, w.part_lse);
   count_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
