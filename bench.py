@@ -183,6 +183,20 @@ def algorithmic_flops(w):
     raise ValueError(w.mode)
 
 
+def summary_form_ablation(w):
+    """Whether the library evaluates the monopole / partial-dipole ablations of this
+    workload in summary form (bfloat16, Dv = 64, D = 64 or 128, Ck <= 128)."""
+    return w.dtype == "bf16" and w.Dv == 64 and w.D in (64, 128) and w.Ck <= 128
+
+
+def summary_output_flops(w, partial):
+    """Flops of the summary-form output kernel per launch (tensor cores): 2 N Ck D for the
+    projections u, 2 N Ck Dv for sum_j p_j mu_v,ij, plus 2 N D Dv for s Cbar_i qt with
+    the partial dipole."""
+    per = 2.0 * w.N * w.Ck * (w.D + w.Dv) + (2.0 * w.N * w.D * w.Dv if partial else 0.0)
+    return w.B * w.H * per
+
+
 def retrieval_flops(w):
     """Algorithmic flops of one retrieval step (all problems): K-means of queries and keys,
     the tilted summaries and the refinement over the whole causal prefix counted as in
@@ -511,17 +525,26 @@ def measure(args, w, steps, warmup, world, rank, local_rank, cpu_baseline):
     # retrieval mode, the remainder), timed live above
     peaks, peak_src = load_peaks()
     kmean = sum(kern_ms) / len(kern_ms)
-    flops = algorithmic_flops(w)
-    achieved = flops / (kmean / 1e3) / 1e12
-    if w.dtype == "bf16":
+    summary_form = (monopole or partial) and summary_form_ablation(w)
+    if summary_form:
+        # the ablations in summary form: the output kernel's products (u = qt . mu_k,
+        # sum_j p_j mu_v,ij, plus s Cbar_i qt for the partial dipole) on the tensor cores
+        flops = summary_output_flops(w, partial)
         peak, bound, unit = float(peaks["bf16_tflops"]), "tensor", "TFLOP/s"
+        kname = "summary-form output (monopole" + (" + covariance)" if partial else ")")
     else:
-        peak, bound, unit = FP32_SIMT_TFLOPS, "alu", "TFLOP/s"
+        flops = algorithmic_flops(w)
+        if w.dtype == "bf16":
+            peak, bound, unit = float(peaks["bf16_tflops"]), "tensor", "TFLOP/s"
+        else:
+            peak, bound, unit = FP32_SIMT_TFLOPS, "alu", "TFLOP/s"
+        kname = "refinement (retrieval remainder)" if w.mode == "retrieval" else "refinement"
+    achieved = flops / (kmean / 1e3) / 1e12
     roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": recorded_traffic(w.name),
-            "kernel": "refinement (retrieval remainder)" if w.mode == "retrieval"
-            else "refinement", "kernel_ms": kmean, "flops_per_launch": flops,
-            "peak_source": f"{peak_src} bf16_tflops (burst)" if w.dtype == "bf16"
+            "frac": achieved / peak,
+            "traffic": None if summary_form else recorded_traffic(w.name),
+            "kernel": kname, "kernel_ms": kmean, "flops_per_launch": flops,
+            "peak_source": f"{peak_src} bf16_tflops (burst)" if bound == "tensor"
             else "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
     if w.mode == "retrieval":
         roof["step_flops"] = retrieval_flops(w)

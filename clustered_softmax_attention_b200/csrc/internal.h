@@ -92,13 +92,36 @@ cudaError_t run_summaries(const MuseTables &mt, int dtype, int D, int Dv, int P,
 cudaError_t run_tilt_weights(const MuseTables &mt, int dtype, int D, int P, float scale,
                              const float *q_centroids, SortedSide ks, const float *logZ, float *W,
                              cudaStream_t st);
+// mu_v[i][j] = sum_{k in S_j} w_ik v_k from the tilt weights W and the cluster-sorted
+// values (row-major).
+cudaError_t run_tilt_values(const MuseTables &mt, int dtype, int Dv, int P, const int32_t *k_offsets,
+                            const float *W, const void *vs_rows, float *mu_v, cudaStream_t st);
 // Partially specialised dipole (acausal tables): Cov_j per key cluster, Cbar_i per query
-// cluster, O += s Cbar_i qt.  ws holds P (Cq + Ck) D Dv floats.
+// cluster, O += s Cbar_i qt.  ws holds P (Cq + Ck) D Dv floats; with O == nullptr only
+// Cov_j and Cbar_i ([P][Cq][Dv][D], at partial_dipole_cbar(ws, ...)) are computed.
 size_t partial_dipole_ws_floats(int P, int Cq, int Ck, int D, int Dv);
+float *partial_dipole_cbar(float *ws, int P, int maxCk, int D, int Dv);
 cudaError_t run_partial_dipole(const MuseTables &mt, int dtype, int D, int Dv, int N, int P,
                                float scale, SortedSide qs, const int32_t *q_perm, SortedSide ks,
                                const void *V, const int32_t *k_perm, const int32_t *k_offsets,
                                const float *logZ, float *ws, void *O, cudaStream_t st);
+// Instances a kernel leaves to another one (bit s: instance s).
+struct InstMask {
+  uint32_t w[kMaxSeg / 32];
+};
+// The coefficients on the tensor cores (coef_tc.cu): bfloat16, D = 64 or 128, Ck <= 256;
+// the instances in `skip` are left out.
+bool coef_tc_supported(int dtype, int D, int maxCk);
+cudaError_t run_coef_tc(const MuseTables &mt, int D, int P, float scale, const void *qs_rows,
+                        const int32_t *q_offsets, const StageBufs &b, const InstMask &skip,
+                        float sdip, int *status, cudaStream_t st);
+// The monopole-only method (cbar == nullptr) and the partially specialised dipole in
+// summary form (coef_tc.cu): O_n = sum_j p_j mu_v,ij (+ s Cbar_i qt_n) with b.mu_v given;
+// bfloat16, D = Dv, no O(N^2) contraction.
+bool coef_out_supported(int dtype, int D, int Dv, int maxCk);
+cudaError_t run_coef_out(const MuseTables &mt, int D, int N, int P, float scale, const void *qs_rows,
+                         const int32_t *q_perm, const int32_t *q_offsets, const StageBufs &b,
+                         const float *cbar, void *O, int *status, cudaStream_t st);
 // sdip: the factor of the dipole terms (the logit scale, or 0 for the monopole only).
 cudaError_t run_coeffs(const MuseTables &mt, int dtype, int D, int P, float scale,
                        SortedSide qs, const int32_t *q_offsets, StageBufs b, float sdip,

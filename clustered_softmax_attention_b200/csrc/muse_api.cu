@@ -363,6 +363,11 @@ static size_t ws_partial_dipole(const muse_dims &d, int Cq, int Ck) {
   return partial_dipole_ws_floats(d.B * d.H, Cq, Ck, d.D, d.Dv) * sizeof(float) + 256;
 }
 
+// the tilted value means of the summary-form ablations (after the forward pass's buffers)
+static size_t ws_value_means(const muse_dims &d, int Cq, int Ck) {
+  return (size_t)d.B * d.H * Cq * Ck * d.Dv * sizeof(float) + 256;
+}
+
 static size_t ws_forward(const muse_dims &d, int Cq, int Ck) {
   MuseTables mt;
   mt.q = whole_side(d.N, Cq);
@@ -403,7 +408,9 @@ extern "C" size_t muse_workspace_size(const char *entry, muse_dims d, int Cq, in
   if (!strcmp(entry, "muse_dipole_refine")) return valid_C(Ck, d.N) ? ws_refine(d, Cq, Ck) : 0;
   if (!strcmp(entry, "muse_forward")) return valid_C(Ck, d.N) ? ws_forward(d, Cq, Ck) : 0;
   if (!strcmp(entry, "muse_forward_ex"))
-    return valid_C(Ck, d.N) ? ws_forward(d, Cq, Ck) + ws_partial_dipole(d, Cq, Ck) : 0;
+    return valid_C(Ck, d.N)
+               ? ws_forward(d, Cq, Ck) + ws_partial_dipole(d, Cq, Ck) + ws_value_means(d, Cq, Ck)
+               : 0;
   if (!strcmp(entry, "muse_causal_blocks")) {
     if (block <= 0 || block % 64 || d.N % block || Cq < 1 || Ck < 1 || Cq > kMaxClusters ||
         Ck > kMaxClusters)
@@ -550,7 +557,10 @@ extern "C" muse_status muse_forward_ex(const void *Q, const void *K, const void 
     if (!p || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
   if (!valid_C(Cq, d.N) || !valid_C(Ck, d.N) || iters < 1 || iters > 1000)
     return MUSE_ERR_INVALID_ARG;
-  const size_t need = ws_forward(d, Cq, Ck) + (partial ? ws_partial_dipole(d, Cq, Ck) : 0);
+  // the ablations in summary form (no O(N^2) contraction) where the output kernel fits
+  const bool summary = flags != 0 && coef_out_supported(d.dtype, d.D, d.Dv, Ck);
+  const size_t need = ws_forward(d, Cq, Ck) + (partial ? ws_partial_dipole(d, Cq, Ck) : 0) +
+                      (summary ? ws_value_means(d, Cq, Ck) : 0);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
   const int P = d.B * d.H;
   MuseTables mt;
@@ -563,12 +573,39 @@ extern "C" muse_status muse_forward_ex(const void *Q, const void *K, const void 
   RefineWs r;
   plan_refine(bp, mt, d, P, r, true);
   float *pd_ws = partial ? bp.take<float>(partial_dipole_ws_floats(P, Cq, Ck, d.D, d.Dv)) : nullptr;
+  float *mu_v = summary ? bp.take<float>((size_t)P * mt.in.z_stride * d.Dv) : nullptr;
   cudaStream_t cs = (cudaStream_t)st;
   int *stat = status_ptr();
   if (run_kmeans_pair(Q, mt.q, kw.q, K, mt.k, kw.k, d.dtype, d.D, d.N, P, iters, kw.scratch, stat,
                       cs) != cudaSuccess) {
     const cudaError_t e_ = cudaGetLastError();
     return cuda_fail(e_ != cudaSuccess ? e_ : cudaErrorUnknown);
+  }
+  if (summary) {
+    // O_n = sum_j p_j mu_v,ij (+ s Cbar_i qt_n) from the summaries: sorted copies (values
+    // row-major), tilt weights / logZ / mu_k, the tilted value means, the aggregated
+    // covariances for the partial dipole, then one output kernel
+    MUSE_TRY(run_sort_side(Q, d.dtype, d.D, d.N, mt.q, P, kw.q.perm, kw.q.offsets, kw.q.centroids,
+                           r.qs, cs));
+    MUSE_TRY(run_sort_side(K, d.dtype, d.D, d.N, mt.k, P, kw.k.perm, kw.k.offsets, nullptr, r.ks, cs));
+    SortedSide vsd{r.vs, r.v_cluster};
+    MUSE_TRY(run_sort_side(V, d.dtype, d.Dv, d.N, mt.k, P, kw.k.perm, kw.k.offsets, nullptr, vsd, cs));
+    StageBufs sb = r.sb;
+    MUSE_TRY(run_summaries(mt, d.dtype, d.D, d.Dv, P, d.scale, kw.q.centroids, r.ks, nullptr,
+                           kw.k.offsets, sb, cs));
+    MUSE_TRY(run_tilt_values(mt, d.dtype, d.Dv, P, kw.k.offsets, sb.W, r.vs, mu_v, cs));
+    sb.mu_v = mu_v;
+    const float *cbar = nullptr;
+    if (partial) {
+      MUSE_TRY(run_partial_dipole(mt, d.dtype, d.D, d.Dv, d.N, P, d.scale, r.qs, kw.q.perm, r.ks, V,
+                                  kw.k.perm, kw.k.offsets, sb.logZ, pd_ws, nullptr, cs));
+      cbar = partial_dipole_cbar(pd_ws, P, mt.k.max_C, d.D, d.Dv);
+    }
+    MUSE_TRY(profile_mark(true, cs));
+    MUSE_TRY(run_coef_out(mt, d.D, d.N, P, d.scale, r.qs.rows, kw.q.perm, kw.q.offsets, sb, cbar, O,
+                          stat, cs));
+    MUSE_TRY(profile_mark(false, cs));
+    return MUSE_OK;
   }
   // the partially specialised dipole adds s Cbar_i qt to the monopole-only result
   muse_status s2 = refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets,

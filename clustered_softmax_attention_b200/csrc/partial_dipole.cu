@@ -152,6 +152,7 @@ pd_correct(MuseTables mt, int N, float scale, const T *__restrict__ qt_rows,
   }
 }
 
+// O == nullptr: Cov_j and Cbar_i only (the summary-form output applies the correction).
 template <typename T, int D, int DV>
 static cudaError_t run_t(const MuseTables &mt, int N, int P, float scale, SortedSide qs,
                          const int32_t *q_perm, SortedSide ks, const void *V,
@@ -160,9 +161,12 @@ static cudaError_t run_t(const MuseTables &mt, int N, int P, float scale, Sorted
   pd_cov<T, D, DV><<<dim3(mt.k.max_C, P), 256, 0, st>>>(mt, N, (const T *)ks.rows, (const T *)V,
                                                         k_perm, k_offsets, cov);
   pd_aggregate<D, DV><<<dim3(mt.q.max_C, P), 256, 0, st>>>(mt, logZ, cov, cbar);
-  pd_correct<T, D, DV><<<dim3((mt.q.max_rows + 63) / 64, P), 256, 0, st>>>(
-      mt, N, scale, (const T *)qs.rows, qs.cluster, q_perm, cbar, (T *)O);
-  count_launches(3);
+  count_launches(2);
+  if (O) {
+    pd_correct<T, D, DV><<<dim3((mt.q.max_rows + 63) / 64, P), 256, 0, st>>>(
+        mt, N, scale, (const T *)qs.rows, qs.cluster, q_perm, cbar, (T *)O);
+    count_launches(1);
+  }
   return cudaGetLastError();
 }
 
@@ -172,13 +176,17 @@ size_t partial_dipole_ws_floats(int P, int Cq, int Ck, int D, int Dv) {
   return (size_t)P * (size_t)(Cq + Ck) * (size_t)D * (size_t)Dv;
 }
 
+float *partial_dipole_cbar(float *ws, int P, int maxCk, int D, int Dv) {
+  return ws + (size_t)P * maxCk * D * Dv;
+}
+
 cudaError_t run_partial_dipole(const MuseTables &mt, int dtype, int D, int Dv, int N, int P,
                                float scale, SortedSide qs, const int32_t *q_perm, SortedSide ks,
                                const void *V, const int32_t *k_perm, const int32_t *k_offsets,
                                const float *logZ, float *ws, void *O, cudaStream_t st) {
   if (mt.in.ninst != 1) return cudaErrorInvalidValue;
   float *cov = ws;
-  float *cbar = ws + (size_t)P * mt.k.max_C * D * Dv;
+  float *cbar = partial_dipole_cbar(ws, P, mt.k.max_C, D, Dv);
   using namespace pdp;
 #define PD_CASE(TT, DD, DVV)                                                                    \
   if (D == DD && Dv == DVV)                                                                     \

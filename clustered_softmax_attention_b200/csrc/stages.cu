@@ -692,11 +692,6 @@ tilt_cov(MuseTables mt, const int32_t *__restrict__ k_offsets, const float *__re
   }
 }
 
-// Instances a kernel leaves to another one (bit s: instance s).
-struct InstMask {
-  uint32_t w[kMaxSeg / 32];
-};
-
 // ---------------------------------------------------------------------------
 // Refinement coefficients for every sorted query position n of cluster i:
 //   a_j = logZ_ij + s u_j, u_j = qt.mu_k,ij;  p = softmax_j(a);
@@ -1418,6 +1413,24 @@ cudaError_t run_summaries(const MuseTables &mt, int dtype, int D, int Dv, int P,
                     b, st);
 }
 
+template <typename T, int DV>
+static cudaError_t values_t(const MuseTables &mt, int P, const int32_t *k_offsets, const float *W,
+                            const void *vs_rows, float *mu_v, cudaStream_t st) {
+  tilt_moments<T, DV><<<dim3(mt.k.max_C, (mt.q.max_C + 63) / 64, P * mt.in.ninst), 256, 0, st>>>(
+      mt, k_offsets, W, (const T *)vs_rows, mu_v);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t run_tilt_values(const MuseTables &mt, int dtype, int Dv, int P, const int32_t *k_offsets,
+                            const float *W, const void *vs_rows, float *mu_v, cudaStream_t st) {
+  if (dtype == MUSE_F32)
+    return Dv == 64 ? values_t<float, 64>(mt, P, k_offsets, W, vs_rows, mu_v, st)
+                    : values_t<float, 128>(mt, P, k_offsets, W, vs_rows, mu_v, st);
+  return Dv == 64 ? values_t<__nv_bfloat16, 64>(mt, P, k_offsets, W, vs_rows, mu_v, st)
+                  : values_t<__nv_bfloat16, 128>(mt, P, k_offsets, W, vs_rows, mu_v, st);
+}
+
 template <typename T, int D>
 static cudaError_t weights_t(const MuseTables &mt, int P, float scale, const float *qcen,
                              SortedSide ks, const float *logZ, float *W, cudaStream_t st) {
@@ -1483,24 +1496,33 @@ static cudaError_t coeffs_grouped_t(const MuseTables &mt, int P, float scale, So
 }
 
 // Instances whose query clusters hold fewer than 32 rows on average take the grouped
-// kernel (passes of 16 rows), the others the tiled one (chunks of 64 rows); both run when
-// the instances differ (the causal squares).
+// kernel (passes of 16 rows), those with at least 64 the tensor-core kernel (bfloat16:
+// one CTA per cluster and 128 rows), the others the tiled one (chunks of 64 rows); the
+// kinds run side by side when the instances differ (the causal squares).
 template <typename T, int D, int JPT>
 static cudaError_t coeffs_split_t(const MuseTables &mt, int P, float scale, SortedSide qs,
                                   const int32_t *q_offsets, StageBufs b, float sdip,
                                   cudaStream_t st) {
-  InstMask small{}, large{};
-  bool any_small = false, any_large = false;
+  const bool tc = std::is_same<T, __nv_bfloat16>::value && coef_tc_supported(MUSE_BF16, D, mt.k.max_C);
+  // each mask lists the instances its kernel skips
+  InstMask not_small{}, not_mid{}, not_large{};
+  bool any[3] = {false, false, false};
   for (int si = 0; si < mt.in.ninst; ++si) {
-    const bool sm = (int64_t)mt.q.nrow[si] < 32ll * mt.q.C[si];
-    (sm ? large : small).w[si >> 5] |= 1u << (si & 31);  // the mask lists the skipped ones
-    any_small |= sm;
-    any_large |= !sm;
+    const int64_t rows = mt.q.nrow[si], C = mt.q.C[si];
+    const int kind = rows < 32 * C ? 0 : (tc && rows >= 64 * C) ? 2 : 1;
+    any[kind] = true;
+    const uint32_t bit = 1u << (si & 31);
+    if (kind != 0) not_small.w[si >> 5] |= bit;
+    if (kind != 1) not_mid.w[si >> 5] |= bit;
+    if (kind != 2) not_large.w[si >> 5] |= bit;
   }
   cudaError_t err = cudaSuccess;
-  if (any_large) err = coeffs_tiled_t<T, D, JPT>(mt, P, scale, qs, q_offsets, b, large, sdip, st);
-  if (err == cudaSuccess && any_small)
-    err = coeffs_grouped_t<T, D, JPT>(mt, P, scale, qs, q_offsets, b, small, sdip, st);
+  if (any[2])
+    err = run_coef_tc(mt, D, P, scale, qs.rows, q_offsets, b, not_large, sdip, device_status_word(), st);
+  if (err == cudaSuccess && any[1])
+    err = coeffs_tiled_t<T, D, JPT>(mt, P, scale, qs, q_offsets, b, not_mid, sdip, st);
+  if (err == cudaSuccess && any[0])
+    err = coeffs_grouped_t<T, D, JPT>(mt, P, scale, qs, q_offsets, b, not_small, sdip, st);
   return err;
 }
 

@@ -193,10 +193,15 @@ muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims 
  *   (same review: "Axioms", the covariance taken without the tilt by the query
  *   centroid; "invented entities", an aggregated covariance per query cluster; the
  *   weights are not printed, this is the reading taken).
+ * Both ablations need only the summaries: for bfloat16 with Dv = 64 (D = 64 or 128) and
+ * Ck <= 128 they are evaluated in that form, O_n = sum_j p_j mu_v,ij (+ s Cbar_i qt_n),
+ * with the tilted value means mu_v and no contraction over all N keys; other shapes run
+ * the pair form of muse_forward with the dipole coefficient set to zero (plus the
+ * covariance correction).
  * Same arguments, layouts and ownership as muse_forward.  Workspace: that of
  * muse_forward, plus B*H*(Cq + Ck)*D*Dv floats and 256 bytes with
- * MUSE_FLAG_PARTIAL_DIPOLE; muse_workspace_size("muse_forward_ex", ...) returns that
- * larger size.  Unknown flag bits, or both flags at once, return MUSE_ERR_INVALID_ARG
+ * MUSE_FLAG_PARTIAL_DIPOLE, plus B*H*Cq*Ck*Dv floats and 256 bytes in summary form;
+ * muse_workspace_size("muse_forward_ex", ...) returns the largest of these sizes.  Unknown flag bits, or both flags at once, return MUSE_ERR_INVALID_ARG
  * before anything is enqueued.
  */
 #define MUSE_FLAG_MONOPOLE 1u

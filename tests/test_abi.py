@@ -42,9 +42,11 @@ def test_workspace_sizes(lib):
     assert lib.muse_workspace_size(b"muse_forward", d, 0, 32, 0, 0, 0) == 0
     assert lib.muse_workspace_size(b"muse_forward", d, 2048, 32, 0, 0, 0) == 0
     # forward_ex: the forward pass's buffers plus the partially specialised dipole's
-    # covariances, B*H*(Cq+Ck)*D*Dv floats and 256 bytes
+    # covariances, B*H*(Cq+Ck)*D*Dv floats and 256 bytes, plus the summary form's tilted
+    # value means, B*H*Cq*Ck*Dv floats and 256 bytes
     assert (lib.muse_workspace_size(b"muse_forward_ex", d, 32, 32, 0, 0, 0)
-            == lib.muse_workspace_size(b"muse_forward", d, 32, 32, 0, 0, 0) + 2 * 64 * 64 * 64 * 4 + 256)
+            == lib.muse_workspace_size(b"muse_forward", d, 32, 32, 0, 0, 0) + 2 * 64 * 64 * 64 * 4 + 256
+            + 2 * 32 * 32 * 64 * 4 + 256)
     # forward = two clusterings + refinement buffers: grows with N
     assert (lib.muse_workspace_size(b"muse_forward", _d(N=2048), 32, 32, 0, 0, 0)
             > lib.muse_workspace_size(b"muse_forward", d, 32, 32, 0, 0, 0))

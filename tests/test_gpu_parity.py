@@ -193,12 +193,15 @@ def test_refine_reports_labels_that_disagree_with_the_permutation():
 # 127-129 and 300 keys (one chunk, several chunks, several clusters per CTA, windows of
 # whole clusters with an empty one inside), 70 centroids (a ragged second group of 64),
 # given directly as a permutation and offsets; Ck = 128 makes most clusters a few keys.
-@pytest.mark.parametrize("dt,D,Ck", [("bf16", 64, 16), ("bf16", 64, 40), ("f32", 64, 40),
-                                      ("bf16", 128, 40), ("f32", 128, 16), ("bf16", 64, 128),
-                                      ("f32", 128, 128)])
-def test_key_means_cluster_layouts(dt, D, Ck, parity):
+# Cq = 200 takes two blocks of 128 query centroids.
+@pytest.mark.parametrize("dt,D,Ck,Cq", [("bf16", 64, 16, 70), ("bf16", 64, 40, 70),
+                                         ("f32", 64, 40, 70), ("bf16", 128, 40, 70),
+                                         ("f32", 128, 16, 70), ("bf16", 64, 128, 70),
+                                         ("f32", 128, 128, 70), ("bf16", 64, 40, 200),
+                                         ("bf16", 128, 128, 200)])
+def test_key_means_cluster_layouts(dt, D, Ck, Cq, parity):
     rng = np.random.Generator(np.random.PCG64(100 + Ck + D))
-    N, Cq, s = 1200, 70, 0.35
+    N, s = 1200, 0.35
     fixed = [300, 0, 1, 15, 0, 16, 17, 64, 65, 127, 128, 129, 0]
     rest = Ck - len(fixed)
     left = N - sum(fixed)
@@ -257,10 +260,14 @@ def test_forward_end_to_end_small_f32(parity):
 
 # the monopole-only ablation (dipole term dropped) against the oracle's same mode, with
 # the GPU's clustering; it must be less accurate than the full method on these inputs
-@pytest.mark.parametrize("dt,D", [("f32", 64), ("bf16", 64), ("bf16", 128)])
-def test_forward_monopole_only(dt, D, parity):
-    N, C, T = 2048, 32, 6
-    Q, K, V = mixture(9, 1, 2, N, D, D, 48, 0.5 / np.sqrt(D), dt)
+# (bfloat16 with Dv = 64 evaluates it in summary form, without the N^2 contraction; C = 128
+# takes the output kernel's 128-cluster variant; D = Dv = 128 runs the pair form)
+@pytest.mark.parametrize("dt,D,Dv,C", [("f32", 64, 64, 32), ("bf16", 64, 64, 32),
+                                       ("bf16", 128, 128, 32), ("bf16", 64, 64, 128),
+                                       ("bf16", 128, 64, 128)])
+def test_forward_monopole_only(dt, D, Dv, C, parity):
+    N, T = 2048, 6
+    Q, K, V = mixture(9, 1, 2, N, D, Dv, 48, 0.5 / np.sqrt(D), dt)
     Qd, Kd, Vd = dev(Q, dt), dev(K, dt), dev(V, dt)
     Om = host(m.muse_forward_ex(Qd, Kd, Vd, C, C, T, 1.0, flags=m.MUSE_FLAG_MONOPOLE))
     Od = host(m.muse_forward_ex(Qd, Kd, Vd, C, C, T, 1.0))
@@ -275,12 +282,13 @@ def test_forward_monopole_only(dt, D, parity):
         assert mo.max_rel_err(Om[0, h], ref_m) <= TOL[dt]
         E = mo.exact_attention(Qf[0, h], Kf[0, h], Vf[0, h], 1.0)
         assert mo.rse(Od[0, h], E) < mo.rse(Om[0, h], E)
+    assert m.muse_last_device_status() == 0
 
 
 # the partially specialised dipole (untilted key-cluster covariances aggregated per query
 # cluster) against the oracle's same reading, with the GPU's clustering
 @pytest.mark.parametrize("dt,D,Dv", [("f32", 64, 64), ("bf16", 64, 64), ("bf16", 128, 128),
-                                     ("f32", 64, 128)])
+                                     ("f32", 64, 128), ("bf16", 128, 64)])
 def test_forward_partial_dipole(dt, D, Dv, parity):
     N, C, T = 2048, 32, 6
     Q, K, V = mixture(10, 1, 2, N, D, Dv, 48, 0.5 / np.sqrt(D), dt)
@@ -294,6 +302,7 @@ def test_forward_partial_dipole(dt, D, Dv, parity):
                                                  kl[0, h].cpu().numpy(), C, C, 1.0)
         parity(f"O h={h}", mo.max_rel_err(Op[0, h], ref), TOL[dt])
         assert mo.max_rel_err(Op[0, h], ref) <= TOL[dt]
+    assert m.muse_last_device_status() == 0
 
 
 def test_forward_bf16_multihead(parity):
