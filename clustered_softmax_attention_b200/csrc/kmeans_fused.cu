@@ -42,16 +42,22 @@ namespace kmf {
 
 constexpr int TM = 128;        // rows per tile
 constexpr int D = 64;          // row width handled by this kernel
-constexpr int NSX = 4;         // row-tile stages
-constexpr int NOH = 2;         // one-hot buffers
 constexpr int CMAX = 128;      // clusters per task
 constexpr int GMAX = 8;        // CTAs per thread-block cluster (at most)
 constexpr int TPC = 8;         // row tiles per CTA that a group size aims for
 constexpr int kEpi = 8;        // epilogue warps
 constexpr int kThreads = 64 + 32 * kEpi;
 constexpr int PLD = D + 4;     // padded row stride (floats) of the partial sums
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSumCol = 256;  // TMEM column of the centroid-sum accumulator
+// Two variants by the largest cluster count CM of a launch: CM = 128, and CM = 64, whose
+// shared memory (two row stages, one 64-cluster block per one-hot buffer) and TMEM fit
+// two CTAs on an SM.
+template <int CM> struct KCfg {
+  static constexpr int NSX = CM == 64 ? 2 : 4;  // row-tile stages
+  static constexpr int NOH = 2;                 // one-hot buffers
+  static constexpr int OHB = CM / 64;           // 64-cluster blocks per one-hot buffer
+  static constexpr uint32_t kTmemCols = CM == 64 ? 256 : 512;
+  static constexpr uint32_t kSumCol = 2 * CM;   // TMEM column of the centroid-sum accumulator
+};
 
 struct PlanEntry {
   uint8_t seg, g;
@@ -71,19 +77,23 @@ struct Params {
   Job job[2];
 };
 
-struct __align__(1024) Smem {
-  __nv_bfloat16 x[NSX][TM * 64];      // row tiles, rows of 128 B, 128-byte swizzle
-  __nv_bfloat16 oh[NOH][2][TM * 64];  // one-hot rows [row][cluster], two 64-cluster blocks
-  __nv_bfloat16 hi[CMAX * 64];        // centroid split, K-major, 128-byte swizzle
-  __nv_bfloat16 lo[CMAX * 64];
-  float part[CMAX * PLD];             // partial sums; the reducer's new centroids in place
-  float cn[CMAX];                     // squared centroid norms (+inf on padding rows)
-  int cnt[CMAX];                      // this CTA's member counts of the round
-  int tot[CMAX];                      // group totals of the clusters this CTA reduces
-  int totall[CMAX];                   // group totals of every cluster
-  int base[CMAX];                     // final sort: next position per cluster
-  int wc[4][CMAX];                    // final sort: members per (warp, cluster) of a tile
-  uint64_t xfull[NSX], xempty[NSX], sfull[2], sfree[2], ohfull[NOH], ohempty[NOH];
+template <int CM> struct __align__(1024) Smem {
+  using Cf = KCfg<CM>;
+  // one-hot rows [row][cluster] in 64-cluster blocks; the row tiles follow them, so that
+  // with one block (CM = 64) the sums contraction's second M block (clusters 64-127, whose
+  // TMEM lanes are never read) reads finite data inside the CTA's shared memory
+  __nv_bfloat16 oh[Cf::NOH][Cf::OHB][TM * 64];
+  __nv_bfloat16 x[Cf::NSX][TM * 64];  // row tiles, rows of 128 B, 128-byte swizzle
+  __nv_bfloat16 hi[CM * 64];          // centroid split, K-major, 128-byte swizzle
+  __nv_bfloat16 lo[CM * 64];
+  float part[CM * PLD];               // partial sums; the reducer's new centroids in place
+  float cn[CM];                       // squared centroid norms (+inf on padding rows)
+  int cnt[CM];                        // this CTA's member counts of the round
+  int tot[CM];                        // group totals of the clusters this CTA reduces
+  int totall[CM];                     // group totals of every cluster
+  int base[CM];                       // final sort: next position per cluster
+  int wc[4][CM];                      // final sort: members per (warp, cluster) of a tile
+  uint64_t xfull[Cf::NSX], xempty[Cf::NSX], sfull[2], sfree[2], ohfull[Cf::NOH], ohempty[Cf::NOH];
   uint64_t sumdone, fin;
   uint32_t tmem_base;
   int abort_flag;
@@ -149,7 +159,8 @@ __host__ __device__ constexpr uint32_t idesc_mn(int M, int N) {
 
 // Writes half h (32 values) of centroid row c into the K-major split operands and
 // returns the partial squared norm.
-__device__ __forceinline__ float put_centroid(Smem &sm, int c, int h, const float (&v)[32]) {
+template <int CM>
+__device__ __forceinline__ float put_centroid(Smem<CM> &sm, int c, int h, const float (&v)[32]) {
   float sq = 0.f;
 #pragma unroll
   for (int j4 = 0; j4 < 4; ++j4) {
@@ -173,12 +184,16 @@ __device__ __forceinline__ float put_centroid(Smem &sm, int c, int h, const floa
   return sq;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int CM>
+__global__ void __launch_bounds__(kThreads, CM == 64 ? 2 : 1)
 km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
          const __grid_constant__ Params prm, int *status) {
+  using Cf = KCfg<CM>;
+  constexpr int NSX = Cf::NSX, NOH = Cf::NOH;
+  constexpr uint32_t kTmemCols = Cf::kTmemCols, kSumCol = Cf::kSumCol;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                       ~(uintptr_t)1023);
+  Smem<CM> &sm = *reinterpret_cast<Smem<CM> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int *abort_flag = &sm.abort_flag;
 
@@ -240,7 +255,7 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
   }
   if (active) {
     // starting centroids: the first C rows of the task
-    for (int tid = threadIdx.x; tid < 2 * CMAX; tid += kThreads) {
+    for (int tid = threadIdx.x; tid < 2 * CM; tid += kThreads) {
       const int c = tid >> 1, h = tid & 1;
       float v[32];
       const __nv_bfloat16 *xr = static_cast<const __nv_bfloat16 *>(J.X) + (grow0 + c) * D + h * 32;
@@ -268,7 +283,7 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
         sm.cnt[c] = 0;
       }
     }
-    for (int e = threadIdx.x; e < 4 * CMAX; e += kThreads) (&sm.wc[0][0])[e] = 0;
+    for (int e = threadIdx.x; e < 4 * CM; e += kThreads) (&sm.wc[0][0])[e] = 0;
   }
   fence_async_smem();
   tc_fence_before();
@@ -312,9 +327,9 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
               tc_fence_after();
               const uint32_t id = idesc(TM, CP);
               for (int kk = 0; kk < D / 16; ++kk)
-                tc_mma(tmem + buf * 128, sdesc(sm.x[st] + kk * 16), sdesc(sm.hi + kk * 16), id, kk > 0 ? 1u : 0u);
+                tc_mma(tmem + buf * CM, sdesc(sm.x[st] + kk * 16), sdesc(sm.hi + kk * 16), id, kk > 0 ? 1u : 0u);
               for (int kk = 0; kk < D / 16; ++kk)
-                tc_mma(tmem + buf * 128, sdesc(sm.x[st] + kk * 16), sdesc(sm.lo + kk * 16), id, 1u);
+                tc_mma(tmem + buf * CM, sdesc(sm.x[st] + kk * 16), sdesc(sm.lo + kk * 16), id, 1u);
               tc_commit(&sm.sfull[buf]);
               ++a;
               progressed = true;
@@ -368,25 +383,27 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
         if (buf != grp) continue;
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.sfull[buf], (u >> 1) & 1, abort_flag, status))) break;
         tc_fence_after();
-        // 16-column chunks in batches of four, one chain per chunk; chains and
-        // batches are merged in column order (strict <: the lowest index wins a tie)
+        // 16-column chunks in batches of NB (four; two in the 64-cluster variant, which
+        // has half the registers), one chain per chunk; chains and batches are merged
+        // in column order (strict <: the lowest index wins a tie)
+        constexpr int NB = CM == 64 ? 2 : 4;
         float bv = CUDART_INF_F;
         int bc = 0;
-        for (int c0 = 0; c0 < CP; c0 += 64) {
-          uint32_t raw[4][16];
+        for (int c0 = 0; c0 < CP; c0 += 16 * NB) {
+          uint32_t raw[NB][16];
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch)
-            if (c0 + ch * 16 < CP) tmem_ld16_async(tmem + lane_base + buf * 128 + c0 + ch * 16, raw[ch]);
+          for (int ch = 0; ch < NB; ++ch)
+            if (c0 + ch * 16 < CP) tmem_ld16_async(tmem + lane_base + buf * CM + c0 + ch * 16, raw[ch]);
           tmem_ld_wait();
-          if (c0 + 64 >= CP) {
+          if (c0 + 16 * NB >= CP) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.sfree[buf]);
           }
-          float best[4];
-          int bi[4];
+          float best[NB];
+          int bi[NB];
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
+          for (int ch = 0; ch < NB; ++ch) {
             best[ch] = CUDART_INF_F;
             bi[ch] = 0;
             if (c0 + ch * 16 < CP) {
@@ -406,7 +423,7 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
             }
           }
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch)
+          for (int ch = 0; ch < NB; ++ch)
             if (best[ch] < bv) {
               bv = best[ch];
               bc = bi[ch];
@@ -426,7 +443,7 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
         const uint32_t one = (L & 1) ? 0x3F800000u : 0x00003F80u;
         const int w = (L & 7) >> 1;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int half = 0; half < Cf::OHB; ++half) {
           unsigned char *dst = reinterpret_cast<unsigned char *>(sm.oh[ob][half]) + rr * 128;
           const int lc = L - half * 64;
           const bool hit = lc >= 0 && lc < 64;
@@ -468,9 +485,11 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0.f;
       }
-      float4 *dst = reinterpret_cast<float4 *>(&sm.part[c * PLD + half * 32]);
+      if (c < CM) {  // (lanes past CM hold the second M block's unused sums)
+        float4 *dst = reinterpret_cast<float4 *>(&sm.part[c * PLD + half * 32]);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+      }
       tc_fence_before();
     }
     __syncwarp();
@@ -509,7 +528,7 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
     cluster_wait();
     // (3) every CTA gathers the new centroids (split operands, norms) and the totals
     if (active) {
-      for (int tid = threadIdx.x; tid < 2 * CMAX; tid += kThreads) {
+      for (int tid = threadIdx.x; tid < 2 * CM; tid += kThreads) {
         const int c = tid >> 1, h = tid & 1;
         const uint32_t q = gb + (uint32_t)(c % g);
         float v[32];
@@ -542,7 +561,7 @@ km_fused(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUten
           int tv[4], s = 0;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            tv[k] = sm.totall[4 * lane + k];
+            tv[k] = 4 * lane + k < CM ? sm.totall[4 * lane + k] : 0;
             s += tv[k];
           }
           int inc = s;
@@ -694,14 +713,15 @@ static int plan_all(Params &prm, int njobs, const void *const *X, const SegTable
 
 }  // namespace kmf
 
-// CTAs of the fused kernel that can be resident at once in clusters of Z (0: not even
-// one cluster fits).
+// CTAs of the fused kernel (variant CM) that can be resident at once in clusters of Z
+// (0: not even one cluster fits).
+template <int CM>
 static int kmf_capacity(int Z) {
   static int cap[kmf::GMAX + 1] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
   if (cap[Z] < 0) {
-    const size_t smem = sizeof(kmf::Smem) + 1024;
+    const size_t smem = sizeof(kmf::Smem<CM>) + 1024;
     int n = 0;
-    if (cudaFuncSetAttribute(kmf::km_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+    if (cudaFuncSetAttribute(kmf::km_fused<CM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
         cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute at[1];
@@ -714,7 +734,7 @@ static int kmf_capacity(int Z) {
       cfg.dynamicSmemBytes = smem;
       cfg.attrs = at;
       cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&n, kmf::km_fused, &cfg) != cudaSuccess) n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kmf::km_fused<CM>, &cfg) != cudaSuccess) n = 0;
     }
     if (n <= 0) cudaGetLastError();  // the multi-launch path takes over; leave no error behind
     cap[Z] = n * Z;
@@ -727,12 +747,13 @@ bool kmeans_fused_supported(int dtype, int D, const SegTable &t) {
   int span = 0;
   for (int s = 0; s < t.nseg; ++s) span += kmf::group_size(t.nrow[s], kmf::TPC, kmf::GMAX);
   if (span > 65535 / 3) return false;  // positions of any plan (groups of 6 are at most 1.5x, padding < 2x) fit 16 bits
-  return kmf_capacity(kmf::GMAX) > 0;
+  return (t.max_C <= 64 ? kmf_capacity<64>(kmf::GMAX) : kmf_capacity<128>(kmf::GMAX)) > 0;
 }
 
-cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *const *tabs,
-                             const KmeansOut *outs, int N, int P, int iters, int *status,
-                             cudaStream_t st) {
+template <int CM>
+static cudaError_t launch_fused(int njobs, const void *const *X, const SegTable *const *tabs,
+                                const KmeansOut *outs, int N, int P, int iters, int *status,
+                                cudaStream_t st) {
   using namespace kmf;
   Params prm{};
   prm.njobs = njobs;
@@ -744,7 +765,7 @@ cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *co
   // clusters of 8 with about 8 tiles per CTA, in several waves.
   int bestZ = GMAX, best_tpc = TPC, best_tiles = 1 << 30;
   for (int Z : {GMAX, 6}) {
-    const int cap = kmf_capacity(Z);
+    const int cap = kmf_capacity<CM>(Z);
     if (cap <= 0) continue;
     for (int tpc = TPC; tpc <= 8 * TPC; tpc *= 2) {
       int tiles = 0;
@@ -762,8 +783,8 @@ cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *co
   if (!ptx::make_map(&m0, X[0], D, (uint64_t)P * N, D, TM) ||
       !ptx::make_map(&m1, X[njobs > 1 ? 1 : 0], D, (uint64_t)P * N, D, TM))
     return cudaErrorInvalidValue;
-  const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(km_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = sizeof(Smem<CM>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(km_fused<CM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute at[1];
@@ -777,10 +798,21 @@ cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *co
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, km_fused, m0, m1, prm, status);
+  e = cudaLaunchKernelEx(&cfg, km_fused<CM>, m0, m1, prm, status);
   count_launches(1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// The 64-cluster variant (two CTAs per SM) when every task of the launch has C <= 64.
+cudaError_t run_kmeans_fused(int njobs, const void *const *X, const SegTable *const *tabs,
+                             const KmeansOut *outs, int N, int P, int iters, int *status,
+                             cudaStream_t st) {
+  int maxC = 0;
+  for (int j = 0; j < njobs; ++j) maxC = std::max(maxC, tabs[j]->max_C);
+  if (maxC <= 64 && kmf_capacity<64>(kmf::GMAX) > 0)
+    return launch_fused<64>(njobs, X, tabs, outs, N, P, iters, status, st);
+  return launch_fused<128>(njobs, X, tabs, outs, N, P, iters, status, st);
 }
 
 }  // namespace muse
