@@ -105,6 +105,11 @@ cudaError_t run_partial_dipole(const MuseTables &mt, int dtype, int D, int Dv, i
                                float scale, SortedSide qs, const int32_t *q_perm, SortedSide ks,
                                const void *V, const int32_t *k_perm, const int32_t *k_offsets,
                                const float *logZ, float *ws, void *O, cudaStream_t st);
+// Tilt logits s qbar_i . k of every instance on the tensor cores (logits_tc.cu), written
+// into W for the tilt stage: bfloat16, D = 64 or 128.
+bool logits_tc_supported(int dtype, int D);
+cudaError_t run_logits_tc(const MuseTables &mt, int D, int P, float scale, const float *q_centroids,
+                          const void *ks_rows, float *W, int *status, cudaStream_t st);
 // Instances a kernel leaves to another one (bit s: instance s).
 struct InstMask {
   uint32_t w[kMaxSeg / 32];

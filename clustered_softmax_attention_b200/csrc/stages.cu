@@ -359,7 +359,9 @@ struct TiltStep {
   int j, je, b, e, pc, pass;
 };
 
-template <typename T, int D>
+// PRE: the logits s qbar_i . k are already in W (logits_tc.cu, tensor cores); the kernel
+// reads them instead of computing them, and overwrites them with the weights.
+template <typename T, int D, bool PRE>
 __global__ void __launch_bounds__(256, 2)
 tilt_fused(MuseTables mt, float scale, const float *__restrict__ qcen, const T *__restrict__ ks,
            const int32_t *__restrict__ k_offsets, float *__restrict__ W, float *__restrict__ logZ,
@@ -384,7 +386,7 @@ tilt_fused(MuseTables mt, float scale, const float *__restrict__ qcen, const T *
   if (j0 >= Ck || i0 >= Cq) return;  // uniform
   const int tid = threadIdx.x, ti = tid >> 4, td = tid & 15;
   if (tid <= j1 - j0) offs[tid] = k_offsets[k.off + j0 + tid];
-  {
+  if (!PRE) {
     constexpr int QU = D / 4, NR = 64 * QU / 256;
     float4 v[NR];
 #pragma unroll
@@ -516,6 +518,15 @@ tilt_fused(MuseTables mt, float scale, const float *__restrict__ qcen, const T *
     auto body = [&](auto ncv) {
       constexpr int NC = decltype(ncv)::value;
       float L[4][NC];
+      if constexpr (PRE) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const int i = i0 + ti * 4 + a;
+#pragma unroll
+          for (int c = 0; c < NC; ++c)
+            L[a][c] = (i < Cq && td + 16 * c < pt) ? wb[(int64_t)i * wl + cur.pc + td + 16 * c] : -CUDART_INF_F;
+        }
+      } else {
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -541,6 +552,7 @@ tilt_fused(MuseTables mt, float scale, const float *__restrict__ qcen, const T *
       for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int c = 0; c < NC; ++c) L[a][c] = td + 16 * c < pt ? scale * L[a][c] : -CUDART_INF_F;
+      }
       if (cur.pass == 3) {
         // a window of whole clusters: the logits go through shared memory, logZ per
         // (cluster, centroid) by a scan of the cluster's keys, then the weights and one
@@ -1334,7 +1346,7 @@ cudaError_t run_sort_side_t(const void *X, int dtype, int width, int N, const Se
   return cudaGetLastError();
 }
 
-template <typename T, int D>
+template <typename T, int D, bool PRE>
 static cudaError_t launch_tilt_fused(const MuseTables &mt, int P, float scale, const float *qcen,
                                      SortedSide ks, const int32_t *k_offsets, StageBufs b,
                                      cudaStream_t st) {
@@ -1348,10 +1360,10 @@ static cudaError_t launch_tilt_fused(const MuseTables &mt, int P, float scale, c
   for (int si = mt.in.ninst + 1; si <= kMaxSeg; ++si) bm.pre[si] = bm.pre[mt.in.ninst];
   bm.total = bm.pre[mt.in.ninst];
   if (bm.total == 0) return cudaSuccess;
-  cudaError_t err = cudaFuncSetAttribute(tilt_fused<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t err = cudaFuncSetAttribute(tilt_fused<T, D, PRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cf::smem);
   if (err != cudaSuccess) return err;
-  tilt_fused<T, D><<<dim3(bm.total, (mt.q.max_C + 63) / 64, P), 256, Cf::smem, st>>>(
+  tilt_fused<T, D, PRE><<<dim3(bm.total, (mt.q.max_C + 63) / 64, P), 256, Cf::smem, st>>>(
       mt, scale, qcen, (const T *)ks.rows, k_offsets, b.W, b.logZ, b.mu_k, bm);
   count_launches(1);
   return cudaGetLastError();
@@ -1364,8 +1376,14 @@ static cudaError_t summaries_t(const MuseTables &mt, int P, float scale, const f
   const int tasks = P * mt.in.ninst;
   const int maxCq = mt.q.max_C, maxCk = mt.k.max_C;
   if (b.mu_k && !b.mu_v && !b.cov) {
-    // the forward pass: logits, log-normalisers, weights and key means in one launch
-    return launch_tilt_fused<T, D>(mt, P, scale, qcen, ks, k_offsets, b, st);
+    // the forward pass: log-normalisers, weights and key means in one launch, from
+    // logits of the tensor cores (bfloat16) or its own (float32)
+    if (std::is_same<T, __nv_bfloat16>::value && logits_tc_supported(MUSE_BF16, D)) {
+      cudaError_t e = run_logits_tc(mt, D, P, scale, qcen, ks.rows, b.W, device_status_word(), st);
+      if (e != cudaSuccess) return e;
+      return launch_tilt_fused<T, D, true>(mt, P, scale, qcen, ks, k_offsets, b, st);
+    }
+    return launch_tilt_fused<T, D, false>(mt, P, scale, qcen, ks, k_offsets, b, st);
   }
   const BlockMap kbm = make_block_map(mt.k, 64);
   tilt_logits<T, D><<<dim3(kbm.total, (maxCq + 63) / 64, P), 256, 0, st>>>(
