@@ -23,7 +23,7 @@ namespace ltc {
 using namespace ptx;
 
 constexpr int TM = 128;     // centroids per CTA, keys per tile
-constexpr int kTiles = 8;   // key tiles per CTA (at most)
+constexpr int kTiles = 2;   // key tiles per CTA (at most): 256 CTAs at N = 8k, 8 heads
 
 template <int D> struct __align__(1024) Smem {
   __nv_bfloat16 c[3][D / 64][TM * 64];  // centroid parts, K-major, 128-byte swizzle

@@ -649,24 +649,39 @@ ret_coeffs(Geo g, float scale, const int32_t *__restrict__ q_perm,
 // block b), merged into the remainder partial of every row of the group (token order):
 // part_lse[p][n], part_o[p][n][:] become the joint (log-normaliser, normalised output) of
 // the remainder and the runs.  One warp per (problem, i, b) group, no block-wide
-// barrier: the warp lists the runs (lanes over the slots, a shuffle scan of their
-// lengths), then for every row of the group walks the runs' keys 32 at a time -- lane k
-// forms the logit of key k against the row's query (held in shared memory), the warp
-// updates the online softmax, and lanes over output columns accumulate p_k v_k (value
-// rows read whole by the warp).
+// barrier.  The warp lists the runs (lanes over the slots, a shuffle scan of their
+// lengths); the runs are the same for every row of the group, so their keys are staged
+// once per chunk of 32 into the warp's shared memory (the keys as sorted, contiguous
+// inside a run; the values by token) and serve up to RB rows at a time: lane k forms the
+// logit of key k against each row's query, the warp updates each row's online softmax,
+// and lanes over output columns accumulate p_k v_k from the staged values.
+template <int D, int DV> struct RunsCfg {
+  static constexpr int WPC = D == 64 && DV == 64 ? 8 : 4;  // warps (groups) per CTA
+  static constexpr int KS = D + 2;                          // staged key row (bf16): 4-byte
+                                                            // reads of lane k hit bank k + d/2
+  static constexpr int RB = 4;                              // rows per pass over the keys
+  static constexpr size_t warp_bytes = (size_t)32 * KS * 2 + (size_t)32 * DV * 2 + (size_t)RB * D * 4;
+  static constexpr size_t smem = WPC * warp_bytes;
+};
+
 template <int D, int DV>
-__global__ void __launch_bounds__(256)
-ret_runs(Geo g, int P, float scale, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
+__global__ void __launch_bounds__(RunsCfg<D, DV>::WPC * 32)
+ret_runs(Geo g, int P, float scale, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ ks,
          const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ q_perm,
          const int32_t *__restrict__ q_offsets, const int32_t *__restrict__ qpend,
          const int32_t *__restrict__ k_perm, const int32_t *__restrict__ k_offsets,
          const int32_t *__restrict__ pend, const int32_t *__restrict__ sel,
          float *__restrict__ part_o, float *__restrict__ part_lse) {
-  constexpr int PV = DV / 32;
-  __shared__ float qsh[8][D];
-  __shared__ int runs[8][64], cum[8][65];
+  using Cf = RunsCfg<D, DV>;
+  constexpr int PV = DV / 32, KS = Cf::KS, RB = Cf::RB;
+  extern __shared__ float4 runs_smem[];
+  __shared__ int runs[Cf::WPC][64], cum[Cf::WPC][65];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t gid = (int64_t)blockIdx.x * 8 + warp;  // (p, i, b)
+  unsigned char *wbase = reinterpret_cast<unsigned char *>(runs_smem) + warp * Cf::warp_bytes;
+  __nv_bfloat16 *Ksh = reinterpret_cast<__nv_bfloat16 *>(wbase);            // [32][KS]
+  __nv_bfloat16 *Vsh = Ksh + 32 * KS;                                       // [32][DV]
+  float *qsh = reinterpret_cast<float *>(Vsh + 32 * DV);                    // [RB][D]
+  const int64_t gid = (int64_t)blockIdx.x * Cf::WPC + warp;  // (p, i, b)
   if (gid >= (int64_t)g.nb * g.Cq * P) return;  // whole warps
   const int b = (int)(gid % g.nb), i = (int)((gid / g.nb) % g.Cq), p = (int)(gid / ((int64_t)g.nb * g.Cq));
   if (b == 0) return;
@@ -711,68 +726,105 @@ ret_runs(Geo g, int P, float scale, const __nv_bfloat16 *__restrict__ Q, const _
   const int total = cum[warp][64];
   if (total == 0) return;
   const int32_t *kperm = k_perm + (int64_t)p * g.N;
-  for (int r = r0; r < r1; ++r) {
-    const int n = q_perm[(int64_t)p * g.N + r];
+  for (int rb = r0; rb < r1; rb += RB) {
+    const int nr = min(RB, r1 - rb);
+    // the batch's queries (scaled), rows past the batch repeat its first row
     __syncwarp();
-    for (int d = lane; d < D; d += 32) qsh[warp][d] = __bfloat162float(Q[((int64_t)p * g.N + n) * D + d]) * scale;
-    __syncwarp();
-    float m = -CUDART_INF_F, l = 0.f, o[PV];
+    for (int x = lane; x < RB * D; x += 32) {
+      const int rr = x / D, d = x % D;
+      const int n = q_perm[(int64_t)p * g.N + rb + (rr < nr ? rr : 0)];
+      qsh[x] = __bfloat162float(Q[((int64_t)p * g.N + n) * D + d]) * scale;
+    }
+    float m[RB], l[RB], o[RB][PV];
 #pragma unroll
-    for (int v = 0; v < PV; ++v) o[v] = 0.f;
-    int rr = 0;  // run of this lane's key (the lane's keys only move forward)
+    for (int rr = 0; rr < RB; ++rr) {
+      m[rr] = -CUDART_INF_F;
+      l[rr] = 0.f;
+#pragma unroll
+      for (int v = 0; v < PV; ++v) o[rr][v] = 0.f;
+    }
+    int run = 0;  // run of this lane's key (the lane's keys only move forward)
     for (int c0 = 0; c0 < total; c0 += 32) {
-      const int gi = c0 + lane;
-      int tok = 0;
-      float x = -CUDART_INF_F;
+      const int gi = c0 + lane, cnt = min(32, total - c0);
+      __syncwarp();  // the previous chunk's keys and values are consumed
       if (gi < total) {
-        while (cum[warp][rr + 1] <= gi) ++rr;
-        tok = kperm[runs[warp][rr] + gi - cum[warp][rr]];
-        const uint4 *kr = reinterpret_cast<const uint4 *>(K + ((int64_t)p * g.N + tok) * D);
-        float a = 0.f;
+        while (cum[warp][run + 1] <= gi) ++run;
+        const int pos = runs[warp][run] + gi - cum[warp][run];  // sorted key position
+        const int tok = kperm[pos];
+        const uint4 *kr = reinterpret_cast<const uint4 *>(ks + ((int64_t)p * g.N + pos) * D);
+        uint32_t *kd = reinterpret_cast<uint32_t *>(Ksh + lane * KS);  // 4-byte aligned rows
 #pragma unroll
         for (int u = 0; u < D / 8; ++u) {
           const uint4 w4 = kr[u];
-          const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&ww[h]);
-            a = fmaf(qsh[warp][8 * u + 2 * h], __low2float(b2), a);
-            a = fmaf(qsh[warp][8 * u + 2 * h + 1], __high2float(b2), a);
-          }
+          kd[4 * u] = w4.x;
+          kd[4 * u + 1] = w4.y;
+          kd[4 * u + 2] = w4.z;
+          kd[4 * u + 3] = w4.w;
         }
-        x = a;
-      }
-      const float mn = fmaxf(m, warp_max(x));
-      const float corr = expf(m - mn);
-      const float pk = gi < total ? expf(x - mn) : 0.f;
-      l = l * corr + warp_sum(pk);
+        const uint4 *vr = reinterpret_cast<const uint4 *>(V + ((int64_t)p * g.N + tok) * DV);
+        uint4 *vd = reinterpret_cast<uint4 *>(Vsh + lane * DV);
 #pragma unroll
-      for (int v = 0; v < PV; ++v) o[v] *= corr;
-      const int cnt = min(32, total - c0);
+        for (int u = 0; u < DV / 8; ++u) vd[u] = vr[u];
+      }
+      __syncwarp();
+      // logits of the lane's key against each row of the batch
+      float x[RB];
+#pragma unroll
+      for (int rr = 0; rr < RB; ++rr) x[rr] = 0.f;
+      if (gi < total) {
+        const __nv_bfloat162 *kk = reinterpret_cast<const __nv_bfloat162 *>(Ksh + lane * KS);
+#pragma unroll 8
+        for (int u = 0; u < D / 2; ++u) {
+          const float2 kf = __bfloat1622float2(kk[u]);
+#pragma unroll
+          for (int rr = 0; rr < RB; ++rr)
+            x[rr] = fmaf(qsh[rr * D + 2 * u], kf.x, fmaf(qsh[rr * D + 2 * u + 1], kf.y, x[rr]));
+        }
+      }
+      float pk[RB];
+#pragma unroll
+      for (int rr = 0; rr < RB; ++rr) {
+        const float xv = gi < total ? x[rr] : -CUDART_INF_F;
+        const float mn = fmaxf(m[rr], warp_max(xv));
+        const float corr = expf(m[rr] - mn);
+        pk[rr] = gi < total ? expf(xv - mn) : 0.f;
+        l[rr] = l[rr] * corr + warp_sum(pk[rr]);
+#pragma unroll
+        for (int v = 0; v < PV; ++v) o[rr][v] *= corr;
+        m[rr] = mn;
+      }
       for (int k = 0; k < cnt; ++k) {
-        const float pkk = __shfl_sync(0xffffffffu, pk, k);
-        const int tk = __shfl_sync(0xffffffffu, tok, k);
-        const __nv_bfloat16 *vr = V + ((int64_t)p * g.N + tk) * DV;
+        float vv[PV];
 #pragma unroll
-        for (int v = 0; v < PV; ++v) o[v] = fmaf(pkk, __bfloat162float(vr[lane + 32 * v]), o[v]);
+        for (int v = 0; v < PV; ++v) vv[v] = __bfloat162float(Vsh[k * DV + lane + 32 * v]);
+#pragma unroll
+        for (int rr = 0; rr < RB; ++rr) {
+          const float pkk = __shfl_sync(0xffffffffu, pk[rr], k);
+#pragma unroll
+          for (int v = 0; v < PV; ++v) o[rr][v] = fmaf(pkk, vv[v], o[rr][v]);
+        }
       }
-      m = mn;
     }
-    // joint softmax with the remainder partial of the row
-    const int64_t at = (int64_t)p * g.N + n;
-    const float L = part_lse[at];
-    float *po = part_o + at * DV;
-    const bool has = L > -CUDART_INF_F;
-    const float mn = has ? fmaxf(m, L) : m;
-    const float ca = expf(m - mn), cb = has ? expf(L - mn) : 0.f;
-    const float lt = l * ca + cb;
+    // joint softmax with the remainder partial of each row
 #pragma unroll
-    for (int v = 0; v < PV; ++v) {
-      const float prev = has ? po[lane + 32 * v] : 0.f;
-      po[lane + 32 * v] = (o[v] * ca + cb * prev) / lt;
+    for (int rr = 0; rr < RB; ++rr) {
+      if (rr >= nr) break;
+      const int n = q_perm[(int64_t)p * g.N + rb + rr];
+      const int64_t at = (int64_t)p * g.N + n;
+      const float L = part_lse[at];
+      float *po = part_o + at * DV;
+      const bool has = L > -CUDART_INF_F;
+      const float mn = has ? fmaxf(m[rr], L) : m[rr];
+      const float ca = expf(m[rr] - mn), cb = has ? expf(L - mn) : 0.f;
+      const float lt = l[rr] * ca + cb;
+#pragma unroll
+      for (int v = 0; v < PV; ++v) {
+        const float prev = has ? po[lane + 32 * v] : 0.f;
+        po[lane + 32 * v] = (o[rr][v] * ca + cb * prev) / lt;
+      }
+      __syncwarp();
+      if (lane == 0) part_lse[at] = mn + logf(lt);
     }
-    __syncwarp();
-    if (lane == 0) part_lse[at] = mn + logf(lt);
   }
 }
 
@@ -943,9 +995,17 @@ static cudaError_t run_tc(const void *Q, const void *K, const void *V, const mus
                              status, st)) != cudaSuccess)
     return e;
   if ((e = profile_mark(false, st)) != cudaSuccess) return e;
-  ret_runs<D, DV><<<(unsigned)(((int64_t)g.nb * g.Cq * P + 7) / 8), 256, 0, st>>>(
-      g, P, d.scale, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V,
-      w.q.perm, w.q.offsets, w.qpend, w.k.perm, w.k.offsets, w.pend, w.sel, w.part_o, w.part_lse);
+  {
+    using Rc = RunsCfg<D, DV>;
+    if ((e = cudaFuncSetAttribute(ret_runs<D, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)Rc::smem)) != cudaSuccess)
+      return e;
+    ret_runs<D, DV><<<(unsigned)(((int64_t)g.nb * g.Cq * P + Rc::WPC - 1) / Rc::WPC), Rc::WPC * 32,
+                      Rc::smem, st>>>(
+        g, P, d.scale, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)w.ks.rows,
+        (const __nv_bfloat16 *)V, w.q.perm, w.q.offsets, w.qpend, w.k.perm, w.k.offsets, w.pend,
+        w.sel, w.part_o, w.part_lse);
+  }
   count_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return run_diag_merge(Q, K, V, d.dtype, D, DV, d.N, P, g.S, -1, d.scale, w.part_o, w.part_lse, O,
