@@ -650,19 +650,32 @@ ret_coeffs(Geo g, float scale, const int32_t *__restrict__ q_perm,
 // part_lse[p][n], part_o[p][n][:] become the joint (log-normaliser, normalised output) of
 // the remainder and the runs.  One warp per (problem, i, b) group, no block-wide
 // barrier.  The warp lists the runs (lanes over the slots, a shuffle scan of their
-// lengths); the runs are the same for every row of the group, so their keys are staged
-// once per chunk of 32 into the warp's shared memory (the keys as sorted, contiguous
-// inside a run; the values by token) and serve up to RB rows at a time: lane k forms the
-// logit of key k against each row's query, the warp updates each row's online softmax,
-// and lanes over output columns accumulate p_k v_k from the staged values.
+// lengths); the runs are the same for every row of the group.  Up to 16 rows at a time
+// form the M side of warp-level tensor-core products (mma.sync m16n8k16, bfloat16 in,
+// float32 accumulate), over chunks of 32 selected keys staged in the warp's shared memory
+// (keys as sorted, contiguous inside a run; values by token, transposed):
+//   S = Q_rows . K_chunk^T (scaled),  online softmax per row,  O += P . V_chunk
+// with P (bfloat16) taken from S's accumulator fragments as the A operand.
 template <int D, int DV> struct RunsCfg {
-  static constexpr int WPC = D == 64 && DV == 64 ? 8 : 4;  // warps (groups) per CTA
-  static constexpr int KS = D + 2;                          // staged key row (bf16): 4-byte
-                                                            // reads of lane k hit bank k + d/2
-  static constexpr int RB = 4;                              // rows per pass over the keys
-  static constexpr size_t warp_bytes = (size_t)32 * KS * 2 + (size_t)32 * DV * 2 + (size_t)RB * D * 4;
+  static constexpr int WPC = 4;       // warps (groups) per CTA
+  static constexpr int QS = D + 8;    // staged row strides (bf16): 4-byte fragment loads of a
+  static constexpr int KS = D + 8;    // quad's 8 rows hit distinct banks
+  static constexpr int VS = 32 + 8;   // transposed values: [DV][VS]
+  static constexpr size_t warp_bytes = ((size_t)16 * QS + 32 * KS + (size_t)DV * VS) * 2;
   static constexpr size_t smem = WPC * warp_bytes;
 };
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
 
 template <int D, int DV>
 __global__ void __launch_bounds__(RunsCfg<D, DV>::WPC * 32)
@@ -673,14 +686,15 @@ ret_runs(Geo g, int P, float scale, const __nv_bfloat16 *__restrict__ Q, const _
          const int32_t *__restrict__ pend, const int32_t *__restrict__ sel,
          float *__restrict__ part_o, float *__restrict__ part_lse) {
   using Cf = RunsCfg<D, DV>;
-  constexpr int PV = DV / 32, KS = Cf::KS, RB = Cf::RB;
+  constexpr int QS = Cf::QS, KS = Cf::KS, VS = Cf::VS, NV = DV / 8;
   extern __shared__ float4 runs_smem[];
   __shared__ int runs[Cf::WPC][64], cum[Cf::WPC][65];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;  // fragment row group and thread in group
   unsigned char *wbase = reinterpret_cast<unsigned char *>(runs_smem) + warp * Cf::warp_bytes;
-  __nv_bfloat16 *Ksh = reinterpret_cast<__nv_bfloat16 *>(wbase);            // [32][KS]
-  __nv_bfloat16 *Vsh = Ksh + 32 * KS;                                       // [32][DV]
-  float *qsh = reinterpret_cast<float *>(Vsh + 32 * DV);                    // [RB][D]
+  __nv_bfloat16 *sQ = reinterpret_cast<__nv_bfloat16 *>(wbase);  // [16][QS]
+  __nv_bfloat16 *sK = sQ + 16 * QS;                                // [32][KS]
+  __nv_bfloat16 *sV = sK + 32 * KS;                                // [DV][VS] (transposed)
   const int64_t gid = (int64_t)blockIdx.x * Cf::WPC + warp;  // (p, i, b)
   if (gid >= (int64_t)g.nb * g.Cq * P) return;  // whole warps
   const int b = (int)(gid % g.nb), i = (int)((gid / g.nb) % g.Cq), p = (int)(gid / ((int64_t)g.nb * g.Cq));
@@ -726,104 +740,164 @@ ret_runs(Geo g, int P, float scale, const __nv_bfloat16 *__restrict__ Q, const _
   const int total = cum[warp][64];
   if (total == 0) return;
   const int32_t *kperm = k_perm + (int64_t)p * g.N;
-  for (int rb = r0; rb < r1; rb += RB) {
-    const int nr = min(RB, r1 - rb);
-    // the batch's queries (scaled), rows past the batch repeat its first row
+  for (int rb = r0; rb < r1; rb += 16) {
+    const int nr = min(16, r1 - rb);
+    // the tile's query rows (rows past the group repeat its first row)
     __syncwarp();
-    for (int x = lane; x < RB * D; x += 32) {
-      const int rr = x / D, d = x % D;
+    for (int x = lane; x < 16 * (D / 8); x += 32) {
+      const int rr = x / (D / 8), c = x % (D / 8);
       const int n = q_perm[(int64_t)p * g.N + rb + (rr < nr ? rr : 0)];
-      qsh[x] = __bfloat162float(Q[((int64_t)p * g.N + n) * D + d]) * scale;
+      const uint4 v = reinterpret_cast<const uint4 *>(Q + ((int64_t)p * g.N + n) * D)[c];
+      uint32_t *dst = reinterpret_cast<uint32_t *>(sQ + rr * QS + 8 * c);
+      dst[0] = v.x;
+      dst[1] = v.y;
+      dst[2] = v.z;
+      dst[3] = v.w;
     }
-    float m[RB], l[RB], o[RB][PV];
+    // rows gq and gq + 8 of the tile: running maximum and sum, output fragments
+    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
+    float o[NV][4];
 #pragma unroll
-    for (int rr = 0; rr < RB; ++rr) {
-      m[rr] = -CUDART_INF_F;
-      l[rr] = 0.f;
+    for (int nt = 0; nt < NV; ++nt)
 #pragma unroll
-      for (int v = 0; v < PV; ++v) o[rr][v] = 0.f;
-    }
+      for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
     int run = 0;  // run of this lane's key (the lane's keys only move forward)
     for (int c0 = 0; c0 < total; c0 += 32) {
-      const int gi = c0 + lane, cnt = min(32, total - c0);
-      __syncwarp();  // the previous chunk's keys and values are consumed
-      if (gi < total) {
-        while (cum[warp][run + 1] <= gi) ++run;
-        const int pos = runs[warp][run] + gi - cum[warp][run];  // sorted key position
-        const int tok = kperm[pos];
-        const uint4 *kr = reinterpret_cast<const uint4 *>(ks + ((int64_t)p * g.N + pos) * D);
-        uint32_t *kd = reinterpret_cast<uint32_t *>(Ksh + lane * KS);  // 4-byte aligned rows
+      const int gi = c0 + lane;
+      __syncwarp();  // the previous chunk is consumed (and the query tile is written)
+      // lane k stages key k of the chunk (zero past the selected keys)
+      {
+        uint4 kv[D / 8], vv[DV / 8];
+        if (gi < total) {
+          while (cum[warp][run + 1] <= gi) ++run;
+          const int pos = runs[warp][run] + gi - cum[warp][run];  // sorted key position
+          const int tok = kperm[pos];
+          const uint4 *kr = reinterpret_cast<const uint4 *>(ks + ((int64_t)p * g.N + pos) * D);
+          const uint4 *vr = reinterpret_cast<const uint4 *>(V + ((int64_t)p * g.N + tok) * DV);
+#pragma unroll
+          for (int u = 0; u < D / 8; ++u) kv[u] = kr[u];
+#pragma unroll
+          for (int u = 0; u < DV / 8; ++u) vv[u] = vr[u];
+        } else {
+#pragma unroll
+          for (int u = 0; u < D / 8; ++u) kv[u] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int u = 0; u < DV / 8; ++u) vv[u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        uint32_t *kd = reinterpret_cast<uint32_t *>(sK + lane * KS);
 #pragma unroll
         for (int u = 0; u < D / 8; ++u) {
-          const uint4 w4 = kr[u];
-          kd[4 * u] = w4.x;
-          kd[4 * u + 1] = w4.y;
-          kd[4 * u + 2] = w4.z;
-          kd[4 * u + 3] = w4.w;
+          kd[4 * u] = kv[u].x;
+          kd[4 * u + 1] = kv[u].y;
+          kd[4 * u + 2] = kv[u].z;
+          kd[4 * u + 3] = kv[u].w;
         }
-        const uint4 *vr = reinterpret_cast<const uint4 *>(V + ((int64_t)p * g.N + tok) * DV);
-        uint4 *vd = reinterpret_cast<uint4 *>(Vsh + lane * DV);
 #pragma unroll
-        for (int u = 0; u < DV / 8; ++u) vd[u] = vr[u];
+        for (int u = 0; u < DV / 8; ++u) {
+          const __nv_bfloat16 *h = reinterpret_cast<const __nv_bfloat16 *>(&vv[u]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) sV[(8 * u + e) * VS + lane] = h[e];
+        }
       }
       __syncwarp();
-      // logits of the lane's key against each row of the batch
-      float x[RB];
+      // S = Q . K^T: 16 rows x 32 keys (four n-tiles of 8)
+      float sacc[4][4];
 #pragma unroll
-      for (int rr = 0; rr < RB; ++rr) x[rr] = 0.f;
-      if (gi < total) {
-        const __nv_bfloat162 *kk = reinterpret_cast<const __nv_bfloat162 *>(Ksh + lane * KS);
-#pragma unroll 8
-        for (int u = 0; u < D / 2; ++u) {
-          const float2 kf = __bfloat1622float2(kk[u]);
+      for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-          for (int rr = 0; rr < RB; ++rr)
-            x[rr] = fmaf(qsh[rr * D + 2 * u], kf.x, fmaf(qsh[rr * D + 2 * u + 1], kf.y, x[rr]));
+        for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t a[4];
+        a[0] = *reinterpret_cast<const uint32_t *>(sQ + gq * QS + kk * 16 + 2 * tq);
+        a[1] = *reinterpret_cast<const uint32_t *>(sQ + (gq + 8) * QS + kk * 16 + 2 * tq);
+        a[2] = *reinterpret_cast<const uint32_t *>(sQ + gq * QS + kk * 16 + 8 + 2 * tq);
+        a[3] = *reinterpret_cast<const uint32_t *>(sQ + (gq + 8) * QS + kk * 16 + 8 + 2 * tq);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+          const __nv_bfloat16 *kr = sK + (nt * 8 + gq) * KS + kk * 16 + 2 * tq;
+          mma_bf16_16816(sacc[nt], a, *reinterpret_cast<const uint32_t *>(kr),
+                         *reinterpret_cast<const uint32_t *>(kr + 8));
         }
       }
-      float pk[RB];
+      // online softmax of rows gq (elements 0, 1) and gq + 8 (elements 2, 3); key of
+      // element e of n-tile nt: nt * 8 + 2 * tq + (e & 1)
+      float mx0 = m0, mx1 = m1;
 #pragma unroll
-      for (int rr = 0; rr < RB; ++rr) {
-        const float xv = gi < total ? x[rr] : -CUDART_INF_F;
-        const float mn = fmaxf(m[rr], warp_max(xv));
-        const float corr = expf(m[rr] - mn);
-        pk[rr] = gi < total ? expf(xv - mn) : 0.f;
-        l[rr] = l[rr] * corr + warp_sum(pk[rr]);
+      for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int v = 0; v < PV; ++v) o[rr][v] *= corr;
-        m[rr] = mn;
+        for (int e = 0; e < 4; ++e) {
+          const bool in = c0 + nt * 8 + 2 * tq + (e & 1) < total;
+          sacc[nt][e] = in ? sacc[nt][e] * scale : -CUDART_INF_F;
+          if (e < 2) mx0 = fmaxf(mx0, sacc[nt][e]);
+          else mx1 = fmaxf(mx1, sacc[nt][e]);
+        }
+#pragma unroll
+      for (int o2 = 1; o2 < 4; o2 <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
       }
-      for (int k = 0; k < cnt; ++k) {
-        float vv[PV];
+      const float cr0 = expf(m0 - mx0), cr1 = expf(m1 - mx1);  // (m = -inf: 0)
+      float s0 = 0.f, s1 = 0.f;
+      uint32_t pa[2][4];  // P as the A operand of two k-steps of 16 keys
 #pragma unroll
-        for (int v = 0; v < PV; ++v) vv[v] = __bfloat162float(Vsh[k * DV + lane + 32 * v]);
+      for (int nt = 0; nt < 4; ++nt) {
+        const float p0 = expf(sacc[nt][0] - mx0), p1 = expf(sacc[nt][1] - mx0);
+        const float p2 = expf(sacc[nt][2] - mx1), p3 = expf(sacc[nt][3] - mx1);
+        s0 += p0 + p1;
+        s1 += p2 + p3;
+        pa[nt >> 1][(nt & 1) * 2] = pack_bf16(p0, p1);
+        pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
+      }
 #pragma unroll
-        for (int rr = 0; rr < RB; ++rr) {
-          const float pkk = __shfl_sync(0xffffffffu, pk[rr], k);
+      for (int o2 = 1; o2 < 4; o2 <<= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o2);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o2);
+      }
+      l0 = l0 * cr0 + s0;
+      l1 = l1 * cr1 + s1;
+      m0 = mx0;
+      m1 = mx1;
 #pragma unroll
-          for (int v = 0; v < PV; ++v) o[rr][v] = fmaf(pkk, vv[v], o[rr][v]);
+      for (int nt = 0; nt < NV; ++nt) {
+        o[nt][0] *= cr0;
+        o[nt][1] *= cr0;
+        o[nt][2] *= cr1;
+        o[nt][3] *= cr1;
+      }
+      // O += P . V: two k-steps of 16 keys, NV n-tiles of 8 output columns
+#pragma unroll
+      for (int ks2 = 0; ks2 < 2; ++ks2) {
+#pragma unroll
+        for (int nt = 0; nt < NV; ++nt) {
+          const __nv_bfloat16 *vr = sV + (nt * 8 + gq) * VS + ks2 * 16 + 2 * tq;
+          mma_bf16_16816(o[nt], pa[ks2], *reinterpret_cast<const uint32_t *>(vr),
+                         *reinterpret_cast<const uint32_t *>(vr + 8));
         }
       }
     }
-    // joint softmax with the remainder partial of each row
+    // joint softmax with the remainder partial of each row: this thread holds columns
+    // nt * 8 + 2 tq (+1) of rows gq and gq + 8
 #pragma unroll
-    for (int rr = 0; rr < RB; ++rr) {
-      if (rr >= nr) break;
+    for (int h = 0; h < 2; ++h) {
+      const int rr = gq + 8 * h;
+      if (rr >= nr) continue;
+      const float m = h ? m1 : m0, l = h ? l1 : l0;
       const int n = q_perm[(int64_t)p * g.N + rb + rr];
       const int64_t at = (int64_t)p * g.N + n;
       const float L = part_lse[at];
       float *po = part_o + at * DV;
       const bool has = L > -CUDART_INF_F;
-      const float mn = has ? fmaxf(m[rr], L) : m[rr];
-      const float ca = expf(m[rr] - mn), cb = has ? expf(L - mn) : 0.f;
-      const float lt = l[rr] * ca + cb;
+      const float mn = has ? fmaxf(m, L) : m;
+      const float ca = expf(m - mn), cb = has ? expf(L - mn) : 0.f;
+      const float lt = l * ca + cb;
 #pragma unroll
-      for (int v = 0; v < PV; ++v) {
-        const float prev = has ? po[lane + 32 * v] : 0.f;
-        po[lane + 32 * v] = (o[rr][v] * ca + cb * prev) / lt;
+      for (int nt = 0; nt < NV; ++nt) {
+        float2 *dst = reinterpret_cast<float2 *>(po + nt * 8 + 2 * tq);
+        const float2 prev = has ? *dst : make_float2(0.f, 0.f);
+        *dst = make_float2((o[nt][2 * h] * ca + cb * prev.x) / lt, (o[nt][2 * h + 1] * ca + cb * prev.y) / lt);
       }
-      __syncwarp();
-      if (lane == 0) part_lse[at] = mn + logf(lt);
+      if (tq == 0) part_lse[at] = mn + logf(lt);
     }
   }
 }
