@@ -106,15 +106,19 @@ coef_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ MuseT
         float scale, const int32_t *__restrict__ q_offsets, const float *__restrict__ logZ,
         const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
         float *__restrict__ lse, const __grid_constant__ InstMask skip, float sdip,
-        const __grid_constant__ CoefOut oa, int *status) {
+        const __grid_constant__ CoefOut oa, const __grid_constant__ BlockMap bm, int *status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Smem<D, CK, OUT> &sm = *reinterpret_cast<Smem<D, CK, OUT> *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
+  // blockIdx.x: a chunk slot of one instance (compact grid over this kernel's instances),
+  // blockIdx.y: the problem
+  int bfirst;
+  const int p = blockIdx.y, s = map_block(bm, mt.in.ninst, blockIdx.x, bfirst);
+  const int chunk = (int)blockIdx.x - bfirst;
   if ((skip.w[s >> 5] >> (s & 31)) & 1u) return;  // uniform: another kernel's instance
   const Task q = make_task(mt.q, p * mt.q.nseg + s), k = make_task(mt.k, p * mt.k.nseg + s);
-  // this CTA's chunk: chunk blockIdx.x of the instance, counting ceil(rows / 128) chunks
+  // this CTA's chunk of the instance, counting ceil(rows / 128) chunks
   // per query cluster in cluster order
   if (warp == 0) {
     int run = 0, found = -1, fr0 = 0;
@@ -132,12 +136,12 @@ coef_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ MuseT
         if (lane >= o) inc += y;
       }
       const int first = run + inc - nch;
-      const bool mine = (int)blockIdx.x >= first && (int)blockIdx.x < first + nch;
+      const bool mine = chunk >= first && chunk < first + nch;
       const unsigned bal = __ballot_sync(0xffffffffu, mine);
       if (bal) {
         const int src = __ffs(bal) - 1;
         found = __shfl_sync(0xffffffffu, c, src);
-        fr0 = __shfl_sync(0xffffffffu, bb + TM * ((int)blockIdx.x - first), src);
+        fr0 = __shfl_sync(0xffffffffu, bb + TM * (chunk - first), src);
       }
       run += __shfl_sync(0xffffffffu, inc, 31);
     }
@@ -418,10 +422,20 @@ static cudaError_t launch(const MuseTables &mt, int P, float scale, const void *
   auto kern = coef_tc<D, CK, OUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  // chunks of an instance: at most rows / 128 + one partial chunk per cluster
-  const int gx = (mt.q.max_rows + TM - 1) / TM + std::min(mt.q.max_C, mt.q.max_rows);
-  kern<<<dim3(gx, P * mt.in.ninst), 2 * TM, smem, st>>>(mq, mt, scale, q_offsets, b.logZ, b.mu_k,
-                                                         b.c0, b.c1, b.lse, skip, sdip, oa, status);
+  // chunk slots of an instance (none for the skipped ones): at most ceil(rows / 128) + one
+  // partial chunk per cluster
+  BlockMap bm;
+  bm.pre[0] = 0;
+  for (int si = 0; si < mt.in.ninst; ++si) {
+    const bool mine = !((skip.w[si >> 5] >> (si & 31)) & 1u);
+    const int n = mt.q.nrow[si];
+    bm.pre[si + 1] = bm.pre[si] + (mine ? (n + TM - 1) / TM + std::min(mt.q.C[si], n) : 0);
+  }
+  for (int si = mt.in.ninst + 1; si <= kMaxSeg; ++si) bm.pre[si] = bm.pre[mt.in.ninst];
+  bm.total = bm.pre[mt.in.ninst];
+  if (bm.total == 0) return cudaSuccess;
+  kern<<<dim3(bm.total, P), 2 * TM, smem, st>>>(mq, mt, scale, q_offsets, b.logZ, b.mu_k, b.c0, b.c1,
+                                                b.lse, skip, sdip, oa, bm, status);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -116,11 +116,12 @@ block_prefix_lse(Geo g, int P, const float *__restrict__ logZb, float *__restric
 }
 
 // One warp per (p, i, b): the selection and the remainder log-normalisers.
-// sel[p][i][b][slot] = (j, b'), slot = t*k2 + u; logZR[p][i][b][j].
+// sel[p][i][b][slot] = (j, b'), slot = t*k2 + u; logZR[p][i][b][j].  MAXJ: key clusters per
+// lane (Ck <= 32 MAXJ).
+template <int MAXJ>
 __global__ void __launch_bounds__(256)
 select_blocks(Geo g, int P, const float *__restrict__ logZb, const float *__restrict__ pref,
               int32_t *__restrict__ sel, float *__restrict__ logZR) {
-  constexpr int MAXJ = kMaxClusters / 32;  // clusters per lane
   const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (wid >= (int64_t)P * g.Cq * g.nb) return;
@@ -222,6 +223,17 @@ select_blocks(Geo g, int P, const float *__restrict__ logZb, const float *__rest
     }
     zr[j] = acc;
   }
+}
+
+static void launch_select(const Geo &g, int P, int64_t ns, const float *logZb, const float *pref,
+                          int32_t *sel, float *logZR, cudaStream_t st) {
+  const unsigned grid = (unsigned)((ns + 7) / 8);
+  if (g.Ck <= 128)
+    select_blocks<4><<<grid, 256, 0, st>>>(g, P, logZb, pref, sel, logZR);
+  else if (g.Ck <= 256)
+    select_blocks<8><<<grid, 256, 0, st>>>(g, P, logZb, pref, sel, logZR);
+  else
+    select_blocks<kMaxClusters / 32><<<grid, 256, 0, st>>>(g, P, logZb, pref, sel, logZR);
 }
 
 // Excluded blocks of cluster j for a query whose selection row is `so` (<= 64 slots).
@@ -474,8 +486,9 @@ exact_merge(Geo g, float scale, const T *__restrict__ Q, const T *__restrict__ K
 // (i, b).  A running sum m1_j = sum_{b' < b} sum_{k in (j, b')} W_ik k over the key blocks
 // gives qt_r.m1_j; a selected cluster's runs are summed once per (i, b) group into e_j
 // and qt_r.(m1_j - e_j) is taken (float32).  One CTA per (problem, query cluster i, group
-// of JPC key clusters); DP = D / 32 threads per cluster, 32 coordinates each; no
-// block-wide barrier (a thread's work varies with its cluster's keys per block).
+// of JPC key clusters); DP = D / 8 threads per cluster, 8 coordinates each (few registers,
+// so many warps hide the latency of the block-by-block walk); no block-wide barrier (a
+// thread's work varies with its cluster's keys per block).
 template <int D>
 __global__ void __launch_bounds__(256)
 ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q_offsets,
@@ -483,7 +496,7 @@ ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q
       const int32_t *__restrict__ k_offsets, const int32_t *__restrict__ pend,
       const float *__restrict__ W, int w_stride, const int32_t *__restrict__ sel,
       float *__restrict__ Tout) {
-  constexpr int DP = D / 32, JPC = 256 / DP;
+  constexpr int CPT = 8, DP = D / CPT, JPC = 256 / DP;
   const int p = blockIdx.z, i = blockIdx.y;
   const int jl = threadIdx.x / DP, dp = threadIdx.x % DP;
   const int j = blockIdx.x * JPC + jl;
@@ -494,28 +507,22 @@ ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q
   const int32_t *pe = pend + ((int64_t)p * g.Ck + jj) * (g.nb + 1);
   const int kbase = k_offsets[(int64_t)p * (g.Ck + 1) + jj];
   const float *wrow = W + (int64_t)p * w_stride + (int64_t)i * w_ld(g.N);
-  const __nv_bfloat16 *kp = ks + (int64_t)p * g.N * D + dp * 32;
+  const __nv_bfloat16 *kp = ks + (int64_t)p * g.N * D + dp * CPT;
   const __nv_bfloat16 *qp = qs + (int64_t)p * g.N * D;
   float *tout = Tout + ((int64_t)p * g.Ck + jj) * g.N;
   const int r_first = qo[i];
-  float m1[32];
+  float m1[CPT];
 #pragma unroll
-  for (int d = 0; d < 32; ++d) m1[d] = 0.f;
-  // acc[d] += w * key[dp * 32 + d] for the key at sorted position pos
-  auto add_key = [&](int pos, float w, float (&acc)[32]) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(kp + (int64_t)pos * D);
-    uint4 u[4];
+  for (int d = 0; d < CPT; ++d) m1[d] = 0.f;
+  // acc[d] += w * key[dp * CPT + d] for the key at sorted position pos
+  auto add_key = [&](int pos, float w, float (&acc)[CPT]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(kp + (int64_t)pos * D);
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int v = 0; v < 4; ++v) u[v] = src[v];
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const uint32_t w4[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
-        acc[8 * v + 2 * h] = fmaf(w, __low2float(b2), acc[8 * v + 2 * h]);
-        acc[8 * v + 2 * h + 1] = fmaf(w, __high2float(b2), acc[8 * v + 2 * h + 1]);
-      }
+    for (int h = 0; h < 4; ++h) {
+      const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
+      acc[2 * h] = fmaf(w, __low2float(b2), acc[2 * h]);
+      acc[2 * h + 1] = fmaf(w, __high2float(b2), acc[2 * h + 1]);
     }
   };
   for (int b = 0; b < g.nb; ++b) {
@@ -538,9 +545,9 @@ ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q
     if (b > 0 && live)
       for (int t = 0; t < g.k1; ++t)
         if (so[2 * t * g.k2] == j) tj = t;
-    float ex[32];
+    float ex[CPT];
 #pragma unroll
-    for (int d = 0; d < 32; ++d) ex[d] = 0.f;
+    for (int d = 0; d < CPT; ++d) ex[d] = 0.f;
     if (tj >= 0) {
       for (int u = 0; u < g.k2; ++u) {
         const int bb = so[2 * (tj * g.k2 + u) + 1];
@@ -548,25 +555,18 @@ ret_T(Geo g, const __nv_bfloat16 *__restrict__ qs, const int32_t *__restrict__ q
         for (int pos = kbase + pe[bb]; pos < kbase + pe[bb + 1]; ++pos) add_key(pos, wrow[pos], ex);
       }
     }
-    // every row of the group: qt.(m1 - e), the thread's 32 coordinates read straight from
-    // the sorted residuals (the same addresses for every thread of a half: L1 broadcast)
+    // every row of the group: qt.(m1 - e), the thread's CPT coordinates read straight from
+    // the sorted residuals (the same addresses for the threads of a coordinate slice)
     for (int r = r0; r < r1; ++r) {
       float acc = 0.f;
       if (b > 0) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(qp + (int64_t)r * D + dp * 32);
-        uint4 u[4];
+        const uint4 u = *reinterpret_cast<const uint4 *>(qp + (int64_t)r * D + dp * CPT);
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int v = 0; v < 4; ++v) u[v] = src[v];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint32_t w4[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
-            const int d = 8 * v + 2 * h;
-            acc = fmaf(__low2float(b2), m1[d] - ex[d], acc);
-            acc = fmaf(__high2float(b2), m1[d + 1] - ex[d + 1], acc);
-          }
+        for (int h = 0; h < 4; ++h) {
+          const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w4[h]);
+          acc = fmaf(__low2float(b2), m1[2 * h] - ex[2 * h], acc);
+          acc = fmaf(__high2float(b2), m1[2 * h + 1] - ex[2 * h + 1], acc);
         }
       }
 #pragma unroll
@@ -1051,8 +1051,8 @@ static cudaError_t run_tc(const void *Q, const void *K, const void *V, const mus
                                                                   w.k.offsets, w.pend, w.logZb);
   block_prefix_lse<<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(g, P, w.logZb, w.pref);
   const int64_t ns = (int64_t)P * g.Cq * g.nb;
-  select_blocks<<<(unsigned)((ns + 7) / 8), 256, 0, st>>>(g, P, w.logZb, w.pref, w.sel, w.logZR);
-  constexpr int JPC = 256 / (D / 32);
+  launch_select(g, P, ns, w.logZb, w.pref, w.sel, w.logZR, st);
+  constexpr int JPC = 256 / (D / 8);  // (ret_T: 8 coordinates per thread)
   ret_T<D><<<dim3((g.Ck + JPC - 1) / JPC, g.Cq, P), 256, 0, st>>>(
       g, (const __nv_bfloat16 *)w.qs.rows, w.q.offsets, w.qpend, (const __nv_bfloat16 *)w.ks.rows,
       w.k.offsets, w.pend, w.W, mt.in.w_stride, w.sel, w.T);
@@ -1118,7 +1118,7 @@ static cudaError_t run_t(const void *Q, const void *K, const void *V, const muse
                                                                   w.k.offsets, w.pend, w.logZb);
   block_prefix_lse<<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(g, P, w.logZb, w.pref);
   const int64_t ns = (int64_t)P * g.Cq * g.nb;
-  select_blocks<<<(unsigned)((ns + 7) / 8), 256, 0, st>>>(g, P, w.logZb, w.pref, w.sel, w.logZR);
+  launch_select(g, P, ns, w.logZb, w.pref, w.sel, w.logZR, st);
   dim3 qg(d.N / 64, P);
   remainder_pass<T, D, DV, 0><<<qg, 256, 0, st>>>(
       g, (const T *)Q, w.q.centroids, w.q.labels, (const T *)w.ks.rows, (const T *)w.vs, w.k.perm,

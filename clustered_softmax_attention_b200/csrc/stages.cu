@@ -803,7 +803,7 @@ __global__ void __launch_bounds__(256)
 refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
                     const int32_t *__restrict__ q_offsets, const float *__restrict__ logZ,
                     const float *__restrict__ mu_k, float *__restrict__ c0, float *__restrict__ c1,
-                    float *__restrict__ lse, InstMask skip, float sdip) {
+                    float *__restrict__ lse, InstMask skip, float sdip, const __grid_constant__ BlockMap bm) {
   constexpr int CJ = 16 * JPT;                         // key clusters (all of them)
   constexpr int MSD = D + 4;                           // row stride of the means (floats)
   constexpr int QRB = D * (int)sizeof(T) + 16;         // row stride of the raw rows (bytes)
@@ -811,7 +811,11 @@ refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
   float *Ms = reinterpret_cast<float *>(tiled_smem);   // [CJ][MSD] tilted key means of cluster i
   float *lz = Ms + CJ * MSD;                           // [CJ]
   unsigned char *Qr = reinterpret_cast<unsigned char *>(lz + CJ);  // [64][QRB] residual rows
-  const int p = blockIdx.y / mt.in.ninst, s = blockIdx.y % mt.in.ninst;
+  // blockIdx.x: a chunk slot of one instance (compact grid over this kernel's instances),
+  // blockIdx.y: the problem
+  int bfirst;
+  const int p = blockIdx.y, s = map_block(bm, mt.in.ninst, blockIdx.x, bfirst);
+  const int chunk = (int)blockIdx.x - bfirst;
   if ((skip.w[s >> 5] >> (s & 31)) & 1u) return;  // uniform: another kernel's instance
   const Task q = q_task(mt, p, s), k = k_task(mt, p, s);
   // this CTA's 64-row chunk: chunk g of the instance, counting ceil(rows/64) chunks
@@ -835,12 +839,12 @@ refine_coeffs_tiled(MuseTables mt, float scale, const T *__restrict__ qt_rows,
         if (lane >= o) inc += y;
       }
       const int first = run + inc - nch;  // chunk index of this cluster's first chunk
-      const bool mine = (int)blockIdx.x >= first && (int)blockIdx.x < first + nch;
+      const bool mine = chunk >= first && chunk < first + nch;
       const unsigned bal = __ballot_sync(0xffffffffu, mine);
       if (bal) {
         const int src = __ffs(bal) - 1;
         found = __shfl_sync(0xffffffffu, c, src);
-        fr0 = __shfl_sync(0xffffffffu, (bb & ~3) + 64 * ((int)blockIdx.x - first), src);
+        fr0 = __shfl_sync(0xffffffffu, (bb & ~3) + 64 * (chunk - first), src);
       }
       run += __shfl_sync(0xffffffffu, inc, 31);
     }
@@ -1481,10 +1485,19 @@ static cudaError_t coeffs_tiled_t(const MuseTables &mt, int P, float scale, Sort
   cudaError_t err = cudaFuncSetAttribute(refine_coeffs_tiled<T, D, JPT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  // chunks of an instance: at most rows/64 + one partial chunk per cluster
-  refine_coeffs_tiled<T, D, JPT><<<dim3((mt.q.max_rows + 63) / 64 + mt.q.max_C, P * mt.in.ninst), 256,
-                                  smem, st>>>(
-      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse, skip, sdip);
+  // chunk slots of an instance (none for the skipped ones): a cluster of n rows starting
+  // up to 3 rows past a 4-row boundary takes at most n / 64 + 2 chunks
+  BlockMap bm;
+  bm.pre[0] = 0;
+  for (int si = 0; si < mt.in.ninst; ++si) {
+    const bool mine = !((skip.w[si >> 5] >> (si & 31)) & 1u);
+    bm.pre[si + 1] = bm.pre[si] + (mine ? mt.q.nrow[si] / 64 + 2 * mt.q.C[si] : 0);
+  }
+  for (int si = mt.in.ninst + 1; si <= kMaxSeg; ++si) bm.pre[si] = bm.pre[mt.in.ninst];
+  bm.total = bm.pre[mt.in.ninst];
+  if (bm.total == 0) return cudaSuccess;
+  refine_coeffs_tiled<T, D, JPT><<<dim3(bm.total, P), 256, smem, st>>>(
+      mt, scale, (const T *)qs.rows, q_offsets, b.logZ, b.mu_k, b.c0, b.c1, b.lse, skip, sdip, bm);
   count_launches(1);
   return cudaGetLastError();
 }
