@@ -185,8 +185,9 @@ def algorithmic_flops(w):
 
 def summary_form_ablation(w):
     """Whether the library evaluates the monopole / partial-dipole ablations of this
-    workload in summary form (bfloat16, Dv = 64, D = 64 or 128, Ck <= 128)."""
-    return w.dtype == "bf16" and w.Dv == 64 and w.D in (64, 128) and w.Ck <= 128
+    workload in summary form (bfloat16, Dv = 64; D = 64 with Ck <= 256, D = 128 with
+    Ck <= 128)."""
+    return w.dtype == "bf16" and w.Dv == 64 and ((w.D == 64 and w.Ck <= 256) or (w.D == 128 and w.Ck <= 128))
 
 
 def summary_output_flops(w, partial):

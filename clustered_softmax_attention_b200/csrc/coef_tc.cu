@@ -164,7 +164,7 @@ coef_tc(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ MuseT
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // TMEM columns: U [0, CK); output mode: O [CK, CK + OV), P (packed) [CK + OV, CK + OV + CK / 2)
-  constexpr uint32_t kCols = OUT ? 256u : (uint32_t)CK;
+  constexpr uint32_t kCols = OUT ? (CK > 128 ? 512u : 256u) : (uint32_t)CK;
   constexpr uint32_t kO = CK, kP = CK + OV;
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -466,7 +466,7 @@ cudaError_t run_coef_tc(const MuseTables &mt, int D, int P, float scale, const v
 }
 
 bool coef_out_supported(int dtype, int D, int Dv, int maxCk) {
-  return dtype == MUSE_BF16 && (D == 64 || D == 128) && Dv == ctc::OV && maxCk <= 128;
+  return dtype == MUSE_BF16 && Dv == ctc::OV && ((D == 64 && maxCk <= 256) || (D == 128 && maxCk <= 128));
 }
 
 cudaError_t run_coef_out(const MuseTables &mt, int D, int N, int P, float scale, const void *qs_rows,
@@ -479,7 +479,8 @@ cudaError_t run_coef_out(const MuseTables &mt, int D, int N, int P, float scale,
   return ctc::launch<DD, CC, true>(mt, P, scale, qs_rows, q_offsets, b, all, 0.f, oa, status, st)
   if (D == 64) {
     if (ck <= 64) MUSE_OUT(64, 64);
-    MUSE_OUT(64, 128);
+    if (ck <= 128) MUSE_OUT(64, 128);
+    MUSE_OUT(64, 256);
   }
   if (ck <= 64) MUSE_OUT(128, 64);
   MUSE_OUT(128, 128);

@@ -193,8 +193,8 @@ muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims 
  *   (same review: "Axioms", the covariance taken without the tilt by the query
  *   centroid; "invented entities", an aggregated covariance per query cluster; the
  *   weights are not printed, this is the reading taken).
- * Both ablations need only the summaries: for bfloat16 with Dv = 64 (D = 64 or 128) and
- * Ck <= 128 they are evaluated in that form, O_n = sum_j p_j mu_v,ij (+ s Cbar_i qt_n),
+ * Both ablations need only the summaries: for bfloat16 with Dv = 64 (D = 64 with
+ * Ck <= 256, D = 128 with Ck <= 128) they are evaluated in that form, O_n = sum_j p_j mu_v,ij (+ s Cbar_i qt_n),
  * with the tilted value means mu_v and no contraction over all N keys; other shapes run
  * the pair form of muse_forward with the dipole coefficient set to zero (plus the
  * covariance correction).

@@ -261,10 +261,10 @@ def test_forward_end_to_end_small_f32(parity):
 # the monopole-only ablation (dipole term dropped) against the oracle's same mode, with
 # the GPU's clustering; it must be less accurate than the full method on these inputs
 # (bfloat16 with Dv = 64 evaluates it in summary form, without the N^2 contraction; C = 128
-# takes the output kernel's 128-cluster variant; D = Dv = 128 runs the pair form)
+# and 256 take the output kernel's wider variants; D = Dv = 128 runs the pair form)
 @pytest.mark.parametrize("dt,D,Dv,C", [("f32", 64, 64, 32), ("bf16", 64, 64, 32),
                                        ("bf16", 128, 128, 32), ("bf16", 64, 64, 128),
-                                       ("bf16", 128, 64, 128)])
+                                       ("bf16", 128, 64, 128), ("bf16", 64, 64, 256)])
 def test_forward_monopole_only(dt, D, Dv, C, parity):
     N, T = 2048, 6
     Q, K, V = mixture(9, 1, 2, N, D, Dv, 48, 0.5 / np.sqrt(D), dt)
