@@ -77,7 +77,10 @@ struct StageBufs {
   float *cov;      // [P][z_stride][Dv][D] (optional)
   float *c0, *c1;  // [P][c_stride]
   float *lse;      // [P][q.row_stride] logsumexp_j a_j per sorted query position
+  float *opart;    // [kSplitCtas][128][Dv] partial outputs of the refinement's split last wave
 };
+// The tensor-core refinement splits at most this many CTAs' key ranges (half an SM count).
+constexpr int kSplitCtas = 256;
 
 cudaError_t run_sort_side(const void *X, int dtype, int width, int N, const SegTable &tab, int P,
                           const int32_t *perm, const int32_t *offsets, const float *centroids,

@@ -190,6 +190,7 @@ static void plan_refine(Bump &bp, const MuseTables &mt, const muse_dims &d, int 
   r.sb.c0 = bp.take<float>((size_t)P * mt.in.c_stride);
   r.sb.c1 = bp.take<float>((size_t)P * mt.in.c_stride);
   r.sb.lse = bp.take<float>(qrows);
+  r.sb.opart = bp.take<float>((size_t)kSplitCtas * 128 * d.Dv);
 }
 
 struct KmWs {

@@ -57,6 +57,7 @@ constexpr int kSlots = 8;    // query clusters per CTA whose tilt weights are st
 constexpr int kTileSegs = 8; // key clusters packed into one tile at most
 constexpr int kComplex = 1 << 13;  // chunk code flag: more than two key clusters in 16 columns
 constexpr int kSBuf = 3;     // S buffers (tile t uses t % 3); P(t) is written over S(t) in place
+constexpr int kSplitSlots = kSplitCtas;  // key-range split: CTAs of half units at most
 
 // Widest key tile: 128 keys when D = Dv = 64, else 64 (shared memory budget).
 template <int D, int DV>
@@ -138,12 +139,15 @@ struct TileIter {
   const int32_t *off;
   const int32_t *live;
   int C;
+  int khi;  // keys from khi on are left to another CTA (a split key range)
   KTile t;
-  __device__ void begin(const int32_t *o, int Ck, const int32_t *lv = nullptr) {
+  __device__ void begin(const int32_t *o, int Ck, const int32_t *lv = nullptr, int klo = -1,
+                        int khi_ = 0x7fffffff) {
     off = o;
     live = lv;
     C = Ck;
-    make(0, off[0]);
+    khi = khi_;
+    make(0, klo >= 0 ? klo : off[0]);
   }
   // The window starting at key c, which lies in cluster j or a later one.
   __device__ void make(int j, int c) {
@@ -159,8 +163,12 @@ struct TileIter {
     t.j = j;
     t.c = c;
     if (j >= C) return;
+    if (c >= khi) {  // the range is done
+      t.j = C;
+      return;
+    }
     t.x0 = c & ~7;
-    int end = min(t.x0 + BN, off[C]);
+    int end = min(min(t.x0 + BN, off[C]), khi);
     if (j + kTileSegs < C) end = min(end, off[j + kTileSegs]);
     int last = j;  // cluster holding key end-1
     if (live) {
@@ -191,6 +199,16 @@ struct RetArgs {
   const int32_t *pend;         // [P][Ck][nb + 1] keys of cluster j in blocks < b'
   const int32_t *sel;          // [P][Cq][nb][K12][2] (cluster, block) pairs selected per (i, b)
   int S, nb, k1, k2, K12, Cq;
+};
+
+// The last wave's key-range split (single-instance output mode).  With tpp > 0 the grid
+// is one-dimensional over units (problem, 128-row tile), unit = p * tpp + tile: CTAs below
+// `full` take a whole unit; the 2 (units - full) CTAs after them take one half of the keys
+// of a unit each, writing float32 partial outputs to opart[slot][row][:] (slot = CTA -
+// full), which refine_halves adds (the pair form is a plain sum over the keys).
+struct SplitArgs {
+  int tpp, full;
+  float *opart;
 };
 
 // RET: columns of chunk cb whose key block precedes the row's block brow (the chunk's
@@ -279,15 +297,35 @@ refine_tc_body(const CUtensorMap &map_q, const CUtensorMap &map_k, const CUtenso
                const float *__restrict__ W, const float *__restrict__ c0g,
                const float *__restrict__ c1g, const float *__restrict__ lse,
                __nv_bfloat16 *__restrict__ O, float *__restrict__ part_o,
-               float *__restrict__ part_lse, int *status, const BlockMap &bm, const RetArgs &ra) {
+               float *__restrict__ part_lse, int *status, const BlockMap &bm, const RetArgs &ra,
+               const SplitArgs &sp) {
   constexpr int BN = TileCfg<D, DV>::BN;
-  // blockIdx.x: a 128-row block of one instance (compact grid), blockIdx.y: the problem
-  int bfirst;
-  const int p = blockIdx.y, s = map_block(bm, mt.in.ninst, blockIdx.x, bfirst);
+  // blockIdx.x: a 128-row block of one instance (compact grid), blockIdx.y: the problem;
+  // or, with the key-range split, a unit or half a unit (SplitArgs)
+  int p, s, r0, half = -1, pslot = 0;  // pslot: this CTA's slot of partial outputs
+  if (sp.tpp > 0) {
+    const int cta = (int)blockIdx.x;
+    int unit = cta;
+    if (cta >= sp.full) {
+      pslot = cta - sp.full;
+      unit = sp.full + (pslot >> 1);
+      half = pslot & 1;
+    }
+    p = unit / sp.tpp;
+    s = 0;
+    r0 = (unit % sp.tpp) * BM;
+  } else {
+    int bfirst;
+    p = blockIdx.y;
+    s = map_block(bm, mt.in.ninst, blockIdx.x, bfirst);
+    r0 = ((int)blockIdx.x - bfirst) * BM;
+  }
   const Task q = make_task(mt.q, p * mt.q.nseg + s);
   const Task k = make_task(mt.k, p * mt.k.nseg + s);
-  const int r0 = ((int)blockIdx.x - bfirst) * BM;
   if (r0 >= q.n) return;  // uniform: nothing allocated yet
+  // this CTA's keys: all, or one half of the instance's sorted keys
+  const int kmid = (k.n / 2) & ~7;
+  const int klo = half == 1 ? kmid : -1, khi = half == 0 ? kmid : 0x7fffffff;
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Smem<D, DV> &sm = *reinterpret_cast<Smem<D, DV> *>(
@@ -370,7 +408,7 @@ refine_tc_body(const CUtensorMap &map_q, const CUtensorMap &map_k, const CUtenso
       uint64_t *full = keys ? sm.fullk : sm.fullv;
       uint64_t *empty = keys ? sm.emptyk : sm.emptyv;
       TileIter<BN> it;
-      it.begin(koff, k.C, kend);
+      it.begin(koff, k.C, kend, klo, khi);
       int t = 0;
       for (; !it.done(); it.next(), ++t) {
         const KTile kt = it.get();
@@ -397,7 +435,7 @@ refine_tc_body(const CUtensorMap &map_q, const CUtensorMap &map_k, const CUtenso
     // warp kEWarp + par stages the tiles of parity par (stages par, par + 2, ...)
     const int par = warp - kEWarp;
     TileIter<BN> it;
-    it.begin(koff, k.C, kend);
+    it.begin(koff, k.C, kend, klo, khi);
     int t = 0;
     for (; !it.done(); it.next(), ++t) {
       if ((t & 1) != par) continue;
@@ -489,7 +527,7 @@ refine_tc_body(const CUtensorMap &map_q, const CUtensorMap &map_k, const CUtenso
       bool ok = mbar_wait<true>(&sm.qbar, 0, abort_flag, status);
       tc_fence_after();
       TileIter<BN> it;
-      it.begin(koff, k.C, kend);
+      it.begin(koff, k.C, kend, klo, khi);
       int g1 = 0, g2 = 0;  // next tile of each contraction
       int idle = 0;
       uint64_t t_idle = 0;
@@ -592,7 +630,7 @@ refine_tc_body(const CUtensorMap &map_q, const CUtensorMap &map_k, const CUtenso
     if constexpr (RET) asm volatile("bar.sync 2, %0;" ::"r"(32 * kEpiWarps) : "memory");
     const bool xfast = ra.k1 <= kSelReg && ra.K12 <= 16;  // selection held in registers/table
     TileIter<BN> it;
-    it.begin(koff, k.C, kend);
+    it.begin(koff, k.C, kend, klo, khi);
     int t = 0;
     bool ok = true;
     for (; !it.done(); it.next(), ++t) {
@@ -740,7 +778,11 @@ refine_tc_body(const CUtensorMap &map_q, const CUtensorMap &map_k, const CUtenso
         float o[16];
         tmem_ld16(tmem_o + lane_base + cb * 16, o);
         if (!valid) continue;
-        if (O) {
+        if (half >= 0) {  // half the keys: a float32 partial, added by refine_halves
+          float4 *dst = reinterpret_cast<float4 *>(sp.opart + ((int64_t)pslot * BM + r) * DV + cb * 16);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) dst[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+        } else if (O) {
           uint32_t pk[8];
 #pragma unroll
           for (int e = 0; e < 16; e += 2) {
@@ -769,6 +811,9 @@ refine_tc_body(const CUtensorMap &map_q, const CUtensorMap &map_k, const CUtenso
         float4 *dst = reinterpret_cast<float4 *>(part_o + rr * DV);
         for (int c = grp; c < DV / 4; c += 2) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (grp == 0) part_lse[rr] = lse[q.lab + n];
+      } else if (half >= 0) {  // a half with no keys: a zero partial
+        float4 *dst = reinterpret_cast<float4 *>(sp.opart + ((int64_t)pslot * BM + r) * DV);
+        for (int c = grp; c < DV / 4; c += 2) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
       } else if (grp == 0) {
         // an instance with no keys cannot occur (every key range is non-empty)
         report(status, MUSE_ERR_DEVICE);
@@ -795,9 +840,32 @@ refine_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                  const float *__restrict__ c0g, const float *__restrict__ c1g,
                  const float *__restrict__ lse, __nv_bfloat16 *__restrict__ O,
                  float *__restrict__ part_o, float *__restrict__ part_lse, int *status,
-                 const __grid_constant__ BlockMap bm, const RetArgs ra) {
+                 const __grid_constant__ BlockMap bm, const RetArgs ra, const SplitArgs sp) {
   refine_tc_body<D, DV, RET>(map_q, map_k, map_vt, mt, N, q_perm, q_cluster, k_offsets, W, c0g,
-                             c1g, lse, O, part_o, part_lse, status, bm, ra);
+                             c1g, lse, O, part_o, part_lse, status, bm, ra, sp);
+}
+
+// O rows of the split units: the two halves' float32 partials added, bf16, natural order.
+// One CTA per split unit, a thread per row.
+template <int DV>
+__global__ void __launch_bounds__(BM)
+refine_halves(MuseTables mt, int N, const int32_t *__restrict__ q_perm, const float *__restrict__ opart,
+              __nv_bfloat16 *__restrict__ O, SplitArgs sp) {
+  const int unit = sp.full + (int)blockIdx.x, p = unit / sp.tpp, r0 = (unit % sp.tpp) * BM;
+  const Task q = make_task(mt.q, p * mt.q.nseg);
+  const int n = r0 + (int)threadIdx.x;
+  if (n >= q.n) return;
+  const int row = q_perm[q.lab + n];
+  const float4 *a = reinterpret_cast<const float4 *>(opart + ((int64_t)(2 * blockIdx.x) * BM + threadIdx.x) * DV);
+  const float4 *b = reinterpret_cast<const float4 *>(opart + ((int64_t)(2 * blockIdx.x + 1) * BM + threadIdx.x) * DV);
+  uint2 *dst = reinterpret_cast<uint2 *>(O + ((int64_t)p * N + row) * DV);
+#pragma unroll 4
+  for (int u = 0; u < DV / 4; ++u) {
+    const float4 x = a[u], y = b[u];
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(x.x + y.x, x.y + y.y);
+    __nv_bfloat162 h1 = __floats2bfloat162_rn(x.z + y.z, x.w + y.w);
+    dst[u] = make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -820,10 +888,34 @@ static cudaError_t launch(const MuseTables &mt, int N, int P, SortedSide qs, con
   if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
   if (fa.maxThreadsPerBlock < kThreads) return cudaErrorLaunchOutOfResources;
   const BlockMap bm = make_block_map(mt.q, BM);
+  // One CTA per SM: with T units (problem, 128-row tile) the last wave holds T % SMs of them.
+  // In the single-instance output mode, when at most half an SM count is left over, those
+  // units are split into key halves so that the last wave is about full and half as long.
+  SplitArgs sp{0, 0, b.opart};
+  int dev = 0, sms = 0;
+  if (!RET && O && mt.in.ninst == 1 && b.opart && cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0) {
+    const int T = bm.total * P, R = T % sms;
+    if (R > 0 && 2 * R <= sms && 2 * R <= kSplitSlots && mt.k.nrow[0] >= 16) {
+      sp.tpp = bm.total;
+      sp.full = T - R;
+    }
+  }
+  cudaGetLastError();  // (attribute queries leave no error behind)
+  if (sp.tpp > 0) {
+    const int R = bm.total * P - sp.full;
+    kern<<<dim3(sp.full + 2 * R), kThreads, smem, st>>>(mq, mk, mv, mt, N, q_perm, qs.cluster, k_offsets,
+                                                         b.W, b.c0, b.c1, b.lse, (__nv_bfloat16 *)O,
+                                                         part_o, part_lse, status, bm, ra, sp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    refine_halves<DV><<<R, BM, 0, st>>>(mt, N, q_perm, sp.opart, (__nv_bfloat16 *)O, sp);
+    count_launches(2);
+    return cudaGetLastError();
+  }
   dim3 grid(bm.total, P);
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mt, N, q_perm, qs.cluster, k_offsets, b.W, b.c0,
                                      b.c1, b.lse, (__nv_bfloat16 *)O, part_o, part_lse, status, bm,
-                                     ra);
+                                     ra, sp);
   count_launches(1);
   return cudaGetLastError();
 }
