@@ -65,6 +65,9 @@ def parse():
                     help="acausal: the monopole-only ablation (dipole term dropped)")
     ap.add_argument("--partial-dipole", action="store_true",
                     help="acausal: the partially specialised dipole (untilted covariances)")
+    ap.add_argument("--refine-form", default="auto", choices=["auto", "summary", "pair"],
+                    help="acausal: the form of the full method's refinement (auto: the "
+                         "library's cost rule)")
     return ap.parse_args()
 
 
@@ -87,7 +90,25 @@ def workload_of(args):
         raise SystemExit("--monopole and --partial-dipole apply to the acausal workloads")
     if args.monopole and args.partial_dipole:
         raise SystemExit("--monopole and --partial-dipole exclude each other")
+    if args.refine_form != "auto" and (w.mode != "acausal" or args.monopole or args.partial_dipole):
+        raise SystemExit("--refine-form applies to the full method on the acausal workloads")
     return w
+
+
+def refine_form_of(w, requested="auto"):
+    """The form in which the library evaluates the full method's refinement: the summary
+    form exists for bfloat16, D = Dv = 128, acausal, Ck <= 256; with "auto" it is taken
+    where it needs under three quarters of the pair form's tensor flops (the library's
+    rule: pair 2 N^2 (D + Dv), summary 2 Dv D N (N / 256 + Cq / 2) + 2 Dv (D + 16) Ck N)."""
+    ok = w.mode == "acausal" and w.dtype == "bf16" and w.D == 128 and w.Dv == 128 and w.Ck <= 256
+    if not ok or requested == "pair":
+        return "pair"
+    if requested == "summary":
+        return "summary"
+    n = float(w.N)
+    pair = 2.0 * n * n * (w.D + w.Dv)
+    summ = 2.0 * w.Dv * w.D * n * (n / 256.0 + w.Cq / 2.0) + 2.0 * w.Dv * (w.D + 16) * w.Ck * n
+    return "summary" if summ < 0.75 * pair else "pair"
 
 
 def dist_info():
@@ -419,7 +440,9 @@ def measure(args, w, steps, warmup, world, rank, local_rank, cpu_baseline):
     if w.mode == "acausal":
         ws = m.workspace("muse_forward_ex", d, w.Cq, w.Ck)
         flags = (m.MUSE_FLAG_MONOPOLE if monopole else 0) | \
-            (m.MUSE_FLAG_PARTIAL_DIPOLE if partial else 0)
+            (m.MUSE_FLAG_PARTIAL_DIPOLE if partial else 0) | \
+            {"auto": 0, "summary": m.MUSE_FLAG_REFINE_SUMMARY,
+             "pair": m.MUSE_FLAG_REFINE_PAIR}[args.refine_form]
 
         def step(Q=Qd, K=Kd, V=Vd, O=Od):
             m.muse_forward_ex(Q, K, V, w.Cq, w.Ck, w.iters, w.scale, flags=flags, out=O, ws=ws)
@@ -540,10 +563,13 @@ def measure(args, w, steps, warmup, world, rank, local_rank, cpu_baseline):
         else:
             peak, bound, unit = FP32_SIMT_TFLOPS, "alu", "TFLOP/s"
         kname = "refinement (retrieval remainder)" if w.mode == "retrieval" else "refinement"
+        if w.mode == "acausal" and not (monopole or partial):
+            form = refine_form_of(w, args.refine_form)
+            kname += f" ({form} form)"
     achieved = flops / (kmean / 1e3) / 1e12
     roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak,
-            "traffic": None if summary_form else recorded_traffic(w.name),
+            "traffic": None if summary_form or "summary form" in kname else recorded_traffic(w.name),
             "kernel": kname, "kernel_ms": kmean, "flops_per_launch": flops,
             "peak_source": f"{peak_src} bf16_tflops (burst)" if bound == "tensor"
             else "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
@@ -574,7 +600,9 @@ def measure(args, w, steps, warmup, world, rank, local_rank, cpu_baseline):
             "ms_per_step": mean_ms, "dtype": w.dtype,
             "config": dict(config_of(w, graph is not None),
                            **({"monopole": True} if monopole else {}),
-                           **({"partial_dipole": True} if partial else {})),
+                           **({"partial_dipole": True} if partial else {}),
+                           **({"refine_form": refine_form_of(w, args.refine_form)}
+                              if w.mode == "acausal" and not (monopole or partial) else {})),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

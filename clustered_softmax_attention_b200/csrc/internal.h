@@ -139,6 +139,15 @@ cudaError_t run_coeffs(const MuseTables &mt, int dtype, int D, int P, float scal
 cudaError_t run_refine(const MuseTables &mt, int dtype, int D, int Dv, int N, int P,
                        SortedSide qs, const int32_t *q_perm, SortedSide ks, const void *vs_rows,
                        StageBufs b, void *O, float *part_o, float *part_lse, cudaStream_t st);
+// The refinement in summary form on the tensor cores (refine_sf.cu): O_n = sum_j c0_nj
+// mu_v,ij + sum_j c1_nj C'_ij qt_n with C'_ij = sum_{k in S_j} w_ik v_k k^T formed on chip per
+// query cluster; bfloat16, D = Dv = 128, one instance (acausal), Ck <= 256.  vt: the
+// transposed sorted values (run_sort_side_t).
+bool refine_sf_supported(int dtype, int D, int Dv, const MuseTables &mt);
+cudaError_t run_refine_sf(const MuseTables &mt, int N, int P, const void *qs_rows,
+                          const int32_t *q_perm, const int32_t *q_offsets, const void *ks_rows,
+                          const int32_t *k_offsets, const void *vt, const StageBufs &b, void *O,
+                          int *status, cudaStream_t st);
 // The refinement from materialised summaries (refine_summaries.cu): O_n = sum_j p_j
 // (mu_v,ij + s C_ij qt) with p = softmax_j(logZ_ij + s qt.mu_k,ij), float32 on the CUDA
 // cores.  q_labels (natural order) is optional; a row whose label disagrees with

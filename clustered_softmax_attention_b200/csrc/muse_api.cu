@@ -233,6 +233,16 @@ cudaError_t profile_mark(bool start, cudaStream_t st) {
   return record_profile_event(start ? ev0 : ev1, st);
 }
 
+// The refinement's two evaluations of the same sum: the pair form costs 2 N^2 (D + Dv)
+// tensor flops per problem; the summary form 2 Dv D N per unit of up to 256 rows of one
+// query cluster (about N / 256 + Cq / 2 units) plus 2 Dv (D + 16) Ck N.  The summary form
+// is taken when it needs under three quarters of the pair form's flops.
+static bool summary_form_cheaper(int N, int Cq, int Ck, int D, int Dv) {
+  const double n = N, pair = 2.0 * n * n * (D + Dv);
+  const double summ = 2.0 * Dv * D * n * (n / 256.0 + Cq / 2.0) + 2.0 * Dv * (D + 16) * (double)Ck * n;
+  return summ < 0.75 * pair;
+}
+
 // The refinement launch sequence shared by every path.
 static muse_status refine_path(const void *Q, const void *K, const void *V, const muse_dims &d,
                                int P, const MuseTables &mt, const float *q_centroids,
@@ -240,7 +250,7 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
                                const int32_t *k_perm, const int32_t *k_offsets,
                                const float *logZ_in, const float *mu_k_in, RefineWs &r, void *O,
                                float *part_o, float *part_lse, cudaStream_t st,
-                               bool monopole = false) {
+                               bool monopole = false, int form = 0) {
   MUSE_TRY(run_sort_side(Q, d.dtype, d.D, d.N, mt.q, P, q_perm, q_offsets, q_centroids, r.qs, st));
   MUSE_TRY(run_sort_side(K, d.dtype, d.D, d.N, mt.k, P, k_perm, k_offsets, nullptr, r.ks, st));
   const bool use_tc = tc_supported(d.dtype, d.D, d.Dv);
@@ -262,7 +272,11 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
   // the dipole terms carry the logit scale; the monopole-only ablation drops them
   MUSE_TRY(run_coeffs(mt, d.dtype, d.D, P, d.scale, r.qs, q_offsets, sb, monopole ? 0.f : d.scale, st));
   MUSE_TRY(profile_mark(true, st));
-  if (use_tc) {
+  if (use_tc && O && !monopole && refine_sf_supported(d.dtype, d.D, d.Dv, mt) &&
+      (form == 1 || (form == 0 && summary_form_cheaper(d.N, mt.q.C[0], mt.k.C[0], d.D, d.Dv)))) {
+    MUSE_TRY(run_refine_sf(mt, d.N, P, r.qs.rows, q_perm, q_offsets, r.ks.rows, k_offsets, r.vs, sb,
+                           O, status_ptr(), st));
+  } else if (use_tc) {
     MUSE_TRY(run_refine_tc(mt, d.D, d.Dv, d.N, P, r.qs, q_perm, r.ks, k_offsets, r.vs, sb, O,
                            part_o, part_lse, status_ptr(), st));
   } else {
@@ -550,16 +564,20 @@ extern "C" muse_status muse_forward_ex(const void *Q, const void *K, const void 
                                        size_t ws_bytes, muse_stream_t st) {
   muse_status s = check_dims(d, true);
   if (s != MUSE_OK) return s;
-  const unsigned known = MUSE_FLAG_MONOPOLE | MUSE_FLAG_PARTIAL_DIPOLE;
-  if ((flags & ~known) || (flags & known) == known) return MUSE_ERR_INVALID_ARG;
+  const unsigned abl = MUSE_FLAG_MONOPOLE | MUSE_FLAG_PARTIAL_DIPOLE;
+  const unsigned frm = MUSE_FLAG_REFINE_SUMMARY | MUSE_FLAG_REFINE_PAIR;
+  if ((flags & ~(abl | frm)) || (flags & abl) == abl || (flags & frm) == frm ||
+      ((flags & abl) && (flags & frm)))
+    return MUSE_ERR_INVALID_ARG;
   const bool partial = (flags & MUSE_FLAG_PARTIAL_DIPOLE) != 0;
+  const int form = (flags & MUSE_FLAG_REFINE_SUMMARY) ? 1 : (flags & MUSE_FLAG_REFINE_PAIR) ? 2 : 0;
   const void *ptrs[] = {Q, K, V, O};
   for (const void *p : ptrs)
     if (!p || !aligned16(p)) return MUSE_ERR_INVALID_ARG;
   if (!valid_C(Cq, d.N) || !valid_C(Ck, d.N) || iters < 1 || iters > 1000)
     return MUSE_ERR_INVALID_ARG;
   // the ablations in summary form (no O(N^2) contraction) where the output kernel fits
-  const bool summary = flags != 0 && coef_out_supported(d.dtype, d.D, d.Dv, Ck);
+  const bool summary = (flags & abl) != 0 && coef_out_supported(d.dtype, d.D, d.Dv, Ck);
   const size_t need = ws_forward(d, Cq, Ck) + (partial ? ws_partial_dipole(d, Cq, Ck) : 0) +
                       (summary ? ws_value_means(d, Cq, Ck) : 0);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MUSE_ERR_WORKSPACE;
@@ -611,7 +629,7 @@ extern "C" muse_status muse_forward_ex(const void *Q, const void *K, const void 
   // the partially specialised dipole adds s Cbar_i qt to the monopole-only result
   muse_status s2 = refine_path(Q, K, V, d, P, mt, kw.q.centroids, kw.q.perm, kw.q.offsets,
                                kw.k.perm, kw.k.offsets, nullptr, nullptr, r, O, nullptr, nullptr,
-                               cs, flags != 0);
+                               cs, (flags & abl) != 0, form);
   if (s2 != MUSE_OK || !partial) return s2;
   MUSE_TRY(run_partial_dipole(mt, d.dtype, d.D, d.Dv, d.N, P, d.scale, r.qs, kw.q.perm, r.ks, V,
                               kw.k.perm, kw.k.offsets, r.sb.logZ, pd_ws, O, cs));

@@ -278,12 +278,15 @@ def muse_forward(Q, K, V, Cq: int, Ck: int, iters: int, scale: float = 1.0,
 
 MUSE_FLAG_MONOPOLE = 1
 MUSE_FLAG_PARTIAL_DIPOLE = 2
+MUSE_FLAG_REFINE_SUMMARY = 4
+MUSE_FLAG_REFINE_PAIR = 8
 
 
 def muse_forward_ex(Q, K, V, Cq: int, Ck: int, iters: int, scale: float = 1.0, flags: int = 0,
                     out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
     """muse_forward with option flags (MUSE_FLAG_MONOPOLE: the monopole-only ablation;
-    MUSE_FLAG_PARTIAL_DIPOLE: the partially specialised dipole)."""
+    MUSE_FLAG_PARTIAL_DIPOLE: the partially specialised dipole; MUSE_FLAG_REFINE_SUMMARY /
+    MUSE_FLAG_REFINE_PAIR: the form of the full method's refinement)."""
     _qkv(Q, K, V, out)
     _contig(Q, K, V, out, ws)
     d = dims(Q, V, scale)

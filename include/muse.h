@@ -150,7 +150,11 @@ muse_status muse_tilted_summaries(const float *q_centroids, const void *K, const
  *     u_j = qt.mu_k,ij the output is computed as
  *       O_n = sum_j sum_{k in S_j} w_ik p_j (1 - s u_j + s qt.k) v_k,
  *     an identity of the definition (sum_k w_ik (k - mu_k,ij) = 0), on the tensor
- *     cores for bfloat16 inputs; the tilt weights w_ik are recomputed from logZ.
+ *     cores for bfloat16 inputs; the tilt weights w_ik are recomputed from logZ.  That
+ *     sum is taken over all keys (the pair form) or, grouped by key cluster, against
+ *     the uncentred summaries C'_ij = sum_{k in S_j} w_ik v_k k^T formed on chip (the
+ *     summary form), as MUSE_FLAG_REFINE_SUMMARY below describes, by the same rule
+ *     as muse_forward with no flags.
  *   - mu_v and cov given: the formula above is evaluated as written from the
  *     caller's materialised summaries (float32, CUDA cores; teacher forcing of the
  *     dipole, or summaries from elsewhere).
@@ -201,11 +205,28 @@ muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims 
  * Same arguments, layouts and ownership as muse_forward.  Workspace: that of
  * muse_forward, plus B*H*(Cq + Ck)*D*Dv floats and 256 bytes with
  * MUSE_FLAG_PARTIAL_DIPOLE, plus B*H*Cq*Ck*Dv floats and 256 bytes in summary form;
- * muse_workspace_size("muse_forward_ex", ...) returns the largest of these sizes.  Unknown flag bits, or both flags at once, return MUSE_ERR_INVALID_ARG
- * before anything is enqueued.
+ * muse_workspace_size("muse_forward_ex", ...) returns the largest of these sizes.  Unknown flag bits, or both ablation flags at once, return
+ * MUSE_ERR_INVALID_ARG before anything is enqueued.
  */
 #define MUSE_FLAG_MONOPOLE 1u
 #define MUSE_FLAG_PARTIAL_DIPOLE 2u
+/*
+ * The form of the full method's refinement (muse_forward, muse_dipole_refine evaluate
+ * the same sum either way; pith.science review of arXiv 2509.10406, "What carries the
+ * argument"):
+ *   pair form: O_n = sum_k w_ik (c0_nj + c1_nj qt_n.k) v_k over all keys, 2 N^2 (D + Dv)
+ *   tensor flops per problem;
+ *   summary form: O_n = sum_j c0_nj mu_v,ij + sum_j c1_nj C'_ij qt_n with
+ *   C'_ij = sum_{k in S_j} w_ik v_k k^T formed on chip for each query cluster and never
+ *   stored, about 2 Dv D N (N / 256 + Cq / 2) + 2 Dv (D + 16) Ck N flops; bfloat16 with
+ *   D = Dv = 128 and Ck <= 256 only.
+ * With neither flag the summary form is taken where it is supported and needs under three
+ * quarters of the pair form's flops; MUSE_FLAG_REFINE_SUMMARY takes it wherever it is
+ * supported, MUSE_FLAG_REFINE_PAIR never.  Both at once, or either with an ablation flag,
+ * return MUSE_ERR_INVALID_ARG.
+ */
+#define MUSE_FLAG_REFINE_SUMMARY 4u
+#define MUSE_FLAG_REFINE_PAIR 8u
 muse_status muse_forward_ex(const void *Q, const void *K, const void *V, muse_dims d, int Cq,
                             int Ck, int iters, unsigned flags, void *O, void *ws,
                             size_t ws_bytes, muse_stream_t st);

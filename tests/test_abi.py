@@ -99,9 +99,15 @@ def test_argument_validation_enqueues_nothing(lib):
     assert lib.muse_causal_blocks(f, f, f, _d(N=1000), 128, 8, 8, 2, f, None, None, f, 1 << 30,
                                   st) == 2
     assert lib.muse_causal_blocks(f, f, f, _d(), 128, 8, 8, 2, f, None, None, f, 0, st) == 4
-    # option flags: unknown bits are refused before the workspace is looked at
-    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 4, f, f, 1 << 30, st) == 1
+    # option flags: unknown bits and contradictory pairs are refused before the workspace
+    # is looked at (both ablations, both refinement forms, an ablation with a form)
+    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 16, f, f, 1 << 30, st) == 1
     assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 3, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 12, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 5, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 10, f, f, 1 << 30, st) == 1
+    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 4, f, f, 16, st) == 4
+    assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 8, f, f, 16, st) == 4
     assert lib.muse_forward_ex(f, f, f, _d(), 8, 8, 2, 1, f, f, 16, st) == 4
     assert lib.muse_forward_ex(f, f, f, _d(D=96), 8, 8, 2, 1, f, f, 1 << 30, st) == 2
 

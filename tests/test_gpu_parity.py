@@ -336,6 +336,32 @@ def test_forward_bf16_unequal_widths(D, Dv, parity):
         assert mo.max_rel_err(O[0, h], ref) <= TOL["bf16"]
 
 
+# The refinement in summary form (C'_ij formed on chip for each query cluster, then one
+# product per query tile against [C'_ij | mu_v,ij]) against the oracle and against the
+# pair form on the same clustering: query clusters of several 256-row units plus ragged
+# ones, key clusters over several tiles and tiles over several key clusters (up to 256),
+# and N = 2996 (the transposed values' padding columns lie inside the last tile).
+@pytest.mark.parametrize("N,Cq,Ck,comps", [(2048, 8, 32, 48), (2996, 5, 40, 48),
+                                           (1536, 64, 256, 96)])
+def test_forward_refine_summary_form(N, Cq, Ck, comps, parity):
+    D = Dv = 128
+    Q, K, V = mixture(14, 1, 2, N, D, Dv, comps, 0.5 / np.sqrt(D), "bf16")
+    Qd, Kd, Vd = dev(Q, "bf16"), dev(K, "bf16"), dev(V, "bf16")
+    Os = host(m.muse_forward_ex(Qd, Kd, Vd, Cq, Ck, 5, 1.0, flags=m.MUSE_FLAG_REFINE_SUMMARY))
+    assert m.muse_last_device_status() == 0
+    Op = host(m.muse_forward_ex(Qd, Kd, Vd, Cq, Ck, 5, 1.0, flags=m.MUSE_FLAG_REFINE_PAIR))
+    ql = m.muse_kmeans(Qd, Cq, 5)[0].cpu().numpy()
+    kl = m.muse_kmeans(Kd, Ck, 5)[0].cpu().numpy()
+    assert np.bincount(ql[0, 0], minlength=Cq).max() > 256 or Cq == 64  # units of 256 rows
+    Qf, Kf, Vf = host(Qd), host(Kd), host(Vd)
+    for h in range(2):
+        ref = mo.muse_from_labels(Qf[0, h], Kf[0, h], Vf[0, h], ql[0, h], kl[0, h], Cq, Ck, 1.0)
+        parity(f"O summary form h={h}", mo.max_rel_err(Os[0, h], ref), TOL["bf16"])
+        assert mo.max_rel_err(Os[0, h], ref) <= TOL["bf16"]
+        parity(f"O pair form h={h}", mo.max_rel_err(Op[0, h], ref), TOL["bf16"])
+        assert mo.max_rel_err(Op[0, h], ref) <= TOL["bf16"]
+
+
 def test_singleton_query_clusters_give_exact_attention_on_gpu(parity):
     Q, K, V = small_problem(21, 256, 64, 64, 16, 0.3)
     Qd, Kd, Vd = (dev(x[None, None], "f32") for x in (Q, K, V))
