@@ -11,20 +11,21 @@
 // 2 Dv D nk (the summaries) + 2 Dv (D + 16) Ck nq (the product), against the pair form's
 // 2 nq nk (D + Dv): the smaller one at long context (N >> Ck D).
 //
-// One CTA = one query cluster i and up to 240 of its sorted rows (a unit).  For every
+// One CTA = one query cluster i and up to 224 of its sorted rows (a unit).  For every
 // non-empty key cluster j, in order:
-//   (a) C'_ij (fp32, TMEM, M = Dv lanes, N = D columns) = (w .* V_j)^T . K_j over key
-//       tiles of 64: the value tile (transposed, TMA) is scaled in place by the tilt
-//       weights of cluster i (zero outside S_j: the tile starts 8-aligned before S_j), the
-//       key tile (TMA, rows of 64 coordinates) is an MN-major B operand; the scaling
-//       threads also sum the scaled values per coordinate in float32: mu_v,ij.
+//   (a) [C'_ij | mu_v,ij] (fp32, TMEM, M = Dv lanes, N = D + 16 columns) =
+//       (w .* V_j)^T . [K_j | 1] over key tiles of 64: the value tile (transposed, TMA) is
+//       scaled in place by the tilt weights of cluster i (zero outside S_j: the tile starts
+//       8-aligned before S_j); the key tile (TMA, rows of 64 coordinates) is an MN-major B
+//       operand, and a constant tile of ones gives the 16 columns of mu_v,ij.
 //   (b) C'_ij is copied as bfloat16 pairs into one of two packed buffers, followed by the
 //       K columns [mu_hi, mu_lo, mu_hi, 0 ...] (the A operand of (c), in TMEM); the
 //       float32 buffer is then free for (a) of the next cluster.
 //   (c) O^T (fp32, TMEM, M = Dv lanes, N = unit rows) += [C'_ij | aux] . [c1 qt_n | c0_hi,
 //       c0_hi, c0_lo, 0 ...]^T, B built per row from the residual (held in registers)
 //       and the coefficients.
-// TMEM columns: C' [0, 128), packed buffers [128, 200) and [200, 272), O^T [272, 512).
+// TMEM columns: C' and mu_v [0, 144), packed buffers [144, 216) and [216, 288), O^T
+// [288, 512).
 // The tensor cores run (a) of cluster j + 1 while (b) of cluster j is copied and the rows
 // of (c) are built; (c) of cluster j follows (a) of cluster j + 1.
 // Warp roles: 0 = TMA producer, 1 = MMA issuer (+ TMEM owner), 2-5 = scaling, 6-13 =
@@ -45,24 +46,24 @@ using namespace ptx;
 constexpr int D = 128, DV = 128;
 constexpr int BN = 64;       // keys per tile
 constexpr int NST = 4;       // tile stages
-constexpr int UR = 240;      // query rows per unit (N of the product (c))
+constexpr int UR = 224;      // query rows per unit (N of the product (c))
 constexpr int kMaxCk = 256;  // key clusters (offsets staged in shared memory)
 constexpr int kScale0 = 2, kRow0 = 6;                // first warp of each role
 constexpr int kRowWarps = 8;                         // 256 threads: rows UR.. are idle
 constexpr int kThreads = 32 * (kRow0 + kRowWarps);   // 448
 constexpr int KA = D / 16 + 1;                       // K steps of (c): D + the aux step
-constexpr uint32_t kPcol = 128, kPstride = D / 2 + 8;  // packed buffers: 72 columns each
-constexpr uint32_t kOcol = kPcol + 2 * kPstride;       // O^T: 240 columns
+constexpr uint32_t kPcol = D + 16, kPstride = D / 2 + 8;  // packed buffers: 72 columns each
+constexpr uint32_t kOcol = kPcol + 2 * kPstride;          // O^T: 224 columns
 
 struct __align__(1024) Smem {
   __nv_bfloat16 k[NST][D / 64][BN * 64];  // key tiles: a row per key, 64 coordinates per block
   __nv_bfloat16 vt[NST][DV * 64];         // value tiles: a row per value coordinate, 64 keys
   __nv_bfloat16 bq[D / 64 + 1][UR * 64];  // B of (c): a row per query row, K-major SW128
   float w[NST][BN];                       // tilt weights of cluster i over each tile's keys
-  float mv[2][DV];                        // mu_v,ij of the clusters in the two C' buffers
+  __nv_bfloat16 ones[16 * 64];            // B of the mu_v columns: 16 K-rows of ones
   int koff[kMaxCk + 1];                   // the key-cluster offsets
   uint64_t full[NST], scaled[NST], empty[NST];
-  uint64_t cfull, cfree, pready[2], mvfull[2], mvfree[2], bqready, bdone;
+  uint64_t cfull, cfree, pready[2], bqready, bdone;
   uint32_t tmem_base;
   int abort_flag;
   int s_i, s_r0, s_nr;
@@ -187,16 +188,15 @@ refine_sf(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUt
     }
     mbar_init(&sm.cfull, 1);
     mbar_init(&sm.cfree, kRowWarps);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.pready[b], kRowWarps);
-      mbar_init(&sm.mvfull[b], 4);
-      mbar_init(&sm.mvfree[b], 4);
-    }
+    for (int b = 0; b < 2; ++b) mbar_init(&sm.pready[b], kRowWarps);
     mbar_init(&sm.bqready, kRowWarps);
     mbar_init(&sm.bdone, 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  for (int u = t; u < 16 * 64 / 8; u += kThreads)  // bfloat16 1.0 = 0x3F80
+    reinterpret_cast<uint4 *>(sm.ones)[u] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // ones -> tensor cores
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      saddr(&sm.tmem_base)),
@@ -263,6 +263,7 @@ refine_sf(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUt
       int g = 0, jj = 0;
       bool ok = true;
       constexpr uint32_t ia = idesc(128, D) | (1u << 16);  // B (the key tile) MN-major
+      constexpr uint32_t i1 = idesc(128, 16) | (1u << 16);  // B: 16 columns of ones
       for (int j = 0; ok && j < Ck; ++j) {
         const int b0 = koff[j], e0 = koff[j + 1];
         if (b0 == e0) continue;
@@ -275,9 +276,12 @@ refine_sf(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUt
           if (!(ok = mbar_wait<true>(&sm.scaled[st], (g / NST) & 1, abort_flag, status))) break;
           tc_fence_after();
           const int nks = (min(BN, e0 - x0) + 15) / 16;
-          for (int kk = 0; kk < nks; ++kk)  // the D/64 blocks of the key tile: BN*128 B apart
-            tc_mma(tmem, sdesc(sm.vt[st] + kk * 16), sdesc_mn(sm.k[st][0] + kk * 16 * 64, BN * 128), ia,
-                   (tl > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < nks; ++kk) {  // the D/64 blocks of the key tile: BN*128 B apart
+            const uint64_t a = sdesc(sm.vt[st] + kk * 16);
+            const uint32_t acc = (tl > 0 || kk > 0) ? 1u : 0u;
+            tc_mma(tmem, a, sdesc_mn(sm.k[st][0] + kk * 16 * 64, BN * 128), ia, acc);
+            tc_mma(tmem + D, a, sdesc_mn(sm.ones, 1024), i1, acc);  // mu_v in all 16 columns
+          }
           tc_commit(&sm.empty[st]);
           lastbar = &sm.empty[st];
           lastpar = (g / NST) & 1;
@@ -297,88 +301,45 @@ refine_sf(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUt
     // ------------------------------------------------------------ scaling
     const int ts = t - 32 * kScale0;
     const int c = ts & 7, rb = ts >> 3;  // 8 keys of the tile; rows rb + 16 m
-    int g = 0, jj = 0;
+    int g = 0;
     bool ok = true;
     for (int j = 0; ok && j < Ck; ++j) {
       const int b0 = koff[j], e0 = koff[j + 1];
-      if (b0 == e0) continue;
-      float acc[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) acc[m] = 0.f;
-      for (int x0 = b0 & ~7; x0 < e0; x0 += BN, ++g) {
+      for (int x0 = b0 & ~7; b0 < e0 && x0 < e0; x0 += BN, ++g) {
         const int st = g % NST;
         const int pos = x0 + 8 * c;
         unsigned in = 0;  // bit e: key pos + e lies in S_j
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           if (pos + e >= b0 && pos + e < e0) in |= 1u << e;
+        uint32_t keep[4];  // per pair: the halves that lie in S_j
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          keep[e] = (((in >> (2 * e)) & 1u) ? 0x0000ffffu : 0u) | (((in >> (2 * e + 1)) & 1u) ? 0xffff0000u : 0u);
         if (!(ok = wait_all(&sm.full[st], (g / NST) & 1, abort_flag, status))) break;
         // (weights past the end of W's row are not copied: they lie outside S_j)
         const float4 wa = *reinterpret_cast<const float4 *>(&sm.w[st][8 * c]);
         const float4 wb = *reinterpret_cast<const float4 *>(&sm.w[st][8 * c + 4]);
-        float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-        if (in != 0xffu) {  // part of the chunk lies outside S_j: zero weights there
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            if (!((in >> e) & 1u)) w[e] = 0.f;
-        }
+        const __nv_bfloat162 w2[4] = {__floats2bfloat162_rn(wa.x, wa.y), __floats2bfloat162_rn(wa.z, wa.w),
+                                      __floats2bfloat162_rn(wb.x, wb.y), __floats2bfloat162_rn(wb.z, wb.w)};
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
           const int v = rb + 16 * m;
           uint4 *ptr = reinterpret_cast<uint4 *>(sm.vt[st] + v * 64 + ((c ^ (v & 7)) << 3));
-          const uint4 x = *ptr;
-          const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
-          uint32_t ys[4];
-          float s0 = 0.f, s1 = 0.f;
+          uint4 x = *ptr;
+          uint32_t *xs = reinterpret_cast<uint32_t *>(&x);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float a0, a1;
-            mul2(a0, a1, __uint_as_float(xs[e] << 16), __uint_as_float(xs[e] & 0xffff0000u), w[2 * e],
-                 w[2 * e + 1]);
-            add2(s0, s1, s0, s1, a0, a1);
-            ys[e] = pack_bf16(a0, a1);
+            const __nv_bfloat162 pr = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&xs[e]), w2[e]);
+            // keys outside S_j (and padding, which may hold anything) become zero
+            xs[e] = *reinterpret_cast<const uint32_t *>(&pr) & keep[e];
           }
-          if (in != 0xffu) {  // padding outside the keys may hold anything: clear it
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t keep = (((in >> (2 * e)) & 1u) ? 0x0000ffffu : 0u) |
-                                    (((in >> (2 * e + 1)) & 1u) ? 0xffff0000u : 0u);
-              ys[e] &= keep;
-            }
-            s0 = 0.f;
-            s1 = 0.f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float a0 = __uint_as_float(xs[e] << 16) * w[2 * e];
-              const float a1 = __uint_as_float(xs[e] & 0xffff0000u) * w[2 * e + 1];
-              s0 += ((in >> (2 * e)) & 1u) ? a0 : 0.f;
-              s1 += ((in >> (2 * e + 1)) & 1u) ? a1 : 0.f;
-            }
-          }
-          acc[m] += s0 + s1;
-          *ptr = make_uint4(ys[0], ys[1], ys[2], ys[3]);
+          *ptr = x;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // scaled tile -> tensor cores
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.scaled[st]);
       }
-      if (!ok) break;
-      // mu_v,ij: the 8 threads of a row group hold parts of the same sums
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 1);
-        acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 2);
-        acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 4);
-      }
-      const int b = jj & 1;
-      if (jj >= 2 && !(ok = wait_all(&sm.mvfree[b], ((jj >> 1) - 1) & 1, abort_flag, status))) break;
-      if (c == 0) {
-#pragma unroll
-        for (int m = 0; m < 8; ++m) sm.mv[b][rb + 16 * m] = acc[m];
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.mvfull[b]);
-      ++jj;
     }
   } else {
     // ------------------------------------------------------------ rows: (b), B of (c), O
@@ -415,7 +376,8 @@ refine_sf(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUt
       const int b = jj & 1;
       const float c0 = valid ? C0[(int64_t)j * cl] : 0.f, c1 = valid ? C1[(int64_t)j * cl] : 0.f;
       // (b) this warp's half of C' (columns [64 h, 64 h + 64)) as bfloat16 pairs into
-      // packed columns [32 h, 32 h + 32) of buffer b; the float32 buffer is then released
+      // packed columns [32 h, 32 h + 32) of buffer b; once mu_v is read too, the float32
+      // buffer is released
       const uint32_t src = tmem + lb + h * 64;
       const uint32_t dst = tmem + lb + kPcol + b * kPstride + h * 32;
       if (!(ok = wait_all(&sm.cfull, jj & 1, abort_flag, status))) break;
@@ -428,14 +390,16 @@ refine_sf(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUt
                                 pack_bf16(x[6], x[7])};
         tmem_st4(dst + 4 * ch, pk);
       }
+      float mu = 0.f;  // h = 1: mu_v,ij of row v (column D; its 16 columns are equal)
+      if (h == 1) {
+        float xm[8];
+        tmem_ld8(tmem + lb + D, xm);
+        mu = xm[0];
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.cfree);
-      if (h == 1) {  // the aux step: [mu_hi, mu_lo, mu_hi, 0 ...]
-        if (!(ok = wait_all(&sm.mvfull[b], (jj >> 1) & 1, abort_flag, status))) break;
-        const float mu = sm.mv[b][v];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.mvfree[b]);
+      if (h == 1) {  // the aux step [mu_hi, mu_lo, mu_hi, 0 ...]
         const float mh = __bfloat162float(__float2bfloat16_rn(mu));
         const uint32_t ax[8] = {pack_bf16(mh, mu - mh), pack_bf16(mh, 0.f), 0u, 0u, 0u, 0u, 0u, 0u};
         tmem_st8(dst + 32, ax);
