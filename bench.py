@@ -65,6 +65,9 @@ def parse():
                     help="acausal: the monopole-only ablation (dipole term dropped)")
     ap.add_argument("--partial-dipole", action="store_true",
                     help="acausal: the partially specialised dipole (untilted covariances)")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the first H (b,h) problems of the workload only (B = 1; the same "
+                         "draws as the full workload's first problems), e.g. for a small profile")
     ap.add_argument("--refine-form", default="auto", choices=["auto", "summary", "pair"],
                     help="acausal: the form of the full method's refinement (auto: the "
                          "library's cost rule)")
@@ -86,6 +89,10 @@ def workload_of(args):
         w = dataclasses.replace(w, Cq=args.clusters, Ck=args.clusters)
     if args.iters:
         w = dataclasses.replace(w, iters=args.iters)
+    if args.heads:
+        if not 1 <= args.heads <= w.B * w.H:
+            raise SystemExit(f"--heads must be in [1, B*H={w.B * w.H}]")
+        w = dataclasses.replace(w, B=1, H=args.heads)
     if (args.monopole or args.partial_dipole) and w.mode != "acausal":
         raise SystemExit("--monopole and --partial-dipole apply to the acausal workloads")
     if args.monopole and args.partial_dipole:
@@ -642,7 +649,8 @@ def main():
     # workload (every rank, same collective steps), reported under its own key
     second = None
     if args.workload == DEFAULT_WORKLOAD and not args.no_second and not (
-            args.block or args.clusters or args.iters or args.monopole or args.partial_dipole):
+            args.block or args.clusters or args.iters or args.heads or args.monopole or
+            args.partial_dipole):
         second = measure(args, WORKLOADS[SECOND_HEADLINE], max(10, args.steps // 4), args.warmup,
                          world, rank, local_rank, cpu_baseline=False)
     if rank == 0:
