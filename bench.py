@@ -103,19 +103,18 @@ def workload_of(args):
 
 
 def refine_form_of(w, requested="auto"):
-    """The form in which the library evaluates the full method's refinement: the summary
-    form exists for bfloat16, D = Dv = 128, acausal, Ck <= 256; with "auto" it is taken
-    where it needs under three quarters of the pair form's tensor flops (the library's
-    rule: pair 2 N^2 (D + Dv), summary 2 Dv D N (N / 256 + Cq / 2) + 2 Dv (D + 16) Ck N)."""
-    ok = w.mode == "acausal" and w.dtype == "bf16" and w.D == 128 and w.Dv == 128 and w.Ck <= 256
-    if not ok or requested == "pair":
+    """The form in which the library evaluates the full method's refinement of workload
+    w ("summary" or "pair"), as the library itself decides it (muse_refine_form)."""
+    from clustered_softmax_attention_b200 import muse as m
+    if w.mode != "acausal":
         return "pair"
-    if requested == "summary":
-        return "summary"
-    n = float(w.N)
-    pair = 2.0 * n * n * (w.D + w.Dv)
-    summ = 2.0 * w.Dv * w.D * n * (n / 256.0 + w.Cq / 2.0) + 2.0 * w.Dv * (w.D + 16) * w.Ck * n
-    return "summary" if summ < 0.75 * pair else "pair"
+    d = m.MuseDims(w.B, w.H, w.N, w.D, w.Dv, m.MUSE_BF16 if w.dtype == "bf16" else m.MUSE_F32,
+                   w.scale)
+    flags = {"auto": 0, "summary": m.MUSE_FLAG_REFINE_SUMMARY, "pair": m.MUSE_FLAG_REFINE_PAIR}[requested]
+    form = m.lib().muse_refine_form(d, w.Cq, w.Ck, flags)
+    if form < 0:
+        raise ValueError(f"muse_refine_form refused {w.name}")
+    return "summary" if form == 1 else "pair"
 
 
 def dist_info():

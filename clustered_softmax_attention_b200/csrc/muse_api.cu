@@ -234,13 +234,22 @@ cudaError_t profile_mark(bool start, cudaStream_t st) {
 }
 
 // The refinement's two evaluations of the same sum: the pair form costs 2 N^2 (D + Dv)
-// tensor flops per problem; the summary form 2 Dv D N per unit of up to 256 rows of one
-// query cluster (about N / 256 + Cq / 2 units) plus 2 Dv (D + 16) Ck N.  The summary form
+// tensor flops per problem; the summary form 2 Dv D N per unit of up to 224 rows of one
+// query cluster (about N / 224 + Cq / 2 units) plus 2 Dv (D + 16) Ck N.  The summary form
 // is taken when it needs under three quarters of the pair form's flops.
 static bool summary_form_cheaper(int N, int Cq, int Ck, int D, int Dv) {
   const double n = N, pair = 2.0 * n * n * (D + Dv);
-  const double summ = 2.0 * Dv * D * n * (n / 256.0 + Cq / 2.0) + 2.0 * Dv * (D + 16) * (double)Ck * n;
+  const double summ = 2.0 * Dv * D * n * (n / 224.0 + Cq / 2.0) + 2.0 * Dv * (D + 16) * (double)Ck * n;
   return summ < 0.75 * pair;
+}
+
+// Whether the full method's refinement runs in summary form.  form: 0 = by the flop rule,
+// 1 = wherever supported, 2 = never; out: the call writes O (not the causal partials).
+static bool use_summary_form(const muse_dims &d, const MuseTables &mt, bool monopole, int form,
+                             bool out) {
+  return out && !monopole && form != 2 && tc_supported(d.dtype, d.D, d.Dv) &&
+         refine_sf_supported(d.dtype, d.D, d.Dv, mt) &&
+         (form == 1 || summary_form_cheaper(d.N, mt.q.C[0], mt.k.C[0], d.D, d.Dv));
 }
 
 // The refinement launch sequence shared by every path.
@@ -272,8 +281,7 @@ static muse_status refine_path(const void *Q, const void *K, const void *V, cons
   // the dipole terms carry the logit scale; the monopole-only ablation drops them
   MUSE_TRY(run_coeffs(mt, d.dtype, d.D, P, d.scale, r.qs, q_offsets, sb, monopole ? 0.f : d.scale, st));
   MUSE_TRY(profile_mark(true, st));
-  if (use_tc && O && !monopole && refine_sf_supported(d.dtype, d.D, d.Dv, mt) &&
-      (form == 1 || (form == 0 && summary_form_cheaper(d.N, mt.q.C[0], mt.k.C[0], d.D, d.Dv)))) {
+  if (use_summary_form(d, mt, monopole, form, O != nullptr)) {
     MUSE_TRY(run_refine_sf(mt, d.N, P, r.qs.rows, q_perm, q_offsets, r.ks.rows, k_offsets, r.vs, sb,
                            O, status_ptr(), st));
   } else if (use_tc) {
@@ -634,6 +642,18 @@ extern "C" muse_status muse_forward_ex(const void *Q, const void *K, const void 
   MUSE_TRY(run_partial_dipole(mt, d.dtype, d.D, d.Dv, d.N, P, d.scale, r.qs, kw.q.perm, r.ks, V,
                               kw.k.perm, kw.k.offsets, r.sb.logZ, pd_ws, O, cs));
   return MUSE_OK;
+}
+
+extern "C" int muse_refine_form(muse_dims d, int Cq, int Ck, unsigned flags) {
+  if (check_dims(d, true) != MUSE_OK || !valid_C(Cq, d.N) || !valid_C(Ck, d.N)) return -1;
+  const unsigned frm = MUSE_FLAG_REFINE_SUMMARY | MUSE_FLAG_REFINE_PAIR;
+  if ((flags & ~frm) || (flags & frm) == frm) return -1;
+  MuseTables mt;
+  mt.q = whole_side(d.N, Cq);
+  mt.k = whole_side(d.N, Ck);
+  mt.in = whole_inst(d.N, Cq, Ck);
+  const int form = (flags & MUSE_FLAG_REFINE_SUMMARY) ? 1 : (flags & MUSE_FLAG_REFINE_PAIR) ? 2 : 0;
+  return use_summary_form(d, mt, false, form, true) ? 1 : 0;
 }
 
 extern "C" muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims d,

@@ -57,6 +57,7 @@ _SIGS = {
     "muse_last_error_detail": [],
     "muse_last_device_status": [_vp],
     "muse_set_test_hooks": [ctypes.c_uint, ctypes.c_uint64],
+    "muse_refine_form": [MuseDims, _i, _i, ctypes.c_uint],
     "muse_backward": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, MuseDims, _i, _i, _vp, _vp, _vp,
                       _vp, _sz, _vp],
 }

@@ -218,7 +218,7 @@ muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims 
  *   tensor flops per problem;
  *   summary form: O_n = sum_j c0_nj mu_v,ij + sum_j c1_nj C'_ij qt_n with
  *   C'_ij = sum_{k in S_j} w_ik v_k k^T formed on chip for each query cluster and never
- *   stored, about 2 Dv D N (N / 256 + Cq / 2) + 2 Dv (D + 16) Ck N flops; bfloat16 with
+ *   stored, about 2 Dv D N (N / 224 + Cq / 2) + 2 Dv (D + 16) Ck N flops; bfloat16 with
  *   D = Dv = 128 and Ck <= 256 only.
  * With neither flag the summary form is taken where it is supported and needs under three
  * quarters of the pair form's flops; MUSE_FLAG_REFINE_SUMMARY takes it wherever it is
@@ -227,6 +227,14 @@ muse_status muse_forward(const void *Q, const void *K, const void *V, muse_dims 
  */
 #define MUSE_FLAG_REFINE_SUMMARY 4u
 #define MUSE_FLAG_REFINE_PAIR 8u
+
+/*
+ * muse_refine_form - the form in which muse_forward_ex (with these flags, 0 or one of the
+ * two form flags) and muse_dipole_refine (flags 0) evaluate the full method's
+ * refinement for these sizes: 1 = summary form, 0 = pair form, -1 = invalid dims, cluster
+ * counts or flags.  Host only (enqueues nothing, needs no device).
+ */
+int muse_refine_form(muse_dims d, int Cq, int Ck, unsigned flags);
 muse_status muse_forward_ex(const void *Q, const void *K, const void *V, muse_dims d, int Cq,
                             int Ck, int iters, unsigned flags, void *O, void *ws,
                             size_t ws_bytes, muse_stream_t st);

@@ -112,6 +112,26 @@ def test_argument_validation_enqueues_nothing(lib):
     assert lib.muse_forward_ex(f, f, f, _d(D=96), 8, 8, 2, 1, f, f, 1 << 30, st) == 2
 
 
+def test_refine_form_query(lib):
+    """muse_refine_form reports the library's own choice between the pair and the summary
+    form of the refinement (host only)."""
+    f = lib.muse_refine_form
+    d64k = _d(H=16, N=65536, D=128, Dv=128)
+    assert f(d64k, 256, 256, 0) == 1                          # long context: summary form
+    assert f(d64k, 256, 256, m.MUSE_FLAG_REFINE_PAIR) == 0
+    assert f(d64k, 256, 300, 0) == 0                          # Ck > 256: pair form only
+    assert f(_d(H=8, N=8192), 128, 128, 0) == 0               # D = 64: pair form
+    assert f(_d(H=8, N=8192), 128, 128, m.MUSE_FLAG_REFINE_SUMMARY) == 0
+    small = _d(N=2048, D=128, Dv=128)
+    assert f(small, 32, 32, 0) == 0                           # short: the pair form is cheaper
+    assert f(small, 32, 32, m.MUSE_FLAG_REFINE_SUMMARY) == 1
+    assert f(_d(N=2048, D=128, Dv=128, dtype=m.MUSE_F32), 32, 32, m.MUSE_FLAG_REFINE_SUMMARY) == 0
+    assert f(small, 32, 32, m.MUSE_FLAG_REFINE_SUMMARY | m.MUSE_FLAG_REFINE_PAIR) == -1
+    assert f(small, 32, 32, m.MUSE_FLAG_MONOPOLE) == -1
+    assert f(_d(D=96), 32, 32, 0) == -1
+    assert f(small, 0, 32, 0) == -1
+
+
 def test_binding_refuses_mismatched_tensors():
     """The binding checks what the C ABI cannot (buffer extents): Q, K, V shapes, dtypes and
     the output's shape, before anything reaches the library."""
