@@ -606,9 +606,7 @@ def measure(args, w, steps, warmup, world, rank, local_rank, cpu_baseline):
             "ms_per_step": mean_ms, "dtype": w.dtype,
             "config": dict(config_of(w, graph is not None),
                            **({"monopole": True} if monopole else {}),
-                           **({"partial_dipole": True} if partial else {}),
-                           **({"refine_form": refine_form_of(w, args.refine_form)}
-                              if w.mode == "acausal" and not (monopole or partial) else {})),
+                           **({"partial_dipole": True} if partial else {})),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
