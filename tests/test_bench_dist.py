@@ -90,10 +90,26 @@ def test_workload_overrides():
                 ["--workload", "causal_n16k_bf16", "--block", "1000"],  # does not divide N
                 ["--workload", "causal_n16k_bf16", "--monopole"],
                 ["--monopole", "--partial-dipole"],
-                ["--clusters", "100000"]):
+                ["--clusters", "100000"],
+                ["--heads", "9"],                                      # 8 problems at 8k
+                ["--refine-form", "summary", "--monopole"],            # forms: full method only
+                ["--workload", "causal_n16k_bf16", "--refine-form", "pair"]):
         bench, a = _args(*bad)
         with pytest.raises(SystemExit):
             bench.workload_of(a)
+
+
+def test_heads_slice_and_refinement_form():
+    """--heads keeps the first H problems of a workload (B = 1); the bench names the
+    refinement form the library chooses (summary form at N = 64k, D = 128 only)."""
+    bench, a = _args("--workload", "acausal_n64k_d128_bf16", "--heads", "2")
+    w = bench.workload_of(a)
+    assert (w.B, w.H, w.N, w.D) == (1, 2, 65536, 128)
+    assert bench.refine_form_of(w) == "summary"
+    assert bench.refine_form_of(w, "pair") == "pair"
+    bench, a = _args()
+    w8 = bench.workload_of(a)
+    assert bench.refine_form_of(w8) == "pair" and bench.refine_form_of(w8, "summary") == "pair"
 
 
 def test_algorithmic_flops_of_the_block_sweep():
